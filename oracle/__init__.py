@@ -1,0 +1,156 @@
+"""CPU oracle for INT8 KV-cache append, dequantization and decode attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and
+the benchmark's CPU-baseline / reference leg may import this package.  It is
+a thin ctypes binding over ``kvq_oracle.c`` (plain scalar C: fp32 IEEE
+quantisation, fp64 attention) and shares nothing with the CUDA library.
+
+Parity pins: every routine here is pinned by ``tests/test_oracle_*.py``
+(worked examples from the pages, closed forms, invariants and an
+independent library routine for attention).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _build
+
+_lib = None
+
+ORACLE_ERR_POS = 1
+ORACLE_ERR_PAGE = 2
+ORACLE_ERR_LEN = 4
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        I64 = ctypes.c_int64
+        lib.oracle_quantize_rows.argtypes = [P, I64, I, I, P, P]
+        lib.oracle_quantize_rows.restype = None
+        lib.oracle_dequant_rows.argtypes = [P, P, I64, I, I, P]
+        lib.oracle_dequant_rows.restype = None
+        lib.oracle_append_contig.argtypes = [P, I, I, I, I, I, P, P, P, I]
+        lib.oracle_append_contig.restype = I
+        lib.oracle_append_paged.argtypes = [P, I, I, I, I, I, P, P, P, P, I, I, I]
+        lib.oracle_append_paged.restype = I
+        lib.oracle_decode_attn.argtypes = [P, I, I, I, I, I, P, P, P, P, I, I, P, I, I, P,
+                                           ctypes.c_double, P]
+        lib.oracle_decode_attn.restype = I
+        lib.oracle_cache_bytes.argtypes = [I64] * 6
+        lib.oracle_cache_bytes.restype = I64
+        lib.oracle_fp32_cache_bytes.argtypes = [I64] * 4
+        lib.oracle_fp32_cache_bytes.restype = I64
+        _lib = lib
+    return _lib
+
+
+def _cpu(t: torch.Tensor, dtype) -> torch.Tensor:
+    assert t.device.type == "cpu", "oracle works on CPU tensors"
+    assert t.dtype == dtype, (t.dtype, dtype)
+    return t.contiguous()
+
+
+def _bits16(x: torch.Tensor) -> torch.Tensor:
+    return _cpu(x, torch.bfloat16).view(torch.int16)
+
+
+def group_of(mode: str, D: int) -> int:
+    if mode == "per_token":
+        return D
+    if mode == "group32":
+        return 32
+    raise ValueError(mode)
+
+
+def quantize(x: torch.Tensor, mode: str = "per_token"):
+    """x bf16 [..., D] -> (u8 [..., D], fp32 scales [..., NG])."""
+    D = x.shape[-1]
+    grp = group_of(mode, D)
+    xb = _bits16(x)
+    rows = xb.numel() // D if D else 0
+    q = torch.empty(x.shape, dtype=torch.uint8)
+    s = torch.empty(*x.shape[:-1], D // grp, dtype=torch.float32)
+    _load().oracle_quantize_rows(xb.data_ptr(), rows, D, grp, q.data_ptr(), s.data_ptr())
+    return q, s
+
+
+def dequant(q: torch.Tensor, scale: torch.Tensor, mode: str = "per_token") -> torch.Tensor:
+    D = q.shape[-1]
+    grp = group_of(mode, D)
+    qc = _cpu(q, torch.uint8)
+    sc = _cpu(scale, torch.float32)
+    rows = qc.numel() // D if D else 0
+    out = torch.empty(q.shape, dtype=torch.float32)
+    _load().oracle_dequant_rows(qc.data_ptr(), sc.data_ptr(), rows, D, grp, out.data_ptr())
+    return out
+
+
+def append_contig(x_new, pos, cache, scale, mode="per_token") -> int:
+    """Quantize x_new bf16 [B,Hk,T,D] into cache u8 [B,Hk,max_seq,D] at pos[b]."""
+    B, Hk, T, D = x_new.shape
+    grp = group_of(mode, D)
+    assert cache.is_contiguous() and scale.is_contiguous()
+    xb = _bits16(x_new)
+    p = _cpu(pos, torch.int32)
+    return _load().oracle_append_contig(xb.data_ptr(), B, Hk, T, D, grp, p.data_ptr(),
+                                        cache.data_ptr(), scale.data_ptr(), cache.shape[2])
+
+
+def append_paged(x_new, pos, arena, scale, table, page_size=16, mode="per_token") -> int:
+    B, Hk, T, D = x_new.shape
+    grp = group_of(mode, D)
+    assert arena.is_contiguous() and scale.is_contiguous()
+    xb = _bits16(x_new)
+    p = _cpu(pos, torch.int32)
+    tb = _cpu(table, torch.int32)
+    return _load().oracle_append_paged(xb.data_ptr(), B, Hk, T, D, grp, p.data_ptr(),
+                                       arena.data_ptr(), scale.data_ptr(), tb.data_ptr(),
+                                       tb.shape[1], arena.shape[0], page_size)
+
+
+def decode_attn(q, k, v, k_scale, v_scale, seq_lens, attn_scale=None, mode="per_token",
+                Hk=None, page_size=0, table=None, return_err=False):
+    """fp64 decode attention over the dequantized INT8 cache.
+
+    q bf16 [B,Hq,D]; contiguous: k/v u8 [B,Hk,max_seq,D]; paged (page_size>0):
+    arenas u8 [num_pages,Hk,page_size,D] plus table int32 [B,max_pages].
+    Returns fp64 [B,Hq,D].
+    """
+    B, Hq, D = q.shape
+    grp = group_of(mode, D)
+    Hk = k.shape[1]
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    qb = _bits16(q)
+    kc, vc = _cpu(k, torch.uint8), _cpu(v, torch.uint8)
+    ks, vs = _cpu(k_scale, torch.float32), _cpu(v_scale, torch.float32)
+    sl = _cpu(seq_lens, torch.int32)
+    out = torch.empty(B, Hq, D, dtype=torch.float64)
+    if page_size > 0:
+        tb = _cpu(table, torch.int32)
+        err = _load().oracle_decode_attn(qb.data_ptr(), B, Hq, Hk, D, grp, kc.data_ptr(),
+                                         vc.data_ptr(), ks.data_ptr(), vs.data_ptr(), 0,
+                                         page_size, tb.data_ptr(), tb.shape[1], kc.shape[0],
+                                         sl.data_ptr(), float(attn_scale), out.data_ptr())
+    else:
+        err = _load().oracle_decode_attn(qb.data_ptr(), B, Hq, Hk, D, grp, kc.data_ptr(),
+                                         vc.data_ptr(), ks.data_ptr(), vs.data_ptr(),
+                                         kc.shape[2], 0, None, 0, 0, sl.data_ptr(),
+                                         float(attn_scale), out.data_ptr())
+    return (out, err) if return_err else out
+
+
+def cache_bytes(layers, Hk, seq, D, group, scale_bytes=4) -> int:
+    return int(_load().oracle_cache_bytes(layers, Hk, seq, D, group, scale_bytes))
+
+
+def fp32_cache_bytes(layers, Hk, seq, D) -> int:
+    return int(_load().oracle_fp32_cache_bytes(layers, Hk, seq, D))

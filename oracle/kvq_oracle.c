@@ -1,0 +1,233 @@
+/*
+ * kvq_oracle.c -- plain, slow CPU oracle for INT8 KV-cache append and decode
+ * attention.  TEST INFRASTRUCTURE ONLY: it exists to check the CUDA library,
+ * and only the tests, the smoke check and the benchmark's CPU-baseline leg
+ * may load it.  It shares no code, header or constant table with the CUDA
+ * library and must never be reached from the product path.
+ *
+ * What it follows (page title, item):
+ *  - Quantize: abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
+ *    CudaQuantizedKvCache::quantize_tensor -- per token, the absolute maximum
+ *    is floored at 1e-8, divided by 127 to give the scale, each element is
+ *    divided by the scale, rounded (Rust f32::round: half away from zero),
+ *    offset by +128 and clamped to [0, 255].  The scale is kept in fp32
+ *    (the page stores bf16; the fp32 reading is the one that makes
+ *    dequantization use the same scale the quantizer used).
+ *    abaddon 0.2.0-rc.2, src/kv_cache_quant.rs, module doc "Quantization
+ *    Strategy" states the same symmetric per-token method.
+ *  - Group-32 variant: realizar 0.8.5, src/cuda/executor/kv_cache_q8_init.rs,
+ *    init_kv_cache_q8_gpu (one fp32 scale per 32 values along head_dim,
+ *    head_dim divisible by 32) and combs-models 0.2.2, src/kv.rs,
+ *    KV_QUANT_GROUP / kv_quantize.  The per-element rule is the per-token one
+ *    applied to each 32-element group.
+ *  - Dequantize: abaddon 0.2.0-rc.2, kv_cache_quant.rs, QuantizedKvCache::
+ *    dequantize -- (u8 - 128) * scale, one fp32 multiply.
+ *  - Attention: combs-models 0.2.2, src/kv.rs, attend and repeat_kv --
+ *    scores = q . k * scale, softmax over the cached window, P . V; query
+ *    head h reads kv head h / (Hq/Hk) (heads repeated consecutively); a
+ *    single decode query attends to every cached position (no mask).
+ *    Computed here in fp64 over the dequantized fp32 cache.
+ *  - Paged layout: combs-models 0.2.2, src/kv.rs, PagedKVCache (arena
+ *    [num_pages, n_kv, page_size, head_dim]; logical token g lives in
+ *    physical page table[g / page_size], slot g % page_size).
+ *  - Memory accounting: realizar 0.8.5, kv_cache_q8_init.rs,
+ *    kv_cache_q8_memory_bytes and kv_cache_fp32_equivalent_bytes.
+ *
+ * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math.
+ * On x86-64 float arithmetic is IEEE single precision (SSE), so '/' is the
+ * correctly rounded fp32 quotient.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Error bits returned by the oracle's append / attention routines. */
+#define ORACLE_ERR_POS 1    /* append position outside [0, capacity - T] */
+#define ORACLE_ERR_PAGE 2   /* page table entry outside [0, num_pages) */
+#define ORACLE_ERR_LEN 4    /* sequence length outside [0, capacity] */
+
+/* bf16 is the upper half of an IEEE binary32; widening is exact. */
+static float widen_bf16(uint16_t h) {
+    uint32_t bits = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return f;
+}
+
+/* One group of n consecutive bf16 values -> n offset-128 bytes + one fp32 scale. */
+static void quantize_group(const uint16_t *x, int n, uint8_t *q, float *scale_out) {
+    float m = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(widen_bf16(x[i]));
+        if (a > m) m = a;
+    }
+    if (m < 1e-8f) m = 1e-8f;            /* max(|x|, 1e-8) */
+    float s = m / 127.0f;                /* scale = max / 127, fp32 division */
+    for (int i = 0; i < n; ++i) {
+        float r = widen_bf16(x[i]) / s;  /* fp32 division */
+        int v = (int)roundf(r) + 128;    /* roundf: half away from zero */
+        if (v < 0) v = 0;
+        if (v > 255) v = 255;
+        q[i] = (uint8_t)v;
+    }
+    *scale_out = s;
+}
+
+/* rows x D values; group = D (per token) or 32 (group-32). */
+void oracle_quantize_rows(const uint16_t *x, int64_t rows, int D, int group,
+                          uint8_t *q, float *scale) {
+    int ng = D / group;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int g = 0; g < ng; ++g)
+            quantize_group(x + r * D + (int64_t)g * group, group,
+                           q + r * D + (int64_t)g * group, scale + r * ng + g);
+}
+
+void oracle_dequant_rows(const uint8_t *q, const float *scale, int64_t rows, int D,
+                         int group, float *out) {
+    int ng = D / group;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int i = 0; i < D; ++i) {
+            float s = scale[r * ng + i / group];
+            out[r * D + i] = (float)((int)q[r * D + i] - 128) * s;
+        }
+}
+
+/*
+ * Contiguous append: new tokens x_new [B, Hk, T, D] go to positions
+ * pos[b] .. pos[b]+T-1 of cache [B, Hk, max_seq, D] / scales
+ * [B, Hk, max_seq, NG].  A batch row whose range leaves the capacity is
+ * skipped and flagged.
+ */
+int oracle_append_contig(const uint16_t *x_new, int B, int Hk, int T, int D, int group,
+                         const int32_t *pos, uint8_t *cache, float *scale, int max_seq) {
+    int err = 0, ng = D / group;
+    for (int b = 0; b < B; ++b) {
+        int64_t p0 = pos[b];
+        if (p0 < 0 || p0 + T > max_seq) { err |= ORACLE_ERR_POS; continue; }
+        for (int h = 0; h < Hk; ++h)
+            for (int t = 0; t < T; ++t) {
+                const uint16_t *src = x_new + (((int64_t)b * Hk + h) * T + t) * D;
+                int64_t row = ((int64_t)b * Hk + h) * max_seq + p0 + t;
+                oracle_quantize_rows(src, 1, D, group, cache + row * D, scale + row * ng);
+            }
+    }
+    return err;
+}
+
+/*
+ * Paged append: logical position g of sequence b goes to physical page
+ * table[b][g / page_size], slot g % page_size, arena [num_pages, Hk,
+ * page_size, D].  Tokens whose page entry is invalid are skipped and
+ * flagged.
+ */
+int oracle_append_paged(const uint16_t *x_new, int B, int Hk, int T, int D, int group,
+                        const int32_t *pos, uint8_t *arena, float *scale,
+                        const int32_t *table, int max_pages, int num_pages, int page_size) {
+    int err = 0, ng = D / group;
+    for (int b = 0; b < B; ++b) {
+        int64_t p0 = pos[b];
+        if (p0 < 0 || p0 + T > (int64_t)max_pages * page_size) { err |= ORACLE_ERR_POS; continue; }
+        for (int t = 0; t < T; ++t) {
+            int64_t g = p0 + t;
+            int32_t phys = table[(int64_t)b * max_pages + g / page_size];
+            int slot = (int)(g % page_size);
+            if (phys < 0 || phys >= num_pages) { err |= ORACLE_ERR_PAGE; continue; }
+            for (int h = 0; h < Hk; ++h) {
+                const uint16_t *src = x_new + (((int64_t)b * Hk + h) * T + t) * D;
+                int64_t row = ((int64_t)phys * Hk + h) * page_size + slot;
+                oracle_quantize_rows(src, 1, D, group, arena + row * D, scale + row * ng);
+            }
+        }
+    }
+    return err;
+}
+
+/*
+ * Decode attention for one new query per (sequence, q head) over the
+ * sequence's whole cached window, in fp64 over the dequantized cache.
+ *   q       bf16 [B, Hq, D]
+ *   page_size == 0: contiguous k/v [B, Hk, max_seq, D], scales [B, Hk, max_seq, NG]
+ *   page_size  > 0: arenas [num_pages, Hk, page_size, D], table [B, max_pages]
+ *   seq_lens int32 [B]; out fp64 [B, Hq, D].  A zero length gives a zero row.
+ */
+int oracle_decode_attn(const uint16_t *q, int B, int Hq, int Hk, int D, int group,
+                       const uint8_t *k, const uint8_t *v, const float *k_scale,
+                       const float *v_scale, int max_seq, int page_size,
+                       const int32_t *table, int max_pages, int num_pages,
+                       const int32_t *seq_lens, double attn_scale, double *out) {
+    int err = 0, ng = D / group, G = Hq / Hk;
+    int64_t cap = page_size > 0 ? (int64_t)max_pages * page_size : max_seq;
+    double *z = NULL, *kh = (double *)malloc(sizeof(double) * D);
+    double *acc = (double *)malloc(sizeof(double) * D);
+    int64_t *rows = NULL;
+    for (int b = 0; b < B; ++b) {
+        int64_t L = seq_lens[b];
+        if (L < 0 || L > cap) { err |= ORACLE_ERR_LEN; L = 0; }
+        /* physical row of each logical position (independent of kv head) */
+        rows = (int64_t *)realloc(rows, sizeof(int64_t) * (L > 0 ? L : 1));
+        z = (double *)realloc(z, sizeof(double) * (L > 0 ? L : 1));
+        int bad = 0;
+        for (int64_t t = 0; t < L; ++t) {
+            if (page_size > 0) {
+                int32_t phys = table[(int64_t)b * max_pages + t / page_size];
+                if (phys < 0 || phys >= num_pages) { bad = 1; break; }
+                rows[t] = (int64_t)phys * Hk * page_size + t % page_size; /* + h*page_size later */
+            } else {
+                rows[t] = (int64_t)b * Hk * max_seq + t;                   /* + h*max_seq later */
+            }
+        }
+        if (bad) { err |= ORACLE_ERR_PAGE; L = 0; }
+        for (int h = 0; h < Hq; ++h) {
+            int hk = h / G;
+            int64_t hstride = page_size > 0 ? page_size : max_seq;
+            double *o = out + ((int64_t)b * Hq + h) * D;
+            if (L == 0) { for (int d = 0; d < D; ++d) o[d] = 0.0; continue; }
+            const uint16_t *qh = q + ((int64_t)b * Hq + h) * D;
+            double zmax = -INFINITY;
+            for (int64_t t = 0; t < L; ++t) {
+                int64_t row = rows[t] + (int64_t)hk * hstride;
+                for (int d = 0; d < D; ++d) {
+                    float s = k_scale[row * ng + d / group];
+                    kh[d] = (double)((float)((int)k[row * D + d] - 128) * s);
+                }
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += (double)widen_bf16(qh[d]) * kh[d];
+                z[t] = dot * attn_scale;
+                if (z[t] > zmax) zmax = z[t];
+            }
+            double l = 0.0;
+            for (int d = 0; d < D; ++d) acc[d] = 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                int64_t row = rows[t] + (int64_t)hk * hstride;
+                double p = exp(z[t] - zmax);
+                l += p;
+                for (int d = 0; d < D; ++d) {
+                    float s = v_scale[row * ng + d / group];
+                    acc[d] += p * (double)((float)((int)v[row * D + d] - 128) * s);
+                }
+            }
+            for (int d = 0; d < D; ++d) o[d] = acc[d] / l;
+        }
+    }
+    free(z); free(kh); free(acc); free(rows);
+    return err;
+}
+
+/*
+ * Bytes of an INT8 cache: layers * 2 (K and V) * (values + scales), with one
+ * byte per value and scale_bytes per scale (4 for fp32), as in
+ * kv_cache_q8_memory_bytes; group = values per scale.
+ */
+int64_t oracle_cache_bytes(int64_t layers, int64_t Hk, int64_t seq, int64_t D, int64_t group,
+                           int64_t scale_bytes) {
+    int64_t values = Hk * seq * D;
+    int64_t scales = Hk * seq * (D / group);
+    return layers * 2 * (values + scales * scale_bytes);
+}
+
+/* fp32 equivalent, as in kv_cache_fp32_equivalent_bytes. */
+int64_t oracle_fp32_cache_bytes(int64_t layers, int64_t Hk, int64_t seq, int64_t D) {
+    return layers * 2 * Hk * seq * D * 4;
+}
