@@ -1,0 +1,563 @@
+#!/usr/bin/env python
+"""Benchmark of the INT8 KV-cache decode hot path on B200.
+
+One step = one pass of the whole hot path over one batch: for every layer of
+the workload, quantise-on-append the new token's K/V into the INT8 cache
+(kvq_append / kvq_append_paged), then decode attention on the INT8 cache
+(kvq_decode_attn: split kernel + combine).  The default workload is one
+Llama-3-8B-shaped decode (B=1, Hq=32, Hk=8, D=128, 4096 cached tokens + 1)
+repeated over 32 independent layer caches (277 MB, larger than the 126 MB L2,
+so consecutive reads of a layer never hit in L2).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+        [--workload llama3_8b_layer|tiny|batched_group32|paged|long_context]
+Multi-GPU: launched by torch.distributed.run, one rank per GPU; every rank
+runs its own replica of the workload (weak scaling, no data-path collective);
+the job time is the max over ranks.
+
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decode-attn INT8-KV GB/s & fraction of HBM peak; tokens/s per layer; append GB/s"
+DEFAULT_WORKLOAD = "llama3_8b_layer"
+LAYERS = {"llama3_8b_layer": 32}
+
+
+# ------------------------------------------------------------------ helpers
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def decode_bytes(wl, seq_lens, page_size=0):
+    """Algorithmic bytes of one decode call: K/V bytes + scales, Q, output,
+    page-table entries."""
+    ng = 1 if wl.mode == "per_token" else wl.D // 32
+    kv = sum(wl.Hk * L * (2 * wl.D + 2 * 4 * ng) for L in seq_lens)
+    qo = wl.B * wl.Hq * wl.D * (2 + 4)
+    pt = sum((L + 15) // 16 * 4 for L in seq_lens) if page_size else 0
+    return kv + qo + pt
+
+
+def append_bytes(wl, T):
+    ng = 1 if wl.mode == "per_token" else wl.D // 32
+    rd = T * wl.B * wl.Hk * wl.D * 2 * 2
+    wr = T * wl.B * wl.Hk * (2 * wl.D + 2 * 4 * ng)
+    return rd + wr
+
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons through NVML (the library
+    nvidia-smi reads) in a background thread while the timed region runs."""
+
+    HW_SLOW = 0x8
+    HW_THERMAL = 0x40
+    SW_THERMAL = 0x20
+    SW_POWER = 0x4
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples = []
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.error = str(e)
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
+        mhz = statistics.median(s[0] for s in self.samples)
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        names = []
+        for bit, name in [(self.HW_SLOW, "hw_slowdown"), (self.HW_THERMAL, "hw_thermal_slowdown"),
+                          (self.SW_THERMAL, "sw_thermal_slowdown"),
+                          (self.SW_POWER, "sw_power_cap")]:
+            if bits & bit:
+                names.append(name)
+        return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+def physical_gpu_index(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        parts = [p.strip() for p in vis.split(",") if p.strip()]
+        if local < len(parts) and parts[local].isdigit():
+            return int(parts[local])
+    return local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def decode_traffic_record():
+    """DRAM bytes per decode launch from a committed ncu summary, valid only if
+    the decode kernel source still has the hash recorded with it."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    src = os.path.join(ROOT, "decode_attention_kvq_b200", "csrc", "kvq_decode.cu")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if rec.get("kvq_decode_cu_sha256") != h:
+        return None
+    return rec
+
+
+# ---------------------------------------------------------------- workload
+class Layer:
+    """One layer's INT8 cache on the GPU with its decode-step inputs."""
+
+    def __init__(self, kvq, wl, inp, dev, keep_host=False):
+        self.wl = wl
+        B, Hk, D = wl.B, wl.Hk, wl.D
+        ng = 1 if wl.mode == "per_token" else D // 32
+        self.paged = wl.layout == "paged"
+        cached = inp.cached
+        self.seq_lens_list = [int(x) for x in inp.seq_lens]
+        self.hint = max(self.seq_lens_list)
+        if self.paged:
+            shape = (inp.num_pages, Hk, 16, D)
+            self.table = inp.page_table.to(dev)
+            self.k = torch.zeros(shape, dtype=torch.uint8, device=dev)
+            self.v = torch.zeros_like(self.k)
+            self.ks = torch.zeros(inp.num_pages, Hk, 16, ng, device=dev)
+            self.vs = torch.zeros_like(self.ks)
+            for b in range(B):
+                L = int(cached[b])
+                kv_k = inp.k_hist[b:b + 1, :, :L].contiguous().to(dev)
+                kv_v = inp.v_hist[b:b + 1, :, :L].contiguous().to(dev)
+                kvq.kvq_append_paged(kv_k, kv_v, torch.zeros(1, dtype=torch.int32, device=dev),
+                                     self.k, self.v, self.ks, self.vs,
+                                     self.table[b:b + 1].contiguous(), 16, wl.mode)
+        else:
+            S = self.hint
+            self.table = None
+            self.k = torch.zeros(B, Hk, S, D, dtype=torch.uint8, device=dev)
+            self.v = torch.zeros_like(self.k)
+            self.ks = torch.zeros(B, Hk, S, ng, device=dev)
+            self.vs = torch.zeros_like(self.ks)
+            Lmax = int(cached.max())
+            chunk = 8192
+            for p0 in range(0, Lmax, chunk):
+                T = min(chunk, Lmax - p0)
+                kvq.kvq_append(inp.k_hist[:, :, p0:p0 + T].contiguous().to(dev),
+                               inp.v_hist[:, :, p0:p0 + T].contiguous().to(dev),
+                               torch.full((B,), p0, dtype=torch.int32, device=dev),
+                               self.k, self.v, self.ks, self.vs, wl.mode)
+        self.k_new = inp.k_new.to(dev)
+        self.v_new = inp.v_new.to(dev)
+        self.q = inp.q.to(dev)
+        self.pos = cached.to(dev)
+        self.seq_lens = inp.seq_lens.to(dev)
+        self.out = torch.empty(B, wl.Hq, D, device=dev)
+        self.view = kvq.cache_view(self.k, self.v, self.ks, self.vs, self.table,
+                                   16 if self.paged else 0)
+        if keep_host:
+            self.host = inp
+        # prefill chunk re-append (long-context workload): rewrite the last chunk
+        self.chunk_T = wl.prefill_chunk
+        if self.chunk_T:
+            p0 = int(cached[0]) - self.chunk_T
+            self.chunk_k = inp.k_hist[:, :, p0:p0 + self.chunk_T].contiguous().to(dev)
+            self.chunk_v = inp.v_hist[:, :, p0:p0 + self.chunk_T].contiguous().to(dev)
+            self.chunk_pos = torch.full((B,), p0, dtype=torch.int32, device=dev)
+
+    def append(self, kvq):
+        if self.chunk_T:
+            kvq.kvq_append(self.chunk_k, self.chunk_v, self.chunk_pos, self.k, self.v, self.ks,
+                           self.vs, self.wl.mode)
+        if self.paged:
+            kvq.kvq_append_paged(self.k_new, self.v_new, self.pos, self.k, self.v, self.ks,
+                                 self.vs, self.table, 16, self.wl.mode)
+        else:
+            kvq.kvq_append(self.k_new, self.v_new, self.pos, self.k, self.v, self.ks, self.vs,
+                           self.wl.mode)
+
+    def decode(self, kvq, workspace):
+        kvq.kvq_decode_attn(self.q, self.k, self.v, self.ks, self.vs, self.seq_lens, self.hint,
+                            mode=self.wl.mode, out=self.out, workspace=workspace,
+                            page_table=self.table, page_size=16 if self.paged else 0,
+                            view=self.view)
+
+
+def build_layers(kvq, wl, n_layers, dev, keep_host=False):
+    layers = []
+    for i in range(n_layers):
+        inp = synth.make_decode_inputs(wl, seed=wl.seed + 7919 * i)
+        layers.append(Layer(kvq, wl, inp, dev, keep_host=keep_host and i == 0))
+        del inp
+    torch.cuda.synchronize(dev)
+    return layers
+
+
+# -------------------------------------------------------------- cpu oracle
+class OracleLayer:
+    """One layer of the workload held by the CPU oracle (single thread): the
+    history is quantised once at set-up; a step quantises the decode token
+    into the cache and runs fp64 decode attention."""
+
+    def __init__(self, wl, seed):
+        import oracle  # test infrastructure: used only by the CPU baseline legs
+        self.oracle = oracle
+        self.wl = wl
+        inp = synth.make_decode_inputs(wl, seed=seed)
+        self.inp = inp
+        B, Hk, D = wl.B, wl.Hk, wl.D
+        ng = 1 if wl.mode == "per_token" else D // 32
+        self.paged = wl.layout == "paged"
+        z1 = torch.zeros(1, dtype=torch.int32)
+        if self.paged:
+            shape = (inp.num_pages, Hk, 16, D)
+            self.k = torch.zeros(shape, dtype=torch.uint8)
+            self.v = torch.zeros_like(self.k)
+            self.ks = torch.zeros(inp.num_pages, Hk, 16, ng)
+            self.vs = torch.zeros_like(self.ks)
+            for b in range(B):
+                L = int(inp.cached[b])
+                tb = inp.page_table[b:b + 1].contiguous()
+                oracle.append_paged(inp.k_hist[b:b + 1, :, :L].contiguous(), z1, self.k, self.ks,
+                                    tb, 16, wl.mode)
+                oracle.append_paged(inp.v_hist[b:b + 1, :, :L].contiguous(), z1, self.v, self.vs,
+                                    tb, 16, wl.mode)
+        else:
+            S = int(inp.seq_lens.max())
+            self.k = torch.zeros(B, Hk, S, D, dtype=torch.uint8)
+            self.v = torch.zeros_like(self.k)
+            self.ks = torch.zeros(B, Hk, S, ng)
+            self.vs = torch.zeros_like(self.ks)
+            Lm = int(inp.cached.max())
+            zb = torch.zeros(B, dtype=torch.int32)
+            oracle.append_contig(inp.k_hist[:, :, :Lm].contiguous(), zb, self.k, self.ks, wl.mode)
+            oracle.append_contig(inp.v_hist[:, :, :Lm].contiguous(), zb, self.v, self.vs, wl.mode)
+        self.scale = float(torch.tensor(1.0 / math.sqrt(D), dtype=torch.float32))
+        self.nbytes = decode_bytes(wl, [int(x) for x in inp.seq_lens], 16 if self.paged else 0)
+        self.inp.k_hist = self.inp.v_hist = None
+
+    def step(self) -> float:
+        o, wl, inp = self.oracle, self.wl, self.inp
+        t0 = time.perf_counter()
+        if self.paged:
+            o.append_paged(inp.k_new, inp.cached, self.k, self.ks, inp.page_table, 16, wl.mode)
+            o.append_paged(inp.v_new, inp.cached, self.v, self.vs, inp.page_table, 16, wl.mode)
+            o.decode_attn(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale,
+                          wl.mode, page_size=16, table=inp.page_table)
+        else:
+            o.append_contig(inp.k_new, inp.cached, self.k, self.ks, wl.mode)
+            o.append_contig(inp.v_new, inp.cached, self.v, self.vs, wl.mode)
+            o.decode_attn(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale,
+                          wl.mode)
+        return time.perf_counter() - t0
+
+
+def oracle_sample(wl, n_steps_max, budget_s, n_distinct=4):
+    """Time the oracle on a bounded sample of the workload: layer steps cycled
+    over a few distinct layers until the time budget or the step cap is hit.
+    Returns (GB/s, sample description)."""
+    layers = [OracleLayer(wl, wl.seed + 7919 * i) for i in range(n_distinct)]
+    done, elapsed, nbytes = 0, 0.0, 0
+    while done < n_steps_max and (elapsed < budget_s or done == 0):
+        ly = layers[done % n_distinct]
+        elapsed += ly.step()
+        nbytes += ly.nbytes
+        done += 1
+    desc = (f"{done} layer steps of {wl.name} (append 1 token + fp64 decode attention) "
+            f"over {n_distinct} distinct layers, single-threaded C oracle, {elapsed:.2f} s timed")
+    return nbytes / elapsed / 1e9, desc
+
+
+# ------------------------------------------------------------------- arms
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    # each step is a bounded sample of the workload: one layer step of the
+    # oracle on a layer prepared once
+    ly = OracleLayer(wl, wl.seed)
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        el = ly.step()
+        if i >= args.warmup:
+            per_step.append((ly.nbytes / el / 1e9, el))
+    desc = (f"1 layer step of {wl.name} per step (append 1 token + fp64 decode attention), "
+            "single-threaded C oracle")
+    value = statistics.median(g for g, _ in per_step)
+    ms = 1000.0 * statistics.median(e for _, e in per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hk": wl.Hk, "D": wl.D,
+                   "seq_len": wl.len_hi + 1, "scale_mode": wl.mode, "layout": wl.layout,
+                   "sample": "1 layer step per step"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_kvq(args, wl):
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    import decode_attention_kvq_b200 as kvq  # fails loudly if libkvq.so is missing
+
+    n_layers = args.layers or LAYERS.get(wl.name, 1)
+    layers = build_layers(kvq, wl, n_layers, dev)
+    L0 = layers[0]
+    ws_bytes = kvq.kvq_decode_workspace_bytes(wl.B, wl.Hq, wl.Hk, wl.D, L0.hint)
+    workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    chunk, splits = kvq.kvq_decode_plan(wl.B, wl.Hk, L0.hint)
+    launches_per_layer = (1 + (1 if wl.prefill_chunk else 0)) + 1 + (1 if splits > 1 else 0)
+
+    stream = torch.cuda.Stream(dev)
+    # warm the library once eagerly, then capture the two phases as graphs
+    with torch.cuda.stream(stream):
+        for ly in layers:
+            ly.append(kvq)
+            ly.decode(kvq, workspace)
+    torch.cuda.synchronize(dev)
+    g_append, g_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_append, stream=stream):
+        for ly in layers:
+            ly.append(kvq)
+    with torch.cuda.graph(g_decode, stream=stream):
+        for ly in layers:
+            ly.decode(kvq, workspace)
+    torch.cuda.synchronize(dev)
+
+    K, W = args.steps, args.warmup
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            g_append.replay()
+            g_decode.replay()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(physical_gpu_index(local))
+    with sampler:
+        with torch.cuda.stream(stream):
+            for i in range(K):
+                ev[i][0].record(stream)
+                g_append.replay()
+                ev[i][1].record(stream)
+                g_decode.replay()
+                ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(dev)
+    t_append = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3          # s over K steps
+    t_decode = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_total = ev[0][0].elapsed_time(ev[-1][2]) / 1e3
+    t_total_max = reduce_max(t_total, dev)
+    t_decode_max = reduce_max(t_decode, dev)
+    t_append_max = reduce_max(t_append, dev)
+
+    dec_b = sum(decode_bytes(wl, ly.seq_lens_list, 16 if ly.paged else 0) for ly in layers)
+    app_b = sum(append_bytes(wl, 1) + (append_bytes(wl, wl.prefill_chunk) if wl.prefill_chunk
+                                       else 0) for _ in layers)
+    value = world * dec_b * K / t_decode_max / 1e9
+    per_layer_decode = t_decode_max / (K * n_layers)
+    per_layer_append = t_append_max / (K * n_layers)
+    tokens_per_s_per_layer = wl.B / (per_layer_append + per_layer_decode)
+    append_gbs = app_b * K / t_append_max / 1e9
+
+    peak, peak_kind = measured_peaks()
+    decode_call_bytes = dec_b / n_layers
+    achieved = decode_call_bytes / per_layer_decode / 1e9
+    traffic = decode_traffic_record()
+    traffic_val = None
+    if traffic and traffic.get("workload") == wl.name:
+        traffic_val = traffic.get("traffic_bytes_per_launch")
+
+    # ---- end to end through the public API from pinned host buffers
+    e2e = run_e2e(kvq, wl, layers, workspace, dev, K, W, world)
+
+    clocks = sampler.summary()
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(1e3 * t_total_max / K, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hk": wl.Hk, "D": wl.D,
+                   "seq_len": L0.hint, "scale_mode": wl.mode, "layout": wl.layout,
+                   "layers_per_step": n_layers, "parallelism": f"replicas x{world}",
+                   "l2": ("inputs larger than L2 (%.0f MB per step)"
+                          % ((dec_b + app_b) / 1e6)),
+                   "split_chunk": chunk, "splits": splits},
+        "tokens_per_s_per_layer": round(tokens_per_s_per_layer, 1),
+        "append_gbs": round(append_gbs, 2),
+        "decode_us_per_layer": round(per_layer_decode * 1e6, 3),
+        "append_us_per_layer": round(per_layer_append * 1e6, 3),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic_val,
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "kernel": "kvq_decode_attn call (split + combine kernels, per layer)",
+                     "algorithmic_bytes_per_launch": int(decode_call_bytes)},
+        "gpu_launches": launches_per_layer * n_layers * K,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, desc = oracle_sample(wl, args.cpu_layers, args.cpu_budget_s)
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1,
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        del g_append, g_decode
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(kvq, wl, layers, workspace, dev, K, W, world):
+    """Same metric through the public Python API with host buffers: each step
+    copies every layer's q / k_new / v_new from pinned host memory, runs
+    kvq_append + kvq_decode_attn eagerly, and copies the outputs back."""
+    n = len(layers)
+    h_q = [ly.q.cpu().pin_memory() for ly in layers]
+    h_k = [ly.k_new.cpu().pin_memory() for ly in layers]
+    h_v = [ly.v_new.cpu().pin_memory() for ly in layers]
+    h_out = [torch.empty_like(ly.out, device="cpu").pin_memory() for ly in layers]
+    h2d = sum(t.numel() * t.element_size() for t in h_q + h_k + h_v)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    stream = torch.cuda.Stream(dev)
+
+    def step():
+        with torch.cuda.stream(stream):
+            for i, ly in enumerate(layers):
+                ly.q.copy_(h_q[i], non_blocking=True)
+                ly.k_new.copy_(h_k[i], non_blocking=True)
+                ly.v_new.copy_(h_v[i], non_blocking=True)
+                ly.append(kvq)
+                ly.decode(kvq, workspace)
+                h_out[i].copy_(ly.out, non_blocking=True)
+
+    for _ in range(max(W, 1)):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(K):
+        step()
+    stop.record(stream)
+    stop.synchronize()
+    t = reduce_max(start.elapsed_time(stop) / 1e3, dev)
+    dec_b = sum(decode_bytes(wl, ly.seq_lens_list, 16 if ly.paged else 0) for ly in layers)
+    return {"value": round(world * dec_b * K / t / 1e9, 3), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(1e3 * t / K, 4), "layers_per_step": n}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
+    ap.add_argument("--workload", choices=list(synth.WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--layers", type=int, default=0, help="layer caches per step (0: default)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--cpu-layers", type=int, default=400)
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)     # timing rule: at least 3 untimed warm-up steps
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_kvq(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

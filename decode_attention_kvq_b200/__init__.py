@@ -1,0 +1,203 @@
+"""Thin Python binding over libkvq (include/kvq.h): INT8 KV-cache append and
+decode attention on B200 (sm_100a).
+
+Every function here only checks tensor arguments and marshals raw device
+pointers into the C ABI; all computation runs in the library's CUDA kernels.
+Importing this package fails loudly if libkvq.so has not been built
+(``python decode_attention_kvq_b200/build.py``); there is no CPU fallback.
+
+Functions take torch CUDA tensors (PyTorch supplies device memory and
+streams) and enqueue on the current CUDA stream unless ``stream`` is given.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional
+
+import torch
+
+from ._lib import KvqError, lib, LIB_PATH, check  # noqa: F401
+
+PER_TOKEN = 0
+GROUP32 = 1
+DEVERR_POS = 1
+DEVERR_PAGE = 2
+DEVERR_LEN = 4
+
+_MODES = {"per_token": PER_TOKEN, "group32": GROUP32, PER_TOKEN: PER_TOKEN, GROUP32: GROUP32}
+
+
+class CacheView(ctypes.Structure):
+    """Mirror of ``kvq_cache_view``."""
+    _fields_ = [
+        ("k", ctypes.c_void_p),
+        ("v", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p),
+        ("v_scale", ctypes.c_void_p),
+        ("page_size", ctypes.c_int32),
+        ("max_seq", ctypes.c_int32),
+        ("page_table", ctypes.c_void_p),
+        ("max_pages", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+    ]
+
+
+def _mode(mode) -> int:
+    try:
+        return _MODES[mode]
+    except KeyError:
+        raise ValueError(f"unknown scale mode {mode!r}") from None
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor") -> int:
+    if t is None:
+        return 0
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream, ref: torch.Tensor) -> int:
+    if stream is None:
+        return torch.cuda.current_stream(ref.device).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def num_groups(mode, D: int) -> int:
+    return 1 if _mode(mode) == PER_TOKEN else D // 32
+
+
+def kvq_append(k_new, v_new, pos, k_cache, v_cache, k_scale, v_scale, mode="per_token",
+               err=None, stream=None):
+    """Quantise k_new/v_new bf16 [B,Hk,T,D] into the contiguous cache at pos[b].
+
+    k_cache/v_cache u8 [B,Hk,max_seq,D]; k_scale/v_scale fp32 [B,Hk,max_seq,NG];
+    pos int32 [B]; err optional int32 [1] device error word.
+    """
+    B, Hk, T, D = k_new.shape
+    check(lib.kvq_append(
+        _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        B, Hk, T, D, _mode(mode), _ptr(pos, torch.int32, "pos"),
+        _ptr(k_cache, torch.uint8, "k_cache"), _ptr(v_cache, torch.uint8, "v_cache"),
+        _ptr(k_scale, torch.float32, "k_scale"), _ptr(v_scale, torch.float32, "v_scale"),
+        k_cache.shape[2], _ptr(err, torch.int32, "err"), _stream(stream, k_new)), "kvq_append")
+
+
+def kvq_append_paged(k_new, v_new, pos, k_arena, v_arena, k_scale, v_scale, page_table,
+                     page_size=16, mode="per_token", err=None, stream=None):
+    """Quantise k_new/v_new bf16 [B,Hk,T,D] into the paged arena.
+
+    k_arena/v_arena u8 [num_pages,Hk,page_size,D]; scales fp32
+    [num_pages,Hk,page_size,NG]; page_table int32 [B,max_pages].
+    """
+    B, Hk, T, D = k_new.shape
+    check(lib.kvq_append_paged(
+        _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        B, Hk, T, D, _mode(mode), _ptr(pos, torch.int32, "pos"),
+        _ptr(k_arena, torch.uint8, "k_arena"), _ptr(v_arena, torch.uint8, "v_arena"),
+        _ptr(k_scale, torch.float32, "k_scale"), _ptr(v_scale, torch.float32, "v_scale"),
+        _ptr(page_table, torch.int32, "page_table"), page_table.shape[1], k_arena.shape[0],
+        page_size, _ptr(err, torch.int32, "err"), _stream(stream, k_new)), "kvq_append_paged")
+
+
+def cache_view(k, v, k_scale, v_scale, page_table=None, page_size=0) -> CacheView:
+    """Build a kvq_cache_view over contiguous caches or paged arenas."""
+    cv = CacheView()
+    cv.k = _ptr(k, torch.uint8, "k")
+    cv.v = _ptr(v, torch.uint8, "v")
+    cv.k_scale = _ptr(k_scale, torch.float32, "k_scale")
+    cv.v_scale = _ptr(v_scale, torch.float32, "v_scale")
+    if page_size:
+        cv.page_size = page_size
+        cv.max_seq = 0
+        cv.page_table = _ptr(page_table, torch.int32, "page_table")
+        cv.max_pages = page_table.shape[1]
+        cv.num_pages = k.shape[0]
+    else:
+        cv.page_size = 0
+        cv.max_seq = k.shape[2]
+        cv.page_table = 0
+        cv.max_pages = 0
+        cv.num_pages = 0
+    return cv
+
+
+def kvq_decode_workspace_bytes(B, Hq, Hk, D, max_seq_len_hint, num_splits=0) -> int:
+    return int(lib.kvq_decode_workspace_bytes(B, Hq, Hk, D, max_seq_len_hint, num_splits))
+
+
+def kvq_decode_plan(B, Hk, max_seq_len_hint, num_splits=0, num_sms=0):
+    """(chunk tokens per split, splits of the longest sequence)."""
+    chunk, splits = ctypes.c_int(0), ctypes.c_int(0)
+    check(lib.kvq_decode_plan(B, Hk, max_seq_len_hint, num_splits, num_sms,
+                              ctypes.byref(chunk), ctypes.byref(splits)), "kvq_decode_plan")
+    return chunk.value, splits.value
+
+
+def kvq_decode_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *, Hk=None,
+                    page_table=None, page_size=0, attn_scale=None, mode="per_token",
+                    out=None, workspace=None, num_splits=0, err=None, stream=None,
+                    view: Optional[CacheView] = None):
+    """Decode attention of q bf16 [B,Hq,D] over the INT8 cache; returns fp32 [B,Hq,D].
+
+    Contiguous cache: k/v u8 [B,Hk,max_seq,D].  Paged: arenas
+    [num_pages,Hk,16,D] with page_table int32 [B,max_pages] and page_size=16.
+    seq_lens int32 [B] counts the cached tokens including the newest one.
+    """
+    B, Hq, D = q.shape
+    if Hk is None:
+        Hk = k.shape[1]
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    if view is None:
+        view = cache_view(k, v, k_scale, v_scale, page_table, page_size)
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
+    need = kvq_decode_workspace_bytes(B, Hq, Hk, D, max_seq_len_hint, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace, None, "workspace") if workspace is not None else 0
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    check(lib.kvq_decode_attn(
+        _ptr(q, torch.bfloat16, "q"), B, Hq, Hk, D, _mode(mode), ctypes.byref(view),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(max_seq_len_hint), float(attn_scale),
+        _ptr(out, torch.float32, "out"), ws_ptr, ws_bytes, int(num_splits),
+        _ptr(err, torch.int32, "err"), _stream(stream, q)), "kvq_decode_attn")
+    return out
+
+
+def kvq_dequant(q, scale, mode="per_token", out=None, stream=None):
+    """fp32 (byte - 128) * scale for q u8 [..., D], scale fp32 [..., NG]."""
+    D = q.shape[-1]
+    rows = q.numel() // D if D else 0
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    check(lib.kvq_dequant(_ptr(q, torch.uint8, "q"), _ptr(scale, torch.float32, "scale"),
+                          rows, D, _mode(mode), _ptr(out, torch.float32, "out"),
+                          _stream(stream, q)), "kvq_dequant")
+    return out
+
+
+def kvq_read_error(err, stream=None) -> int:
+    """Synchronise, return and clear the device error bits."""
+    bits = ctypes.c_int32(0)
+    st = lib.kvq_read_error(_ptr(err, torch.int32, "err"), ctypes.byref(bits),
+                            _stream(stream, err))
+    if st not in (0, 4):
+        check(st, "kvq_read_error")
+    return bits.value
+
+
+def kvq_cache_bytes(layers, Hk, seq, D, mode="per_token") -> int:
+    return int(lib.kvq_cache_bytes(layers, Hk, seq, D, _mode(mode)))
+
+
+def kvq_version() -> str:
+    return lib.kvq_version().decode()

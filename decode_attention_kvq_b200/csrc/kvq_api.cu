@@ -1,0 +1,219 @@
+// kvq_api.cu -- the extern "C" entry points declared in include/kvq.h:
+// argument validation, split planning and kernel launches.  No allocation,
+// no host<->device copies and no synchronisation happen here, except in
+// kvq_read_error, whose job is to read the device error word.
+#include <stdint.h>
+
+#include "kvq_internal.cuh"
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+constexpr int kMaxSplits = 4096;     // bound on splits per sequence (combine smem)
+
+kvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+kvq_status check_append_common(const uint16_t* k_new, const uint16_t* v_new, int B, int Hk, int T,
+                               int D, kvq_scale_mode mode, const int32_t* d_pos,
+                               const void* kd, const void* vd, const float* ks,
+                               const float* vs, const int32_t* d_err) {
+    if (!k_new || !v_new || !d_pos || !kd || !vd || !ks || !vs) return KVQ_ERR_INVALID_ARG;
+    if (B < 1 || Hk < 1 || T < 1 || D < 16 || D > 256 || (D % 16) != 0) return KVQ_ERR_INVALID_ARG;
+    if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_INVALID_ARG;
+    if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(kd, 16) || !aligned(vd, 16) ||
+        !aligned(ks, 4) || !aligned(vs, 4) || !aligned(d_pos, 4) || !aligned(d_err, 4))
+        return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
+kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk_out,
+                int* splits_out) {
+    if (B < 0 || Hk < 1 || hint < 0 || num_splits < 0) return KVQ_ERR_INVALID_ARG;
+    if (num_sms <= 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+    }
+    int64_t chunk;
+    if (hint <= 16) {
+        chunk = 16;
+    } else if (num_splits > 0) {
+        const int64_t s = num_splits < ceil_div(hint, 16) ? num_splits : ceil_div(hint, 16);
+        chunk = ceil_div(ceil_div(hint, s), 16) * 16;
+    } else {
+        // about two CTAs per SM over all (sequence, kv head) units, splits of
+        // 64..1024 tokens
+        const int64_t units = static_cast<int64_t>(B > 0 ? B : 1) * Hk;
+        const int64_t want = ceil_div(2ll * num_sms, units);
+        chunk = ceil_div(ceil_div(hint, want), 64) * 64;
+        if (chunk < 64) chunk = 64;
+        if (chunk > 1024) chunk = 1024;
+    }
+    if (ceil_div(hint, chunk) > kMaxSplits) chunk = ceil_div(ceil_div(hint, kMaxSplits), 16) * 16;
+    int64_t splits = ceil_div(hint, chunk);
+    if (splits < 1) splits = 1;
+    *chunk_out = static_cast<int>(chunk);
+    *splits_out = static_cast<int>(splits);
+    return KVQ_OK;
+}
+
+size_t workspace_for(int B, int Hq, int D, int splits) {
+    if (splits <= 1) return 0;
+    return static_cast<size_t>(B) * Hq * splits * (D + 2) * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_append(const uint16_t* k_new, const uint16_t* v_new, int B, int Hk, int T, int D,
+                      kvq_scale_mode mode, const int32_t* d_pos, uint8_t* k_cache,
+                      uint8_t* v_cache, float* k_scale, float* v_scale, int max_seq,
+                      int32_t* d_err, kvq_stream_t stream) {
+    kvq_status st = check_append_common(k_new, v_new, B, Hk, T, D, mode, d_pos, k_cache, v_cache,
+                                        k_scale, v_scale, d_err);
+    if (st != KVQ_OK) return st;
+    if (max_seq < 1) return KVQ_ERR_INVALID_ARG;
+    kvq::AppendParams p{};
+    p.k_new = k_new; p.v_new = v_new; p.k_dst = k_cache; p.v_dst = v_cache;
+    p.k_scale = k_scale; p.v_scale = v_scale; p.pos = d_pos; p.table = nullptr; p.d_err = d_err;
+    p.B = B; p.Hk = Hk; p.T = T; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
+    p.max_seq = max_seq; p.page_size = 0;
+    return from_cuda(kvq::launch_append(p, static_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_append_paged(const uint16_t* k_new, const uint16_t* v_new, int B, int Hk, int T,
+                            int D, kvq_scale_mode mode, const int32_t* d_pos, uint8_t* k_arena,
+                            uint8_t* v_arena, float* k_scale, float* v_scale,
+                            const int32_t* page_table, int max_pages, int num_pages,
+                            int page_size, int32_t* d_err, kvq_stream_t stream) {
+    kvq_status st = check_append_common(k_new, v_new, B, Hk, T, D, mode, d_pos, k_arena, v_arena,
+                                        k_scale, v_scale, d_err);
+    if (st != KVQ_OK) return st;
+    if (!page_table || !aligned(page_table, 4) || max_pages < 1 || num_pages < 1 ||
+        page_size != 16)
+        return KVQ_ERR_INVALID_ARG;
+    kvq::AppendParams p{};
+    p.k_new = k_new; p.v_new = v_new; p.k_dst = k_arena; p.v_dst = v_arena;
+    p.k_scale = k_scale; p.v_scale = v_scale; p.pos = d_pos; p.table = page_table;
+    p.d_err = d_err; p.B = B; p.Hk = Hk; p.T = T; p.D = D;
+    p.group32 = mode == KVQ_SCALE_GROUP32; p.max_seq = 0; p.page_size = page_size;
+    p.max_pages = max_pages; p.num_pages = num_pages;
+    return from_cuda(kvq::launch_append(p, static_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_decode_plan(int B, int Hk, int max_seq_len_hint, int num_splits, int num_sms,
+                           int* chunk, int* splits) {
+    if (!chunk || !splits) return KVQ_ERR_INVALID_ARG;
+    return plan(B, Hk, max_seq_len_hint, num_splits, num_sms, chunk, splits);
+}
+
+size_t kvq_decode_workspace_bytes(int B, int Hq, int Hk, int D, int max_seq_len_hint,
+                                  int num_splits) {
+    int chunk = 0, splits = 0;
+    if (B < 1 || Hq < 1 || D < 1) return 0;
+    if (plan(B, Hk, max_seq_len_hint, num_splits, 0, &chunk, &splits) != KVQ_OK) return 0;
+    return workspace_for(B, Hq, D, splits);
+}
+
+kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_scale_mode mode,
+                           const kvq_cache_view* kv, const int32_t* d_seq_lens,
+                           int max_seq_len_hint, float attn_scale, float* out, void* workspace,
+                           size_t workspace_bytes, int num_splits, int32_t* d_err,
+                           kvq_stream_t stream) {
+    if (!q || !kv || !kv->k || !kv->v || !kv->k_scale || !kv->v_scale || !d_seq_lens || !out)
+        return KVQ_ERR_INVALID_ARG;
+    if (B < 0 || Hq < 1 || Hk < 1 || (Hq % Hk) != 0 || D < 16 || (D % 16) != 0 ||
+        max_seq_len_hint < 0 || num_splits < 0 || B > 65535 || Hk > 65535)
+        return KVQ_ERR_INVALID_ARG;
+    if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_INVALID_ARG;
+    if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
+    if (kv->page_size == 16) {
+        if (!kv->page_table || !aligned(kv->page_table, 4) || kv->max_pages < 1 ||
+            kv->num_pages < 1)
+            return KVQ_ERR_INVALID_ARG;
+    } else if (kv->page_size == 0) {
+        if (kv->max_seq < 1) return KVQ_ERR_INVALID_ARG;
+    } else {
+        return KVQ_ERR_INVALID_ARG;
+    }
+    if (!aligned(q, 16) || !aligned(kv->k, 16) || !aligned(kv->v, 16) ||
+        !aligned(kv->k_scale, 4) || !aligned(kv->v_scale, 4) || !aligned(d_seq_lens, 4) ||
+        !aligned(out, 16) || !aligned(workspace, 16) || !aligned(d_err, 4))
+        return KVQ_ERR_INVALID_ARG;
+    const int G = Hq / Hk;
+    if (D != 64 && D != 128) return KVQ_ERR_UNSUPPORTED;
+    if (G > 8) return KVQ_ERR_UNSUPPORTED;
+    if (B == 0) return KVQ_OK;
+
+    int chunk = 0, splits = 0;
+    kvq_status st = plan(B, Hk, max_seq_len_hint, num_splits, 0, &chunk, &splits);
+    if (st != KVQ_OK) return st;
+    const size_t need = workspace_for(B, Hq, D, splits);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return KVQ_ERR_INVALID_ARG;
+
+    kvq::DecodeParams p{};
+    p.q = q; p.k = kv->k; p.v = kv->v; p.k_scale = kv->k_scale; p.v_scale = kv->v_scale;
+    p.table = kv->page_table; p.seq_lens = d_seq_lens; p.out = out; p.d_err = d_err;
+    float* ws = static_cast<float*>(workspace);
+    const size_t n_part = static_cast<size_t>(B) * Hq * splits;
+    p.ws_o = ws;
+    p.ws_m = ws ? ws + n_part * D : nullptr;
+    p.ws_l = ws ? ws + n_part * (D + 1) : nullptr;
+    p.B = B; p.Hq = Hq; p.Hk = Hk; p.G = G; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
+    p.page_size = kv->page_size; p.max_seq = kv->max_seq; p.max_pages = kv->max_pages;
+    p.num_pages = kv->num_pages; p.chunk = chunk; p.splits = splits;
+    p.scale_log2 = attn_scale * 1.4426950408889634f;
+    return from_cuda(kvq::launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_dequant(const uint8_t* q, const float* scale, int64_t rows, int D,
+                       kvq_scale_mode mode, float* out, kvq_stream_t stream) {
+    if (rows < 0 || D < 16 || (D % 16) != 0) return KVQ_ERR_INVALID_ARG;
+    if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_INVALID_ARG;
+    if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
+    if (rows == 0) return KVQ_OK;
+    if (!q || !scale || !out || !aligned(q, 16) || !aligned(out, 16) || !aligned(scale, 4))
+        return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_dequant(q, scale, rows, D, mode == KVQ_SCALE_GROUP32, out,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+const char* kvq_status_string(kvq_status status) {
+    switch (status) {
+        case KVQ_OK: return "KVQ_OK";
+        case KVQ_ERR_INVALID_ARG: return "KVQ_ERR_INVALID_ARG";
+        case KVQ_ERR_UNSUPPORTED: return "KVQ_ERR_UNSUPPORTED";
+        case KVQ_ERR_CUDA: return "KVQ_ERR_CUDA";
+        case KVQ_ERR_DEVICE_FLAG: return "KVQ_ERR_DEVICE_FLAG";
+    }
+    return "KVQ_UNKNOWN_STATUS";
+}
+
+kvq_status kvq_read_error(int32_t* d_err, int32_t* bits, kvq_stream_t stream) {
+    if (!d_err || !aligned(d_err, 4)) return KVQ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t h = 0;
+    if (cudaMemcpyAsync(&h, d_err, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    if (cudaMemsetAsync(d_err, 0, sizeof(int32_t), s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    if (bits) *bits = h;
+    return h ? KVQ_ERR_DEVICE_FLAG : KVQ_OK;
+}
+
+int64_t kvq_cache_bytes(int64_t layers, int64_t Hk, int64_t seq, int D, kvq_scale_mode mode) {
+    const int64_t ng = mode == KVQ_SCALE_GROUP32 ? D / 32 : 1;
+    return layers * 2 * Hk * seq * (static_cast<int64_t>(D) + 4 * ng);
+}
+
+const char* kvq_version(void) { return "kvq 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

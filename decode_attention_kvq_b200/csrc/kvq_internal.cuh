@@ -1,0 +1,68 @@
+// kvq_internal.cuh -- declarations shared by the CUDA translation units of
+// libkvq (launchers, parameter blocks, small device helpers).  Not part of
+// the public ABI; the public declarations live in include/kvq.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+// bf16 bits -> fp32 (exact widening: bf16 is the top half of binary32).
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h16) {
+    return __uint_as_float(h16 << 16);
+}
+
+__device__ __forceinline__ void raise_flag(int32_t* d_err, uint32_t bits) {
+    if (d_err) atomicOr(reinterpret_cast<int*>(d_err), static_cast<int>(bits));
+}
+
+// ---------------------------------------------------------------- append
+struct AppendParams {
+    const uint16_t* k_new;   // [B, Hk, T, D] bf16
+    const uint16_t* v_new;
+    uint8_t* k_dst;          // contiguous cache or paged arena
+    uint8_t* v_dst;
+    float* k_scale;
+    float* v_scale;
+    const int32_t* pos;      // [B]
+    const int32_t* table;    // paged only: [B, max_pages]
+    int32_t* d_err;
+    int B, Hk, T, D;
+    int group32;             // 1: 32-value groups, 0: one scale per row
+    int max_seq;             // contiguous capacity
+    int page_size;           // 0: contiguous, else paged
+    int max_pages, num_pages;
+};
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+
+// --------------------------------------------------------------- dequant
+cudaError_t launch_dequant(const uint8_t* q, const float* scale, int64_t rows, int D,
+                           int group32, float* out, cudaStream_t s);
+
+// ---------------------------------------------------------------- decode
+struct DecodeParams {
+    const uint16_t* q;       // [B, Hq, D] bf16
+    const uint8_t* k;        // cache / arena
+    const uint8_t* v;
+    const float* k_scale;
+    const float* v_scale;
+    const int32_t* table;    // paged: [B, max_pages]
+    const int32_t* seq_lens; // [B]
+    float* out;              // [B, Hq, D]
+    float* ws_o;             // [B*Hq, splits, D] partial outputs (unnormalised)
+    float* ws_m;             // [B*Hq, splits] running max (log2 domain)
+    float* ws_l;             // [B*Hq, splits] running sum
+    int32_t* d_err;
+    int B, Hq, Hk, G, D;
+    int group32;
+    int page_size, max_seq, max_pages, num_pages;
+    int chunk;               // KV tokens per split
+    int splits;              // splits of the longest sequence (grid.x)
+    float scale_log2;        // attn_scale * log2(e)
+};
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+
+}  // namespace kvq

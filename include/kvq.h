@@ -1,0 +1,214 @@
+/*
+ * kvq.h -- C ABI of libkvq: INT8 KV-cache quantisation on append and decode
+ * attention computed directly on the INT8 cache, for NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ *  - All tensor arguments are raw pointers to caller-owned DEVICE memory,
+ *    densely packed in the row-major layout given for each argument.  The
+ *    library never allocates, frees or copies host<->device inside these
+ *    calls, and never synchronises the stream (except kvq_read_error).
+ *  - bf16 tensors are passed as uint16_t* (the raw bf16 bits).
+ *  - Every pointer that is read or written with vector loads must be 16-byte
+ *    aligned (all tensor arguments except d_pos, d_seq_lens, page_table and
+ *    d_err, which need 4-byte alignment).  torch allocations satisfy this.
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *    default stream.  All work is enqueued on it, in order.
+ *  - Argument faults the host can see are reported synchronously as
+ *    KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED before anything is enqueued.
+ *    A failed launch returns KVQ_ERR_CUDA.
+ *  - Faults only the device can see (a write position beyond the cache
+ *    capacity, a page-table entry outside the arena, a sequence length
+ *    beyond the capacity) never trap: the offending row / page is skipped
+ *    and the matching KVQ_DEVERR_* bit is OR-ed into *d_err when d_err is
+ *    not NULL.  kvq_read_error fetches and clears that word.
+ *
+ * Quantisation (both append calls), per (token, kv head) or per 32-value
+ * group along head_dim: m = max(max_i |x_i|, 1e-8); s = m / 127 (IEEE fp32
+ * division); byte_i = clamp(round_half_away_from_zero(x_i / s) + 128, 0, 255)
+ * with x_i / s an IEEE fp32 division; s is stored as fp32.  The result is
+ * bit-exact with that definition.  Source: abaddon 0.2.0-rc.1,
+ * src/kv_cache_quant_cuda.rs, CudaQuantizedKvCache::quantize_tensor (per
+ * token, offset-128 bytes); abaddon 0.2.0-rc.2, src/kv_cache_quant.rs, module
+ * doc "Quantization Strategy"; group-32 fp32 scales as in realizar 0.8.5,
+ * src/cuda/executor/kv_cache_q8_init.rs, init_kv_cache_q8_gpu, and
+ * combs-models 0.2.2, src/kv.rs, kv_quantize (KV_QUANT_GROUP = 32).
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvq_status {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, too small workspace */
+    KVQ_ERR_UNSUPPORTED = 2,   /* valid but not built: head_dim or GQA group outside the kernels' set */
+    KVQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    KVQ_ERR_DEVICE_FLAG = 4    /* kvq_read_error found device-side error bits */
+} kvq_status;
+
+typedef enum kvq_scale_mode {
+    KVQ_SCALE_PER_TOKEN = 0,   /* one fp32 scale per (token, kv head): NG = 1 */
+    KVQ_SCALE_GROUP32 = 1      /* one fp32 scale per 32 values along head_dim: NG = D / 32 */
+} kvq_scale_mode;
+
+/* Device-side error bits (OR-ed into *d_err). */
+#define KVQ_DEVERR_POS 1u    /* append range [pos, pos + T) outside [0, capacity) */
+#define KVQ_DEVERR_PAGE 2u   /* page-table entry outside [0, num_pages) in the used range */
+#define KVQ_DEVERR_LEN 4u    /* decode sequence length outside [0, capacity] */
+
+typedef void *kvq_stream_t;  /* cudaStream_t */
+
+/*
+ * kvq_append -- quantise T new tokens per (sequence, kv head) and write them
+ * in place into a contiguous INT8 cache.
+ *   k_new, v_new  bf16 [B, Hk, T, D]        new keys / values (read)
+ *   d_pos         int32 [B]                 first write position of each sequence
+ *   k_cache, v_cache  u8 [B, Hk, max_seq, D]   offset-128 bytes (written at
+ *                                              positions d_pos[b] .. d_pos[b]+T-1)
+ *   k_scale, v_scale  fp32 [B, Hk, max_seq, NG]
+ *   d_err         int32 [1] or NULL         device error word (KVQ_DEVERR_POS)
+ * Requirements: B, Hk, T >= 1; 16 <= D <= 256, D % 16 == 0; GROUP32 needs
+ * D % 32 == 0; max_seq >= 1.  Positions are arbitrary within capacity (a
+ * later append may overwrite a slot); a sequence whose range leaves
+ * [0, max_seq) is skipped and flagged.
+ * Source: abaddon 0.2.0-rc.1, kv_cache_quant_cuda.rs, CudaQuantizedKvCache::
+ * append (input layout [batch, kv_heads, new_seq, head_dim]); realizar 0.8.5,
+ * kv_cache_q8_init.rs, write_kv_q8 (write at an explicit position below the
+ * capacity, capacity-strided per head).
+ */
+kvq_status kvq_append(const uint16_t *k_new, const uint16_t *v_new, int B, int Hk, int T, int D,
+                      kvq_scale_mode mode, const int32_t *d_pos, uint8_t *k_cache,
+                      uint8_t *v_cache, float *k_scale, float *v_scale, int max_seq,
+                      int32_t *d_err, kvq_stream_t stream);
+
+/*
+ * kvq_append_paged -- as kvq_append, but the cache is a paged arena.
+ *   k_arena, v_arena  u8 [num_pages, Hk, page_size, D]
+ *   k_scale, v_scale  fp32 [num_pages, Hk, page_size, NG]
+ *   page_table    int32 [B, max_pages]      physical page of each logical page
+ * Logical position g of sequence b is stored in physical page
+ * page_table[b][g / page_size], slot g % page_size.  page_size must be 16.
+ * A token whose page entry is outside [0, num_pages) is skipped and flagged
+ * with KVQ_DEVERR_PAGE; a range beyond max_pages * page_size with
+ * KVQ_DEVERR_POS.
+ * Source: combs-models 0.2.2, src/kv.rs, PagedKVCache (arena layout,
+ * DEFAULT_PAGE_SIZE = 16) and PagedKVCache::attention_opts (slot arithmetic;
+ * each token quantised once, never re-quantised).
+ */
+kvq_status kvq_append_paged(const uint16_t *k_new, const uint16_t *v_new, int B, int Hk, int T,
+                            int D, kvq_scale_mode mode, const int32_t *d_pos, uint8_t *k_arena,
+                            uint8_t *v_arena, float *k_scale, float *v_scale,
+                            const int32_t *page_table, int max_pages, int num_pages,
+                            int page_size, int32_t *d_err, kvq_stream_t stream);
+
+/*
+ * Where decode attention finds the INT8 cache.  page_size == 0 selects the
+ * contiguous layout of kvq_append, page_size == 16 the arena of
+ * kvq_append_paged.  Unused fields are ignored.
+ */
+typedef struct kvq_cache_view {
+    const uint8_t *k;          /* [B, Hk, max_seq, D] or [num_pages, Hk, page_size, D] */
+    const uint8_t *v;
+    const float *k_scale;      /* [B, Hk, max_seq, NG] or [num_pages, Hk, page_size, NG] */
+    const float *v_scale;
+    int32_t page_size;         /* 0 (contiguous) or 16 (paged) */
+    int32_t max_seq;           /* contiguous: capacity per (sequence, kv head) */
+    const int32_t *page_table; /* paged: int32 [B, max_pages] (device) */
+    int32_t max_pages;         /* paged */
+    int32_t num_pages;         /* paged: pages in the arena */
+} kvq_cache_view;
+
+/*
+ * kvq_decode_attn -- one decode query per (sequence, q head) attending to
+ * the sequence's whole cached window, with dequantisation fused into Q.K^T
+ * and P.V:
+ *   z_t = attn_scale * sum_d q_d * (k_t,d - 128) * sk_t,grp(d)
+ *   out = sum_t softmax(z)_t * (v_t,d - 128) * sv_t,grp(d)
+ * Query head h reads kv head h / (Hq / Hk) (GQA, heads repeated
+ * consecutively).  A decode query is the newest position, so the causal
+ * window is the whole cache: no mask is applied.
+ *   q           bf16 [B, Hq, D]
+ *   kv          cache view (see above)
+ *   d_seq_lens  int32 [B]   cached length of each sequence INCLUDING the token
+ *                           just appended; 0 gives a zero output row
+ *   max_seq_len_hint  host upper bound of d_seq_lens (plans the split-K grid;
+ *                     positions beyond it are not read)
+ *   attn_scale  usually 1 / sqrt(D)
+ *   out         fp32 [B, Hq, D]
+ *   workspace   device scratch of at least kvq_decode_workspace_bytes(...)
+ *               bytes (same B, Hq, Hk, D, hint, num_splits), 16-byte
+ *               aligned; may be NULL when that size is 0.  Contents on entry
+ *               are ignored.
+ *   num_splits  0 = automatic; otherwise the requested number of KV splits
+ *               per sequence (split-K / flash-decoding)
+ *   d_err       int32 [1] or NULL (KVQ_DEVERR_LEN, KVQ_DEVERR_PAGE)
+ * Requirements: Hq % Hk == 0 and Hq / Hk <= 16; D in {64, 128}; GROUP32
+ * needs D % 32 == 0.
+ * Source: abaddon 0.2.0-rc.1, kv_cache_quant_cuda.rs, module doc "Fused
+ * approach" and CudaQuantizedKvCache::forward_attention (scores with
+ * on-the-fly K dequantisation, softmax, P.V with on-the-fly V
+ * dequantisation); combs-models 0.2.2, src/kv.rs, attend and repeat_kv
+ * (scale applied after the dot product, GQA mapping, a single decode query
+ * needs no mask).  Split-K with an online softmax and a combine step is this
+ * library's own (flash-decoding), not from those pages.
+ */
+kvq_status kvq_decode_attn(const uint16_t *q, int B, int Hq, int Hk, int D, kvq_scale_mode mode,
+                           const kvq_cache_view *kv, const int32_t *d_seq_lens,
+                           int max_seq_len_hint, float attn_scale, float *out, void *workspace,
+                           size_t workspace_bytes, int num_splits, int32_t *d_err,
+                           kvq_stream_t stream);
+
+/* Workspace bytes kvq_decode_attn needs for these arguments (0 when no split is needed). */
+size_t kvq_decode_workspace_bytes(int B, int Hq, int Hk, int D, int max_seq_len_hint,
+                                  int num_splits);
+
+/*
+ * Split plan kvq_decode_attn uses: KV tokens per split (*chunk) and the
+ * largest number of splits of any sequence (*splits).  num_sms <= 0 means the
+ * current device's SM count.  Returns KVQ_ERR_INVALID_ARG on bad sizes.
+ */
+kvq_status kvq_decode_plan(int B, int Hk, int max_seq_len_hint, int num_splits, int num_sms,
+                           int *chunk, int *splits);
+
+/*
+ * kvq_dequant -- x = (byte - 128) * scale, one fp32 multiply per element,
+ * bit-exact.
+ *   q      u8 [rows, D];  scale fp32 [rows, NG];  out fp32 [rows, D]
+ * Requirements: rows >= 0; 16 <= D, D % 16 == 0; GROUP32 needs D % 32 == 0.
+ * Source: abaddon 0.2.0-rc.2, kv_cache_quant.rs, QuantizedKvCache::
+ * dequantize; abaddon 0.2.0-rc.1, kv_cache_quant_cuda.rs, int8_dequant_bf16
+ * (this library writes fp32 instead of bf16); realizar 0.8.5,
+ * kv_cache_q8_init.rs, read_kv_q8.
+ */
+kvq_status kvq_dequant(const uint8_t *q, const float *scale, int64_t rows, int D,
+                       kvq_scale_mode mode, float *out, kvq_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char *kvq_status_string(kvq_status status);
+
+/*
+ * Synchronises `stream`, copies the device error word to *bits (may be NULL)
+ * and clears it.  Returns KVQ_OK when it was 0, KVQ_ERR_DEVICE_FLAG when any
+ * bit was set, KVQ_ERR_CUDA on a runtime failure.
+ */
+kvq_status kvq_read_error(int32_t *d_err, int32_t *bits, kvq_stream_t stream);
+
+/*
+ * Bytes of an INT8 cache with fp32 scales: layers * 2 * Hk * seq * (D + 4 * NG).
+ * Source: realizar 0.8.5, kv_cache_q8_init.rs, kv_cache_q8_memory_bytes.
+ */
+int64_t kvq_cache_bytes(int64_t layers, int64_t Hk, int64_t seq, int D, kvq_scale_mode mode);
+
+/* Library version string. */
+const char *kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */
