@@ -148,7 +148,11 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
         return KVQ_ERR_INVALID_ARG;
     const int G = Hq / Hk;
     if (D != 64 && D != 128) return KVQ_ERR_UNSUPPORTED;
-    if (G > 8) return KVQ_ERR_UNSUPPORTED;
+    if (G > 16) return KVQ_ERR_UNSUPPORTED;
+    // TMA row coordinates are 32-bit
+    const int64_t rows = kv->page_size ? static_cast<int64_t>(kv->num_pages) * Hk * 16
+                                       : static_cast<int64_t>(B) * Hk * kv->max_seq;
+    if (rows >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
     if (B == 0) return KVQ_OK;
 
     int chunk = 0, splits = 0;

@@ -1,0 +1,691 @@
+// kvq_decode_tc.cu -- split-K decode attention on the INT8 cache for sm_100a:
+// TMA-staged K/V tiles, tensor-core Q.K^T and P.V on exact integer operands
+// with the dequantisation scales applied outside the MMA.
+//
+// Method (what is computed): abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
+// module doc "Fused approach" -- Q.K^T with K dequantised on the fly,
+// softmax, P.V with V dequantised on the fly; combs-models 0.2.2, src/kv.rs,
+// attend / repeat_kv -- scale after the dot product, query head h reads kv
+// head h / G, a decode query attends to the whole cache.  Split-K with an
+// online softmax is this library's own (flash-decoding).
+//
+// How (sm_100a):
+//  * CTA = 4 consumer warps + 1 producer warp, one CTA per (sequence, kv
+//    head, split).  The producer streams 64-token stages of K and V bytes
+//    into shared memory with TMA tile loads (2-D tensor maps over the cache
+//    rows, 128-byte swizzle for D=128) and the fp32 scales with cp.async;
+//    both complete on the stage's mbarrier.  4 stages are in flight.
+//  * Consumer warp w owns the stages w, w+4, ...: for each 16-token slice it
+//    runs S = Q.K^T with mma.sync m16n8k16 (f16 in, f32 accumulate), rows =
+//    query heads of the GQA group (padded to 16), columns = tokens.  The
+//    operands are exact: K enters as the integers (byte - 128) built in
+//    registers (1024 + byte spliced into an f16 mantissa, minus 1152), and Q
+//    enters as f16 after a per-head power-of-two prescale (bf16 has 8
+//    significant bits, f16 has 11, so q * 2^s is exact), so the f32
+//    accumulators hold sum_d q_d (k_d - 128) up to accumulation rounding.
+//    The K scale (per token, or per 32-value group with one accumulator per
+//    group), 2^-s, attn_scale and log2(e) are applied to the accumulator.
+//  * Online softmax in base 2 per head row; P' = 2^(z-m) * v_scale(token) is
+//    rounded to f16 and multiplied with the exact integers (v - 128), so the
+//    V scale is folded into P (per 32-value group in group-32 mode).
+//  * Token order inside each 16-token slice and the d order of the MMA
+//    k-dimension are permuted so that every shared-memory load of the
+//    swizzled tiles is free of bank conflicts (sigma below).
+//  * The four warps' (m, l, o) are merged in shared memory; the CTA writes
+//    its split (o, m, l) or, for a single-split sequence, the final row.
+#include <cuda.h>
+#include <math.h>
+
+#include "kvq_internal.cuh"
+#include "kvq_ptx.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int TT = 64;                 // tokens per stage
+constexpr int NCW = 4;                 // consumer warps
+constexpr int NTHREADS = (NCW + 1) * 32;
+constexpr int NST = 4;                 // stages in flight
+
+// Row (inside an 8-token group) that holds MMA column n of the K operand and
+// MMA k-index n of the V operand: sigma = {0, 2, 4, 6, 3, 1, 7, 5}.  Under the
+// 128-byte swizzle (16-byte chunk index XOR row % 8) this makes the K loads
+// (rows sigma(g), 8 bytes at 32*G + 8*t) and the V loads (rows sigma(2t),
+// sigma(2t+1), 16 bytes at 16*g) of a warp hit distinct banks: the rows a
+// load instruction touches differ in bits 1..2.
+__device__ __forceinline__ int sigma(int x) { return x < 4 ? 2 * x : ((2 * x - 7) ^ 2); }
+
+template <int D, bool G32>
+struct Layout {
+    static constexpr int NG = G32 ? D / 32 : 1;
+    static constexpr int KV_BYTES = TT * D;
+    static constexpr int SC_FLOATS = TT * NG;
+    static constexpr int STAGE = ((2 * KV_BYTES + 2 * SC_FLOATS * 4) + 1023) / 1024 * 1024;
+    static constexpr int BAR_OFF = NST * STAGE;
+    static constexpr int SMEM = BAR_OFF + 2 * NST * 8 + 1024;   // + base alignment slack
+};
+
+// byte offset of (row, byte) inside a swizzled K or V stage tile
+template <int D>
+__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t byte) {
+    if constexpr (D == 128) {
+        return row * 128u + ((((byte >> 4) ^ row) & 7u) << 4) + (byte & 15u);
+    } else {  // D == 64, 64-byte swizzle
+        return row * 64u + ((((byte >> 4) ^ (row >> 1)) & 3u) << 4) + (byte & 15u);
+    }
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float ldsf(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
+}
+
+template <int D, bool G32, bool PAGED, bool G16>
+__global__ void __launch_bounds__(NTHREADS)
+decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                DecodeParams p) {
+    using Lay = Layout<D, G32>;
+    constexpr int NG = Lay::NG;
+    constexpr int KS = D / 16;          // MMA k-steps over head_dim
+    constexpr int NGRP = D / 32;        // 32-value groups over head_dim
+    constexpr int NTD = D / 8;          // output n-tiles over head_dim
+    constexpr int NACC = G32 ? NG : 1;  // score accumulators per n-tile
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.G;
+
+    const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
+    const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
+    int L = p.seq_lens[b];
+    if (L < 0 || L > lim) {
+        if (j == 0 && hk == 0 && threadIdx.x == 0) raise_flag(p.d_err, KVQ_DEVERR_LEN);
+        L = 0;
+    }
+    if (L == 0) {
+        if (j == 0)
+            for (int i = threadIdx.x; i < G * D; i += NTHREADS)
+                p.out[(static_cast<int64_t>(b) * p.Hq + hk * G) * D + i] = 0.f;
+        return;
+    }
+    const int t0 = j * p.chunk;
+    if (t0 >= L) return;
+    const int t1 = min(t0 + p.chunk, L);
+    const int nsplit = (L + p.chunk - 1) / p.chunk;
+    const int ntiles = (t1 - t0 + TT - 1) / TT;
+
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const uint32_t bar_full = sbase + Lay::BAR_OFF;
+    const uint32_t bar_empty = bar_full + NST * 8;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            ptx::mbar_init(bar_full + 8 * s, 1 + 32);   // expect_tx arrive + 32 cp.async arrivals
+            ptx::mbar_init(bar_empty + 8 * s, 1);
+        }
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+
+    // ------------------------------------------------------------ producer
+    if (warp == NCW) {
+        if (lane == 0) {
+            ptx::prefetch_tensormap(&tm_k);
+            ptx::prefetch_tensormap(&tm_v);
+        }
+        const uint64_t pol = ptx::policy_evict_first();
+        for (int i = 0; i < ntiles; ++i) {
+            const int s = i % NST;
+            const uint32_t full = bar_full + 8 * s;
+            if (i >= NST && !ptx::mbar_wait(bar_empty + 8 * s, ((i / NST) - 1) & 1)) {
+                if (lane == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
+                break;
+            }
+            const int tt0 = t0 + i * TT;
+            const int ntok = min(TT, t1 - tt0);
+            const uint32_t sk = sbase + s * Lay::STAGE;
+            const uint32_t sv = sk + Lay::KV_BYTES;
+            const uint32_t sks = sv + Lay::KV_BYTES;
+            const uint32_t svs = sks + Lay::SC_FLOATS * 4;
+            if (!PAGED) {
+                const int64_t row0 = (static_cast<int64_t>(b) * p.Hk + hk) * p.max_seq + tt0;
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(full, 2 * Lay::KV_BYTES);
+                    ptx::tma_load_2d(sk, &tm_k, 0, static_cast<int>(row0), full, pol);
+                    ptx::tma_load_2d(sv, &tm_v, 0, static_cast<int>(row0), full, pol);
+                }
+                for (int k = lane; k < ntok; k += 32) {
+                    const int64_t r = row0 + k;
+                    if (G32) {
+                        ptx::cp_async_16(sks + k * 16, p.k_scale + r * NG);
+                        ptx::cp_async_16(svs + k * 16, p.v_scale + r * NG);
+                    } else {
+                        ptx::cp_async_4(sks + k * 4, p.k_scale + r);
+                        ptx::cp_async_4(svs + k * 4, p.v_scale + r);
+                    }
+                }
+            } else {
+                const int np = (ntok + 15) >> 4;
+                int32_t pg = -1;
+                if (lane < np) {
+                    pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tt0 >> 4) + lane];
+                    if (pg < 0 || pg >= p.num_pages) {
+                        raise_flag(p.d_err, KVQ_DEVERR_PAGE);
+                        pg = -1;
+                    }
+                }
+                const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
+                int pgs[TT / 16];
+#pragma unroll
+                for (int q = 0; q < TT / 16; ++q) pgs[q] = __shfl_sync(0xffffffffu, pg, q);
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(full, __popc(valid) * 2 * 16 * D);
+                    for (int q = 0; q < np; ++q) {
+                        const int pq = pgs[q];
+                        if (pq < 0) continue;
+                        const int y = (pq * p.Hk + hk) * 16;
+                        ptx::tma_load_2d(sk + q * 16 * D, &tm_k, 0, y, full, pol);
+                        ptx::tma_load_2d(sv + q * 16 * D, &tm_v, 0, y, full, pol);
+                    }
+                }
+                for (int k = lane; k < TT; k += 32) {
+                    const int pk = __shfl_sync(0xffffffffu, pg, k >> 4);
+                    if (k < ntok && pk >= 0) {
+                        const int64_t r = (static_cast<int64_t>(pk) * p.Hk + hk) * 16 + (k & 15);
+                        if (G32) {
+                            ptx::cp_async_16(sks + k * 16, p.k_scale + r * NG);
+                            ptx::cp_async_16(svs + k * 16, p.v_scale + r * NG);
+                        } else {
+                            ptx::cp_async_4(sks + k * 4, p.k_scale + r);
+                            ptx::cp_async_4(svs + k * 4, p.v_scale + r);
+                        }
+                    }
+                }
+            }
+            ptx::cp_async_arrive_noinc(full);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        return;
+    }
+
+    // ------------------------------------------------------------ consumers
+    const int g = lane >> 2, t = lane & 3;
+    const int tid = threadIdx.x;                 // 0..127
+
+    // Q fragments: rows = heads g (lo) and g + 8 (hi), pre-scaled by 2^s
+    uint32_t qa0[KS], qa2[KS], qa1[KS], qa3[KS];
+    float zs_lo = 0.f, zs_hi = 0.f;
+    const float sc_log2 = p.scale_log2;
+    auto load_q = [&](int h, uint32_t* f0, uint32_t* f2, float& zs) {
+        float qf[NGRP][8];
+        float amax = 0.f;
+        if (h < G) {
+            const uint16_t* qrow = p.q + (static_cast<int64_t>(b) * p.Hq + hk * G + h) * D;
+#pragma unroll
+            for (int gi = 0; gi < NGRP; ++gi) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(qrow + 32 * gi + 8 * t);
+                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    qf[gi][2 * e] = bf16_bits_to_f32(w[e] & 0xffffu);
+                    qf[gi][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(qf[gi][e]));
+            }
+        } else {
+#pragma unroll
+            for (int gi = 0; gi < NGRP; ++gi)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) qf[gi][e] = 0.f;
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        // power-of-two prescale: max |q| * 2^s in [2^14, 2^15)
+        int sh = 0;
+        if (amax > 0.f) {
+            const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+            sh = min(max(14 - e, -100), 100);
+        }
+        const float up = ldexpf(1.f, sh);
+        zs = ldexpf(1.f, -sh) * sc_log2;
+#pragma unroll
+        for (int gi = 0; gi < NGRP; ++gi)
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                f0[2 * gi + h2] = ptx::pack_f16x2(qf[gi][4 * h2] * up, qf[gi][4 * h2 + 1] * up);
+                f2[2 * gi + h2] = ptx::pack_f16x2(qf[gi][4 * h2 + 2] * up, qf[gi][4 * h2 + 3] * up);
+            }
+    };
+    load_q(g, qa0, qa2, zs_lo);
+    if (G16) {
+        load_q(g + 8, qa1, qa3, zs_hi);
+    } else {
+#pragma unroll
+        for (int k = 0; k < KS; ++k) qa1[k] = qa3[k] = 0u;
+    }
+
+    float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
+    float o_lo[NTD][2], o_hi[NTD][2];
+#pragma unroll
+    for (int n = 0; n < NTD; ++n) o_lo[n][0] = o_lo[n][1] = o_hi[n][0] = o_hi[n][1] = 0.f;
+
+    const int sig_g = sigma(g);
+    const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
+    bool timed_out = false;
+
+    for (int i = warp; i < ntiles; i += NCW) {
+        const int s = i % NST;
+        if (!ptx::mbar_wait(bar_full + 8 * s, (i / NST) & 1)) {
+            if (lane == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
+            timed_out = true;
+            break;
+        }
+        const int tt0 = t0 + i * TT;
+        const uint32_t sk = sbase + s * Lay::STAGE;
+        const uint32_t sv = sk + Lay::KV_BYTES;
+        const uint32_t sks = sv + Lay::KV_BYTES;
+        const uint32_t svs = sks + Lay::SC_FLOATS * 4;
+
+#pragma unroll 1
+        for (int sub = 0; sub < TT / 16; ++sub) {
+            const int tok0 = tt0 + 16 * sub;
+            if (tok0 >= t1) break;
+            bool page_ok = true;
+            if (PAGED) {
+                const int32_t pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tok0 >> 4)];
+                page_ok = pg >= 0 && pg < p.num_pages;
+            }
+            // ---- S = Q.K^T on 16 tokens: two n-tiles of 8
+            float sacc[2][NACC][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int a = 0; a < NACC; ++a)
+                    sacc[nt][a][0] = sacc[nt][a][1] = sacc[nt][a][2] = sacc[nt][a][3] = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const uint32_t row = 16 * sub + 8 * nt + sig_g;
+                uint2 kw[NGRP];
+#pragma unroll
+                for (int gi = 0; gi < NGRP; ++gi) kw[gi] = lds64(sk + swz<D>(row, 32 * gi + 8 * t));
+#pragma unroll
+                for (int gi = 0; gi < NGRP; ++gi)
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const uint32_t w = h2 ? kw[gi].y : kw[gi].x;
+                        const uint32_t b0 = ptx::bytes_to_f16x2(w, 0x4140u);
+                        const uint32_t b1 = ptx::bytes_to_f16x2(w, 0x4342u);
+                        const int ks = 2 * gi + h2;
+                        ptx::mma_f16(sacc[nt][G32 ? gi : 0], qa0[ks], qa1[ks], qa2[ks], qa3[ks],
+                                     b0, b1);
+                    }
+            }
+            // ---- scores (log2 domain), masked
+            float z_lo[2][2], z_hi[2][2];
+            bool ok[2][2];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int r = 16 * sub + 8 * nt + (c ? sig_b : sig_a);
+                    ok[nt][c] = page_ok && (tt0 + r < t1);
+                    float zl, zh;
+                    if (G32) {
+                        zl = 0.f;
+                        zh = 0.f;
+#pragma unroll
+                        for (int a = 0; a < NACC; ++a) {
+                            const float ksc = ldsf(sks + (r * NG + a) * 4);
+                            zl = fmaf(sacc[nt][a][c], ksc, zl);
+                            zh = fmaf(sacc[nt][a][2 + c], ksc, zh);
+                        }
+                    } else {
+                        const float ksc = ldsf(sks + r * 4);
+                        zl = sacc[nt][0][c] * ksc;
+                        zh = sacc[nt][0][2 + c] * ksc;
+                    }
+                    z_lo[nt][c] = ok[nt][c] ? zl * zs_lo : -INFINITY;
+                    z_hi[nt][c] = ok[nt][c] ? zh * zs_hi : -INFINITY;
+                }
+            // ---- online softmax, rows g (lo) and g + 8 (hi)
+            float mx_lo = fmaxf(fmaxf(z_lo[0][0], z_lo[0][1]), fmaxf(z_lo[1][0], z_lo[1][1]));
+            mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
+            mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
+            const float mn_lo = fmaxf(m_lo, mx_lo);
+            const float al_lo = (mn_lo == -INFINITY) ? 1.f : ptx::ex2(m_lo - mn_lo);
+            float pr_lo[2][2], pr_hi[2][2];
+            float ps_lo = 0.f, ps_hi = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    pr_lo[nt][c] = ok[nt][c] ? ptx::ex2(z_lo[nt][c] - mn_lo) : 0.f;
+                    ps_lo += pr_lo[nt][c];
+                }
+            l_lo = l_lo * al_lo + ps_lo;
+            m_lo = mn_lo;
+            float al_hi = 1.f;
+            if (G16) {
+                float mx_hi = fmaxf(fmaxf(z_hi[0][0], z_hi[0][1]), fmaxf(z_hi[1][0], z_hi[1][1]));
+                mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
+                mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
+                const float mn_hi = fmaxf(m_hi, mx_hi);
+                al_hi = (mn_hi == -INFINITY) ? 1.f : ptx::ex2(m_hi - mn_hi);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        pr_hi[nt][c] = ok[nt][c] ? ptx::ex2(z_hi[nt][c] - mn_hi) : 0.f;
+                        ps_hi += pr_hi[nt][c];
+                    }
+                l_hi = l_hi * al_hi + ps_hi;
+                m_hi = mn_hi;
+            }
+#pragma unroll
+            for (int n = 0; n < NTD; ++n) {
+                o_lo[n][0] *= al_lo;
+                o_lo[n][1] *= al_lo;
+                if (G16) {
+                    o_hi[n][0] *= al_hi;
+                    o_hi[n][1] *= al_hi;
+                }
+            }
+            // ---- P . V with P' = p * v_scale folded in
+            const int R0 = 16 * sub + sig_a, R1 = 16 * sub + sig_b;
+            const int R2 = R0 + 8, R3 = R1 + 8;
+            const int rr[2][2] = {{R0, R1}, {R2, R3}};
+            if (!G32) {
+                float vsc[2][2];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        vsc[nt][c] = ok[nt][c] ? ldsf(svs + rr[nt][c] * 4) : 0.f;
+                const uint32_t a0 = ptx::pack_f16x2(pr_lo[0][0] * vsc[0][0], pr_lo[0][1] * vsc[0][1]);
+                const uint32_t a2 = ptx::pack_f16x2(pr_lo[1][0] * vsc[1][0], pr_lo[1][1] * vsc[1][1]);
+                uint32_t a1 = 0u, a3 = 0u;
+                if (G16) {
+                    a1 = ptx::pack_f16x2(pr_hi[0][0] * vsc[0][0], pr_hi[0][1] * vsc[0][1]);
+                    a3 = ptx::pack_f16x2(pr_hi[1][0] * vsc[1][0], pr_hi[1][1] * vsc[1][1]);
+                }
+                // D == 128: thread g owns head_dim bytes [16g, 16g + 16) of each row,
+                // so output n-tile n, MMA column c is head_dim 16c + n.
+                // D == 64: thread g owns bytes [8g, 8g + 8); column c is 8c + n.
+                if constexpr (D == 128) {
+                    const uint32_t col = 16 * g;
+                    const uint4 v0 = lds128(sv + swz<D>(R0, col));
+                    const uint4 v1 = lds128(sv + swz<D>(R1, col));
+                    const uint4 v2 = lds128(sv + swz<D>(R2, col));
+                    const uint4 v3 = lds128(sv + swz<D>(R3, col));
+                    const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w};
+                    const uint32_t w1[4] = {v1.x, v1.y, v1.z, v1.w};
+                    const uint32_t w2[4] = {v2.x, v2.y, v2.z, v2.w};
+                    const uint32_t w3[4] = {v3.x, v3.y, v3.z, v3.w};
+#pragma unroll
+                    for (int wi = 0; wi < 4; ++wi) {
+                        const uint32_t xl01 = ptx::prmt(w0[wi], w1[wi], 0x5140u);
+                        const uint32_t xh01 = ptx::prmt(w0[wi], w1[wi], 0x7362u);
+                        const uint32_t xl23 = ptx::prmt(w2[wi], w3[wi], 0x5140u);
+                        const uint32_t xh23 = ptx::prmt(w2[wi], w3[wi], 0x7362u);
+                        const uint32_t b0s[4] = {ptx::bytes_to_f16x2(xl01, 0x4140u),
+                                                 ptx::bytes_to_f16x2(xl01, 0x4342u),
+                                                 ptx::bytes_to_f16x2(xh01, 0x4140u),
+                                                 ptx::bytes_to_f16x2(xh01, 0x4342u)};
+                        const uint32_t b1s[4] = {ptx::bytes_to_f16x2(xl23, 0x4140u),
+                                                 ptx::bytes_to_f16x2(xl23, 0x4342u),
+                                                 ptx::bytes_to_f16x2(xh23, 0x4140u),
+                                                 ptx::bytes_to_f16x2(xh23, 0x4342u)};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float acc[4] = {o_lo[4 * wi + e][0], o_lo[4 * wi + e][1],
+                                            o_hi[4 * wi + e][0], o_hi[4 * wi + e][1]};
+                            ptx::mma_f16(acc, a0, a1, a2, a3, b0s[e], b1s[e]);
+                            o_lo[4 * wi + e][0] = acc[0];
+                            o_lo[4 * wi + e][1] = acc[1];
+                            o_hi[4 * wi + e][0] = acc[2];
+                            o_hi[4 * wi + e][1] = acc[3];
+                        }
+                    }
+                } else {
+                    const uint32_t c64 = 8 * g;
+                    const uint2 v0 = lds64(sv + swz<D>(R0, c64));
+                    const uint2 v1 = lds64(sv + swz<D>(R1, c64));
+                    const uint2 v2 = lds64(sv + swz<D>(R2, c64));
+                    const uint2 v3 = lds64(sv + swz<D>(R3, c64));
+                    const uint32_t w0[2] = {v0.x, v0.y}, w1[2] = {v1.x, v1.y};
+                    const uint32_t w2[2] = {v2.x, v2.y}, w3[2] = {v3.x, v3.y};
+#pragma unroll
+                    for (int wi = 0; wi < 2; ++wi) {
+                        const uint32_t xl01 = ptx::prmt(w0[wi], w1[wi], 0x5140u);
+                        const uint32_t xh01 = ptx::prmt(w0[wi], w1[wi], 0x7362u);
+                        const uint32_t xl23 = ptx::prmt(w2[wi], w3[wi], 0x5140u);
+                        const uint32_t xh23 = ptx::prmt(w2[wi], w3[wi], 0x7362u);
+                        const uint32_t b0s[4] = {ptx::bytes_to_f16x2(xl01, 0x4140u),
+                                                 ptx::bytes_to_f16x2(xl01, 0x4342u),
+                                                 ptx::bytes_to_f16x2(xh01, 0x4140u),
+                                                 ptx::bytes_to_f16x2(xh01, 0x4342u)};
+                        const uint32_t b1s[4] = {ptx::bytes_to_f16x2(xl23, 0x4140u),
+                                                 ptx::bytes_to_f16x2(xl23, 0x4342u),
+                                                 ptx::bytes_to_f16x2(xh23, 0x4140u),
+                                                 ptx::bytes_to_f16x2(xh23, 0x4342u)};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float acc[4] = {o_lo[4 * wi + e][0], o_lo[4 * wi + e][1],
+                                            o_hi[4 * wi + e][0], o_hi[4 * wi + e][1]};
+                            ptx::mma_f16(acc, a0, a1, a2, a3, b0s[e], b1s[e]);
+                            o_lo[4 * wi + e][0] = acc[0];
+                            o_lo[4 * wi + e][1] = acc[1];
+                            o_hi[4 * wi + e][0] = acc[2];
+                            o_hi[4 * wi + e][1] = acc[3];
+                        }
+                    }
+                }
+            } else {
+                // group-32: n-tile 4*gv + e covers head_dim 32*gv + 4*n + e (n = MMA column),
+                // so thread g reads 4 bytes at 32*gv + 4*g of each row.
+#pragma unroll
+                for (int gv = 0; gv < NGRP; ++gv) {
+                    float vsc[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int c = 0; c < 2; ++c)
+                            vsc[nt][c] = ok[nt][c] ? ldsf(svs + (rr[nt][c] * NG + gv) * 4) : 0.f;
+                    const uint32_t a0 =
+                        ptx::pack_f16x2(pr_lo[0][0] * vsc[0][0], pr_lo[0][1] * vsc[0][1]);
+                    const uint32_t a2 =
+                        ptx::pack_f16x2(pr_lo[1][0] * vsc[1][0], pr_lo[1][1] * vsc[1][1]);
+                    uint32_t a1 = 0u, a3 = 0u;
+                    if (G16) {
+                        a1 = ptx::pack_f16x2(pr_hi[0][0] * vsc[0][0], pr_hi[0][1] * vsc[0][1]);
+                        a3 = ptx::pack_f16x2(pr_hi[1][0] * vsc[1][0], pr_hi[1][1] * vsc[1][1]);
+                    }
+                    const uint32_t cb = 32 * gv + 4 * g;
+                    const uint32_t w0 = lds32(sv + swz<D>(R0, cb));
+                    const uint32_t w1 = lds32(sv + swz<D>(R1, cb));
+                    const uint32_t w2 = lds32(sv + swz<D>(R2, cb));
+                    const uint32_t w3 = lds32(sv + swz<D>(R3, cb));
+                    const uint32_t xl01 = ptx::prmt(w0, w1, 0x5140u);
+                    const uint32_t xh01 = ptx::prmt(w0, w1, 0x7362u);
+                    const uint32_t xl23 = ptx::prmt(w2, w3, 0x5140u);
+                    const uint32_t xh23 = ptx::prmt(w2, w3, 0x7362u);
+                    const uint32_t b0s[4] = {ptx::bytes_to_f16x2(xl01, 0x4140u),
+                                             ptx::bytes_to_f16x2(xl01, 0x4342u),
+                                             ptx::bytes_to_f16x2(xh01, 0x4140u),
+                                             ptx::bytes_to_f16x2(xh01, 0x4342u)};
+                    const uint32_t b1s[4] = {ptx::bytes_to_f16x2(xl23, 0x4140u),
+                                             ptx::bytes_to_f16x2(xl23, 0x4342u),
+                                             ptx::bytes_to_f16x2(xh23, 0x4140u),
+                                             ptx::bytes_to_f16x2(xh23, 0x4342u)};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int n = 4 * gv + e;
+                        float acc[4] = {o_lo[n][0], o_lo[n][1], o_hi[n][0], o_hi[n][1]};
+                        ptx::mma_f16(acc, a0, a1, a2, a3, b0s[e], b1s[e]);
+                        o_lo[n][0] = acc[0];
+                        o_lo[n][1] = acc[1];
+                        o_hi[n][0] = acc[2];
+                        o_hi[n][1] = acc[3];
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar_empty + 8 * s);
+    }
+    (void)timed_out;
+
+    // ---- merge the four warps' (m, l, o) and write the split / final row
+    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+    ptx::named_bar_sync(1, NCW * 32);             // all stages consumed: reuse shared memory
+    constexpr int RS = D + 4;                     // padded row stride (floats)
+    float* red = reinterpret_cast<float*>(smem);  // [NCW][16][RS]
+    float* red_m = red + NCW * 16 * RS;           // [NCW][16]
+    float* red_l = red_m + NCW * 16;
+    // head_dim index of output n-tile n, column c (0/1) of this thread
+    auto dcol = [&](int n, int c) -> int {
+        if (G32) return 32 * (n >> 2) + 4 * (2 * t + c) + (n & 3);
+        return (D == 128 ? 16 : 8) * (2 * t + c) + n;
+    };
+#pragma unroll
+    for (int n = 0; n < NTD; ++n)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            red[(warp * 16 + g) * RS + dcol(n, c)] = o_lo[n][c];
+            if (G16) red[(warp * 16 + g + 8) * RS + dcol(n, c)] = o_hi[n][c];
+        }
+    if (t == 0) {
+        red_m[warp * 16 + g] = m_lo;
+        red_l[warp * 16 + g] = l_lo;
+        red_m[warp * 16 + g + 8] = G16 ? m_hi : -INFINITY;
+        red_l[warp * 16 + g + 8] = G16 ? l_hi : 0.f;
+    }
+    ptx::named_bar_sync(1, NCW * 32);
+    for (int idx = tid; idx < G * D; idx += NCW * 32) {
+        const int h = idx / D, d = idx - h * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NCW; ++w) M = fmaxf(M, red_m[w * 16 + h]);
+        float acc = 0.f, lsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < NCW; ++w) {
+            const float mw = red_m[w * 16 + h];
+            const float f = (mw == -INFINITY) ? 0.f : ptx::ex2(mw - M);
+            acc = fmaf(f, red[(w * 16 + h) * RS + d], acc);
+            lsum = fmaf(f, red_l[w * 16 + h], lsum);
+        }
+        const int64_t bh = static_cast<int64_t>(b) * p.Hq + hk * G + h;
+        if (nsplit == 1) {
+            p.out[bh * D + d] = lsum > 0.f ? acc / lsum : 0.f;
+        } else {
+            p.ws_o[(bh * p.splits + j) * D + d] = acc;
+            if (d == 0) {
+                p.ws_m[bh * p.splits + j] = M;
+                p.ws_l[bh * p.splits + j] = lsum;
+            }
+        }
+    }
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(ptr);
+    }
+    return fn;
+}
+
+// 2-D u8 tensor map over `rows` rows of D bytes, box of box_rows rows.
+cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, int box_rows) {
+    EncodeFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw =
+        D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D, bool G32, bool PAGED, bool G16>
+cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
+    using Lay = Layout<D, G32>;
+    static bool attr_done = false;
+    auto kern = decode_split_tc<D, G32, PAGED, G16>;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Lay::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    CUtensorMap mk, mv;
+    const int64_t rows = PAGED ? static_cast<int64_t>(p.num_pages) * p.Hk * 16
+                               : static_cast<int64_t>(p.B) * p.Hk * p.max_seq;
+    const int box = PAGED ? 16 : TT;
+    cudaError_t e = make_map(&mk, p.k, D, rows, box);
+    if (e == cudaSuccess) e = make_map(&mv, p.v, D, rows, box);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.splits, p.Hk, p.B);
+    kern<<<grid, NTHREADS, Lay::SMEM, s>>>(mk, mv, p);
+    return cudaGetLastError();
+}
+
+template <int D, bool G32, bool PAGED>
+cudaError_t pick_g(const DecodeParams& p, cudaStream_t s) {
+    return p.G > 8 ? launch_tc<D, G32, PAGED, true>(p, s) : launch_tc<D, G32, PAGED, false>(p, s);
+}
+
+template <int D>
+cudaError_t pick_layout(const DecodeParams& p, cudaStream_t s) {
+    if (p.page_size)
+        return p.group32 ? pick_g<D, true, true>(p, s) : pick_g<D, false, true>(p, s);
+    return p.group32 ? pick_g<D, true, false>(p, s) : pick_g<D, false, false>(p, s);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s) {
+    if (p.D == 128) return pick_layout<128>(p, s);
+    if (p.D == 64) return pick_layout<64>(p, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kvq

@@ -64,5 +64,7 @@ struct DecodeParams {
     float scale_log2;        // attn_scale * log2(e)
 };
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+// tensor-core split kernel (kvq_decode_tc.cu)
+cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s);
 
 }  // namespace kvq

@@ -60,6 +60,7 @@ typedef enum kvq_scale_mode {
 #define KVQ_DEVERR_POS 1u    /* append range [pos, pos + T) outside [0, capacity) */
 #define KVQ_DEVERR_PAGE 2u   /* page-table entry outside [0, num_pages) in the used range */
 #define KVQ_DEVERR_LEN 4u    /* decode sequence length outside [0, capacity] */
+#define KVQ_DEVERR_TIMEOUT 8u /* a bounded wait inside a kernel gave up (never expected) */
 
 typedef void *kvq_stream_t;  /* cudaStream_t */
 
@@ -148,7 +149,8 @@ typedef struct kvq_cache_view {
  *               per sequence (split-K / flash-decoding)
  *   d_err       int32 [1] or NULL (KVQ_DEVERR_LEN, KVQ_DEVERR_PAGE)
  * Requirements: Hq % Hk == 0 and Hq / Hk <= 16; D in {64, 128}; GROUP32
- * needs D % 32 == 0.
+ * needs D % 32 == 0; B * Hk * max_seq (contiguous) or num_pages * Hk * 16
+ * (paged) below 2^31 rows.
  * Source: abaddon 0.2.0-rc.1, kv_cache_quant_cuda.rs, module doc "Fused
  * approach" and CudaQuantizedKvCache::forward_attention (scores with
  * on-the-fly K dequantisation, softmax, P.V with on-the-fly V

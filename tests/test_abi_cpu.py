@@ -139,7 +139,7 @@ def test_decode_rejects_bad_arguments(kvq):
     assert call(mode=1, D=48) == 1
     assert call(D=256) == 2                 # valid, kernel not built for it
     assert call(D=32) == 2
-    assert call(Hq=8 * 16, Hk=8) == 2       # GQA group above the built tile
+    assert call(Hq=8 * 32, Hk=8) == 2       # GQA group above the built tile (16)
     assert call(out=FAKE + 4) == 1          # misaligned output
     assert call(hint=-1) == 1
     bad_page = kvq.CacheView(FAKE, FAKE, FAKE, FAKE, 32, 0, FAKE, 4, 4)

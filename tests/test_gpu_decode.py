@@ -28,7 +28,7 @@ def _fill_contig(B, Hq, Hk, D, mode, lens, seed, sigma=1.0, outlier=None):
 
 @pytest.mark.parametrize("mode", ["per_token", "group32"])
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("G", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 8, 12, 16])
 def test_decode_contig_small(mode, D, G):
     B, Hk = 3, 2
     lens = [1, 130, 517]
@@ -107,9 +107,9 @@ def test_decode_outlier_channels():
 
 
 @pytest.mark.parametrize("mode", ["per_token", "group32"])
-@pytest.mark.parametrize("G", [1, 4, 8])
-def test_decode_paged_matches_oracle(mode, G):
-    B, Hk, D, ps = 3, 2, 128, 16
+@pytest.mark.parametrize("G,D", [(1, 128), (4, 128), (8, 128), (16, 128), (4, 64)])
+def test_decode_paged_matches_oracle(mode, G, D):
+    B, Hk, ps = 3, 2, 16
     lens = [16, 47, 300]
     need = [(L + ps - 1) // ps for L in lens]
     gen = torch.Generator().manual_seed(G)
@@ -163,3 +163,32 @@ def test_decode_bad_page_is_flagged_not_read():
     q = bf16_randn((1, 2, 64), seed=3)
     c.decode(q, torch.tensor([40], dtype=torch.int32), 48)
     assert kvq().kvq_read_error(c.err) & kvq().DEVERR_PAGE
+
+
+@pytest.mark.parametrize("G", [4, 8])
+def test_decode_peaky_softmax(G):
+    """One key per sequence aligned with the query dominates the softmax."""
+    B, Hk, D, L = 2, 2, 128, 300
+    c, q = _fill_contig(B, Hk * G, Hk, D, "per_token", [L, L], seed=21)
+    kq = q.view(B, Hk, G, D)[:, :, 0]                       # first query head of each group
+    k_hot = (kq.float() * 6).to(torch.bfloat16)[:, :, None]  # [B, Hk, 1, D]
+    v_hot = bf16_randn((B, Hk, 1, D), seed=22, sigma=4.0)
+    assert c.append(k_hot, v_hot, torch.tensor([137, 5], dtype=torch.int32)) == 0
+    sl = torch.tensor([L, L], dtype=torch.int32)
+    out = c.decode(q, sl, L, attn_scale=f32_scale(D))
+    assert_attn_close(out, c.oracle_decode(q, sl, f32_scale(D)), "peaky")
+
+
+def test_decode_large_query_magnitudes():
+    """Query rows of very different magnitude (the per-head f16 prescale)."""
+    B, Hk, G, D, L = 1, 2, 8, 128, 200
+    c, q = _fill_contig(B, Hk * G, Hk, D, "group32", [L], seed=23)
+    qf = q.float()
+    qf[0, 0] *= 1e-20
+    qf[0, 1] *= 3e4
+    qf[0, 2] = 0
+    qf[0, 3, :5] = 1e-30
+    q = qf.to(torch.bfloat16)
+    sl = torch.tensor([L], dtype=torch.int32)
+    out = c.decode(q, sl, L, attn_scale=1e-4)
+    assert_attn_close(out, c.oracle_decode(q, sl, 1e-4), "q magnitudes")
