@@ -25,7 +25,7 @@ kvq_status check_append_common(const uint16_t* k_new, const uint16_t* v_new, int
     if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_INVALID_ARG;
     if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
     if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(kd, 16) || !aligned(vd, 16) ||
-        !aligned(ks, 4) || !aligned(vs, 4) || !aligned(d_pos, 4) || !aligned(d_err, 4))
+        !aligned(ks, 16) || !aligned(vs, 16) || !aligned(d_pos, 4) || !aligned(d_err, 4))
         return KVQ_ERR_INVALID_ARG;
     return KVQ_OK;
 }
@@ -143,7 +143,7 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
         return KVQ_ERR_INVALID_ARG;
     }
     if (!aligned(q, 16) || !aligned(kv->k, 16) || !aligned(kv->v, 16) ||
-        !aligned(kv->k_scale, 4) || !aligned(kv->v_scale, 4) || !aligned(d_seq_lens, 4) ||
+        !aligned(kv->k_scale, 16) || !aligned(kv->v_scale, 16) || !aligned(d_seq_lens, 4) ||
         !aligned(out, 16) || !aligned(workspace, 16) || !aligned(d_err, 4))
         return KVQ_ERR_INVALID_ARG;
     const int G = Hq / Hk;
@@ -182,7 +182,7 @@ kvq_status kvq_dequant(const uint8_t* q, const float* scale, int64_t rows, int D
     if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_INVALID_ARG;
     if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
     if (rows == 0) return KVQ_OK;
-    if (!q || !scale || !out || !aligned(q, 16) || !aligned(out, 16) || !aligned(scale, 4))
+    if (!q || !scale || !out || !aligned(q, 16) || !aligned(out, 16) || !aligned(scale, 16))
         return KVQ_ERR_INVALID_ARG;
     return from_cuda(kvq::launch_dequant(q, scale, rows, D, mode == KVQ_SCALE_GROUP32, out,
                                          static_cast<cudaStream_t>(stream)));

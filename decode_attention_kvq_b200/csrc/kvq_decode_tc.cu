@@ -97,6 +97,16 @@ __device__ __forceinline__ float ldsf(uint32_t a) {
     return v;
 }
 
+// The NG fp32 scales of one token (4, 8 or 16 bytes, aligned to their size
+// because the scale array is 16-byte aligned and rows are NG floats apart).
+template <int NG>
+__device__ __forceinline__ void copy_scales(uint32_t dst, const float* src) {
+    static_assert(NG == 1 || NG == 2 || NG == 4, "scales per token");
+    if constexpr (NG == 1) ptx::cp_async_4(dst, src);
+    else if constexpr (NG == 2) ptx::cp_async_8(dst, src);
+    else ptx::cp_async_16(dst, src);
+}
+
 template <int D, bool G32, bool PAGED, bool G16>
 __global__ void __launch_bounds__(NTHREADS)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -176,13 +186,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
                 for (int k = lane; k < ntok; k += 32) {
                     const int64_t r = row0 + k;
-                    if (G32) {
-                        ptx::cp_async_16(sks + k * 16, p.k_scale + r * NG);
-                        ptx::cp_async_16(svs + k * 16, p.v_scale + r * NG);
-                    } else {
-                        ptx::cp_async_4(sks + k * 4, p.k_scale + r);
-                        ptx::cp_async_4(svs + k * 4, p.v_scale + r);
-                    }
+                    copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
+                    copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
                 }
             } else {
                 const int np = (ntok + 15) >> 4;
@@ -212,13 +217,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const int pk = __shfl_sync(0xffffffffu, pg, k >> 4);
                     if (k < ntok && pk >= 0) {
                         const int64_t r = (static_cast<int64_t>(pk) * p.Hk + hk) * 16 + (k & 15);
-                        if (G32) {
-                            ptx::cp_async_16(sks + k * 16, p.k_scale + r * NG);
-                            ptx::cp_async_16(svs + k * 16, p.v_scale + r * NG);
-                        } else {
-                            ptx::cp_async_4(sks + k * 4, p.k_scale + r);
-                            ptx::cp_async_4(svs + k * 4, p.v_scale + r);
-                        }
+                        copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
+                        copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
                     }
                 }
             }

@@ -111,6 +111,7 @@ def test_append_rejects_bad_arguments(kvq):
     assert call(T=0) == 1
     assert call(mode=7) == 1
     assert call(k=FAKE + 2) == 1            # misaligned vector source
+    assert call(ks=FAKE + 4) == 1           # scale arrays need 16-byte alignment
     assert call(max_seq=0) == 1
 
 
@@ -141,6 +142,8 @@ def test_decode_rejects_bad_arguments(kvq):
     assert call(D=32) == 2
     assert call(Hq=8 * 32, Hk=8) == 2       # GQA group above the built tile (16)
     assert call(out=FAKE + 4) == 1          # misaligned output
+    cv_bad_scale = kvq.CacheView(FAKE, FAKE, FAKE + 8, FAKE, 0, 4096, 0, 0, 0)
+    assert call(kv=ctypes.byref(cv_bad_scale)) == 1
     assert call(hint=-1) == 1
     bad_page = kvq.CacheView(FAKE, FAKE, FAKE, FAKE, 32, 0, FAKE, 4, 4)
     assert call(kv=ctypes.byref(bad_page)) == 1
