@@ -25,9 +25,12 @@
 //    accumulators hold sum_d q_d (k_d - 128) up to accumulation rounding.
 //    The K scale (per token, or per 32-value group with one accumulator per
 //    group), 2^-s, attn_scale and log2(e) are applied to the accumulator.
-//  * Online softmax in base 2 per head row; P' = 2^(z-m) * v_scale(token) is
-//    rounded to f16 and multiplied with the exact integers (v - 128), so the
-//    V scale is folded into P (per 32-value group in group-32 mode).
+//  * Online softmax in base 2 per head row.  The V scale is folded into P:
+//    P'' = 2^(z-m) * v_scale(token) * 2^kv (per 32-value group in group-32
+//    mode), with a running per-warp power of two 2^kv that keeps P'' inside
+//    the f16 normal range.  P'' is split into f16 hi + lo parts (about 22
+//    significant bits together) and both are multiplied with the exact
+//    integers (v - 128), so P.V carries no f16 rounding of P beyond ~2^-22.
 //  * Token order inside each 16-token slice and the d order of the MMA
 //    k-dimension are permuted so that every shared-memory load of the
 //    swizzled tiles is free of bank conflicts (sigma below).
@@ -97,6 +100,16 @@ __device__ __forceinline__ float ldsf(uint32_t a) {
     return v;
 }
 
+// (a, b) -> f16x2 hi = rn(a, b) and lo = rn(a - hi, b - hi): hi + lo carries
+// about 22 significant bits of each value.
+__device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const __half2 h = __floats2half2_rn(a, b);
+    const float2 f = __half22float2(h);
+    const __half2 l = __floats2half2_rn(a - f.x, b - f.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 // The NG fp32 scales of one token (4, 8 or 16 bytes, aligned to their size
 // because the scale array is 16-byte aligned and rows are NG floats apart).
 template <int NG>
@@ -117,6 +130,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     constexpr int NGRP = D / 32;        // 32-value groups over head_dim
     constexpr int NTD = D / 8;          // output n-tiles over head_dim
     constexpr int NACC = G32 ? NG : 1;  // score accumulators per n-tile
+    constexpr int NGV = G32 ? NG : 1;   // V scales per token
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -290,6 +304,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
     for (int n = 0; n < NTD; ++n) o_lo[n][0] = o_lo[n][1] = o_hi[n][0] = o_hi[n][1] = 0.f;
 
+    int kv = 64;                         // running P'' prescale exponent (per warp)
     const int sig_g = sigma(g);
     const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
     bool timed_out = false;
@@ -381,6 +396,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     pr_lo[nt][c] = ok[nt][c] ? ptx::ex2(z_lo[nt][c] - mn_lo) : 0.f;
+                    pr_hi[nt][c] = 0.f;
                     ps_lo += pr_lo[nt][c];
                 }
             l_lo = l_lo * al_lo + ps_lo;
@@ -402,152 +418,118 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 l_hi = l_hi * al_hi + ps_hi;
                 m_hi = mn_hi;
             }
-#pragma unroll
-            for (int n = 0; n < NTD; ++n) {
-                o_lo[n][0] *= al_lo;
-                o_lo[n][1] *= al_lo;
-                if (G16) {
-                    o_hi[n][0] *= al_hi;
-                    o_hi[n][1] *= al_hi;
-                }
-            }
-            // ---- P . V with P' = p * v_scale folded in
+
+            // ---- V scales of this slice and the running power-of-two prescale:
+            // P'' = p * v_scale * 2^kv with kv chosen so that the largest
+            // v_scale * 2^kv seen by this warp lies in [2^14, 2^15); when kv
+            // drops, the accumulated O is rescaled by the same power of two.
             const int R0 = 16 * sub + sig_a, R1 = 16 * sub + sig_b;
             const int R2 = R0 + 8, R3 = R1 + 8;
             const int rr[2][2] = {{R0, R1}, {R2, R3}};
-            if (!G32) {
-                float vsc[2][2];
+            float vsc[2][2][NGV];
+            float vmax = 0.f;
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                    for (int c = 0; c < 2; ++c)
-                        vsc[nt][c] = ok[nt][c] ? ldsf(svs + rr[nt][c] * 4) : 0.f;
-                const uint32_t a0 = ptx::pack_f16x2(pr_lo[0][0] * vsc[0][0], pr_lo[0][1] * vsc[0][1]);
-                const uint32_t a2 = ptx::pack_f16x2(pr_lo[1][0] * vsc[1][0], pr_lo[1][1] * vsc[1][1]);
-                uint32_t a1 = 0u, a3 = 0u;
-                if (G16) {
-                    a1 = ptx::pack_f16x2(pr_hi[0][0] * vsc[0][0], pr_hi[0][1] * vsc[0][1]);
-                    a3 = ptx::pack_f16x2(pr_hi[1][0] * vsc[1][0], pr_hi[1][1] * vsc[1][1]);
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int gv = 0; gv < NGV; ++gv) {
+                        vsc[nt][c][gv] = ok[nt][c] ? ldsf(svs + (rr[nt][c] * NG + gv) * 4) : 0.f;
+                        vmax = fmaxf(vmax, vsc[nt][c][gv]);
+                    }
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 1));
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 2));
+            float f_lo = al_lo, f_hi = al_hi;     // factors applied to O
+            if (vmax > 0.f) {
+                const int ev = static_cast<int>((__float_as_uint(vmax) >> 23) & 0xffu) - 127;
+                const int kn = min(kv, 14 - ev);
+                if (kn < kv) {
+                    const float drop = ldexpf(1.f, kn - kv);
+                    f_lo *= drop;
+                    f_hi *= drop;
+                    kv = kn;
                 }
-                // D == 128: thread g owns head_dim bytes [16g, 16g + 16) of each row,
-                // so output n-tile n, MMA column c is head_dim 16c + n.
-                // D == 64: thread g owns bytes [8g, 8g + 8); column c is 8c + n.
+            }
+            const float up = ldexpf(1.f, kv);
+#pragma unroll
+            for (int n = 0; n < NTD; ++n) {
+                o_lo[n][0] *= f_lo;
+                o_lo[n][1] *= f_lo;
+                if (G16) {
+                    o_hi[n][0] *= f_hi;
+                    o_hi[n][1] *= f_hi;
+                }
+            }
+            // A fragments of P'' split into f16 hi + lo (P'' = hi + lo to ~2^-22)
+            uint32_t ah[NGV][4], al[NGV][4];
+#pragma unroll
+            for (int gv = 0; gv < NGV; ++gv) {
+                split_f16x2(pr_lo[0][0] * vsc[0][0][gv] * up, pr_lo[0][1] * vsc[0][1][gv] * up,
+                            ah[gv][0], al[gv][0]);
+                split_f16x2(pr_lo[1][0] * vsc[1][0][gv] * up, pr_lo[1][1] * vsc[1][1][gv] * up,
+                            ah[gv][2], al[gv][2]);
+                if (G16) {
+                    split_f16x2(pr_hi[0][0] * vsc[0][0][gv] * up, pr_hi[0][1] * vsc[0][1][gv] * up,
+                                ah[gv][1], al[gv][1]);
+                    split_f16x2(pr_hi[1][0] * vsc[1][0][gv] * up, pr_hi[1][1] * vsc[1][1][gv] * up,
+                                ah[gv][3], al[gv][3]);
+                } else {
+                    ah[gv][1] = ah[gv][3] = al[gv][1] = al[gv][3] = 0u;
+                }
+            }
+            auto pv = [&](int n, int gv, uint32_t b0, uint32_t b1) {
+                float acc[4] = {o_lo[n][0], o_lo[n][1], o_hi[n][0], o_hi[n][1]};
+                ptx::mma_f16(acc, ah[gv][0], ah[gv][1], ah[gv][2], ah[gv][3], b0, b1);
+                ptx::mma_f16(acc, al[gv][0], al[gv][1], al[gv][2], al[gv][3], b0, b1);
+                o_lo[n][0] = acc[0];
+                o_lo[n][1] = acc[1];
+                o_hi[n][0] = acc[2];
+                o_hi[n][1] = acc[3];
+            };
+            // B fragments from two pairs of V words: rows (R0, R1) give b0,
+            // rows (R2, R3) give b1; byte e of the words is n-tile offset e.
+            auto pv_words = [&](int n0, int gv, uint32_t w0, uint32_t w1, uint32_t w2,
+                                uint32_t w3) {
+                const uint32_t xl01 = ptx::prmt(w0, w1, 0x5140u);
+                const uint32_t xh01 = ptx::prmt(w0, w1, 0x7362u);
+                const uint32_t xl23 = ptx::prmt(w2, w3, 0x5140u);
+                const uint32_t xh23 = ptx::prmt(w2, w3, 0x7362u);
+                pv(n0 + 0, gv, ptx::bytes_to_f16x2(xl01, 0x4140u), ptx::bytes_to_f16x2(xl23, 0x4140u));
+                pv(n0 + 1, gv, ptx::bytes_to_f16x2(xl01, 0x4342u), ptx::bytes_to_f16x2(xl23, 0x4342u));
+                pv(n0 + 2, gv, ptx::bytes_to_f16x2(xh01, 0x4140u), ptx::bytes_to_f16x2(xh23, 0x4140u));
+                pv(n0 + 3, gv, ptx::bytes_to_f16x2(xh01, 0x4342u), ptx::bytes_to_f16x2(xh23, 0x4342u));
+            };
+            if (!G32) {
                 if constexpr (D == 128) {
+                    // thread g owns head_dim bytes [16g, 16g + 16): n-tile n, MMA column c
+                    // is head_dim 16c + n
                     const uint32_t col = 16 * g;
                     const uint4 v0 = lds128(sv + swz<D>(R0, col));
                     const uint4 v1 = lds128(sv + swz<D>(R1, col));
                     const uint4 v2 = lds128(sv + swz<D>(R2, col));
                     const uint4 v3 = lds128(sv + swz<D>(R3, col));
-                    const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w};
-                    const uint32_t w1[4] = {v1.x, v1.y, v1.z, v1.w};
-                    const uint32_t w2[4] = {v2.x, v2.y, v2.z, v2.w};
-                    const uint32_t w3[4] = {v3.x, v3.y, v3.z, v3.w};
-#pragma unroll
-                    for (int wi = 0; wi < 4; ++wi) {
-                        const uint32_t xl01 = ptx::prmt(w0[wi], w1[wi], 0x5140u);
-                        const uint32_t xh01 = ptx::prmt(w0[wi], w1[wi], 0x7362u);
-                        const uint32_t xl23 = ptx::prmt(w2[wi], w3[wi], 0x5140u);
-                        const uint32_t xh23 = ptx::prmt(w2[wi], w3[wi], 0x7362u);
-                        const uint32_t b0s[4] = {ptx::bytes_to_f16x2(xl01, 0x4140u),
-                                                 ptx::bytes_to_f16x2(xl01, 0x4342u),
-                                                 ptx::bytes_to_f16x2(xh01, 0x4140u),
-                                                 ptx::bytes_to_f16x2(xh01, 0x4342u)};
-                        const uint32_t b1s[4] = {ptx::bytes_to_f16x2(xl23, 0x4140u),
-                                                 ptx::bytes_to_f16x2(xl23, 0x4342u),
-                                                 ptx::bytes_to_f16x2(xh23, 0x4140u),
-                                                 ptx::bytes_to_f16x2(xh23, 0x4342u)};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float acc[4] = {o_lo[4 * wi + e][0], o_lo[4 * wi + e][1],
-                                            o_hi[4 * wi + e][0], o_hi[4 * wi + e][1]};
-                            ptx::mma_f16(acc, a0, a1, a2, a3, b0s[e], b1s[e]);
-                            o_lo[4 * wi + e][0] = acc[0];
-                            o_lo[4 * wi + e][1] = acc[1];
-                            o_hi[4 * wi + e][0] = acc[2];
-                            o_hi[4 * wi + e][1] = acc[3];
-                        }
-                    }
+                    pv_words(0, 0, v0.x, v1.x, v2.x, v3.x);
+                    pv_words(4, 0, v0.y, v1.y, v2.y, v3.y);
+                    pv_words(8, 0, v0.z, v1.z, v2.z, v3.z);
+                    pv_words(12, 0, v0.w, v1.w, v2.w, v3.w);
                 } else {
-                    const uint32_t c64 = 8 * g;
-                    const uint2 v0 = lds64(sv + swz<D>(R0, c64));
-                    const uint2 v1 = lds64(sv + swz<D>(R1, c64));
-                    const uint2 v2 = lds64(sv + swz<D>(R2, c64));
-                    const uint2 v3 = lds64(sv + swz<D>(R3, c64));
-                    const uint32_t w0[2] = {v0.x, v0.y}, w1[2] = {v1.x, v1.y};
-                    const uint32_t w2[2] = {v2.x, v2.y}, w3[2] = {v3.x, v3.y};
-#pragma unroll
-                    for (int wi = 0; wi < 2; ++wi) {
-                        const uint32_t xl01 = ptx::prmt(w0[wi], w1[wi], 0x5140u);
-                        const uint32_t xh01 = ptx::prmt(w0[wi], w1[wi], 0x7362u);
-                        const uint32_t xl23 = ptx::prmt(w2[wi], w3[wi], 0x5140u);
-                        const uint32_t xh23 = ptx::prmt(w2[wi], w3[wi], 0x7362u);
-                        const uint32_t b0s[4] = {ptx::bytes_to_f16x2(xl01, 0x4140u),
-                                                 ptx::bytes_to_f16x2(xl01, 0x4342u),
-                                                 ptx::bytes_to_f16x2(xh01, 0x4140u),
-                                                 ptx::bytes_to_f16x2(xh01, 0x4342u)};
-                        const uint32_t b1s[4] = {ptx::bytes_to_f16x2(xl23, 0x4140u),
-                                                 ptx::bytes_to_f16x2(xl23, 0x4342u),
-                                                 ptx::bytes_to_f16x2(xh23, 0x4140u),
-                                                 ptx::bytes_to_f16x2(xh23, 0x4342u)};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float acc[4] = {o_lo[4 * wi + e][0], o_lo[4 * wi + e][1],
-                                            o_hi[4 * wi + e][0], o_hi[4 * wi + e][1]};
-                            ptx::mma_f16(acc, a0, a1, a2, a3, b0s[e], b1s[e]);
-                            o_lo[4 * wi + e][0] = acc[0];
-                            o_lo[4 * wi + e][1] = acc[1];
-                            o_hi[4 * wi + e][0] = acc[2];
-                            o_hi[4 * wi + e][1] = acc[3];
-                        }
-                    }
+                    // D == 64: thread g owns bytes [8g, 8g + 8): column c is 8c + n
+                    const uint32_t col = 8 * g;
+                    const uint2 v0 = lds64(sv + swz<D>(R0, col));
+                    const uint2 v1 = lds64(sv + swz<D>(R1, col));
+                    const uint2 v2 = lds64(sv + swz<D>(R2, col));
+                    const uint2 v3 = lds64(sv + swz<D>(R3, col));
+                    pv_words(0, 0, v0.x, v1.x, v2.x, v3.x);
+                    pv_words(4, 0, v0.y, v1.y, v2.y, v3.y);
                 }
             } else {
-                // group-32: n-tile 4*gv + e covers head_dim 32*gv + 4*n + e (n = MMA column),
-                // so thread g reads 4 bytes at 32*gv + 4*g of each row.
+                // group-32: n-tile 4*gv + e covers head_dim 32*gv + 4*c + e (c = MMA
+                // column), so thread g reads 4 bytes at 32*gv + 4*g of each row
 #pragma unroll
                 for (int gv = 0; gv < NGRP; ++gv) {
-                    float vsc[2][2];
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                        for (int c = 0; c < 2; ++c)
-                            vsc[nt][c] = ok[nt][c] ? ldsf(svs + (rr[nt][c] * NG + gv) * 4) : 0.f;
-                    const uint32_t a0 =
-                        ptx::pack_f16x2(pr_lo[0][0] * vsc[0][0], pr_lo[0][1] * vsc[0][1]);
-                    const uint32_t a2 =
-                        ptx::pack_f16x2(pr_lo[1][0] * vsc[1][0], pr_lo[1][1] * vsc[1][1]);
-                    uint32_t a1 = 0u, a3 = 0u;
-                    if (G16) {
-                        a1 = ptx::pack_f16x2(pr_hi[0][0] * vsc[0][0], pr_hi[0][1] * vsc[0][1]);
-                        a3 = ptx::pack_f16x2(pr_hi[1][0] * vsc[1][0], pr_hi[1][1] * vsc[1][1]);
-                    }
                     const uint32_t cb = 32 * gv + 4 * g;
-                    const uint32_t w0 = lds32(sv + swz<D>(R0, cb));
-                    const uint32_t w1 = lds32(sv + swz<D>(R1, cb));
-                    const uint32_t w2 = lds32(sv + swz<D>(R2, cb));
-                    const uint32_t w3 = lds32(sv + swz<D>(R3, cb));
-                    const uint32_t xl01 = ptx::prmt(w0, w1, 0x5140u);
-                    const uint32_t xh01 = ptx::prmt(w0, w1, 0x7362u);
-                    const uint32_t xl23 = ptx::prmt(w2, w3, 0x5140u);
-                    const uint32_t xh23 = ptx::prmt(w2, w3, 0x7362u);
-                    const uint32_t b0s[4] = {ptx::bytes_to_f16x2(xl01, 0x4140u),
-                                             ptx::bytes_to_f16x2(xl01, 0x4342u),
-                                             ptx::bytes_to_f16x2(xh01, 0x4140u),
-                                             ptx::bytes_to_f16x2(xh01, 0x4342u)};
-                    const uint32_t b1s[4] = {ptx::bytes_to_f16x2(xl23, 0x4140u),
-                                             ptx::bytes_to_f16x2(xl23, 0x4342u),
-                                             ptx::bytes_to_f16x2(xh23, 0x4140u),
-                                             ptx::bytes_to_f16x2(xh23, 0x4342u)};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int n = 4 * gv + e;
-                        float acc[4] = {o_lo[n][0], o_lo[n][1], o_hi[n][0], o_hi[n][1]};
-                        ptx::mma_f16(acc, a0, a1, a2, a3, b0s[e], b1s[e]);
-                        o_lo[n][0] = acc[0];
-                        o_lo[n][1] = acc[1];
-                        o_hi[n][0] = acc[2];
-                        o_hi[n][1] = acc[3];
-                    }
+                    pv_words(4 * gv, gv, lds32(sv + swz<D>(R0, cb)), lds32(sv + swz<D>(R1, cb)),
+                             lds32(sv + swz<D>(R2, cb)), lds32(sv + swz<D>(R3, cb)));
                 }
             }
         }
@@ -561,6 +543,16 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
     l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
     l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+    {
+        const float down = ldexpf(1.f, -kv);         // undo the P'' prescale
+#pragma unroll
+        for (int n = 0; n < NTD; ++n) {
+            o_lo[n][0] *= down;
+            o_lo[n][1] *= down;
+            o_hi[n][0] *= down;
+            o_hi[n][1] *= down;
+        }
+    }
     ptx::named_bar_sync(1, NCW * 32);             // all stages consumed: reuse shared memory
     constexpr int RS = D + 4;                     // padded row stride (floats)
     float* red = reinterpret_cast<float*>(smem);  // [NCW][16][RS]
