@@ -397,8 +397,11 @@ def run_kvq(args, wl):
     L0 = layers[0]
     ws_bytes = kvq.kvq_decode_workspace_bytes(wl.B, wl.Hq, wl.Hk, wl.D, L0.hint)
     workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    # a cluster of splits combines in distributed shared memory: no workspace
     chunk, splits = kvq.kvq_decode_plan(wl.B, wl.Hk, L0.hint)
-    launches_per_layer = (1 + (1 if wl.prefill_chunk else 0)) + 1 + (1 if splits > 1 else 0)
+    # append (+ prefill-chunk append) + split kernel (+ combine kernel when the
+    # splits do not fit one cluster and go through the workspace)
+    launches_per_layer = (1 + (1 if wl.prefill_chunk else 0)) + 1 + (1 if ws_bytes > 0 else 0)
 
     stream = torch.cuda.Stream(dev)
     # warm the library once eagerly, then capture the two phases as graphs

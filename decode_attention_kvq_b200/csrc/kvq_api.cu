@@ -30,6 +30,8 @@ kvq_status check_append_common(const uint16_t* k_new, const uint16_t* v_new, int
     return KVQ_OK;
 }
 
+constexpr int kClusterSplits = 16;   // splits combined inside one thread-block cluster
+
 kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk_out,
                 int* splits_out) {
     if (B < 0 || Hk < 1 || hint < 0 || num_splits < 0) return KVQ_ERR_INVALID_ARG;
@@ -46,13 +48,12 @@ kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk
         const int64_t s = num_splits < ceil_div(hint, 16) ? num_splits : ceil_div(hint, 16);
         chunk = ceil_div(ceil_div(hint, s), 16) * 16;
     } else {
-        // about two CTAs per SM over all (sequence, kv head) units, splits of
-        // 64..1024 tokens
+        // about two CTAs per SM over all (sequence, kv head) units, at most
+        // one cluster of splits per unit
         const int64_t units = static_cast<int64_t>(B > 0 ? B : 1) * Hk;
-        const int64_t want = ceil_div(2ll * num_sms, units);
-        chunk = ceil_div(ceil_div(hint, want), 64) * 64;
-        if (chunk < 64) chunk = 64;
-        if (chunk > 1024) chunk = 1024;
+        int64_t want = ceil_div(2ll * num_sms, units);
+        if (want > kClusterSplits) want = kClusterSplits;
+        chunk = ceil_div(ceil_div(hint, want), 16) * 16;
     }
     if (ceil_div(hint, chunk) > kMaxSplits) chunk = ceil_div(ceil_div(hint, kMaxSplits), 16) * 16;
     int64_t splits = ceil_div(hint, chunk);
@@ -62,8 +63,14 @@ kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk
     return KVQ_OK;
 }
 
+// splits combined in a cluster (no workspace), or 1 when the combine kernel is used
+int cluster_for(int splits) {
+    if (splits <= 1) return 1;
+    return splits <= kvq::decode_max_cluster() ? splits : 1;
+}
+
 size_t workspace_for(int B, int Hq, int D, int splits) {
-    if (splits <= 1) return 0;
+    if (splits <= 1 || cluster_for(splits) > 1) return 0;
     return static_cast<size_t>(B) * Hq * splits * (D + 2) * sizeof(float);
 }
 
@@ -172,6 +179,7 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
     p.B = B; p.Hq = Hq; p.Hk = Hk; p.G = G; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
     p.page_size = kv->page_size; p.max_seq = kv->max_seq; p.max_pages = kv->max_pages;
     p.num_pages = kv->num_pages; p.chunk = chunk; p.splits = splits;
+    p.cluster = cluster_for(splits);
     p.scale_log2 = attn_scale * 1.4426950408889634f;
     return from_cuda(kvq::launch_decode(p, static_cast<cudaStream_t>(stream)));
 }

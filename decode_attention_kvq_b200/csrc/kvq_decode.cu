@@ -1,6 +1,7 @@
 // kvq_decode.cu -- decode attention driver: the split kernel
-// (kvq_decode_tc.cu) followed, when any sequence has more than one split, by
-// the combine kernel below.
+// (kvq_decode_tc.cu), which combines up to 16 splits inside a thread-block
+// cluster, followed -- only when more splits than one cluster holds were
+// requested -- by the combine kernel below.
 //
 // Combine (flash-decoding): for each (sequence, q head) with splits j =
 // 0..ns-1 holding unnormalised (o_j, m_j, l_j) in base 2,
@@ -80,7 +81,7 @@ decode_combine(DecodeParams p) {
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
     cudaError_t e = launch_decode_split_tc(p, s);
-    if (e != cudaSuccess || p.splits <= 1) return e;
+    if (e != cudaSuccess || p.splits <= 1 || p.cluster > 1) return e;
     const size_t smem = static_cast<size_t>(p.splits) * sizeof(float);
     decode_combine<<<p.B * p.Hq, kThreads, smem, s>>>(p);
     return cudaGetLastError();

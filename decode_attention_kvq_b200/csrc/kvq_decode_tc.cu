@@ -1,24 +1,29 @@
-// kvq_decode_tc.cu -- split-K decode attention on the INT8 cache for sm_100a:
+// kvq_decode_tc.cu -- decode attention on the INT8 cache for sm_100a:
 // TMA-staged K/V tiles, tensor-core Q.K^T and P.V on exact integer operands
-// with the dequantisation scales applied outside the MMA.
+// with the dequantisation scales applied outside the MMA, split-K across the
+// CTAs of a thread-block cluster combined through distributed shared memory.
 //
 // Method (what is computed): abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
 // module doc "Fused approach" -- Q.K^T with K dequantised on the fly,
 // softmax, P.V with V dequantised on the fly; combs-models 0.2.2, src/kv.rs,
 // attend / repeat_kv -- scale after the dot product, query head h reads kv
 // head h / G, a decode query attends to the whole cache.  Split-K with an
-// online softmax is this library's own (flash-decoding).
+// online softmax and the combine are this library's own (flash-decoding).
 //
 // How (sm_100a):
-//  * CTA = 4 consumer warps + 1 producer warp, one CTA per (sequence, kv
-//    head, split).  The producer streams 64-token stages of K and V bytes
-//    into shared memory with TMA tile loads (2-D tensor maps over the cache
-//    rows, 128-byte swizzle for D=128) and the fp32 scales with cp.async;
-//    both complete on the stage's mbarrier.  4 stages are in flight.
-//  * Consumer warp w owns the stages w, w+4, ...: for each 16-token slice it
-//    runs S = Q.K^T with mma.sync m16n8k16 (f16 in, f32 accumulate), rows =
-//    query heads of the GQA group (padded to 16), columns = tokens.  The
-//    operands are exact: K enters as the integers (byte - 128) built in
+//  * Grid (S, Hk, B): S splits of the KV range per (sequence, kv head).  With
+//    2 <= S <= 16 the S CTAs form one thread-block cluster and merge their
+//    partial softmax states through distributed shared memory (no global
+//    workspace, no second kernel).  Larger S (only on request) writes the
+//    partials to a workspace for the combine kernel in kvq_decode.cu.
+//  * CTA = 4 warps.  Warp 0 streams 64-token stages of K and V bytes into
+//    shared memory with TMA tile loads (2-D tensor maps over the cache rows,
+//    128-byte swizzle for D=128, 64-byte for D=64) and the fp32 scales with
+//    cp.async; both complete on the stage's mbarrier; 4 stages in flight.
+//    Every warp takes one 16-token slice of each stage.
+//  * Per slice: S = Q.K^T with mma.sync m16n8k16 (f16 in, f32 accumulate),
+//    rows = query heads of the GQA group (padded to 16), columns = tokens.
+//    The operands are exact: K enters as the integers (byte - 128) built in
 //    registers (1024 + byte spliced into an f16 mantissa, minus 1152), and Q
 //    enters as f16 after a per-head power-of-two prescale (bf16 has 8
 //    significant bits, f16 has 11, so q * 2^s is exact), so the f32
@@ -34,8 +39,8 @@
 //  * Token order inside each 16-token slice and the d order of the MMA
 //    k-dimension are permuted so that every shared-memory load of the
 //    swizzled tiles is free of bank conflicts (sigma below).
-//  * The four warps' (m, l, o) are merged in shared memory; the CTA writes
-//    its split (o, m, l) or, for a single-split sequence, the final row.
+//  * Every wait on an mbarrier is bounded; a wait that gives up sets
+//    KVQ_DEVERR_TIMEOUT and the kernel finishes without hanging.
 #include <cuda.h>
 #include <math.h>
 
@@ -45,10 +50,11 @@
 namespace kvq {
 namespace {
 
-constexpr int TT = 64;                 // tokens per stage
-constexpr int NCW = 4;                 // consumer warps
-constexpr int NTHREADS = (NCW + 1) * 32;
+constexpr int TT = 64;                 // tokens per stage: one 16-token slice per warp
+constexpr int NW = 4;                  // warps per CTA
+constexpr int NTHREADS = NW * 32;
 constexpr int NST = 4;                 // stages in flight
+constexpr int kMaxCluster = 16;        // largest cluster the combine supports
 
 // Row (inside an 8-token group) that holds MMA column n of the K operand and
 // MMA k-index n of the V operand: sigma = {0, 2, 4, 6, 3, 1, 7, 5}.  Under the
@@ -58,15 +64,6 @@ constexpr int NST = 4;                 // stages in flight
 // load instruction touches differ in bits 1..2.
 __device__ __forceinline__ int sigma(int x) { return x < 4 ? 2 * x : ((2 * x - 7) ^ 2); }
 
-template <int D, bool G32>
-struct Layout {
-    static constexpr int NG = G32 ? D / 32 : 1;
-    static constexpr int KV_BYTES = TT * D;
-    static constexpr int SC_FLOATS = TT * NG;
-    static constexpr int STAGE = ((2 * KV_BYTES + 2 * SC_FLOATS * 4) + 1023) / 1024 * 1024;
-    static constexpr int BAR_OFF = NST * STAGE;
-    static constexpr int SMEM = BAR_OFF + 2 * NST * 8 + 1024;   // + base alignment slack
-};
 
 // byte offset of (row, byte) inside a swizzled K or V stage tile
 template <int D>
@@ -120,8 +117,64 @@ __device__ __forceinline__ void copy_scales(uint32_t dst, const float* src) {
     else ptx::cp_async_16(dst, src);
 }
 
+template <int D, bool G32>
+struct Layout {
+    static constexpr int NG = G32 ? D / 32 : 1;
+    static constexpr int KV_BYTES = TT * D;
+    static constexpr int SC_FLOATS = TT * NG;
+    static constexpr int STAGE = ((2 * KV_BYTES + 2 * SC_FLOATS * 4) + 1023) / 1024 * 1024;
+    static constexpr int BAR_OFF = NST * STAGE;
+    static constexpr int NBAR = 2 * NST + 2;               // full[], empty[], done, read
+    static constexpr int SMEM = BAR_OFF + NBAR * 8 + 1024;  // + base alignment slack
+    // epilogue buffers, in floats, reusing the stage area once every stage is consumed
+    static constexpr int RS = D + 4;                       // warp-merge row stride
+    static constexpr int RED_M = NW * 16 * RS;             // [NW][16] running max
+    static constexpr int RED_L = RED_M + NW * 16;          // [NW][16] running sum
+    static constexpr int CPS = D + 2;                      // CTA partial row: o[D], m, l
+    static constexpr int CP = RED_L + NW * 16;             // [16][CPS]
+    static constexpr int CW = CP + 16 * CPS;               // [kMaxCluster][16] peer max / weights
+    static constexpr int CL = CW + kMaxCluster * 16;       // [kMaxCluster][16] peer sums
+    static constexpr int CSUM = CL + kMaxCluster * 16;     // [16] combined sums
+    static constexpr int EPI_FLOATS = CSUM + 16;
+    static_assert(EPI_FLOATS * 4 <= BAR_OFF, "epilogue buffers fit in the stage area");
+};
+
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+// Bounded wait with cluster-scope acquire (sees stores released by peers).
+__device__ __forceinline__ bool wait_cluster(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < ptx::kSpinLimit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+
 template <int D, bool G32, bool PAGED, bool G16>
-__global__ void __launch_bounds__(NTHREADS)
+__global__ void __launch_bounds__(NTHREADS, G16 ? 2 : 3)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 DecodeParams p) {
     using Lay = Layout<D, G32>;
@@ -138,114 +191,109 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tid = threadIdx.x;
     const int G = p.G;
+    const int S = p.cluster;            // CTAs in this kernel's cluster (1: none)
 
     const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
     const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
     int L = p.seq_lens[b];
     if (L < 0 || L > lim) {
-        if (j == 0 && hk == 0 && threadIdx.x == 0) raise_flag(p.d_err, KVQ_DEVERR_LEN);
+        if (j == 0 && hk == 0 && tid == 0) raise_flag(p.d_err, KVQ_DEVERR_LEN);
         L = 0;
     }
-    if (L == 0) {
-        if (j == 0)
-            for (int i = threadIdx.x; i < G * D; i += NTHREADS)
-                p.out[(static_cast<int64_t>(b) * p.Hq + hk * G) * D + i] = 0.f;
-        return;
-    }
+    // No CTA leaves early: in a cluster every CTA takes part in the combine.
     const int t0 = j * p.chunk;
-    if (t0 >= L) return;
-    const int t1 = min(t0 + p.chunk, L);
+    const bool active = t0 < L;
+    const int t1 = active ? min(t0 + p.chunk, L) : t0;
     const int nsplit = (L + p.chunk - 1) / p.chunk;
-    const int ntiles = (t1 - t0 + TT - 1) / TT;
+    const int ntiles = active ? (t1 - t0 + TT - 1) / TT : 0;
 
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t bar_full = sbase + Lay::BAR_OFF;
     const uint32_t bar_empty = bar_full + NST * 8;
-    if (threadIdx.x == 0) {
+    const uint32_t bar_done = bar_empty + NST * 8;     // all peers' partials are ready
+    const uint32_t bar_read = bar_done + 8;             // all peers finished reading ours
+    if (tid == 0) {
         for (int s = 0; s < NST; ++s) {
             ptx::mbar_init(bar_full + 8 * s, 1 + 32);   // expect_tx arrive + 32 cp.async arrivals
-            ptx::mbar_init(bar_empty + 8 * s, 1);
+            ptx::mbar_init(bar_empty + 8 * s, NW);
         }
+        ptx::mbar_init(bar_done, S);
+        ptx::mbar_init(bar_read, S);
         ptx::fence_mbar_init();
     }
     __syncthreads();
+    // peers arrive on our barriers only after every CTA has initialised them
+    if (S > 1) cluster_sync_all();
 
-    // ------------------------------------------------------------ producer
-    if (warp == NCW) {
-        if (lane == 0) {
-            ptx::prefetch_tensormap(&tm_k);
-            ptx::prefetch_tensormap(&tm_v);
-        }
-        const uint64_t pol = ptx::policy_evict_first();
-        for (int i = 0; i < ntiles; ++i) {
-            const int s = i % NST;
-            const uint32_t full = bar_full + 8 * s;
-            if (i >= NST && !ptx::mbar_wait(bar_empty + 8 * s, ((i / NST) - 1) & 1)) {
-                if (lane == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
-                break;
+    // ---- warp 0 issues stage i: TMA for K/V bytes, cp.async for the scales
+    const uint64_t pol = ptx::policy_evict_first();
+    auto issue = [&](int i) {
+        const int s = i % NST;
+        const uint32_t full = bar_full + 8 * s;
+        const int tt0 = t0 + i * TT;
+        const int ntok = min(TT, t1 - tt0);
+        const uint32_t sk = sbase + s * Lay::STAGE;
+        const uint32_t sv = sk + Lay::KV_BYTES;
+        const uint32_t sks = sv + Lay::KV_BYTES;
+        const uint32_t svs = sks + Lay::SC_FLOATS * 4;
+        if (!PAGED) {
+            const int64_t row0 = (static_cast<int64_t>(b) * p.Hk + hk) * p.max_seq + tt0;
+            if (lane == 0) {
+                ptx::mbar_arrive_expect_tx(full, 2 * Lay::KV_BYTES);
+                ptx::tma_load_2d(sk, &tm_k, 0, static_cast<int>(row0), full, pol);
+                ptx::tma_load_2d(sv, &tm_v, 0, static_cast<int>(row0), full, pol);
             }
-            const int tt0 = t0 + i * TT;
-            const int ntok = min(TT, t1 - tt0);
-            const uint32_t sk = sbase + s * Lay::STAGE;
-            const uint32_t sv = sk + Lay::KV_BYTES;
-            const uint32_t sks = sv + Lay::KV_BYTES;
-            const uint32_t svs = sks + Lay::SC_FLOATS * 4;
-            if (!PAGED) {
-                const int64_t row0 = (static_cast<int64_t>(b) * p.Hk + hk) * p.max_seq + tt0;
-                if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(full, 2 * Lay::KV_BYTES);
-                    ptx::tma_load_2d(sk, &tm_k, 0, static_cast<int>(row0), full, pol);
-                    ptx::tma_load_2d(sv, &tm_v, 0, static_cast<int>(row0), full, pol);
+            for (int k = lane; k < ntok; k += 32) {
+                const int64_t r = row0 + k;
+                copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
+                copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
+            }
+        } else {
+            const int np = (ntok + 15) >> 4;
+            int32_t pg = -1;
+            if (lane < np) {
+                pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tt0 >> 4) + lane];
+                if (pg < 0 || pg >= p.num_pages) {
+                    raise_flag(p.d_err, KVQ_DEVERR_PAGE);
+                    pg = -1;
                 }
-                for (int k = lane; k < ntok; k += 32) {
-                    const int64_t r = row0 + k;
+            }
+            const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
+            int pgs[TT / 16];
+#pragma unroll
+            for (int q = 0; q < TT / 16; ++q) pgs[q] = __shfl_sync(0xffffffffu, pg, q);
+            if (lane == 0) {
+                ptx::mbar_arrive_expect_tx(full, __popc(valid) * 2 * 16 * D);
+                for (int q = 0; q < np; ++q) {
+                    const int pq = pgs[q];
+                    if (pq < 0) continue;
+                    const int y = (pq * p.Hk + hk) * 16;
+                    ptx::tma_load_2d(sk + q * 16 * D, &tm_k, 0, y, full, pol);
+                    ptx::tma_load_2d(sv + q * 16 * D, &tm_v, 0, y, full, pol);
+                }
+            }
+            for (int k = lane; k < TT; k += 32) {
+                const int pk = __shfl_sync(0xffffffffu, pg, k >> 4);
+                if (k < ntok && pk >= 0) {
+                    const int64_t r = (static_cast<int64_t>(pk) * p.Hk + hk) * 16 + (k & 15);
                     copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
                     copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
                 }
-            } else {
-                const int np = (ntok + 15) >> 4;
-                int32_t pg = -1;
-                if (lane < np) {
-                    pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tt0 >> 4) + lane];
-                    if (pg < 0 || pg >= p.num_pages) {
-                        raise_flag(p.d_err, KVQ_DEVERR_PAGE);
-                        pg = -1;
-                    }
-                }
-                const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
-                int pgs[TT / 16];
-#pragma unroll
-                for (int q = 0; q < TT / 16; ++q) pgs[q] = __shfl_sync(0xffffffffu, pg, q);
-                if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(full, __popc(valid) * 2 * 16 * D);
-                    for (int q = 0; q < np; ++q) {
-                        const int pq = pgs[q];
-                        if (pq < 0) continue;
-                        const int y = (pq * p.Hk + hk) * 16;
-                        ptx::tma_load_2d(sk + q * 16 * D, &tm_k, 0, y, full, pol);
-                        ptx::tma_load_2d(sv + q * 16 * D, &tm_v, 0, y, full, pol);
-                    }
-                }
-                for (int k = lane; k < TT; k += 32) {
-                    const int pk = __shfl_sync(0xffffffffu, pg, k >> 4);
-                    if (k < ntok && pk >= 0) {
-                        const int64_t r = (static_cast<int64_t>(pk) * p.Hk + hk) * 16 + (k & 15);
-                        copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
-                        copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
-                    }
-                }
             }
-            ptx::cp_async_arrive_noinc(full);
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        return;
+        ptx::cp_async_arrive_noinc(full);
+    };
+    if (warp == 0) {
+        if (lane == 0 && ntiles > 0) {
+            ptx::prefetch_tensormap(&tm_k);
+            ptx::prefetch_tensormap(&tm_v);
+        }
+        for (int i = 0; i < min(NST, ntiles); ++i) issue(i);
     }
 
-    // ------------------------------------------------------------ consumers
     const int g = lane >> 2, t = lane & 3;
-    const int tid = threadIdx.x;                 // 0..127
-
     // Q fragments: rows = heads g (lo) and g + 8 (hi), pre-scaled by 2^s
     uint32_t qa0[KS], qa2[KS], qa1[KS], qa3[KS];
     float zs_lo = 0.f, zs_hi = 0.f;
@@ -291,12 +339,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 f2[2 * gi + h2] = ptx::pack_f16x2(qf[gi][4 * h2 + 2] * up, qf[gi][4 * h2 + 3] * up);
             }
     };
-    load_q(g, qa0, qa2, zs_lo);
-    if (G16) {
-        load_q(g + 8, qa1, qa3, zs_hi);
-    } else {
 #pragma unroll
-        for (int k = 0; k < KS; ++k) qa1[k] = qa3[k] = 0u;
+    for (int k = 0; k < KS; ++k) qa0[k] = qa1[k] = qa2[k] = qa3[k] = 0u;
+    if (ntiles > 0) {
+        load_q(g, qa0, qa2, zs_lo);
+        if (G16) load_q(g + 8, qa1, qa3, zs_hi);
     }
 
     float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
@@ -307,13 +354,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     int kv = 64;                         // running P'' prescale exponent (per warp)
     const int sig_g = sigma(g);
     const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
-    bool timed_out = false;
 
-    for (int i = warp; i < ntiles; i += NCW) {
+    for (int i = 0; i < ntiles; ++i) {
         const int s = i % NST;
         if (!ptx::mbar_wait(bar_full + 8 * s, (i / NST) & 1)) {
             if (lane == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
-            timed_out = true;
             break;
         }
         const int tt0 = t0 + i * TT;
@@ -321,11 +366,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const uint32_t sv = sk + Lay::KV_BYTES;
         const uint32_t sks = sv + Lay::KV_BYTES;
         const uint32_t svs = sks + Lay::SC_FLOATS * 4;
-
-#pragma unroll 1
-        for (int sub = 0; sub < TT / 16; ++sub) {
-            const int tok0 = tt0 + 16 * sub;
-            if (tok0 >= t1) break;
+        const int tok0 = tt0 + 16 * warp;             // this warp's 16-token slice
+        if (tok0 < t1) {
             bool page_ok = true;
             if (PAGED) {
                 const int32_t pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tok0 >> 4)];
@@ -340,7 +382,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     sacc[nt][a][0] = sacc[nt][a][1] = sacc[nt][a][2] = sacc[nt][a][3] = 0.f;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                const uint32_t row = 16 * sub + 8 * nt + sig_g;
+                const uint32_t row = 16 * warp + 8 * nt + sig_g;
                 uint2 kw[NGRP];
 #pragma unroll
                 for (int gi = 0; gi < NGRP; ++gi) kw[gi] = lds64(sk + swz<D>(row, 32 * gi + 8 * t));
@@ -363,7 +405,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    const int r = 16 * sub + 8 * nt + (c ? sig_b : sig_a);
+                    const int r = 16 * warp + 8 * nt + (c ? sig_b : sig_a);
                     ok[nt][c] = page_ok && (tt0 + r < t1);
                     float zl, zh;
                     if (G32) {
@@ -423,7 +465,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // P'' = p * v_scale * 2^kv with kv chosen so that the largest
             // v_scale * 2^kv seen by this warp lies in [2^14, 2^15); when kv
             // drops, the accumulated O is rescaled by the same power of two.
-            const int R0 = 16 * sub + sig_a, R1 = 16 * sub + sig_b;
+            const int R0 = 16 * warp + sig_a, R1 = 16 * warp + sig_b;
             const int R2 = R0 + 8, R3 = R1 + 8;
             const int rr[2][2] = {{R0, R1}, {R2, R3}};
             float vsc[2][2][NGV];
@@ -535,14 +577,18 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar_empty + 8 * s);
+        if (warp == 0 && i + NST < ntiles) {
+            // refill slot s once all four warps have released it
+            if (!ptx::mbar_wait(bar_empty + 8 * s, (i / NST) & 1)) {
+                if (lane == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
+                break;
+            }
+            issue(i + NST);
+        }
     }
-    (void)timed_out;
+    if (warp == 0) asm volatile("cp.async.wait_all;" ::: "memory");
 
-    // ---- merge the four warps' (m, l, o) and write the split / final row
-    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
-    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
-    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
-    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+    // ---- merge the four warps' (m, l, o) into the CTA partial
     {
         const float down = ldexpf(1.f, -kv);         // undo the P'' prescale
 #pragma unroll
@@ -553,11 +599,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             o_hi[n][1] *= down;
         }
     }
-    ptx::named_bar_sync(1, NCW * 32);             // all stages consumed: reuse shared memory
-    constexpr int RS = D + 4;                     // padded row stride (floats)
-    float* red = reinterpret_cast<float*>(smem);  // [NCW][16][RS]
-    float* red_m = red + NCW * 16 * RS;           // [NCW][16]
-    float* red_l = red_m + NCW * 16;
+    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+    __syncthreads();                              // every stage consumed: reuse shared memory
+    float* red = reinterpret_cast<float*>(smem);  // [NW][16][RS]
+    float* red_m = red + Lay::RED_M;
+    float* red_l = red + Lay::RED_L;
     // head_dim index of output n-tile n, column c (0/1) of this thread
     auto dcol = [&](int n, int c) -> int {
         if (G32) return 32 * (n >> 2) + 4 * (2 * t + c) + (n & 3);
@@ -567,8 +616,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     for (int n = 0; n < NTD; ++n)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            red[(warp * 16 + g) * RS + dcol(n, c)] = o_lo[n][c];
-            if (G16) red[(warp * 16 + g + 8) * RS + dcol(n, c)] = o_hi[n][c];
+            red[(warp * 16 + g) * Lay::RS + dcol(n, c)] = o_lo[n][c];
+            if (G16) red[(warp * 16 + g + 8) * Lay::RS + dcol(n, c)] = o_hi[n][c];
         }
     if (t == 0) {
         red_m[warp * 16 + g] = m_lo;
@@ -576,28 +625,87 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         red_m[warp * 16 + g + 8] = G16 ? m_hi : -INFINITY;
         red_l[warp * 16 + g + 8] = G16 ? l_hi : 0.f;
     }
-    ptx::named_bar_sync(1, NCW * 32);
-    for (int idx = tid; idx < G * D; idx += NCW * 32) {
+    __syncthreads();
+    float* cp = red + Lay::CP;                    // [16][CPS]: o (unnormalised), m, l
+    for (int idx = tid; idx < G * D; idx += NTHREADS) {
         const int h = idx / D, d = idx - h * D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < NCW; ++w) M = fmaxf(M, red_m[w * 16 + h]);
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * 16 + h]);
         float acc = 0.f, lsum = 0.f;
 #pragma unroll
-        for (int w = 0; w < NCW; ++w) {
+        for (int w = 0; w < NW; ++w) {
             const float mw = red_m[w * 16 + h];
             const float f = (mw == -INFINITY) ? 0.f : ptx::ex2(mw - M);
-            acc = fmaf(f, red[(w * 16 + h) * RS + d], acc);
+            acc = fmaf(f, red[(w * 16 + h) * Lay::RS + d], acc);
             lsum = fmaf(f, red_l[w * 16 + h], lsum);
         }
-        const int64_t bh = static_cast<int64_t>(b) * p.Hq + hk * G + h;
-        if (nsplit == 1) {
-            p.out[bh * D + d] = lsum > 0.f ? acc / lsum : 0.f;
-        } else {
-            p.ws_o[(bh * p.splits + j) * D + d] = acc;
+        cp[h * Lay::CPS + d] = acc;
+        if (d == 0) {
+            cp[h * Lay::CPS + D] = M;
+            cp[h * Lay::CPS + D + 1] = lsum;
+        }
+    }
+    __syncthreads();
+
+    const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
+    if (S > 1) {
+        // ---- cluster combine: partial j lives in CTA j's shared memory
+        const uint32_t cp_addr = ptx::smem_u32(cp);
+        if (tid < S) arrive_remote(mapa(bar_done, tid));
+        if (!wait_cluster(bar_done, 0) && tid == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
+        float* cw = red + Lay::CW;                // [S][16] peer max, then weights
+        float* cl = red + Lay::CL;                // [S][16] peer sums
+        float* csum = red + Lay::CSUM;            // [16]
+        for (int idx = tid; idx < S * G; idx += NTHREADS) {
+            const int r = idx / G, h = idx - r * G;
+            const uint32_t a = mapa(cp_addr + (h * Lay::CPS + D) * 4, r);
+            cw[r * 16 + h] = ld_cluster_f32(a);
+            cl[r * 16 + h] = ld_cluster_f32(a + 4);
+        }
+        __syncthreads();
+        if (tid < G) {
+            float M = -INFINITY;
+            for (int r = 0; r < S; ++r) M = fmaxf(M, cw[r * 16 + tid]);
+            float lsum = 0.f;
+            for (int r = 0; r < S; ++r) {
+                const float mr = cw[r * 16 + tid];
+                const float w = (mr == -INFINITY) ? 0.f : ptx::ex2(mr - M);
+                cw[r * 16 + tid] = w;
+                lsum = fmaf(w, cl[r * 16 + tid], lsum);
+            }
+            csum[tid] = lsum;
+        }
+        __syncthreads();
+        // this CTA writes outputs j*128 + tid, stepping by S*128
+        for (int idx = j * NTHREADS + tid; idx < G * D; idx += S * NTHREADS) {
+            const int h = idx / D, d = idx - h * D;
+            const uint32_t a = cp_addr + (h * Lay::CPS + d) * 4;
+            float acc = 0.f;
+            for (int r = 0; r < S; ++r) acc = fmaf(cw[r * 16 + h], ld_cluster_f32(mapa(a, r)), acc);
+            const float lsum = csum[h];
+            p.out[(bh0 + h) * D + d] = lsum > 0.f ? acc / lsum : 0.f;
+        }
+        __syncthreads();
+        // keep this CTA's shared memory alive until every peer has read it
+        if (tid < S) arrive_remote(mapa(bar_read, tid));
+        if (!wait_cluster(bar_read, 0) && tid == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
+    } else if (nsplit <= 1) {
+        // single split (or empty sequence): the final row
+        if (j == 0)
+            for (int idx = tid; idx < G * D; idx += NTHREADS) {
+                const int h = idx / D, d = idx - h * D;
+                const float lsum = cp[h * Lay::CPS + D + 1];
+                p.out[(bh0 + h) * D + d] = lsum > 0.f ? cp[h * Lay::CPS + d] / lsum : 0.f;
+            }
+    } else if (active) {
+        // many splits without a cluster: partials for the combine kernel
+        for (int idx = tid; idx < G * D; idx += NTHREADS) {
+            const int h = idx / D, d = idx - h * D;
+            p.ws_o[((bh0 + h) * p.splits + j) * D + d] = cp[h * Lay::CPS + d];
             if (d == 0) {
-                p.ws_m[bh * p.splits + j] = M;
-                p.ws_l[bh * p.splits + j] = lsum;
+                p.ws_m[(bh0 + h) * p.splits + j] = cp[h * Lay::CPS + D];
+                p.ws_l[(bh0 + h) * p.splits + j] = cp[h * Lay::CPS + D + 1];
             }
         }
     }
@@ -638,26 +746,48 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
 }
 
 template <int D, bool G32, bool PAGED, bool G16>
+cudaError_t set_attrs() {
+    using Lay = Layout<D, G32>;
+    static bool done = false;
+    if (done) return cudaSuccess;
+    auto kern = decode_split_tc<D, G32, PAGED, G16>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e == cudaSuccess) done = true;
+    return e;
+}
+
+template <int D, bool G32, bool PAGED, bool G16>
 cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     using Lay = Layout<D, G32>;
-    static bool attr_done = false;
-    auto kern = decode_split_tc<D, G32, PAGED, G16>;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Lay::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+    cudaError_t e = set_attrs<D, G32, PAGED, G16>();
+    if (e != cudaSuccess) return e;
     CUtensorMap mk, mv;
     const int64_t rows = PAGED ? static_cast<int64_t>(p.num_pages) * p.Hk * 16
                                : static_cast<int64_t>(p.B) * p.Hk * p.max_seq;
     const int box = PAGED ? 16 : TT;
-    cudaError_t e = make_map(&mk, p.k, D, rows, box);
+    e = make_map(&mk, p.k, D, rows, box);
     if (e == cudaSuccess) e = make_map(&mv, p.v, D, rows, box);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.splits, p.Hk, p.B);
-    kern<<<grid, NTHREADS, Lay::SMEM, s>>>(mk, mv, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.splits, p.Hk, p.B);
+    cfg.blockDim = dim3(NTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = Lay::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    if (p.cluster > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = p.cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16>, mk, mv, p);
 }
 
 template <int D, bool G32, bool PAGED>
@@ -675,9 +805,37 @@ cudaError_t pick_layout(const DecodeParams& p, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s) {
+    if (p.cluster > kMaxCluster || (p.cluster > 1 && p.cluster != p.splits))
+        return cudaErrorInvalidValue;
     if (p.D == 128) return pick_layout<128>(p, s);
     if (p.D == 64) return pick_layout<64>(p, s);
     return cudaErrorInvalidValue;
+}
+
+int decode_max_cluster() {
+    static int cached = 0;
+    if (cached) return cached;
+    // the most demanding variant (registers, shared memory) bounds every other
+    auto kern = decode_split_tc<128, true, true, true>;
+    int n = 0;
+    if (set_attrs<128, true, true, true>() == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kMaxCluster, 1, 1);
+        cfg.blockDim = dim3(NTHREADS, 1, 1);
+        cfg.dynamicSmemBytes = Layout<128, true>::SMEM;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kMaxCluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxPotentialClusterSize(&n, kern, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();                           // a failed query leaves no sticky error
+    n = n < 1 ? 1 : (n > kMaxCluster ? kMaxCluster : n);
+    cached = n;
+    return n;
 }
 
 }  // namespace kvq

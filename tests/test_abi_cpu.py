@@ -69,11 +69,17 @@ def test_decode_plan_covers_hint(kvq, B, Hk, hint, ns):
 
 
 def test_decode_plan_fills_the_machine(kvq):
-    # one Llama-3-8B layer: 8 (sequence, kv head) units need splits to fill 148 SMs
+    # few (sequence, kv head) units: up to one 16-CTA cluster of splits per unit
     chunk, splits = kvq.kvq_decode_plan(1, 8, 4097, 0, num_sms=148)
-    assert 8 * splits >= 148
+    assert splits == 16 and chunk == 272
     chunk, splits = kvq.kvq_decode_plan(1, 8, 131073, 0, num_sms=148)
-    assert 8 * splits >= 148
+    assert splits == 16
+    # enough units to fill the machine twice over: no split at all
+    chunk, splits = kvq.kvq_decode_plan(37, 8, 16385, 0, num_sms=148)
+    assert splits == 1
+    # explicit split counts beyond one cluster are honoured (combine kernel path)
+    chunk, splits = kvq.kvq_decode_plan(1, 8, 4097, 64, num_sms=148)
+    assert 16 < splits <= 64
 
 
 def test_workspace_formula(kvq):
