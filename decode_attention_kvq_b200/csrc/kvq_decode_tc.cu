@@ -16,31 +16,34 @@
 //    partial softmax states through distributed shared memory (no global
 //    workspace, no second kernel).  Larger S (only on request) writes the
 //    partials to a workspace for the combine kernel in kvq_decode.cu.
-//  * CTA = 4 warps.  Warp 0 streams 64-token stages of K and V bytes into
+//  * CTA = 8 warps.  Warp 0 streams 128-token stages of K and V bytes into
 //    shared memory with TMA tile loads (2-D tensor maps over the cache rows,
 //    128-byte swizzle for D=128, 64-byte for D=64) and the fp32 scales with
-//    cp.async; both complete on the stage's mbarrier; 4 stages in flight.
+//    cp.async; both complete on the stage's mbarrier; 3 stages in flight.
 //    Every warp takes one 16-token slice of each stage.
-//  * Per slice: S = Q.K^T with mma.sync m16n8k16 (f16 in, f32 accumulate),
-//    rows = query heads of the GQA group (padded to 16), columns = tokens.
-//    The operands are exact: K enters as the integers (byte - 128) built in
+//  * Per slice, on mma.sync m16n8k16 (f16 in, f32 accumulate), with the
+//    query heads of the GQA group as the N = 8 dimension (two n-tiles when
+//    G > 8):  S^T = K . Q^T (M = 16 tokens, K = head_dim) and
+//    O^T += V^T . P^T (M = 16 head_dim rows, K = 16 tokens).  The operands
+//    are exact: K and V enter as the integers (byte - 128) built in
 //    registers (1024 + byte spliced into an f16 mantissa, minus 1152), and Q
 //    enters as f16 after a per-head power-of-two prescale (bf16 has 8
-//    significant bits, f16 has 11, so q * 2^s is exact), so the f32
-//    accumulators hold sum_d q_d (k_d - 128) up to accumulation rounding.
-//    The K scale (per token, or per 32-value group with one accumulator per
-//    group), 2^-s, attn_scale and log2(e) are applied to the accumulator.
-//  * Online softmax in base 2 per head row.  The V scale is folded into P:
+//    significant bits, f16 has 11, so q * 2^s is exact).  The K scale (per
+//    token, or per 32-value group with one accumulator per group), 2^-s,
+//    attn_scale and log2(e) are applied to the f32 scores.
+//  * Online softmax in base 2 per head.  The V scale is folded into P:
 //    P'' = 2^(z-m) * v_scale(token) * 2^kv (per 32-value group in group-32
 //    mode), with a running per-warp power of two 2^kv that keeps P'' inside
 //    the f16 normal range.  P'' is split into f16 hi + lo parts (about 22
-//    significant bits together) and both are multiplied with the exact
-//    integers (v - 128), so P.V carries no f16 rounding of P beyond ~2^-22.
-//  * Token order inside each 16-token slice and the d order of the MMA
-//    k-dimension are permuted so that every shared-memory load of the
+//    significant bits together); each part is transposed from the score
+//    accumulator layout into the P^T operand layout with movmatrix and
+//    multiplied with the exact (v - 128) integers.
+//  * Token order inside each 16-token slice and the head_dim order of the
+//    MMA k-dimension are permuted so that every shared-memory load of the
 //    swizzled tiles is free of bank conflicts (sigma below).
-//  * Every wait on an mbarrier is bounded; a wait that gives up sets
-//    KVQ_DEVERR_TIMEOUT and the kernel finishes without hanging.
+//  * mbarrier waits are bounded (KVQ_DEVERR_TIMEOUT when one gives up); the
+//    only unbounded waits are the CTA and cluster barriers, which every
+//    thread of every CTA reaches unconditionally.
 #include <cuda.h>
 #include <math.h>
 
@@ -50,20 +53,69 @@
 namespace kvq {
 namespace {
 
-constexpr int TT = 64;                 // tokens per stage: one 16-token slice per warp
-constexpr int NW = 4;                  // warps per CTA
+constexpr int NW = 8;                  // warps per CTA
 constexpr int NTHREADS = NW * 32;
-constexpr int NST = 4;                 // stages in flight
+constexpr int TT = 16 * NW;            // tokens per stage: one 16-token slice per warp
+constexpr int NST = 3;                 // stages in flight
 constexpr int kMaxCluster = 16;        // largest cluster the combine supports
 
-// Row (inside an 8-token group) that holds MMA column n of the K operand and
-// MMA k-index n of the V operand: sigma = {0, 2, 4, 6, 3, 1, 7, 5}.  Under the
-// 128-byte swizzle (16-byte chunk index XOR row % 8) this makes the K loads
+// Row (inside an 8-token half of a slice) that holds MMA row r of the K
+// operand and MMA k-index r of the V operand: sigma = {0, 2, 4, 6, 3, 1, 7, 5}.
+// Under the 128-byte swizzle (16-byte chunk index XOR row % 8) the rows that
+// one load instruction touches then differ in bits 1..2, so the K loads
 // (rows sigma(g), 8 bytes at 32*G + 8*t) and the V loads (rows sigma(2t),
-// sigma(2t+1), 16 bytes at 16*g) of a warp hit distinct banks: the rows a
-// load instruction touches differ in bits 1..2.
+// sigma(2t+1), 16 bytes at 16*g) of a warp hit distinct banks.
 __device__ __forceinline__ int sigma(int x) { return x < 4 ? 2 * x : ((2 * x - 7) ^ 2); }
 
+// (a, b) -> f16x2 hi = rn(a, b) and lo = rn(a - hi, b - hi): hi + lo carries
+// about 22 significant bits of each value.
+__device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const __half2 h = __floats2half2_rn(a, b);
+    const float2 f = __half22float2(h);
+    const __half2 l = __floats2half2_rn(a - f.x, b - f.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// 8x8 b16 transpose across the warp (fragment of row lane/4, columns
+// 2*(lane%4) and +1, in and out).
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// The NG fp32 scales of one token (4, 8 or 16 bytes, aligned to their size
+// because the scale array is 16-byte aligned and rows are NG floats apart).
+template <int NG>
+__device__ __forceinline__ void copy_scales(uint32_t dst, const float* src) {
+    static_assert(NG == 1 || NG == 2 || NG == 4, "scales per token");
+    if constexpr (NG == 1) ptx::cp_async_4(dst, src);
+    else if constexpr (NG == 2) ptx::cp_async_8(dst, src);
+    else ptx::cp_async_16(dst, src);
+}
+
+template <int D, bool G32>
+struct Layout {
+    static constexpr int NG = G32 ? D / 32 : 1;
+    static constexpr int KV_BYTES = TT * D;
+    static constexpr int SC_FLOATS = TT * NG;
+    static constexpr int STAGE = ((2 * KV_BYTES + 2 * SC_FLOATS * 4) + 1023) / 1024 * 1024;
+    static constexpr int BAR_OFF = NST * STAGE;
+    static constexpr int NBAR = 2 * NST;                   // full[], empty[]
+    static constexpr int SMEM = BAR_OFF + NBAR * 8 + 1024;  // + base alignment slack
+    // epilogue buffers, in floats, reusing the stage area once every stage is consumed
+    static constexpr int RS = D + 4;                       // warp-merge row stride
+    static constexpr int RED_M = NW * 16 * RS;             // [NW][16] running max
+    static constexpr int RED_L = RED_M + NW * 16;          // [NW][16] running sum
+    static constexpr int CPS = D + 2;                      // CTA partial row: o[D], m, l
+    static constexpr int CP = RED_L + NW * 16;             // [16][CPS]
+    static constexpr int CW = CP + 16 * CPS;               // [kMaxCluster][16] peer max / weights
+    static constexpr int CL = CW + kMaxCluster * 16;       // [kMaxCluster][16] peer sums
+    static constexpr int CSUM = CL + kMaxCluster * 16;     // [16] combined sums
+    static constexpr int EPI_FLOATS = CSUM + 16;
+    static_assert(EPI_FLOATS * 4 <= BAR_OFF, "epilogue buffers fit in the stage area");
+};
 
 // byte offset of (row, byte) inside a swizzled K or V stage tile
 template <int D>
@@ -97,48 +149,6 @@ __device__ __forceinline__ float ldsf(uint32_t a) {
     return v;
 }
 
-// (a, b) -> f16x2 hi = rn(a, b) and lo = rn(a - hi, b - hi): hi + lo carries
-// about 22 significant bits of each value.
-__device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
-    const __half2 h = __floats2half2_rn(a, b);
-    const float2 f = __half22float2(h);
-    const __half2 l = __floats2half2_rn(a - f.x, b - f.y);
-    hi = *reinterpret_cast<const uint32_t*>(&h);
-    lo = *reinterpret_cast<const uint32_t*>(&l);
-}
-
-// The NG fp32 scales of one token (4, 8 or 16 bytes, aligned to their size
-// because the scale array is 16-byte aligned and rows are NG floats apart).
-template <int NG>
-__device__ __forceinline__ void copy_scales(uint32_t dst, const float* src) {
-    static_assert(NG == 1 || NG == 2 || NG == 4, "scales per token");
-    if constexpr (NG == 1) ptx::cp_async_4(dst, src);
-    else if constexpr (NG == 2) ptx::cp_async_8(dst, src);
-    else ptx::cp_async_16(dst, src);
-}
-
-template <int D, bool G32>
-struct Layout {
-    static constexpr int NG = G32 ? D / 32 : 1;
-    static constexpr int KV_BYTES = TT * D;
-    static constexpr int SC_FLOATS = TT * NG;
-    static constexpr int STAGE = ((2 * KV_BYTES + 2 * SC_FLOATS * 4) + 1023) / 1024 * 1024;
-    static constexpr int BAR_OFF = NST * STAGE;
-    static constexpr int NBAR = 2 * NST + 2;               // full[], empty[], done, read
-    static constexpr int SMEM = BAR_OFF + NBAR * 8 + 1024;  // + base alignment slack
-    // epilogue buffers, in floats, reusing the stage area once every stage is consumed
-    static constexpr int RS = D + 4;                       // warp-merge row stride
-    static constexpr int RED_M = NW * 16 * RS;             // [NW][16] running max
-    static constexpr int RED_L = RED_M + NW * 16;          // [NW][16] running sum
-    static constexpr int CPS = D + 2;                      // CTA partial row: o[D], m, l
-    static constexpr int CP = RED_L + NW * 16;             // [16][CPS]
-    static constexpr int CW = CP + 16 * CPS;               // [kMaxCluster][16] peer max / weights
-    static constexpr int CL = CW + kMaxCluster * 16;       // [kMaxCluster][16] peer sums
-    static constexpr int CSUM = CL + kMaxCluster * 16;     // [16] combined sums
-    static constexpr int EPI_FLOATS = CSUM + 16;
-    static_assert(EPI_FLOATS * 4 <= BAR_OFF, "epilogue buffers fit in the stage area");
-};
-
 __device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
@@ -149,39 +159,23 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
     return v;
 }
-__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
-}
-// Bounded wait with cluster-scope acquire (sees stores released by peers).
-__device__ __forceinline__ bool wait_cluster(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < ptx::kSpinLimit; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (done) return true;
-    }
-    return false;
-}
+// Cluster-wide barrier: stores before it (release) are visible to every CTA
+// of the cluster after it (acquire).
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                  ::: "memory");
 }
 
 template <int D, bool G32, bool PAGED, bool G16>
-__global__ void __launch_bounds__(NTHREADS, G16 ? 2 : 3)
+__global__ void __launch_bounds__(NTHREADS, G16 ? 1 : 2)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 DecodeParams p) {
     using Lay = Layout<D, G32>;
     constexpr int NG = Lay::NG;
-    constexpr int KS = D / 16;          // MMA k-steps over head_dim
+    constexpr int KS = D / 16;          // MMA k-steps over head_dim (QK)
     constexpr int NGRP = D / 32;        // 32-value groups over head_dim
-    constexpr int NTD = D / 8;          // output n-tiles over head_dim
+    constexpr int MT = D / 16;          // m-tiles of O^T over head_dim (PV)
+    constexpr int NT = G16 ? 2 : 1;     // n-tiles of 8 query heads
     constexpr int NACC = G32 ? NG : 1;  // score accumulators per n-tile
     constexpr int NGV = G32 ? NG : 1;   // V scales per token
 
@@ -192,6 +186,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tid = threadIdx.x;
+    const int g = lane >> 2, t = lane & 3;
     const int G = p.G;
     const int S = p.cluster;            // CTAs in this kernel's cluster (1: none)
 
@@ -212,20 +207,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t bar_full = sbase + Lay::BAR_OFF;
     const uint32_t bar_empty = bar_full + NST * 8;
-    const uint32_t bar_done = bar_empty + NST * 8;     // all peers' partials are ready
-    const uint32_t bar_read = bar_done + 8;             // all peers finished reading ours
     if (tid == 0) {
         for (int s = 0; s < NST; ++s) {
             ptx::mbar_init(bar_full + 8 * s, 1 + 32);   // expect_tx arrive + 32 cp.async arrivals
             ptx::mbar_init(bar_empty + 8 * s, NW);
         }
-        ptx::mbar_init(bar_done, S);
-        ptx::mbar_init(bar_read, S);
         ptx::fence_mbar_init();
     }
     __syncthreads();
-    // peers arrive on our barriers only after every CTA has initialised them
-    if (S > 1) cluster_sync_all();
 
     // ---- warp 0 issues stage i: TMA for K/V bytes, cp.async for the scales
     const uint64_t pol = ptx::policy_evict_first();
@@ -251,6 +240,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
             }
         } else {
+            constexpr int PPS = TT / 16;                // pages per stage
             const int np = (ntok + 15) >> 4;
             int32_t pg = -1;
             if (lane < np) {
@@ -261,14 +251,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
             }
             const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
-            int pgs[TT / 16];
+            if (lane == 0) ptx::mbar_arrive_expect_tx(full, __popc(valid) * 2 * 16 * D);
 #pragma unroll
-            for (int q = 0; q < TT / 16; ++q) pgs[q] = __shfl_sync(0xffffffffu, pg, q);
-            if (lane == 0) {
-                ptx::mbar_arrive_expect_tx(full, __popc(valid) * 2 * 16 * D);
-                for (int q = 0; q < np; ++q) {
-                    const int pq = pgs[q];
-                    if (pq < 0) continue;
+            for (int q = 0; q < PPS; ++q) {
+                const int pq = __shfl_sync(0xffffffffu, pg, q);
+                if (lane == 0 && pq >= 0) {
                     const int y = (pq * p.Hk + hk) * 16;
                     ptx::tma_load_2d(sk + q * 16 * D, &tm_k, 0, y, full, pol);
                     ptx::tma_load_2d(sv + q * 16 * D, &tm_v, 0, y, full, pol);
@@ -293,67 +280,90 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int i = 0; i < min(NST, ntiles); ++i) issue(i);
     }
 
-    const int g = lane >> 2, t = lane & 3;
-    // Q fragments: rows = heads g (lo) and g + 8 (hi), pre-scaled by 2^s
-    uint32_t qa0[KS], qa2[KS], qa1[KS], qa3[KS];
-    float zs_lo = 0.f, zs_hi = 0.f;
-    const float sc_log2 = p.scale_log2;
-    auto load_q = [&](int h, uint32_t* f0, uint32_t* f2, float& zs) {
-        float qf[NGRP][8];
-        float amax = 0.f;
-        if (h < G) {
-            const uint16_t* qrow = p.q + (static_cast<int64_t>(b) * p.Hq + hk * G + h) * D;
+    // ---- Q^T operand: column n = g of n-tile nt is query head 8*nt + g,
+    // pre-scaled by 2^sh so that max |q| * 2^sh lies in [2^14, 2^15).
+    // B fragment rows 2t, 2t+1 (qb0) and 2t+8, 2t+9 (qb1) of k-step 2*gi + h2
+    // hold head_dim 32*gi + 8*t + 4*h2 + {0, 1} and {2, 3}.
+    uint32_t qb0[NT][KS], qb1[NT][KS];
+    float zsq[NT];                      // 2^-sh * attn_scale * log2(e) of head 8*nt + g
 #pragma unroll
-            for (int gi = 0; gi < NGRP; ++gi) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(qrow + 32 * gi + 8 * t);
-                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    for (int nt = 0; nt < NT; ++nt) {
+        zsq[nt] = 0.f;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    qf[gi][2 * e] = bf16_bits_to_f32(w[e] & 0xffffu);
-                    qf[gi][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
+        for (int k = 0; k < KS; ++k) qb0[nt][k] = qb1[nt][k] = 0u;
+    }
+    if (ntiles > 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int h = 8 * nt + g;
+            float qf[NGRP][8];
+            float amax = 0.f;
+            if (h < G) {
+                const uint16_t* qrow = p.q + (static_cast<int64_t>(b) * p.Hq + hk * G + h) * D;
+#pragma unroll
+                for (int gi = 0; gi < NGRP; ++gi) {
+                    const uint4 raw = *reinterpret_cast<const uint4*>(qrow + 32 * gi + 8 * t);
+                    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        qf[gi][2 * e] = bf16_bits_to_f32(w[e] & 0xffffu);
+                        qf[gi][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(qf[gi][e]));
                 }
+            } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(qf[gi][e]));
+                for (int gi = 0; gi < NGRP; ++gi)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) qf[gi][e] = 0.f;
             }
-        } else {
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            int sh = 0;
+            if (amax > 0.f) {
+                const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+                sh = min(max(14 - e, -100), 100);
+            }
+            const float up = ldexpf(1.f, sh);
+            zsq[nt] = ldexpf(1.f, -sh) * p.scale_log2;
 #pragma unroll
             for (int gi = 0; gi < NGRP; ++gi)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) qf[gi][e] = 0.f;
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    qb0[nt][2 * gi + h2] =
+                        ptx::pack_f16x2(qf[gi][4 * h2] * up, qf[gi][4 * h2 + 1] * up);
+                    qb1[nt][2 * gi + h2] =
+                        ptx::pack_f16x2(qf[gi][4 * h2 + 2] * up, qf[gi][4 * h2 + 3] * up);
+                }
         }
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        // power-of-two prescale: max |q| * 2^s in [2^14, 2^15)
-        int sh = 0;
-        if (amax > 0.f) {
-            const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
-            sh = min(max(14 - e, -100), 100);
-        }
-        const float up = ldexpf(1.f, sh);
-        zs = ldexpf(1.f, -sh) * sc_log2;
+    }
+    // score factor of the two heads (columns 2t, 2t+1) this thread accumulates
+    float zs[NT][2];
 #pragma unroll
-        for (int gi = 0; gi < NGRP; ++gi)
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                f0[2 * gi + h2] = ptx::pack_f16x2(qf[gi][4 * h2] * up, qf[gi][4 * h2 + 1] * up);
-                f2[2 * gi + h2] = ptx::pack_f16x2(qf[gi][4 * h2 + 2] * up, qf[gi][4 * h2 + 3] * up);
-            }
-    };
-#pragma unroll
-    for (int k = 0; k < KS; ++k) qa0[k] = qa1[k] = qa2[k] = qa3[k] = 0u;
-    if (ntiles > 0) {
-        load_q(g, qa0, qa2, zs_lo);
-        if (G16) load_q(g + 8, qa1, qa3, zs_hi);
+    for (int nt = 0; nt < NT; ++nt) {
+        zs[nt][0] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t));
+        zs[nt][1] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t + 1));
     }
 
-    float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
-    float o_lo[NTD][2], o_hi[NTD][2];
+    // ---- per-warp online softmax state: heads 8*nt + 2t + c
+    float m[NT][2], l[NT][2];
+    float o[MT][NT][4];                 // O^T C fragments: rows = head_dim, columns = heads
 #pragma unroll
-    for (int n = 0; n < NTD; ++n) o_lo[n][0] = o_lo[n][1] = o_hi[n][0] = o_hi[n][1] = 0.f;
-
+    for (int nt = 0; nt < NT; ++nt) {
+        m[nt][0] = m[nt][1] = -INFINITY;
+        l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+    }
     int kv = 64;                         // running P'' prescale exponent (per warp)
+
     const int sig_g = sigma(g);
     const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
+    const int rowA = 16 * warp + sig_g;           // MMA row g     of this warp's slice
+    const int rowB = rowA + 8;                    // MMA row g + 8
+    const int R0 = 16 * warp + sig_a, R1 = 16 * warp + sig_b;   // V rows of k 2t, 2t+1
+    const int R2 = R0 + 8, R3 = R1 + 8;                         // V rows of k 2t+8, 2t+9
 
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % NST;
@@ -366,211 +376,198 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const uint32_t sv = sk + Lay::KV_BYTES;
         const uint32_t sks = sv + Lay::KV_BYTES;
         const uint32_t svs = sks + Lay::SC_FLOATS * 4;
-        const int tok0 = tt0 + 16 * warp;             // this warp's 16-token slice
+        const int tok0 = tt0 + 16 * warp;             // first token of this warp's slice
         if (tok0 < t1) {
             bool page_ok = true;
             if (PAGED) {
                 const int32_t pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tok0 >> 4)];
                 page_ok = pg >= 0 && pg < p.num_pages;
             }
-            // ---- S = Q.K^T on 16 tokens: two n-tiles of 8
-            float sacc[2][NACC][4];
+            const bool okA = page_ok && (tok0 + sig_g < t1);
+            const bool okB = page_ok && (tok0 + 8 + sig_g < t1);
+
+            // ---- S^T = K . Q^T: rows tokens (rowA, rowB), columns heads
+            float sacc[NT][NACC][4];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int a = 0; a < NACC; ++a)
                     sacc[nt][a][0] = sacc[nt][a][1] = sacc[nt][a][2] = sacc[nt][a][3] = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const uint32_t row = 16 * warp + 8 * nt + sig_g;
-                uint2 kw[NGRP];
+            for (int gi = 0; gi < NGRP; ++gi) {
+                const uint2 wa = lds64(sk + swz<D>(rowA, 32 * gi + 8 * t));
+                const uint2 wb = lds64(sk + swz<D>(rowB, 32 * gi + 8 * t));
 #pragma unroll
-                for (int gi = 0; gi < NGRP; ++gi) kw[gi] = lds64(sk + swz<D>(row, 32 * gi + 8 * t));
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const uint32_t xa = h2 ? wa.y : wa.x;
+                    const uint32_t xb = h2 ? wb.y : wb.x;
+                    const uint32_t a0 = ptx::bytes_to_f16x2(xa, 0x4140u);
+                    const uint32_t a2 = ptx::bytes_to_f16x2(xa, 0x4342u);
+                    const uint32_t a1 = ptx::bytes_to_f16x2(xb, 0x4140u);
+                    const uint32_t a3 = ptx::bytes_to_f16x2(xb, 0x4342u);
 #pragma unroll
-                for (int gi = 0; gi < NGRP; ++gi)
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const uint32_t w = h2 ? kw[gi].y : kw[gi].x;
-                        const uint32_t b0 = ptx::bytes_to_f16x2(w, 0x4140u);
-                        const uint32_t b1 = ptx::bytes_to_f16x2(w, 0x4342u);
-                        const int ks = 2 * gi + h2;
-                        ptx::mma_f16(sacc[nt][G32 ? gi : 0], qa0[ks], qa1[ks], qa2[ks], qa3[ks],
-                                     b0, b1);
-                    }
+                    for (int nt = 0; nt < NT; ++nt)
+                        ptx::mma_f16(sacc[nt][G32 ? gi : 0], a0, a1, a2, a3, qb0[nt][2 * gi + h2],
+                                     qb1[nt][2 * gi + h2]);
+                }
             }
-            // ---- scores (log2 domain), masked
-            float z_lo[2][2], z_hi[2][2];
-            bool ok[2][2];
+            // ---- scores z (log2 domain): [nt][0..1] token rowA, [nt][2..3] token rowB
+            float z[NT][4];
+            if (G32) {
+                float ksa[NG], ksb[NG];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+                for (int a = 0; a < NG; ++a) {
+                    ksa[a] = ldsf(sks + (rowA * NG + a) * 4);
+                    ksb[a] = ldsf(sks + (rowB * NG + a) * 4);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float za0 = 0.f, za1 = 0.f, zb0 = 0.f, zb1 = 0.f;
+#pragma unroll
+                    for (int a = 0; a < NACC; ++a) {
+                        za0 = fmaf(sacc[nt][a][0], ksa[a], za0);
+                        za1 = fmaf(sacc[nt][a][1], ksa[a], za1);
+                        zb0 = fmaf(sacc[nt][a][2], ksb[a], zb0);
+                        zb1 = fmaf(sacc[nt][a][3], ksb[a], zb1);
+                    }
+                    z[nt][0] = okA ? za0 * zs[nt][0] : -INFINITY;
+                    z[nt][1] = okA ? za1 * zs[nt][1] : -INFINITY;
+                    z[nt][2] = okB ? zb0 * zs[nt][0] : -INFINITY;
+                    z[nt][3] = okB ? zb1 * zs[nt][1] : -INFINITY;
+                }
+            } else {
+                const float ksa = ldsf(sks + rowA * 4), ksb = ldsf(sks + rowB * 4);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    z[nt][0] = okA ? sacc[nt][0][0] * ksa * zs[nt][0] : -INFINITY;
+                    z[nt][1] = okA ? sacc[nt][0][1] * ksa * zs[nt][1] : -INFINITY;
+                    z[nt][2] = okB ? sacc[nt][0][2] * ksb * zs[nt][0] : -INFINITY;
+                    z[nt][3] = okB ? sacc[nt][0][3] * ksb * zs[nt][1] : -INFINITY;
+                }
+            }
+            // ---- online softmax per head: max over the slice's 16 tokens
+            float pr[NT][4];
+            float f[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    const int r = 16 * warp + 8 * nt + (c ? sig_b : sig_a);
-                    ok[nt][c] = page_ok && (tt0 + r < t1);
-                    float zl, zh;
-                    if (G32) {
-                        zl = 0.f;
-                        zh = 0.f;
-#pragma unroll
-                        for (int a = 0; a < NACC; ++a) {
-                            const float ksc = ldsf(sks + (r * NG + a) * 4);
-                            zl = fmaf(sacc[nt][a][c], ksc, zl);
-                            zh = fmaf(sacc[nt][a][2 + c], ksc, zh);
-                        }
-                    } else {
-                        const float ksc = ldsf(sks + r * 4);
-                        zl = sacc[nt][0][c] * ksc;
-                        zh = sacc[nt][0][2 + c] * ksc;
-                    }
-                    z_lo[nt][c] = ok[nt][c] ? zl * zs_lo : -INFINITY;
-                    z_hi[nt][c] = ok[nt][c] ? zh * zs_hi : -INFINITY;
+                    float mx = fmaxf(z[nt][c], z[nt][2 + c]);
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    const float mn = fmaxf(m[nt][c], mx);
+                    const float al = (mn == -INFINITY) ? 1.f : ptx::ex2(m[nt][c] - mn);
+                    pr[nt][c] = okA ? ptx::ex2(z[nt][c] - mn) : 0.f;
+                    pr[nt][2 + c] = okB ? ptx::ex2(z[nt][2 + c] - mn) : 0.f;
+                    l[nt][c] = l[nt][c] * al + pr[nt][c] + pr[nt][2 + c];
+                    m[nt][c] = mn;
+                    f[nt][c] = al;
                 }
-            // ---- online softmax, rows g (lo) and g + 8 (hi)
-            float mx_lo = fmaxf(fmaxf(z_lo[0][0], z_lo[0][1]), fmaxf(z_lo[1][0], z_lo[1][1]));
-            mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
-            mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
-            const float mn_lo = fmaxf(m_lo, mx_lo);
-            const float al_lo = (mn_lo == -INFINITY) ? 1.f : ptx::ex2(m_lo - mn_lo);
-            float pr_lo[2][2], pr_hi[2][2];
-            float ps_lo = 0.f, ps_hi = 0.f;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    pr_lo[nt][c] = ok[nt][c] ? ptx::ex2(z_lo[nt][c] - mn_lo) : 0.f;
-                    pr_hi[nt][c] = 0.f;
-                    ps_lo += pr_lo[nt][c];
-                }
-            l_lo = l_lo * al_lo + ps_lo;
-            m_lo = mn_lo;
-            float al_hi = 1.f;
-            if (G16) {
-                float mx_hi = fmaxf(fmaxf(z_hi[0][0], z_hi[0][1]), fmaxf(z_hi[1][0], z_hi[1][1]));
-                mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
-                mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
-                const float mn_hi = fmaxf(m_hi, mx_hi);
-                al_hi = (mn_hi == -INFINITY) ? 1.f : ptx::ex2(m_hi - mn_hi);
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        pr_hi[nt][c] = ok[nt][c] ? ptx::ex2(z_hi[nt][c] - mn_hi) : 0.f;
-                        ps_hi += pr_hi[nt][c];
-                    }
-                l_hi = l_hi * al_hi + ps_hi;
-                m_hi = mn_hi;
-            }
-
-            // ---- V scales of this slice and the running power-of-two prescale:
-            // P'' = p * v_scale * 2^kv with kv chosen so that the largest
-            // v_scale * 2^kv seen by this warp lies in [2^14, 2^15); when kv
-            // drops, the accumulated O is rescaled by the same power of two.
-            const int R0 = 16 * warp + sig_a, R1 = 16 * warp + sig_b;
-            const int R2 = R0 + 8, R3 = R1 + 8;
-            const int rr[2][2] = {{R0, R1}, {R2, R3}};
-            float vsc[2][2][NGV];
+            // ---- V scales of the thread's two tokens and the running prescale 2^kv
+            float vsa[NGV], vsb[NGV];
             float vmax = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-#pragma unroll
-                    for (int gv = 0; gv < NGV; ++gv) {
-                        vsc[nt][c][gv] = ok[nt][c] ? ldsf(svs + (rr[nt][c] * NG + gv) * 4) : 0.f;
-                        vmax = fmaxf(vmax, vsc[nt][c][gv]);
-                    }
-            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 1));
-            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 2));
-            float f_lo = al_lo, f_hi = al_hi;     // factors applied to O
+            for (int gv = 0; gv < NGV; ++gv) {
+                vsa[gv] = okA ? ldsf(svs + (rowA * NG + gv) * 4) : 0.f;
+                vsb[gv] = okB ? ldsf(svs + (rowB * NG + gv) * 4) : 0.f;
+                vmax = fmaxf(vmax, fmaxf(vsa[gv], vsb[gv]));
+            }
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 8));
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 16));
             if (vmax > 0.f) {
                 const int ev = static_cast<int>((__float_as_uint(vmax) >> 23) & 0xffu) - 127;
                 const int kn = min(kv, 14 - ev);
                 if (kn < kv) {
                     const float drop = ldexpf(1.f, kn - kv);
-                    f_lo *= drop;
-                    f_hi *= drop;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        f[nt][0] *= drop;
+                        f[nt][1] *= drop;
+                    }
                     kv = kn;
                 }
             }
             const float up = ldexpf(1.f, kv);
 #pragma unroll
-            for (int n = 0; n < NTD; ++n) {
-                o_lo[n][0] *= f_lo;
-                o_lo[n][1] *= f_lo;
-                if (G16) {
-                    o_hi[n][0] *= f_hi;
-                    o_hi[n][1] *= f_hi;
-                }
-            }
-            // A fragments of P'' split into f16 hi + lo (P'' = hi + lo to ~2^-22)
-            uint32_t ah[NGV][4], al[NGV][4];
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int gv = 0; gv < NGV; ++gv) {
-                split_f16x2(pr_lo[0][0] * vsc[0][0][gv] * up, pr_lo[0][1] * vsc[0][1][gv] * up,
-                            ah[gv][0], al[gv][0]);
-                split_f16x2(pr_lo[1][0] * vsc[1][0][gv] * up, pr_lo[1][1] * vsc[1][1][gv] * up,
-                            ah[gv][2], al[gv][2]);
-                if (G16) {
-                    split_f16x2(pr_hi[0][0] * vsc[0][0][gv] * up, pr_hi[0][1] * vsc[0][1][gv] * up,
-                                ah[gv][1], al[gv][1]);
-                    split_f16x2(pr_hi[1][0] * vsc[1][0][gv] * up, pr_hi[1][1] * vsc[1][1][gv] * up,
-                                ah[gv][3], al[gv][3]);
-                } else {
-                    ah[gv][1] = ah[gv][3] = al[gv][1] = al[gv][3] = 0u;
+                for (int nt = 0; nt < NT; ++nt) {
+                    o[mt][nt][0] *= f[nt][0];
+                    o[mt][nt][1] *= f[nt][1];
+                    o[mt][nt][2] *= f[nt][0];
+                    o[mt][nt][3] *= f[nt][1];
                 }
-            }
-            auto pv = [&](int n, int gv, uint32_t b0, uint32_t b1) {
-                float acc[4] = {o_lo[n][0], o_lo[n][1], o_hi[n][0], o_hi[n][1]};
-                ptx::mma_f16(acc, ah[gv][0], ah[gv][1], ah[gv][2], ah[gv][3], b0, b1);
-                ptx::mma_f16(acc, al[gv][0], al[gv][1], al[gv][2], al[gv][3], b0, b1);
-                o_lo[n][0] = acc[0];
-                o_lo[n][1] = acc[1];
-                o_hi[n][0] = acc[2];
-                o_hi[n][1] = acc[3];
-            };
-            // B fragments from two pairs of V words: rows (R0, R1) give b0,
-            // rows (R2, R3) give b1; byte e of the words is n-tile offset e.
-            auto pv_words = [&](int n0, int gv, uint32_t w0, uint32_t w1, uint32_t w2,
+            // ---- P^T operand: P'' hi / lo, transposed from the score layout
+            // (row = token, column = head) into B fragments (k = token, n = head)
+            uint32_t pbh[NGV][NT][2], pbl[NGV][NT][2];
+#pragma unroll
+            for (int gv = 0; gv < NGV; ++gv)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    uint32_t ha, la, hb, lb;
+                    split_f16x2(pr[nt][0] * vsa[gv] * up, pr[nt][1] * vsa[gv] * up, ha, la);
+                    split_f16x2(pr[nt][2] * vsb[gv] * up, pr[nt][3] * vsb[gv] * up, hb, lb);
+                    pbh[gv][nt][0] = transpose8x8(ha);
+                    pbl[gv][nt][0] = transpose8x8(la);
+                    pbh[gv][nt][1] = transpose8x8(hb);
+                    pbl[gv][nt][1] = transpose8x8(lb);
+                }
+            // ---- O^T += V^T . P^T.  V^T A fragment of m-tile mt: rows g, g+8 are
+            // head_dim d(mt, g), d(mt, g) + 1; columns 2t, 2t+1 / 2t+8, 2t+9 are the
+            // V rows R0, R1 / R2, R3.  Byte pairs of two rows are interleaved with
+            // prmt and turned into exact (v - 128) f16 pairs.
+            auto pv_words = [&](int mt0, int gv, uint32_t w0, uint32_t w1, uint32_t w2,
                                 uint32_t w3) {
                 const uint32_t xl01 = ptx::prmt(w0, w1, 0x5140u);
                 const uint32_t xh01 = ptx::prmt(w0, w1, 0x7362u);
                 const uint32_t xl23 = ptx::prmt(w2, w3, 0x5140u);
                 const uint32_t xh23 = ptx::prmt(w2, w3, 0x7362u);
-                pv(n0 + 0, gv, ptx::bytes_to_f16x2(xl01, 0x4140u), ptx::bytes_to_f16x2(xl23, 0x4140u));
-                pv(n0 + 1, gv, ptx::bytes_to_f16x2(xl01, 0x4342u), ptx::bytes_to_f16x2(xl23, 0x4342u));
-                pv(n0 + 2, gv, ptx::bytes_to_f16x2(xh01, 0x4140u), ptx::bytes_to_f16x2(xh23, 0x4140u));
-                pv(n0 + 3, gv, ptx::bytes_to_f16x2(xh01, 0x4342u), ptx::bytes_to_f16x2(xh23, 0x4342u));
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint32_t x01 = hh ? xh01 : xl01;
+                    const uint32_t x23 = hh ? xh23 : xl23;
+                    const uint32_t a0 = ptx::bytes_to_f16x2(x01, 0x4140u);
+                    const uint32_t a1 = ptx::bytes_to_f16x2(x01, 0x4342u);
+                    const uint32_t a2 = ptx::bytes_to_f16x2(x23, 0x4140u);
+                    const uint32_t a3 = ptx::bytes_to_f16x2(x23, 0x4342u);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        ptx::mma_f16(o[mt0 + hh][nt], a0, a1, a2, a3, pbh[gv][nt][0],
+                                     pbh[gv][nt][1]);
+                        ptx::mma_f16(o[mt0 + hh][nt], a0, a1, a2, a3, pbl[gv][nt][0],
+                                     pbl[gv][nt][1]);
+                    }
+                }
             };
             if (!G32) {
                 if constexpr (D == 128) {
-                    // thread g owns head_dim bytes [16g, 16g + 16): n-tile n, MMA column c
-                    // is head_dim 16c + n
-                    const uint32_t col = 16 * g;
-                    const uint4 v0 = lds128(sv + swz<D>(R0, col));
-                    const uint4 v1 = lds128(sv + swz<D>(R1, col));
-                    const uint4 v2 = lds128(sv + swz<D>(R2, col));
-                    const uint4 v3 = lds128(sv + swz<D>(R3, col));
+                    // thread g owns head_dim [16g, 16g + 16): d(mt, g) = 16g + 2mt
+                    const uint4 v0 = lds128(sv + swz<D>(R0, 16 * g));
+                    const uint4 v1 = lds128(sv + swz<D>(R1, 16 * g));
+                    const uint4 v2 = lds128(sv + swz<D>(R2, 16 * g));
+                    const uint4 v3 = lds128(sv + swz<D>(R3, 16 * g));
                     pv_words(0, 0, v0.x, v1.x, v2.x, v3.x);
-                    pv_words(4, 0, v0.y, v1.y, v2.y, v3.y);
-                    pv_words(8, 0, v0.z, v1.z, v2.z, v3.z);
-                    pv_words(12, 0, v0.w, v1.w, v2.w, v3.w);
+                    pv_words(2, 0, v0.y, v1.y, v2.y, v3.y);
+                    pv_words(4, 0, v0.z, v1.z, v2.z, v3.z);
+                    pv_words(6, 0, v0.w, v1.w, v2.w, v3.w);
                 } else {
-                    // D == 64: thread g owns bytes [8g, 8g + 8): column c is 8c + n
-                    const uint32_t col = 8 * g;
-                    const uint2 v0 = lds64(sv + swz<D>(R0, col));
-                    const uint2 v1 = lds64(sv + swz<D>(R1, col));
-                    const uint2 v2 = lds64(sv + swz<D>(R2, col));
-                    const uint2 v3 = lds64(sv + swz<D>(R3, col));
+                    // D == 64: thread g owns head_dim [8g, 8g + 8): d(mt, g) = 8g + 2mt
+                    const uint2 v0 = lds64(sv + swz<D>(R0, 8 * g));
+                    const uint2 v1 = lds64(sv + swz<D>(R1, 8 * g));
+                    const uint2 v2 = lds64(sv + swz<D>(R2, 8 * g));
+                    const uint2 v3 = lds64(sv + swz<D>(R3, 8 * g));
                     pv_words(0, 0, v0.x, v1.x, v2.x, v3.x);
-                    pv_words(4, 0, v0.y, v1.y, v2.y, v3.y);
+                    pv_words(2, 0, v0.y, v1.y, v2.y, v3.y);
                 }
             } else {
-                // group-32: n-tile 4*gv + e covers head_dim 32*gv + 4*c + e (c = MMA
-                // column), so thread g reads 4 bytes at 32*gv + 4*g of each row
+                // group-32: m-tiles 2*gv, 2*gv + 1 stay inside group gv:
+                // d(2gv + hh, g) = 32*gv + 4*g + 2*hh
 #pragma unroll
                 for (int gv = 0; gv < NGRP; ++gv) {
                     const uint32_t cb = 32 * gv + 4 * g;
-                    pv_words(4 * gv, gv, lds32(sv + swz<D>(R0, cb)), lds32(sv + swz<D>(R1, cb)),
+                    pv_words(2 * gv, gv, lds32(sv + swz<D>(R0, cb)), lds32(sv + swz<D>(R1, cb)),
                              lds32(sv + swz<D>(R2, cb)), lds32(sv + swz<D>(R3, cb)));
                 }
             }
@@ -578,7 +575,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar_empty + 8 * s);
         if (warp == 0 && i + NST < ntiles) {
-            // refill slot s once all four warps have released it
+            // refill slot s once all eight warps have released it
             if (!ptx::mbar_wait(bar_empty + 8 * s, (i / NST) & 1)) {
                 if (lane == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
                 break;
@@ -588,42 +585,51 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
     if (warp == 0) asm volatile("cp.async.wait_all;" ::: "memory");
 
-    // ---- merge the four warps' (m, l, o) into the CTA partial
+    // ---- per-warp totals: undo the P'' prescale, sum l over the 8 row groups
     {
-        const float down = ldexpf(1.f, -kv);         // undo the P'' prescale
+        const float down = ldexpf(1.f, -kv);
 #pragma unroll
-        for (int n = 0; n < NTD; ++n) {
-            o_lo[n][0] *= down;
-            o_lo[n][1] *= down;
-            o_hi[n][0] *= down;
-            o_hi[n][1] *= down;
-        }
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[mt][nt][e] *= down;
     }
-    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
-    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
-    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
-    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 4);
+            l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 8);
+            l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 16);
+        }
     __syncthreads();                              // every stage consumed: reuse shared memory
     float* red = reinterpret_cast<float*>(smem);  // [NW][16][RS]
     float* red_m = red + Lay::RED_M;
     float* red_l = red + Lay::RED_L;
-    // head_dim index of output n-tile n, column c (0/1) of this thread
-    auto dcol = [&](int n, int c) -> int {
-        if (G32) return 32 * (n >> 2) + 4 * (2 * t + c) + (n & 3);
-        return (D == 128 ? 16 : 8) * (2 * t + c) + n;
+    // head_dim of O^T m-tile mt, row g (e = 0) or g + 8 (e = 1) of this thread
+    auto drow = [&](int mt, int e) -> int {
+        if (G32) return 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + e;
+        return (D == 128 ? 16 : 8) * g + 2 * mt + e;
     };
 #pragma unroll
-    for (int n = 0; n < NTD; ++n)
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            red[(warp * 16 + g) * Lay::RS + dcol(n, c)] = o_lo[n][c];
-            if (G16) red[(warp * 16 + g + 8) * Lay::RS + dcol(n, c)] = o_hi[n][c];
+        for (int nt = 0; nt < NT; ++nt) {
+            const int h0 = 8 * nt + 2 * t;
+            red[(warp * 16 + h0) * Lay::RS + drow(mt, 0)] = o[mt][nt][0];
+            red[(warp * 16 + h0 + 1) * Lay::RS + drow(mt, 0)] = o[mt][nt][1];
+            red[(warp * 16 + h0) * Lay::RS + drow(mt, 1)] = o[mt][nt][2];
+            red[(warp * 16 + h0 + 1) * Lay::RS + drow(mt, 1)] = o[mt][nt][3];
         }
-    if (t == 0) {
-        red_m[warp * 16 + g] = m_lo;
-        red_l[warp * 16 + g] = l_lo;
-        red_m[warp * 16 + g + 8] = G16 ? m_hi : -INFINITY;
-        red_l[warp * 16 + g + 8] = G16 ? l_hi : 0.f;
+    if (g == 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                red_m[warp * 16 + 8 * nt + 2 * t + c] = m[nt][c];
+                red_l[warp * 16 + 8 * nt + 2 * t + c] = l[nt][c];
+            }
     }
     __syncthreads();
     float* cp = red + Lay::CP;                    // [16][CPS]: o (unnormalised), m, l
@@ -636,9 +642,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
             const float mw = red_m[w * 16 + h];
-            const float f = (mw == -INFINITY) ? 0.f : ptx::ex2(mw - M);
-            acc = fmaf(f, red[(w * 16 + h) * Lay::RS + d], acc);
-            lsum = fmaf(f, red_l[w * 16 + h], lsum);
+            const float fw = (mw == -INFINITY) ? 0.f : ptx::ex2(mw - M);
+            acc = fmaf(fw, red[(w * 16 + h) * Lay::RS + d], acc);
+            lsum = fmaf(fw, red_l[w * 16 + h], lsum);
         }
         cp[h * Lay::CPS + d] = acc;
         if (d == 0) {
@@ -650,10 +656,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
     if (S > 1) {
-        // ---- cluster combine: partial j lives in CTA j's shared memory
+        // ---- cluster combine: partial r lives in CTA r's shared memory
+        cluster_sync_all();                       // every partial of the cluster is written
         const uint32_t cp_addr = ptx::smem_u32(cp);
-        if (tid < S) arrive_remote(mapa(bar_done, tid));
-        if (!wait_cluster(bar_done, 0) && tid == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
         float* cw = red + Lay::CW;                // [S][16] peer max, then weights
         float* cl = red + Lay::CL;                // [S][16] peer sums
         float* csum = red + Lay::CSUM;            // [16]
@@ -677,7 +682,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             csum[tid] = lsum;
         }
         __syncthreads();
-        // this CTA writes outputs j*128 + tid, stepping by S*128
+        // this CTA writes outputs j*256 + tid, stepping by S*256
         for (int idx = j * NTHREADS + tid; idx < G * D; idx += S * NTHREADS) {
             const int h = idx / D, d = idx - h * D;
             const uint32_t a = cp_addr + (h * Lay::CPS + d) * 4;
@@ -686,10 +691,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const float lsum = csum[h];
             p.out[(bh0 + h) * D + d] = lsum > 0.f ? acc / lsum : 0.f;
         }
-        __syncthreads();
-        // keep this CTA's shared memory alive until every peer has read it
-        if (tid < S) arrive_remote(mapa(bar_read, tid));
-        if (!wait_cluster(bar_read, 0) && tid == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
+        cluster_sync_all();                       // peers are done reading this CTA's partial
     } else if (nsplit <= 1) {
         // single split (or empty sequence): the final row
         if (j == 0)
