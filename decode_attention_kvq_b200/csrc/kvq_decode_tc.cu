@@ -16,11 +16,13 @@
 //    partial softmax states through distributed shared memory (no global
 //    workspace, no second kernel).  Larger S (only on request) writes the
 //    partials to a workspace for the combine kernel in kvq_decode.cu.
-//  * CTA = 8 warps.  Warp 0 streams 128-token stages of K and V bytes into
-//    shared memory with TMA tile loads (2-D tensor maps over the cache rows,
-//    128-byte swizzle for D=128, 64-byte for D=64) and the fp32 scales with
-//    cp.async; both complete on the stage's mbarrier; 3 stages in flight.
-//    Every warp takes one 16-token slice of each stage.
+//  * CTA = 8 warps, one CTA per SM.  Warp 0 streams 128-token stages of K
+//    and V bytes into shared memory with TMA tile loads (2-D tensor maps over
+//    the cache rows, 128-byte swizzle for D=128, 64-byte for D=64) and the
+//    fp32 scales with cp.async; both complete on the stage's mbarrier; 5-6
+//    stages (~200 KB) are in flight per SM.  The first stage is issued before
+//    the sequence length is read.  Every warp takes one 16-token slice of
+//    each stage.
 //  * Per slice, on mma.sync m16n8k16 (f16 in, f32 accumulate), with the
 //    query heads of the GQA group as the N = 8 dimension (two n-tiles when
 //    G > 8):  S^T = K . Q^T (M = 16 tokens, K = head_dim) and
@@ -41,6 +43,10 @@
 //  * Token order inside each 16-token slice and the head_dim order of the
 //    MMA k-dimension are permuted so that every shared-memory load of the
 //    swizzled tiles is free of bank conflicts (sigma below).
+//  * Cluster combine: each CTA owns a slice of the outputs; every CTA stores
+//    its partial values of each slice into the owner's receive buffer
+//    (st.shared::cluster), one cluster barrier publishes them, and owners
+//    combine locally, so no CTA reads a peer's memory after the barrier.
 //  * mbarrier waits are bounded (KVQ_DEVERR_TIMEOUT when one gives up); the
 //    only unbounded waits are the CTA and cluster barriers, which every
 //    thread of every CTA reaches unconditionally.
@@ -56,7 +62,6 @@ namespace {
 constexpr int NW = 8;                  // warps per CTA
 constexpr int NTHREADS = NW * 32;
 constexpr int TT = 16 * NW;            // tokens per stage: one 16-token slice per warp
-constexpr int NST = 3;                 // stages in flight
 constexpr int kMaxCluster = 16;        // largest cluster the combine supports
 
 // Row (inside an 8-token half of a slice) that holds MMA row r of the K
@@ -95,26 +100,35 @@ __device__ __forceinline__ void copy_scales(uint32_t dst, const float* src) {
     else ptx::cp_async_16(dst, src);
 }
 
+// Shared-memory plan: NST stages (one CTA per SM, as many stages as fit so
+// that enough bytes are in flight per SM), the stage mbarriers, and a
+// receive buffer for the cluster combine that nothing else touches.
 template <int D, bool G32>
 struct Layout {
     static constexpr int NG = G32 ? D / 32 : 1;
     static constexpr int KV_BYTES = TT * D;
     static constexpr int SC_FLOATS = TT * NG;
     static constexpr int STAGE = ((2 * KV_BYTES + 2 * SC_FLOATS * 4) + 1023) / 1024 * 1024;
+    static constexpr int NST = (D == 128 && G32) ? 5 : 6;  // stages in flight
     static constexpr int BAR_OFF = NST * STAGE;
     static constexpr int NBAR = 2 * NST;                   // full[], empty[]
-    static constexpr int SMEM = BAR_OFF + NBAR * 8 + 1024;  // + base alignment slack
+    static constexpr int RECV_OFF = BAR_OFF + 128;
+    // per owner and source CTA: its owned outputs (<= ceil(16*D/2)) plus m, l of 16 heads,
+    // over at most 16 sources: <= 16*D + 15 + 2*16*16 floats
+    static constexpr int RECV_FLOATS = 16 * D + 16 + 2 * 16 * 16;
+    static constexpr int SMEM = RECV_OFF + RECV_FLOATS * 4 + 1024;  // + base alignment slack
     // epilogue buffers, in floats, reusing the stage area once every stage is consumed
     static constexpr int RS = D + 4;                       // warp-merge row stride
     static constexpr int RED_M = NW * 16 * RS;             // [NW][16] running max
     static constexpr int RED_L = RED_M + NW * 16;          // [NW][16] running sum
+    static constexpr int WT = RED_L + NW * 16;             // [NW][16] warp weights
     static constexpr int CPS = D + 2;                      // CTA partial row: o[D], m, l
-    static constexpr int CP = RED_L + NW * 16;             // [16][CPS]
-    static constexpr int CW = CP + 16 * CPS;               // [kMaxCluster][16] peer max / weights
-    static constexpr int CL = CW + kMaxCluster * 16;       // [kMaxCluster][16] peer sums
-    static constexpr int CSUM = CL + kMaxCluster * 16;     // [16] combined sums
+    static constexpr int CP = WT + NW * 16;                // [16][CPS]
+    static constexpr int CW = CP + 16 * CPS;               // [kMaxCluster][16] peer weights
+    static constexpr int CSUM = CW + kMaxCluster * 16;     // [16] combined sums
     static constexpr int EPI_FLOATS = CSUM + 16;
     static_assert(EPI_FLOATS * 4 <= BAR_OFF, "epilogue buffers fit in the stage area");
+    static_assert(SMEM <= 227 * 1024, "fits one SM");
 };
 
 // byte offset of (row, byte) inside a swizzled K or V stage tile
@@ -154,10 +168,8 @@ __device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
 }
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 // Cluster-wide barrier: stores before it (release) are visible to every CTA
 // of the cluster after it (acquire).
@@ -167,7 +179,7 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 
 template <int D, bool G32, bool PAGED, bool G16>
-__global__ void __launch_bounds__(NTHREADS, G16 ? 1 : 2)
+__global__ void __launch_bounds__(NTHREADS, 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 DecodeParams p) {
     using Lay = Layout<D, G32>;
@@ -176,7 +188,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     constexpr int NGRP = D / 32;        // 32-value groups over head_dim
     constexpr int MT = D / 16;          // m-tiles of O^T over head_dim (PV)
     constexpr int NT = G16 ? 2 : 1;     // n-tiles of 8 query heads
-    constexpr int NACC = G32 ? NG : 1;  // score accumulators per n-tile
+    constexpr int NACC = G32 ? NG : 2;  // score accumulators per n-tile (two chains per token)
+    constexpr int NST = Lay::NST;
     constexpr int NGV = G32 ? NG : 1;   // V scales per token
 
     extern __shared__ uint8_t smem_raw[];
@@ -192,17 +205,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
     const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
-    int L = p.seq_lens[b];
-    if (L < 0 || L > lim) {
-        if (j == 0 && hk == 0 && tid == 0) raise_flag(p.d_err, KVQ_DEVERR_LEN);
-        L = 0;
-    }
-    // No CTA leaves early: in a cluster every CTA takes part in the combine.
     const int t0 = j * p.chunk;
-    const bool active = t0 < L;
-    const int t1 = active ? min(t0 + p.chunk, L) : t0;
-    const int nsplit = (L + p.chunk - 1) / p.chunk;
-    const int ntiles = active ? (t1 - t0 + TT - 1) / TT : 0;
+    // the first stage is issued before the sequence length is known: tokens
+    // [t0, spec_end) are inside the cache's capacity, so every load is in bounds
+    const int spec_end = static_cast<int>(min(static_cast<int64_t>(t0) + TT, lim));
+    const bool spec = t0 < spec_end;
 
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t bar_full = sbase + Lay::BAR_OFF;
@@ -216,13 +223,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
     __syncthreads();
 
-    // ---- warp 0 issues stage i: TMA for K/V bytes, cp.async for the scales
+    // ---- warp 0 issues stage i (tokens up to t_end): TMA for K/V bytes,
+    // cp.async for the scales
     const uint64_t pol = ptx::policy_evict_first();
-    auto issue = [&](int i) {
+    auto issue = [&](int i, int t_end) {
         const int s = i % NST;
         const uint32_t full = bar_full + 8 * s;
         const int tt0 = t0 + i * TT;
-        const int ntok = min(TT, t1 - tt0);
+        const int ntok = min(TT, t_end - tt0);
         const uint32_t sk = sbase + s * Lay::STAGE;
         const uint32_t sv = sk + Lay::KV_BYTES;
         const uint32_t sks = sv + Lay::KV_BYTES;
@@ -244,11 +252,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int np = (ntok + 15) >> 4;
             int32_t pg = -1;
             if (lane < np) {
+                // a bad entry is skipped here and reported by the consumers,
+                // which know the sequence's true length
                 pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tt0 >> 4) + lane];
-                if (pg < 0 || pg >= p.num_pages) {
-                    raise_flag(p.d_err, KVQ_DEVERR_PAGE);
-                    pg = -1;
-                }
+                if (pg < 0 || pg >= p.num_pages) pg = -1;
             }
             const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
             if (lane == 0) ptx::mbar_arrive_expect_tx(full, __popc(valid) * 2 * 16 * D);
@@ -272,13 +279,20 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         ptx::cp_async_arrive_noinc(full);
     };
-    if (warp == 0) {
-        if (lane == 0 && ntiles > 0) {
-            ptx::prefetch_tensormap(&tm_k);
-            ptx::prefetch_tensormap(&tm_v);
-        }
-        for (int i = 0; i < min(NST, ntiles); ++i) issue(i);
+    if (warp == 0 && spec) issue(0, spec_end);
+
+    int L = p.seq_lens[b];
+    if (L < 0 || L > lim) {
+        if (j == 0 && hk == 0 && tid == 0) raise_flag(p.d_err, KVQ_DEVERR_LEN);
+        L = 0;
     }
+    // No CTA leaves early: in a cluster every CTA takes part in the combine.
+    const bool active = t0 < L;
+    const int t1 = active ? min(t0 + p.chunk, L) : t0;
+    const int nsplit = (L + p.chunk - 1) / p.chunk;
+    const int ntiles = active ? (t1 - t0 + TT - 1) / TT : 0;
+    if (warp == 0)
+        for (int i = spec ? 1 : 0; i < min(NST, ntiles); ++i) issue(i, t1);
 
     // ---- Q^T operand: column n = g of n-tile nt is query head 8*nt + g,
     // pre-scaled by 2^sh so that max |q| * 2^sh lies in [2^14, 2^15).
@@ -382,6 +396,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (PAGED) {
                 const int32_t pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tok0 >> 4)];
                 page_ok = pg >= 0 && pg < p.num_pages;
+                if (!page_ok && lane == 0) raise_flag(p.d_err, KVQ_DEVERR_PAGE);
             }
             const bool okA = page_ok && (tok0 + sig_g < t1);
             const bool okB = page_ok && (tok0 + 8 + sig_g < t1);
@@ -407,8 +422,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const uint32_t a3 = ptx::bytes_to_f16x2(xb, 0x4342u);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
-                        ptx::mma_f16(sacc[nt][G32 ? gi : 0], a0, a1, a2, a3, qb0[nt][2 * gi + h2],
-                                     qb1[nt][2 * gi + h2]);
+                        ptx::mma_f16(sacc[nt][G32 ? gi : (gi & 1)], a0, a1, a2, a3,
+                                     qb0[nt][2 * gi + h2], qb1[nt][2 * gi + h2]);
                 }
             }
             // ---- scores z (log2 domain): [nt][0..1] token rowA, [nt][2..3] token rowB
@@ -439,10 +454,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const float ksa = ldsf(sks + rowA * 4), ksb = ldsf(sks + rowB * 4);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    z[nt][0] = okA ? sacc[nt][0][0] * ksa * zs[nt][0] : -INFINITY;
-                    z[nt][1] = okA ? sacc[nt][0][1] * ksa * zs[nt][1] : -INFINITY;
-                    z[nt][2] = okB ? sacc[nt][0][2] * ksb * zs[nt][0] : -INFINITY;
-                    z[nt][3] = okB ? sacc[nt][0][3] * ksb * zs[nt][1] : -INFINITY;
+                    const float s0 = sacc[nt][0][0] + sacc[nt][1][0];
+                    const float s1 = sacc[nt][0][1] + sacc[nt][1][1];
+                    const float s2 = sacc[nt][0][2] + sacc[nt][1][2];
+                    const float s3 = sacc[nt][0][3] + sacc[nt][1][3];
+                    z[nt][0] = okA ? s0 * ksa * zs[nt][0] : -INFINITY;
+                    z[nt][1] = okA ? s1 * ksa * zs[nt][1] : -INFINITY;
+                    z[nt][2] = okB ? s2 * ksb * zs[nt][0] : -INFINITY;
+                    z[nt][3] = okB ? s3 * ksb * zs[nt][1] : -INFINITY;
                 }
             }
             // ---- online softmax per head: max over the slice's 16 tokens
@@ -490,15 +509,20 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
             }
             const float up = ldexpf(1.f, kv);
+            bool unit = true;
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
+            for (int nt = 0; nt < NT; ++nt) unit = unit && f[nt][0] == 1.f && f[nt][1] == 1.f;
+            if (!__all_sync(0xffffffffu, unit)) {       // the running max moved: rescale O
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    o[mt][nt][0] *= f[nt][0];
-                    o[mt][nt][1] *= f[nt][1];
-                    o[mt][nt][2] *= f[nt][0];
-                    o[mt][nt][3] *= f[nt][1];
-                }
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        o[mt][nt][0] *= f[nt][0];
+                        o[mt][nt][1] *= f[nt][1];
+                        o[mt][nt][2] *= f[nt][0];
+                        o[mt][nt][3] *= f[nt][1];
+                    }
+            }
             // ---- P^T operand: P'' hi / lo, transposed from the score layout
             // (row = token, column = head) into B fragments (k = token, n = head)
             uint32_t pbh[NGV][NT][2], pbl[NGV][NT][2];
@@ -580,10 +604,15 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 if (lane == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
                 break;
             }
-            issue(i + NST);
+            issue(i + NST, t1);
         }
     }
-    if (warp == 0) asm volatile("cp.async.wait_all;" ::: "memory");
+    if (warp == 0) {
+        // a speculative first stage of an inactive CTA still lands in shared memory
+        if (spec && ntiles == 0 && !ptx::mbar_wait(bar_full, 0) && lane == 0)
+            raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    }
 
     // ---- per-warp totals: undo the P'' prescale, sum l over the 8 row groups
     {
@@ -633,65 +662,79 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
     __syncthreads();
     float* cp = red + Lay::CP;                    // [16][CPS]: o (unnormalised), m, l
-    for (int idx = tid; idx < G * D; idx += NTHREADS) {
-        const int h = idx / D, d = idx - h * D;
+    float* wt = red + Lay::WT;                    // [NW][16] weight of each warp's state
+    if (tid < G) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * 16 + h]);
-        float acc = 0.f, lsum = 0.f;
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * 16 + tid]);
+        float lsum = 0.f;
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
-            const float mw = red_m[w * 16 + h];
+            const float mw = red_m[w * 16 + tid];
             const float fw = (mw == -INFINITY) ? 0.f : ptx::ex2(mw - M);
-            acc = fmaf(fw, red[(w * 16 + h) * Lay::RS + d], acc);
-            lsum = fmaf(fw, red_l[w * 16 + h], lsum);
+            wt[w * 16 + tid] = fw;
+            lsum = fmaf(fw, red_l[w * 16 + tid], lsum);
         }
+        cp[tid * Lay::CPS + D] = M;
+        cp[tid * Lay::CPS + D + 1] = lsum;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < G * D; idx += NTHREADS) {
+        const int h = idx / D, d = idx - h * D;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) acc = fmaf(wt[w * 16 + h], red[(w * 16 + h) * Lay::RS + d], acc);
         cp[h * Lay::CPS + d] = acc;
-        if (d == 0) {
-            cp[h * Lay::CPS + D] = M;
-            cp[h * Lay::CPS + D + 1] = lsum;
-        }
     }
     __syncthreads();
 
     const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
     if (S > 1) {
-        // ---- cluster combine: partial r lives in CTA r's shared memory
-        cluster_sync_all();                       // every partial of the cluster is written
-        const uint32_t cp_addr = ptx::smem_u32(cp);
-        float* cw = red + Lay::CW;                // [S][16] peer max, then weights
-        float* cl = red + Lay::CL;                // [S][16] peer sums
-        float* csum = red + Lay::CSUM;            // [16]
+        // ---- cluster combine.  CTA r owns outputs [r*OPC, (r+1)*OPC) of the
+        // flattened (head, head_dim) row; every CTA stores its partial values of
+        // those outputs and its (m, l) of every head into row j of the owner's
+        // receive buffer, one cluster barrier publishes all of them, and each
+        // owner combines its outputs from local shared memory.
+        const int GD = G * D;
+        const int OPC = (GD + S - 1) / S;
+        const int RW = OPC + 2 * G;
+        const uint32_t recv = sbase + Lay::RECV_OFF;
+        for (int idx = tid; idx < GD; idx += NTHREADS) {
+            const int r = idx / OPC, off = idx - r * OPC;
+            const int h = idx / D, d = idx - h * D;
+            st_cluster_f32(mapa(recv + (j * RW + off) * 4, r), cp[h * Lay::CPS + d]);
+        }
         for (int idx = tid; idx < S * G; idx += NTHREADS) {
             const int r = idx / G, h = idx - r * G;
-            const uint32_t a = mapa(cp_addr + (h * Lay::CPS + D) * 4, r);
-            cw[r * 16 + h] = ld_cluster_f32(a);
-            cl[r * 16 + h] = ld_cluster_f32(a + 4);
+            st_cluster_f32(mapa(recv + (j * RW + OPC + h) * 4, r), cp[h * Lay::CPS + D]);
+            st_cluster_f32(mapa(recv + (j * RW + OPC + G + h) * 4, r), cp[h * Lay::CPS + D + 1]);
         }
-        __syncthreads();
+        cluster_sync_all();                       // every CTA's pushes are visible
+        const float* rv = reinterpret_cast<const float*>(smem + Lay::RECV_OFF);
+        float* cw = red + Lay::CW;                // [S][16] weights
+        float* csum = red + Lay::CSUM;            // [16]
         if (tid < G) {
             float M = -INFINITY;
-            for (int r = 0; r < S; ++r) M = fmaxf(M, cw[r * 16 + tid]);
+            for (int r = 0; r < S; ++r) M = fmaxf(M, rv[r * RW + OPC + tid]);
             float lsum = 0.f;
             for (int r = 0; r < S; ++r) {
-                const float mr = cw[r * 16 + tid];
+                const float mr = rv[r * RW + OPC + tid];
                 const float w = (mr == -INFINITY) ? 0.f : ptx::ex2(mr - M);
                 cw[r * 16 + tid] = w;
-                lsum = fmaf(w, cl[r * 16 + tid], lsum);
+                lsum = fmaf(w, rv[r * RW + OPC + G + tid], lsum);
             }
             csum[tid] = lsum;
         }
         __syncthreads();
-        // this CTA writes outputs j*256 + tid, stepping by S*256
-        for (int idx = j * NTHREADS + tid; idx < G * D; idx += S * NTHREADS) {
+        for (int off = tid; off < OPC; off += NTHREADS) {
+            const int idx = j * OPC + off;
+            if (idx >= GD) break;
             const int h = idx / D, d = idx - h * D;
-            const uint32_t a = cp_addr + (h * Lay::CPS + d) * 4;
             float acc = 0.f;
-            for (int r = 0; r < S; ++r) acc = fmaf(cw[r * 16 + h], ld_cluster_f32(mapa(a, r)), acc);
+            for (int r = 0; r < S; ++r) acc = fmaf(cw[r * 16 + h], rv[r * RW + off], acc);
             const float lsum = csum[h];
             p.out[(bh0 + h) * D + d] = lsum > 0.f ? acc / lsum : 0.f;
         }
-        cluster_sync_all();                       // peers are done reading this CTA's partial
     } else if (nsplit <= 1) {
         // single split (or empty sequence): the final row
         if (j == 0)
