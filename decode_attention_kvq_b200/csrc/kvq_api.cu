@@ -30,8 +30,6 @@ kvq_status check_append_common(const uint16_t* k_new, const uint16_t* v_new, int
     return KVQ_OK;
 }
 
-constexpr int kClusterSplits = 16;   // splits combined inside one thread-block cluster
-
 kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk_out,
                 int* splits_out) {
     if (B < 0 || Hk < 1 || hint < 0 || num_splits < 0) return KVQ_ERR_INVALID_ARG;
@@ -48,12 +46,19 @@ kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk
         const int64_t s = num_splits < ceil_div(hint, 16) ? num_splits : ceil_div(hint, 16);
         chunk = ceil_div(ceil_div(hint, s), 16) * 16;
     } else {
-        // about two CTAs per SM over all (sequence, kv head) units, at most
-        // one cluster of splits per unit
+        // Small problems: about one chunk per SM over all (sequence, kv head)
+        // units.  Large ones: chunks of at least 512 tokens, about 16 per SM,
+        // so that the persistent CTAs share the work evenly.
         const int64_t units = static_cast<int64_t>(B > 0 ? B : 1) * Hk;
-        int64_t want = ceil_div(2ll * num_sms, units);
-        if (want > kClusterSplits) want = kClusterSplits;
-        chunk = ceil_div(ceil_div(hint, want), 16) * 16;
+        int64_t per_unit = num_sms / units;
+        if (per_unit < 1) per_unit = 1;
+        chunk = ceil_div(ceil_div(hint, per_unit), 16) * 16;
+        if (chunk > 1024) {
+            chunk = ceil_div(ceil_div(static_cast<int64_t>(hint) * units, 16ll * num_sms), 16) * 16;
+            if (chunk < 512) chunk = 512;
+        }
+        const int64_t cap = ceil_div(hint, 16) * 16;
+        if (chunk > cap) chunk = cap;
     }
     if (ceil_div(hint, chunk) > kMaxSplits) chunk = ceil_div(ceil_div(hint, kMaxSplits), 16) * 16;
     int64_t splits = ceil_div(hint, chunk);
@@ -63,14 +68,8 @@ kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk
     return KVQ_OK;
 }
 
-// splits combined in a cluster (no workspace), or 1 when the combine kernel is used
-int cluster_for(int splits) {
-    if (splits <= 1) return 1;
-    return splits <= kvq::decode_max_cluster() ? splits : 1;
-}
-
 size_t workspace_for(int B, int Hq, int D, int splits) {
-    if (splits <= 1 || cluster_for(splits) > 1) return 0;
+    if (splits <= 1) return 0;
     return static_cast<size_t>(B) * Hq * splits * (D + 2) * sizeof(float);
 }
 
@@ -179,7 +178,14 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
     p.B = B; p.Hq = Hq; p.Hk = Hk; p.G = G; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
     p.page_size = kv->page_size; p.max_seq = kv->max_seq; p.max_pages = kv->max_pages;
     p.num_pages = kv->num_pages; p.chunk = chunk; p.splits = splits;
-    p.cluster = cluster_for(splits);
+    {
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        const int64_t items = static_cast<int64_t>(B) * Hk * splits;
+        p.grid = static_cast<int>(items < sms ? items : sms);   // persistent: one CTA per SM
+    }
     p.scale_log2 = attn_scale * 1.4426950408889634f;
     return from_cuda(kvq::launch_decode(p, static_cast<cudaStream_t>(stream)));
 }

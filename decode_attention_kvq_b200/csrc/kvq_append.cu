@@ -14,7 +14,8 @@
 // 8 bf16 (16 bytes) and storing 8 bytes; the absolute maximum is reduced
 // with xor shuffles inside the row (per token) or inside each 4-lane
 // quarter that covers 32 values (group-32).  The kernel is HBM-bound: per
-// row it reads 2*D bytes and writes D + 4*NG bytes.
+// row it reads 2*D bytes and writes D + 4*NG bytes.  It is launched as a
+// programmatic dependent (waits for the preceding grid before reading).
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -24,6 +25,8 @@ constexpr int kAppendThreads = 256;
 
 __global__ void __launch_bounds__(kAppendThreads)
 append_kernel(AppendParams p, int lanes_log2) {
+    grid_dep_wait();                             // inputs written by the preceding grid
+    grid_dep_launch();
     const int P = 1 << lanes_log2;               // lanes per row
     const int lane = threadIdx.x & 31;
     const int sub = lane & (P - 1);              // lane index inside the row
@@ -117,8 +120,16 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
     const int rows_per_block = (kAppendThreads / 32) * (32 >> lanes_log2);
     const int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
     if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
-    append_kernel<<<static_cast<unsigned>(blocks), kAppendThreads, 0, s>>>(p, lanes_log2);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    cfg.blockDim = dim3(kAppendThreads, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, append_kernel, p, lanes_log2);
 }
 
 }  // namespace kvq

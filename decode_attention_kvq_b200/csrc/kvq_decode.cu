@@ -1,7 +1,7 @@
-// kvq_decode.cu -- decode attention driver: the split kernel
-// (kvq_decode_tc.cu), which combines up to 16 splits inside a thread-block
-// cluster, followed -- only when more splits than one cluster holds were
-// requested -- by the combine kernel below.
+// kvq_decode.cu -- decode attention driver: the persistent split kernel
+// (kvq_decode_tc.cu) followed, when some sequence spans more than one chunk,
+// by the combine kernel below (launched as a programmatic dependent so its
+// launch overlaps the split kernel).
 //
 // Combine (flash-decoding): for each (sequence, q head) with splits j =
 // 0..ns-1 holding unnormalised (o_j, m_j, l_j) in base 2,
@@ -24,6 +24,7 @@ decode_combine(DecodeParams p) {
     extern __shared__ float s_w[];                 // [splits] weights
     __shared__ float s_red[kWarps];
     __shared__ __align__(16) float s_acc[kWarps][256];
+    grid_dep_wait();                    // the split kernel's partials are complete
     const int64_t bh = blockIdx.x;
     const int b = static_cast<int>(bh / p.Hq);
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -81,10 +82,18 @@ decode_combine(DecodeParams p) {
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
     cudaError_t e = launch_decode_split_tc(p, s);
-    if (e != cudaSuccess || p.splits <= 1 || p.cluster > 1) return e;
-    const size_t smem = static_cast<size_t>(p.splits) * sizeof(float);
-    decode_combine<<<p.B * p.Hq, kThreads, smem, s>>>(p);
-    return cudaGetLastError();
+    if (e != cudaSuccess || p.splits <= 1) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.B * p.Hq, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(p.splits) * sizeof(float);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_combine, p);
 }
 
 }  // namespace kvq

@@ -1,7 +1,7 @@
 // kvq_decode_tc.cu -- decode attention on the INT8 cache for sm_100a:
-// TMA-staged K/V tiles, tensor-core Q.K^T and P.V on exact integer operands
-// with the dequantisation scales applied outside the MMA, split-K across the
-// CTAs of a thread-block cluster combined through distributed shared memory.
+// a persistent split-K kernel with TMA-staged K/V tiles and tensor-core
+// Q.K^T and P.V on exact integer operands, the dequantisation scales applied
+// outside the MMA.
 //
 // Method (what is computed): abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
 // module doc "Fused approach" -- Q.K^T with K dequantised on the fly,
@@ -11,18 +11,20 @@
 // online softmax and the combine are this library's own (flash-decoding).
 //
 // How (sm_100a):
-//  * Grid (S, Hk, B): S splits of the KV range per (sequence, kv head).  With
-//    2 <= S <= 16 the S CTAs form one thread-block cluster and merge their
-//    partial softmax states through distributed shared memory (no global
-//    workspace, no second kernel).  Larger S (only on request) writes the
-//    partials to a workspace for the combine kernel in kvq_decode.cu.
-//  * CTA = 8 warps, one CTA per SM.  Warp 0 streams 128-token stages of K
-//    and V bytes into shared memory with TMA tile loads (2-D tensor maps over
-//    the cache rows, 128-byte swizzle for D=128, 64-byte for D=64) and the
-//    fp32 scales with cp.async; both complete on the stage's mbarrier; 5-6
-//    stages (~200 KB) are in flight per SM.  The first stage is issued before
-//    the sequence length is read.  Every warp takes one 16-token slice of
-//    each stage.
+//  * Work items are (sequence b, kv head, chunk j) with chunk = p.chunk
+//    tokens.  The grid is persistent (at most one CTA per SM); CTA c takes the
+//    items c, c + gridDim.x, ... of the list ordered (j, b, kv head), so long
+//    and short sequences spread over all SMs.  An item that is a whole
+//    sequence writes the final rows; otherwise it writes its partial softmax
+//    state (o, m, l) for the combine kernel (kvq_decode.cu).
+//  * CTA = 8 warps.  Warp 0 streams 128-token stages into a ring of 4-8
+//    stages (~200 KB of shared memory, so one CTA fills an SM): K and V
+//    bytes by TMA tile loads (2-D tensor maps over the cache rows, 128-byte
+//    swizzle for D=128, 64-byte for D=64), the fp32 scales and, with an
+//    item's first stage, the item's query rows by cp.async; all complete on
+//    the stage's mbarrier.  The ring runs across item boundaries, so the
+//    memory pipe stays busy while the warps merge an item.  Every warp takes
+//    one 16-token slice of each stage.
 //  * Per slice, on mma.sync m16n8k16 (f16 in, f32 accumulate), with the
 //    query heads of the GQA group as the N = 8 dimension (two n-tiles when
 //    G > 8):  S^T = K . Q^T (M = 16 tokens, K = head_dim) and
@@ -43,13 +45,14 @@
 //  * Token order inside each 16-token slice and the head_dim order of the
 //    MMA k-dimension are permuted so that every shared-memory load of the
 //    swizzled tiles is free of bank conflicts (sigma below).
-//  * Cluster combine: each CTA owns a slice of the outputs; every CTA stores
-//    its partial values of each slice into the owner's receive buffer
-//    (st.shared::cluster), one cluster barrier publishes them, and owners
-//    combine locally, so no CTA reads a peer's memory after the barrier.
-//  * mbarrier waits are bounded (KVQ_DEVERR_TIMEOUT when one gives up); the
-//    only unbounded waits are the CTA and cluster barriers, which every
-//    thread of every CTA reaches unconditionally.
+//  * An item's eight warp states are merged by a pairwise tree through a
+//    small dedicated buffer (deterministic: no atomics).
+//  * Programmatic dependent launch: the kernel waits for its predecessor in
+//    the stream before touching memory and lets its successor (the combine
+//    kernel) launch early.
+//  * mbarrier waits are bounded (KVQ_DEVERR_TIMEOUT when one gives up, after
+//    which every wait of the CTA returns at once); CTA barriers are reached
+//    by every thread unconditionally.
 #include <cuda.h>
 #include <math.h>
 
@@ -62,7 +65,6 @@ namespace {
 constexpr int NW = 8;                  // warps per CTA
 constexpr int NTHREADS = NW * 32;
 constexpr int TT = 16 * NW;            // tokens per stage: one 16-token slice per warp
-constexpr int kMaxCluster = 16;        // largest cluster the combine supports
 
 // Row (inside an 8-token half of a slice) that holds MMA row r of the K
 // operand and MMA k-index r of the V operand: sigma = {0, 2, 4, 6, 3, 1, 7, 5}.
@@ -100,34 +102,26 @@ __device__ __forceinline__ void copy_scales(uint32_t dst, const float* src) {
     else ptx::cp_async_16(dst, src);
 }
 
-// Shared-memory plan: NST stages (one CTA per SM, as many stages as fit so
-// that enough bytes are in flight per SM), the stage mbarriers, and a
-// receive buffer for the cluster combine that nothing else touches.
-template <int D, bool G32>
+// Shared-memory plan (one CTA per SM): a ring of NST stages, each holding K
+// and V bytes of 128 tokens, their scales and room for one item's query rows;
+// the merge buffer; the stage mbarriers and the per-warp head maxima.
+template <int D, bool G32, bool G16>
 struct Layout {
     static constexpr int NG = G32 ? D / 32 : 1;
     static constexpr int KV_BYTES = TT * D;
     static constexpr int SC_FLOATS = TT * NG;
-    static constexpr int STAGE = ((2 * KV_BYTES + 2 * SC_FLOATS * 4) + 1023) / 1024 * 1024;
-    static constexpr int NST = (D == 128 && G32) ? 5 : 6;  // stages in flight
-    static constexpr int BAR_OFF = NST * STAGE;
-    static constexpr int NBAR = 2 * NST;                   // full[], empty[]
-    static constexpr int RECV_OFF = BAR_OFF + 128;
-    // per owner and source CTA: its owned outputs (<= ceil(16*D/2)) plus m, l of 16 heads,
-    // over at most 16 sources: <= 16*D + 15 + 2*16*16 floats
-    static constexpr int RECV_FLOATS = 16 * D + 16 + 2 * 16 * 16;
-    static constexpr int SMEM = RECV_OFF + RECV_FLOATS * 4 + 1024;  // + base alignment slack
-    // epilogue buffers, in floats, reusing the stage area once every stage is consumed
-    static constexpr int RS = D + 4;                       // warp-merge row stride
-    static constexpr int RED_M = NW * 16 * RS;             // [NW][16] running max
-    static constexpr int RED_L = RED_M + NW * 16;          // [NW][16] running sum
-    static constexpr int WT = RED_L + NW * 16;             // [NW][16] warp weights
-    static constexpr int CPS = D + 2;                      // CTA partial row: o[D], m, l
-    static constexpr int CP = WT + NW * 16;                // [16][CPS]
-    static constexpr int CW = CP + 16 * CPS;               // [kMaxCluster][16] peer weights
-    static constexpr int CSUM = CW + kMaxCluster * 16;     // [16] combined sums
-    static constexpr int EPI_FLOATS = CSUM + 16;
-    static_assert(EPI_FLOATS * 4 <= BAR_OFF, "epilogue buffers fit in the stage area");
+    static constexpr int Q_OFF = 2 * KV_BYTES + 2 * SC_FLOATS * 4;   // within a stage
+    static constexpr int Q_BYTES = 16 * D * 2;                        // up to 16 bf16 rows
+    static constexpr int STAGE = ((Q_OFF + Q_BYTES) + 1023) / 1024 * 1024;
+    static constexpr int NV = (G16 ? 2 : 1) * (D / 16) * 4 + 4;      // merged floats per thread
+    static constexpr int MERGE_BYTES = 4 * NV * 32 * 4;             // 4 warp slots
+    static constexpr int MISC_BYTES = 1024;                         // barriers, maxima, abort flag
+    static constexpr int BUDGET = 227 * 1024 - 1024 - MERGE_BYTES - MISC_BYTES;
+    static constexpr int NST = (BUDGET / STAGE) > 8 ? 8 : (BUDGET / STAGE);
+    static_assert(NST >= 3, "at least three stages");
+    static constexpr int MERGE_OFF = NST * STAGE;
+    static constexpr int MISC_OFF = MERGE_OFF + MERGE_BYTES;
+    static constexpr int SMEM = MISC_OFF + MISC_BYTES + 1024;       // + base alignment slack
     static_assert(SMEM <= 227 * 1024, "fits one SM");
 };
 
@@ -163,78 +157,120 @@ __device__ __forceinline__ float ldsf(uint32_t a) {
     return v;
 }
 
-__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-// Cluster-wide barrier: stores before it (release) are visible to every CTA
-// of the cluster after it (acquire).
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
-                 ::: "memory");
+// The items of one CTA: dense indices first, first + step, ... of the list
+// (j, b, kv head), skipping chunks past a sequence's end.  A sequence of
+// length 0 yields one item with t0 == t1 (its output rows are zero).
+struct Walk {
+    int64_t dense;
+    int b, hk, j, L, t0, t1;
+};
+
+__device__ __forceinline__ bool walk_next(Walk& w, const DecodeParams& p, int64_t lim,
+                                          int64_t first, int64_t step, int64_t total) {
+    const int64_t per_j = static_cast<int64_t>(p.B) * p.Hk;
+    for (;;) {
+        w.dense = w.dense < 0 ? first : w.dense + step;
+        if (w.dense >= total) return false;
+        w.j = static_cast<int>(w.dense / per_j);
+        const int rem = static_cast<int>(w.dense - static_cast<int64_t>(w.j) * per_j);
+        w.b = rem / p.Hk;
+        w.hk = rem - w.b * p.Hk;
+        int L = p.seq_lens[w.b];
+        if (L < 0 || L > lim) L = 0;
+        w.L = L;
+        const int ns = (L + p.chunk - 1) / p.chunk;
+        if (ns == 0) {
+            if (w.j != 0) continue;
+            w.t0 = w.t1 = 0;
+            return true;
+        }
+        if (w.j >= ns) continue;
+        w.t0 = w.j * p.chunk;
+        w.t1 = min(w.t0 + p.chunk, L);
+        return true;
+    }
 }
 
 template <int D, bool G32, bool PAGED, bool G16>
 __global__ void __launch_bounds__(NTHREADS, 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 DecodeParams p) {
-    using Lay = Layout<D, G32>;
+    using Lay = Layout<D, G32, G16>;
     constexpr int NG = Lay::NG;
+    constexpr int NST = Lay::NST;
     constexpr int KS = D / 16;          // MMA k-steps over head_dim (QK)
     constexpr int NGRP = D / 32;        // 32-value groups over head_dim
     constexpr int MT = D / 16;          // m-tiles of O^T over head_dim (PV)
     constexpr int NT = G16 ? 2 : 1;     // n-tiles of 8 query heads
     constexpr int NACC = G32 ? NG : 2;  // score accumulators per n-tile (two chains per token)
-    constexpr int NST = Lay::NST;
     constexpr int NGV = G32 ? NG : 1;   // V scales per token
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
-    const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tid = threadIdx.x;
     const int g = lane >> 2, t = lane & 3;
     const int G = p.G;
-    const int S = p.cluster;            // CTAs in this kernel's cluster (1: none)
-
-    const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
-    const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
-    const int t0 = j * p.chunk;
-    // the first stage is issued before the sequence length is known: tokens
-    // [t0, spec_end) are inside the cache's capacity, so every load is in bounds
-    const int spec_end = static_cast<int>(min(static_cast<int64_t>(t0) + TT, lim));
-    const bool spec = t0 < spec_end;
 
     const uint32_t sbase = ptx::smem_u32(smem);
-    const uint32_t bar_full = sbase + Lay::BAR_OFF;
+    const uint32_t bar_full = sbase + Lay::MISC_OFF;
     const uint32_t bar_empty = bar_full + NST * 8;
+    float* mrg_m = reinterpret_cast<float*>(smem + Lay::MISC_OFF + 2 * NST * 8);   // [NW][16]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_m + NW * 16);
+    float* mbuf = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);                // [4][NV][32]
+
     if (tid == 0) {
         for (int s = 0; s < NST; ++s) {
             ptx::mbar_init(bar_full + 8 * s, 1 + 32);   // expect_tx arrive + 32 cp.async arrivals
             ptx::mbar_init(bar_empty + 8 * s, NW);
         }
+        *abort_flag = 0;
         ptx::fence_mbar_init();
     }
     __syncthreads();
+    grid_dep_wait();                    // the predecessor's writes (q, cache, lengths) are visible
+    grid_dep_launch();                  // the combine kernel may be scheduled now
 
-    // ---- warp 0 issues stage i (tokens up to t_end): TMA for K/V bytes,
-    // cp.async for the scales
+    const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
+    const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
+    const int64_t total = static_cast<int64_t>(p.splits) * p.B * p.Hk;
+    const int64_t first = blockIdx.x, step = gridDim.x;
+
+    // bounded wait that gives up at once after any earlier timeout of this CTA
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+        if (*abort_flag) return;
+        if (!ptx::mbar_wait(bar, parity)) {
+            *abort_flag = 1;
+            if (lane == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
+        }
+    };
+
+    // ---- producer state (warp 0): next tile to issue
+    Walk pw;
+    pw.dense = -1;
+    bool p_valid = walk_next(pw, p, lim, first, step, total);
+    int p_tile = 0;                     // tile within pw's item
+    int p_count = 0;                    // tiles issued so far (ring position)
     const uint64_t pol = ptx::policy_evict_first();
-    auto issue = [&](int i, int t_end) {
-        const int s = i % NST;
+
+    // issue the next tile of this CTA's item list into the ring (warp 0, all lanes)
+    auto produce = [&]() {
+        while (p_valid && pw.t0 + p_tile * TT >= pw.t1) {
+            p_valid = walk_next(pw, p, lim, first, step, total);
+            p_tile = 0;
+        }
+        if (!p_valid) return;
+        const int s = p_count % NST;
         const uint32_t full = bar_full + 8 * s;
-        const int tt0 = t0 + i * TT;
-        const int ntok = min(TT, t_end - tt0);
+        const int tt0 = pw.t0 + p_tile * TT;
+        const int ntok = min(TT, pw.t1 - tt0);
         const uint32_t sk = sbase + s * Lay::STAGE;
         const uint32_t sv = sk + Lay::KV_BYTES;
         const uint32_t sks = sv + Lay::KV_BYTES;
         const uint32_t svs = sks + Lay::SC_FLOATS * 4;
+        const int b = pw.b, hk = pw.hk;
         if (!PAGED) {
             const int64_t row0 = (static_cast<int64_t>(b) * p.Hk + hk) * p.max_seq + tt0;
             if (lane == 0) {
@@ -252,8 +288,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int np = (ntok + 15) >> 4;
             int32_t pg = -1;
             if (lane < np) {
-                // a bad entry is skipped here and reported by the consumers,
-                // which know the sequence's true length
+                // a bad entry is skipped here and reported by the consumers
                 pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tt0 >> 4) + lane];
                 if (pg < 0 || pg >= p.num_pages) pg = -1;
             }
@@ -277,101 +312,20 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
             }
         }
-        ptx::cp_async_arrive_noinc(full);
-    };
-    if (warp == 0 && spec) issue(0, spec_end);
-
-    int L = p.seq_lens[b];
-    if (L < 0 || L > lim) {
-        if (j == 0 && hk == 0 && tid == 0) raise_flag(p.d_err, KVQ_DEVERR_LEN);
-        L = 0;
-    }
-    // No CTA leaves early: in a cluster every CTA takes part in the combine.
-    const bool active = t0 < L;
-    const int t1 = active ? min(t0 + p.chunk, L) : t0;
-    const int nsplit = (L + p.chunk - 1) / p.chunk;
-    const int ntiles = active ? (t1 - t0 + TT - 1) / TT : 0;
-    if (warp == 0)
-        for (int i = spec ? 1 : 0; i < min(NST, ntiles); ++i) issue(i, t1);
-
-    // ---- Q^T operand: column n = g of n-tile nt is query head 8*nt + g,
-    // pre-scaled by 2^sh so that max |q| * 2^sh lies in [2^14, 2^15).
-    // B fragment rows 2t, 2t+1 (qb0) and 2t+8, 2t+9 (qb1) of k-step 2*gi + h2
-    // hold head_dim 32*gi + 8*t + 4*h2 + {0, 1} and {2, 3}.
-    uint32_t qb0[NT][KS], qb1[NT][KS];
-    float zsq[NT];                      // 2^-sh * attn_scale * log2(e) of head 8*nt + g
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        zsq[nt] = 0.f;
-#pragma unroll
-        for (int k = 0; k < KS; ++k) qb0[nt][k] = qb1[nt][k] = 0u;
-    }
-    if (ntiles > 0) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int h = 8 * nt + g;
-            float qf[NGRP][8];
-            float amax = 0.f;
-            if (h < G) {
-                const uint16_t* qrow = p.q + (static_cast<int64_t>(b) * p.Hq + hk * G + h) * D;
-#pragma unroll
-                for (int gi = 0; gi < NGRP; ++gi) {
-                    const uint4 raw = *reinterpret_cast<const uint4*>(qrow + 32 * gi + 8 * t);
-                    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        qf[gi][2 * e] = bf16_bits_to_f32(w[e] & 0xffffu);
-                        qf[gi][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
-                    }
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(qf[gi][e]));
-                }
-            } else {
-#pragma unroll
-                for (int gi = 0; gi < NGRP; ++gi)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) qf[gi][e] = 0.f;
-            }
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-            int sh = 0;
-            if (amax > 0.f) {
-                const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
-                sh = min(max(14 - e, -100), 100);
-            }
-            const float up = ldexpf(1.f, sh);
-            zsq[nt] = ldexpf(1.f, -sh) * p.scale_log2;
-#pragma unroll
-            for (int gi = 0; gi < NGRP; ++gi)
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    qb0[nt][2 * gi + h2] =
-                        ptx::pack_f16x2(qf[gi][4 * h2] * up, qf[gi][4 * h2 + 1] * up);
-                    qb1[nt][2 * gi + h2] =
-                        ptx::pack_f16x2(qf[gi][4 * h2 + 2] * up, qf[gi][4 * h2 + 3] * up);
-                }
+        if (p_tile == 0) {
+            // the item's G query rows (contiguous bf16) ride with its first stage
+            const uint16_t* qsrc = p.q + (static_cast<int64_t>(b) * p.Hq + hk * G) * D;
+            const uint32_t sq = sk + Lay::Q_OFF;
+            for (int c = lane; c < G * D / 8; c += 32) ptx::cp_async_16(sq + c * 16, qsrc + c * 8);
         }
-    }
-    // score factor of the two heads (columns 2t, 2t+1) this thread accumulates
-    float zs[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        zs[nt][0] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t));
-        zs[nt][1] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t + 1));
-    }
+        ptx::cp_async_arrive_noinc(full);
+        ++p_tile;
+        ++p_count;
+    };
+    if (warp == 0)
+        for (int k = 0; k < NST; ++k) produce();
 
-    // ---- per-warp online softmax state: heads 8*nt + 2t + c
-    float m[NT][2], l[NT][2];
-    float o[MT][NT][4];                 // O^T C fragments: rows = head_dim, columns = heads
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        m[nt][0] = m[nt][1] = -INFINITY;
-        l[nt][0] = l[nt][1] = 0.f;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
-    }
-    int kv = 64;                         // running P'' prescale exponent (per warp)
-
+    // ---- consumers: all eight warps
     const int sig_g = sigma(g);
     const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
     const int rowA = 16 * warp + sig_g;           // MMA row g     of this warp's slice
@@ -379,19 +333,100 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int R0 = 16 * warp + sig_a, R1 = 16 * warp + sig_b;   // V rows of k 2t, 2t+1
     const int R2 = R0 + 8, R3 = R1 + 8;                         // V rows of k 2t+8, 2t+9
 
-    for (int i = 0; i < ntiles; ++i) {
-        const int s = i % NST;
-        if (!ptx::mbar_wait(bar_full + 8 * s, (i / NST) & 1)) {
-            if (lane == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
-            break;
+    Walk cw;
+    cw.dense = -1;
+    int c_count = 0;                    // tiles consumed so far (ring position)
+    while (walk_next(cw, p, lim, first, step, total)) {
+        const int b = cw.b, hk = cw.hk;
+        const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
+        if (cw.t0 == cw.t1) {
+            // empty (or rejected) sequence: zero rows
+            if (hk == 0 && tid == 0) {
+                const int Lraw = p.seq_lens[b];
+                if (Lraw < 0 || Lraw > lim) raise_flag(p.d_err, KVQ_DEVERR_LEN);
+            }
+            for (int idx = tid; idx < G * D; idx += NTHREADS) p.out[bh0 * D + idx] = 0.f;
+            continue;
         }
-        const int tt0 = t0 + i * TT;
-        const uint32_t sk = sbase + s * Lay::STAGE;
-        const uint32_t sv = sk + Lay::KV_BYTES;
-        const uint32_t sks = sv + Lay::KV_BYTES;
-        const uint32_t svs = sks + Lay::SC_FLOATS * 4;
-        const int tok0 = tt0 + 16 * warp;             // first token of this warp's slice
-        if (tok0 < t1) {
+        const int t0 = cw.t0, t1 = cw.t1;
+        const int nsplit = (cw.L + p.chunk - 1) / p.chunk;
+        const int ntiles = (t1 - t0 + TT - 1) / TT;
+
+        uint32_t qb0[NT][KS], qb1[NT][KS];
+        float zs[NT][2];
+        float m[NT][2], l[NT][2];
+        float o[MT][NT][4];             // O^T C fragments: rows = head_dim, columns = heads
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            m[nt][0] = m[nt][1] = -INFINITY;
+            l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+                o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+        }
+        int kv = 64;                    // running P'' prescale exponent (per warp)
+
+        for (int it = 0; it < ntiles; ++it, ++c_count) {
+            const int s = c_count % NST;
+            wait(bar_full + 8 * s, (c_count / NST) & 1);
+            const int tt0 = t0 + it * TT;
+            const uint32_t sk = sbase + s * Lay::STAGE;
+            const uint32_t sv = sk + Lay::KV_BYTES;
+            const uint32_t sks = sv + Lay::KV_BYTES;
+            const uint32_t svs = sks + Lay::SC_FLOATS * 4;
+            if (it == 0) {
+                // ---- Q^T operand from the stage: column n = g of n-tile nt is query
+                // head 8*nt + g, pre-scaled by 2^sh so max |q| * 2^sh is in [2^14, 2^15).
+                // B fragment rows 2t, 2t+1 (qb0) and 2t+8, 2t+9 (qb1) of k-step
+                // 2*gi + h2 hold head_dim 32*gi + 8*t + 4*h2 + {0, 1} and {2, 3}.
+                const uint32_t sq = sk + Lay::Q_OFF;
+                float zsq[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int h = 8 * nt + g;
+                    float qf[NGRP][8];
+                    float amax = 0.f;
+#pragma unroll
+                    for (int gi = 0; gi < NGRP; ++gi) {
+                        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+                        if (h < G) raw = lds128(sq + (h * D + 32 * gi + 8 * t) * 2);
+                        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            qf[gi][2 * e] = bf16_bits_to_f32(w[e] & 0xffffu);
+                            qf[gi][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(qf[gi][e]));
+                    }
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                    int sh = 0;
+                    if (amax > 0.f) {
+                        const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+                        sh = min(max(14 - e, -100), 100);
+                    }
+                    const float up = ldexpf(1.f, sh);
+                    zsq[nt] = ldexpf(1.f, -sh) * p.scale_log2;
+#pragma unroll
+                    for (int gi = 0; gi < NGRP; ++gi)
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            qb0[nt][2 * gi + h2] =
+                                ptx::pack_f16x2(qf[gi][4 * h2] * up, qf[gi][4 * h2 + 1] * up);
+                            qb1[nt][2 * gi + h2] =
+                                ptx::pack_f16x2(qf[gi][4 * h2 + 2] * up, qf[gi][4 * h2 + 3] * up);
+                        }
+                }
+                // score factor of the two heads (columns 2t, 2t+1) this thread accumulates
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    zs[nt][0] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t));
+                    zs[nt][1] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t + 1));
+                }
+            }
+            const int tok0 = tt0 + 16 * warp;             // first token of this warp's slice
+            if (tok0 < t1) {
             bool page_ok = true;
             if (PAGED) {
                 const int32_t pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tok0 >> 4)];
@@ -595,165 +630,128 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                              lds32(sv + swz<D>(R2, cb)), lds32(sv + swz<D>(R3, cb)));
                 }
             }
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar_empty + 8 * s);
-        if (warp == 0 && i + NST < ntiles) {
-            // refill slot s once all eight warps have released it
-            if (!ptx::mbar_wait(bar_empty + 8 * s, (i / NST) & 1)) {
-                if (lane == 0) raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
-                break;
             }
-            issue(i + NST, t1);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_empty + 8 * s);
+            if (warp == 0) {
+                // refill slot s once all eight warps have released it
+                wait(bar_empty + 8 * s, (c_count / NST) & 1);
+                produce();
+            }
         }
-    }
-    if (warp == 0) {
-        // a speculative first stage of an inactive CTA still lands in shared memory
-        if (spec && ntiles == 0 && !ptx::mbar_wait(bar_full, 0) && lane == 0)
-            raise_flag(p.d_err, KVQ_DEVERR_TIMEOUT);
-        asm volatile("cp.async.wait_all;" ::: "memory");
-    }
 
-    // ---- per-warp totals: undo the P'' prescale, sum l over the 8 row groups
-    {
-        const float down = ldexpf(1.f, -kv);
+        // ---- merge the eight warps' states of this item
+        {
+            const float down = ldexpf(1.f, -kv);         // undo the P'' prescale
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) o[mt][nt][e] *= down;
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 4);
-            l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 8);
-            l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 16);
+                    for (int e = 0; e < 4; ++e) o[mt][nt][e] *= down;
         }
-    __syncthreads();                              // every stage consumed: reuse shared memory
-    float* red = reinterpret_cast<float*>(smem);  // [NW][16][RS]
-    float* red_m = red + Lay::RED_M;
-    float* red_l = red + Lay::RED_L;
-    // head_dim of O^T m-tile mt, row g (e = 0) or g + 8 (e = 1) of this thread
-    auto drow = [&](int mt, int e) -> int {
-        if (G32) return 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + e;
-        return (D == 128 ? 16 : 8) * g + 2 * mt + e;
-    };
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int h0 = 8 * nt + 2 * t;
-            red[(warp * 16 + h0) * Lay::RS + drow(mt, 0)] = o[mt][nt][0];
-            red[(warp * 16 + h0 + 1) * Lay::RS + drow(mt, 0)] = o[mt][nt][1];
-            red[(warp * 16 + h0) * Lay::RS + drow(mt, 1)] = o[mt][nt][2];
-            red[(warp * 16 + h0 + 1) * Lay::RS + drow(mt, 1)] = o[mt][nt][3];
-        }
-    if (g == 0) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                red_m[warp * 16 + 8 * nt + 2 * t + c] = m[nt][c];
-                red_l[warp * 16 + 8 * nt + 2 * t + c] = l[nt][c];
+                l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 4);
+                l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 8);
+                l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 16);
+                if (g == 0) mrg_m[warp * 16 + 8 * nt + 2 * t + c] = m[nt][c];
             }
-    }
-    __syncthreads();
-    float* cp = red + Lay::CP;                    // [16][CPS]: o (unnormalised), m, l
-    float* wt = red + Lay::WT;                    // [NW][16] weight of each warp's state
-    if (tid < G) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * 16 + tid]);
-        float lsum = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-            const float mw = red_m[w * 16 + tid];
-            const float fw = (mw == -INFINITY) ? 0.f : ptx::ex2(mw - M);
-            wt[w * 16 + tid] = fw;
-            lsum = fmaf(fw, red_l[w * 16 + tid], lsum);
-        }
-        cp[tid * Lay::CPS + D] = M;
-        cp[tid * Lay::CPS + D + 1] = lsum;
-    }
-    __syncthreads();
-    for (int idx = tid; idx < G * D; idx += NTHREADS) {
-        const int h = idx / D, d = idx - h * D;
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) acc = fmaf(wt[w * 16 + h], red[(w * 16 + h) * Lay::RS + d], acc);
-        cp[h * Lay::CPS + d] = acc;
-    }
-    __syncthreads();
-
-    const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
-    if (S > 1) {
-        // ---- cluster combine.  CTA r owns outputs [r*OPC, (r+1)*OPC) of the
-        // flattened (head, head_dim) row; every CTA stores its partial values of
-        // those outputs and its (m, l) of every head into row j of the owner's
-        // receive buffer, one cluster barrier publishes all of them, and each
-        // owner combines its outputs from local shared memory.
-        const int GD = G * D;
-        const int OPC = (GD + S - 1) / S;
-        const int RW = OPC + 2 * G;
-        const uint32_t recv = sbase + Lay::RECV_OFF;
-        for (int idx = tid; idx < GD; idx += NTHREADS) {
-            const int r = idx / OPC, off = idx - r * OPC;
-            const int h = idx / D, d = idx - h * D;
-            st_cluster_f32(mapa(recv + (j * RW + off) * 4, r), cp[h * Lay::CPS + d]);
-        }
-        for (int idx = tid; idx < S * G; idx += NTHREADS) {
-            const int r = idx / G, h = idx - r * G;
-            st_cluster_f32(mapa(recv + (j * RW + OPC + h) * 4, r), cp[h * Lay::CPS + D]);
-            st_cluster_f32(mapa(recv + (j * RW + OPC + G + h) * 4, r), cp[h * Lay::CPS + D + 1]);
-        }
-        cluster_sync_all();                       // every CTA's pushes are visible
-        const float* rv = reinterpret_cast<const float*>(smem + Lay::RECV_OFF);
-        float* cw = red + Lay::CW;                // [S][16] weights
-        float* csum = red + Lay::CSUM;            // [16]
-        if (tid < G) {
-            float M = -INFINITY;
-            for (int r = 0; r < S; ++r) M = fmaxf(M, rv[r * RW + OPC + tid]);
-            float lsum = 0.f;
-            for (int r = 0; r < S; ++r) {
-                const float mr = rv[r * RW + OPC + tid];
-                const float w = (mr == -INFINITY) ? 0.f : ptx::ex2(mr - M);
-                cw[r * 16 + tid] = w;
-                lsum = fmaf(w, rv[r * RW + OPC + G + tid], lsum);
-            }
-            csum[tid] = lsum;
-        }
         __syncthreads();
-        for (int off = tid; off < OPC; off += NTHREADS) {
-            const int idx = j * OPC + off;
-            if (idx >= GD) break;
-            const int h = idx / D, d = idx - h * D;
-            float acc = 0.f;
-            for (int r = 0; r < S; ++r) acc = fmaf(cw[r * 16 + h], rv[r * RW + off], acc);
-            const float lsum = csum[h];
-            p.out[(bh0 + h) * D + d] = lsum > 0.f ? acc / lsum : 0.f;
+        // rescale this warp's state to the common maximum of each head
+        float Mh[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int h = 8 * nt + 2 * t + c;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) M = fmaxf(M, mrg_m[w * 16 + h]);
+                Mh[nt][c] = M;
+                const float f = (m[nt][c] == -INFINITY) ? 0.f : ptx::ex2(m[nt][c] - M);
+                l[nt][c] *= f;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    o[mt][nt][c] *= f;
+                    o[mt][nt][2 + c] *= f;
+                }
+            }
+        // pairwise tree over the warps: 8 -> 4 -> 2 -> 1 (register order, conflict-free)
+#pragma unroll
+        for (int half = NW / 2; half >= 1; half >>= 1) {
+            if (warp >= half && warp < 2 * half) {
+                float* slot = mbuf + (warp - half) * Lay::NV * 32 + lane;
+                int v = 0;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) slot[(v++) * 32] = o[mt][nt][e];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    slot[(v++) * 32] = l[nt][0];
+                    slot[(v++) * 32] = l[nt][1];
+                }
+            }
+            __syncthreads();
+            if (warp < half) {
+                const float* slot = mbuf + warp * Lay::NV * 32 + lane;
+                int v = 0;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o[mt][nt][e] += slot[(v++) * 32];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    l[nt][0] += slot[(v++) * 32];
+                    l[nt][1] += slot[(v++) * 32];
+                }
+            }
+            __syncthreads();
         }
-    } else if (nsplit <= 1) {
-        // single split (or empty sequence): the final row
-        if (j == 0)
-            for (int idx = tid; idx < G * D; idx += NTHREADS) {
-                const int h = idx / D, d = idx - h * D;
-                const float lsum = cp[h * Lay::CPS + D + 1];
-                p.out[(bh0 + h) * D + d] = lsum > 0.f ? cp[h * Lay::CPS + d] / lsum : 0.f;
-            }
-    } else if (active) {
-        // many splits without a cluster: partials for the combine kernel
-        for (int idx = tid; idx < G * D; idx += NTHREADS) {
-            const int h = idx / D, d = idx - h * D;
-            p.ws_o[((bh0 + h) * p.splits + j) * D + d] = cp[h * Lay::CPS + d];
-            if (d == 0) {
-                p.ws_m[(bh0 + h) * p.splits + j] = cp[h * Lay::CPS + D];
-                p.ws_l[(bh0 + h) * p.splits + j] = cp[h * Lay::CPS + D + 1];
-            }
+        // warp 0 holds the item's (o, l); write the final rows or the partial
+        if (warp == 0) {
+            auto drow = [&](int mt, int e) -> int {
+                if (G32) return 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + e;
+                return (D == 128 ? 16 : 8) * g + 2 * mt + e;
+            };
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int h = 8 * nt + 2 * t + c;
+                    if (h >= G) continue;
+                    const int64_t row = bh0 + h;
+                    if (nsplit == 1) {
+                        const float inv_ok = l[nt][c] > 0.f ? 1.f : 0.f;
+                        const float lden = l[nt][c] > 0.f ? l[nt][c] : 1.f;
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            p.out[row * D + drow(mt, 0)] = inv_ok * (o[mt][nt][c] / lden);
+                            p.out[row * D + drow(mt, 1)] = inv_ok * (o[mt][nt][2 + c] / lden);
+                        }
+                    } else {
+                        float* wo = p.ws_o + (row * p.splits + cw.j) * D;
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            wo[drow(mt, 0)] = o[mt][nt][c];
+                            wo[drow(mt, 1)] = o[mt][nt][2 + c];
+                        }
+                        if (g == 0) {
+                            p.ws_m[row * p.splits + cw.j] = Mh[nt][c];
+                            p.ws_l[row * p.splits + cw.j] = l[nt][c];
+                        }
+                    }
+                }
         }
     }
+    if (warp == 0) asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -792,7 +790,7 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
 
 template <int D, bool G32, bool PAGED, bool G16>
 cudaError_t set_attrs() {
-    using Lay = Layout<D, G32>;
+    using Lay = Layout<D, G32, G16>;
     static bool done = false;
     if (done) return cudaSuccess;
     auto kern = decode_split_tc<D, G32, PAGED, G16>;
@@ -800,15 +798,13 @@ cudaError_t set_attrs() {
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e == cudaSuccess) done = true;
     return e;
 }
 
 template <int D, bool G32, bool PAGED, bool G16>
 cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
-    using Lay = Layout<D, G32>;
+    using Lay = Layout<D, G32, G16>;
     cudaError_t e = set_attrs<D, G32, PAGED, G16>();
     if (e != cudaSuccess) return e;
     CUtensorMap mk, mv;
@@ -819,19 +815,15 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     if (e == cudaSuccess) e = make_map(&mv, p.v, D, rows, box);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.splits, p.Hk, p.B);
+    cfg.gridDim = dim3(p.grid, 1, 1);
     cfg.blockDim = dim3(NTHREADS, 1, 1);
     cfg.dynamicSmemBytes = Lay::SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
-    if (p.cluster > 1) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = p.cluster;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16>, mk, mv, p);
 }
 
@@ -850,37 +842,10 @@ cudaError_t pick_layout(const DecodeParams& p, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s) {
-    if (p.cluster > kMaxCluster || (p.cluster > 1 && p.cluster != p.splits))
-        return cudaErrorInvalidValue;
+    if (p.grid < 1) return cudaErrorInvalidValue;
     if (p.D == 128) return pick_layout<128>(p, s);
     if (p.D == 64) return pick_layout<64>(p, s);
     return cudaErrorInvalidValue;
-}
-
-int decode_max_cluster() {
-    static int cached = 0;
-    if (cached) return cached;
-    // the most demanding variant (registers, shared memory) bounds every other
-    auto kern = decode_split_tc<128, true, true, true>;
-    int n = 0;
-    if (set_attrs<128, true, true, true>() == cudaSuccess) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(kMaxCluster, 1, 1);
-        cfg.blockDim = dim3(NTHREADS, 1, 1);
-        cfg.dynamicSmemBytes = Layout<128, true>::SMEM;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = kMaxCluster;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaOccupancyMaxPotentialClusterSize(&n, kern, &cfg) != cudaSuccess) n = 0;
-    }
-    cudaGetLastError();                           // a failed query leaves no sticky error
-    n = n < 1 ? 1 : (n > kMaxCluster ? kMaxCluster : n);
-    cached = n;
-    return n;
 }
 
 }  // namespace kvq

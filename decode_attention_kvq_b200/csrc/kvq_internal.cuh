@@ -60,15 +60,19 @@ struct DecodeParams {
     int group32;
     int page_size, max_seq, max_pages, num_pages;
     int chunk;               // KV tokens per split
-    int splits;              // splits of the longest sequence (grid.x)
-    int cluster;             // > 1: the splits form one thread-block cluster and
-                             // combine in distributed shared memory (cluster == splits)
+    int splits;              // chunks of the longest sequence
+    int grid;                // persistent CTAs of the split kernel
     float scale_log2;        // attn_scale * log2(e)
 };
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 // tensor-core split kernel (kvq_decode_tc.cu)
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s);
-// largest cluster of split CTAs the current device can co-schedule (1..16)
-int decode_max_cluster();
+
+// Programmatic dependent launch: wait for the preceding grid's writes, and
+// let the next grid in the stream be scheduled early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 }  // namespace kvq

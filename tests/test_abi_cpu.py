@@ -69,15 +69,16 @@ def test_decode_plan_covers_hint(kvq, B, Hk, hint, ns):
 
 
 def test_decode_plan_fills_the_machine(kvq):
-    # few (sequence, kv head) units: up to one 16-CTA cluster of splits per unit
+    # few (sequence, kv head) units and a short cache: about one chunk per SM
     chunk, splits = kvq.kvq_decode_plan(1, 8, 4097, 0, num_sms=148)
-    assert splits == 16 and chunk == 272
+    assert (chunk, splits) == (240, 18) and 8 * splits <= 148
+    # long cache: chunks of >= 512 tokens, about 16 per SM
     chunk, splits = kvq.kvq_decode_plan(1, 8, 131073, 0, num_sms=148)
-    assert splits == 16
-    # enough units to fill the machine twice over: no split at all
+    assert chunk == 512 and splits == 257
+    # many units: still >= 512-token chunks that spread over the persistent CTAs
     chunk, splits = kvq.kvq_decode_plan(37, 8, 16385, 0, num_sms=148)
-    assert splits == 1
-    # explicit split counts beyond one cluster are honoured (combine kernel path)
+    assert chunk % 16 == 0 and chunk >= 512 and splits == -(-16385 // chunk)
+    # explicit split counts are honoured up to the 16-token rounding of the chunk
     chunk, splits = kvq.kvq_decode_plan(1, 8, 4097, 64, num_sms=148)
     assert 16 < splits <= 64
 
