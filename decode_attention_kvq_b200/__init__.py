@@ -173,6 +173,30 @@ def kvq_decode_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *, Hk
     return out
 
 
+def kvq_decode_attn_noalloc(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *,
+                            Hk=None, page_table=None, page_size=0, attn_scale=None,
+                            mode="per_token", out=None, num_splits=0, err=None, stream=None,
+                            view: Optional[CacheView] = None):
+    """kvq_decode_attn without a caller workspace: the split-K scratch is the
+    library's own fixed array (for callers that cannot allocate device memory;
+    see include/kvq.h).  `out` must be given by callers that cannot allocate."""
+    B, Hq, D = q.shape
+    if Hk is None:
+        Hk = k.shape[1]
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    if view is None:
+        view = cache_view(k, v, k_scale, v_scale, page_table, page_size)
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
+    check(lib.kvq_decode_attn_noalloc(
+        _ptr(q, torch.bfloat16, "q"), B, Hq, Hk, D, _mode(mode), ctypes.byref(view),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(max_seq_len_hint), float(attn_scale),
+        _ptr(out, torch.float32, "out"), int(num_splits), _ptr(err, torch.int32, "err"),
+        _stream(stream, q)), "kvq_decode_attn_noalloc")
+    return out
+
+
 def kvq_dequant(q, scale, mode="per_token", out=None, stream=None):
     """fp32 (byte - 128) * scale for q u8 [..., D], scale fp32 [..., NG]."""
     D = q.shape[-1]

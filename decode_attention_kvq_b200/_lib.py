@@ -31,6 +31,8 @@ _PROTOS = {
     "kvq_read_error": (_I, [_P, _P, _P]),
     "kvq_cache_bytes": (_I64, [_I64, _I64, _I64, _I, _I]),
     "kvq_version": (ctypes.c_char_p, []),
+    "kvq_decode_attn_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _I, _P, _P]),
+    "kvq_noalloc_scratch_bytes": (_SZ, []),
 }
 
 for _name, (_res, _args) in _PROTOS.items():

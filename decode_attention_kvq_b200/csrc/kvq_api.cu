@@ -209,6 +209,7 @@ const char* kvq_status_string(kvq_status status) {
         case KVQ_ERR_UNSUPPORTED: return "KVQ_ERR_UNSUPPORTED";
         case KVQ_ERR_CUDA: return "KVQ_ERR_CUDA";
         case KVQ_ERR_DEVICE_FLAG: return "KVQ_ERR_DEVICE_FLAG";
+        case KVQ_ERR_SCRATCH_TOO_SMALL: return "KVQ_ERR_SCRATCH_TOO_SMALL";
     }
     return "KVQ_UNKNOWN_STATUS";
 }

@@ -48,7 +48,9 @@ typedef enum kvq_status {
     KVQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, too small workspace */
     KVQ_ERR_UNSUPPORTED = 2,   /* valid but not built: head_dim or GQA group outside the kernels' set */
     KVQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
-    KVQ_ERR_DEVICE_FLAG = 4    /* kvq_read_error found device-side error bits */
+    KVQ_ERR_DEVICE_FLAG = 4,   /* kvq_read_error found device-side error bits */
+    KVQ_ERR_SCRATCH_TOO_SMALL = 5  /* kvq_decode_attn_noalloc: the problem needs more split-K
+                                      scratch than the library's fixed array holds */
 } kvq_status;
 
 typedef enum kvq_scale_mode {
@@ -189,6 +191,40 @@ kvq_status kvq_decode_plan(int B, int Hk, int max_seq_len_hint, int num_splits, 
  */
 kvq_status kvq_dequant(const uint8_t *q, const float *scale, int64_t rows, int D,
                        kvq_scale_mode mode, float *out, kvq_stream_t stream);
+
+/*
+ * kvq_decode_attn_noalloc -- kvq_decode_attn for callers that cannot allocate
+ * device memory.  The pages this library follows have no counterpart of this
+ * call; it exists for integration.  Some callers cannot call cudaMalloc (or
+ * any allocator) where they run attention: code inside a CUDA graph capture
+ * that must not allocate, plugin or embedded hosts that only hand over their
+ * own input and output buffers, runtimes whose allocator this C interface
+ * cannot reach.  This entry point takes the same arguments as
+ * kvq_decode_attn minus the workspace, and uses instead a split-K scratch
+ * array that lives inside the library: a file-scope __device__ array of
+ * kvq_noalloc_scratch_bytes() bytes (16 MiB), present on every GPU that loads
+ * the library until the process exits.
+ *  - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
+ *    library routine is called.
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress (with that device current) and caches it; make that
+ *    first call before any stream capture.
+ *  - Problems whose split-K scratch (kvq_decode_workspace_bytes for the same
+ *    arguments) exceeds the array return KVQ_ERR_SCRATCH_TOO_SMALL before
+ *    anything is enqueued.
+ *  - Every call on a device shares the one array and leaves its last
+ *    contents in it (nothing in it needs to start at zero).  Calls whose GPU
+ *    work overlaps (different streams without ordering, or concurrent host
+ *    threads on different streams) race on the array; serialise them.
+ */
+kvq_status kvq_decode_attn_noalloc(const uint16_t *q, int B, int Hq, int Hk, int D,
+                                   kvq_scale_mode mode, const kvq_cache_view *kv,
+                                   const int32_t *d_seq_lens, int max_seq_len_hint,
+                                   float attn_scale, float *out, int num_splits, int32_t *d_err,
+                                   kvq_stream_t stream);
+
+/* Size in bytes of the scratch array kvq_decode_attn_noalloc uses (no counterpart on the pages). */
+size_t kvq_noalloc_scratch_bytes(void);
 
 /* Human-readable name of a status code (static string). */
 const char *kvq_status_string(kvq_status status);
