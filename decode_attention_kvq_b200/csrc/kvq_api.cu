@@ -13,6 +13,7 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 constexpr int kMaxSplits = 4096;     // bound on splits per sequence (combine smem)
+constexpr int kMaxBatch = 1024;      // sequences per decode call (split kernel smem)
 
 kvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
 
@@ -155,6 +156,8 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
     const int G = Hq / Hk;
     if (D != 64 && D != 128) return KVQ_ERR_UNSUPPORTED;
     if (G > 16) return KVQ_ERR_UNSUPPORTED;
+    // the split kernel keeps every sequence length in shared memory
+    if (B > kMaxBatch) return KVQ_ERR_UNSUPPORTED;
     // TMA row coordinates are 32-bit
     const int64_t rows = kv->page_size ? static_cast<int64_t>(kv->num_pages) * Hk * 16
                                        : static_cast<int64_t>(B) * Hk * kv->max_seq;
@@ -164,6 +167,8 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
     int chunk = 0, splits = 0;
     kvq_status st = plan(B, Hk, max_seq_len_hint, num_splits, 0, &chunk, &splits);
     if (st != KVQ_OK) return st;
+    // work items (sequence, kv head, chunk) are counted in 32-bit integers
+    if (static_cast<int64_t>(B) * Hk * splits >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
     const size_t need = workspace_for(B, Hq, D, splits);
     if (need > 0 && (!workspace || workspace_bytes < need)) return KVQ_ERR_INVALID_ARG;
 

@@ -3,10 +3,14 @@
 // by the combine kernel below (launched as a programmatic dependent so its
 // launch overlaps the split kernel).
 //
-// Combine (flash-decoding): for each (sequence, q head) with splits j =
+// Combine (flash-decoding): for each (sequence, q head) with chunk slots j =
 // 0..ns-1 holding unnormalised (o_j, m_j, l_j) in base 2,
 //   M = max_j m_j,  w_j = 2^(m_j - M),  out = sum_j w_j o_j / sum_j w_j l_j.
-// Sequences with a single split were finished by the split kernel.
+// The split kernel merges consecutive chunks it owns into the slot of the
+// first of them and marks the others empty (m = -inf, l = 0); a slot of
+// weight zero is skipped, never multiplied (its o was not written).  A
+// sequence finished whole by one CTA carries l_0 = -1 and is left alone, as
+// are sequences with a single chunk.
 #include <math.h>
 
 #include "kvq_internal.cuh"
@@ -16,14 +20,17 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
+constexpr int kBatch = 8;                       // slots in flight per warp
+constexpr int kDirect = kWarps * kBatch;        // up to this many slots: one round of loads
+constexpr int kMaxList = 4096;                  // = the planner's bound on splits
 
-// One CTA per (b, q head).  Warp w folds splits w, w+4, ... with 16-byte
-// loads (lane l owns head_dim [4l, 4l+4)), then the four warps are summed.
+// One CTA per (b, q head); lane l of a warp owns head_dim [4l, 4l + 4).
 __global__ void __launch_bounds__(kThreads)
 decode_combine(DecodeParams p) {
-    extern __shared__ float s_w[];                 // [splits] weights
-    __shared__ float s_red[kWarps];
-    __shared__ __align__(16) float s_acc[kWarps][256];
+    __shared__ float s_m[kWarps], s_l[kWarps];
+    __shared__ __align__(16) float s_acc[kWarps][128];
+    __shared__ int s_cnt[kWarps];
+    __shared__ int s_list[kMaxList];            // slots of non-zero weight (long sequences)
     grid_dep_wait();                    // the split kernel's partials are complete
     const int64_t bh = blockIdx.x;
     const int b = static_cast<int>(bh / p.Hq);
@@ -37,43 +44,102 @@ decode_combine(DecodeParams p) {
 
     const float* m = p.ws_m + bh * p.splits;
     const float* lv = p.ws_l + bh * p.splits;
-    float M = -INFINITY;
-    for (int j = tid; j < ns; j += kThreads) M = fmaxf(M, m[j]);
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if (lane == 0) s_red[w] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-    __syncthreads();
-    float lsum = 0.f;
-    for (int j = tid; j < ns; j += kThreads) {
-        const float wj = (M == -INFINITY) ? 0.f : exp2f(m[j] - M);
-        s_w[j] = wj;
-        lsum = fmaf(wj, lv[j], lsum);
-    }
-    for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-    if (lane == 0) s_red[w] = lsum;
-    __syncthreads();
-    lsum = s_red[0] + s_red[1] + s_red[2] + s_red[3];
-
     const int D = p.D;
     const bool active = lane * 4 < D;
+    const float* o = p.ws_o + bh * p.splits * D + lane * 4;
+    const bool finished = lv[0] < 0.f;
+
+    // per-warp online fold over a list of slots: running max Mw, sums lw, acc
+    float Mw = -INFINITY, lw = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float* o = p.ws_o + bh * p.splits * D;
-    if (active) {
-#pragma unroll 4
-        for (int j = w; j < ns; j += kWarps) {
-            const float4 v = *reinterpret_cast<const float4*>(o + static_cast<int64_t>(j) * D + lane * 4);
-            const float wj = s_w[j];
-            acc.x = fmaf(wj, v.x, acc.x);
-            acc.y = fmaf(wj, v.y, acc.y);
-            acc.z = fmaf(wj, v.z, acc.z);
-            acc.w = fmaf(wj, v.w, acc.w);
+    auto fold = [&](const float (&mj)[kBatch], const float (&lj)[kBatch],
+                    const float4 (&oj)[kBatch]) {
+        float Mn = Mw;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) Mn = fmaxf(Mn, mj[u]);
+        if (Mn == -INFINITY) return;
+        const float a = exp2f(Mw - Mn);                   // 0 while Mw is -inf
+        acc.x *= a; acc.y *= a; acc.z *= a; acc.w *= a;
+        lw *= a;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            if (mj[u] == -INFINITY) continue;             // empty slot: o unwritten
+            const float wj = exp2f(mj[u] - Mn);
+            acc.x = fmaf(wj, oj[u].x, acc.x);
+            acc.y = fmaf(wj, oj[u].y, acc.y);
+            acc.z = fmaf(wj, oj[u].z, acc.z);
+            acc.w = fmaf(wj, oj[u].w, acc.w);
+            lw = fmaf(wj, lj[u], lw);
         }
-        *reinterpret_cast<float4*>(&s_acc[w][lane * 4]) = acc;
+        Mw = Mn;
+    };
+
+    if (ns <= kDirect) {
+        // one round: every slot's m, l and o are loaded together
+        float mj[kBatch], lj[kBatch];
+        float4 oj[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int j = w + u * kWarps;
+            const bool in = j < ns;
+            mj[u] = in ? m[j] : -INFINITY;
+            lj[u] = in ? lv[j] : 0.f;
+            oj[u] = (in && active) ? *reinterpret_cast<const float4*>(o + static_cast<int64_t>(j) * D)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (!finished) fold(mj, lj, oj);
+    } else if (!finished) {
+        // long sequences: list the slots that hold a partial (in slot order),
+        // then load only those
+        int n = 0;
+        for (int base = 0; base < ns; base += kThreads) {
+            const int j = base + tid;
+            const bool live = j < ns && m[j] != -INFINITY;
+            const uint32_t bal = __ballot_sync(0xffffffffu, live);
+            if (lane == 0) s_cnt[w] = __popc(bal);
+            __syncthreads();
+            int off = n;
+            for (int x = 0; x < w; ++x) off += s_cnt[x];
+            if (live) s_list[off + __popc(bal & ((1u << lane) - 1u))] = j;
+            for (int x = 0; x < kWarps; ++x) n += s_cnt[x];
+            __syncthreads();
+        }
+        for (int u0 = w; u0 < n; u0 += kWarps * kBatch) {
+            float mj[kBatch], lj[kBatch];
+            float4 oj[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int k = u0 + u * kWarps;
+                const int j = k < n ? s_list[k] : 0;
+                mj[u] = k < n ? m[j] : -INFINITY;
+                lj[u] = k < n ? lv[j] : 0.f;
+                oj[u] = (k < n && active)
+                            ? *reinterpret_cast<const float4*>(o + static_cast<int64_t>(j) * D)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            fold(mj, lj, oj);
+        }
     }
+    if (finished) return;                           // uniform over the CTA
+    if (lane == 0) {
+        s_m[w] = Mw;
+        s_l[w] = lw;
+    }
+    if (active) *reinterpret_cast<float4*>(&s_acc[w][lane * 4]) = acc;
     __syncthreads();
+    float M = s_m[0];
+#pragma unroll
+    for (int x = 1; x < kWarps; ++x) M = fmaxf(M, s_m[x]);
+    float f[kWarps], lsum = 0.f;
+#pragma unroll
+    for (int x = 0; x < kWarps; ++x) {
+        f[x] = s_m[x] == -INFINITY ? 0.f : exp2f(s_m[x] - M);
+        lsum = fmaf(f[x], s_l[x], lsum);
+    }
     for (int d = tid; d < D; d += kThreads) {
-        const float sum = s_acc[0][d] + s_acc[1][d] + s_acc[2][d] + s_acc[3][d];
+        float sum = 0.f;
+#pragma unroll
+        for (int x = 0; x < kWarps; ++x) sum = fmaf(f[x], s_acc[x][d], sum);
         p.out[bh * D + d] = lsum > 0.f ? sum / lsum : 0.f;
     }
 }
@@ -86,7 +152,7 @@ cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.B * p.Hq, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(p.splits) * sizeof(float);
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

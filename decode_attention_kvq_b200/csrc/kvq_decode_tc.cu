@@ -1,7 +1,7 @@
 // kvq_decode_tc.cu -- decode attention on the INT8 cache for sm_100a:
-// a persistent split-K kernel with TMA-staged K/V tiles and tensor-core
-// Q.K^T and P.V on exact integer operands, the dequantisation scales applied
-// outside the MMA.
+// a persistent split-K kernel with a TMA-fed shared-memory ring and
+// tensor-core Q.K^T and P.V on exact integer operands, the dequantisation
+// scales applied outside the MMA.
 //
 // Method (what is computed): abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
 // module doc "Fused approach" -- Q.K^T with K dequantised on the fly,
@@ -12,19 +12,24 @@
 //
 // How (sm_100a):
 //  * Work items are (sequence b, kv head, chunk j) with chunk = p.chunk
-//    tokens.  The grid is persistent (at most one CTA per SM); CTA c takes the
-//    items c, c + gridDim.x, ... of the list ordered (j, b, kv head), so long
-//    and short sequences spread over all SMs.  An item that is a whole
-//    sequence writes the final rows; otherwise it writes its partial softmax
-//    state (o, m, l) for the combine kernel (kvq_decode.cu).
-//  * CTA = 8 warps.  Warp 0 streams 128-token stages into a ring of 4-8
-//    stages (~200 KB of shared memory, so one CTA fills an SM): K and V
-//    bytes by TMA tile loads (2-D tensor maps over the cache rows, 128-byte
-//    swizzle for D=128, 64-byte for D=64), the fp32 scales and, with an
-//    item's first stage, the item's query rows by cp.async; all complete on
-//    the stage's mbarrier.  The ring runs across item boundaries, so the
-//    memory pipe stays busy while the warps merge an item.  Every warp takes
-//    one 16-token slice of each stage.
+//    tokens, listed in (b, kv head, j) order.  The grid is persistent (at
+//    most one CTA per SM) and CTA c takes the contiguous block
+//    [c*T/grid, (c+1)*T/grid) of the T items, found from a prefix sum of the
+//    per-sequence chunk counts (sequence lengths cached in shared memory).
+//    Consecutive chunks of one (b, kv head) inside a CTA's block form a
+//    segment and share one softmax state; a segment that is a whole
+//    sequence writes the final rows, any other writes one partial state
+//    (o, m, l) into the slot of its first chunk and marks the slots of its
+//    other chunks empty for the combine kernel (kvq_decode.cu).
+//  * CTA = 8 consumer warps + 1 producer warp.  The producer streams
+//    128-token stages into a ring of 3-8 stages (~150-180 KB of shared
+//    memory, one CTA per SM): K and V bytes by TMA tile loads (2-D tensor
+//    maps over the cache rows, 128-byte swizzle for D=128, 64-byte for
+//    D=64), the fp32 scales and, with a segment's first stage, its query
+//    rows by cp.async; all complete on the stage's mbarrier.  It refills a
+//    slot as soon as all consumers released it, independent of their
+//    progress elsewhere.  Every consumer warp takes one 16-token slice of
+//    each stage.
 //  * Per slice, on mma.sync m16n8k16 (f16 in, f32 accumulate), with the
 //    query heads of the GQA group as the N = 8 dimension (two n-tiles when
 //    G > 8):  S^T = K . Q^T (M = 16 tokens, K = head_dim) and
@@ -45,14 +50,14 @@
 //  * Token order inside each 16-token slice and the head_dim order of the
 //    MMA k-dimension are permuted so that every shared-memory load of the
 //    swizzled tiles is free of bank conflicts (sigma below).
-//  * An item's eight warp states are merged by a pairwise tree through a
-//    small dedicated buffer (deterministic: no atomics).
+//  * A segment's eight warp states are merged in one round through eight
+//    shared-memory slots in register order (deterministic: no atomics).
 //  * Programmatic dependent launch: the kernel waits for its predecessor in
-//    the stream before touching memory and lets its successor (the combine
-//    kernel) launch early.
+//    the stream before touching inputs and lets the combine kernel launch
+//    early.
 //  * mbarrier waits are bounded (KVQ_DEVERR_TIMEOUT when one gives up, after
-//    which every wait of the CTA returns at once); CTA barriers are reached
-//    by every thread unconditionally.
+//    which every wait of the CTA returns at once); barriers are reached by
+//    every participating thread unconditionally.
 #include <cuda.h>
 #include <math.h>
 
@@ -62,9 +67,11 @@
 namespace kvq {
 namespace {
 
-constexpr int NW = 8;                  // warps per CTA
-constexpr int NTHREADS = NW * 32;
+constexpr int NW = 8;                  // consumer warps per CTA
+constexpr int NCONS = NW * 32;         // consumer threads
+constexpr int NTHREADS = NCONS + 32;   // + the producer warp
 constexpr int TT = 16 * NW;            // tokens per stage: one 16-token slice per warp
+constexpr int kMaxB = 1024;            // sequences whose lengths are cached in shared memory
 
 // Row (inside an 8-token half of a slice) that holds MMA row r of the K
 // operand and MMA k-index r of the V operand: sigma = {0, 2, 4, 6, 3, 1, 7, 5}.
@@ -102,25 +109,28 @@ __device__ __forceinline__ void copy_scales(uint32_t dst, const float* src) {
     else ptx::cp_async_16(dst, src);
 }
 
-// Shared-memory plan (one CTA per SM): a ring of NST stages, each holding K
-// and V bytes of 128 tokens, their scales and room for one item's query rows;
-// the merge buffer; the stage mbarriers and the per-warp head maxima.
+// Shared-memory plan (one CTA per SM): a ring of NST stages (K and V bytes of
+// 128 tokens, their scales, room for one segment's query rows), the merge
+// slots, the cached lengths and chunk prefix sums, the stage mbarriers and
+// per-warp head maxima.
 template <int D, bool G32, bool G16>
 struct Layout {
     static constexpr int NG = G32 ? D / 32 : 1;
     static constexpr int KV_BYTES = TT * D;
     static constexpr int SC_FLOATS = TT * NG;
     static constexpr int Q_OFF = 2 * KV_BYTES + 2 * SC_FLOATS * 4;   // within a stage
-    static constexpr int Q_BYTES = 16 * D * 2;                        // up to 16 bf16 rows
+    static constexpr int Q_BYTES = (G16 ? 16 : 8) * D * 2;           // bf16 query rows
     static constexpr int STAGE = ((Q_OFF + Q_BYTES) + 1023) / 1024 * 1024;
-    static constexpr int NV = (G16 ? 2 : 1) * (D / 16) * 4 + 4;      // merged floats per thread
-    static constexpr int MERGE_BYTES = 4 * NV * 32 * 4;             // 4 warp slots
-    static constexpr int MISC_BYTES = 1024;                         // barriers, maxima, abort flag
-    static constexpr int BUDGET = 227 * 1024 - 1024 - MERGE_BYTES - MISC_BYTES;
+    static constexpr int NV = (G16 ? 2 : 1) * (D / 16) * 4 + (G16 ? 4 : 2);   // floats per lane
+    static constexpr int MERGE_BYTES = NW * NV * 32 * 4;
+    static constexpr int LENS_BYTES = 2 * (kMaxB + 1) * 4;          // lengths, prefix sums
+    static constexpr int MISC_BYTES = 2048;                         // barriers, maxima, flags
+    static constexpr int BUDGET = 227 * 1024 - 1024 - MERGE_BYTES - LENS_BYTES - MISC_BYTES;
     static constexpr int NST = (BUDGET / STAGE) > 8 ? 8 : (BUDGET / STAGE);
     static_assert(NST >= 3, "at least three stages");
     static constexpr int MERGE_OFF = NST * STAGE;
-    static constexpr int MISC_OFF = MERGE_OFF + MERGE_BYTES;
+    static constexpr int LENS_OFF = MERGE_OFF + MERGE_BYTES;
+    static constexpr int MISC_OFF = LENS_OFF + LENS_BYTES;
     static constexpr int SMEM = MISC_OFF + MISC_BYTES + 1024;       // + base alignment slack
     static_assert(SMEM <= 227 * 1024, "fits one SM");
 };
@@ -157,38 +167,31 @@ __device__ __forceinline__ float ldsf(uint32_t a) {
     return v;
 }
 
-// The items of one CTA: dense indices first, first + step, ... of the list
-// (j, b, kv head), skipping chunks past a sequence's end.  A sequence of
-// length 0 yields one item with t0 == t1 (its output rows are zero).
-struct Walk {
-    int64_t dense;
-    int b, hk, j, L, t0, t1;
+// One work item of a CTA's block: item index -> (b, kv head, chunk j).
+struct Item {
+    int b, hk, j, ns, L, t0, t1;   // ns = chunks of the sequence (0: empty sequence)
 };
 
-__device__ __forceinline__ bool walk_next(Walk& w, const DecodeParams& p, int64_t lim,
-                                          int64_t first, int64_t step, int64_t total) {
-    const int64_t per_j = static_cast<int64_t>(p.B) * p.Hk;
-    for (;;) {
-        w.dense = w.dense < 0 ? first : w.dense + step;
-        if (w.dense >= total) return false;
-        w.j = static_cast<int>(w.dense / per_j);
-        const int rem = static_cast<int>(w.dense - static_cast<int64_t>(w.j) * per_j);
-        w.b = rem / p.Hk;
-        w.hk = rem - w.b * p.Hk;
-        int L = p.seq_lens[w.b];
-        if (L < 0 || L > lim) L = 0;
-        w.L = L;
-        const int ns = (L + p.chunk - 1) / p.chunk;
-        if (ns == 0) {
-            if (w.j != 0) continue;
-            w.t0 = w.t1 = 0;
-            return true;
-        }
-        if (w.j >= ns) continue;
-        w.t0 = w.j * p.chunk;
-        w.t1 = min(w.t0 + p.chunk, L);
-        return true;
+// cum[b] = items of sequences < b (each sequence has Hk * max(1, ns_b) items)
+__device__ __forceinline__ Item item_at(int64_t i, const int* lens, const int* cum, int B,
+                                        int Hk, int chunk) {
+    int lo = 0, hi = B;                  // largest b with cum[b] <= i
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cum[mid] <= i) lo = mid;
+        else hi = mid;
     }
+    Item it;
+    it.b = lo;
+    it.L = lens[lo];
+    it.ns = (it.L + chunk - 1) / chunk;
+    const int per = it.ns > 0 ? it.ns : 1;
+    const int r = static_cast<int>(i - cum[lo]);
+    it.hk = r / per;
+    it.j = r - it.hk * per;
+    it.t0 = it.j * chunk;
+    it.t1 = it.ns > 0 ? min(it.t0 + chunk, it.L) : 0;
+    return it;
 }
 
 template <int D, bool G32, bool PAGED, bool G16>
@@ -198,6 +201,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     using Lay = Layout<D, G32, G16>;
     constexpr int NG = Lay::NG;
     constexpr int NST = Lay::NST;
+    constexpr int NV = Lay::NV;
     constexpr int KS = D / 16;          // MMA k-steps over head_dim (QK)
     constexpr int NGRP = D / 32;        // 32-value groups over head_dim
     constexpr int MT = D / 16;          // m-tiles of O^T over head_dim (PV)
@@ -217,11 +221,18 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t bar_full = sbase + Lay::MISC_OFF;
     const uint32_t bar_empty = bar_full + NST * 8;
-    float* mrg_m = reinterpret_cast<float*>(smem + Lay::MISC_OFF + 2 * NST * 8);   // [NW][16]
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_m + NW * 16);
-    float* mbuf = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);                // [4][NV][32]
+    // per-warp head maxima of a segment, double-buffered: a warp that has
+    // finished one segment's merge may write the next one's while slower warps
+    // still read the previous buffer (two merges apart, barrier 1 orders them)
+    float* mrg_m0 = reinterpret_cast<float*>(smem + Lay::MISC_OFF + 2 * NST * 8);  // [2][NW][16]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_m0 + 2 * NW * 16);
+    float* mslot = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);               // [NW][NV][32]
+    int* lens = reinterpret_cast<int*>(smem + Lay::LENS_OFF);                     // [B]
+    int* cum = lens + (kMaxB + 1);                                               // [B + 1]
 
     if (tid == 0) {
+        ptx::prefetch_tensormap(&tm_k);     // kernel parameters: safe before the dependency wait
+        ptx::prefetch_tensormap(&tm_v);
         for (int s = 0; s < NST; ++s) {
             ptx::mbar_init(bar_full + 8 * s, 1 + 32);   // expect_tx arrive + 32 cp.async arrivals
             ptx::mbar_init(bar_empty + 8 * s, NW);
@@ -229,14 +240,42 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    __syncthreads();
     grid_dep_wait();                    // the predecessor's writes (q, cache, lengths) are visible
     grid_dep_launch();                  // the combine kernel may be scheduled now
 
+    // ---- lengths and chunk prefix sums (items per sequence: Hk * max(1, chunks))
     const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
     const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
-    const int64_t total = static_cast<int64_t>(p.splits) * p.B * p.Hk;
-    const int64_t first = blockIdx.x, step = gridDim.x;
+    const int B = p.B;
+    for (int b = tid; b < B; b += NTHREADS) {
+        int L = p.seq_lens[b];
+        if (L < 0 || L > lim) {
+            if (blockIdx.x == 0) raise_flag(p.d_err, KVQ_DEVERR_LEN);
+            L = 0;
+        }
+        lens[b] = L;
+        const int ns = (L + p.chunk - 1) / p.chunk;
+        cum[b + 1] = p.Hk * (ns > 0 ? ns : 1);
+    }
+    __syncthreads();
+    if (warp == 0) {                    // inclusive scan of cum[1..B] by one warp
+        int carry = 0;
+        for (int base = 0; base < B; base += 32) {
+            int v = base + lane < B ? cum[base + lane + 1] : 0;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, v, off);
+                if (lane >= off) v += u;
+            }
+            if (base + lane < B) cum[base + lane + 1] = v + carry;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (lane == 0) cum[0] = 0;
+    }
+    __syncthreads();
+    const int64_t T = cum[B];
+    const int64_t ibeg = T * blockIdx.x / gridDim.x;
+    const int64_t iend = T * (blockIdx.x + 1) / gridDim.x;
 
     // bounded wait that gives up at once after any earlier timeout of this CTA
     auto wait = [&](uint32_t bar, uint32_t parity) {
@@ -247,85 +286,88 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
     };
 
-    // ---- producer state (warp 0): next tile to issue
-    Walk pw;
-    pw.dense = -1;
-    bool p_valid = walk_next(pw, p, lim, first, step, total);
-    int p_tile = 0;                     // tile within pw's item
-    int p_count = 0;                    // tiles issued so far (ring position)
-    const uint64_t pol = ptx::policy_evict_first();
-
-    // issue the next tile of this CTA's item list into the ring (warp 0, all lanes)
-    auto produce = [&]() {
-        while (p_valid && pw.t0 + p_tile * TT >= pw.t1) {
-            p_valid = walk_next(pw, p, lim, first, step, total);
-            p_tile = 0;
-        }
-        if (!p_valid) return;
-        const int s = p_count % NST;
-        const uint32_t full = bar_full + 8 * s;
-        const int tt0 = pw.t0 + p_tile * TT;
-        const int ntok = min(TT, pw.t1 - tt0);
-        const uint32_t sk = sbase + s * Lay::STAGE;
-        const uint32_t sv = sk + Lay::KV_BYTES;
-        const uint32_t sks = sv + Lay::KV_BYTES;
-        const uint32_t svs = sks + Lay::SC_FLOATS * 4;
-        const int b = pw.b, hk = pw.hk;
-        if (!PAGED) {
-            const int64_t row0 = (static_cast<int64_t>(b) * p.Hk + hk) * p.max_seq + tt0;
-            if (lane == 0) {
-                ptx::mbar_arrive_expect_tx(full, 2 * Lay::KV_BYTES);
-                ptx::tma_load_2d(sk, &tm_k, 0, static_cast<int>(row0), full, pol);
-                ptx::tma_load_2d(sv, &tm_v, 0, static_cast<int>(row0), full, pol);
-            }
-            for (int k = lane; k < ntok; k += 32) {
-                const int64_t r = row0 + k;
-                copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
-                copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
-            }
-        } else {
-            constexpr int PPS = TT / 16;                // pages per stage
-            const int np = (ntok + 15) >> 4;
-            int32_t pg = -1;
-            if (lane < np) {
-                // a bad entry is skipped here and reported by the consumers
-                pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tt0 >> 4) + lane];
-                if (pg < 0 || pg >= p.num_pages) pg = -1;
-            }
-            const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
-            if (lane == 0) ptx::mbar_arrive_expect_tx(full, __popc(valid) * 2 * 16 * D);
+    // ------------------------------------------------------------ producer
+    if (warp == NW) {
+        const uint64_t pol = ptx::policy_evict_first();
+        int count = 0;                  // tiles issued (ring position)
+        int pb = -1, phk = -1;
+        for (int64_t i = ibeg; i < iend; ++i) {
+            const Item itm = item_at(i, lens, cum, B, p.Hk, p.chunk);
+            if (itm.ns == 0) continue;
+            const bool seg_first = itm.b != pb || itm.hk != phk;
+            pb = itm.b;
+            phk = itm.hk;
+            const int b = itm.b, hk = itm.hk;
+            for (int tt0 = itm.t0; tt0 < itm.t1; tt0 += TT, ++count) {
+                const int s = count % NST;
+                const uint32_t full = bar_full + 8 * s;
+                if (count >= NST) wait(bar_empty + 8 * s, ((count / NST) - 1) & 1);
+                const int ntok = min(TT, itm.t1 - tt0);
+                const uint32_t sk = sbase + s * Lay::STAGE;
+                const uint32_t sv = sk + Lay::KV_BYTES;
+                const uint32_t sks = sv + Lay::KV_BYTES;
+                const uint32_t svs = sks + Lay::SC_FLOATS * 4;
+                if (!PAGED) {
+                    const int64_t row0 = (static_cast<int64_t>(b) * p.Hk + hk) * p.max_seq + tt0;
+                    if (lane == 0) {
+                        ptx::mbar_arrive_expect_tx(full, 2 * Lay::KV_BYTES);
+                        ptx::tma_load_2d(sk, &tm_k, 0, static_cast<int>(row0), full, pol);
+                        ptx::tma_load_2d(sv, &tm_v, 0, static_cast<int>(row0), full, pol);
+                    }
+                    for (int k = lane; k < ntok; k += 32) {
+                        const int64_t r = row0 + k;
+                        copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
+                        copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
+                    }
+                } else {
+                    constexpr int PPS = TT / 16;                // pages per stage
+                    const int np = (ntok + 15) >> 4;
+                    int32_t pg = -1;
+                    if (lane < np) {
+                        // a bad entry is skipped here and reported by the consumers
+                        pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tt0 >> 4) + lane];
+                        if (pg < 0 || pg >= p.num_pages) pg = -1;
+                    }
+                    const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
+                    if (lane == 0) ptx::mbar_arrive_expect_tx(full, __popc(valid) * 2 * 16 * D);
 #pragma unroll
-            for (int q = 0; q < PPS; ++q) {
-                const int pq = __shfl_sync(0xffffffffu, pg, q);
-                if (lane == 0 && pq >= 0) {
-                    const int y = (pq * p.Hk + hk) * 16;
-                    ptx::tma_load_2d(sk + q * 16 * D, &tm_k, 0, y, full, pol);
-                    ptx::tma_load_2d(sv + q * 16 * D, &tm_v, 0, y, full, pol);
+                    for (int q = 0; q < PPS; ++q) {
+                        const int pq = __shfl_sync(0xffffffffu, pg, q);
+                        if (lane == 0 && pq >= 0) {
+                            const int y = (pq * p.Hk + hk) * 16;
+                            ptx::tma_load_2d(sk + q * 16 * D, &tm_k, 0, y, full, pol);
+                            ptx::tma_load_2d(sv + q * 16 * D, &tm_v, 0, y, full, pol);
+                        }
+                    }
+                    for (int k = lane; k < TT; k += 32) {
+                        const int pk = __shfl_sync(0xffffffffu, pg, k >> 4);
+                        if (k < ntok && pk >= 0) {
+                            const int64_t r = (static_cast<int64_t>(pk) * p.Hk + hk) * 16 + (k & 15);
+                            copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
+                            copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
+                        }
+                    }
                 }
-            }
-            for (int k = lane; k < TT; k += 32) {
-                const int pk = __shfl_sync(0xffffffffu, pg, k >> 4);
-                if (k < ntok && pk >= 0) {
-                    const int64_t r = (static_cast<int64_t>(pk) * p.Hk + hk) * 16 + (k & 15);
-                    copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
-                    copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
+                if (seg_first && tt0 == itm.t0) {
+                    // the segment's G query rows (contiguous bf16) ride with its first stage
+                    const uint16_t* qsrc = p.q + (static_cast<int64_t>(b) * p.Hq + hk * G) * D;
+                    const uint32_t sq = sk + Lay::Q_OFF;
+                    for (int c = lane; c < G * D / 8; c += 32)
+                        ptx::cp_async_16(sq + c * 16, qsrc + c * 8);
                 }
+                ptx::cp_async_arrive_noinc(full);
             }
         }
-        if (p_tile == 0) {
-            // the item's G query rows (contiguous bf16) ride with its first stage
-            const uint16_t* qsrc = p.q + (static_cast<int64_t>(b) * p.Hq + hk * G) * D;
-            const uint32_t sq = sk + Lay::Q_OFF;
-            for (int c = lane; c < G * D / 8; c += 32) ptx::cp_async_16(sq + c * 16, qsrc + c * 8);
-        }
-        ptx::cp_async_arrive_noinc(full);
-        ++p_tile;
-        ++p_count;
-    };
-    if (warp == 0)
-        for (int k = 0; k < NST; ++k) produce();
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        // the last tile of every slot has landed (normally long consumed; after a
+        // timeout this keeps the CTA alive until its bulk copies are done)
+        if (lane == 0)
+            for (int c = count - 1; c >= 0 && c >= count - NST; --c)
+                ptx::mbar_wait(bar_full + 8 * (c % NST), (c / NST) & 1);
+        return;                         // consumers synchronise among themselves (barrier 1)
+    }
 
-    // ---- consumers: all eight warps
+    // ------------------------------------------------------------ consumers
     const int sig_g = sigma(g);
     const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
     const int rowA = 16 * warp + sig_g;           // MMA row g     of this warp's slice
@@ -333,39 +375,39 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int R0 = 16 * warp + sig_a, R1 = 16 * warp + sig_b;   // V rows of k 2t, 2t+1
     const int R2 = R0 + 8, R3 = R1 + 8;                         // V rows of k 2t+8, 2t+9
 
-    Walk cw;
-    cw.dense = -1;
-    int c_count = 0;                    // tiles consumed so far (ring position)
-    while (walk_next(cw, p, lim, first, step, total)) {
-        const int b = cw.b, hk = cw.hk;
+    uint32_t qb0[NT][KS], qb1[NT][KS];
+    float zs[NT][2];
+    float m[NT][2], l[NT][2];
+    float o[MT][NT][4];                 // O^T C fragments: rows = head_dim, columns = heads
+    int kv = 64;                        // running P'' prescale exponent (per warp)
+    int c_count = 0;                    // tiles consumed (ring position)
+    bool open = false;                  // a segment's state is live
+    int seg_j0 = 0;                     // first chunk of the open segment
+    int merges = 0;                     // segments merged so far (selects the maxima buffer)
+
+    for (int64_t i = ibeg; i < iend; ++i) {
+        const Item itm = item_at(i, lens, cum, B, p.Hk, p.chunk);
+        const int b = itm.b, hk = itm.hk;
         const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
-        if (cw.t0 == cw.t1) {
+        if (itm.ns == 0) {
             // empty (or rejected) sequence: zero rows
-            if (hk == 0 && tid == 0) {
-                const int Lraw = p.seq_lens[b];
-                if (Lraw < 0 || Lraw > lim) raise_flag(p.d_err, KVQ_DEVERR_LEN);
-            }
-            for (int idx = tid; idx < G * D; idx += NTHREADS) p.out[bh0 * D + idx] = 0.f;
+            for (int idx = tid; idx < G * D; idx += NCONS) p.out[bh0 * D + idx] = 0.f;
             continue;
         }
-        const int t0 = cw.t0, t1 = cw.t1;
-        const int nsplit = (cw.L + p.chunk - 1) / p.chunk;
-        const int ntiles = (t1 - t0 + TT - 1) / TT;
-
-        uint32_t qb0[NT][KS], qb1[NT][KS];
-        float zs[NT][2];
-        float m[NT][2], l[NT][2];
-        float o[MT][NT][4];             // O^T C fragments: rows = head_dim, columns = heads
+        if (!open) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            m[nt][0] = m[nt][1] = -INFINITY;
-            l[nt][0] = l[nt][1] = 0.f;
+            for (int nt = 0; nt < NT; ++nt) {
+                m[nt][0] = m[nt][1] = -INFINITY;
+                l[nt][0] = l[nt][1] = 0.f;
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-                o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+                for (int mt = 0; mt < MT; ++mt)
+                    o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+            }
+            kv = 64;
+            seg_j0 = itm.j;
         }
-        int kv = 64;                    // running P'' prescale exponent (per warp)
-
+        const int t0 = itm.t0, t1 = itm.t1;
+        const int ntiles = (t1 - t0 + TT - 1) / TT;
         for (int it = 0; it < ntiles; ++it, ++c_count) {
             const int s = c_count % NST;
             wait(bar_full + 8 * s, (c_count / NST) & 1);
@@ -374,7 +416,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const uint32_t sv = sk + Lay::KV_BYTES;
             const uint32_t sks = sv + Lay::KV_BYTES;
             const uint32_t svs = sks + Lay::SC_FLOATS * 4;
-            if (it == 0) {
+            if (!open && it == 0) {
                 // ---- Q^T operand from the stage: column n = g of n-tile nt is query
                 // head 8*nt + g, pre-scaled by 2^sh so max |q| * 2^sh is in [2^14, 2^15).
                 // B fragment rows 2t, 2t+1 (qb0) and 2t+8, 2t+9 (qb1) of k-step
@@ -633,14 +675,17 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bar_empty + 8 * s);
-            if (warp == 0) {
-                // refill slot s once all eight warps have released it
-                wait(bar_empty + 8 * s, (c_count / NST) & 1);
-                produce();
-            }
         }
+        open = true;
+        // the segment continues if the next item is the next chunk of this (b, kv head)
+        if (i + 1 < iend) {
+            const Item nx = item_at(i + 1, lens, cum, B, p.Hk, p.chunk);
+            if (nx.b == b && nx.hk == hk) continue;
+        }
+        open = false;
 
-        // ---- merge the eight warps' states of this item
+        // ---- merge the eight warps' states of the segment (one round)
+        float* mrg_m = mrg_m0 + (merges++ & 1) * NW * 16;
         {
             const float down = ldexpf(1.f, -kv);         // undo the P'' prescale
 #pragma unroll
@@ -659,99 +704,86 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 16);
                 if (g == 0) mrg_m[warp * 16 + 8 * nt + 2 * t + c] = m[nt][c];
             }
-        __syncthreads();
-        // rescale this warp's state to the common maximum of each head
-        float Mh[NT][2];
+        ptx::named_bar_sync(1, NCONS);
+        {
+            float* slot = mslot + warp * NV * 32 + lane;
+            int v = 0;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int h = 8 * nt + 2 * t + c;
-                float M = -INFINITY;
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int w = 0; w < NW; ++w) M = fmaxf(M, mrg_m[w * 16 + h]);
-                Mh[nt][c] = M;
-                const float f = (m[nt][c] == -INFINITY) ? 0.f : ptx::ex2(m[nt][c] - M);
-                l[nt][c] *= f;
+                    for (int e = 0; e < 4; ++e) {
+                        const int h = 8 * nt + 2 * t + (e & 1);
+                        float M = -INFINITY;
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    o[mt][nt][c] *= f;
-                    o[mt][nt][2 + c] *= f;
-                }
-            }
-        // pairwise tree over the warps: 8 -> 4 -> 2 -> 1 (register order, conflict-free)
-#pragma unroll
-        for (int half = NW / 2; half >= 1; half >>= 1) {
-            if (warp >= half && warp < 2 * half) {
-                float* slot = mbuf + (warp - half) * Lay::NV * 32 + lane;
-                int v = 0;
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) slot[(v++) * 32] = o[mt][nt][e];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    slot[(v++) * 32] = l[nt][0];
-                    slot[(v++) * 32] = l[nt][1];
-                }
-            }
-            __syncthreads();
-            if (warp < half) {
-                const float* slot = mbuf + warp * Lay::NV * 32 + lane;
-                int v = 0;
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) o[mt][nt][e] += slot[(v++) * 32];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    l[nt][0] += slot[(v++) * 32];
-                    l[nt][1] += slot[(v++) * 32];
-                }
-            }
-            __syncthreads();
-        }
-        // warp 0 holds the item's (o, l); write the final rows or the partial
-        if (warp == 0) {
-            auto drow = [&](int mt, int e) -> int {
-                if (G32) return 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + e;
-                return (D == 128 ? 16 : 8) * g + 2 * mt + e;
-            };
+                        for (int w = 0; w < NW; ++w) M = fmaxf(M, mrg_m[w * 16 + h]);
+                        const float mv = m[nt][e & 1];
+                        const float f = (mv == -INFINITY) ? 0.f : ptx::ex2(mv - M);
+                        slot[(v++) * 32] = o[mt][nt][e] * f;
+                    }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const int h = 8 * nt + 2 * t + c;
-                    if (h >= G) continue;
-                    const int64_t row = bh0 + h;
-                    if (nsplit == 1) {
-                        const float inv_ok = l[nt][c] > 0.f ? 1.f : 0.f;
-                        const float lden = l[nt][c] > 0.f ? l[nt][c] : 1.f;
+                    float M = -INFINITY;
 #pragma unroll
-                        for (int mt = 0; mt < MT; ++mt) {
-                            p.out[row * D + drow(mt, 0)] = inv_ok * (o[mt][nt][c] / lden);
-                            p.out[row * D + drow(mt, 1)] = inv_ok * (o[mt][nt][2 + c] / lden);
-                        }
-                    } else {
-                        float* wo = p.ws_o + (row * p.splits + cw.j) * D;
-#pragma unroll
-                        for (int mt = 0; mt < MT; ++mt) {
-                            wo[drow(mt, 0)] = o[mt][nt][c];
-                            wo[drow(mt, 1)] = o[mt][nt][2 + c];
-                        }
-                        if (g == 0) {
-                            p.ws_m[row * p.splits + cw.j] = Mh[nt][c];
-                            p.ws_l[row * p.splits + cw.j] = l[nt][c];
-                        }
-                    }
+                    for (int w = 0; w < NW; ++w) M = fmaxf(M, mrg_m[w * 16 + h]);
+                    const float f = (m[nt][c] == -INFINITY) ? 0.f : ptx::ex2(m[nt][c] - M);
+                    slot[(v++) * 32] = l[nt][c] * f;
                 }
         }
+        ptx::named_bar_sync(1, NCONS);
+        // sum the eight slots position by position and write the rows; a
+        // segment that is the whole sequence writes the final rows (and, when
+        // the sequence has several chunks, a marker l = -1 in slot 0 that tells
+        // the combine kernel to leave them alone)
+        const bool final_rows = itm.ns == 1 || (seg_j0 == 0 && itm.j == itm.ns - 1);
+        for (int pos = tid; pos < NV * 32; pos += NCONS) {
+            const int v = pos >> 5, ln = pos & 31;
+            const int pg_ = ln >> 2, pt = ln & 3;
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) sum += mslot[(w * NV + v) * 32 + ln];
+            if (v < MT * NT * 4) {
+                const int mt = v / (NT * 4), nt = (v / 4) % NT, e = v & 3;
+                const int h = 8 * nt + 2 * pt + (e & 1);
+                if (h >= G) continue;
+                const int d = G32 ? 32 * (mt >> 1) + 4 * pg_ + 2 * (mt & 1) + (e >> 1)
+                                  : (D == 128 ? 16 : 8) * pg_ + 2 * mt + (e >> 1);
+                const int64_t row = bh0 + h;
+                if (final_rows) {
+                    // the head's sum l sits at position (MT*NT*4 + 2*nt + c, lane pt)
+                    const int vl = MT * NT * 4 + 2 * nt + (e & 1);
+                    float lsum = 0.f;
+#pragma unroll
+                    for (int w = 0; w < NW; ++w) lsum += mslot[(w * NV + vl) * 32 + pt];
+                    p.out[row * D + d] = lsum > 0.f ? sum / lsum : 0.f;
+                } else {
+                    p.ws_o[(row * p.splits + seg_j0) * D + d] = sum;
+                }
+            } else if (pg_ == 0 && (!final_rows || itm.ns > 1)) {
+                const int k = v - MT * NT * 4, nt = k >> 1, c = k & 1;
+                const int h = 8 * nt + 2 * pt + c;
+                if (h >= G) continue;
+                if (final_rows) {
+                    p.ws_l[(bh0 + h) * p.splits] = -1.f;
+                    continue;
+                }
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) M = fmaxf(M, mrg_m[w * 16 + h]);
+                const int64_t row = bh0 + h;
+                p.ws_m[row * p.splits + seg_j0] = M;
+                p.ws_l[row * p.splits + seg_j0] = sum;
+                for (int jj = seg_j0 + 1; jj <= itm.j; ++jj) {     // chunks merged into seg_j0
+                    p.ws_m[row * p.splits + jj] = -INFINITY;
+                    p.ws_l[row * p.splits + jj] = 0.f;
+                }
+            }
+        }
     }
-    if (warp == 0) asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

@@ -152,7 +152,8 @@ typedef struct kvq_cache_view {
  *   d_err       int32 [1] or NULL (KVQ_DEVERR_LEN, KVQ_DEVERR_PAGE)
  * Requirements: Hq % Hk == 0 and Hq / Hk <= 16; D in {64, 128}; GROUP32
  * needs D % 32 == 0; B * Hk * max_seq (contiguous) or num_pages * Hk * 16
- * (paged) below 2^31 rows.
+ * (paged) below 2^31 rows; B <= 1024 and B * Hk * splits below 2^31
+ * (otherwise KVQ_ERR_UNSUPPORTED).
  * Source: abaddon 0.2.0-rc.1, kv_cache_quant_cuda.rs, module doc "Fused
  * approach" and CudaQuantizedKvCache::forward_attention (scores with
  * on-the-fly K dequantisation, softmax, P.V with on-the-fly V

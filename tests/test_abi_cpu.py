@@ -148,6 +148,7 @@ def test_decode_rejects_bad_arguments(kvq):
     assert call(D=256) == 2                 # valid, kernel not built for it
     assert call(D=32) == 2
     assert call(Hq=8 * 32, Hk=8) == 2       # GQA group above the built tile (16)
+    assert call(B=1025) == 2                # more sequences than the split kernel caches
     assert call(out=FAKE + 4) == 1          # misaligned output
     cv_bad_scale = kvq.CacheView(FAKE, FAKE, FAKE + 8, FAKE, 0, 4096, 0, 0, 0)
     assert call(kv=ctypes.byref(cv_bad_scale)) == 1
