@@ -35,19 +35,12 @@ decode_combine(DecodeParams p) {
     const int64_t bh = blockIdx.x;
     const int b = static_cast<int>(bh / p.Hq);
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int64_t cap = p.page_size ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
-    const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
-    int L = p.seq_lens[b];
-    if (L < 0 || L > lim) L = 0;
-    const int ns = (L + p.chunk - 1) / p.chunk;
-    if (ns <= 1) return;
-
+    const int L0 = p.seq_lens[b];
     const float* m = p.ws_m + bh * p.splits;
     const float* lv = p.ws_l + bh * p.splits;
     const int D = p.D;
     const bool active = lane * 4 < D;
     const float* o = p.ws_o + bh * p.splits * D + lane * 4;
-    const bool finished = lv[0] < 0.f;
 
     // per-warp online fold over a list of slots: running max Mw, sums lw, acc
     float Mw = -INFINITY, lw = 0.f;
@@ -74,21 +67,38 @@ decode_combine(DecodeParams p) {
         Mw = Mn;
     };
 
-    if (ns <= kDirect) {
-        // one round: every slot's m, l and o are loaded together
+    const int64_t cap = p.page_size ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
+    const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
+    bool finished;
+    if (p.splits <= kDirect) {
+        // one round: every slot of the workspace row is loaded together with the
+        // length (slots past the sequence's chunk count are in bounds and masked
+        // afterwards, before any arithmetic reads them)
         float mj[kBatch], lj[kBatch];
         float4 oj[kBatch];
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int j = w + u * kWarps;
-            const bool in = j < ns;
+            const bool in = j < p.splits;
             mj[u] = in ? m[j] : -INFINITY;
             lj[u] = in ? lv[j] : 0.f;
             oj[u] = (in && active) ? *reinterpret_cast<const float4*>(o + static_cast<int64_t>(j) * D)
                                    : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        if (!finished) fold(mj, lj, oj);
-    } else if (!finished) {
+        finished = lv[0] < 0.f;
+        const int L = (L0 < 0 || L0 > lim) ? 0 : L0;
+        const int ns = (L + p.chunk - 1) / p.chunk;
+        if (ns <= 1 || finished) return;               // uniform over the CTA
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+            if (w + u * kWarps >= ns) mj[u] = -INFINITY;
+        fold(mj, lj, oj);
+    } else {
+        const int L = (L0 < 0 || L0 > lim) ? 0 : L0;
+        const int ns = (L + p.chunk - 1) / p.chunk;
+        if (ns <= 1) return;
+        finished = lv[0] < 0.f;
+        if (finished) return;                          // uniform over the CTA
         // long sequences: list the slots that hold a partial (in slot order),
         // then load only those
         int n = 0;
@@ -120,7 +130,6 @@ decode_combine(DecodeParams p) {
             fold(mj, lj, oj);
         }
     }
-    if (finished) return;                           // uniform over the CTA
     if (lane == 0) {
         s_m[w] = Mw;
         s_l[w] = lw;

@@ -121,7 +121,7 @@ struct Layout {
     static constexpr int Q_OFF = 2 * KV_BYTES + 2 * SC_FLOATS * 4;   // within a stage
     static constexpr int Q_BYTES = (G16 ? 16 : 8) * D * 2;           // bf16 query rows
     static constexpr int STAGE = ((Q_OFF + Q_BYTES) + 1023) / 1024 * 1024;
-    static constexpr int NV = (G16 ? 2 : 1) * (D / 16) * 4 + (G16 ? 4 : 2);   // floats per lane
+    static constexpr int NV = (G16 ? 2 : 1) * (D / 16) * 4;        // o floats per lane
     static constexpr int MERGE_BYTES = NW * NV * 32 * 4;
     static constexpr int LENS_BYTES = 2 * (kMaxB + 1) * 4;          // lengths, prefix sums
     static constexpr int MISC_BYTES = 2048;                         // barriers, maxima, flags
@@ -221,11 +221,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t bar_full = sbase + Lay::MISC_OFF;
     const uint32_t bar_empty = bar_full + NST * 8;
-    // per-warp head maxima of a segment, double-buffered: a warp that has
-    // finished one segment's merge may write the next one's while slower warps
-    // still read the previous buffer (two merges apart, barrier 1 orders them)
-    float* mrg_m0 = reinterpret_cast<float*>(smem + Lay::MISC_OFF + 2 * NST * 8);  // [2][NW][16]
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_m0 + 2 * NW * 16);
+    // per-warp head maxima and sums of a segment (read only between the two
+    // merge barriers, so the next segment's writes cannot overtake a reader)
+    float* mrg_m = reinterpret_cast<float*>(smem + Lay::MISC_OFF + 2 * NST * 8);  // [NW][16]
+    float* mrg_l = mrg_m + NW * 16;                                               // [NW][16]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_l + NW * 16);
     float* mslot = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);               // [NW][NV][32]
     int* lens = reinterpret_cast<int*>(smem + Lay::LENS_OFF);                     // [B]
     int* cum = lens + (kMaxB + 1);                                               // [B + 1]
@@ -383,7 +383,6 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     int c_count = 0;                    // tiles consumed (ring position)
     bool open = false;                  // a segment's state is live
     int seg_j0 = 0;                     // first chunk of the open segment
-    int merges = 0;                     // segments merged so far (selects the maxima buffer)
 
     for (int64_t i = ibeg; i < iend; ++i) {
         const Item itm = item_at(i, lens, cum, B, p.Hk, p.chunk);
@@ -685,16 +684,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         open = false;
 
         // ---- merge the eight warps' states of the segment (one round)
-        float* mrg_m = mrg_m0 + (merges++ & 1) * NW * 16;
-        {
-            const float down = ldexpf(1.f, -kv);         // undo the P'' prescale
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) o[mt][nt][e] *= down;
-        }
+        // a segment that is the whole sequence writes the final rows (and,
+        // when the sequence has several chunks, a marker l = -1 in slot 0 that
+        // tells the combine kernel to leave them alone)
+        const bool final_rows = itm.ns == 1 || (seg_j0 == 0 && itm.j == itm.ns - 1);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -702,86 +695,77 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 4);
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 8);
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 16);
-                if (g == 0) mrg_m[warp * 16 + 8 * nt + 2 * t + c] = m[nt][c];
+                if (g == 0) {
+                    mrg_m[warp * 16 + 8 * nt + 2 * t + c] = m[nt][c];
+                    mrg_l[warp * 16 + 8 * nt + 2 * t + c] = l[nt][c];
+                }
             }
         ptx::named_bar_sync(1, NCONS);
+        // per head of this thread: segment max M, segment sum Ls, and the factor
+        // for this warp's o (2^(m - M) undoing the P'' prescale, divided by Ls
+        // when the rows are final)
+        float fo[NT][2];
         {
-            float* slot = mslot + warp * NV * 32 + lane;
-            int v = 0;
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int h = 8 * nt + 2 * t + (e & 1);
-                        float M = -INFINITY;
-#pragma unroll
-                        for (int w = 0; w < NW; ++w) M = fmaxf(M, mrg_m[w * 16 + h]);
-                        const float mv = m[nt][e & 1];
-                        const float f = (mv == -INFINITY) ? 0.f : ptx::ex2(mv - M);
-                        slot[(v++) * 32] = o[mt][nt][e] * f;
-                    }
+            const float down = ldexpf(1.f, -kv);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const int h = 8 * nt + 2 * t + c;
+                    float mw[NW];
                     float M = -INFINITY;
 #pragma unroll
-                    for (int w = 0; w < NW; ++w) M = fmaxf(M, mrg_m[w * 16 + h]);
-                    const float f = (m[nt][c] == -INFINITY) ? 0.f : ptx::ex2(m[nt][c] - M);
-                    slot[(v++) * 32] = l[nt][c] * f;
+                    for (int w = 0; w < NW; ++w) {
+                        mw[w] = mrg_m[w * 16 + h];
+                        M = fmaxf(M, mw[w]);
+                    }
+                    float Ls = 0.f;
+#pragma unroll
+                    for (int w = 0; w < NW; ++w)
+                        if (mw[w] != -INFINITY) Ls = fmaf(mrg_l[w * 16 + h], ptx::ex2(mw[w] - M), Ls);
+                    const float f = (m[nt][c] == -INFINITY) ? 0.f : ptx::ex2(m[nt][c] - M) * down;
+                    fo[nt][c] = final_rows ? (Ls > 0.f ? f / Ls : 0.f) : f;
+                    if (warp == 0 && g == 0 && itm.ns > 1 && h < G) {
+                        const int64_t row = bh0 + h;
+                        if (final_rows) {
+                            p.ws_l[row * p.splits] = -1.f;
+                        } else {
+                            p.ws_m[row * p.splits + seg_j0] = M;
+                            p.ws_l[row * p.splits + seg_j0] = Ls;
+                            for (int jj = seg_j0 + 1; jj <= itm.j; ++jj) {   // merged into seg_j0
+                                p.ws_m[row * p.splits + jj] = -INFINITY;
+                                p.ws_l[row * p.splits + jj] = 0.f;
+                            }
+                        }
+                    }
                 }
         }
+        {
+            float* slot = mslot + warp * NV * 32 + lane;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        slot[((mt * NT + nt) * 4 + e) * 32] = o[mt][nt][e] * fo[nt][e & 1];
+        }
         ptx::named_bar_sync(1, NCONS);
-        // sum the eight slots position by position and write the rows; a
-        // segment that is the whole sequence writes the final rows (and, when
-        // the sequence has several chunks, a marker l = -1 in slot 0 that tells
-        // the combine kernel to leave them alone)
-        const bool final_rows = itm.ns == 1 || (seg_j0 == 0 && itm.j == itm.ns - 1);
+        // sum the eight slots position by position and write the rows
         for (int pos = tid; pos < NV * 32; pos += NCONS) {
             const int v = pos >> 5, ln = pos & 31;
             const int pg_ = ln >> 2, pt = ln & 3;
+            const int mt = v / (NT * 4), nt = (v / 4) % NT, e = v & 3;
+            const int h = 8 * nt + 2 * pt + (e & 1);
+            if (h >= G) continue;
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < NW; ++w) sum += mslot[(w * NV + v) * 32 + ln];
-            if (v < MT * NT * 4) {
-                const int mt = v / (NT * 4), nt = (v / 4) % NT, e = v & 3;
-                const int h = 8 * nt + 2 * pt + (e & 1);
-                if (h >= G) continue;
-                const int d = G32 ? 32 * (mt >> 1) + 4 * pg_ + 2 * (mt & 1) + (e >> 1)
-                                  : (D == 128 ? 16 : 8) * pg_ + 2 * mt + (e >> 1);
-                const int64_t row = bh0 + h;
-                if (final_rows) {
-                    // the head's sum l sits at position (MT*NT*4 + 2*nt + c, lane pt)
-                    const int vl = MT * NT * 4 + 2 * nt + (e & 1);
-                    float lsum = 0.f;
-#pragma unroll
-                    for (int w = 0; w < NW; ++w) lsum += mslot[(w * NV + vl) * 32 + pt];
-                    p.out[row * D + d] = lsum > 0.f ? sum / lsum : 0.f;
-                } else {
-                    p.ws_o[(row * p.splits + seg_j0) * D + d] = sum;
-                }
-            } else if (pg_ == 0 && (!final_rows || itm.ns > 1)) {
-                const int k = v - MT * NT * 4, nt = k >> 1, c = k & 1;
-                const int h = 8 * nt + 2 * pt + c;
-                if (h >= G) continue;
-                if (final_rows) {
-                    p.ws_l[(bh0 + h) * p.splits] = -1.f;
-                    continue;
-                }
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < NW; ++w) M = fmaxf(M, mrg_m[w * 16 + h]);
-                const int64_t row = bh0 + h;
-                p.ws_m[row * p.splits + seg_j0] = M;
-                p.ws_l[row * p.splits + seg_j0] = sum;
-                for (int jj = seg_j0 + 1; jj <= itm.j; ++jj) {     // chunks merged into seg_j0
-                    p.ws_m[row * p.splits + jj] = -INFINITY;
-                    p.ws_l[row * p.splits + jj] = 0.f;
-                }
-            }
+            const int d = G32 ? 32 * (mt >> 1) + 4 * pg_ + 2 * (mt & 1) + (e >> 1)
+                              : (D == 128 ? 16 : 8) * pg_ + 2 * mt + (e >> 1);
+            const int64_t row = bh0 + h;
+            if (final_rows) p.out[row * D + d] = sum;
+            else p.ws_o[(row * p.splits + seg_j0) * D + d] = sum;
         }
     }
 }
