@@ -13,23 +13,23 @@
 // How (sm_100a):
 //  * Work items are (sequence b, kv head, chunk j) with chunk = p.chunk
 //    tokens, listed in (b, kv head, j) order.  The grid is persistent (at
-//    most one CTA per SM) and CTA c takes the contiguous block
-//    [c*T/grid, (c+1)*T/grid) of the T items, found from a prefix sum of the
-//    per-sequence chunk counts (sequence lengths cached in shared memory).
-//    Consecutive chunks of one (b, kv head) inside a CTA's block form a
-//    segment and share one softmax state; a segment that is a whole
-//    sequence writes the final rows, any other writes one partial state
-//    (o, m, l) into the slot of its first chunk and marks the slots of its
-//    other chunks empty for the combine kernel (kvq_decode.cu).
-//  * CTA = 8 consumer warps + 1 producer warp.  The producer streams
-//    128-token stages into a ring of 3-8 stages (~150-180 KB of shared
-//    memory, one CTA per SM): K and V bytes by TMA tile loads (2-D tensor
-//    maps over the cache rows, 128-byte swizzle for D=128, 64-byte for
-//    D=64), the fp32 scales and, with a segment's first stage, its query
-//    rows by cp.async; all complete on the stage's mbarrier.  It refills a
-//    slot as soon as all consumers released it, independent of their
-//    progress elsewhere.  Every consumer warp takes one 16-token slice of
-//    each stage.
+//    most one CTA per SM) and CTA c takes a contiguous block of the T items
+//    (T / grid each, the first T % grid CTAs one more), found from a prefix
+//    sum of the per-sequence chunk counts (lengths cached in shared memory).
+//    The items of one (b, kv head) inside a CTA's block form a segment: one
+//    token range, one softmax state.  A segment that is a whole sequence
+//    writes the final rows, any other writes one partial state (o, m, l)
+//    into the slot of its first chunk and marks the slots of its other
+//    chunks empty for the combine kernel (kvq_decode.cu).
+//  * CTA = 1 producer warp (warp 0) + 8 consumer warps.  One producer lane
+//    streams 128-token stages into a ring of 3-8 stages (~150-220 KB of
+//    shared memory, one CTA per SM): K and V bytes by TMA tile loads (2-D
+//    tensor maps over the cache rows, 128-byte swizzle for D=128, 64-byte
+//    for D=64), the fp32 scales and, with a segment's first two stages, its
+//    query rows by 1-D bulk copies; all complete on the stage's mbarrier.
+//    It refills a slot as soon as its consumers released it.  The consumers
+//    form two groups of four warps that take alternate stages; a warp takes
+//    32 tokens of its group's stage as two 16-token MMA tiles.
 //  * Per slice, on mma.sync m16n8k16 (f16 in, f32 accumulate), with the
 //    query heads of the GQA group as the N = 8 dimension (two n-tiles when
 //    G > 8):  S^T = K . Q^T (M = 16 tokens, K = head_dim) and
@@ -47,7 +47,7 @@
 //    significant bits together); each part is transposed from the score
 //    accumulator layout into the P^T operand layout with movmatrix and
 //    multiplied with the exact (v - 128) integers.
-//  * Token order inside each 16-token slice and the head_dim order of the
+//  * Token order inside each 16-token MMA tile and the head_dim order of the
 //    MMA k-dimension are permuted so that every shared-memory load of the
 //    swizzled tiles is free of bank conflicts (sigma below).
 //  * A segment's eight warp states are merged in one round through eight
@@ -70,7 +70,8 @@ namespace {
 constexpr int NW = 8;                  // consumer warps per CTA
 constexpr int NCONS = NW * 32;         // consumer threads
 constexpr int NTHREADS = NCONS + 32;   // + the producer warp
-constexpr int TT = 16 * NW;            // tokens per stage: one 16-token slice per warp
+constexpr int WPG = 4;                 // consumer warps per group (a group works one stage)
+constexpr int TT = 32 * WPG;           // tokens per stage: one 32-token slice per warp of a group
 constexpr int kMaxB = 1024;            // sequences whose lengths are cached in shared memory
 
 // Row (inside an 8-token half of a slice) that holds MMA row r of the K
@@ -99,16 +100,6 @@ __device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
     return y;
 }
 
-// The NG fp32 scales of one token (4, 8 or 16 bytes, aligned to their size
-// because the scale array is 16-byte aligned and rows are NG floats apart).
-template <int NG>
-__device__ __forceinline__ void copy_scales(uint32_t dst, const float* src) {
-    static_assert(NG == 1 || NG == 2 || NG == 4, "scales per token");
-    if constexpr (NG == 1) ptx::cp_async_4(dst, src);
-    else if constexpr (NG == 2) ptx::cp_async_8(dst, src);
-    else ptx::cp_async_16(dst, src);
-}
-
 // Shared-memory plan (one CTA per SM): a ring of NST stages (K and V bytes of
 // 128 tokens, their scales, room for one segment's query rows), the merge
 // slots, the cached lengths and chunk prefix sums, the stage mbarriers and
@@ -117,20 +108,24 @@ template <int D, bool G32, bool G16>
 struct Layout {
     static constexpr int NG = G32 ? D / 32 : 1;
     static constexpr int KV_BYTES = TT * D;
-    static constexpr int SC_FLOATS = TT * NG;
+    static constexpr int SC_FLOATS = TT * NG + 4;   // + room for a 16-byte alignment offset
     static constexpr int Q_OFF = 2 * KV_BYTES + 2 * SC_FLOATS * 4;   // within a stage
     static constexpr int Q_BYTES = (G16 ? 16 : 8) * D * 2;           // bf16 query rows
-    static constexpr int STAGE = ((Q_OFF + Q_BYTES) + 1023) / 1024 * 1024;
+    static constexpr int MASK_OFF = Q_OFF + Q_BYTES;                 // paged: valid-page bits
+    static constexpr int STAGE = ((MASK_OFF + 16) + 1023) / 1024 * 1024;
     static constexpr int NV = (G16 ? 2 : 1) * (D / 16) * 4;        // o floats per lane
     static constexpr int MERGE_BYTES = NW * NV * 32 * 4;
-    static constexpr int LENS_BYTES = 2 * (kMaxB + 1) * 4;          // lengths, prefix sums
-    static constexpr int MISC_BYTES = 2048;                         // barriers, maxima, flags
-    static constexpr int BUDGET = 227 * 1024 - 1024 - MERGE_BYTES - LENS_BYTES - MISC_BYTES;
+    static constexpr int LENS_BYTES = (3 * kMaxB + 1) * 4;          // lengths, chunks, prefix sums
+    static constexpr int PARAM_BYTES = 256;                         // the kernel parameters
+    static constexpr int MISC_BYTES = 1536;                         // barriers, maxima, flags
+    static constexpr int BUDGET =
+        227 * 1024 - 1024 - MERGE_BYTES - LENS_BYTES - PARAM_BYTES - MISC_BYTES;
     static constexpr int NST = (BUDGET / STAGE) > 8 ? 8 : (BUDGET / STAGE);
     static_assert(NST >= 3, "at least three stages");
     static constexpr int MERGE_OFF = NST * STAGE;
     static constexpr int LENS_OFF = MERGE_OFF + MERGE_BYTES;
-    static constexpr int MISC_OFF = LENS_OFF + LENS_BYTES;
+    static constexpr int PARAM_OFF = (LENS_OFF + LENS_BYTES + 15) / 16 * 16;
+    static constexpr int MISC_OFF = PARAM_OFF + PARAM_BYTES;
     static constexpr int SMEM = MISC_OFF + MISC_BYTES + 1024;       // + base alignment slack
     static_assert(SMEM <= 227 * 1024, "fits one SM");
 };
@@ -161,43 +156,57 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
     return v;
 }
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
 __device__ __forceinline__ float ldsf(uint32_t a) {
     float v;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
     return v;
 }
 
-// One work item of a CTA's block: item index -> (b, kv head, chunk j).
-struct Item {
-    int b, hk, j, ns, L, t0, t1;   // ns = chunks of the sequence (0: empty sequence)
+// The run of work items of one (sequence, kv head) that starts at item i and
+// stays inside [i, iend): chunks j0..j1 of sequence b, kv head hk, i.e.
+// tokens [t0, t1).  Items are listed in (b, kv head, chunk) order and
+// cum[b] counts the items of sequences before b (Hk * max(1, ns) each).
+// 2^e for -126 <= e <= 127, exact.
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+
+struct Seg {
+    int b, hk, ns, j0, j1, t0, t1;
+    int next;                      // first item after the run
 };
 
-// cum[b] = items of sequences < b (each sequence has Hk * max(1, ns_b) items)
-__device__ __forceinline__ Item item_at(int64_t i, const int* lens, const int* cum, int B,
-                                        int Hk, int chunk) {
-    int lo = 0, hi = B;                  // largest b with cum[b] <= i
+__device__ __forceinline__ Seg seg_at(int i, int iend, const int* lens, const int* nsv,
+                                      const int* cum, int B, int chunk) {
+    int lo = 0, hi = B;            // largest b with cum[b] <= i
+#pragma unroll 1
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (cum[mid] <= i) lo = mid;
         else hi = mid;
     }
-    Item it;
-    it.b = lo;
-    it.L = lens[lo];
-    it.ns = (it.L + chunk - 1) / chunk;
-    const int per = it.ns > 0 ? it.ns : 1;
-    const int r = static_cast<int>(i - cum[lo]);
-    it.hk = r / per;
-    it.j = r - it.hk * per;
-    it.t0 = it.j * chunk;
-    it.t1 = it.ns > 0 ? min(it.t0 + chunk, it.L) : 0;
-    return it;
+    Seg sg;
+    sg.b = lo;
+    sg.ns = nsv[lo];
+    const int per = sg.ns > 0 ? sg.ns : 1;
+    const int r = i - cum[lo];
+    sg.hk = r / per;
+    sg.j0 = r - sg.hk * per;
+    sg.next = min(iend, cum[lo] + (sg.hk + 1) * per);
+    sg.j1 = sg.j0 + (sg.next - i) - 1;
+    sg.t0 = sg.j0 * chunk;
+    sg.t1 = sg.ns > 0 ? min((sg.j1 + 1) * chunk, lens[lo]) : 0;
+    return sg;
 }
 
 template <int D, bool G32, bool PAGED, bool G16>
 __global__ void __launch_bounds__(NTHREADS, 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                DecodeParams p) {
+                const __grid_constant__ DecodeParams prm) {
     using Lay = Layout<D, G32, G16>;
     constexpr int NG = Lay::NG;
     constexpr int NST = Lay::NST;
@@ -216,7 +225,6 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tid = threadIdx.x;
     const int g = lane >> 2, t = lane & 3;
-    const int G = p.G;
 
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t bar_full = sbase + Lay::MISC_OFF;
@@ -225,17 +233,31 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     // merge barriers, so the next segment's writes cannot overtake a reader)
     float* mrg_m = reinterpret_cast<float*>(smem + Lay::MISC_OFF + 2 * NST * 8);  // [NW][16]
     float* mrg_l = mrg_m + NW * 16;                                               // [NW][16]
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_l + NW * 16);
+    float* seg_M = mrg_l + NW * 16;     // [16] a segment's per-head max and sum, for the
+    float* seg_L = seg_M + 16;          // [16] partial-state writes after the merge
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(seg_L + 16);
+    static_assert(2 * NST * 8 + (2 * NW * 16 + 32) * 4 + 4 <= Lay::MISC_BYTES,
+                  "barriers, maxima, flag");
     float* mslot = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);               // [NW][NV][32]
     int* lens = reinterpret_cast<int*>(smem + Lay::LENS_OFF);                     // [B]
-    int* cum = lens + (kMaxB + 1);                                               // [B + 1]
+    int* nsv = lens + kMaxB;                                                     // [B] chunks
+    int* cum = nsv + kMaxB;                                                      // [B + 1]
+    DecodeParams* sprm = reinterpret_cast<DecodeParams*>(smem + Lay::PARAM_OFF);
 
+    // the parameters are copied to shared memory in one parallel round of
+    // parameter-space reads (their latency overlaps the dependency wait);
+    // every later use is a shared-memory load
+    static_assert(sizeof(DecodeParams) % 4 == 0 && sizeof(DecodeParams) <= Lay::PARAM_BYTES,
+                  "the parameters fit their shared-memory copy");
+    if (tid < static_cast<int>(sizeof(DecodeParams) / 4))
+        reinterpret_cast<uint32_t*>(sprm)[tid] = reinterpret_cast<const uint32_t*>(&prm)[tid];
     if (tid == 0) {
         ptx::prefetch_tensormap(&tm_k);     // kernel parameters: safe before the dependency wait
         ptx::prefetch_tensormap(&tm_v);
+#pragma unroll 1
         for (int s = 0; s < NST; ++s) {
-            ptx::mbar_init(bar_full + 8 * s, 1 + 32);   // expect_tx arrive + 32 cp.async arrivals
-            ptx::mbar_init(bar_empty + 8 * s, NW);
+            ptx::mbar_init(bar_full + 8 * s, 1);        // the producer's expect_tx arrival
+            ptx::mbar_init(bar_empty + 8 * s, WPG);
         }
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -244,22 +266,29 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     grid_dep_launch();                  // the combine kernel may be scheduled now
 
     // ---- lengths and chunk prefix sums (items per sequence: Hk * max(1, chunks))
-    const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
-    const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
-    const int B = p.B;
-    for (int b = tid; b < B; b += NTHREADS) {
-        int L = p.seq_lens[b];
-        if (L < 0 || L > lim) {
-            if (blockIdx.x == 0) raise_flag(p.d_err, KVQ_DEVERR_LEN);
-            L = 0;
+    {
+        const int64_t cap = PAGED ? static_cast<int64_t>(prm.max_pages) * prm.page_size : prm.max_seq;
+        const int64_t lim = min(cap, static_cast<int64_t>(prm.splits) * prm.chunk);
+#pragma unroll 1
+        for (int b = tid; b < prm.B; b += NTHREADS) {
+            int L = prm.seq_lens[b];
+            if (L < 0 || L > lim) {
+                if (blockIdx.x == 0) raise_flag(prm.d_err, KVQ_DEVERR_LEN);
+                L = 0;
+            }
+            lens[b] = L;
+            const int ns = (L + prm.chunk - 1) / prm.chunk;
+            nsv[b] = ns;
+            cum[b + 1] = prm.Hk * (ns > 0 ? ns : 1);
         }
-        lens[b] = L;
-        const int ns = (L + p.chunk - 1) / p.chunk;
-        cum[b + 1] = p.Hk * (ns > 0 ? ns : 1);
     }
     __syncthreads();
+    const DecodeParams& p = *sprm;
+    const int B = p.B;
+    const int G = p.G;
     if (warp == 0) {                    // inclusive scan of cum[1..B] by one warp
         int carry = 0;
+#pragma unroll 1
         for (int base = 0; base < B; base += 32) {
             int v = base + lane < B ? cum[base + lane + 1] : 0;
 #pragma unroll
@@ -273,9 +302,13 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (lane == 0) cum[0] = 0;
     }
     __syncthreads();
-    const int64_t T = cum[B];
-    const int64_t ibeg = T * blockIdx.x / gridDim.x;
-    const int64_t iend = T * (blockIdx.x + 1) / gridDim.x;
+    // CTA c takes items [c*q + min(c, r), ...) with q = T / grid, r = T % grid
+    // (the first r CTAs one item more); T < 2^31 is checked by the host
+    const int T = cum[B];
+    const int ibeg = static_cast<int>(blockIdx.x) * (T / static_cast<int>(gridDim.x)) +
+                     min(static_cast<int>(blockIdx.x), T % static_cast<int>(gridDim.x));
+    const int iend = ibeg + T / static_cast<int>(gridDim.x) +
+                     (static_cast<int>(blockIdx.x) < T % static_cast<int>(gridDim.x) ? 1 : 0);
 
     // bounded wait that gives up at once after any earlier timeout of this CTA
     auto wait = [&](uint32_t bar, uint32_t parity) {
@@ -287,139 +320,190 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     };
 
     // ------------------------------------------------------------ producer
-    if (warp == NW) {
+    if (warp == 0) {
+        // one lane issues every copy of a stage (TMA tiles for K and V, 1-D bulk
+        // copies for the scales and the query rows); all complete on the stage's
+        // mbarrier, whose single arrival is the expect_tx below
         const uint64_t pol = ptx::policy_evict_first();
+        // the parameters this loop uses live in registers: the asm statements
+        // below clobber memory, so reads through p would be repeated after each
+        // of them (shared-memory loads queued behind the consumers' traffic)
+        const int Hk = p.Hk, Hq = p.Hq, chunk = p.chunk, max_seq = p.max_seq;
+        const int max_pages = p.max_pages, num_pages = p.num_pages;
+        const float* const k_scale = p.k_scale;
+        const float* const v_scale = p.v_scale;
+        const uint16_t* const qg = p.q;
+        const int32_t* const table = p.table;
+        int32_t* const d_err = p.d_err;
+        // floats in each scale array (contiguous layout)
+        const int64_t sc_total = static_cast<int64_t>(B) * Hk * max_seq * NG;
+        const uint32_t q_bytes = static_cast<uint32_t>(G * D * 2);
         int count = 0;                  // tiles issued (ring position)
-        int pb = -1, phk = -1;
-        for (int64_t i = ibeg; i < iend; ++i) {
-            const Item itm = item_at(i, lens, cum, B, p.Hk, p.chunk);
-            if (itm.ns == 0) continue;
-            const bool seg_first = itm.b != pb || itm.hk != phk;
-            pb = itm.b;
-            phk = itm.hk;
-            const int b = itm.b, hk = itm.hk;
-            for (int tt0 = itm.t0; tt0 < itm.t1; tt0 += TT, ++count) {
+#pragma unroll 1
+        for (int i = ibeg; i < iend;) {
+            const Seg sg = seg_at(i, iend, lens, nsv, cum, B, chunk);
+            i = sg.next;
+            if (sg.ns == 0) continue;
+            const int b = sg.b, hk = sg.hk;
+            const uint16_t* qsrc = qg + (static_cast<int64_t>(b) * Hq + hk * G) * D;
+            int seg_tiles = 0;          // tiles issued for this segment
+#pragma unroll 1
+            for (int tt0 = sg.t0; tt0 < sg.t1; tt0 += TT, ++count, ++seg_tiles) {
                 const int s = count % NST;
                 const uint32_t full = bar_full + 8 * s;
-                if (count >= NST) wait(bar_empty + 8 * s, ((count / NST) - 1) & 1);
-                const int ntok = min(TT, itm.t1 - tt0);
+                if (count >= NST && lane == 0) wait(bar_empty + 8 * s, ((count / NST) - 1) & 1);
+                __syncwarp();
+                const int ntok = min(TT, sg.t1 - tt0);
                 const uint32_t sk = sbase + s * Lay::STAGE;
                 const uint32_t sv = sk + Lay::KV_BYTES;
                 const uint32_t sks = sv + Lay::KV_BYTES;
                 const uint32_t svs = sks + Lay::SC_FLOATS * 4;
+                // the segment's G query rows (contiguous bf16) ride with its first
+                // two stages: each consumer group builds its Q operand from the
+                // first stage it works in the segment
+                const bool with_q = seg_tiles < 2;
                 if (!PAGED) {
-                    const int64_t row0 = (static_cast<int64_t>(b) * p.Hk + hk) * p.max_seq + tt0;
                     if (lane == 0) {
-                        ptx::mbar_arrive_expect_tx(full, 2 * Lay::KV_BYTES);
+                        const int64_t row0 = (static_cast<int64_t>(b) * Hk + hk) * max_seq + tt0;
+                        // scales: whole 16-byte chunks from the aligned float at or
+                        // below the tile's first one; where the last chunk would run
+                        // past the end of the scale array its 1-3 floats are copied
+                        // by plain loads (before the arrival that publishes them)
+                        const int64_t f0 = row0 * NG;
+                        const int off = static_cast<int>(f0 & 3);
+                        const int64_t c0 = f0 - off;
+                        const int nf = ntok * NG + off;
+                        int nb = (nf + 3) & ~3;
+                        if (c0 + nb > sc_total) {
+                            nb = nf & ~3;
+#pragma unroll 1
+                            for (int e = nb; e < nf; ++e) {
+                                sts_f32(sks + 4 * e, k_scale[c0 + e]);
+                                sts_f32(svs + 4 * e, v_scale[c0 + e]);
+                            }
+                        }
+                        ptx::mbar_arrive_expect_tx(
+                            full, 2 * Lay::KV_BYTES + 8 * nb + (with_q ? q_bytes : 0u));
                         ptx::tma_load_2d(sk, &tm_k, 0, static_cast<int>(row0), full, pol);
                         ptx::tma_load_2d(sv, &tm_v, 0, static_cast<int>(row0), full, pol);
-                    }
-                    for (int k = lane; k < ntok; k += 32) {
-                        const int64_t r = row0 + k;
-                        copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
-                        copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
+                        if (nb > 0) {
+                            ptx::bulk_load(sks, k_scale + c0, 4 * nb, full);
+                            ptx::bulk_load(svs, v_scale + c0, 4 * nb, full);
+                        }
+                        if (with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
                     }
                 } else {
                     constexpr int PPS = TT / 16;                // pages per stage
+                    constexpr uint32_t PAGE_BYTES = 2 * 16 * D + 2 * 64 * NG;
                     const int np = (ntok + 15) >> 4;
                     int32_t pg = -1;
                     if (lane < np) {
-                        // a bad entry is skipped here and reported by the consumers
-                        pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tt0 >> 4) + lane];
-                        if (pg < 0 || pg >= p.num_pages) pg = -1;
+                        // a bad entry is skipped (its tokens are masked)
+                        pg = table[static_cast<int64_t>(b) * max_pages + (tt0 >> 4) + lane];
+                        if (pg < 0 || pg >= num_pages) pg = -1;
                     }
                     const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
-                    if (lane == 0) ptx::mbar_arrive_expect_tx(full, __popc(valid) * 2 * 16 * D);
+                    if (lane == 0) {
+                        // the consumers mask the tokens of pages that were not
+                        // loaded; a bad table entry is reported here
+                        if (valid != (1u << np) - 1u) raise_flag(d_err, KVQ_DEVERR_PAGE);
+                        sts_u32(sk + Lay::MASK_OFF, valid);
+                        ptx::mbar_arrive_expect_tx(
+                            full, __popc(valid) * PAGE_BYTES + (with_q ? q_bytes : 0u));
+                    }
 #pragma unroll
                     for (int q = 0; q < PPS; ++q) {
                         const int pq = __shfl_sync(0xffffffffu, pg, q);
                         if (lane == 0 && pq >= 0) {
-                            const int y = (pq * p.Hk + hk) * 16;
+                            // a page holds 16 rows of this kv head; its scales are
+                            // 16 * NG aligned floats
+                            const int y = (pq * Hk + hk) * 16;
                             ptx::tma_load_2d(sk + q * 16 * D, &tm_k, 0, y, full, pol);
                             ptx::tma_load_2d(sv + q * 16 * D, &tm_v, 0, y, full, pol);
+                            const int64_t fc = static_cast<int64_t>(y) * NG;
+                            ptx::bulk_load(sks + q * 64 * NG, k_scale + fc, 64 * NG, full);
+                            ptx::bulk_load(svs + q * 64 * NG, v_scale + fc, 64 * NG, full);
                         }
                     }
-                    for (int k = lane; k < TT; k += 32) {
-                        const int pk = __shfl_sync(0xffffffffu, pg, k >> 4);
-                        if (k < ntok && pk >= 0) {
-                            const int64_t r = (static_cast<int64_t>(pk) * p.Hk + hk) * 16 + (k & 15);
-                            copy_scales<NG>(sks + k * NG * 4, p.k_scale + r * NG);
-                            copy_scales<NG>(svs + k * NG * 4, p.v_scale + r * NG);
-                        }
-                    }
+                    if (lane == 0 && with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
                 }
-                if (seg_first && tt0 == itm.t0) {
-                    // the segment's G query rows (contiguous bf16) ride with its first stage
-                    const uint16_t* qsrc = p.q + (static_cast<int64_t>(b) * p.Hq + hk * G) * D;
-                    const uint32_t sq = sk + Lay::Q_OFF;
-                    for (int c = lane; c < G * D / 8; c += 32)
-                        ptx::cp_async_16(sq + c * 16, qsrc + c * 8);
-                }
-                ptx::cp_async_arrive_noinc(full);
             }
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
         // the last tile of every slot has landed (normally long consumed; after a
         // timeout this keeps the CTA alive until its bulk copies are done)
         if (lane == 0)
+#pragma unroll 1
             for (int c = count - 1; c >= 0 && c >= count - NST; --c)
                 ptx::mbar_wait(bar_full + 8 * (c % NST), (c / NST) & 1);
         return;                         // consumers synchronise among themselves (barrier 1)
     }
 
     // ------------------------------------------------------------ consumers
+    // Two groups of four warps take alternate stages (tile c of the CTA goes
+    // to group c % 2), so two stages are in work at once.  Inside a stage,
+    // warp wg of the group owns rows [32 wg, 32 wg + 32) as two 16-token MMA
+    // tiles u = 0, 1 that share one online-softmax step.
+    const int cw = warp - 1;            // consumer warp index
+    const int ctid = tid - 32;          // consumer thread index
+    const int grp = cw / WPG, wg = cw % WPG;
     const int sig_g = sigma(g);
     const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
-    const int rowA = 16 * warp + sig_g;           // MMA row g     of this warp's slice
-    const int rowB = rowA + 8;                    // MMA row g + 8
-    const int R0 = 16 * warp + sig_a, R1 = 16 * warp + sig_b;   // V rows of k 2t, 2t+1
-    const int R2 = R0 + 8, R3 = R1 + 8;                         // V rows of k 2t+8, 2t+9
 
     uint32_t qb0[NT][KS], qb1[NT][KS];
     float zs[NT][2];
     float m[NT][2], l[NT][2];
     float o[MT][NT][4];                 // O^T C fragments: rows = head_dim, columns = heads
     int kv = 64;                        // running P'' prescale exponent (per warp)
-    int c_count = 0;                    // tiles consumed (ring position)
-    bool open = false;                  // a segment's state is live
-    int seg_j0 = 0;                     // first chunk of the open segment
+    int c_count = 0;                    // tiles of the CTA seen so far (ring position)
 
-    for (int64_t i = ibeg; i < iend; ++i) {
-        const Item itm = item_at(i, lens, cum, B, p.Hk, p.chunk);
-        const int b = itm.b, hk = itm.hk;
+#pragma unroll 1
+    for (int i = ibeg; i < iend;) {
+        const Seg sg = seg_at(i, iend, lens, nsv, cum, B, p.chunk);
+        i = sg.next;
+        const int b = sg.b, hk = sg.hk;
         const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
-        if (itm.ns == 0) {
+        if (sg.ns == 0) {
             // empty (or rejected) sequence: zero rows
-            for (int idx = tid; idx < G * D; idx += NCONS) p.out[bh0 * D + idx] = 0.f;
+#pragma unroll 1
+            for (int idx = ctid; idx < G * D; idx += NCONS) p.out[bh0 * D + idx] = 0.f;
             continue;
         }
-        if (!open) {
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                m[nt][0] = m[nt][1] = -INFINITY;
-                l[nt][0] = l[nt][1] = 0.f;
+        for (int nt = 0; nt < NT; ++nt) {
+            m[nt][0] = m[nt][1] = -INFINITY;
+            l[nt][0] = l[nt][1] = 0.f;
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-                    o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
-            }
-            kv = 64;
-            seg_j0 = itm.j;
+            for (int mt = 0; mt < MT; ++mt)
+                o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
         }
-        const int t0 = itm.t0, t1 = itm.t1;
+        kv = 64;
+        bool have_q = false;            // Q fragments of this segment are built
+        // contiguous layout: the stage's scales start sc_off bytes in (the copies
+        // start at the 16-byte aligned float at or below the tile's first; tiles
+        // start at multiples of 16 tokens, so the offset is the segment's)
+        const uint32_t sc_off =
+            PAGED ? 0u
+                  : ((static_cast<uint32_t>(b * p.Hk + hk) * static_cast<uint32_t>(p.max_seq) *
+                      static_cast<uint32_t>(NG)) & 3u) * 4u;
+        const int t0 = sg.t0, t1 = sg.t1;
         const int ntiles = (t1 - t0 + TT - 1) / TT;
+#pragma unroll 1
         for (int it = 0; it < ntiles; ++it, ++c_count) {
+            if ((c_count & 1) != grp) continue;           // the other group's stage
             const int s = c_count % NST;
             wait(bar_full + 8 * s, (c_count / NST) & 1);
             const int tt0 = t0 + it * TT;
             const uint32_t sk = sbase + s * Lay::STAGE;
             const uint32_t sv = sk + Lay::KV_BYTES;
-            const uint32_t sks = sv + Lay::KV_BYTES;
-            const uint32_t svs = sks + Lay::SC_FLOATS * 4;
-            if (!open && it == 0) {
-                // ---- Q^T operand from the stage: column n = g of n-tile nt is query
-                // head 8*nt + g, pre-scaled by 2^sh so max |q| * 2^sh is in [2^14, 2^15).
-                // B fragment rows 2t, 2t+1 (qb0) and 2t+8, 2t+9 (qb1) of k-step
+            const uint32_t sks = sv + Lay::KV_BYTES + sc_off;
+            const uint32_t svs = sv + Lay::KV_BYTES + Lay::SC_FLOATS * 4 + sc_off;
+            if (!have_q) {
+                // ---- Q^T operand (the segment's query rows ride with its first
+                // two stages): column n = g of n-tile nt is query head 8*nt + g,
+                // pre-scaled by 2^sh so max |q| * 2^sh is in [2^14, 2^15).  B
+                // fragment rows 2t, 2t+1 (qb0) and 2t+8, 2t+9 (qb1) of k-step
                 // 2*gi + h2 hold head_dim 32*gi + 8*t + 4*h2 + {0, 1} and {2, 3}.
+                have_q = true;
                 const uint32_t sq = sk + Lay::Q_OFF;
                 float zsq[NT];
 #pragma unroll
@@ -447,8 +531,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
                         sh = min(max(14 - e, -100), 100);
                     }
-                    const float up = ldexpf(1.f, sh);
-                    zsq[nt] = ldexpf(1.f, -sh) * p.scale_log2;
+                    const float up = pow2i(sh);                  // |sh| <= 100
+                    zsq[nt] = pow2i(-sh) * p.scale_log2;
 #pragma unroll
                     for (int gi = 0; gi < NGRP; ++gi)
 #pragma unroll
@@ -466,228 +550,257 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     zs[nt][1] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t + 1));
                 }
             }
-            const int tok0 = tt0 + 16 * warp;             // first token of this warp's slice
+            const int tok0 = tt0 + 32 * wg;               // first token of this warp's slice
             if (tok0 < t1) {
-            bool page_ok = true;
-            if (PAGED) {
-                const int32_t pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tok0 >> 4)];
-                page_ok = pg >= 0 && pg < p.num_pages;
-                if (!page_ok && lane == 0) raise_flag(p.d_err, KVQ_DEVERR_PAGE);
-            }
-            const bool okA = page_ok && (tok0 + sig_g < t1);
-            const bool okB = page_ok && (tok0 + 8 + sig_g < t1);
+                // stage rows of MMA tile u: K rows g, g + 8; V rows of k 2t, 2t+1, 2t+8, 2t+9
+                int rA[2], rB[2], V0[2], V1[2];
+                bool okA[2], okB[2];
+                const uint32_t pmask = PAGED ? lds32(sk + Lay::MASK_OFF) : 0u;
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int base = 32 * wg + 16 * u;
+                    rA[u] = base + sig_g;
+                    rB[u] = rA[u] + 8;
+                    V0[u] = base + sig_a;
+                    V1[u] = base + sig_b;
+                    const int tk = tok0 + 16 * u;
+                    bool page_ok = tk < t1;
+                    // paged: page 2 wg + u of the stage was loaded (the producer
+                    // checked the table entry)
+                    if (PAGED) page_ok = page_ok && ((pmask >> (2 * wg + u)) & 1u);
+                    okA[u] = page_ok && (tk + sig_g < t1);
+                    okB[u] = page_ok && (tk + 8 + sig_g < t1);
+                }
 
-            // ---- S^T = K . Q^T: rows tokens (rowA, rowB), columns heads
-            float sacc[NT][NACC][4];
+                // ---- S^T = K . Q^T per MMA tile: rows tokens (rA, rB), columns heads
+                float sacc[2][NT][NACC][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int a = 0; a < NACC; ++a)
-                    sacc[nt][a][0] = sacc[nt][a][1] = sacc[nt][a][2] = sacc[nt][a][3] = 0.f;
-#pragma unroll
-            for (int gi = 0; gi < NGRP; ++gi) {
-                const uint2 wa = lds64(sk + swz<D>(rowA, 32 * gi + 8 * t));
-                const uint2 wb = lds64(sk + swz<D>(rowB, 32 * gi + 8 * t));
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const uint32_t xa = h2 ? wa.y : wa.x;
-                    const uint32_t xb = h2 ? wb.y : wb.x;
-                    const uint32_t a0 = ptx::bytes_to_f16x2(xa, 0x4140u);
-                    const uint32_t a2 = ptx::bytes_to_f16x2(xa, 0x4342u);
-                    const uint32_t a1 = ptx::bytes_to_f16x2(xb, 0x4140u);
-                    const uint32_t a3 = ptx::bytes_to_f16x2(xb, 0x4342u);
+                for (int u = 0; u < 2; ++u)
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
-                        ptx::mma_f16(sacc[nt][G32 ? gi : (gi & 1)], a0, a1, a2, a3,
-                                     qb0[nt][2 * gi + h2], qb1[nt][2 * gi + h2]);
-                }
-            }
-            // ---- scores z (log2 domain): [nt][0..1] token rowA, [nt][2..3] token rowB
-            float z[NT][4];
-            if (G32) {
-                float ksa[NG], ksb[NG];
 #pragma unroll
-                for (int a = 0; a < NG; ++a) {
-                    ksa[a] = ldsf(sks + (rowA * NG + a) * 4);
-                    ksb[a] = ldsf(sks + (rowB * NG + a) * 4);
-                }
+                        for (int a = 0; a < NACC; ++a)
+                            sacc[u][nt][a][0] = sacc[u][nt][a][1] = sacc[u][nt][a][2] =
+                                sacc[u][nt][a][3] = 0.f;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    float za0 = 0.f, za1 = 0.f, zb0 = 0.f, zb1 = 0.f;
+                for (int gi = 0; gi < NGRP; ++gi)
 #pragma unroll
-                    for (int a = 0; a < NACC; ++a) {
-                        za0 = fmaf(sacc[nt][a][0], ksa[a], za0);
-                        za1 = fmaf(sacc[nt][a][1], ksa[a], za1);
-                        zb0 = fmaf(sacc[nt][a][2], ksb[a], zb0);
-                        zb1 = fmaf(sacc[nt][a][3], ksb[a], zb1);
+                    for (int u = 0; u < 2; ++u) {
+                        const uint2 wa = lds64(sk + swz<D>(rA[u], 32 * gi + 8 * t));
+                        const uint2 wb = lds64(sk + swz<D>(rB[u], 32 * gi + 8 * t));
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            const uint32_t xa = h2 ? wa.y : wa.x;
+                            const uint32_t xb = h2 ? wb.y : wb.x;
+                            const uint32_t a0 = ptx::bytes_to_f16x2(xa, 0x4140u);
+                            const uint32_t a2 = ptx::bytes_to_f16x2(xa, 0x4342u);
+                            const uint32_t a1 = ptx::bytes_to_f16x2(xb, 0x4140u);
+                            const uint32_t a3 = ptx::bytes_to_f16x2(xb, 0x4342u);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+                                ptx::mma_f16(sacc[u][nt][G32 ? gi : (gi & 1)], a0, a1, a2, a3,
+                                             qb0[nt][2 * gi + h2], qb1[nt][2 * gi + h2]);
+                        }
                     }
-                    z[nt][0] = okA ? za0 * zs[nt][0] : -INFINITY;
-                    z[nt][1] = okA ? za1 * zs[nt][1] : -INFINITY;
-                    z[nt][2] = okB ? zb0 * zs[nt][0] : -INFINITY;
-                    z[nt][3] = okB ? zb1 * zs[nt][1] : -INFINITY;
-                }
-            } else {
-                const float ksa = ldsf(sks + rowA * 4), ksb = ldsf(sks + rowB * 4);
+                // ---- scores z (log2 domain): [u][nt][0..1] token rA[u], [u][nt][2..3] token rB[u]
+                float z[2][NT][4];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const float s0 = sacc[nt][0][0] + sacc[nt][1][0];
-                    const float s1 = sacc[nt][0][1] + sacc[nt][1][1];
-                    const float s2 = sacc[nt][0][2] + sacc[nt][1][2];
-                    const float s3 = sacc[nt][0][3] + sacc[nt][1][3];
-                    z[nt][0] = okA ? s0 * ksa * zs[nt][0] : -INFINITY;
-                    z[nt][1] = okA ? s1 * ksa * zs[nt][1] : -INFINITY;
-                    z[nt][2] = okB ? s2 * ksb * zs[nt][0] : -INFINITY;
-                    z[nt][3] = okB ? s3 * ksb * zs[nt][1] : -INFINITY;
-                }
-            }
-            // ---- online softmax per head: max over the slice's 16 tokens
-            float pr[NT][4];
-            float f[NT][2];
+                for (int u = 0; u < 2; ++u) {
+                    if (G32) {
+                        float ksa[NG], ksb[NG];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+                        for (int a = 0; a < NG; ++a) {
+                            ksa[a] = ldsf(sks + (rA[u] * NG + a) * 4);
+                            ksb[a] = ldsf(sks + (rB[u] * NG + a) * 4);
+                        }
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    float mx = fmaxf(z[nt][c], z[nt][2 + c]);
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                    const float mn = fmaxf(m[nt][c], mx);
-                    const float al = (mn == -INFINITY) ? 1.f : ptx::ex2(m[nt][c] - mn);
-                    pr[nt][c] = okA ? ptx::ex2(z[nt][c] - mn) : 0.f;
-                    pr[nt][2 + c] = okB ? ptx::ex2(z[nt][2 + c] - mn) : 0.f;
-                    l[nt][c] = l[nt][c] * al + pr[nt][c] + pr[nt][2 + c];
-                    m[nt][c] = mn;
-                    f[nt][c] = al;
-                }
-            // ---- V scales of the thread's two tokens and the running prescale 2^kv
-            float vsa[NGV], vsb[NGV];
-            float vmax = 0.f;
+                        for (int nt = 0; nt < NT; ++nt) {
+                            float za0 = 0.f, za1 = 0.f, zb0 = 0.f, zb1 = 0.f;
 #pragma unroll
-            for (int gv = 0; gv < NGV; ++gv) {
-                vsa[gv] = okA ? ldsf(svs + (rowA * NG + gv) * 4) : 0.f;
-                vsb[gv] = okB ? ldsf(svs + (rowB * NG + gv) * 4) : 0.f;
-                vmax = fmaxf(vmax, fmaxf(vsa[gv], vsb[gv]));
-            }
-            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
-            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 8));
-            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 16));
-            if (vmax > 0.f) {
-                const int ev = static_cast<int>((__float_as_uint(vmax) >> 23) & 0xffu) - 127;
-                const int kn = min(kv, 14 - ev);
-                if (kn < kv) {
-                    const float drop = ldexpf(1.f, kn - kv);
+                            for (int a = 0; a < NACC; ++a) {
+                                za0 = fmaf(sacc[u][nt][a][0], ksa[a], za0);
+                                za1 = fmaf(sacc[u][nt][a][1], ksa[a], za1);
+                                zb0 = fmaf(sacc[u][nt][a][2], ksb[a], zb0);
+                                zb1 = fmaf(sacc[u][nt][a][3], ksb[a], zb1);
+                            }
+                            z[u][nt][0] = okA[u] ? za0 * zs[nt][0] : -INFINITY;
+                            z[u][nt][1] = okA[u] ? za1 * zs[nt][1] : -INFINITY;
+                            z[u][nt][2] = okB[u] ? zb0 * zs[nt][0] : -INFINITY;
+                            z[u][nt][3] = okB[u] ? zb1 * zs[nt][1] : -INFINITY;
+                        }
+                    } else {
+                        const float ksa = ldsf(sks + rA[u] * 4), ksb = ldsf(sks + rB[u] * 4);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        f[nt][0] *= drop;
-                        f[nt][1] *= drop;
-                    }
-                    kv = kn;
-                }
-            }
-            const float up = ldexpf(1.f, kv);
-            bool unit = true;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) unit = unit && f[nt][0] == 1.f && f[nt][1] == 1.f;
-            if (!__all_sync(0xffffffffu, unit)) {       // the running max moved: rescale O
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        o[mt][nt][0] *= f[nt][0];
-                        o[mt][nt][1] *= f[nt][1];
-                        o[mt][nt][2] *= f[nt][0];
-                        o[mt][nt][3] *= f[nt][1];
-                    }
-            }
-            // ---- P^T operand: P'' hi / lo, transposed from the score layout
-            // (row = token, column = head) into B fragments (k = token, n = head)
-            uint32_t pbh[NGV][NT][2], pbl[NGV][NT][2];
-#pragma unroll
-            for (int gv = 0; gv < NGV; ++gv)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    uint32_t ha, la, hb, lb;
-                    split_f16x2(pr[nt][0] * vsa[gv] * up, pr[nt][1] * vsa[gv] * up, ha, la);
-                    split_f16x2(pr[nt][2] * vsb[gv] * up, pr[nt][3] * vsb[gv] * up, hb, lb);
-                    pbh[gv][nt][0] = transpose8x8(ha);
-                    pbl[gv][nt][0] = transpose8x8(la);
-                    pbh[gv][nt][1] = transpose8x8(hb);
-                    pbl[gv][nt][1] = transpose8x8(lb);
-                }
-            // ---- O^T += V^T . P^T.  V^T A fragment of m-tile mt: rows g, g+8 are
-            // head_dim d(mt, g), d(mt, g) + 1; columns 2t, 2t+1 / 2t+8, 2t+9 are the
-            // V rows R0, R1 / R2, R3.  Byte pairs of two rows are interleaved with
-            // prmt and turned into exact (v - 128) f16 pairs.
-            auto pv_words = [&](int mt0, int gv, uint32_t w0, uint32_t w1, uint32_t w2,
-                                uint32_t w3) {
-                const uint32_t xl01 = ptx::prmt(w0, w1, 0x5140u);
-                const uint32_t xh01 = ptx::prmt(w0, w1, 0x7362u);
-                const uint32_t xl23 = ptx::prmt(w2, w3, 0x5140u);
-                const uint32_t xh23 = ptx::prmt(w2, w3, 0x7362u);
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const uint32_t x01 = hh ? xh01 : xl01;
-                    const uint32_t x23 = hh ? xh23 : xl23;
-                    const uint32_t a0 = ptx::bytes_to_f16x2(x01, 0x4140u);
-                    const uint32_t a1 = ptx::bytes_to_f16x2(x01, 0x4342u);
-                    const uint32_t a2 = ptx::bytes_to_f16x2(x23, 0x4140u);
-                    const uint32_t a3 = ptx::bytes_to_f16x2(x23, 0x4342u);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        ptx::mma_f16(o[mt0 + hh][nt], a0, a1, a2, a3, pbh[gv][nt][0],
-                                     pbh[gv][nt][1]);
-                        ptx::mma_f16(o[mt0 + hh][nt], a0, a1, a2, a3, pbl[gv][nt][0],
-                                     pbl[gv][nt][1]);
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const float s0 = sacc[u][nt][0][0] + sacc[u][nt][1][0];
+                            const float s1 = sacc[u][nt][0][1] + sacc[u][nt][1][1];
+                            const float s2 = sacc[u][nt][0][2] + sacc[u][nt][1][2];
+                            const float s3 = sacc[u][nt][0][3] + sacc[u][nt][1][3];
+                            z[u][nt][0] = okA[u] ? s0 * ksa * zs[nt][0] : -INFINITY;
+                            z[u][nt][1] = okA[u] ? s1 * ksa * zs[nt][1] : -INFINITY;
+                            z[u][nt][2] = okB[u] ? s2 * ksb * zs[nt][0] : -INFINITY;
+                            z[u][nt][3] = okB[u] ? s3 * ksb * zs[nt][1] : -INFINITY;
+                        }
                     }
                 }
-            };
-            if (!G32) {
-                if constexpr (D == 128) {
-                    // thread g owns head_dim [16g, 16g + 16): d(mt, g) = 16g + 2mt
-                    const uint4 v0 = lds128(sv + swz<D>(R0, 16 * g));
-                    const uint4 v1 = lds128(sv + swz<D>(R1, 16 * g));
-                    const uint4 v2 = lds128(sv + swz<D>(R2, 16 * g));
-                    const uint4 v3 = lds128(sv + swz<D>(R3, 16 * g));
-                    pv_words(0, 0, v0.x, v1.x, v2.x, v3.x);
-                    pv_words(2, 0, v0.y, v1.y, v2.y, v3.y);
-                    pv_words(4, 0, v0.z, v1.z, v2.z, v3.z);
-                    pv_words(6, 0, v0.w, v1.w, v2.w, v3.w);
-                } else {
-                    // D == 64: thread g owns head_dim [8g, 8g + 8): d(mt, g) = 8g + 2mt
-                    const uint2 v0 = lds64(sv + swz<D>(R0, 8 * g));
-                    const uint2 v1 = lds64(sv + swz<D>(R1, 8 * g));
-                    const uint2 v2 = lds64(sv + swz<D>(R2, 8 * g));
-                    const uint2 v3 = lds64(sv + swz<D>(R3, 8 * g));
-                    pv_words(0, 0, v0.x, v1.x, v2.x, v3.x);
-                    pv_words(2, 0, v0.y, v1.y, v2.y, v3.y);
-                }
-            } else {
-                // group-32: m-tiles 2*gv, 2*gv + 1 stay inside group gv:
-                // d(2gv + hh, g) = 32*gv + 4*g + 2*hh
+                // ---- online softmax per head: max over the slice's 32 tokens
+                float pr[2][NT][4];
+                float f[NT][2];
 #pragma unroll
-                for (int gv = 0; gv < NGRP; ++gv) {
-                    const uint32_t cb = 32 * gv + 4 * g;
-                    pv_words(2 * gv, gv, lds32(sv + swz<D>(R0, cb)), lds32(sv + swz<D>(R1, cb)),
-                             lds32(sv + swz<D>(R2, cb)), lds32(sv + swz<D>(R3, cb)));
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        float mx = fmaxf(fmaxf(z[0][nt][c], z[0][nt][2 + c]),
+                                         fmaxf(z[1][nt][c], z[1][nt][2 + c]));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                        const float mn = fmaxf(m[nt][c], mx);
+                        const float al = (mn == -INFINITY) ? 1.f : ptx::ex2(m[nt][c] - mn);
+                        float add = 0.f;
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            pr[u][nt][c] = okA[u] ? ptx::ex2(z[u][nt][c] - mn) : 0.f;
+                            pr[u][nt][2 + c] = okB[u] ? ptx::ex2(z[u][nt][2 + c] - mn) : 0.f;
+                            add += pr[u][nt][c] + pr[u][nt][2 + c];
+                        }
+                        l[nt][c] = l[nt][c] * al + add;
+                        m[nt][c] = mn;
+                        f[nt][c] = al;
+                    }
+                // ---- V scales of the thread's four tokens and the running prescale 2^kv
+                float vsa[2][NGV], vsb[2][NGV];
+                float vmax = 0.f;
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int gv = 0; gv < NGV; ++gv) {
+                        vsa[u][gv] = okA[u] ? ldsf(svs + (rA[u] * NG + gv) * 4) : 0.f;
+                        vsb[u][gv] = okB[u] ? ldsf(svs + (rB[u] * NG + gv) * 4) : 0.f;
+                        vmax = fmaxf(vmax, fmaxf(vsa[u][gv], vsb[u][gv]));
+                    }
+                vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
+                vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 8));
+                vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 16));
+                if (vmax > 0.f) {
+                    const int ev = static_cast<int>((__float_as_uint(vmax) >> 23) & 0xffu) - 127;
+                    const int kn = max(min(kv, 14 - ev), -120);   // kv stays in [-120, 64]
+                    if (kn < kv) {
+                        const float drop = ldexpf(1.f, kn - kv);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            f[nt][0] *= drop;
+                            f[nt][1] *= drop;
+                        }
+                        kv = kn;
+                    }
                 }
-            }
+                const float up = pow2i(kv);
+                bool unit = true;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) unit = unit && f[nt][0] == 1.f && f[nt][1] == 1.f;
+                if (!__all_sync(0xffffffffu, unit)) {       // the running max moved: rescale O
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            o[mt][nt][0] *= f[nt][0];
+                            o[mt][nt][1] *= f[nt][1];
+                            o[mt][nt][2] *= f[nt][0];
+                            o[mt][nt][3] *= f[nt][1];
+                        }
+                }
+                // ---- O^T += V^T . P^T, one k-step of 16 tokens per MMA tile u.  P^T
+                // operand: P'' hi / lo transposed from the score layout (row = token,
+                // column = head) into B fragments (k = token, n = head).  V^T A
+                // fragment of m-tile mt: rows g, g+8 are head_dim d(mt, g),
+                // d(mt, g) + 1; columns 2t, 2t+1 / 2t+8, 2t+9 are the V rows
+                // V0, V1 / V0 + 8, V1 + 8.  Byte pairs of two rows are interleaved
+                // with prmt and turned into exact (v - 128) f16 pairs.
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    uint32_t pbh[NGV][NT][2], pbl[NGV][NT][2];
+#pragma unroll
+                    for (int gv = 0; gv < NGV; ++gv)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            uint32_t ha, la, hb, lb;
+                            split_f16x2(pr[u][nt][0] * vsa[u][gv] * up,
+                                        pr[u][nt][1] * vsa[u][gv] * up, ha, la);
+                            split_f16x2(pr[u][nt][2] * vsb[u][gv] * up,
+                                        pr[u][nt][3] * vsb[u][gv] * up, hb, lb);
+                            pbh[gv][nt][0] = transpose8x8(ha);
+                            pbl[gv][nt][0] = transpose8x8(la);
+                            pbh[gv][nt][1] = transpose8x8(hb);
+                            pbl[gv][nt][1] = transpose8x8(lb);
+                        }
+                    auto pv_words = [&](int mt0, int gv, uint32_t w0, uint32_t w1, uint32_t w2,
+                                        uint32_t w3) {
+                        const uint32_t xl01 = ptx::prmt(w0, w1, 0x5140u);
+                        const uint32_t xh01 = ptx::prmt(w0, w1, 0x7362u);
+                        const uint32_t xl23 = ptx::prmt(w2, w3, 0x5140u);
+                        const uint32_t xh23 = ptx::prmt(w2, w3, 0x7362u);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t x01 = hh ? xh01 : xl01;
+                            const uint32_t x23 = hh ? xh23 : xl23;
+                            const uint32_t a0 = ptx::bytes_to_f16x2(x01, 0x4140u);
+                            const uint32_t a1 = ptx::bytes_to_f16x2(x01, 0x4342u);
+                            const uint32_t a2 = ptx::bytes_to_f16x2(x23, 0x4140u);
+                            const uint32_t a3 = ptx::bytes_to_f16x2(x23, 0x4342u);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                ptx::mma_f16(o[mt0 + hh][nt], a0, a1, a2, a3, pbh[gv][nt][0],
+                                             pbh[gv][nt][1]);
+                                ptx::mma_f16(o[mt0 + hh][nt], a0, a1, a2, a3, pbl[gv][nt][0],
+                                             pbl[gv][nt][1]);
+                            }
+                        }
+                    };
+                    const int R0 = V0[u], R1 = V1[u], R2 = V0[u] + 8, R3 = V1[u] + 8;
+                    if (!G32) {
+                        if constexpr (D == 128) {
+                            // thread g owns head_dim [16g, 16g + 16): d(mt, g) = 16g + 2mt
+                            const uint4 v0 = lds128(sv + swz<D>(R0, 16 * g));
+                            const uint4 v1 = lds128(sv + swz<D>(R1, 16 * g));
+                            const uint4 v2 = lds128(sv + swz<D>(R2, 16 * g));
+                            const uint4 v3 = lds128(sv + swz<D>(R3, 16 * g));
+                            pv_words(0, 0, v0.x, v1.x, v2.x, v3.x);
+                            pv_words(2, 0, v0.y, v1.y, v2.y, v3.y);
+                            pv_words(4, 0, v0.z, v1.z, v2.z, v3.z);
+                            pv_words(6, 0, v0.w, v1.w, v2.w, v3.w);
+                        } else {
+                            // D == 64: thread g owns head_dim [8g, 8g + 8): d(mt, g) = 8g + 2mt
+                            const uint2 v0 = lds64(sv + swz<D>(R0, 8 * g));
+                            const uint2 v1 = lds64(sv + swz<D>(R1, 8 * g));
+                            const uint2 v2 = lds64(sv + swz<D>(R2, 8 * g));
+                            const uint2 v3 = lds64(sv + swz<D>(R3, 8 * g));
+                            pv_words(0, 0, v0.x, v1.x, v2.x, v3.x);
+                            pv_words(2, 0, v0.y, v1.y, v2.y, v3.y);
+                        }
+                    } else {
+                        // group-32: m-tiles 2*gv, 2*gv + 1 stay inside group gv:
+                        // d(2gv + hh, g) = 32*gv + 4*g + 2*hh
+#pragma unroll
+                        for (int gv = 0; gv < NGRP; ++gv) {
+                            const uint32_t cb = 32 * gv + 4 * g;
+                            pv_words(2 * gv, gv, lds32(sv + swz<D>(R0, cb)),
+                                     lds32(sv + swz<D>(R1, cb)), lds32(sv + swz<D>(R2, cb)),
+                                     lds32(sv + swz<D>(R3, cb)));
+                        }
+                    }
+                }
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bar_empty + 8 * s);
         }
-        open = true;
-        // the segment continues if the next item is the next chunk of this (b, kv head)
-        if (i + 1 < iend) {
-            const Item nx = item_at(i + 1, lens, cum, B, p.Hk, p.chunk);
-            if (nx.b == b && nx.hk == hk) continue;
-        }
-        open = false;
 
         // ---- merge the eight warps' states of the segment (one round)
         // a segment that is the whole sequence writes the final rows (and,
         // when the sequence has several chunks, a marker l = -1 in slot 0 that
         // tells the combine kernel to leave them alone)
-        const bool final_rows = itm.ns == 1 || (seg_j0 == 0 && itm.j == itm.ns - 1);
+        const bool final_rows = sg.j0 == 0 && sg.j1 == sg.ns - 1;
+        const int seg_j0 = sg.j0;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -696,8 +809,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 8);
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 16);
                 if (g == 0) {
-                    mrg_m[warp * 16 + 8 * nt + 2 * t + c] = m[nt][c];
-                    mrg_l[warp * 16 + 8 * nt + 2 * t + c] = l[nt][c];
+                    mrg_m[cw * 16 + 8 * nt + 2 * t + c] = m[nt][c];
+                    mrg_l[cw * 16 + 8 * nt + 2 * t + c] = l[nt][c];
                 }
             }
         ptx::named_bar_sync(1, NCONS);
@@ -706,7 +819,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // when the rows are final)
         float fo[NT][2];
         {
-            const float down = ldexpf(1.f, -kv);
+            const float down = pow2i(-kv);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -724,24 +837,15 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     for (int w = 0; w < NW; ++w)
                         if (mw[w] != -INFINITY) Ls = fmaf(mrg_l[w * 16 + h], ptx::ex2(mw[w] - M), Ls);
                     const float f = (m[nt][c] == -INFINITY) ? 0.f : ptx::ex2(m[nt][c] - M) * down;
-                    fo[nt][c] = final_rows ? (Ls > 0.f ? f / Ls : 0.f) : f;
-                    if (warp == 0 && g == 0 && itm.ns > 1 && h < G) {
-                        const int64_t row = bh0 + h;
-                        if (final_rows) {
-                            p.ws_l[row * p.splits] = -1.f;
-                        } else {
-                            p.ws_m[row * p.splits + seg_j0] = M;
-                            p.ws_l[row * p.splits + seg_j0] = Ls;
-                            for (int jj = seg_j0 + 1; jj <= itm.j; ++jj) {   // merged into seg_j0
-                                p.ws_m[row * p.splits + jj] = -INFINITY;
-                                p.ws_l[row * p.splits + jj] = 0.f;
-                            }
-                        }
+                    fo[nt][c] = final_rows ? (Ls > 0.f ? f * __frcp_rn(Ls) : 0.f) : f;
+                    if (cw == 0 && g == 0) {
+                        seg_M[h] = M;
+                        seg_L[h] = Ls;
                     }
                 }
         }
         {
-            float* slot = mslot + warp * NV * 32 + lane;
+            float* slot = mslot + cw * NV * 32 + lane;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -752,7 +856,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         ptx::named_bar_sync(1, NCONS);
         // sum the eight slots position by position and write the rows
-        for (int pos = tid; pos < NV * 32; pos += NCONS) {
+#pragma unroll 1
+        for (int pos = ctid; pos < NV * 32; pos += NCONS) {
             const int v = pos >> 5, ln = pos & 31;
             const int pg_ = ln >> 2, pt = ln & 3;
             const int mt = v / (NT * 4), nt = (v / 4) % NT, e = v & 3;
@@ -766,6 +871,23 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int64_t row = bh0 + h;
             if (final_rows) p.out[row * D + d] = sum;
             else p.ws_o[(row * p.splits + seg_j0) * D + d] = sum;
+        }
+        // the partial's (m, l) and the empty markers of the chunks merged into
+        // slot seg_j0, or the finished marker (l = -1 in slot 0)
+        if (!final_rows || sg.ns > 1) {
+            const int nrow = final_rows ? 1 : sg.j1 - seg_j0 + 1;
+#pragma unroll 1
+            for (int idx = ctid; idx < G * nrow; idx += NCONS) {
+                const int k = idx / G, h = idx - k * G;
+                float* const wm = p.ws_m + (bh0 + h) * p.splits + seg_j0 + k;
+                float* const wl = p.ws_l + (bh0 + h) * p.splits + seg_j0 + k;
+                if (final_rows) {
+                    *wl = -1.f;
+                } else {
+                    *wm = k == 0 ? seg_M[h] : -INFINITY;
+                    *wl = k == 0 ? seg_L[h] : 0.f;
+                }
+            }
         }
     }
 }

@@ -192,3 +192,22 @@ def test_decode_large_query_magnitudes():
     sl = torch.tensor([L], dtype=torch.int32)
     out = c.decode(q, sl, L, attn_scale=1e-4)
     assert_attn_close(out, c.oracle_decode(q, sl, 1e-4), "q magnitudes")
+
+
+@pytest.mark.parametrize("mode,D", [("per_token", 128), ("per_token", 64), ("group32", 64)])
+@pytest.mark.parametrize("S", [257, 130, 131])
+def test_decode_full_cache_unaligned_capacity(mode, D, S):
+    """Every sequence fills its whole capacity S, and S * (scales per token) is
+    not a multiple of 4: the scale rows of a (sequence, kv head) start off a
+    16-byte boundary and the last tile ends at the end of the scale array."""
+    B, Hk, G = 2, 3, 2
+    c = ContigCache(B, Hk, S, D, mode)
+    k = bf16_randn((B, Hk, S, D), seed=S, sigma=0.7)
+    v = bf16_randn((B, Hk, S, D), seed=S + 1, sigma=0.7)
+    assert c.append(k, v, torch.zeros(B, dtype=torch.int32)) == 0
+    q = bf16_randn((B, Hk * G, D), seed=S + 2)
+    sl = torch.tensor([S, S], dtype=torch.int32)
+    for ns in (0, 1, 3):
+        out = c.decode(q, sl, S, attn_scale=f32_scale(D), num_splits=ns)
+        assert_attn_close(out, c.oracle_decode(q, sl, f32_scale(D)), f"S={S} ns={ns}")
+    assert kvq().kvq_read_error(c.err) == 0
