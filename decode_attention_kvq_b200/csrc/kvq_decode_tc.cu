@@ -256,7 +256,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         ptx::prefetch_tensormap(&tm_v);
 #pragma unroll 1
         for (int s = 0; s < NST; ++s) {
-            ptx::mbar_init(bar_full + 8 * s, 1);        // the producer's expect_tx arrival
+            // the producer's expect_tx arrival (+ one cp.async arrival per lane
+            // of the producer warp for the paged scales)
+            ptx::mbar_init(bar_full + 8 * s, PAGED ? 1 + 32 : 1);
             ptx::mbar_init(bar_empty + 8 * s, WPG);
         }
         *abort_flag = 0;
@@ -347,6 +349,24 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int b = sg.b, hk = sg.hk;
             const uint16_t* qsrc = qg + (static_cast<int64_t>(b) * Hq + hk * G) * D;
             int seg_tiles = 0;          // tiles issued for this segment
+            // paged: the segment's page ids, 32 pages (4 stages) per register,
+            // loaded one group of 4 stages ahead so the table read is off the
+            // issue path; lane i holds page pbase + i (-1: none or out of range)
+            int pbase = sg.t0 >> 4;
+            int32_t pg_cur = -1, pg_nxt = -1;
+            auto load_pages = [&](int first) {
+                const int idx = first + lane;
+                int32_t v = -1;
+                if (16 * idx < sg.t1) {
+                    v = table[static_cast<int64_t>(b) * max_pages + idx];
+                    if (v < 0 || v >= num_pages) v = -1;
+                }
+                return v;
+            };
+            if (PAGED) {
+                pg_cur = load_pages(pbase);
+                pg_nxt = load_pages(pbase + 32);
+            }
 #pragma unroll 1
             for (int tt0 = sg.t0; tt0 < sg.t1; tt0 += TT, ++count, ++seg_tiles) {
                 const int s = count % NST;
@@ -393,15 +413,16 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         if (with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
                     }
                 } else {
-                    constexpr int PPS = TT / 16;                // pages per stage
-                    constexpr uint32_t PAGE_BYTES = 2 * 16 * D + 2 * 64 * NG;
+                    constexpr uint32_t PAGE_BYTES = 2 * 16 * D;   // TMA bytes (scales by cp.async)
                     const int np = (ntok + 15) >> 4;
-                    int32_t pg = -1;
-                    if (lane < np) {
-                        // a bad entry is skipped (its tokens are masked)
-                        pg = table[static_cast<int64_t>(b) * max_pages + (tt0 >> 4) + lane];
-                        if (pg < 0 || pg >= num_pages) pg = -1;
+                    if ((tt0 >> 4) >= pbase + 32) {
+                        pbase += 32;
+                        pg_cur = pg_nxt;
+                        pg_nxt = load_pages(pbase + 32);
                     }
+                    // a bad entry is skipped (its tokens are masked)
+                    int32_t pg = __shfl_sync(0xffffffffu, pg_cur, (tt0 >> 4) - pbase + (lane & 7));
+                    if (lane >= np) pg = -1;
                     const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
                     if (lane == 0) {
                         // the consumers mask the tokens of pages that were not
@@ -410,27 +431,36 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         sts_u32(sk + Lay::MASK_OFF, valid);
                         ptx::mbar_arrive_expect_tx(
                             full, __popc(valid) * PAGE_BYTES + (with_q ? q_bytes : 0u));
+                        if (with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
+                    }
+                    __syncwarp();
+                    // lane q < 8 loads page q's K and V rows (16 rows of this kv
+                    // head per page); every lane copies 16-byte chunks of the
+                    // pages' scales (16 * NG aligned floats per page), chunk c of
+                    // the stage being page c / (4 NG)
+                    if (pg >= 0) {
+                        const int y = (pg * Hk + hk) * 16;
+                        ptx::tma_load_2d(sk + lane * 16 * D, &tm_k, 0, y, full, pol);
+                        ptx::tma_load_2d(sv + lane * 16 * D, &tm_v, 0, y, full, pol);
                     }
 #pragma unroll
-                    for (int q = 0; q < PPS; ++q) {
+                    for (int it = 0; it < NG; ++it) {
+                        const int c = lane + 32 * it;
+                        const int q = c / (4 * NG), cc = c % (4 * NG);
                         const int pq = __shfl_sync(0xffffffffu, pg, q);
-                        if (lane == 0 && pq >= 0) {
-                            // a page holds 16 rows of this kv head; its scales are
-                            // 16 * NG aligned floats
-                            const int y = (pq * Hk + hk) * 16;
-                            ptx::tma_load_2d(sk + q * 16 * D, &tm_k, 0, y, full, pol);
-                            ptx::tma_load_2d(sv + q * 16 * D, &tm_v, 0, y, full, pol);
-                            const int64_t fc = static_cast<int64_t>(y) * NG;
-                            ptx::bulk_load(sks + q * 64 * NG, k_scale + fc, 64 * NG, full);
-                            ptx::bulk_load(svs + q * 64 * NG, v_scale + fc, 64 * NG, full);
+                        if (pq >= 0) {
+                            const int64_t fc = static_cast<int64_t>((pq * Hk + hk) * 16) * NG + 4 * cc;
+                            ptx::cp_async_16(sks + 16 * c, k_scale + fc);
+                            ptx::cp_async_16(svs + 16 * c, v_scale + fc);
                         }
                     }
-                    if (lane == 0 && with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
+                    ptx::cp_async_arrive_noinc(full);
                 }
             }
         }
         // the last tile of every slot has landed (normally long consumed; after a
         // timeout this keeps the CTA alive until its bulk copies are done)
+        if (PAGED) asm volatile("cp.async.wait_all;" ::: "memory");
         if (lane == 0)
 #pragma unroll 1
             for (int c = count - 1; c >= 0 && c >= count - NST; --c)
