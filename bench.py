@@ -167,15 +167,22 @@ def decode_traffic_record():
     """DRAM bytes per decode launch from a committed ncu summary, valid only if
     the decode kernel source still has the hash recorded with it."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    src = os.path.join(ROOT, "decode_attention_kvq_b200", "csrc", "kvq_decode.cu")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if rec.get("kvq_decode_cu_sha256") != h:
+    if rec.get("decode_sources_sha256") != decode_sources_hash():
         return None
     return rec
+
+
+def decode_sources_hash():
+    """sha256 over the decode kernels' sources (split kernel, combine, PTX helpers)."""
+    h = hashlib.sha256()
+    for name in ("kvq_decode_tc.cu", "kvq_decode.cu", "kvq_ptx.cuh", "kvq_internal.cuh"):
+        with open(os.path.join(ROOT, "decode_attention_kvq_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 # ---------------------------------------------------------------- workload
@@ -397,10 +404,9 @@ def run_kvq(args, wl):
     L0 = layers[0]
     ws_bytes = kvq.kvq_decode_workspace_bytes(wl.B, wl.Hq, wl.Hk, wl.D, L0.hint)
     workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    # a cluster of splits combines in distributed shared memory: no workspace
     chunk, splits = kvq.kvq_decode_plan(wl.B, wl.Hk, L0.hint)
-    # append (+ prefill-chunk append) + split kernel (+ combine kernel when the
-    # splits do not fit one cluster and go through the workspace)
+    # append (+ prefill-chunk append) + split kernel (+ combine kernel when a
+    # sequence spans several chunks: then the call has a workspace)
     launches_per_layer = (1 + (1 if wl.prefill_chunk else 0)) + 1 + (1 if ws_bytes > 0 else 0)
 
     stream = torch.cuda.Stream(dev)
