@@ -211,11 +211,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     constexpr int NG = Lay::NG;
     constexpr int NST = Lay::NST;
     constexpr int NV = Lay::NV;
-    constexpr int KS = D / 16;          // MMA k-steps over head_dim (QK)
     constexpr int NGRP = D / 32;        // 32-value groups over head_dim
     constexpr int MT = D / 16;          // m-tiles of O^T over head_dim (PV)
     constexpr int NT = G16 ? 2 : 1;     // n-tiles of 8 query heads
-    constexpr int NACC = G32 ? NG : 2;  // score accumulators per n-tile (two chains per token)
     constexpr int NGV = G32 ? NG : 1;   // V scales per token
 
     extern __shared__ uint8_t smem_raw[];
@@ -479,7 +477,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int sig_g = sigma(g);
     const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
 
-    uint32_t qb0[NT][KS], qb1[NT][KS];
+    constexpr int NCG = G32 ? NGRP : 1;   // offset terms per head (per 32-value group)
+    uint32_t qh0[NT][NGRP], qh1[NT][NGRP], ql0[NT][NGRP], ql1[NT][NGRP];   // Q digits
+    int qc[NT][2][NCG];                   // 128 * sum(Qi) of the thread's two heads
     float zs[NT][2];
     float m[NT][2], l[NT][2];
     float o[MT][NT][4];                 // O^T C fragments: rows = head_dim, columns = heads
@@ -529,13 +529,18 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const uint32_t svs = sv + Lay::KV_BYTES + Lay::SC_FLOATS * 4 + sc_off;
             if (!have_q) {
                 // ---- Q^T operand (the segment's query rows ride with its first
-                // two stages): column n = g of n-tile nt is query head 8*nt + g,
-                // pre-scaled by 2^sh so max |q| * 2^sh is in [2^14, 2^15).  B
-                // fragment rows 2t, 2t+1 (qb0) and 2t+8, 2t+9 (qb1) of k-step
-                // 2*gi + h2 hold head_dim 32*gi + 8*t + 4*h2 + {0, 1} and {2, 3}.
+                // two stages).  Column n = g of n-tile nt is query head 8*nt + g.
+                // Each head is scaled by 2^sh so max |q| * 2^sh is in [2^14, 2^15)
+                // and rounded to a 16-bit integer Qi = 256 * hi + lo (hi signed,
+                // lo unsigned byte); the relative error per element is at most
+                // 2^-15 of the head's max |q|.  B fragment rows 4t..4t+3 (b0) and
+                // 16+4t..16+4t+3 (b1) of k-step gi hold head_dim 32*gi + 8*t +
+                // {0..3} and {4..7}: the same permutation of head_dim as the
+                // K operand's bytes, so the dot products are unchanged.
                 have_q = true;
                 const uint32_t sq = sk + Lay::Q_OFF;
                 float zsq[NT];
+                int csq[NT][NCG];              // sum of the head's Qi (per 32-value group)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int h = 8 * nt + g;
@@ -564,21 +569,40 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const float up = pow2i(sh);                  // |sh| <= 100
                     zsq[nt] = pow2i(-sh) * p.scale_log2;
 #pragma unroll
-                    for (int gi = 0; gi < NGRP; ++gi)
+                    for (int c = 0; c < NCG; ++c) csq[nt][c] = 0;
 #pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) {
-                            qb0[nt][2 * gi + h2] =
-                                ptx::pack_f16x2(qf[gi][4 * h2] * up, qf[gi][4 * h2 + 1] * up);
-                            qb1[nt][2 * gi + h2] =
-                                ptx::pack_f16x2(qf[gi][4 * h2 + 2] * up, qf[gi][4 * h2 + 3] * up);
+                    for (int gi = 0; gi < NGRP; ++gi) {
+                        uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int qi = min(max(__float2int_rn(qf[gi][e] * up), -32767), 32767);
+                            csq[nt][G32 ? gi : 0] += qi;
+                            hw[e >> 2] |= (static_cast<uint32_t>(qi >> 8) & 0xffu) << (8 * (e & 3));
+                            lw[e >> 2] |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * (e & 3));
                         }
-                }
-                // score factor of the two heads (columns 2t, 2t+1) this thread accumulates
+                        qh0[nt][gi] = hw[0];
+                        qh1[nt][gi] = hw[1];
+                        ql0[nt][gi] = lw[0];
+                        ql1[nt][gi] = lw[1];
+                    }
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    zs[nt][0] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t));
-                    zs[nt][1] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t + 1));
+                    for (int c = 0; c < NCG; ++c) {
+                        csq[nt][c] += __shfl_xor_sync(0xffffffffu, csq[nt][c], 1);
+                        csq[nt][c] += __shfl_xor_sync(0xffffffffu, csq[nt][c], 2);
+                    }
                 }
+                // per-head factors of the two heads (columns 2t, 2t+1) this thread
+                // accumulates: score scale, and the offset term 128 * sum(Qi) of
+                // sum Qi * (byte - 128) = sum Qi * byte - 128 * sum Qi
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        zs[nt][c] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t + c));
+#pragma unroll
+                        for (int k = 0; k < NCG; ++k)
+                            qc[nt][c][k] = 128 * __shfl_sync(0xffffffffu, csq[nt][k], 4 * (2 * t + c));
+                    }
             }
             const int tok0 = tt0 + 32 * wg;               // first token of this warp's slice
             if (tok0 < t1) {
@@ -602,77 +626,72 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     okB[u] = page_ok && (tk + 8 + sig_g < t1);
                 }
 
-                // ---- S^T = K . Q^T per MMA tile: rows tokens (rA, rB), columns heads
-                float sacc[2][NT][NACC][4];
+                // ---- S^T = K . Q^T per MMA tile on the integer MMA: the K bytes
+                // are the A operand as loaded (rows tokens rA, rB; 8 bytes at
+                // 32*gi + 8*t are k = 4t..4t+3 and 16+4t..16+4t+3), times the two
+                // Q digits; S = 256 * S_hi + S_lo - 128 * sum(Qi) is exact in s32.
+                // ---- scores z (log2 domain): [u][nt][0..1] token rA[u], [u][nt][2..3] token rB[u]
+                float z[2][NT][4];
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
+                        z[u][nt][0] = z[u][nt][1] = z[u][nt][2] = z[u][nt][3] = 0.f;
+                int ah[2][NT][4], al[2][NT][4];
+                auto zero_acc = [&]() {
 #pragma unroll
-                        for (int a = 0; a < NACC; ++a)
-                            sacc[u][nt][a][0] = sacc[u][nt][a][1] = sacc[u][nt][a][2] =
-                                sacc[u][nt][a][3] = 0.f;
+                    for (int u = 0; u < 2; ++u)
 #pragma unroll
-                for (int gi = 0; gi < NGRP; ++gi)
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) ah[u][nt][e] = al[u][nt][e] = 0;
+                };
+                // fold the integer scores of head_dim group kg into z, times the K
+                // scale of the token (per token: kg = 0, once after all groups)
+                auto fold = [&](int kg) {
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const float ksa = ldsf(sks + (rA[u] * NG + kg) * 4);
+                        const float ksb = ldsf(sks + (rB[u] * NG + kg) * 4);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int S = ah[u][nt][e] * 256 + al[u][nt][e] - qc[nt][e & 1][kg];
+                                z[u][nt][e] = fmaf(static_cast<float>(S), e < 2 ? ksa : ksb, z[u][nt][e]);
+                            }
+                    }
+                };
+                zero_acc();
+#pragma unroll
+                for (int gi = 0; gi < NGRP; ++gi) {
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const uint2 wa = lds64(sk + swz<D>(rA[u], 32 * gi + 8 * t));
                         const uint2 wb = lds64(sk + swz<D>(rB[u], 32 * gi + 8 * t));
 #pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) {
-                            const uint32_t xa = h2 ? wa.y : wa.x;
-                            const uint32_t xb = h2 ? wb.y : wb.x;
-                            const uint32_t a0 = ptx::bytes_to_f16x2(xa, 0x4140u);
-                            const uint32_t a2 = ptx::bytes_to_f16x2(xa, 0x4342u);
-                            const uint32_t a1 = ptx::bytes_to_f16x2(xb, 0x4140u);
-                            const uint32_t a3 = ptx::bytes_to_f16x2(xb, 0x4342u);
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt)
-                                ptx::mma_f16(sacc[u][nt][G32 ? gi : (gi & 1)], a0, a1, a2, a3,
-                                             qb0[nt][2 * gi + h2], qb1[nt][2 * gi + h2]);
+                        for (int nt = 0; nt < NT; ++nt) {
+                            ptx::mma_u8<true>(ah[u][nt], wa.x, wb.x, wa.y, wb.y, qh0[nt][gi],
+                                              qh1[nt][gi]);
+                            ptx::mma_u8<false>(al[u][nt], wa.x, wb.x, wa.y, wb.y, ql0[nt][gi],
+                                               ql1[nt][gi]);
                         }
                     }
-                // ---- scores z (log2 domain): [u][nt][0..1] token rA[u], [u][nt][2..3] token rB[u]
-                float z[2][NT][4];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
                     if (G32) {
-                        float ksa[NG], ksb[NG];
-#pragma unroll
-                        for (int a = 0; a < NG; ++a) {
-                            ksa[a] = ldsf(sks + (rA[u] * NG + a) * 4);
-                            ksb[a] = ldsf(sks + (rB[u] * NG + a) * 4);
-                        }
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            float za0 = 0.f, za1 = 0.f, zb0 = 0.f, zb1 = 0.f;
-#pragma unroll
-                            for (int a = 0; a < NACC; ++a) {
-                                za0 = fmaf(sacc[u][nt][a][0], ksa[a], za0);
-                                za1 = fmaf(sacc[u][nt][a][1], ksa[a], za1);
-                                zb0 = fmaf(sacc[u][nt][a][2], ksb[a], zb0);
-                                zb1 = fmaf(sacc[u][nt][a][3], ksb[a], zb1);
-                            }
-                            z[u][nt][0] = okA[u] ? za0 * zs[nt][0] : -INFINITY;
-                            z[u][nt][1] = okA[u] ? za1 * zs[nt][1] : -INFINITY;
-                            z[u][nt][2] = okB[u] ? zb0 * zs[nt][0] : -INFINITY;
-                            z[u][nt][3] = okB[u] ? zb1 * zs[nt][1] : -INFINITY;
-                        }
-                    } else {
-                        const float ksa = ldsf(sks + rA[u] * 4), ksb = ldsf(sks + rB[u] * 4);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            const float s0 = sacc[u][nt][0][0] + sacc[u][nt][1][0];
-                            const float s1 = sacc[u][nt][0][1] + sacc[u][nt][1][1];
-                            const float s2 = sacc[u][nt][0][2] + sacc[u][nt][1][2];
-                            const float s3 = sacc[u][nt][0][3] + sacc[u][nt][1][3];
-                            z[u][nt][0] = okA[u] ? s0 * ksa * zs[nt][0] : -INFINITY;
-                            z[u][nt][1] = okA[u] ? s1 * ksa * zs[nt][1] : -INFINITY;
-                            z[u][nt][2] = okB[u] ? s2 * ksb * zs[nt][0] : -INFINITY;
-                            z[u][nt][3] = okB[u] ? s3 * ksb * zs[nt][1] : -INFINITY;
-                        }
+                        fold(gi);
+                        zero_acc();
                     }
                 }
+                if (!G32) fold(0);
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        z[u][nt][0] = okA[u] ? z[u][nt][0] * zs[nt][0] : -INFINITY;
+                        z[u][nt][1] = okA[u] ? z[u][nt][1] * zs[nt][1] : -INFINITY;
+                        z[u][nt][2] = okB[u] ? z[u][nt][2] * zs[nt][0] : -INFINITY;
+                        z[u][nt][3] = okB[u] ? z[u][nt][3] * zs[nt][1] : -INFINITY;
+                    }
                 // ---- online softmax per head: max over the slice's 32 tokens
                 float pr[2][NT][4];
                 float f[NT][2];
