@@ -47,16 +47,16 @@ kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk
         const int64_t s = num_splits < ceil_div(hint, 16) ? num_splits : ceil_div(hint, 16);
         chunk = ceil_div(ceil_div(hint, s), 16) * 16;
     } else {
-        // Small problems: about one chunk per SM over all (sequence, kv head)
-        // units.  Large ones: chunks of at least 512 tokens, about 16 per SM,
-        // so that the persistent CTAs share the work evenly.
+        // Few (sequence, kv head) units: one chunk per CTA, units * per_unit <=
+        // #SM chunks of equal length.  Many units: 128-token chunks (one
+        // stage), so that the contiguous item blocks of the persistent CTAs
+        // hold equal numbers of stages whatever the length mix.
         const int64_t units = static_cast<int64_t>(B > 0 ? B : 1) * Hk;
-        int64_t per_unit = num_sms / units;
-        if (per_unit < 1) per_unit = 1;
-        chunk = ceil_div(ceil_div(hint, per_unit), 16) * 16;
-        if (chunk > 1024) {
-            chunk = ceil_div(ceil_div(static_cast<int64_t>(hint) * units, 16ll * num_sms), 16) * 16;
-            if (chunk < 512) chunk = 512;
+        const int64_t per_unit = num_sms / units;
+        if (per_unit >= 8) {
+            chunk = ceil_div(ceil_div(hint, per_unit), 16) * 16;
+        } else {
+            chunk = 128;
         }
         const int64_t cap = ceil_div(hint, 16) * 16;
         if (chunk > cap) chunk = cap;

@@ -69,7 +69,10 @@ namespace {
 
 constexpr int NW = 8;                  // consumer warps per CTA
 constexpr int NCONS = NW * 32;         // consumer threads
-constexpr int NTHREADS = NCONS + 32;   // + the producer warp
+// producer warps: one; two for paged caches (K pages and V pages), whose
+// stages take sixteen page copies
+constexpr int nprod(bool paged) { return paged ? 2 : 1; }
+constexpr int nthreads(bool paged) { return NCONS + 32 * nprod(paged); }
 constexpr int WPG = 4;                 // consumer warps per group (a group works one stage)
 constexpr int TT = 32 * WPG;           // tokens per stage: one 32-token slice per warp of a group
 constexpr int kMaxB = 1024;            // sequences whose lengths are cached in shared memory
@@ -204,7 +207,7 @@ __device__ __forceinline__ Seg seg_at(int i, int iend, const int* lens, const in
 }
 
 template <int D, bool G32, bool PAGED, bool G16>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(nthreads(PAGED), 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ DecodeParams prm) {
     using Lay = Layout<D, G32, G16>;
@@ -254,9 +257,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         ptx::prefetch_tensormap(&tm_v);
 #pragma unroll 1
         for (int s = 0; s < NST; ++s) {
-            // the producer's expect_tx arrival (+ one cp.async arrival per lane
-            // of the producer warp for the paged scales)
-            ptx::mbar_init(bar_full + 8 * s, PAGED ? 1 + 32 : 1);
+            // the producer's expect_tx arrival (paged: one per producer warp, plus
+            // one cp.async arrival per lane of producer warp 0 for the scales)
+            ptx::mbar_init(bar_full + 8 * s, PAGED ? 2 + 32 : 1);
             ptx::mbar_init(bar_empty + 8 * s, WPG);
         }
         *abort_flag = 0;
@@ -270,7 +273,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int64_t cap = PAGED ? static_cast<int64_t>(prm.max_pages) * prm.page_size : prm.max_seq;
         const int64_t lim = min(cap, static_cast<int64_t>(prm.splits) * prm.chunk);
 #pragma unroll 1
-        for (int b = tid; b < prm.B; b += NTHREADS) {
+        for (int b = tid; b < prm.B; b += nthreads(PAGED)) {
             int L = prm.seq_lens[b];
             if (L < 0 || L > lim) {
                 if (blockIdx.x == 0) raise_flag(prm.d_err, KVQ_DEVERR_LEN);
@@ -320,7 +323,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     };
 
     // ------------------------------------------------------------ producer
-    if (warp == 0) {
+    if (warp < nprod(PAGED)) {
+        const int pw = warp;            // producer warp index
         // one lane issues every copy of a stage (TMA tiles for K and V, 1-D bulk
         // copies for the scales and the query rows); all complete on the stage's
         // mbarrier, whose single arrival is the expect_tx below
@@ -411,7 +415,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         if (with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
                     }
                 } else {
-                    constexpr uint32_t PAGE_BYTES = 2 * 16 * D;   // TMA bytes (scales by cp.async)
+                    constexpr uint32_t PAGE_BYTES = 16 * D;   // TMA bytes of K (or V) per page
                     const int np = (ntok + 15) >> 4;
                     if ((tt0 >> 4) >= pbase + 32) {
                         pbase += 32;
@@ -422,6 +426,16 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     int32_t pg = __shfl_sync(0xffffffffu, pg_cur, (tt0 >> 4) - pbase + (lane & 7));
                     if (lane >= np) pg = -1;
                     const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
+                    if (pw == 1) {
+                        // producer warp 1: the V rows of the pages (lane q < 8 loads
+                        // page q: 16 rows of this kv head), its own byte count
+                        if (lane == 0) ptx::mbar_arrive_expect_tx(full, __popc(valid) * PAGE_BYTES);
+                        __syncwarp();
+                        if (pg >= 0)
+                            ptx::tma_load_2d(sv + lane * 16 * D, &tm_v, 0, (pg * Hk + hk) * 16, full,
+                                             pol);
+                        continue;
+                    }
                     if (lane == 0) {
                         // the consumers mask the tokens of pages that were not
                         // loaded; a bad table entry is reported here
@@ -432,15 +446,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         if (with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
                     }
                     __syncwarp();
-                    // lane q < 8 loads page q's K and V rows (16 rows of this kv
-                    // head per page); every lane copies 16-byte chunks of the
-                    // pages' scales (16 * NG aligned floats per page), chunk c of
-                    // the stage being page c / (4 NG)
-                    if (pg >= 0) {
-                        const int y = (pg * Hk + hk) * 16;
-                        ptx::tma_load_2d(sk + lane * 16 * D, &tm_k, 0, y, full, pol);
-                        ptx::tma_load_2d(sv + lane * 16 * D, &tm_v, 0, y, full, pol);
-                    }
+                    // producer warp 0: lane q < 8 loads page q's K rows; every lane
+                    // copies 16-byte chunks of the pages' scales (16 * NG aligned
+                    // floats per page), chunk c of the stage being page c / (4 NG)
+                    if (pg >= 0)
+                        ptx::tma_load_2d(sk + lane * 16 * D, &tm_k, 0, (pg * Hk + hk) * 16, full, pol);
 #pragma unroll
                     for (int it = 0; it < NG; ++it) {
                         const int c = lane + 32 * it;
@@ -471,8 +481,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     // to group c % 2), so two stages are in work at once.  Inside a stage,
     // warp wg of the group owns rows [32 wg, 32 wg + 32) as two 16-token MMA
     // tiles u = 0, 1 that share one online-softmax step.
-    const int cw = warp - 1;            // consumer warp index
-    const int ctid = tid - 32;          // consumer thread index
+    const int cw = warp - nprod(PAGED);            // consumer warp index
+    const int ctid = tid - 32 * nprod(PAGED);      // consumer thread index
     const int grp = cw / WPG, wg = cw % WPG;
     const int sig_g = sigma(g);
     const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
@@ -874,17 +884,19 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const int h = 8 * nt + 2 * t + c;
-                    float mw[NW];
-                    float M = -INFINITY;
+                    float mw[NW], lw[NW];
 #pragma unroll
                     for (int w = 0; w < NW; ++w) {
                         mw[w] = mrg_m[w * 16 + h];
-                        M = fmaxf(M, mw[w]);
+                        lw[w] = mrg_l[w * 16 + h];
                     }
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int w = 0; w < NW; ++w) M = fmaxf(M, mw[w]);
                     float Ls = 0.f;
 #pragma unroll
                     for (int w = 0; w < NW; ++w)
-                        if (mw[w] != -INFINITY) Ls = fmaf(mrg_l[w * 16 + h], ptx::ex2(mw[w] - M), Ls);
+                        Ls += mw[w] == -INFINITY ? 0.f : lw[w] * ptx::ex2(mw[w] - M);
                     const float f = (m[nt][c] == -INFINITY) ? 0.f : ptx::ex2(m[nt][c] - M) * down;
                     fo[nt][c] = final_rows ? (Ls > 0.f ? f * __frcp_rn(Ls) : 0.f) : f;
                     if (cw == 0 && g == 0) {
@@ -904,9 +916,12 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         slot[((mt * NT + nt) * 4 + e) * 32] = o[mt][nt][e] * fo[nt][e & 1];
         }
         ptx::named_bar_sync(1, NCONS);
-        // sum the eight slots position by position and write the rows
-#pragma unroll 1
-        for (int pos = ctid; pos < NV * 32; pos += NCONS) {
+        // sum the eight slots position by position and write the rows (all
+        // loads of a thread's positions issued together)
+        static_assert((NV * 32) % NCONS == 0, "positions per consumer thread");
+#pragma unroll
+        for (int it = 0; it < NV * 32 / NCONS; ++it) {
+            const int pos = ctid + it * NCONS;
             const int v = pos >> 5, ln = pos & 31;
             const int pg_ = ln >> 2, pt = ln & 3;
             const int mt = v / (NT * 4), nt = (v / 4) % NT, e = v & 3;
@@ -1003,7 +1018,7 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid, 1, 1);
-    cfg.blockDim = dim3(NTHREADS, 1, 1);
+    cfg.blockDim = dim3(nthreads(PAGED), 1, 1);
     cfg.dynamicSmemBytes = Lay::SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

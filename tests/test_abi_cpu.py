@@ -69,15 +69,19 @@ def test_decode_plan_covers_hint(kvq, B, Hk, hint, ns):
 
 
 def test_decode_plan_fills_the_machine(kvq):
-    # few (sequence, kv head) units and a short cache: about one chunk per SM
+    # few (sequence, kv head) units: one equal chunk per CTA, at most one per SM
     chunk, splits = kvq.kvq_decode_plan(1, 8, 4097, 0, num_sms=148)
     assert (chunk, splits) == (240, 18) and 8 * splits <= 148
-    # long cache: chunks of >= 512 tokens, about 16 per SM
     chunk, splits = kvq.kvq_decode_plan(1, 8, 131073, 0, num_sms=148)
-    assert chunk == 512 and splits == 257
-    # many units: still >= 512-token chunks that spread over the persistent CTAs
+    assert (chunk, splits) == (7296, 18) and 8 * splits <= 148
+    # many units: one-stage (128-token) chunks balance the CTAs' blocks
     chunk, splits = kvq.kvq_decode_plan(37, 8, 16385, 0, num_sms=148)
-    assert chunk % 16 == 0 and chunk >= 512 and splits == -(-16385 // chunk)
+    assert chunk == 128 and splits == -(-16385 // 128)
+    chunk, splits = kvq.kvq_decode_plan(16, 8, 8193, 0, num_sms=148)
+    assert chunk == 128 and splits == 65
+    # the split count stays bounded for very long caches
+    chunk, splits = kvq.kvq_decode_plan(64, 8, 10_000_000, 0, num_sms=148)
+    assert splits <= 4096 and chunk % 16 == 0
     # explicit split counts are honoured up to the 16-token rounding of the chunk
     chunk, splits = kvq.kvq_decode_plan(1, 8, 4097, 64, num_sms=148)
     assert 16 < splits <= 64

@@ -211,3 +211,21 @@ def test_decode_full_cache_unaligned_capacity(mode, D, S):
         out = c.decode(q, sl, S, attn_scale=f32_scale(D), num_splits=ns)
         assert_attn_close(out, c.oracle_decode(q, sl, f32_scale(D)), f"S={S} ns={ns}")
     assert kvq().kvq_read_error(c.err) == 0
+
+
+
+def test_one_workspace_serves_calls_of_any_shape():
+    """One workspace, reused across calls of different shapes and split counts,
+    gives the oracle's answer every time (its contents on entry are ignored)."""
+    m = kvq()
+    ws = torch.full((8 << 20,), 0xFF, dtype=torch.uint8, device="cuda")   # NaN bit patterns
+    cases = [(2, 8, 2, 128, "per_token", [1000, 333]), (3, 16, 2, 64, "group32", [517, 1, 130]),
+             (1, 32, 8, 128, "per_token", [4097])]
+    for rep in range(2):
+        for i, (B, Hq, Hk, D, mode, lens) in enumerate(cases):
+            c, q = _fill_contig(B, Hq, Hk, D, mode, lens, seed=100 + i)
+            sl = torch.tensor(lens, dtype=torch.int32)
+            need = m.kvq_decode_workspace_bytes(B, Hq, Hk, D, max(lens), 7)
+            assert 0 < need <= ws.numel()
+            out = c.decode(q, sl, max(lens), attn_scale=f32_scale(D), num_splits=7, workspace=ws)
+            assert_attn_close(out, c.oracle_decode(q, sl, f32_scale(D)), f"case {i} rep {rep}")
