@@ -13,7 +13,6 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 constexpr int kMaxSplits = 4096;     // bound on splits per sequence (combine smem)
-constexpr int kMaxBatch = 1024;      // sequences per decode call (split kernel smem)
 
 kvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
 
@@ -71,7 +70,7 @@ kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk
 
 size_t workspace_for(int B, int Hq, int D, int splits) {
     if (splits <= 1) return 0;
-    return static_cast<size_t>(B) * Hq * splits * (D + 2) * sizeof(float);
+    return kvq::kHdrBytes + static_cast<size_t>(B) * Hq * splits * (D + 2) * sizeof(float);
 }
 
 }  // namespace
@@ -157,7 +156,7 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
     if (D != 64 && D != 128) return KVQ_ERR_UNSUPPORTED;
     if (G > 16) return KVQ_ERR_UNSUPPORTED;
     // the split kernel keeps every sequence length in shared memory
-    if (B > kMaxBatch) return KVQ_ERR_UNSUPPORTED;
+    if (B > kvq::kMaxBatch) return KVQ_ERR_UNSUPPORTED;
     // TMA row coordinates are 32-bit
     const int64_t rows = kv->page_size ? static_cast<int64_t>(kv->num_pages) * Hk * 16
                                        : static_cast<int64_t>(B) * Hk * kv->max_seq;
@@ -175,8 +174,11 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
     kvq::DecodeParams p{};
     p.q = q; p.k = kv->k; p.v = kv->v; p.k_scale = kv->k_scale; p.v_scale = kv->v_scale;
     p.table = kv->page_table; p.seq_lens = d_seq_lens; p.out = out; p.d_err = d_err;
-    float* ws = static_cast<float*>(workspace);
+    // [partition header: kHdrBytes][o: n_part * D][m: n_part][l: n_part]
+    float* ws = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kvq::kHdrBytes)
+                          : nullptr;
     const size_t n_part = static_cast<size_t>(B) * Hq * splits;
+    p.ws_hdr = static_cast<int*>(workspace);
     p.ws_o = ws;
     p.ws_m = ws ? ws + n_part * D : nullptr;
     p.ws_l = ws ? ws + n_part * (D + 1) : nullptr;

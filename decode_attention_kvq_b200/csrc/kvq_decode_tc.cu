@@ -17,10 +17,11 @@
 //    (T / grid each, the first T % grid CTAs one more), found from a prefix
 //    sum of the per-sequence chunk counts (lengths cached in shared memory).
 //    The items of one (b, kv head) inside a CTA's block form a segment: one
-//    token range, one softmax state.  A segment that is a whole sequence
-//    writes the final rows, any other writes one partial state (o, m, l)
-//    into the slot of its first chunk and marks the slots of its other
-//    chunks empty for the combine kernel (kvq_decode.cu).
+//    token range, one softmax state.  A segment that is a whole (b, kv head)
+//    writes the final rows; any other writes one partial state (o, m, l)
+//    into the workspace slot of its first chunk.  CTA 0 publishes the
+//    partition (item prefix sums, chunk counts), from which the combine
+//    kernel (kvq_decode.cu) finds the slots that hold a unit's partials.
 //  * CTA = 1 producer warp (warp 0) + 8 consumer warps.  One producer lane
 //    streams 128-token stages into a ring of 3-8 stages (~150-220 KB of
 //    shared memory, one CTA per SM): K and V bytes by TMA tile loads (2-D
@@ -75,7 +76,7 @@ constexpr int nprod(bool paged) { return paged ? 2 : 1; }
 constexpr int nthreads(bool paged) { return NCONS + 32 * nprod(paged); }
 constexpr int WPG = 4;                 // consumer warps per group (a group works one stage)
 constexpr int TT = 32 * WPG;           // tokens per stage: one 32-token slice per warp of a group
-constexpr int kMaxB = 1024;            // sequences whose lengths are cached in shared memory
+constexpr int kMaxB = kMaxBatch;       // sequences whose lengths are cached in shared memory
 
 // Row (inside an 8-token half of a slice) that holds MMA row r of the K
 // operand and MMA k-index r of the V operand: sigma = {0, 2, 4, 6, 3, 1, 7, 5}.
@@ -308,6 +309,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     // CTA c takes items [c*q + min(c, r), ...) with q = T / grid, r = T % grid
     // (the first r CTAs one item more); T < 2^31 is checked by the host
     const int T = cum[B];
+    if (blockIdx.x == 0 && p.splits > 1) {
+        // publish the partition for the combine kernel: T, the item prefix sums
+        // and the chunk counts (it finds each unit's partials from them)
+        int* hdr = p.ws_hdr;
+        if (tid == 0) hdr[0] = T;
+        for (int b = tid; b <= B; b += nthreads(PAGED)) hdr[2 + b] = cum[b];
+        for (int b = tid; b < B; b += nthreads(PAGED)) hdr[2 + kMaxB + 1 + b] = nsv[b];
+    }
     const int ibeg = static_cast<int>(blockIdx.x) * (T / static_cast<int>(gridDim.x)) +
                      min(static_cast<int>(blockIdx.x), T % static_cast<int>(gridDim.x));
     const int iend = ibeg + T / static_cast<int>(gridDim.x) +
@@ -854,10 +863,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (lane == 0) ptx::mbar_arrive(bar_empty + 8 * s);
         }
 
-        // ---- merge the eight warps' states of the segment (one round)
-        // a segment that is the whole sequence writes the final rows (and,
-        // when the sequence has several chunks, a marker l = -1 in slot 0 that
-        // tells the combine kernel to leave them alone)
+        // ---- merge the eight warps' states of the segment (one round); a
+        // segment that is the whole (b, kv head) writes the final rows
         const bool final_rows = sg.j0 == 0 && sg.j1 == sg.ns - 1;
         const int seg_j0 = sg.j0;
 #pragma unroll
@@ -936,22 +943,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (final_rows) p.out[row * D + d] = sum;
             else p.ws_o[(row * p.splits + seg_j0) * D + d] = sum;
         }
-        // the partial's (m, l) and the empty markers of the chunks merged into
-        // slot seg_j0, or the finished marker (l = -1 in slot 0)
-        if (!final_rows || sg.ns > 1) {
-            const int nrow = final_rows ? 1 : sg.j1 - seg_j0 + 1;
-#pragma unroll 1
-            for (int idx = ctid; idx < G * nrow; idx += NCONS) {
-                const int k = idx / G, h = idx - k * G;
-                float* const wm = p.ws_m + (bh0 + h) * p.splits + seg_j0 + k;
-                float* const wl = p.ws_l + (bh0 + h) * p.splits + seg_j0 + k;
-                if (final_rows) {
-                    *wl = -1.f;
-                } else {
-                    *wm = k == 0 ? seg_M[h] : -INFINITY;
-                    *wl = k == 0 ? seg_L[h] : 0.f;
-                }
-            }
+        // the partial's (m, l), in the slot of the segment's first chunk
+        if (!final_rows && ctid < G) {
+            p.ws_m[(bh0 + ctid) * p.splits + seg_j0] = seg_M[ctid];
+            p.ws_l[(bh0 + ctid) * p.splits + seg_j0] = seg_L[ctid];
         }
     }
 }

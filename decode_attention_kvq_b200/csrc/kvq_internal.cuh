@@ -55,6 +55,7 @@ struct DecodeParams {
     float* ws_o;             // [B*Hq, splits, D] partial outputs (unnormalised)
     float* ws_m;             // [B*Hq, splits] running max (log2 domain)
     float* ws_l;             // [B*Hq, splits] running sum
+    int* ws_hdr;             // the split kernel's partition: T, -, cum[kMaxB + 1], ns[kMaxB]
     int32_t* d_err;
     int B, Hq, Hk, G, D;
     int group32;
@@ -64,6 +65,11 @@ struct DecodeParams {
     int grid;                // persistent CTAs of the split kernel
     float scale_log2;        // attn_scale * log2(e)
 };
+// Split-K workspace: the partition header (written by the split kernel, read
+// by the combine kernel), then the partials.
+constexpr int kMaxBatch = 1024;                              // sequences per call
+constexpr int kHdrInts = 2 + (kMaxBatch + 1) + kMaxBatch;    // T, unused, cum, ns
+constexpr size_t kHdrBytes = (kHdrInts * 4 + 255) / 256 * 256;
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 // tensor-core split kernel (kvq_decode_tc.cu)
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s);
