@@ -167,7 +167,7 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
     kvq_status st = plan(B, Hk, max_seq_len_hint, num_splits, 0, &chunk, &splits);
     if (st != KVQ_OK) return st;
     // work items (sequence, kv head, chunk) are counted in 32-bit integers
-    if (static_cast<int64_t>(B) * Hk * splits >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(B) * Hk * (splits + 3) >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
     const size_t need = workspace_for(B, Hq, D, splits);
     if (need > 0 && (!workspace || workspace_bytes < need)) return KVQ_ERR_INVALID_ARG;
 
@@ -192,8 +192,13 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
             return KVQ_ERR_CUDA;
         const int64_t items = static_cast<int64_t>(B) * Hk * splits;
         p.grid = static_cast<int>(items < sms ? items : sms);   // persistent: one CTA per SM
+        if (p.grid > kvq::kMaxGrid) p.grid = kvq::kMaxGrid;
     }
     p.scale_log2 = attn_scale * 1.4426950408889634f;
+    // one-stage chunks (many units): a CTA pays about three stages of time
+    // for every (sequence, kv head) it starts (merge, query set-up), so each
+    // unit start weighs three items when the items are divided among the CTAs
+    p.seg_w = chunk <= 128 ? 3 : 0;
     return from_cuda(kvq::launch_decode(p, static_cast<cudaStream_t>(stream)));
 }
 

@@ -308,19 +308,50 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     __syncthreads();
     // CTA c takes items [c*q + min(c, r), ...) with q = T / grid, r = T % grid
     // (the first r CTAs one item more); T < 2^31 is checked by the host
+    // ---- the CTA's block of items.  Every (sequence, kv head) unit weighs its
+    // items plus W, the cost of starting it; CTA c takes the equal share
+    // [c * TW / grid, (c + 1) * TW / grid) of the total weight TW (the first
+    // TW % grid CTAs one more), mapped back to items.
     const int T = cum[B];
-    if (blockIdx.x == 0 && p.splits > 1) {
-        // publish the partition for the combine kernel: T, the item prefix sums
-        // and the chunk counts (it finds each unit's partials from them)
+    const int W = p.seg_w;
+    const int HkW = p.Hk * W;
+    const int TW = T + HkW * B;
+    auto item_of = [&](int x) {          // first item at or after weight position x
+        if (x >= TW) return T;
+        int lo = 0, hi = B;              // largest b with wcum(b) <= x
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (cum[mid] + HkW * mid <= x) lo = mid;
+            else hi = mid;
+        }
+        const int per = max(nsv[lo], 1);
+        const int r = x - (cum[lo] + HkW * lo);
+        const int hk = r / (per + W);
+        const int jw = r - hk * (per + W);
+        return cum[lo] + hk * per + max(jw - W, 0);
+    };
+    const int grid = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    const int wq = TW / grid, wr = TW % grid;
+    const int ibeg = W ? item_of(c * wq + min(c, wr)) : c * wq + min(c, wr);
+    const int iend = W ? item_of((c + 1) * wq + min(c + 1, wr)) : (c + 1) * wq + min(c + 1, wr);
+    if (p.splits > 1) {
+        // publish the partition for the combine kernel: T, the item prefix sums,
+        // the chunk counts and every CTA's first item (it finds each unit's
+        // partials from them); written by a consumer thread, off the producer's
+        // path to its first load
         int* hdr = p.ws_hdr;
-        if (tid == 0) hdr[0] = T;
-        for (int b = tid; b <= B; b += nthreads(PAGED)) hdr[2 + b] = cum[b];
-        for (int b = tid; b < B; b += nthreads(PAGED)) hdr[2 + kMaxB + 1 + b] = nsv[b];
+        if (tid == 32) {
+            if (W) hdr[kHdrStart + c] = ibeg;
+            if (c == 0) {
+                hdr[0] = T;
+                hdr[kHdrStart + grid] = T;
+            }
+        }
+        if (c == 0) {
+            for (int b = tid; b <= B; b += nthreads(PAGED)) hdr[kHdrCum + b] = cum[b];
+            for (int b = tid; b < B; b += nthreads(PAGED)) hdr[kHdrNs + b] = nsv[b];
+        }
     }
-    const int ibeg = static_cast<int>(blockIdx.x) * (T / static_cast<int>(gridDim.x)) +
-                     min(static_cast<int>(blockIdx.x), T % static_cast<int>(gridDim.x));
-    const int iend = ibeg + T / static_cast<int>(gridDim.x) +
-                     (static_cast<int>(blockIdx.x) < T % static_cast<int>(gridDim.x) ? 1 : 0);
 
     // bounded wait that gives up at once after any earlier timeout of this CTA
     auto wait = [&](uint32_t bar, uint32_t parity) {

@@ -55,7 +55,7 @@ struct DecodeParams {
     float* ws_o;             // [B*Hq, splits, D] partial outputs (unnormalised)
     float* ws_m;             // [B*Hq, splits] running max (log2 domain)
     float* ws_l;             // [B*Hq, splits] running sum
-    int* ws_hdr;             // the split kernel's partition: T, -, cum[kMaxB + 1], ns[kMaxB]
+    int* ws_hdr;             // the split kernel's partition: T, -, cum, ns, CTA starts
     int32_t* d_err;
     int B, Hq, Hk, G, D;
     int group32;
@@ -63,12 +63,17 @@ struct DecodeParams {
     int chunk;               // KV tokens per split
     int splits;              // chunks of the longest sequence
     int grid;                // persistent CTAs of the split kernel
+    int seg_w;               // partition weight of a (sequence, kv head) start, in items
     float scale_log2;        // attn_scale * log2(e)
 };
 // Split-K workspace: the partition header (written by the split kernel, read
 // by the combine kernel), then the partials.
 constexpr int kMaxBatch = 1024;                              // sequences per call
-constexpr int kHdrInts = 2 + (kMaxBatch + 1) + kMaxBatch;    // T, unused, cum, ns
+constexpr int kMaxGrid = 1024;                               // persistent CTAs
+constexpr int kHdrCum = 2;                                   // [kMaxBatch + 1] item prefix sums
+constexpr int kHdrNs = kHdrCum + kMaxBatch + 1;              // [kMaxBatch] chunk counts
+constexpr int kHdrStart = kHdrNs + kMaxBatch;                // [grid + 1] first item of CTA c
+constexpr int kHdrInts = kHdrStart + kMaxGrid + 1;
 constexpr size_t kHdrBytes = (kHdrInts * 4 + 255) / 256 * 256;
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 // tensor-core split kernel (kvq_decode_tc.cu)
