@@ -32,6 +32,7 @@ decode_combine_even(DecodeParams p) {
     __shared__ float s_m[kWarps], s_l[kWarps];
     __shared__ __align__(16) float s_acc[kWarps][128];
     grid_dep_wait();                    // the split kernel's partials are complete
+    grid_dep_launch();                  // the next kernel may run its prologue now
     const int64_t bh = blockIdx.x;
     const int b = static_cast<int>(bh / p.Hq);
     const int hk = static_cast<int>(bh % p.Hq) / p.G;
@@ -172,6 +173,7 @@ decode_combine_weighted(DecodeParams p) {
     extern __shared__ int s_dyn[];
     int* const s_start = s_dyn;                 // [grid + 1]
     grid_dep_wait();                    // the split kernel's partials are complete
+    grid_dep_launch();                  // the next kernel may run its prologue now
     const int64_t bh = blockIdx.x;
     const int b = static_cast<int>(bh / p.Hq);
     const int hk = static_cast<int>(bh % p.Hq) / p.G;

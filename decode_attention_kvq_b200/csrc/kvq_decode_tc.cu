@@ -622,18 +622,22 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     for (int c = 0; c < NCG; ++c) csq[nt][c] = 0;
 #pragma unroll
                     for (int gi = 0; gi < NGRP; ++gi) {
-                        uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+                        uint32_t qi[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            const int qi = min(max(__float2int_rn(qf[gi][e] * up), -32767), 32767);
-                            csq[nt][G32 ? gi : 0] += qi;
-                            hw[e >> 2] |= (static_cast<uint32_t>(qi >> 8) & 0xffu) << (8 * (e & 3));
-                            lw[e >> 2] |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * (e & 3));
+                            const int v = min(max(__float2int_rn(qf[gi][e] * up), -32767), 32767);
+                            csq[nt][G32 ? gi : 0] += v;
+                            qi[e] = static_cast<uint32_t>(v);
                         }
-                        qh0[nt][gi] = hw[0];
-                        qh1[nt][gi] = hw[1];
-                        ql0[nt][gi] = lw[0];
-                        ql1[nt][gi] = lw[1];
+                        // byte 1 (hi digit) and byte 0 (lo digit) of four values each
+                        auto pick4 = [&](int e0, uint32_t sel2) {
+                            return ptx::prmt(ptx::prmt(qi[e0], qi[e0 + 1], sel2),
+                                             ptx::prmt(qi[e0 + 2], qi[e0 + 3], sel2), 0x5410u);
+                        };
+                        qh0[nt][gi] = pick4(0, 0x0051u);
+                        qh1[nt][gi] = pick4(4, 0x0051u);
+                        ql0[nt][gi] = pick4(0, 0x0040u);
+                        ql1[nt][gi] = pick4(4, 0x0040u);
                     }
 #pragma unroll
                     for (int c = 0; c < NCG; ++c) {
