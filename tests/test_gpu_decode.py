@@ -229,3 +229,25 @@ def test_one_workspace_serves_calls_of_any_shape():
             assert 0 < need <= ws.numel()
             out = c.decode(q, sl, max(lens), attn_scale=f32_scale(D), num_splits=7, workspace=ws)
             assert_attn_close(out, c.oracle_decode(q, sl, f32_scale(D)), f"case {i} rep {rep}")
+
+
+@pytest.mark.parametrize("mode", ["per_token", "group32"])
+@pytest.mark.parametrize("num_splits,top", [(0, 4100), (40, 4100), (300, 4100), (0, 2000)])
+def test_decode_many_units_ragged_with_empty_sequences(mode, num_splits, top):
+    """Many (sequence, kv head) units of very different lengths, some empty:
+    one-stage chunks, the weighted CTA partition, units split over several
+    CTAs and units finished inside one, and both combine paths (up to 32 slots
+    in one round of loads, more through the slot list)."""
+    import random
+    rnd = random.Random(num_splits + (7 if mode == "group32" else 0))
+    B, Hk, G, D = 40, 4, 2, 64
+    lens = [rnd.choice([0, 1, 17, 130, 600, 2000, top]) for _ in range(B)]
+    lens[3] = 0
+    c, q = _fill_contig(B, Hk * G, Hk, D, mode, lens, seed=90 + num_splits)
+    sl = torch.tensor(lens, dtype=torch.int32)
+    out = c.decode(q, sl, max(lens), attn_scale=f32_scale(D), num_splits=num_splits).cpu()
+    assert_attn_close(out, c.oracle_decode(q, sl, f32_scale(D)), f"splits={num_splits} {mode}")
+    for b, L in enumerate(lens):
+        if L == 0:
+            assert torch.all(out[b] == 0)
+    assert kvq().kvq_read_error(c.err) == 0
