@@ -193,12 +193,13 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
         const int64_t items = static_cast<int64_t>(B) * Hk * splits;
         p.grid = static_cast<int>(items < sms ? items : sms);   // persistent: one CTA per SM
         if (p.grid > kvq::kMaxGrid) p.grid = kvq::kMaxGrid;
+        p.one_item = items <= p.grid ? 1 : 0;
     }
     p.scale_log2 = attn_scale * 1.4426950408889634f;
     // one-stage chunks (many units): a CTA pays about three stages of time
     // for every (sequence, kv head) it starts (merge, query set-up), so each
     // unit start weighs three items when the items are divided among the CTAs
-    p.seg_w = chunk <= 128 ? 3 : 0;
+    p.seg_w = (chunk <= 128 && !p.one_item) ? 3 : 0;
     return from_cuda(kvq::launch_decode(p, static_cast<cudaStream_t>(stream)));
 }
 

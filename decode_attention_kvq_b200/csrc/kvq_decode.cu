@@ -24,6 +24,99 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kBatch = 8;                       // slots in flight per warp
 
+// One item per CTA (one_item): CTA c of the split kernel held item c of the
+// plan, so chunk j < ns of every unit holds a partial and nothing else does.
+// One CTA per (b, q head); lane l of a warp owns head_dim [4l, 4l + 4).
+__global__ void __launch_bounds__(kThreads)
+decode_combine_one(DecodeParams p) {
+    __shared__ float s_m[kWarps], s_l[kWarps];
+    __shared__ __align__(16) float s_acc[kWarps][128];
+    grid_dep_wait();                    // the split kernel's partials are complete
+    grid_dep_launch();                  // the next kernel may run its prologue now
+    const int64_t bh = blockIdx.x;
+    const int b = static_cast<int>(bh / p.Hq);
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const float* m = p.ws_m + bh * p.splits;
+    const float* lv = p.ws_l + bh * p.splits;
+    const int D = p.D;
+    const bool active = lane * 4 < D;
+    const float* o = p.ws_o + bh * p.splits * D + lane * 4;
+    const int64_t cap = p.page_size ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
+    const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
+    const int L0 = p.seq_lens[b];
+
+    float Mw = -INFINITY, lw = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float mj[kBatch], lj[kBatch];
+    float4 oj[kBatch];
+    auto load = [&](int k0) {                   // slots k0 + u * kWarps
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int j = k0 + u * kWarps;
+            const bool in = j < p.splits;
+            mj[u] = in ? m[j] : -INFINITY;
+            lj[u] = in ? lv[j] : 0.f;
+            oj[u] = (in && active) ? *reinterpret_cast<const float4*>(o + static_cast<int64_t>(j) * D)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto fold = [&](int k0, int ns) {           // slots past the chunk count are dropped
+        float Mn = Mw;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            if (k0 + u * kWarps >= ns) mj[u] = -INFINITY;
+            Mn = fmaxf(Mn, mj[u]);
+        }
+        if (Mn == -INFINITY) return;
+        const float a = exp2f(Mw - Mn);                   // 0 while Mw is -inf
+        acc.x *= a; acc.y *= a; acc.z *= a; acc.w *= a;
+        lw *= a;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            if (mj[u] == -INFINITY) continue;             // no weight: o not used
+            const float wj = exp2f(mj[u] - Mn);
+            acc.x = fmaf(wj, oj[u].x, acc.x);
+            acc.y = fmaf(wj, oj[u].y, acc.y);
+            acc.z = fmaf(wj, oj[u].z, acc.z);
+            acc.w = fmaf(wj, oj[u].w, acc.w);
+            lw = fmaf(wj, lj[u], lw);
+        }
+        Mw = Mn;
+    };
+    // the first round of loads is issued together with the length
+    load(w);
+    const int L = (L0 < 0 || L0 > lim) ? 0 : L0;
+    const int ns = (L + p.chunk - 1) / p.chunk;
+    if (ns <= 1) return;                        // finished by the split kernel
+    fold(w, ns);
+#pragma unroll 1
+    for (int k0 = w + kWarps * kBatch; k0 < ns; k0 += kWarps * kBatch) {
+        load(k0);
+        fold(k0, ns);
+    }
+    if (lane == 0) {
+        s_m[w] = Mw;
+        s_l[w] = lw;
+    }
+    if (active) *reinterpret_cast<float4*>(&s_acc[w][lane * 4]) = acc;
+    __syncthreads();
+    float M = s_m[0];
+#pragma unroll
+    for (int x = 1; x < kWarps; ++x) M = fmaxf(M, s_m[x]);
+    float f[kWarps], lsum = 0.f;
+#pragma unroll
+    for (int x = 0; x < kWarps; ++x) {
+        f[x] = s_m[x] == -INFINITY ? 0.f : exp2f(s_m[x] - M);
+        lsum = fmaf(f[x], s_l[x], lsum);
+    }
+    for (int d = tid; d < D; d += kThreads) {
+        float sum = 0.f;
+#pragma unroll
+        for (int x = 0; x < kWarps; ++x) sum = fmaf(f[x], s_acc[x][d], sum);
+        p.out[bh * D + d] = lsum > 0.f ? sum / lsum : 0.f;
+    }
+}
+
 // Unweighted partition (seg_w == 0): CTA c of the split kernel starts at item
 // c * (T / grid) + min(c, T % grid), so the live slots follow arithmetically.
 // One CTA per (b, q head); lane l of a warp owns head_dim [4l, 4l + 4).
@@ -330,6 +423,10 @@ cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (p.one_item) {
+        cfg.dynamicSmemBytes = 0;
+        return cudaLaunchKernelEx(&cfg, decode_combine_one, p);
+    }
     if (p.seg_w == 0) {
         cfg.dynamicSmemBytes = 0;
         return cudaLaunchKernelEx(&cfg, decode_combine_even, p);

@@ -269,8 +269,12 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     grid_dep_wait();                    // the predecessor's writes (q, cache, lengths) are visible
     grid_dep_launch();                  // the combine kernel may be scheduled now
 
+    // one item per CTA (the plan's items fit the grid): CTA c takes item c of
+    // the plan, (b, kv head, chunk j) = c in (b, kv head, j) order, whatever the
+    // lengths; the producer issues its first stage before the length arrives
+    const bool one = prm.one_item != 0;
     // ---- lengths and chunk prefix sums (items per sequence: Hk * max(1, chunks))
-    {
+    if (!one) {
         const int64_t cap = PAGED ? static_cast<int64_t>(prm.max_pages) * prm.page_size : prm.max_seq;
         const int64_t lim = min(cap, static_cast<int64_t>(prm.splits) * prm.chunk);
 #pragma unroll 1
@@ -290,7 +294,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const DecodeParams& p = *sprm;
     const int B = p.B;
     const int G = p.G;
-    if (warp == 0) {                    // inclusive scan of cum[1..B] by one warp
+    if (!one && warp == 0) {            // inclusive scan of cum[1..B] by one warp
         int carry = 0;
 #pragma unroll 1
         for (int base = 0; base < B; base += 32) {
@@ -305,7 +309,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         if (lane == 0) cum[0] = 0;
     }
-    __syncthreads();
+    if (!one) __syncthreads();
     // CTA c takes items [c*q + min(c, r), ...) with q = T / grid, r = T % grid
     // (the first r CTAs one item more); T < 2^31 is checked by the host
     // ---- the CTA's block of items.  Every (sequence, kv head) unit weighs its
@@ -332,9 +336,35 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     };
     const int grid = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
     const int wq = TW / grid, wr = TW % grid;
-    const int ibeg = W ? item_of(c * wq + min(c, wr)) : c * wq + min(c, wr);
-    const int iend = W ? item_of((c + 1) * wq + min(c + 1, wr)) : (c + 1) * wq + min(c + 1, wr);
-    if (p.splits > 1) {
+    const int ibeg = one ? c : W ? item_of(c * wq + min(c, wr)) : c * wq + min(c, wr);
+    const int iend = one ? c + 1
+                         : W ? item_of((c + 1) * wq + min(c + 1, wr)) : (c + 1) * wq + min(c + 1, wr);
+    // one item per CTA: the item, and its length read straight from the caller
+    const int one_b = c / max(p.Hk * p.splits, 1);
+    const int one_r = c - one_b * p.Hk * p.splits;
+    const int one_hk = one_r / p.splits, one_j = one_r - one_hk * p.splits;
+    auto one_len = [&]() {
+        const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
+        const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
+        int L = p.seq_lens[one_b];
+        if (L < 0 || L > lim) {
+            if (one_j == 0 && one_hk == 0 && tid == 0) raise_flag(p.d_err, KVQ_DEVERR_LEN);
+            L = 0;
+        }
+        return L;
+    };
+    auto one_seg = [&](int L) {
+        Seg sg;
+        sg.b = one_b;
+        sg.hk = one_hk;
+        sg.j0 = sg.j1 = one_j;
+        sg.ns = (L + p.chunk - 1) / p.chunk;
+        sg.t0 = one_j * p.chunk;
+        sg.t1 = max(sg.t0, min(sg.t0 + p.chunk, L));
+        sg.next = iend;
+        return sg;
+    };
+    if (!one && p.splits > 1) {
         // publish the partition for the combine kernel: T, the item prefix sums,
         // the chunk counts and every CTA's first item (it finds each unit's
         // partials from them); written by a consumer thread, off the producer's
@@ -385,9 +415,15 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         int count = 0;                  // tiles issued (ring position)
 #pragma unroll 1
         for (int i = ibeg; i < iend;) {
-            const Seg sg = seg_at(i, iend, lens, nsv, cum, B, chunk);
+            // one item per CTA: the length load is issued first and used only
+            // after the first stage is on its way (the chunk's end stands in)
+            int Lone = 0;
+            if (one) Lone = one_len();
+            const Seg sg = one ? one_seg((one_j + 1) * chunk) : seg_at(i, iend, lens, nsv, cum, B, chunk);
             i = sg.next;
             if (sg.ns == 0) continue;
+            int t1 = sg.t1;
+            uint32_t spec_valid = ~0u;      // paged, one item: the first stage's loaded pages
             const int b = sg.b, hk = sg.hk;
             const uint16_t* qsrc = qg + (static_cast<int64_t>(b) * Hq + hk * G) * D;
             int seg_tiles = 0;          // tiles issued for this segment
@@ -399,7 +435,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             auto load_pages = [&](int first) {
                 const int idx = first + lane;
                 int32_t v = -1;
-                if (16 * idx < sg.t1) {
+                if (16 * idx < t1 && idx < max_pages) {
                     v = table[static_cast<int64_t>(b) * max_pages + idx];
                     if (v < 0 || v >= num_pages) v = -1;
                 }
@@ -410,12 +446,13 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 pg_nxt = load_pages(pbase + 32);
             }
 #pragma unroll 1
-            for (int tt0 = sg.t0; tt0 < sg.t1; tt0 += TT, ++count, ++seg_tiles) {
+            for (int tt0 = sg.t0; tt0 < t1; tt0 += TT, ++count, ++seg_tiles,
+                     t1 = (one && seg_tiles == 1) ? max(sg.t0, min(sg.t0 + chunk, Lone)) : t1) {
                 const int s = count % NST;
                 const uint32_t full = bar_full + 8 * s;
                 if (count >= NST && lane == 0) wait(bar_empty + 8 * s, ((count / NST) - 1) & 1);
                 __syncwarp();
-                const int ntok = min(TT, sg.t1 - tt0);
+                const int ntok = min(TT, t1 - tt0);
                 const uint32_t sk = sbase + s * Lay::STAGE;
                 const uint32_t sv = sk + Lay::KV_BYTES;
                 const uint32_t sks = sv + Lay::KV_BYTES;
@@ -479,7 +516,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     if (lane == 0) {
                         // the consumers mask the tokens of pages that were not
                         // loaded; a bad table entry is reported here
-                        if (valid != (1u << np) - 1u) raise_flag(d_err, KVQ_DEVERR_PAGE);
+                        // (one item per CTA: the first stage's range is the chunk's, not
+                        // yet the length's; its pages are checked once the length is known)
+                        if (one && seg_tiles == 0) spec_valid = valid;
+                        else if (valid != (1u << np) - 1u) raise_flag(d_err, KVQ_DEVERR_PAGE);
                         sts_u32(sk + Lay::MASK_OFF, valid);
                         ptx::mbar_arrive_expect_tx(
                             full, __popc(valid) * PAGE_BYTES + (with_q ? q_bytes : 0u));
@@ -504,6 +544,12 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     }
                     ptx::cp_async_arrive_noinc(full);
                 }
+            }
+            if (PAGED && one && lane == 0) {
+                // the first stage's pages inside the sequence must all have loaded
+                const int nreal = min(max(t1 - sg.t0, 0), TT);
+                const uint32_t need = nreal >= 16 * 32 ? ~0u : (1u << ((nreal + 15) >> 4)) - 1u;
+                if ((spec_valid & need) != need) raise_flag(d_err, KVQ_DEVERR_PAGE);
             }
         }
         // the last tile of every slot has landed (normally long consumed; after a
@@ -538,11 +584,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 #pragma unroll 1
     for (int i = ibeg; i < iend;) {
-        const Seg sg = seg_at(i, iend, lens, nsv, cum, B, p.chunk);
+        const Seg sg = one ? one_seg(one_len()) : seg_at(i, iend, lens, nsv, cum, B, p.chunk);
         i = sg.next;
         const int b = sg.b, hk = sg.hk;
         const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
-        if (sg.ns == 0) {
+        if (!one && sg.ns == 0) {
             // empty (or rejected) sequence: zero rows
 #pragma unroll 1
             for (int idx = ctid; idx < G * D; idx += NCONS) p.out[bh0 * D + idx] = 0.f;
@@ -566,7 +612,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                   : ((static_cast<uint32_t>(b * p.Hk + hk) * static_cast<uint32_t>(p.max_seq) *
                       static_cast<uint32_t>(NG)) & 3u) * 4u;
         const int t0 = sg.t0, t1 = sg.t1;
-        const int ntiles = (t1 - t0 + TT - 1) / TT;
+        // one item per CTA: at least the one stage the producer issued before
+        // it knew the length
+        const int ntiles = max(one ? 1 : 0, (t1 - t0 + TT - 1) / TT);
 #pragma unroll 1
         for (int it = 0; it < ntiles; ++it, ++c_count) {
             if ((c_count & 1) != grp) continue;           // the other group's stage
@@ -900,7 +948,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
         // ---- merge the eight warps' states of the segment (one round); a
         // segment that is the whole (b, kv head) writes the final rows
-        const bool final_rows = sg.j0 == 0 && sg.j1 == sg.ns - 1;
+        // (one item per CTA: the final rows of a one-chunk or empty sequence come
+        // from its chunk 0; chunks past the length write nothing)
+        const bool final_rows = one ? sg.j0 == 0 && sg.ns <= 1 : sg.j0 == 0 && sg.j1 == sg.ns - 1;
+        const bool part_rows = one ? sg.ns > 1 && sg.j0 < sg.ns : !final_rows;
         const int seg_j0 = sg.j0;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -976,10 +1027,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                               : (D == 128 ? 16 : 8) * pg_ + 2 * mt + (e >> 1);
             const int64_t row = bh0 + h;
             if (final_rows) p.out[row * D + d] = sum;
-            else p.ws_o[(row * p.splits + seg_j0) * D + d] = sum;
+            else if (part_rows) p.ws_o[(row * p.splits + seg_j0) * D + d] = sum;
         }
         // the partial's (m, l), in the slot of the segment's first chunk
-        if (!final_rows && ctid < G) {
+        if (part_rows && ctid < G) {
             p.ws_m[(bh0 + ctid) * p.splits + seg_j0] = seg_M[ctid];
             p.ws_l[(bh0 + ctid) * p.splits + seg_j0] = seg_L[ctid];
         }

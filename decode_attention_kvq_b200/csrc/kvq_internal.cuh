@@ -64,6 +64,7 @@ struct DecodeParams {
     int splits;              // chunks of the longest sequence
     int grid;                // persistent CTAs of the split kernel
     int seg_w;               // partition weight of a (sequence, kv head) start, in items
+    int one_item;            // the plan's items fit the grid: CTA c takes item c
     float scale_log2;        // attn_scale * log2(e)
 };
 // Split-K workspace: the partition header (written by the split kernel, read
