@@ -335,20 +335,25 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         return cum[lo] + hk * per + max(jw - W, 0);
     };
     const int grid = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-    const int wq = TW / grid, wr = TW % grid;
-    const int ibeg = one ? c : W ? item_of(c * wq + min(c, wr)) : c * wq + min(c, wr);
-    const int iend = one ? c + 1
-                         : W ? item_of((c + 1) * wq + min(c + 1, wr)) : (c + 1) * wq + min(c + 1, wr);
+    int ibeg = c, iend = c + 1;
+    if (!one) {
+        const int wq = TW / grid, wr = TW % grid;
+        ibeg = W ? item_of(c * wq + min(c, wr)) : c * wq + min(c, wr);
+        iend = W ? item_of((c + 1) * wq + min(c + 1, wr)) : (c + 1) * wq + min(c + 1, wr);
+    }
     // one item per CTA: the item, and its length read straight from the caller
     const int one_b = c / max(p.Hk * p.splits, 1);
     const int one_r = c - one_b * p.Hk * p.splits;
     const int one_hk = one_r / p.splits, one_j = one_r - one_hk * p.splits;
-    auto one_len = [&]() {
+    // the length as read, and as used: a length beyond the capacity or the
+    // planned window reads as 0 (flagged once, by the first consumer thread of
+    // the sequence's first CTA)
+    auto one_raw = [&]() { return p.seq_lens[one_b]; };
+    auto one_valid = [&](int L) {
         const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
         const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
-        int L = p.seq_lens[one_b];
         if (L < 0 || L > lim) {
-            if (one_j == 0 && one_hk == 0 && tid == 0) raise_flag(p.d_err, KVQ_DEVERR_LEN);
+            if (one_j == 0 && one_hk == 0 && tid == 32 * nprod(PAGED)) raise_flag(p.d_err, KVQ_DEVERR_LEN);
             L = 0;
         }
         return L;
@@ -418,7 +423,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // one item per CTA: the length load is issued first and used only
             // after the first stage is on its way (the chunk's end stands in)
             int Lone = 0;
-            if (one) Lone = one_len();
+            if (one) Lone = one_raw();
             const Seg sg = one ? one_seg((one_j + 1) * chunk) : seg_at(i, iend, lens, nsv, cum, B, chunk);
             i = sg.next;
             if (sg.ns == 0) continue;
@@ -447,7 +452,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
 #pragma unroll 1
             for (int tt0 = sg.t0; tt0 < t1; tt0 += TT, ++count, ++seg_tiles,
-                     t1 = (one && seg_tiles == 1) ? max(sg.t0, min(sg.t0 + chunk, Lone)) : t1) {
+                     t1 = (one && seg_tiles == 1) ? max(sg.t0, min(sg.t0 + chunk, one_valid(Lone))) : t1) {
                 const int s = count % NST;
                 const uint32_t full = bar_full + 8 * s;
                 if (count >= NST && lane == 0) wait(bar_empty + 8 * s, ((count / NST) - 1) & 1);
@@ -584,7 +589,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 #pragma unroll 1
     for (int i = ibeg; i < iend;) {
-        const Seg sg = one ? one_seg(one_len()) : seg_at(i, iend, lens, nsv, cum, B, p.chunk);
+        const Seg sg = one ? one_seg(one_valid(one_raw())) : seg_at(i, iend, lens, nsv, cum, B, p.chunk);
         i = sg.next;
         const int b = sg.b, hk = sg.hk;
         const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
