@@ -179,6 +179,21 @@ __device__ __forceinline__ float ldsf(uint32_t a) {
 // 2^e for -126 <= e <= 127, exact.
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
 
+// Merge-slot swizzle: chunk k (16 bytes) of head h's row is stored at
+// k ^ mswz(h).  The eight lanes of a quarter warp store chunks of heads
+// 2t + c (t = lane % 4) whose unswizzled indices differ only in one bit
+// (bit 2 per-token at D = 128, bit 1 at D = 64, bit 0 in group-32 mode);
+// XOR-ing t into the two other low bits makes the eight chunks fall into
+// eight different bank quads.  mswz(h) < 8, so an aligned run of eight
+// chunks of one row stays a run of eight distinct quads for the readers.
+template <int D, bool G32>
+__device__ __forceinline__ int mswz(int h) {
+    const int t = (h >> 1) & 3;
+    if constexpr (G32) return t << 1;
+    else if constexpr (D == 128) return t;
+    else return (t & 1) | ((t & 2) << 1);
+}
+
 struct Seg {
     int b, hk, ns, j0, j1, t0, t1;
     int next;                      // first item after the run
@@ -233,14 +248,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t bar_empty = bar_full + NST * 8;
     // per-warp head maxima and sums of a segment (read only between the two
     // merge barriers, so the next segment's writes cannot overtake a reader)
-    float* mrg_m = reinterpret_cast<float*>(smem + Lay::MISC_OFF + 2 * NST * 8);  // [NW][16]
-    float* mrg_l = mrg_m + NW * 16;                                               // [NW][16]
-    float* seg_M = mrg_l + NW * 16;     // [16] a segment's per-head max and sum, for the
-    float* seg_L = seg_M + 16;          // [16] partial-state writes after the merge
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(seg_L + 16);
-    static_assert(2 * NST * 8 + (2 * NW * 16 + 32) * 4 + 4 <= Lay::MISC_BYTES,
+    float* mrg_m = reinterpret_cast<float*>(smem + Lay::MISC_OFF + 2 * NST * 8);  // [16][NW]
+    float* mrg_l = mrg_m + 16 * NW;                                               // [16][NW]
+    // completes when all consumer warps have read a segment's maxima and slots
+    const uint32_t bar_mfree = ptx::smem_u32(mrg_l + 16 * NW);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_l + 16 * NW + 2);
+    static_assert(2 * NST * 8 + 2 * 16 * NW * 4 + 8 + 4 <= Lay::MISC_BYTES,
                   "barriers, maxima, flag");
-    float* mslot = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);               // [NW][NV][32]
+    float* mslot = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);   // [NW][8 NT heads][D]
     int* lens = reinterpret_cast<int*>(smem + Lay::LENS_OFF);                     // [B]
     int* nsv = lens + kMaxB;                                                     // [B] chunks
     int* cum = nsv + kMaxB;                                                      // [B + 1]
@@ -263,6 +278,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             ptx::mbar_init(bar_full + 8 * s, PAGED ? 2 + 32 : 1);
             ptx::mbar_init(bar_empty + 8 * s, WPG);
         }
+        ptx::mbar_init(bar_mfree, NW);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -586,6 +602,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     float o[MT][NT][4];                 // O^T C fragments: rows = head_dim, columns = heads
     int kv = 64;                        // running P'' prescale exponent (per warp)
     int c_count = 0;                    // tiles of the CTA seen so far (ring position)
+    int merges = 0;                     // segment merges of the CTA so far
 
 #pragma unroll 1
     for (int i = ibeg; i < iend;) {
@@ -951,13 +968,15 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (lane == 0) ptx::mbar_arrive(bar_empty + 8 * s);
         }
 
-        // ---- merge the eight warps' states of the segment (one round); a
+        // ---- merge the eight warps' states of the segment (one barrier); a
         // segment that is the whole (b, kv head) writes the final rows
         // (one item per CTA: the final rows of a one-chunk or empty sequence come
         // from its chunk 0; chunks past the length write nothing)
         const bool final_rows = one ? sg.j0 == 0 && sg.ns <= 1 : sg.j0 == 0 && sg.j1 == sg.ns - 1;
         const bool part_rows = one ? sg.ns > 1 && sg.j0 < sg.ns : !final_rows;
         const int seg_j0 = sg.j0;
+        // the previous segment's readers are done with the maxima and the slots
+        if (merges > 0) wait(bar_mfree, (merges - 1) & 1);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -966,79 +985,91 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 8);
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 16);
                 if (g == 0) {
-                    mrg_m[cw * 16 + 8 * nt + 2 * t + c] = m[nt][c];
-                    mrg_l[cw * 16 + 8 * nt + 2 * t + c] = l[nt][c];
+                    mrg_m[(8 * nt + 2 * t + c) * NW + cw] = m[nt][c];
+                    mrg_l[(8 * nt + 2 * t + c) * NW + cw] = l[nt][c];
                 }
             }
-        ptx::named_bar_sync(1, NCONS);
-        // per head of this thread: segment max M, segment sum Ls, and the factor
-        // for this warp's o (2^(m - M) undoing the P'' prescale, divided by Ls
-        // when the rows are final)
-        float fo[NT][2];
+        // this warp's o, prescale 2^kv undone, into its slot: one row of D
+        // floats per head, stored as 16-byte chunks, chunk k of head h at
+        // k ^ mswz(h).  A thread holds four consecutive head_dim values of a
+        // head in o[2a][nt][c], o[2a][nt][c+2], o[2a+1][nt][c], o[2a+1][nt][c+2]
+        // (one chunk), and the swizzle puts the eight chunks of a quarter warp
+        // in eight different bank quads.
         {
             const float down = pow2i(-kv);
+            float* slot = mslot + cw * NV * 32;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const int h = 8 * nt + 2 * t + c;
-                    float mw[NW], lw[NW];
 #pragma unroll
-                    for (int w = 0; w < NW; ++w) {
-                        mw[w] = mrg_m[w * 16 + h];
-                        lw[w] = mrg_l[w * 16 + h];
-                    }
-                    float M = -INFINITY;
-#pragma unroll
-                    for (int w = 0; w < NW; ++w) M = fmaxf(M, mw[w]);
-                    float Ls = 0.f;
-#pragma unroll
-                    for (int w = 0; w < NW; ++w)
-                        Ls += mw[w] == -INFINITY ? 0.f : lw[w] * ptx::ex2(mw[w] - M);
-                    const float f = (m[nt][c] == -INFINITY) ? 0.f : ptx::ex2(m[nt][c] - M) * down;
-                    fo[nt][c] = final_rows ? (Ls > 0.f ? f * __frcp_rn(Ls) : 0.f) : f;
-                    if (cw == 0 && g == 0) {
-                        seg_M[h] = M;
-                        seg_L[h] = Ls;
+                    for (int a = 0; a < D / 32; ++a) {
+                        const int k = G32 ? 8 * a + g : (D / 32) * g + a;
+                        *reinterpret_cast<float4*>(slot + h * D + 4 * (k ^ mswz<D, G32>(h))) =
+                            make_float4(o[2 * a][nt][c] * down, o[2 * a][nt][c + 2] * down,
+                                        o[2 * a + 1][nt][c] * down, o[2 * a + 1][nt][c + 2] * down);
                     }
                 }
         }
-        {
-            float* slot = mslot + cw * NV * 32 + lane;
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        slot[((mt * NT + nt) * 4 + e) * 32] = o[mt][nt][e] * fo[nt][e & 1];
-        }
         ptx::named_bar_sync(1, NCONS);
-        // sum the eight slots position by position and write the rows (all
-        // loads of a thread's positions issued together)
-        static_assert((NV * 32) % NCONS == 0, "positions per consumer thread");
+        // one thread per (head, 16-byte chunk of its row): the head's segment
+        // max M and sum Ls over the eight warps, the weights 2^(m_w - M) (over
+        // Ls when the rows are final), and the weighted sum of the eight slots
+        constexpr int NCH = D / 4;
+        constexpr int NITEM = 8 * NT * NCH;
+        static_assert(NW == 8, "two 16-byte loads of per-warp maxima and sums");
 #pragma unroll
-        for (int it = 0; it < NV * 32 / NCONS; ++it) {
-            const int pos = ctid + it * NCONS;
-            const int v = pos >> 5, ln = pos & 31;
-            const int pg_ = ln >> 2, pt = ln & 3;
-            const int mt = v / (NT * 4), nt = (v / 4) % NT, e = v & 3;
-            const int h = 8 * nt + 2 * pt + (e & 1);
-            if (h >= G) continue;
-            float sum = 0.f;
+        for (int it = 0; it < (NITEM + NCONS - 1) / NCONS; ++it) {
+            const int idx = ctid + it * NCONS;
+            const int h = idx / NCH, k = idx % NCH;
+            if (idx >= NITEM || h >= G) continue;
+            float mw[NW], fw[NW], lw[NW];
+            *reinterpret_cast<float4*>(mw) = *reinterpret_cast<const float4*>(mrg_m + h * NW);
+            *reinterpret_cast<float4*>(mw + 4) = *reinterpret_cast<const float4*>(mrg_m + h * NW + 4);
+            *reinterpret_cast<float4*>(lw) = *reinterpret_cast<const float4*>(mrg_l + h * NW);
+            *reinterpret_cast<float4*>(lw + 4) = *reinterpret_cast<const float4*>(mrg_l + h * NW + 4);
+            float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < NW; ++w) sum += mslot[(w * NV + v) * 32 + ln];
-            const int d = G32 ? 32 * (mt >> 1) + 4 * pg_ + 2 * (mt & 1) + (e >> 1)
-                              : (D == 128 ? 16 : 8) * pg_ + 2 * mt + (e >> 1);
+            for (int w = 0; w < NW; ++w) M = fmaxf(M, mw[w]);
+            float Ls = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                fw[w] = mw[w] == -INFINITY ? 0.f : ptx::ex2(mw[w] - M);
+                Ls += lw[w] * fw[w];
+            }
+            if (final_rows) {
+                const float r = Ls > 0.f ? __frcp_rn(Ls) : 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) fw[w] *= r;
+            }
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+            const float* src = mslot + h * D + 4 * (k ^ mswz<D, G32>(h));
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float4 v = *reinterpret_cast<const float4*>(src + w * NV * 32);
+                s0 = fmaf(fw[w], v.x, s0);
+                s1 = fmaf(fw[w], v.y, s1);
+                s2 = fmaf(fw[w], v.z, s2);
+                s3 = fmaf(fw[w], v.w, s3);
+            }
             const int64_t row = bh0 + h;
-            if (final_rows) p.out[row * D + d] = sum;
-            else if (part_rows) p.ws_o[(row * p.splits + seg_j0) * D + d] = sum;
+            if (final_rows) {
+                *reinterpret_cast<float4*>(p.out + row * D + 4 * k) = make_float4(s0, s1, s2, s3);
+            } else if (part_rows) {
+                // the partial, with its (m, l) in the slot of the segment's first chunk
+                *reinterpret_cast<float4*>(p.ws_o + (row * p.splits + seg_j0) * D + 4 * k) =
+                    make_float4(s0, s1, s2, s3);
+                if (k == 0) {
+                    p.ws_m[row * p.splits + seg_j0] = M;
+                    p.ws_l[row * p.splits + seg_j0] = Ls;
+                }
+            }
         }
-        // the partial's (m, l), in the slot of the segment's first chunk
-        if (part_rows && ctid < G) {
-            p.ws_m[(bh0 + ctid) * p.splits + seg_j0] = seg_M[ctid];
-            p.ws_l[(bh0 + ctid) * p.splits + seg_j0] = seg_L[ctid];
-        }
+        // this warp has read the maxima and the slots
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar_mfree);
+        ++merges;
     }
 }
 
