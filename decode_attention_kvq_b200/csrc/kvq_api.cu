@@ -70,7 +70,7 @@ kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk
 
 size_t workspace_for(int B, int Hq, int D, int splits) {
     if (splits <= 1) return 0;
-    return kvq::kHdrBytes + static_cast<size_t>(B) * Hq * splits * (D + 2) * sizeof(float);
+    return static_cast<size_t>(B) * Hq * splits * (D + 2) * sizeof(float);
 }
 
 }  // namespace
@@ -174,11 +174,9 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
     kvq::DecodeParams p{};
     p.q = q; p.k = kv->k; p.v = kv->v; p.k_scale = kv->k_scale; p.v_scale = kv->v_scale;
     p.table = kv->page_table; p.seq_lens = d_seq_lens; p.out = out; p.d_err = d_err;
-    // [partition header: kHdrBytes][o: n_part * D][m: n_part][l: n_part]
-    float* ws = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kvq::kHdrBytes)
-                          : nullptr;
+    // [o: n_part * D][m: n_part][l: n_part]
+    float* ws = static_cast<float*>(workspace);
     const size_t n_part = static_cast<size_t>(B) * Hq * splits;
-    p.ws_hdr = static_cast<int*>(workspace);
     p.ws_o = ws;
     p.ws_m = ws ? ws + n_part * D : nullptr;
     p.ws_l = ws ? ws + n_part * (D + 1) : nullptr;

@@ -282,6 +282,37 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
+    if (!PAGED && prm.one_item && tid == 32) {
+        // one item per CTA, contiguous cache: the item's first two stages of K
+        // and V rows (and their scales) do not depend on the length, so they
+        // are prefetched into L2 while the predecessor finishes (more than two
+        // stages holds up the CTA's own first loads behind the prefetch).  A prefetch moves
+        // nothing into this SM: the loads after the dependency wait still see
+        // every write the predecessor makes.
+        const int c = blockIdx.x;
+        const int pb = c / max(prm.Hk * prm.splits, 1);
+        const int pr = c - pb * prm.Hk * prm.splits;
+        const int phk = pr / prm.splits;
+        const int64_t pt0 = static_cast<int64_t>(pr - phk * prm.splits) * prm.chunk;
+        const int64_t prow = static_cast<int64_t>(pb * prm.Hk + phk) * prm.max_seq;
+        const int64_t nrow = min(static_cast<int64_t>(min(prm.chunk, 2 * TT)), prm.max_seq - pt0);
+        if (nrow > 0) {
+            const uint32_t kvb = static_cast<uint32_t>(nrow * D);
+            ptx::prefetch_l2(prm.k + (prow + pt0) * D, kvb);
+            ptx::prefetch_l2(prm.v + (prow + pt0) * D, kvb);
+            // scales: the 16-byte aligned span that covers the rows' floats
+            // and stays inside the scale arrays
+            const int64_t f0 = (prow + pt0) * Lay::NG;
+            const int64_t f1 = min((prow + pt0 + nrow) * Lay::NG + 3,
+                                   static_cast<int64_t>(prm.B) * prm.Hk * prm.max_seq * Lay::NG) &
+                               ~static_cast<int64_t>(3);
+            const int64_t a0 = f0 & ~static_cast<int64_t>(3);
+            if (f1 > a0) {
+                ptx::prefetch_l2(prm.k_scale + a0, static_cast<uint32_t>((f1 - a0) * 4));
+                ptx::prefetch_l2(prm.v_scale + a0, static_cast<uint32_t>((f1 - a0) * 4));
+            }
+        }
+    }
     grid_dep_wait();                    // the predecessor's writes (q, cache, lengths) are visible
     grid_dep_launch();                  // the combine kernel may be scheduled now
 
@@ -385,25 +416,6 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         sg.next = iend;
         return sg;
     };
-    if (!one && p.splits > 1) {
-        // publish the partition for the combine kernel: T, the item prefix sums,
-        // the chunk counts and every CTA's first item (it finds each unit's
-        // partials from them); written by a consumer thread, off the producer's
-        // path to its first load
-        int* hdr = p.ws_hdr;
-        if (tid == 32) {
-            if (W) hdr[kHdrStart + c] = ibeg;
-            if (c == 0) {
-                hdr[0] = T;
-                hdr[kHdrStart + grid] = T;
-            }
-        }
-        if (c == 0) {
-            for (int b = tid; b <= B; b += nthreads(PAGED)) hdr[kHdrCum + b] = cum[b];
-            for (int b = tid; b < B; b += nthreads(PAGED)) hdr[kHdrNs + b] = nsv[b];
-        }
-    }
-
     // bounded wait that gives up at once after any earlier timeout of this CTA
     auto wait = [&](uint32_t bar, uint32_t parity) {
         if (*abort_flag) return;
@@ -1064,6 +1076,15 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     p.ws_m[row * p.splits + seg_j0] = M;
                     p.ws_l[row * p.splits + seg_j0] = Ls;
                 }
+            }
+            // blocks of several items: every other chunk slot the segment covers
+            // gets m = -inf ("no partial here"), so the combine kernel finds a
+            // unit's partials from its m slots alone (one item per CTA: every
+            // chunk below the chunk count holds a partial)
+            if (!one && p.splits > 1 && sg.ns > 1) {
+#pragma unroll 1
+                for (int j = seg_j0 + (part_rows ? 1 : 0) + k; j <= sg.j1; j += NCH)
+                    p.ws_m[row * p.splits + j] = -INFINITY;
             }
         }
         // this warp has read the maxima and the slots

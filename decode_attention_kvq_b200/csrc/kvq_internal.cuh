@@ -55,7 +55,6 @@ struct DecodeParams {
     float* ws_o;             // [B*Hq, splits, D] partial outputs (unnormalised)
     float* ws_m;             // [B*Hq, splits] running max (log2 domain)
     float* ws_l;             // [B*Hq, splits] running sum
-    int* ws_hdr;             // the split kernel's partition: T, -, cum, ns, CTA starts
     int32_t* d_err;
     int B, Hq, Hk, G, D;
     int group32;
@@ -67,15 +66,8 @@ struct DecodeParams {
     int one_item;            // the plan's items fit the grid: CTA c takes item c
     float scale_log2;        // attn_scale * log2(e)
 };
-// Split-K workspace: the partition header (written by the split kernel, read
-// by the combine kernel), then the partials.
 constexpr int kMaxBatch = 1024;                              // sequences per call
 constexpr int kMaxGrid = 1024;                               // persistent CTAs
-constexpr int kHdrCum = 2;                                   // [kMaxBatch + 1] item prefix sums
-constexpr int kHdrNs = kHdrCum + kMaxBatch + 1;              // [kMaxBatch] chunk counts
-constexpr int kHdrStart = kHdrNs + kMaxBatch;                // [grid + 1] first item of CTA c
-constexpr int kHdrInts = kHdrStart + kMaxGrid + 1;
-constexpr size_t kHdrBytes = (kHdrInts * 4 + 255) / 256 * 256;
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 // tensor-core split kernel (kvq_decode_tc.cu)
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s);
