@@ -313,7 +313,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
         }
     }
-    grid_dep_wait();                    // the predecessor's writes (q, cache, lengths) are visible
+    // the predecessor's writes (q, cache, lengths) are visible after the
+    // dependency wait.  One item per CTA: nothing before the roles reads
+    // them, so each role waits just before its first global access and the
+    // producer's set-up overlaps the predecessor's tail.
+    if (!prm.one_item) grid_dep_wait();
     grid_dep_launch();                  // the combine kernel may be scheduled now
 
     // one item per CTA (the plan's items fit the grid): CTA c takes item c of
@@ -446,6 +450,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int64_t sc_total = static_cast<int64_t>(B) * Hk * max_seq * NG;
         const uint32_t q_bytes = static_cast<uint32_t>(G * D * 2);
         int count = 0;                  // tiles issued (ring position)
+        if (one) grid_dep_wait();       // before the length, table, q and cache reads
 #pragma unroll 1
         for (int i = ibeg; i < iend;) {
             // one item per CTA: the length load is issued first and used only
@@ -602,6 +607,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     // tiles u = 0, 1 that share one online-softmax step.
     const int cw = warp - nprod(PAGED);            // consumer warp index
     const int ctid = tid - 32 * nprod(PAGED);      // consumer thread index
+    if (one) grid_dep_wait();           // before the length read and any global write
     const int grp = cw / WPG, wg = cw % WPG;
     const int sig_g = sigma(g);
     const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
