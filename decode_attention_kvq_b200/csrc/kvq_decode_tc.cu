@@ -252,8 +252,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     float* mrg_l = mrg_m + 16 * NW;                                               // [16][NW]
     // completes when all consumer warps have read a segment's maxima and slots
     const uint32_t bar_mfree = ptx::smem_u32(mrg_l + 16 * NW);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_l + 16 * NW + 2);
-    static_assert(2 * NST * 8 + 2 * 16 * NW * 4 + 8 + 4 <= Lay::MISC_BYTES,
+    // one item per CTA: the query rows' own barrier (they land ahead of stage 0)
+    const uint32_t bar_q = bar_mfree + 8;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_l + 16 * NW + 4);
+    static_assert(2 * NST * 8 + 2 * 16 * NW * 4 + 16 + 4 <= Lay::MISC_BYTES,
                   "barriers, maxima, flag");
     float* mslot = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);   // [NW][8 NT heads][D]
     int* lens = reinterpret_cast<int*>(smem + Lay::LENS_OFF);                     // [B]
@@ -279,6 +281,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             ptx::mbar_init(bar_empty + 8 * s, WPG);
         }
         ptx::mbar_init(bar_mfree, NW);
+        ptx::mbar_init(bar_q, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -465,6 +468,13 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int b = sg.b, hk = sg.hk;
             const uint16_t* qsrc = qg + (static_cast<int64_t>(b) * Hq + hk * G) * D;
             int seg_tiles = 0;          // tiles issued for this segment
+            if (one && pw == 0 && lane == 0) {
+                // one item per CTA: the query rows go first, on their own
+                // barrier, into stage 0's query area (no stage carries them), so
+                // the consumers build their Q operand while K and V are in flight
+                ptx::mbar_arrive_expect_tx(bar_q, q_bytes);
+                ptx::bulk_load(sbase + Lay::Q_OFF, qsrc, q_bytes, bar_q);
+            }
             // paged: the segment's page ids, 32 pages (4 stages) per register,
             // loaded one group of 4 stages ahead so the table read is off the
             // issue path; lane i holds page pbase + i (-1: none or out of range)
@@ -497,8 +507,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const uint32_t svs = sks + Lay::SC_FLOATS * 4;
                 // the segment's G query rows (contiguous bf16) ride with its first
                 // two stages: each consumer group builds its Q operand from the
-                // first stage it works in the segment
-                const bool with_q = seg_tiles < 2;
+                // first stage it works in the segment (one item per CTA: they
+                // came first, on their own barrier)
+                const bool with_q = !one && seg_tiles < 2;
                 if (!PAGED) {
                     if (lane == 0) {
                         const int64_t row0 = (static_cast<int64_t>(b) * Hk + hk) * max_seq + tt0;
@@ -597,6 +608,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll 1
             for (int c = count - 1; c >= 0 && c >= count - NST; --c)
                 ptx::mbar_wait(bar_full + 8 * (c % NST), (c / NST) & 1);
+        if (one && pw == 0 && lane == 0) ptx::mbar_wait(bar_q, 0);
         return;                         // consumers synchronise among themselves (barrier 1)
     }
 
@@ -622,6 +634,87 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     int c_count = 0;                    // tiles of the CTA seen so far (ring position)
     int merges = 0;                     // segment merges of the CTA so far
 
+    // ---- Q^T operand from the segment's query rows at sq (they ride with its
+    // first two stages; one item per CTA: they come ahead of stage 0).
+    // Column n = g of n-tile nt is query head 8*nt + g.
+    // Each head is scaled by 2^sh so max |q| * 2^sh is in [2^14, 2^15)
+    // and rounded to a 16-bit integer Qi = 256 * hi + lo (hi signed,
+    // lo unsigned byte); the relative error per element is at most
+    // 2^-15 of the head's max |q|.  B fragment rows 4t..4t+3 (b0) and
+    // 16+4t..16+4t+3 (b1) of k-step gi hold head_dim 32*gi + 8*t +
+    // {0..3} and {4..7}: the same permutation of head_dim as the
+    // K operand's bytes, so the dot products are unchanged.
+    auto build_q = [&](uint32_t sq) {
+        float zsq[NT];
+        int csq[NT][NCG];              // sum of the head's Qi (per 32-value group)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int h = 8 * nt + g;
+            float qf[NGRP][8];
+            float amax = 0.f;
+#pragma unroll
+            for (int gi = 0; gi < NGRP; ++gi) {
+                uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+                if (h < G) raw = lds128(sq + (h * D + 32 * gi + 8 * t) * 2);
+                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    qf[gi][2 * e] = bf16_bits_to_f32(w[e] & 0xffffu);
+                    qf[gi][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(qf[gi][e]));
+            }
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            int sh = 0;
+            if (amax > 0.f) {
+                const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+                sh = min(max(14 - e, -100), 100);
+            }
+            const float up = pow2i(sh);                  // |sh| <= 100
+            zsq[nt] = pow2i(-sh) * p.scale_log2;
+#pragma unroll
+            for (int c = 0; c < NCG; ++c) csq[nt][c] = 0;
+#pragma unroll
+            for (int gi = 0; gi < NGRP; ++gi) {
+                uint32_t qi[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int v = min(max(__float2int_rn(qf[gi][e] * up), -32767), 32767);
+                    csq[nt][G32 ? gi : 0] += v;
+                    qi[e] = static_cast<uint32_t>(v);
+                }
+                // byte 1 (hi digit) and byte 0 (lo digit) of four values each
+                auto pick4 = [&](int e0, uint32_t sel2) {
+                    return ptx::prmt(ptx::prmt(qi[e0], qi[e0 + 1], sel2),
+                                     ptx::prmt(qi[e0 + 2], qi[e0 + 3], sel2), 0x5410u);
+                };
+                qh0[nt][gi] = pick4(0, 0x0051u);
+                qh1[nt][gi] = pick4(4, 0x0051u);
+                ql0[nt][gi] = pick4(0, 0x0040u);
+                ql1[nt][gi] = pick4(4, 0x0040u);
+            }
+#pragma unroll
+            for (int c = 0; c < NCG; ++c) {
+                csq[nt][c] += __shfl_xor_sync(0xffffffffu, csq[nt][c], 1);
+                csq[nt][c] += __shfl_xor_sync(0xffffffffu, csq[nt][c], 2);
+            }
+        }
+        // per-head factors of the two heads (columns 2t, 2t+1) this thread
+        // accumulates: score scale, and the offset term 128 * sum(Qi) of
+        // sum Qi * (byte - 128) = sum Qi * byte - 128 * sum Qi
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                zs[nt][c] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t + c));
+#pragma unroll
+                for (int k = 0; k < NCG; ++k)
+                    qc[nt][c][k] = 128 * __shfl_sync(0xffffffffu, csq[nt][k], 4 * (2 * t + c));
+            }
+    };
+
 #pragma unroll 1
     for (int i = ibeg; i < iend;) {
         const Seg sg = one ? one_seg(one_valid(one_raw())) : seg_at(i, iend, lens, nsv, cum, B, p.chunk);
@@ -644,6 +737,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         kv = 64;
         bool have_q = false;            // Q fragments of this segment are built
+        if (one) {                      // the query rows came ahead of stage 0
+            wait(bar_q, 0);
+            build_q(sbase + Lay::Q_OFF);
+            have_q = true;
+        }
         // contiguous layout: the stage's scales start sc_off bytes in (the copies
         // start at the 16-byte aligned float at or below the tile's first; tiles
         // start at multiples of 16 tokens, so the offset is the segment's)
@@ -666,85 +764,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const uint32_t sks = sv + Lay::KV_BYTES + sc_off;
             const uint32_t svs = sv + Lay::KV_BYTES + Lay::SC_FLOATS * 4 + sc_off;
             if (!have_q) {
-                // ---- Q^T operand (the segment's query rows ride with its first
-                // two stages).  Column n = g of n-tile nt is query head 8*nt + g.
-                // Each head is scaled by 2^sh so max |q| * 2^sh is in [2^14, 2^15)
-                // and rounded to a 16-bit integer Qi = 256 * hi + lo (hi signed,
-                // lo unsigned byte); the relative error per element is at most
-                // 2^-15 of the head's max |q|.  B fragment rows 4t..4t+3 (b0) and
-                // 16+4t..16+4t+3 (b1) of k-step gi hold head_dim 32*gi + 8*t +
-                // {0..3} and {4..7}: the same permutation of head_dim as the
-                // K operand's bytes, so the dot products are unchanged.
                 have_q = true;
-                const uint32_t sq = sk + Lay::Q_OFF;
-                float zsq[NT];
-                int csq[NT][NCG];              // sum of the head's Qi (per 32-value group)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const int h = 8 * nt + g;
-                    float qf[NGRP][8];
-                    float amax = 0.f;
-#pragma unroll
-                    for (int gi = 0; gi < NGRP; ++gi) {
-                        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-                        if (h < G) raw = lds128(sq + (h * D + 32 * gi + 8 * t) * 2);
-                        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            qf[gi][2 * e] = bf16_bits_to_f32(w[e] & 0xffffu);
-                            qf[gi][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
-                        }
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(qf[gi][e]));
-                    }
-                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                    int sh = 0;
-                    if (amax > 0.f) {
-                        const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
-                        sh = min(max(14 - e, -100), 100);
-                    }
-                    const float up = pow2i(sh);                  // |sh| <= 100
-                    zsq[nt] = pow2i(-sh) * p.scale_log2;
-#pragma unroll
-                    for (int c = 0; c < NCG; ++c) csq[nt][c] = 0;
-#pragma unroll
-                    for (int gi = 0; gi < NGRP; ++gi) {
-                        uint32_t qi[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int v = min(max(__float2int_rn(qf[gi][e] * up), -32767), 32767);
-                            csq[nt][G32 ? gi : 0] += v;
-                            qi[e] = static_cast<uint32_t>(v);
-                        }
-                        // byte 1 (hi digit) and byte 0 (lo digit) of four values each
-                        auto pick4 = [&](int e0, uint32_t sel2) {
-                            return ptx::prmt(ptx::prmt(qi[e0], qi[e0 + 1], sel2),
-                                             ptx::prmt(qi[e0 + 2], qi[e0 + 3], sel2), 0x5410u);
-                        };
-                        qh0[nt][gi] = pick4(0, 0x0051u);
-                        qh1[nt][gi] = pick4(4, 0x0051u);
-                        ql0[nt][gi] = pick4(0, 0x0040u);
-                        ql1[nt][gi] = pick4(4, 0x0040u);
-                    }
-#pragma unroll
-                    for (int c = 0; c < NCG; ++c) {
-                        csq[nt][c] += __shfl_xor_sync(0xffffffffu, csq[nt][c], 1);
-                        csq[nt][c] += __shfl_xor_sync(0xffffffffu, csq[nt][c], 2);
-                    }
-                }
-                // per-head factors of the two heads (columns 2t, 2t+1) this thread
-                // accumulates: score scale, and the offset term 128 * sum(Qi) of
-                // sum Qi * (byte - 128) = sum Qi * byte - 128 * sum Qi
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        zs[nt][c] = __shfl_sync(0xffffffffu, zsq[nt], 4 * (2 * t + c));
-#pragma unroll
-                        for (int k = 0; k < NCG; ++k)
-                            qc[nt][c][k] = 128 * __shfl_sync(0xffffffffu, csq[nt][k], 4 * (2 * t + c));
-                    }
+                build_q(sk + Lay::Q_OFF);
             }
             const int tok0 = tt0 + 32 * wg;               // first token of this warp's slice
             if (tok0 < t1) {
