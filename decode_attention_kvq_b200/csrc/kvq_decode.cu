@@ -14,6 +14,8 @@
 // one CTA took whole (and finished itself) has no finite m at all.
 #include <math.h>
 
+#include <atomic>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -208,6 +210,48 @@ decode_combine_live(DecodeParams p) {
     finish_row<true>(p.out + bh * D, D, Mw, lw, acc, s_m, s_l, s_acc);
 }
 
+// Dynamic shared memory for decode_combine_one so that at most k =
+// ceil(rows / SMs) of its CTAs share an SM.  The combine launches early, next
+// to the split kernel, and without this its CTAs crowd onto the few SMs the
+// split kernel leaves idle, where the L2 reads of the partials queue behind
+// one another.  0 when the attributes cannot be read or k > 2.  The device
+// figures are read once per device.
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_spread_state[kMaxDevices];   // 0 not read, 1 ready, -1 unavailable
+int g_spread_sms[kMaxDevices];
+int g_spread_dyn[kMaxDevices][2];                // bytes for k = 1, 2
+
+size_t combine_one_spread_smem(int rows) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    int st = g_spread_state[dev].load(std::memory_order_acquire);
+    if (st == 0) {
+        int sms = 0, cap = 0, reserved = 0;
+        cudaFuncAttributes fa;
+        st = -1;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&cap, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) ==
+                cudaSuccess &&
+            cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) ==
+                cudaSuccess &&
+            cudaFuncGetAttributes(&fa, decode_combine_one) == cudaSuccess && sms > 0) {
+            // a CTA's footprint F = cap / k: k of them fit on an SM, k + 1 do not
+            for (int k = 1; k <= 2; ++k)
+                g_spread_dyn[dev][k - 1] = static_cast<int>(
+                    (cap / k - static_cast<long long>(fa.sharedSizeBytes) - reserved) / 16 * 16);
+            g_spread_sms[dev] = sms;
+            if (g_spread_dyn[dev][1] > 0 &&
+                cudaFuncSetAttribute(decode_combine_one, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     g_spread_dyn[dev][0]) == cudaSuccess)
+                st = 1;
+        }
+        g_spread_state[dev].store(st, std::memory_order_release);
+    }
+    if (st < 0) return 0;
+    const int k = (rows + g_spread_sms[dev] - 1) / g_spread_sms[dev];
+    return k <= 2 ? static_cast<size_t>(g_spread_dyn[dev][k - 1]) : 0;
+}
+
 }  // namespace
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
@@ -223,7 +267,10 @@ cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (p.one_item) return cudaLaunchKernelEx(&cfg, decode_combine_one, p);
+    if (p.one_item) {
+        cfg.dynamicSmemBytes = combine_one_spread_smem(p.B * p.Hq);
+        return cudaLaunchKernelEx(&cfg, decode_combine_one, p);
+    }
     return cudaLaunchKernelEx(&cfg, decode_combine_live, p);
 }
 
