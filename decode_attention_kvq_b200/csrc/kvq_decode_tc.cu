@@ -222,7 +222,14 @@ __device__ __forceinline__ Seg seg_at(int i, int iend, const int* lens, const in
     return sg;
 }
 
-template <int D, bool G32, bool PAGED, bool G16>
+// PK (group-32, G <= 4): the 8 columns of an MMA n-tile carry the G heads
+// twice, columns 4*par + h for the two parities par of the 32-value groups.
+// A Q.K^T k-step over group gi fills only the columns of parity gi % 2 (the
+// others' Q digits are zero), so groups 2a and 2a + 1 share one accumulator
+// and one fold; lanes t and t ^ 2 (the two parities) add their scores.  P''
+// is built once per group pair, each column with its own parity's V scale;
+// the P.V output columns of the other parity are not used.
+template <int D, bool G32, bool PAGED, bool G16, bool PK>
 __global__ void __launch_bounds__(nthreads(PAGED), 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ DecodeParams prm) {
@@ -234,6 +241,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     constexpr int MT = D / 16;          // m-tiles of O^T over head_dim (PV)
     constexpr int NT = G16 ? 2 : 1;     // n-tiles of 8 query heads
     constexpr int NGV = G32 ? NG : 1;   // V scales per token
+    static_assert(!PK || (G32 && !G16), "packing: group-32 scales, at most 4 heads");
+    constexpr int NVS = PK ? NGRP / 2 : NGV;   // P'' operand sets (PK: group pairs)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -242,6 +251,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tid = threadIdx.x;
     const int g = lane >> 2, t = lane & 3;
+    const int par = PK ? (t >> 1) : 0;  // PK: parity of this thread's MMA columns
 
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t bar_full = sbase + Lay::MISC_OFF;
@@ -649,7 +659,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         int csq[NT][NCG];              // sum of the head's Qi (per 32-value group)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const int h = 8 * nt + g;
+            const int h = PK ? (g & 3) : 8 * nt + g;
             float qf[NGRP][8];
             float amax = 0.f;
 #pragma unroll
@@ -681,7 +691,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 uint32_t qi[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int v = min(max(__float2int_rn(qf[gi][e] * up), -32767), 32767);
+                    // PK: column g carries group parity g / 4 only
+                    const int v = (PK && (g >> 2) != (gi & 1))
+                                      ? 0
+                                      : min(max(__float2int_rn(qf[gi][e] * up), -32767), 32767);
                     csq[nt][G32 ? gi : 0] += v;
                     qi[e] = static_cast<uint32_t>(v);
                 }
@@ -801,31 +814,40 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     for (int nt = 0; nt < NT; ++nt)
                         z[u][nt][0] = z[u][nt][1] = z[u][nt][2] = z[u][nt][3] = 0.f;
                 int ah[2][NT][4], al[2][NT][4];
-                auto zero_acc = [&]() {
+                // accumulators of fold kg (a head_dim group; PK: a group pair,
+                // whose lo digit starts at the pair's offset term -128 * sum(Qi))
+                auto zero_acc = [&](int kg) {
 #pragma unroll
                     for (int u = 0; u < 2; ++u)
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) ah[u][nt][e] = al[u][nt][e] = 0;
+                            for (int e = 0; e < 4; ++e) {
+                                ah[u][nt][e] = 0;
+                                al[u][nt][e] =
+                                    PK ? -(qc[nt][e & 1][2 * kg] + qc[nt][e & 1][2 * kg + 1]) : 0;
+                            }
                 };
-                // fold the integer scores of head_dim group kg into z, times the K
-                // scale of the token (per token: kg = 0, once after all groups)
+                // fold the integer scores of fold kg into z, times the K scale of
+                // the token and of the column's group (per token: kg = 0, once
+                // after all groups; PK: group 2 kg + par)
                 auto fold = [&](int kg) {
+                    const int cg = PK ? 2 * kg + par : kg;
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const float ksa = ldsf(sks + (rA[u] * NG + kg) * 4);
-                        const float ksb = ldsf(sks + (rB[u] * NG + kg) * 4);
+                        const float ksa = ldsf(sks + (rA[u] * NG + cg) * 4);
+                        const float ksb = ldsf(sks + (rB[u] * NG + cg) * 4);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                const int S = ah[u][nt][e] * 256 + al[u][nt][e] - qc[nt][e & 1][kg];
+                                const int S = ah[u][nt][e] * 256 + al[u][nt][e] -
+                                              (PK ? 0 : qc[nt][e & 1][kg]);
                                 z[u][nt][e] = fmaf(static_cast<float>(S), e < 2 ? ksa : ksb, z[u][nt][e]);
                             }
                     }
                 };
-                zero_acc();
+                zero_acc(0);
 #pragma unroll
                 for (int gi = 0; gi < NGRP; ++gi) {
 #pragma unroll
@@ -840,20 +862,36 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                                                ql1[nt][gi]);
                         }
                     }
-                    if (G32) {
-                        fold(gi);
-                        zero_acc();
+                    if constexpr (G32) {
+                        if (!PK || (gi & 1)) {
+                            const int kg = PK ? gi >> 1 : gi;
+                            fold(kg);
+                            if (gi + 1 < NGRP) zero_acc(kg + 1);
+                        }
                     }
                 }
-                if (!G32) fold(0);
+                if constexpr (!G32) fold(0);
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        z[u][nt][0] = okA[u] ? z[u][nt][0] * zs[nt][0] : -INFINITY;
-                        z[u][nt][1] = okA[u] ? z[u][nt][1] * zs[nt][1] : -INFINITY;
-                        z[u][nt][2] = okB[u] ? z[u][nt][2] * zs[nt][0] : -INFINITY;
-                        z[u][nt][3] = okB[u] ? z[u][nt][3] * zs[nt][1] : -INFINITY;
+                        if constexpr (PK) {
+                            // this parity's groups, then the other parity's (lane t ^ 2)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float zz = z[u][nt][e] * zs[nt][e & 1];
+                                z[u][nt][e] = zz + __shfl_xor_sync(0xffffffffu, zz, 2);
+                            }
+                            z[u][nt][0] = okA[u] ? z[u][nt][0] : -INFINITY;
+                            z[u][nt][1] = okA[u] ? z[u][nt][1] : -INFINITY;
+                            z[u][nt][2] = okB[u] ? z[u][nt][2] : -INFINITY;
+                            z[u][nt][3] = okB[u] ? z[u][nt][3] : -INFINITY;
+                        } else {
+                            z[u][nt][0] = okA[u] ? z[u][nt][0] * zs[nt][0] : -INFINITY;
+                            z[u][nt][1] = okA[u] ? z[u][nt][1] * zs[nt][1] : -INFINITY;
+                            z[u][nt][2] = okB[u] ? z[u][nt][2] * zs[nt][0] : -INFINITY;
+                            z[u][nt][3] = okB[u] ? z[u][nt][3] * zs[nt][1] : -INFINITY;
+                        }
                     }
                 // ---- online softmax per head: max over the slice's 32 tokens
                 float pr[2][NT][4];
@@ -881,16 +919,19 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         f[nt][c] = al;
                     }
                 // ---- V scales of the thread's four tokens and the running prescale 2^kv
-                float vsa[2][NGV], vsb[2][NGV];
+                // (PK: set gv is group pair gv, this thread's column group 2 gv + par)
+                float vsa[2][NVS], vsb[2][NVS];
                 float vmax = 0.f;
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
-                    for (int gv = 0; gv < NGV; ++gv) {
-                        vsa[u][gv] = okA[u] ? ldsf(svs + (rA[u] * NG + gv) * 4) : 0.f;
-                        vsb[u][gv] = okB[u] ? ldsf(svs + (rB[u] * NG + gv) * 4) : 0.f;
+                    for (int gv = 0; gv < NVS; ++gv) {
+                        const int cg = PK ? 2 * gv + par : gv;
+                        vsa[u][gv] = okA[u] ? ldsf(svs + (rA[u] * NG + cg) * 4) : 0.f;
+                        vsb[u][gv] = okB[u] ? ldsf(svs + (rB[u] * NG + cg) * 4) : 0.f;
                         vmax = fmaxf(vmax, fmaxf(vsa[u][gv], vsb[u][gv]));
                     }
+                if constexpr (PK) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 2));
                 vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
                 vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 8));
                 vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 16));
@@ -931,9 +972,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 // with prmt and turned into exact (v - 128) f16 pairs.
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    uint32_t pbh[NGV][NT][2], pbl[NGV][NT][2];
+                    uint32_t pbh[NVS][NT][2], pbl[NVS][NT][2];
 #pragma unroll
-                    for (int gv = 0; gv < NGV; ++gv)
+                    for (int gv = 0; gv < NVS; ++gv)
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
                             uint32_t ha, la, hb, lb;
@@ -996,7 +1037,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
                         for (int gv = 0; gv < NGRP; ++gv) {
                             const uint32_t cb = 32 * gv + 4 * g;
-                            pv_words(2 * gv, gv, lds32(sv + swz<D>(R0, cb)),
+                            pv_words(2 * gv, PK ? gv >> 1 : gv, lds32(sv + swz<D>(R0, cb)),
                                      lds32(sv + swz<D>(R1, cb)), lds32(sv + swz<D>(R2, cb)),
                                      lds32(sv + swz<D>(R3, cb)));
                         }
@@ -1024,8 +1065,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 8);
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 16);
                 if (g == 0) {
-                    mrg_m[(8 * nt + 2 * t + c) * NW + cw] = m[nt][c];
-                    mrg_l[(8 * nt + 2 * t + c) * NW + cw] = l[nt][c];
+                    const int hm = PK ? 2 * (t & 1) + c : 8 * nt + 2 * t + c;
+                    mrg_m[hm * NW + cw] = m[nt][c];
+                    mrg_l[hm * NW + cw] = l[nt][c];
                 }
             }
         // this warp's o, prescale 2^kv undone, into its slot: one row of D
@@ -1041,9 +1083,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    const int h = 8 * nt + 2 * t + c;
+                    const int h = PK ? 2 * (t & 1) + c : 8 * nt + 2 * t + c;
 #pragma unroll
                     for (int a = 0; a < D / 32; ++a) {
+                        if (PK && (a & 1) != par) continue;   // the other parity's group
                         const int k = G32 ? 8 * a + g : (D / 32) * g + a;
                         *reinterpret_cast<float4*>(slot + h * D + 4 * (k ^ mswz<D, G32>(h))) =
                             make_float4(o[2 * a][nt][c] * down, o[2 * a][nt][c + 2] * down,
@@ -1155,12 +1198,12 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D, bool G32, bool PAGED, bool G16>
+template <int D, bool G32, bool PAGED, bool G16, bool PK>
 cudaError_t set_attrs() {
     using Lay = Layout<D, G32, G16>;
     static bool done = false;
     if (done) return cudaSuccess;
-    auto kern = decode_split_tc<D, G32, PAGED, G16>;
+    auto kern = decode_split_tc<D, G32, PAGED, G16, PK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -1169,10 +1212,10 @@ cudaError_t set_attrs() {
     return e;
 }
 
-template <int D, bool G32, bool PAGED, bool G16>
+template <int D, bool G32, bool PAGED, bool G16, bool PK>
 cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     using Lay = Layout<D, G32, G16>;
-    cudaError_t e = set_attrs<D, G32, PAGED, G16>();
+    cudaError_t e = set_attrs<D, G32, PAGED, G16, PK>();
     if (e != cudaSuccess) return e;
     CUtensorMap mk, mv;
     const int64_t rows = PAGED ? static_cast<int64_t>(p.num_pages) * p.Hk * 16
@@ -1191,12 +1234,15 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16>, mk, mv, p);
+    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16, PK>, mk, mv, p);
 }
 
 template <int D, bool G32, bool PAGED>
 cudaError_t pick_g(const DecodeParams& p, cudaStream_t s) {
-    return p.G > 8 ? launch_tc<D, G32, PAGED, true>(p, s) : launch_tc<D, G32, PAGED, false>(p, s);
+    if (p.G > 8) return launch_tc<D, G32, PAGED, true, false>(p, s);
+    if constexpr (G32)
+        if (p.G <= 4) return launch_tc<D, G32, PAGED, false, true>(p, s);
+    return launch_tc<D, G32, PAGED, false, false>(p, s);
 }
 
 template <int D>

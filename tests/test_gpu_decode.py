@@ -179,9 +179,11 @@ def test_decode_peaky_softmax(G):
     assert_attn_close(out, c.oracle_decode(q, sl, f32_scale(D)), "peaky")
 
 
-def test_decode_large_query_magnitudes():
-    """Query rows of very different magnitude (the per-head f16 prescale)."""
-    B, Hk, G, D, L = 1, 2, 8, 128, 200
+@pytest.mark.parametrize("G", [4, 8])
+def test_decode_large_query_magnitudes(G):
+    """Query rows of very different magnitude (the per-head integer prescale;
+    G = 4 also runs the group-pair packing of group-32 scales)."""
+    B, Hk, D, L = 1, 2, 128, 200
     c, q = _fill_contig(B, Hk * G, Hk, D, "group32", [L], seed=23)
     qf = q.float()
     qf[0, 0] *= 1e-20
