@@ -62,6 +62,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "kvq_internal.cuh"
 #include "kvq_ptx.cuh"
 
@@ -462,163 +464,170 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // floats in each scale array (contiguous layout)
         const int64_t sc_total = static_cast<int64_t>(B) * Hk * max_seq * NG;
         const uint32_t q_bytes = static_cast<uint32_t>(G * D * 2);
-        int count = 0;                  // tiles issued (ring position)
-        if (one) grid_dep_wait();       // before the length, table, q and cache reads
+        // the issue loop is compiled once for blocks of items and once for one
+        // item per CTA, so the former carries none of the latter's bookkeeping
+        auto produce = [&](auto one_tag) {
+            constexpr bool ONE = decltype(one_tag)::value;
+            int count = 0;                  // tiles issued (ring position)
+            if (ONE) grid_dep_wait();       // before the length, table, q and cache reads
 #pragma unroll 1
-        for (int i = ibeg; i < iend;) {
-            // one item per CTA: the length load is issued first and used only
-            // after the first stage is on its way (the chunk's end stands in)
-            int Lone = 0;
-            if (one) Lone = one_raw();
-            const Seg sg = one ? one_seg((one_j + 1) * chunk) : seg_at(i, iend, lens, nsv, cum, B, chunk);
-            i = sg.next;
-            if (sg.ns == 0) continue;
-            int t1 = sg.t1;
-            uint32_t spec_valid = ~0u;      // paged, one item: the first stage's loaded pages
-            const int b = sg.b, hk = sg.hk;
-            const uint16_t* qsrc = qg + (static_cast<int64_t>(b) * Hq + hk * G) * D;
-            int seg_tiles = 0;          // tiles issued for this segment
-            if (one && pw == 0 && lane == 0) {
-                // one item per CTA: the query rows go first, on their own
-                // barrier, into stage 0's query area (no stage carries them), so
-                // the consumers build their Q operand while K and V are in flight
-                ptx::mbar_arrive_expect_tx(bar_q, q_bytes);
-                ptx::bulk_load(sbase + Lay::Q_OFF, qsrc, q_bytes, bar_q);
-            }
-            // paged: the segment's page ids, 32 pages (4 stages) per register,
-            // loaded one group of 4 stages ahead so the table read is off the
-            // issue path; lane i holds page pbase + i (-1: none or out of range)
-            int pbase = sg.t0 >> 4;
-            int32_t pg_cur = -1, pg_nxt = -1;
-            auto load_pages = [&](int first) {
-                const int idx = first + lane;
-                int32_t v = -1;
-                if (16 * idx < t1 && idx < max_pages) {
-                    v = table[static_cast<int64_t>(b) * max_pages + idx];
-                    if (v < 0 || v >= num_pages) v = -1;
+            for (int i = ibeg; i < iend;) {
+                // one item per CTA: the length load is issued first and used only
+                // after the first stage is on its way (the chunk's end stands in)
+                int Lone = 0;
+                if (ONE) Lone = one_raw();
+                const Seg sg = ONE ? one_seg((one_j + 1) * chunk) : seg_at(i, iend, lens, nsv, cum, B, chunk);
+                i = sg.next;
+                if (sg.ns == 0) continue;
+                int t1 = sg.t1;
+                uint32_t spec_valid = ~0u;      // paged, ONE item: the first stage's loaded pages
+                const int b = sg.b, hk = sg.hk;
+                const uint16_t* qsrc = qg + (static_cast<int64_t>(b) * Hq + hk * G) * D;
+                int seg_tiles = 0;          // tiles issued for this segment
+                if (ONE && pw == 0 && lane == 0) {
+                    // one item per CTA: the query rows go first, on their own
+                    // barrier, into stage 0's query area (no stage carries them), so
+                    // the consumers build their Q operand while K and V are in flight
+                    ptx::mbar_arrive_expect_tx(bar_q, q_bytes);
+                    ptx::bulk_load(sbase + Lay::Q_OFF, qsrc, q_bytes, bar_q);
                 }
-                return v;
-            };
-            if (PAGED) {
-                pg_cur = load_pages(pbase);
-                pg_nxt = load_pages(pbase + 32);
-            }
+                // paged: the segment's page ids, 32 pages (4 stages) per register,
+                // loaded ONE group of 4 stages ahead so the table read is off the
+                // issue path; lane i holds page pbase + i (-1: none or out of range)
+                int pbase = sg.t0 >> 4;
+                int32_t pg_cur = -1, pg_nxt = -1;
+                auto load_pages = [&](int first) {
+                    const int idx = first + lane;
+                    int32_t v = -1;
+                    if (16 * idx < t1 && idx < max_pages) {
+                        v = table[static_cast<int64_t>(b) * max_pages + idx];
+                        if (v < 0 || v >= num_pages) v = -1;
+                    }
+                    return v;
+                };
+                if (PAGED) {
+                    pg_cur = load_pages(pbase);
+                    pg_nxt = load_pages(pbase + 32);
+                }
 #pragma unroll 1
-            for (int tt0 = sg.t0; tt0 < t1; tt0 += TT, ++count, ++seg_tiles,
-                     t1 = (one && seg_tiles == 1) ? max(sg.t0, min(sg.t0 + chunk, one_valid(Lone))) : t1) {
-                const int s = count % NST;
-                const uint32_t full = bar_full + 8 * s;
-                if (count >= NST && lane == 0) wait(bar_empty + 8 * s, ((count / NST) - 1) & 1);
-                __syncwarp();
-                const int ntok = min(TT, t1 - tt0);
-                const uint32_t sk = sbase + s * Lay::STAGE;
-                const uint32_t sv = sk + Lay::KV_BYTES;
-                const uint32_t sks = sv + Lay::KV_BYTES;
-                const uint32_t svs = sks + Lay::SC_FLOATS * 4;
-                // the segment's G query rows (contiguous bf16) ride with its first
-                // two stages: each consumer group builds its Q operand from the
-                // first stage it works in the segment (one item per CTA: they
-                // came first, on their own barrier)
-                const bool with_q = !one && seg_tiles < 2;
-                if (!PAGED) {
-                    if (lane == 0) {
-                        const int64_t row0 = (static_cast<int64_t>(b) * Hk + hk) * max_seq + tt0;
-                        // scales: whole 16-byte chunks from the aligned float at or
-                        // below the tile's first one; where the last chunk would run
-                        // past the end of the scale array its 1-3 floats are copied
-                        // by plain loads (before the arrival that publishes them)
-                        const int64_t f0 = row0 * NG;
-                        const int off = static_cast<int>(f0 & 3);
-                        const int64_t c0 = f0 - off;
-                        const int nf = ntok * NG + off;
-                        int nb = (nf + 3) & ~3;
-                        if (c0 + nb > sc_total) {
-                            nb = nf & ~3;
+                for (int tt0 = sg.t0; tt0 < t1; tt0 += TT, ++count, ++seg_tiles,
+                         t1 = (ONE && seg_tiles == 1) ? max(sg.t0, min(sg.t0 + chunk, one_valid(Lone))) : t1) {
+                    const int s = count % NST;
+                    const uint32_t full = bar_full + 8 * s;
+                    if (count >= NST && lane == 0) wait(bar_empty + 8 * s, ((count / NST) - 1) & 1);
+                    __syncwarp();
+                    const int ntok = min(TT, t1 - tt0);
+                    const uint32_t sk = sbase + s * Lay::STAGE;
+                    const uint32_t sv = sk + Lay::KV_BYTES;
+                    const uint32_t sks = sv + Lay::KV_BYTES;
+                    const uint32_t svs = sks + Lay::SC_FLOATS * 4;
+                    // the segment's G query rows (contiguous bf16) ride with its first
+                    // two stages: each consumer group builds its Q operand from the
+                    // first stage it works in the segment (one item per CTA: they
+                    // came first, on their own barrier)
+                    const bool with_q = !ONE && seg_tiles < 2;
+                    if (!PAGED) {
+                        if (lane == 0) {
+                            const int64_t row0 = (static_cast<int64_t>(b) * Hk + hk) * max_seq + tt0;
+                            // scales: whole 16-byte chunks from the aligned float at or
+                            // below the tile's first ONE; where the last chunk would run
+                            // past the end of the scale array its 1-3 floats are copied
+                            // by plain loads (before the arrival that publishes them)
+                            const int64_t f0 = row0 * NG;
+                            const int off = static_cast<int>(f0 & 3);
+                            const int64_t c0 = f0 - off;
+                            const int nf = ntok * NG + off;
+                            int nb = (nf + 3) & ~3;
+                            if (c0 + nb > sc_total) {
+                                nb = nf & ~3;
 #pragma unroll 1
-                            for (int e = nb; e < nf; ++e) {
-                                sts_f32(sks + 4 * e, k_scale[c0 + e]);
-                                sts_f32(svs + 4 * e, v_scale[c0 + e]);
+                                for (int e = nb; e < nf; ++e) {
+                                    sts_f32(sks + 4 * e, k_scale[c0 + e]);
+                                    sts_f32(svs + 4 * e, v_scale[c0 + e]);
+                                }
+                            }
+                            ptx::mbar_arrive_expect_tx(
+                                full, 2 * Lay::KV_BYTES + 8 * nb + (with_q ? q_bytes : 0u));
+                            ptx::tma_load_2d(sk, &tm_k, 0, static_cast<int>(row0), full, pol);
+                            ptx::tma_load_2d(sv, &tm_v, 0, static_cast<int>(row0), full, pol);
+                            if (nb > 0) {
+                                ptx::bulk_load(sks, k_scale + c0, 4 * nb, full);
+                                ptx::bulk_load(svs, v_scale + c0, 4 * nb, full);
+                            }
+                            if (with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
+                        }
+                    } else {
+                        constexpr uint32_t PAGE_BYTES = 16 * D;   // TMA bytes of K (or V) per page
+                        const int np = (ntok + 15) >> 4;
+                        if ((tt0 >> 4) >= pbase + 32) {
+                            pbase += 32;
+                            pg_cur = pg_nxt;
+                            pg_nxt = load_pages(pbase + 32);
+                        }
+                        // a bad entry is skipped (its tokens are masked)
+                        int32_t pg = __shfl_sync(0xffffffffu, pg_cur, (tt0 >> 4) - pbase + (lane & 7));
+                        if (lane >= np) pg = -1;
+                        const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
+                        if (pw == 1) {
+                            // producer warp 1: the V rows of the pages (lane q < 8 loads
+                            // page q: 16 rows of this kv head), its own byte count
+                            if (lane == 0) ptx::mbar_arrive_expect_tx(full, __popc(valid) * PAGE_BYTES);
+                            __syncwarp();
+                            if (pg >= 0)
+                                ptx::tma_load_2d(sv + lane * 16 * D, &tm_v, 0, (pg * Hk + hk) * 16, full,
+                                                 pol);
+                            continue;
+                        }
+                        if (lane == 0) {
+                            // the consumers mask the tokens of pages that were not
+                            // loaded; a bad table entry is reported here
+                            // (one item per CTA: the first stage's range is the chunk's, not
+                            // yet the length's; its pages are checked once the length is known)
+                            if (ONE && seg_tiles == 0) spec_valid = valid;
+                            else if (valid != (1u << np) - 1u) raise_flag(d_err, KVQ_DEVERR_PAGE);
+                            sts_u32(sk + Lay::MASK_OFF, valid);
+                            ptx::mbar_arrive_expect_tx(
+                                full, __popc(valid) * PAGE_BYTES + (with_q ? q_bytes : 0u));
+                            if (with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
+                        }
+                        __syncwarp();
+                        // producer warp 0: lane q < 8 loads page q's K rows; every lane
+                        // copies 16-byte chunks of the pages' scales (16 * NG aligned
+                        // floats per page), chunk c of the stage being page c / (4 NG)
+                        if (pg >= 0)
+                            ptx::tma_load_2d(sk + lane * 16 * D, &tm_k, 0, (pg * Hk + hk) * 16, full, pol);
+#pragma unroll
+                        for (int it = 0; it < NG; ++it) {
+                            const int c = lane + 32 * it;
+                            const int q = c / (4 * NG), cc = c % (4 * NG);
+                            const int pq = __shfl_sync(0xffffffffu, pg, q);
+                            if (pq >= 0) {
+                                const int64_t fc = static_cast<int64_t>((pq * Hk + hk) * 16) * NG + 4 * cc;
+                                ptx::cp_async_16(sks + 16 * c, k_scale + fc);
+                                ptx::cp_async_16(svs + 16 * c, v_scale + fc);
                             }
                         }
-                        ptx::mbar_arrive_expect_tx(
-                            full, 2 * Lay::KV_BYTES + 8 * nb + (with_q ? q_bytes : 0u));
-                        ptx::tma_load_2d(sk, &tm_k, 0, static_cast<int>(row0), full, pol);
-                        ptx::tma_load_2d(sv, &tm_v, 0, static_cast<int>(row0), full, pol);
-                        if (nb > 0) {
-                            ptx::bulk_load(sks, k_scale + c0, 4 * nb, full);
-                            ptx::bulk_load(svs, v_scale + c0, 4 * nb, full);
-                        }
-                        if (with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
+                        ptx::cp_async_arrive_noinc(full);
                     }
-                } else {
-                    constexpr uint32_t PAGE_BYTES = 16 * D;   // TMA bytes of K (or V) per page
-                    const int np = (ntok + 15) >> 4;
-                    if ((tt0 >> 4) >= pbase + 32) {
-                        pbase += 32;
-                        pg_cur = pg_nxt;
-                        pg_nxt = load_pages(pbase + 32);
-                    }
-                    // a bad entry is skipped (its tokens are masked)
-                    int32_t pg = __shfl_sync(0xffffffffu, pg_cur, (tt0 >> 4) - pbase + (lane & 7));
-                    if (lane >= np) pg = -1;
-                    const uint32_t valid = __ballot_sync(0xffffffffu, pg >= 0);
-                    if (pw == 1) {
-                        // producer warp 1: the V rows of the pages (lane q < 8 loads
-                        // page q: 16 rows of this kv head), its own byte count
-                        if (lane == 0) ptx::mbar_arrive_expect_tx(full, __popc(valid) * PAGE_BYTES);
-                        __syncwarp();
-                        if (pg >= 0)
-                            ptx::tma_load_2d(sv + lane * 16 * D, &tm_v, 0, (pg * Hk + hk) * 16, full,
-                                             pol);
-                        continue;
-                    }
-                    if (lane == 0) {
-                        // the consumers mask the tokens of pages that were not
-                        // loaded; a bad table entry is reported here
-                        // (one item per CTA: the first stage's range is the chunk's, not
-                        // yet the length's; its pages are checked once the length is known)
-                        if (one && seg_tiles == 0) spec_valid = valid;
-                        else if (valid != (1u << np) - 1u) raise_flag(d_err, KVQ_DEVERR_PAGE);
-                        sts_u32(sk + Lay::MASK_OFF, valid);
-                        ptx::mbar_arrive_expect_tx(
-                            full, __popc(valid) * PAGE_BYTES + (with_q ? q_bytes : 0u));
-                        if (with_q) ptx::bulk_load(sk + Lay::Q_OFF, qsrc, q_bytes, full);
-                    }
-                    __syncwarp();
-                    // producer warp 0: lane q < 8 loads page q's K rows; every lane
-                    // copies 16-byte chunks of the pages' scales (16 * NG aligned
-                    // floats per page), chunk c of the stage being page c / (4 NG)
-                    if (pg >= 0)
-                        ptx::tma_load_2d(sk + lane * 16 * D, &tm_k, 0, (pg * Hk + hk) * 16, full, pol);
-#pragma unroll
-                    for (int it = 0; it < NG; ++it) {
-                        const int c = lane + 32 * it;
-                        const int q = c / (4 * NG), cc = c % (4 * NG);
-                        const int pq = __shfl_sync(0xffffffffu, pg, q);
-                        if (pq >= 0) {
-                            const int64_t fc = static_cast<int64_t>((pq * Hk + hk) * 16) * NG + 4 * cc;
-                            ptx::cp_async_16(sks + 16 * c, k_scale + fc);
-                            ptx::cp_async_16(svs + 16 * c, v_scale + fc);
-                        }
-                    }
-                    ptx::cp_async_arrive_noinc(full);
+                }
+                if (PAGED && ONE && lane == 0) {
+                    // the first stage's pages inside the sequence must all have loaded
+                    const int nreal = min(max(t1 - sg.t0, 0), TT);
+                    const uint32_t need = nreal >= 16 * 32 ? ~0u : (1u << ((nreal + 15) >> 4)) - 1u;
+                    if ((spec_valid & need) != need) raise_flag(d_err, KVQ_DEVERR_PAGE);
                 }
             }
-            if (PAGED && one && lane == 0) {
-                // the first stage's pages inside the sequence must all have loaded
-                const int nreal = min(max(t1 - sg.t0, 0), TT);
-                const uint32_t need = nreal >= 16 * 32 ? ~0u : (1u << ((nreal + 15) >> 4)) - 1u;
-                if ((spec_valid & need) != need) raise_flag(d_err, KVQ_DEVERR_PAGE);
-            }
-        }
-        // the last tile of every slot has landed (normally long consumed; after a
-        // timeout this keeps the CTA alive until its bulk copies are done)
-        if (PAGED) asm volatile("cp.async.wait_all;" ::: "memory");
-        if (lane == 0)
+            // the last tile of every slot has landed (normally long consumed; after a
+            // timeout this keeps the CTA alive until its bulk copies are done)
+            if (PAGED) asm volatile("cp.async.wait_all;" ::: "memory");
+            if (lane == 0)
 #pragma unroll 1
-            for (int c = count - 1; c >= 0 && c >= count - NST; --c)
-                ptx::mbar_wait(bar_full + 8 * (c % NST), (c / NST) & 1);
-        if (one && pw == 0 && lane == 0) ptx::mbar_wait(bar_q, 0);
+                for (int c = count - 1; c >= 0 && c >= count - NST; --c)
+                    ptx::mbar_wait(bar_full + 8 * (c % NST), (c / NST) & 1);
+            if (ONE && pw == 0 && lane == 0) ptx::mbar_wait(bar_q, 0);
+        };
+        if (one) produce(std::true_type{});
+        else produce(std::false_type{});
         return;                         // consumers synchronise among themselves (barrier 1)
     }
 
