@@ -244,22 +244,25 @@ class Layer:
             self.chunk_v = inp.v_hist[:, :, p0:p0 + self.chunk_T].contiguous().to(dev)
             self.chunk_pos = torch.full((B,), p0, dtype=torch.int32, device=dev)
 
-    def append(self, kvq):
+    def append(self, kvq, k_new=None, v_new=None, stream=None):
+        k_new = self.k_new if k_new is None else k_new
+        v_new = self.v_new if v_new is None else v_new
         if self.chunk_T:
             kvq.kvq_append(self.chunk_k, self.chunk_v, self.chunk_pos, self.k, self.v, self.ks,
-                           self.vs, self.wl.mode)
+                           self.vs, self.wl.mode, stream=stream)
         if self.paged:
-            kvq.kvq_append_paged(self.k_new, self.v_new, self.pos, self.k, self.v, self.ks,
-                                 self.vs, self.table, 16, self.wl.mode)
+            kvq.kvq_append_paged(k_new, v_new, self.pos, self.k, self.v, self.ks,
+                                 self.vs, self.table, 16, self.wl.mode, stream=stream)
         else:
-            kvq.kvq_append(self.k_new, self.v_new, self.pos, self.k, self.v, self.ks, self.vs,
-                           self.wl.mode)
+            kvq.kvq_append(k_new, v_new, self.pos, self.k, self.v, self.ks, self.vs,
+                           self.wl.mode, stream=stream)
 
-    def decode(self, kvq, workspace):
-        kvq.kvq_decode_attn(self.q, self.k, self.v, self.ks, self.vs, self.seq_lens, self.hint,
-                            mode=self.wl.mode, out=self.out, workspace=workspace,
+    def decode(self, kvq, workspace, q=None, out=None, stream=None):
+        kvq.kvq_decode_attn(self.q if q is None else q, self.k, self.v, self.ks, self.vs,
+                            self.seq_lens, self.hint, mode=self.wl.mode,
+                            out=self.out if out is None else out, workspace=workspace,
                             page_table=self.table, page_size=16 if self.paged else 0,
-                            view=self.view)
+                            view=self.view, stream=stream)
 
 
 def build_layers(kvq, wl, n_layers, dev, keep_host=False):
@@ -511,26 +514,37 @@ def run_kvq(args, wl):
 
 def run_e2e(kvq, wl, layers, workspace, dev, K, W, world):
     """Same metric through the public Python API with host buffers: each step
-    copies every layer's q / k_new / v_new from pinned host memory, runs
-    kvq_append + kvq_decode_attn eagerly, and copies the outputs back."""
+    copies every layer's q / k_new / v_new from pinned host memory (one packed
+    copy for the step), runs kvq_append + kvq_decode_attn eagerly for every
+    layer, and copies all the outputs back (one packed copy)."""
     n = len(layers)
-    h_q = [ly.q.cpu().pin_memory() for ly in layers]
-    h_k = [ly.k_new.cpu().pin_memory() for ly in layers]
-    h_v = [ly.v_new.cpu().pin_memory() for ly in layers]
-    h_out = [torch.empty_like(ly.out, device="cpu").pin_memory() for ly in layers]
-    h2d = sum(t.numel() * t.element_size() for t in h_q + h_k + h_v)
-    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    # the step's inputs, packed layer after layer: q, k_new, v_new (bf16)
+    parts = [t for ly in layers for t in (ly.q, ly.k_new, ly.v_new)]
+    h_in = torch.cat([t.reshape(-1).cpu() for t in parts]).pin_memory()
+    d_in = torch.empty_like(h_in, device=dev)
+    views, off = [], 0
+    for t in parts:
+        views.append(d_in[off:off + t.numel()].view(t.shape))
+        off += t.numel()
+    outs = [ly.out for ly in layers]
+    d_out = torch.empty(sum(t.numel() for t in outs), dtype=torch.float32, device=dev)
+    h_out = torch.empty(d_out.numel(), dtype=torch.float32).pin_memory()
+    out_views, off = [], 0
+    for t in outs:
+        out_views.append(d_out[off:off + t.numel()].view(t.shape))
+        off += t.numel()
+    h2d = h_in.numel() * h_in.element_size()
+    d2h = h_out.numel() * h_out.element_size()
     stream = torch.cuda.Stream(dev)
 
     def step():
         with torch.cuda.stream(stream):
+            d_in.copy_(h_in, non_blocking=True)
             for i, ly in enumerate(layers):
-                ly.q.copy_(h_q[i], non_blocking=True)
-                ly.k_new.copy_(h_k[i], non_blocking=True)
-                ly.v_new.copy_(h_v[i], non_blocking=True)
-                ly.append(kvq)
-                ly.decode(kvq, workspace)
-                h_out[i].copy_(ly.out, non_blocking=True)
+                q, k_new, v_new = views[3 * i:3 * i + 3]
+                ly.append(kvq, k_new, v_new, stream=stream)
+                ly.decode(kvq, workspace, q=q, out=out_views[i], stream=stream)
+            h_out.copy_(d_out, non_blocking=True)
 
     for _ in range(max(W, 1)):
         step()

@@ -62,8 +62,16 @@ def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor") -> int:
     return t.data_ptr()
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream, ref: torch.Tensor) -> int:
     if stream is None:
+        # the current stream of the tensor's device, as a raw handle (the
+        # Stream object that torch.cuda.current_stream builds costs more
+        # than the rest of a call)
+        if _raw_stream is not None:
+            return _raw_stream(ref.device.index)
         return torch.cuda.current_stream(ref.device).cuda_stream
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
@@ -160,9 +168,10 @@ def kvq_decode_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *, Hk
         view = cache_view(k, v, k_scale, v_scale, page_table, page_size)
     if out is None:
         out = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
-    need = kvq_decode_workspace_bytes(B, Hq, Hk, D, max_seq_len_hint, num_splits)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:               # (a given workspace's size is checked by the call)
+        need = kvq_decode_workspace_bytes(B, Hq, Hk, D, max_seq_len_hint, num_splits)
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _ptr(workspace, None, "workspace") if workspace is not None else 0
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     check(lib.kvq_decode_attn(
