@@ -63,6 +63,7 @@
 #include <math.h>
 
 #include <type_traits>
+#include <unordered_map>
 
 #include "kvq_internal.cuh"
 #include "kvq_ptx.cuh"
@@ -1191,8 +1192,35 @@ EncodeFn encode_fn() {
     return fn;
 }
 
-// 2-D u8 tensor map over `rows` rows of D bytes, box of box_rows rows.
+// The inputs a tensor map is encoded from (everything else is fixed).
+struct MapKey {
+    uintptr_t base;
+    int64_t rows;
+    int D, box_rows;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && rows == o.rows && D == o.D && box_rows == o.box_rows;
+    }
+};
+struct MapKeyHash {
+    size_t operator()(const MapKey& k) const {
+        uint64_t h = k.base * 0x9E3779B97F4A7C15ull;
+        h ^= static_cast<uint64_t>(k.rows) + 0x7F4A7C15ull + (h << 6) + (h >> 2);
+        h ^= static_cast<uint64_t>(k.D * 1031 + k.box_rows) + (h << 6) + (h >> 2);
+        return static_cast<size_t>(h);
+    }
+};
+
+// 2-D u8 tensor map over `rows` rows of D bytes, box of box_rows rows.  The
+// encoded maps are kept per host thread, keyed by every input of the
+// encoding, so a cached map is the one the encoder would produce again.
 cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, int box_rows) {
+    thread_local std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+    const MapKey key{reinterpret_cast<uintptr_t>(base), rows, D, box_rows};
+    const auto it = cache.find(key);
+    if (it != cache.end()) {
+        *map = it->second;
+        return cudaSuccess;
+    }
     EncodeFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
@@ -1204,7 +1232,10 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    if (cache.size() >= 4096) cache.clear();
+    cache.emplace(key, *map);
+    return cudaSuccess;
 }
 
 template <int D, bool G32, bool PAGED, bool G16, bool PK>
