@@ -13,46 +13,48 @@
 // How (sm_100a):
 //  * Work items are (sequence b, kv head, chunk j) with chunk = p.chunk
 //    tokens, listed in (b, kv head, j) order.  The grid is persistent (at
-//    most one CTA per SM) and CTA c takes a contiguous block of the T items
-//    (T / grid each, the first T % grid CTAs one more), found from a prefix
-//    sum of the per-sequence chunk counts (lengths cached in shared memory).
-//    The items of one (b, kv head) inside a CTA's block form a segment: one
-//    token range, one softmax state.  A segment that is a whole (b, kv head)
-//    writes the final rows; any other writes one partial state (o, m, l)
-//    into the workspace slot of its first chunk.  CTA 0 publishes the
-//    partition (item prefix sums, chunk counts), from which the combine
-//    kernel (kvq_decode.cu) finds the slots that hold a unit's partials.
-//  * CTA = 1 producer warp (warp 0) + 8 consumer warps.  One producer lane
-//    streams 128-token stages into a ring of 3-8 stages (~150-220 KB of
-//    shared memory, one CTA per SM): K and V bytes by TMA tile loads (2-D
-//    tensor maps over the cache rows, 128-byte swizzle for D=128, 64-byte
-//    for D=64), the fp32 scales and, with a segment's first two stages, its
-//    query rows by 1-D bulk copies; all complete on the stage's mbarrier.
-//    It refills a slot as soon as its consumers released it.  The consumers
-//    form two groups of four warps that take alternate stages; a warp takes
-//    32 tokens of its group's stage as two 16-token MMA tiles.
-//  * Per slice, on mma.sync m16n8k16 (f16 in, f32 accumulate), with the
-//    query heads of the GQA group as the N = 8 dimension (two n-tiles when
-//    G > 8):  S^T = K . Q^T (M = 16 tokens, K = head_dim) and
-//    O^T += V^T . P^T (M = 16 head_dim rows, K = 16 tokens).  The operands
-//    are exact: K and V enter as the integers (byte - 128) built in
-//    registers (1024 + byte spliced into an f16 mantissa, minus 1152), and Q
-//    enters as f16 after a per-head power-of-two prescale (bf16 has 8
-//    significant bits, f16 has 11, so q * 2^s is exact).  The K scale (per
-//    token, or per 32-value group with one accumulator per group), 2^-s,
-//    attn_scale and log2(e) are applied to the f32 scores.
+//    most one CTA per SM).  When the items fit the grid, CTA c takes item c
+//    (one item per CTA); otherwise CTA c takes a contiguous block of items
+//    whose weight (items, plus W per (b, kv head) started) is an equal share
+//    of the total, found from prefix sums of the per-sequence chunk counts
+//    (lengths cached in shared memory).  The items of one (b, kv head)
+//    inside a CTA's block form a segment: one token range, one softmax
+//    state.  A segment that is a whole (b, kv head) writes the final rows;
+//    any other writes one partial state (o, m, l) into the workspace slot of
+//    its first chunk, and with blocks of several items m = -inf into the
+//    other slots it covers, so the combine kernel (kvq_decode.cu) finds a
+//    unit's partials from its m slots.
+//  * CTA = 1 producer warp (2 for the paged cache) + 8 consumer warps.  One
+//    producer lane streams 128-token stages into a ring of 3-8 stages
+//    (~150-220 KB of shared memory, one CTA per SM): K and V bytes by TMA
+//    tile loads (2-D tensor maps over the cache rows, 128-byte swizzle for
+//    D=128, 64-byte for D=64), the fp32 scales and, with a segment's first
+//    two stages, its query rows by 1-D bulk copies; all complete on the
+//    stage's mbarrier.  It refills a slot as soon as its consumers released
+//    it.  The consumers form two groups of four warps that take alternate
+//    stages; a warp takes 32 tokens of its group's stage as two 16-token MMA
+//    tiles.
+//  * S^T = K . Q^T on the integer MMA (mma.sync m16n8k32, s32 accumulate),
+//    with the query heads of the GQA group as the N = 8 dimension (two
+//    n-tiles when G > 8): the K bytes are the A operand as loaded, and Q is
+//    a per-head power-of-two prescaled 16-bit integer in two byte digits, so
+//    S = 256 S_hi + S_lo - 128 sum(Qi) is exact.  The K scale (per token, or
+//    per 32-value group with one fold per group), the prescale, attn_scale
+//    and log2(e) are applied to the f32 scores.
 //  * Online softmax in base 2 per head.  The V scale is folded into P:
 //    P'' = 2^(z-m) * v_scale(token) * 2^kv (per 32-value group in group-32
 //    mode), with a running per-warp power of two 2^kv that keeps P'' inside
 //    the f16 normal range.  P'' is split into f16 hi + lo parts (about 22
 //    significant bits together); each part is transposed from the score
 //    accumulator layout into the P^T operand layout with movmatrix and
-//    multiplied with the exact (v - 128) integers.
+//    multiplied on mma.sync m16n8k16 (f32 accumulate) with the exact
+//    (v - 128) integers, O^T += V^T . P^T (M = 16 head_dim rows, K = 16
+//    tokens).
 //  * Token order inside each 16-token MMA tile and the head_dim order of the
 //    MMA k-dimension are permuted so that every shared-memory load of the
 //    swizzled tiles is free of bank conflicts (sigma below).
-//  * A segment's eight warp states are merged in one round through eight
-//    shared-memory slots in register order (deterministic: no atomics).
+//  * A segment's eight warp states are merged behind one named barrier
+//    through head-major shared-memory rows (deterministic: no atomics).
 //  * Programmatic dependent launch: the kernel waits for its predecessor in
 //    the stream before touching inputs and lets the combine kernel launch
 //    early.

@@ -238,8 +238,8 @@ def test_one_workspace_serves_calls_of_any_shape():
 def test_decode_many_units_ragged_with_empty_sequences(mode, num_splits, top):
     """Many (sequence, kv head) units of very different lengths, some empty:
     one-stage chunks, the weighted CTA partition, units split over several
-    CTAs and units finished inside one, and both combine paths (up to 32 slots
-    in one round of loads, more through the slot list)."""
+    CTAs and units finished inside one, and the combine that finds a unit's
+    partials from its m slots (within the first 128 slots and past them)."""
     import random
     rnd = random.Random(num_splits + (7 if mode == "group32" else 0))
     B, Hk, G, D = 40, 4, 2, 64
