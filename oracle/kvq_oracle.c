@@ -216,6 +216,84 @@ int oracle_decode_attn(const uint16_t *q, int B, int Hq, int Hk, int D, int grou
 }
 
 /*
+ * Attention of a chunk of T new queries per (sequence, q head) over the
+ * sequence's cache, causal from the chunk's end, in fp64 over the
+ * dequantized cache.  seq_lens[b] = L counts every cached token including
+ * the chunk's T, so query i sits at position L - T + i and attends to the
+ * positions 0 .. L - T + i.  (abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
+ * forward_attention: cache_offset = seq_len - q_len, query q_pos sees KV
+ * positions up to cache_offset + q_pos; combs-models 0.2.2, src/kv.rs,
+ * attend: a query at global position p attends the keys at positions <= p.)
+ *   q   bf16 [B, Hq, T, D]; out fp64 [B, Hq, T, D]; cache arguments as in
+ *   oracle_decode_attn.  L = 0 gives zero rows; 0 < L < T (a chunk longer
+ *   than the cache it sits in) is a length error and gives zero rows.
+ */
+int oracle_chunk_attn(const uint16_t *q, int B, int Hq, int Hk, int T, int D, int group,
+                      const uint8_t *k, const uint8_t *v, const float *k_scale,
+                      const float *v_scale, int max_seq, int page_size,
+                      const int32_t *table, int max_pages, int num_pages,
+                      const int32_t *seq_lens, double attn_scale, double *out) {
+    int err = 0, ng = D / group, G = Hq / Hk;
+    int64_t cap = page_size > 0 ? (int64_t)max_pages * page_size : max_seq;
+    double *z = NULL, *kh = (double *)malloc(sizeof(double) * D);
+    double *acc = (double *)malloc(sizeof(double) * D);
+    int64_t *rows = NULL;
+    for (int b = 0; b < B; ++b) {
+        int64_t L = seq_lens[b];
+        if (L < 0 || L > cap || (L > 0 && L < T)) { err |= ORACLE_ERR_LEN; L = 0; }
+        rows = (int64_t *)realloc(rows, sizeof(int64_t) * (L > 0 ? L : 1));
+        z = (double *)realloc(z, sizeof(double) * (L > 0 ? L : 1));
+        int bad = 0;
+        for (int64_t t = 0; t < L; ++t) {
+            if (page_size > 0) {
+                int32_t phys = table[(int64_t)b * max_pages + t / page_size];
+                if (phys < 0 || phys >= num_pages) { bad = 1; break; }
+                rows[t] = (int64_t)phys * Hk * page_size + t % page_size;
+            } else {
+                rows[t] = (int64_t)b * Hk * max_seq + t;
+            }
+        }
+        if (bad) { err |= ORACLE_ERR_PAGE; L = 0; }
+        for (int h = 0; h < Hq; ++h) {
+            int hk = h / G;
+            int64_t hstride = page_size > 0 ? page_size : max_seq;
+            for (int i = 0; i < T; ++i) {
+                double *o = out + (((int64_t)b * Hq + h) * T + i) * D;
+                if (L == 0) { for (int d = 0; d < D; ++d) o[d] = 0.0; continue; }
+                const uint16_t *qh = q + (((int64_t)b * Hq + h) * T + i) * D;
+                int64_t visible = L - T + i + 1;          /* positions 0 .. L - T + i */
+                double zmax = -INFINITY;
+                for (int64_t t = 0; t < visible; ++t) {
+                    int64_t row = rows[t] + (int64_t)hk * hstride;
+                    for (int d = 0; d < D; ++d) {
+                        float s = k_scale[row * ng + d / group];
+                        kh[d] = (double)((float)((int)k[row * D + d] - 128) * s);
+                    }
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += (double)widen_bf16(qh[d]) * kh[d];
+                    z[t] = dot * attn_scale;
+                    if (z[t] > zmax) zmax = z[t];
+                }
+                double l = 0.0;
+                for (int d = 0; d < D; ++d) acc[d] = 0.0;
+                for (int64_t t = 0; t < visible; ++t) {
+                    int64_t row = rows[t] + (int64_t)hk * hstride;
+                    double p = exp(z[t] - zmax);
+                    l += p;
+                    for (int d = 0; d < D; ++d) {
+                        float s = v_scale[row * ng + d / group];
+                        acc[d] += p * (double)((float)((int)v[row * D + d] - 128) * s);
+                    }
+                }
+                for (int d = 0; d < D; ++d) o[d] = acc[d] / l;
+            }
+        }
+    }
+    free(z); free(kh); free(acc); free(rows);
+    return err;
+}
+
+/*
  * Bytes of an INT8 cache: layers * 2 (K and V) * (values + scales), with one
  * byte per value and scale_bytes per scale (4 for fp32), as in
  * kv_cache_q8_memory_bytes; group = values per scale.
