@@ -10,7 +10,10 @@ repeated over 32 independent layer caches (277 MB, larger than the 126 MB L2,
 so consecutive reads of a layer never hit in L2).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
-        [--workload llama3_8b_layer|tiny|batched_group32|paged|long_context]
+        [--workload llama3_8b_layer|tiny|batched_group32|paged|long_context] [--qlen T]
+--qlen T > 1 times chunk steps instead: every layer appends a chunk of T new
+tokens and runs kvq_chunk_attn with T queries per head (causal from the
+chunk's end).
 Multi-GPU: launched by torch.distributed.run, one rank per GPU; every rank
 runs its own replica of the workload (weak scaling, no data-path collective);
 the job time is the max over ranks.
@@ -38,6 +41,7 @@ import synth  # noqa: E402
 
 METRIC = "decode-attn INT8-KV GB/s & fraction of HBM peak; tokens/s per layer; append GB/s"
 DEFAULT_WORKLOAD = "llama3_8b_layer"
+QLEN = 1                                  # queries per (sequence, q head) per step (--qlen)
 LAYERS = {"llama3_8b_layer": 32}
 
 
@@ -56,7 +60,7 @@ def decode_bytes(wl, seq_lens, page_size=0):
     page-table entries."""
     ng = 1 if wl.mode == "per_token" else wl.D // 32
     kv = sum(wl.Hk * L * (2 * wl.D + 2 * 4 * ng) for L in seq_lens)
-    qo = wl.B * wl.Hq * wl.D * (2 + 4)
+    qo = wl.B * wl.Hq * wl.D * (2 + 4) * QLEN
     pt = sum((L + 15) // 16 * 4 for L in seq_lens) if page_size else 0
     return kv + qo + pt
 
@@ -231,7 +235,8 @@ class Layer:
         self.q = inp.q.to(dev)
         self.pos = cached.to(dev)
         self.seq_lens = inp.seq_lens.to(dev)
-        self.out = torch.empty(B, wl.Hq, D, device=dev)
+        self.qlen = QLEN
+        self.out = torch.empty((B, wl.Hq, D) if QLEN == 1 else (B, wl.Hq, QLEN, D), device=dev)
         self.view = kvq.cache_view(self.k, self.v, self.ks, self.vs, self.table,
                                    16 if self.paged else 0)
         if keep_host:
@@ -258,7 +263,8 @@ class Layer:
                            self.wl.mode, stream=stream)
 
     def decode(self, kvq, workspace, q=None, out=None, stream=None):
-        kvq.kvq_decode_attn(self.q if q is None else q, self.k, self.v, self.ks, self.vs,
+        call = kvq.kvq_decode_attn if self.qlen == 1 else kvq.kvq_chunk_attn
+        call(self.q if q is None else q, self.k, self.v, self.ks, self.vs,
                             self.seq_lens, self.hint, mode=self.wl.mode,
                             out=self.out if out is None else out, workspace=workspace,
                             page_table=self.table, page_size=16 if self.paged else 0,
@@ -268,7 +274,7 @@ class Layer:
 def build_layers(kvq, wl, n_layers, dev, keep_host=False):
     layers = []
     for i in range(n_layers):
-        inp = synth.make_decode_inputs(wl, seed=wl.seed + 7919 * i)
+        inp = synth.make_decode_inputs(wl, seed=wl.seed + 7919 * i, qlen=QLEN)
         layers.append(Layer(kvq, wl, inp, dev, keep_host=keep_host and i == 0))
         del inp
     torch.cuda.synchronize(dev)
@@ -285,7 +291,7 @@ class OracleLayer:
         import oracle  # test infrastructure: used only by the CPU baseline legs
         self.oracle = oracle
         self.wl = wl
-        inp = synth.make_decode_inputs(wl, seed=seed)
+        inp = synth.make_decode_inputs(wl, seed=seed, qlen=QLEN)
         self.inp = inp
         B, Hk, D = wl.B, wl.Hk, wl.D
         ng = 1 if wl.mode == "per_token" else D // 32
@@ -324,13 +330,14 @@ class OracleLayer:
         if self.paged:
             o.append_paged(inp.k_new, inp.cached, self.k, self.ks, inp.page_table, 16, wl.mode)
             o.append_paged(inp.v_new, inp.cached, self.v, self.vs, inp.page_table, 16, wl.mode)
-            o.decode_attn(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale,
-                          wl.mode, page_size=16, table=inp.page_table)
+            attn = o.decode_attn if QLEN == 1 else o.chunk_attn
+            attn(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale, wl.mode,
+                 page_size=16, table=inp.page_table)
         else:
             o.append_contig(inp.k_new, inp.cached, self.k, self.ks, wl.mode)
             o.append_contig(inp.v_new, inp.cached, self.v, self.vs, wl.mode)
-            o.decode_attn(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale,
-                          wl.mode)
+            attn = o.decode_attn if QLEN == 1 else o.chunk_attn
+            attn(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale, wl.mode)
         return time.perf_counter() - t0
 
 
@@ -374,8 +381,8 @@ def run_reference(args, wl):
         "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hk": wl.Hk, "D": wl.D,
-                   "seq_len": wl.len_hi + 1, "scale_mode": wl.mode, "layout": wl.layout,
-                   "sample": "1 layer step per step"},
+                   "seq_len": wl.len_hi + QLEN, "scale_mode": wl.mode, "layout": wl.layout,
+                   "q_len": QLEN, "sample": "1 layer step per step"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -405,7 +412,8 @@ def run_kvq(args, wl):
     n_layers = args.layers or LAYERS.get(wl.name, 1)
     layers = build_layers(kvq, wl, n_layers, dev)
     L0 = layers[0]
-    ws_bytes = kvq.kvq_decode_workspace_bytes(wl.B, wl.Hq, wl.Hk, wl.D, L0.hint)
+    ws_bytes = (kvq.kvq_decode_workspace_bytes(wl.B, wl.Hq, wl.Hk, wl.D, L0.hint) if QLEN == 1
+                else kvq.kvq_chunk_workspace_bytes(wl.B, wl.Hq, wl.Hk, QLEN, wl.D, L0.hint))
     workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     chunk, splits = kvq.kvq_decode_plan(wl.B, wl.Hk, L0.hint)
     # append (+ prefill-chunk append) + split kernel (+ combine kernel when a
@@ -456,12 +464,12 @@ def run_kvq(args, wl):
     t_append_max = reduce_max(t_append, dev)
 
     dec_b = sum(decode_bytes(wl, ly.seq_lens_list, 16 if ly.paged else 0) for ly in layers)
-    app_b = sum(append_bytes(wl, 1) + (append_bytes(wl, wl.prefill_chunk) if wl.prefill_chunk
+    app_b = sum(append_bytes(wl, QLEN) + (append_bytes(wl, wl.prefill_chunk) if wl.prefill_chunk
                                        else 0) for _ in layers)
     value = world * dec_b * K / t_decode_max / 1e9
     per_layer_decode = t_decode_max / (K * n_layers)
     per_layer_append = t_append_max / (K * n_layers)
-    tokens_per_s_per_layer = wl.B / (per_layer_append + per_layer_decode)
+    tokens_per_s_per_layer = wl.B * QLEN / (per_layer_append + per_layer_decode)
     append_gbs = app_b * K / t_append_max / 1e9
 
     peak, peak_kind = measured_peaks()
@@ -482,7 +490,8 @@ def run_kvq(args, wl):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
         "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hk": wl.Hk, "D": wl.D,
-                   "seq_len": L0.hint, "scale_mode": wl.mode, "layout": wl.layout,
+                   "seq_len": L0.hint, "q_len": QLEN, "scale_mode": wl.mode,
+                   "layout": wl.layout,
                    "layers_per_step": n_layers, "parallelism": f"replicas x{world}",
                    "l2": ("inputs larger than L2 (%.0f MB per step)"
                           % ((dec_b + app_b) / 1e6)),
@@ -574,7 +583,13 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--cpu-layers", type=int, default=400)
+    ap.add_argument("--qlen", type=int, default=1,
+                    help="queries per head per step: > 1 runs chunk attention steps")
     args = ap.parse_args(argv)
+    global QLEN
+    if args.qlen < 1:
+        ap.error("--qlen must be at least 1")
+    QLEN = args.qlen
     args.warmup = max(args.warmup, 3)     # timing rule: at least 3 untimed warm-up steps
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":

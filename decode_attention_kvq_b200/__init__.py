@@ -182,6 +182,44 @@ def kvq_decode_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *, Hk
     return out
 
 
+def kvq_chunk_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *, Hk=None,
+                   page_table=None, page_size=0, attn_scale=None, mode="per_token",
+                   out=None, workspace=None, num_splits=0, err=None, stream=None,
+                   view: Optional[CacheView] = None):
+    """Attention of a chunk of T queries per (sequence, q head), causal from
+    the chunk's end; returns fp32 [B,Hq,T,D].
+
+    q bf16 [B,Hq,T,D]; seq_lens int32 [B] counts the cached tokens including
+    the chunk's T.  Cache arguments as for kvq_decode_attn.
+    """
+    B, Hq, T, D = q.shape
+    if Hk is None:
+        Hk = k.shape[1]
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    if view is None:
+        view = cache_view(k, v, k_scale, v_scale, page_table, page_size)
+    if out is None:
+        out = torch.empty(B, Hq, T, D, dtype=torch.float32, device=q.device)
+    if workspace is None:               # (a given workspace's size is checked by the call)
+        need = kvq_chunk_workspace_bytes(B, Hq, Hk, T, D, max_seq_len_hint, num_splits)
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace, None, "workspace") if workspace is not None else 0
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    check(lib.kvq_chunk_attn(
+        _ptr(q, torch.bfloat16, "q"), B, Hq, Hk, T, D, _mode(mode), ctypes.byref(view),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(max_seq_len_hint), float(attn_scale),
+        _ptr(out, torch.float32, "out"), ws_ptr, ws_bytes, int(num_splits),
+        _ptr(err, torch.int32, "err"), _stream(stream, q)), "kvq_chunk_attn")
+    return out
+
+
+def kvq_chunk_workspace_bytes(B, Hq, Hk, T, D, max_seq_len_hint, num_splits=0) -> int:
+    return int(lib.kvq_chunk_workspace_bytes(B, Hq, Hk, T, D, int(max_seq_len_hint),
+                                             int(num_splits)))
+
+
 def kvq_decode_attn_noalloc(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *,
                             Hk=None, page_table=None, page_size=0, attn_scale=None,
                             mode="per_token", out=None, num_splits=0, err=None, stream=None,

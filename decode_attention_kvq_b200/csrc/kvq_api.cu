@@ -4,6 +4,8 @@
 // kvq_read_error, whose job is to read the device error word.
 #include <stdint.h>
 
+#include <cstdint>
+
 #include "kvq_internal.cuh"
 
 namespace {
@@ -73,6 +75,84 @@ size_t workspace_for(int B, int Hq, int D, int splits) {
     return static_cast<size_t>(B) * Hq * splits * (D + 2) * sizeof(float);
 }
 
+// Decode (T = 1) and chunk (T > 1) attention: the T queries of a (sequence,
+// q head) ride as T rows of the GQA group, so the split kernel sees Hq * T
+// heads, G * T per kv head, and masks each row causally.
+kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_scale_mode mode,
+                  const kvq_cache_view* kv, const int32_t* d_seq_lens, int max_seq_len_hint,
+                  float attn_scale, float* out, void* workspace, size_t workspace_bytes,
+                  int num_splits, int32_t* d_err, kvq_stream_t stream) {
+    if (!q || !kv || !kv->k || !kv->v || !kv->k_scale || !kv->v_scale || !d_seq_lens || !out)
+        return KVQ_ERR_INVALID_ARG;
+    if (B < 0 || Hq < 1 || Hk < 1 || (Hq % Hk) != 0 || D < 16 || (D % 16) != 0 ||
+        max_seq_len_hint < 0 || num_splits < 0 || B > 65535 || Hk > 65535)
+        return KVQ_ERR_INVALID_ARG;
+    if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_INVALID_ARG;
+    if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
+    if (kv->page_size == 16) {
+        if (!kv->page_table || !aligned(kv->page_table, 4) || kv->max_pages < 1 ||
+            kv->num_pages < 1)
+            return KVQ_ERR_INVALID_ARG;
+    } else if (kv->page_size == 0) {
+        if (kv->max_seq < 1) return KVQ_ERR_INVALID_ARG;
+    } else {
+        return KVQ_ERR_INVALID_ARG;
+    }
+    if (!aligned(q, 16) || !aligned(kv->k, 16) || !aligned(kv->v, 16) ||
+        !aligned(kv->k_scale, 16) || !aligned(kv->v_scale, 16) || !aligned(d_seq_lens, 4) ||
+        !aligned(out, 16) || !aligned(workspace, 16) || !aligned(d_err, 4))
+        return KVQ_ERR_INVALID_ARG;
+    if (T > 16 || Hq > 65535) return KVQ_ERR_UNSUPPORTED;
+    const int G = Hq / Hk * T;          // rows per kv head: (head, query), query fastest
+    if (D != 64 && D != 128) return KVQ_ERR_UNSUPPORTED;
+    if (G > 16) return KVQ_ERR_UNSUPPORTED;
+    // the split kernel keeps every sequence length in shared memory
+    if (B > kvq::kMaxBatch) return KVQ_ERR_UNSUPPORTED;
+    // TMA row coordinates are 32-bit
+    const int64_t rows = kv->page_size ? static_cast<int64_t>(kv->num_pages) * Hk * 16
+                                       : static_cast<int64_t>(B) * Hk * kv->max_seq;
+    if (rows >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+    if (B == 0) return KVQ_OK;
+
+    int chunk = 0, splits = 0;
+    kvq_status st = plan(B, Hk, max_seq_len_hint, num_splits, 0, &chunk, &splits);
+    if (st != KVQ_OK) return st;
+    // work items (sequence, kv head, chunk) are counted in 32-bit integers
+    if (static_cast<int64_t>(B) * Hk * (splits + 3) >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+    const size_t need = workspace_for(B, Hq * T, D, splits);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return KVQ_ERR_INVALID_ARG;
+
+    kvq::DecodeParams p{};
+    p.q = q; p.k = kv->k; p.v = kv->v; p.k_scale = kv->k_scale; p.v_scale = kv->v_scale;
+    p.table = kv->page_table; p.seq_lens = d_seq_lens; p.out = out; p.d_err = d_err;
+    // [o: n_part * D][m: n_part][l: n_part]
+    float* ws = static_cast<float*>(workspace);
+    const size_t n_part = static_cast<size_t>(B) * Hq * T * splits;
+    p.ws_o = ws;
+    p.ws_m = ws ? ws + n_part * D : nullptr;
+    p.ws_l = ws ? ws + n_part * (D + 1) : nullptr;
+    p.B = B; p.Hq = Hq * T; p.Hk = Hk; p.G = G; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
+    p.qlen = T;
+    p.page_size = kv->page_size; p.max_seq = kv->max_seq; p.max_pages = kv->max_pages;
+    p.num_pages = kv->num_pages; p.chunk = chunk; p.splits = splits;
+    {
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        const int64_t items = static_cast<int64_t>(B) * Hk * splits;
+        p.grid = static_cast<int>(items < sms ? items : sms);   // persistent: one CTA per SM
+        if (p.grid > kvq::kMaxGrid) p.grid = kvq::kMaxGrid;
+        p.one_item = items <= p.grid ? 1 : 0;
+    }
+    p.scale_log2 = attn_scale * 1.4426950408889634f;
+    // one-stage chunks (many units): a CTA pays about three stages of time
+    // for every (sequence, kv head) it starts (merge, query set-up), so each
+    // unit start weighs three items when the items are divided among the CTAs
+    p.seg_w = (chunk <= 128 && !p.one_item) ? 3 : 0;
+    return from_cuda(kvq::launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
 }  // namespace
 
 extern "C" {
@@ -132,73 +212,24 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
                            int max_seq_len_hint, float attn_scale, float* out, void* workspace,
                            size_t workspace_bytes, int num_splits, int32_t* d_err,
                            kvq_stream_t stream) {
-    if (!q || !kv || !kv->k || !kv->v || !kv->k_scale || !kv->v_scale || !d_seq_lens || !out)
-        return KVQ_ERR_INVALID_ARG;
-    if (B < 0 || Hq < 1 || Hk < 1 || (Hq % Hk) != 0 || D < 16 || (D % 16) != 0 ||
-        max_seq_len_hint < 0 || num_splits < 0 || B > 65535 || Hk > 65535)
-        return KVQ_ERR_INVALID_ARG;
-    if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_INVALID_ARG;
-    if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
-    if (kv->page_size == 16) {
-        if (!kv->page_table || !aligned(kv->page_table, 4) || kv->max_pages < 1 ||
-            kv->num_pages < 1)
-            return KVQ_ERR_INVALID_ARG;
-    } else if (kv->page_size == 0) {
-        if (kv->max_seq < 1) return KVQ_ERR_INVALID_ARG;
-    } else {
-        return KVQ_ERR_INVALID_ARG;
-    }
-    if (!aligned(q, 16) || !aligned(kv->k, 16) || !aligned(kv->v, 16) ||
-        !aligned(kv->k_scale, 16) || !aligned(kv->v_scale, 16) || !aligned(d_seq_lens, 4) ||
-        !aligned(out, 16) || !aligned(workspace, 16) || !aligned(d_err, 4))
-        return KVQ_ERR_INVALID_ARG;
-    const int G = Hq / Hk;
-    if (D != 64 && D != 128) return KVQ_ERR_UNSUPPORTED;
-    if (G > 16) return KVQ_ERR_UNSUPPORTED;
-    // the split kernel keeps every sequence length in shared memory
-    if (B > kvq::kMaxBatch) return KVQ_ERR_UNSUPPORTED;
-    // TMA row coordinates are 32-bit
-    const int64_t rows = kv->page_size ? static_cast<int64_t>(kv->num_pages) * Hk * 16
-                                       : static_cast<int64_t>(B) * Hk * kv->max_seq;
-    if (rows >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
-    if (B == 0) return KVQ_OK;
+    return attend(q, B, Hq, Hk, 1, D, mode, kv, d_seq_lens, max_seq_len_hint, attn_scale, out,
+                  workspace, workspace_bytes, num_splits, d_err, stream);
+}
 
-    int chunk = 0, splits = 0;
-    kvq_status st = plan(B, Hk, max_seq_len_hint, num_splits, 0, &chunk, &splits);
-    if (st != KVQ_OK) return st;
-    // work items (sequence, kv head, chunk) are counted in 32-bit integers
-    if (static_cast<int64_t>(B) * Hk * (splits + 3) >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
-    const size_t need = workspace_for(B, Hq, D, splits);
-    if (need > 0 && (!workspace || workspace_bytes < need)) return KVQ_ERR_INVALID_ARG;
+kvq_status kvq_chunk_attn(const uint16_t* q, int B, int Hq, int Hk, int T, int D,
+                          kvq_scale_mode mode, const kvq_cache_view* kv,
+                          const int32_t* d_seq_lens, int max_seq_len_hint, float attn_scale,
+                          float* out, void* workspace, size_t workspace_bytes, int num_splits,
+                          int32_t* d_err, kvq_stream_t stream) {
+    if (T < 1) return KVQ_ERR_INVALID_ARG;
+    return attend(q, B, Hq, Hk, T, D, mode, kv, d_seq_lens, max_seq_len_hint, attn_scale, out,
+                  workspace, workspace_bytes, num_splits, d_err, stream);
+}
 
-    kvq::DecodeParams p{};
-    p.q = q; p.k = kv->k; p.v = kv->v; p.k_scale = kv->k_scale; p.v_scale = kv->v_scale;
-    p.table = kv->page_table; p.seq_lens = d_seq_lens; p.out = out; p.d_err = d_err;
-    // [o: n_part * D][m: n_part][l: n_part]
-    float* ws = static_cast<float*>(workspace);
-    const size_t n_part = static_cast<size_t>(B) * Hq * splits;
-    p.ws_o = ws;
-    p.ws_m = ws ? ws + n_part * D : nullptr;
-    p.ws_l = ws ? ws + n_part * (D + 1) : nullptr;
-    p.B = B; p.Hq = Hq; p.Hk = Hk; p.G = G; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
-    p.page_size = kv->page_size; p.max_seq = kv->max_seq; p.max_pages = kv->max_pages;
-    p.num_pages = kv->num_pages; p.chunk = chunk; p.splits = splits;
-    {
-        int dev = 0, sms = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return KVQ_ERR_CUDA;
-        const int64_t items = static_cast<int64_t>(B) * Hk * splits;
-        p.grid = static_cast<int>(items < sms ? items : sms);   // persistent: one CTA per SM
-        if (p.grid > kvq::kMaxGrid) p.grid = kvq::kMaxGrid;
-        p.one_item = items <= p.grid ? 1 : 0;
-    }
-    p.scale_log2 = attn_scale * 1.4426950408889634f;
-    // one-stage chunks (many units): a CTA pays about three stages of time
-    // for every (sequence, kv head) it starts (merge, query set-up), so each
-    // unit start weighs three items when the items are divided among the CTAs
-    p.seg_w = (chunk <= 128 && !p.one_item) ? 3 : 0;
-    return from_cuda(kvq::launch_decode(p, static_cast<cudaStream_t>(stream)));
+size_t kvq_chunk_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_seq_len_hint,
+                                 int num_splits) {
+    if (T < 1 || Hq > INT32_MAX / T) return 0;
+    return kvq_decode_workspace_bytes(B, Hq * T, Hk, D, max_seq_len_hint, num_splits);
 }
 
 kvq_status kvq_dequant(const uint8_t* q, const float* scale, int64_t rows, int D,

@@ -234,7 +234,10 @@ __device__ __forceinline__ Seg seg_at(int i, int iend, const int* lens, const in
 // and one fold; lanes t and t ^ 2 (the two parities) add their scores.  P''
 // is built once per group pair, each column with its own parity's V scale;
 // the P.V output columns of the other parity are not used.
-template <int D, bool G32, bool PAGED, bool G16, bool PK>
+// CAUSAL (a chunk of T = p.qlen queries per sequence and q head): the G
+// columns are (head, query i) rows, query fastest, and column i of a sequence
+// of length L sees the positions <= L - T + i (L counts the chunk's tokens).
+template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL>
 __global__ void __launch_bounds__(nthreads(PAGED), 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ DecodeParams prm) {
@@ -247,6 +250,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     constexpr int NT = G16 ? 2 : 1;     // n-tiles of 8 query heads
     constexpr int NGV = G32 ? NG : 1;   // V scales per token
     static_assert(!PK || (G32 && !G16), "packing: group-32 scales, at most 4 heads");
+    static_assert(!(PK && CAUSAL), "chunk queries: unpacked columns");
     constexpr int NVS = PK ? NGRP / 2 : NGV;   // P'' operand sets (PK: group pairs)
 
     extern __shared__ uint8_t smem_raw[];
@@ -349,7 +353,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll 1
         for (int b = tid; b < prm.B; b += nthreads(PAGED)) {
             int L = prm.seq_lens[b];
-            if (L < 0 || L > lim) {
+            // (a chunk of queries needs its own tokens in the cache: L >= T)
+            if (L < 0 || L > lim || (CAUSAL && L > 0 && L < prm.qlen)) {
                 if (blockIdx.x == 0) raise_flag(prm.d_err, KVQ_DEVERR_LEN);
                 L = 0;
             }
@@ -421,7 +426,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     auto one_valid = [&](int L) {
         const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
         const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
-        if (L < 0 || L > lim) {
+        if (L < 0 || L > lim || (CAUSAL && L > 0 && L < p.qlen)) {
             if (one_j == 0 && one_hk == 0 && tid == 32 * nprod(PAGED)) raise_flag(p.d_err, KVQ_DEVERR_LEN);
             L = 0;
         }
@@ -746,6 +751,16 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         i = sg.next;
         const int b = sg.b, hk = sg.hk;
         const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
+        // chunk of queries: the last position column 8 nt + 2 t + c may see
+        int lim_col[NT][2];
+        if constexpr (CAUSAL) {
+            const int Lseq = one ? one_valid(one_raw()) : lens[b];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    lim_col[nt][c] = Lseq - p.qlen + (8 * nt + 2 * t + c) % p.qlen;
+        }
         if (!one && sg.ns == 0) {
             // empty (or rejected) sequence: zero rows
 #pragma unroll 1
@@ -904,6 +919,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                             z[u][nt][2] = okB[u] ? z[u][nt][2] * zs[nt][0] : -INFINITY;
                             z[u][nt][3] = okB[u] ? z[u][nt][3] * zs[nt][1] : -INFINITY;
                         }
+                        if constexpr (CAUSAL) {
+                            // positions past the column's query are masked
+                            const int ta = tt0 + rA[u], tb = tt0 + rB[u];
+                            if (ta > lim_col[nt][0]) z[u][nt][0] = -INFINITY;
+                            if (ta > lim_col[nt][1]) z[u][nt][1] = -INFINITY;
+                            if (tb > lim_col[nt][0]) z[u][nt][2] = -INFINITY;
+                            if (tb > lim_col[nt][1]) z[u][nt][3] = -INFINITY;
+                        }
                     }
                 // ---- online softmax per head: max over the slice's 32 tokens
                 float pr[2][NT][4];
@@ -920,10 +943,13 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         const float mn = fmaxf(m[nt][c], mx);
                         const float al = (mn == -INFINITY) ? 1.f : ptx::ex2(m[nt][c] - mn);
                         float add = 0.f;
+                        // (a chunk query can have seen no position yet: its
+                        // masked scores then give 2^-inf = 0, not NaN)
+                        const float mb = (CAUSAL && mn == -INFINITY) ? 0.f : mn;
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
-                            pr[u][nt][c] = okA[u] ? ptx::ex2(z[u][nt][c] - mn) : 0.f;
-                            pr[u][nt][2 + c] = okB[u] ? ptx::ex2(z[u][nt][2 + c] - mn) : 0.f;
+                            pr[u][nt][c] = okA[u] ? ptx::ex2(z[u][nt][c] - mb) : 0.f;
+                            pr[u][nt][2 + c] = okB[u] ? ptx::ex2(z[u][nt][2 + c] - mb) : 0.f;
                             add += pr[u][nt][c] + pr[u][nt][2 + c];
                         }
                         l[nt][c] = l[nt][c] * al + add;
@@ -1240,12 +1266,12 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
     return cudaSuccess;
 }
 
-template <int D, bool G32, bool PAGED, bool G16, bool PK>
+template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL>
 cudaError_t set_attrs() {
     using Lay = Layout<D, G32, G16>;
     static bool done = false;
     if (done) return cudaSuccess;
-    auto kern = decode_split_tc<D, G32, PAGED, G16, PK>;
+    auto kern = decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -1254,10 +1280,10 @@ cudaError_t set_attrs() {
     return e;
 }
 
-template <int D, bool G32, bool PAGED, bool G16, bool PK>
+template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL>
 cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     using Lay = Layout<D, G32, G16>;
-    cudaError_t e = set_attrs<D, G32, PAGED, G16, PK>();
+    cudaError_t e = set_attrs<D, G32, PAGED, G16, PK, CAUSAL>();
     if (e != cudaSuccess) return e;
     CUtensorMap mk, mv;
     const int64_t rows = PAGED ? static_cast<int64_t>(p.num_pages) * p.Hk * 16
@@ -1276,15 +1302,18 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16, PK>, mk, mv, p);
+    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL>, mk, mv, p);
 }
 
 template <int D, bool G32, bool PAGED>
 cudaError_t pick_g(const DecodeParams& p, cudaStream_t s) {
-    if (p.G > 8) return launch_tc<D, G32, PAGED, true, false>(p, s);
+    if (p.qlen > 1)                     // a chunk of queries: causal columns
+        return p.G > 8 ? launch_tc<D, G32, PAGED, true, false, true>(p, s)
+                       : launch_tc<D, G32, PAGED, false, false, true>(p, s);
+    if (p.G > 8) return launch_tc<D, G32, PAGED, true, false, false>(p, s);
     if constexpr (G32)
-        if (p.G <= 4) return launch_tc<D, G32, PAGED, false, true>(p, s);
-    return launch_tc<D, G32, PAGED, false, false>(p, s);
+        if (p.G <= 4) return launch_tc<D, G32, PAGED, false, true, false>(p, s);
+    return launch_tc<D, G32, PAGED, false, false, false>(p, s);
 }
 
 template <int D>

@@ -64,6 +64,8 @@ struct DecodeParams {
     int grid;                // persistent CTAs of the split kernel
     int seg_w;               // partition weight of a (sequence, kv head) start, in items
     int one_item;            // the plan's items fit the grid: CTA c takes item c
+    int qlen;                // queries per (sequence, q head): 1 for decode, T for a chunk
+                             // (Hq and G then count (head, query) rows, query fastest)
     float scale_log2;        // attn_scale * log2(e)
 };
 constexpr int kMaxBatch = 1024;                              // sequences per call

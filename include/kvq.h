@@ -173,6 +173,40 @@ size_t kvq_decode_workspace_bytes(int B, int Hq, int Hk, int D, int max_seq_len_
                                   int num_splits);
 
 /*
+ * kvq_chunk_attn -- a chunk of T new queries per (sequence, q head), causal
+ * from the chunk's end: the chunk's T tokens are the last T positions of the
+ * sequence (appended before the call), so query i sits at position
+ * L - T + i and attends to positions 0 .. L - T + i, with the same fused
+ * dequantisation as kvq_decode_attn.  T = 1 is kvq_decode_attn.
+ *   q           bf16 [B, Hq, T, D]
+ *   kv          cache view (see above)
+ *   d_seq_lens  int32 [B]   L, the cached length INCLUDING the chunk's T
+ *                           tokens; 0 gives zero output rows, and 0 < L < T
+ *                           is a length error (KVQ_DEVERR_LEN, zero rows)
+ *   out         fp32 [B, Hq, T, D]
+ *   workspace   at least kvq_chunk_workspace_bytes(...) bytes, as for
+ *               kvq_decode_attn
+ *   the other arguments as for kvq_decode_attn.
+ * Requirements: those of kvq_decode_attn with the GQA group counted in
+ * (head, query) rows: (Hq / Hk) * T <= 16 (otherwise KVQ_ERR_UNSUPPORTED).
+ * T < 1 is KVQ_ERR_INVALID_ARG.
+ * Source: abaddon 0.2.0-rc.1, kv_cache_quant_cuda.rs,
+ * CudaQuantizedKvCache::forward_attention (prefill with q_len > 1: the cache
+ * offset is seq_len - q_len and query q_pos sees the positions up to
+ * cache_offset + q_pos); combs-models 0.2.2, src/kv.rs, attend (a query at
+ * global position p attends the keys at positions <= p).
+ */
+kvq_status kvq_chunk_attn(const uint16_t *q, int B, int Hq, int Hk, int T, int D,
+                          kvq_scale_mode mode, const kvq_cache_view *kv,
+                          const int32_t *d_seq_lens, int max_seq_len_hint, float attn_scale,
+                          float *out, void *workspace, size_t workspace_bytes, int num_splits,
+                          int32_t *d_err, kvq_stream_t stream);
+
+/* Workspace bytes kvq_chunk_attn needs for these arguments (0 when no split is needed). */
+size_t kvq_chunk_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_seq_len_hint,
+                                 int num_splits);
+
+/*
  * Split plan kvq_decode_attn uses: KV tokens per split (*chunk) and the
  * largest number of splits of any sequence (*splits).  num_sms <= 0 means the
  * current device's SM count.  Returns KVQ_ERR_INVALID_ARG on bad sizes.

@@ -153,8 +153,10 @@ class DecodeInputs:
 
 def make_decode_inputs(wl: Workload, *, B: Optional[int] = None, len_lo: Optional[int] = None,
                        len_hi: Optional[int] = None, seed: Optional[int] = None,
-                       page_size: int = 16) -> DecodeInputs:
-    """Seeded decode-step inputs for a workload (optionally shrunk)."""
+                       page_size: int = 16, qlen: int = 1) -> DecodeInputs:
+    """Seeded decode-step inputs for a workload (optionally shrunk).  qlen > 1:
+    a chunk of qlen new tokens (k_new/v_new [B, Hk, qlen, D]) and qlen queries
+    per head (q [B, Hq, qlen, D]); qlen = 1 draws exactly the decode inputs."""
     B = wl.B if B is None else B
     lo = wl.len_lo if len_lo is None else len_lo
     hi = wl.len_hi if len_hi is None else len_hi
@@ -164,10 +166,10 @@ def make_decode_inputs(wl: Workload, *, B: Optional[int] = None, len_lo: Optiona
     chans = outlier_channels(wl.Hk, wl.D, wl.outlier_frac, g)
     k_hist = apply_outliers(bf16_normal((B, wl.Hk, Lmax, wl.D), wl.sigma, g), chans, wl.outlier_factor)
     v_hist = apply_outliers(bf16_normal((B, wl.Hk, Lmax, wl.D), wl.sigma, g), chans, wl.outlier_factor)
-    k_new = apply_outliers(bf16_normal((B, wl.Hk, 1, wl.D), wl.sigma, g), chans, wl.outlier_factor)
-    v_new = apply_outliers(bf16_normal((B, wl.Hk, 1, wl.D), wl.sigma, g), chans, wl.outlier_factor)
-    q = bf16_normal((B, wl.Hq, wl.D), 1.0, g)
-    seq_lens = (cached + 1).to(torch.int32)
+    k_new = apply_outliers(bf16_normal((B, wl.Hk, qlen, wl.D), wl.sigma, g), chans, wl.outlier_factor)
+    v_new = apply_outliers(bf16_normal((B, wl.Hk, qlen, wl.D), wl.sigma, g), chans, wl.outlier_factor)
+    q = bf16_normal((B, wl.Hq, wl.D) if qlen == 1 else (B, wl.Hq, qlen, wl.D), 1.0, g)
+    seq_lens = (cached + qlen).to(torch.int32)
     table, npages = (None, 0)
     if wl.layout == "paged":
         table, npages = page_table_for(seq_lens.tolist(), page_size, g)

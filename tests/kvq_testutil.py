@@ -79,6 +79,16 @@ class ContigCache:
         return oracle.decode_attn(q, self.ok, self.ov, self.oks, self.ovs, seq_lens,
                                   attn_scale, self.mode)
 
+    def chunk(self, q, seq_lens, hint, **kw):
+        m = kvq()
+        dev = self.k.device
+        return m.kvq_chunk_attn(q.to(dev), self.k, self.v, self.ks, self.vs, seq_lens.to(dev),
+                                hint, mode=self.mode, err=self.err, **kw)
+
+    def oracle_chunk(self, q, seq_lens, attn_scale):
+        return oracle.chunk_attn(q, self.ok, self.ov, self.oks, self.ovs, seq_lens, attn_scale,
+                                 self.mode)
+
 
 class PagedCache:
     """Paged INT8 arena on the GPU plus its oracle twin."""
@@ -127,6 +137,17 @@ class PagedCache:
     def oracle_decode(self, q, seq_lens, attn_scale):
         return oracle.decode_attn(q, self.ok, self.ov, self.oks, self.ovs, seq_lens, attn_scale,
                                   self.mode, page_size=self.ps, table=self.table_cpu)
+
+    def chunk(self, q, seq_lens, hint, **kw):
+        m = kvq()
+        dev = self.k.device
+        return m.kvq_chunk_attn(q.to(dev), self.k, self.v, self.ks, self.vs, seq_lens.to(dev),
+                                hint, page_table=self.table, page_size=self.ps, mode=self.mode,
+                                err=self.err, **kw)
+
+    def oracle_chunk(self, q, seq_lens, attn_scale):
+        return oracle.chunk_attn(q, self.ok, self.ov, self.oks, self.ovs, seq_lens, attn_scale,
+                                 self.mode, page_size=self.ps, table=self.table_cpu)
 
 
 def f32_scale(D):

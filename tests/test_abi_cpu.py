@@ -164,6 +164,32 @@ def test_decode_rejects_bad_arguments(kvq):
 
 
 @needs_no_gpu
+def test_chunk_rejects_bad_arguments(kvq):
+    lib = kvq.lib
+    cv = kvq.CacheView(FAKE, FAKE, FAKE, FAKE, 0, 4096, 0, 0, 0)
+    ok = dict(q=FAKE, B=1, Hq=32, Hk=8, T=4, D=128, mode=0, kv=ctypes.byref(cv), sl=FAKE,
+              hint=4096, scale=0.088, out=FAKE, ws=FAKE, wsb=1 << 30, ns=0, err=None, s=None)
+
+    def call(**over):
+        a = dict(ok)
+        a.update(over)
+        return lib.kvq_chunk_attn(*a.values())
+    assert call(T=0) == 1
+    assert call(q=None) == 1
+    assert call(T=5) == 2                   # (Hq / Hk) * T = 20 rows per kv head
+    assert call(Hq=64, T=3) == 2            # 24 rows
+    assert call(out=FAKE + 4) == 1
+
+
+def test_chunk_workspace_is_the_decode_workspace_of_the_rows(kvq):
+    for B, Hq, Hk, T, D, hint, ns in [(1, 32, 8, 4, 128, 4097, 0), (3, 8, 2, 2, 64, 999, 5),
+                                      (16, 32, 8, 1, 128, 8193, 0)]:
+        assert kvq.kvq_chunk_workspace_bytes(B, Hq, Hk, T, D, hint, ns) == \
+            kvq.kvq_decode_workspace_bytes(B, Hq * T, Hk, D, hint, ns)
+    assert kvq.kvq_chunk_workspace_bytes(1, 32, 8, 0, 128, 4097, 0) == 0
+
+
+@needs_no_gpu
 def test_dequant_rejects_bad_arguments(kvq):
     lib = kvq.lib
     assert lib.kvq_dequant(FAKE, FAKE, 10, 24, 0, FAKE, None) == 1
