@@ -1,4 +1,5 @@
-"""CPU oracle for INT8 KV-cache append, dequantization and decode attention.
+"""CPU oracle for INT8 KV-cache append, dequantization, decode attention and
+chunk attention.
 
 TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and
 the benchmark's CPU-baseline / reference leg may import this package.  It is

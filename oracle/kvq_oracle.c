@@ -27,6 +27,11 @@
  *    head h reads kv head h / (Hq/Hk) (heads repeated consecutively); a
  *    single decode query attends to every cached position (no mask).
  *    Computed here in fp64 over the dequantized fp32 cache.
+ *  - Chunk attention (T new queries): abaddon 0.2.0-rc.1,
+ *    src/kv_cache_quant_cuda.rs, forward_attention (prefill with q_len > 1:
+ *    the cache offset is seq_len - q_len and query q_pos sees the positions
+ *    up to offset + q_pos) and combs-models 0.2.2, src/kv.rs, attend (a
+ *    query at global position p attends the keys at positions <= p).
  *  - Paged layout: combs-models 0.2.2, src/kv.rs, PagedKVCache (arena
  *    [num_pages, n_kv, page_size, head_dim]; logical token g lives in
  *    physical page table[g / page_size], slot g % page_size).
