@@ -100,3 +100,21 @@ def test_reference_arm_prints_one_line_from_rank_zero():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_runs_chunk_steps():
+    """--qlen T: the CPU oracle leg times chunk steps (T new tokens, T queries
+    per head) and the line records the chunk length."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                        "--qlen", "3", "--steps", "1", "--warmup", "0"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    d = json.loads(lines[-1])
+    assert d["impl"] == "reference" and d["value"] > 0
+    assert d["config"]["q_len"] == 3 and d["config"]["seq_len"] == 256 + 3
+    bad = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                          "--qlen", "0"], cwd=ROOT, env=env, capture_output=True, text=True,
+                         timeout=120)
+    assert bad.returncode != 0
