@@ -265,8 +265,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t bar_full = sbase + Lay::MISC_OFF;
     const uint32_t bar_empty = bar_full + NST * 8;
-    // per-warp head maxima and sums of a segment (read only between the two
-    // merge barriers, so the next segment's writes cannot overtake a reader)
+    // per-warp head maxima and sums of a segment (read after the merge
+    // barrier; the next segment's writers first wait on bar_mfree, which
+    // completes once every consumer warp has read them and the slots)
     float* mrg_m = reinterpret_cast<float*>(smem + Lay::MISC_OFF + 2 * NST * 8);  // [16][NW]
     float* mrg_l = mrg_m + 16 * NW;                                               // [16][NW]
     // completes when all consumer warps have read a segment's maxima and slots
