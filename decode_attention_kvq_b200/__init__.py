@@ -8,6 +8,17 @@ Importing this package fails loudly if libkvq.so has not been built
 
 Functions take torch CUDA tensors (PyTorch supplies device memory and
 streams) and enqueue on the current CUDA stream unless ``stream`` is given.
+
+A decode step on a contiguous cache (B sequences, Hk kv heads, head_dim D):
+
+    k = torch.zeros(B, Hk, S, D, dtype=torch.uint8, device="cuda"); v = torch.zeros_like(k)
+    ks = torch.zeros(B, Hk, S, 1, device="cuda"); vs = torch.zeros_like(ks)   # D // 32 for group32
+    kvq_append(k_new, v_new, pos, k, v, ks, vs)        # bf16 [B, Hk, T, D] at pos[b]
+    out = kvq_decode_attn(q, k, v, ks, vs, seq_lens, max_len)   # q bf16 [B, Hq, D]
+    out = kvq_chunk_attn(qc, k, v, ks, vs, seq_lens, max_len)   # qc bf16 [B, Hq, T, D]
+
+``seq_lens`` (int32 [B], on the device) counts the cached tokens including
+the ones just appended; ``max_len`` is a host upper bound of it.
 """
 from __future__ import annotations
 
