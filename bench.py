@@ -18,6 +18,13 @@ Multi-GPU: launched by torch.distributed.run, one rank per GPU; every rank
 runs its own replica of the workload (weak scaling, no data-path collective);
 the job time is the max over ranks.
 
+The line's headline fields time exactly K steps of the chosen workload.
+Its "per_config" object then times every workload on its own (median over
+at least 10 repeats, enough of them to span a quarter of a second), each
+with its roofline, append rate, end-to-end rate and clock record.  The CPU
+baseline is the oracle on this host: all cores (OpenMP over independent
+(sequence, kv head) units) and one core.
+
 Prints ONE JSON line on rank 0.
 """
 from __future__ import annotations
@@ -81,13 +88,15 @@ class ClockSampler:
     SW_THERMAL = 0x20
     SW_POWER = 0x4
 
-    def __init__(self, device_index: int, period_s: float = 0.002):
+    def __init__(self, device_index: int, period_s: float = 0.002, enabled: bool = True):
         self.samples = []
         self.max_mhz = None
         self.period = period_s
         self._stop = threading.Event()
         self._thread = None
         self.ok = False
+        if not enabled:
+            return
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -282,10 +291,24 @@ def build_layers(kvq, wl, n_layers, dev, keep_host=False):
 
 
 # -------------------------------------------------------------- cpu oracle
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 class OracleLayer:
-    """One layer of the workload held by the CPU oracle (single thread): the
-    history is quantised once at set-up; a step quantises the decode token
-    into the cache and runs fp64 decode attention."""
+    """One layer of the workload held by the CPU oracle: the history is
+    quantised once at set-up; a step quantises the decode token into the
+    cache and runs fp64 decode attention, either single-threaded (the pinned
+    oracle as it stands) or as one pinned-oracle call per (sequence, kv head)
+    on `threads` host threads (the oracle's all-core baseline build)."""
 
     def __init__(self, wl, seed):
         import oracle  # test infrastructure: used only by the CPU baseline legs
@@ -310,6 +333,7 @@ class OracleLayer:
                                     tb, 16, wl.mode)
                 oracle.append_paged(inp.v_hist[b:b + 1, :, :L].contiguous(), z1, self.v, self.vs,
                                     tb, 16, wl.mode)
+            self.utables = oracle.unit_tables(inp.page_table, Hk, inp.num_pages)
         else:
             S = int(inp.seq_lens.max())
             self.k = torch.zeros(B, Hk, S, D, dtype=torch.uint8)
@@ -320,28 +344,35 @@ class OracleLayer:
             zb = torch.zeros(B, dtype=torch.int32)
             oracle.append_contig(inp.k_hist[:, :, :Lm].contiguous(), zb, self.k, self.ks, wl.mode)
             oracle.append_contig(inp.v_hist[:, :, :Lm].contiguous(), zb, self.v, self.vs, wl.mode)
+            self.utables = None
         self.scale = float(torch.tensor(1.0 / math.sqrt(D), dtype=torch.float32))
         self.nbytes = decode_bytes(wl, [int(x) for x in inp.seq_lens], 16 if self.paged else 0)
         self.inp.k_hist = self.inp.v_hist = None
 
-    def step(self) -> float:
+    def step(self, threads: int = 1) -> float:
         o, wl, inp = self.oracle, self.wl, self.inp
         t0 = time.perf_counter()
         if self.paged:
             o.append_paged(inp.k_new, inp.cached, self.k, self.ks, inp.page_table, 16, wl.mode)
             o.append_paged(inp.v_new, inp.cached, self.v, self.vs, inp.page_table, 16, wl.mode)
-            attn = o.decode_attn if QLEN == 1 else o.chunk_attn
-            attn(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale, wl.mode,
-                 page_size=16, table=inp.page_table)
         else:
             o.append_contig(inp.k_new, inp.cached, self.k, self.ks, wl.mode)
             o.append_contig(inp.v_new, inp.cached, self.v, self.vs, wl.mode)
+        if threads <= 1:
             attn = o.decode_attn if QLEN == 1 else o.chunk_attn
-            attn(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale, wl.mode)
+            if self.paged:
+                attn(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale, wl.mode,
+                     page_size=16, table=inp.page_table)
+            else:
+                attn(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale, wl.mode)
+        else:
+            o.attn_units(inp.q, self.k, self.v, self.ks, self.vs, inp.seq_lens, self.scale,
+                         wl.mode, page_size=16 if self.paged else 0, utables=self.utables,
+                         num_pages=inp.num_pages, threads=threads)
         return time.perf_counter() - t0
 
 
-def oracle_sample(wl, n_steps_max, budget_s, n_distinct=4):
+def oracle_sample(wl, n_steps_max, budget_s, threads=1, n_distinct=4):
     """Time the oracle on a bounded sample of the workload: layer steps cycled
     over a few distinct layers until the time budget or the step cap is hit.
     Returns (GB/s, sample description)."""
@@ -349,12 +380,26 @@ def oracle_sample(wl, n_steps_max, budget_s, n_distinct=4):
     done, elapsed, nbytes = 0, 0.0, 0
     while done < n_steps_max and (elapsed < budget_s or done == 0):
         ly = layers[done % n_distinct]
-        elapsed += ly.step()
+        elapsed += ly.step(threads)
         nbytes += ly.nbytes
         done += 1
-    desc = (f"{done} layer steps of {wl.name} (append 1 token + fp64 decode attention) "
-            f"over {n_distinct} distinct layers, single-threaded C oracle, {elapsed:.2f} s timed")
+    how = ("single-threaded C oracle" if threads <= 1 else
+           f"C oracle, one call per (sequence, kv head) unit on {threads} OpenMP threads")
+    desc = (f"{done} layer steps of {wl.name} (append {QLEN} token(s) + fp64 attention) "
+            f"over {n_distinct} distinct layers, {how}, {elapsed:.2f} s timed")
     return nbytes / elapsed / 1e9, desc
+
+
+def cpu_baseline(wl, args):
+    """The oracle timed on this host: all cores (OpenMP over independent
+    (sequence, kv head) units, the headline value) and one core."""
+    threads = os.cpu_count() or 1
+    gbs_all, desc_all = oracle_sample(wl, args.cpu_layers, args.cpu_budget_s, threads=threads)
+    gbs_one, desc_one = oracle_sample(wl, args.cpu_layers, args.cpu_budget_s, threads=1)
+    return {"value": round(gbs_all, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": desc_all, "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+            "single_thread": {"value": round(gbs_one, 4), "unit": "GB/s", "cores": 1,
+                              "sample": desc_one}}
 
 
 # ------------------------------------------------------------------- arms
@@ -364,15 +409,16 @@ def run_reference(args, wl):
     if rank != 0:
         return 0
     # each step is a bounded sample of the workload: one layer step of the
-    # oracle on a layer prepared once
+    # oracle, on all host cores, on a layer prepared once
+    threads = os.cpu_count() or 1
     ly = OracleLayer(wl, wl.seed)
     per_step = []
     for i in range(args.warmup + args.steps):
-        el = ly.step()
+        el = ly.step(threads)
         if i >= args.warmup:
             per_step.append((ly.nbytes / el / 1e9, el))
-    desc = (f"1 layer step of {wl.name} per step (append 1 token + fp64 decode attention), "
-            "single-threaded C oracle")
+    desc = (f"1 layer step of {wl.name} per step (append {QLEN} token(s) + fp64 attention), "
+            f"C oracle, one call per (sequence, kv head) unit on {threads} OpenMP threads")
     value = statistics.median(g for g, _ in per_step)
     ms = 1000.0 * statistics.median(e for _, e in per_step)
     line = {
@@ -383,13 +429,152 @@ def run_reference(args, wl):
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hk": wl.Hk, "D": wl.D,
                    "seq_len": wl.len_hi + QLEN, "scale_mode": wl.mode, "layout": wl.layout,
                    "q_len": QLEN, "sample": "1 layer step per step"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
-                         "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": desc, "cpu_model": cpu_model(),
+                         "host_cpus": os.cpu_count()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+NOMINAL_HBM_GBS = 8000.0                  # B200 HBM3e, nominal
+
+
+class GpuWorkload:
+    """One workload resident on the GPU: its layer caches, the decode
+    workspace and the step's two phases captured as CUDA graphs (every
+    layer's append, then every layer's decode attention)."""
+
+    def __init__(self, kvq, wl, dev, n_layers):
+        self.kvq, self.wl, self.dev = kvq, wl, dev
+        self.layers = build_layers(kvq, wl, n_layers, dev)
+        self.n_layers = n_layers
+        L0 = self.layers[0]
+        self.hint = L0.hint
+        ws_bytes = (kvq.kvq_decode_workspace_bytes(wl.B, wl.Hq, wl.Hk, wl.D, L0.hint)
+                    if QLEN == 1 else
+                    kvq.kvq_chunk_workspace_bytes(wl.B, wl.Hq, wl.Hk, QLEN, wl.D, L0.hint))
+        self.workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.chunk, self.splits = kvq.kvq_decode_plan(wl.B, wl.Hk, L0.hint)
+        # append (+ prefill-chunk append) + split kernel (+ combine kernel when a
+        # sequence spans several chunks: then the call has a workspace)
+        self.launches_per_layer = ((1 + (1 if wl.prefill_chunk else 0)) + 1 +
+                                   (1 if ws_bytes > 0 else 0))
+        self.stream = torch.cuda.Stream(dev)
+        with torch.cuda.stream(self.stream):       # warm the library once eagerly
+            for ly in self.layers:
+                ly.append(kvq)
+                ly.decode(kvq, self.workspace)
+        torch.cuda.synchronize(dev)
+        self.g_append, self.g_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_append, stream=self.stream):
+            for ly in self.layers:
+                ly.append(kvq)
+        with torch.cuda.graph(self.g_decode, stream=self.stream):
+            for ly in self.layers:
+                ly.decode(kvq, self.workspace)
+        torch.cuda.synchronize(dev)
+        self.dec_b = sum(decode_bytes(wl, ly.seq_lens_list, 16 if ly.paged else 0)
+                         for ly in self.layers)
+        self.app_b = n_layers * (append_bytes(wl, QLEN) +
+                                 (append_bytes(wl, wl.prefill_chunk) if wl.prefill_chunk else 0))
+
+    def warm(self, W):
+        with torch.cuda.stream(self.stream):
+            for _ in range(W):
+                self.g_append.replay()
+                self.g_decode.replay()
+        torch.cuda.synchronize(self.dev)
+
+    def timed(self, reps, sampler):
+        """reps steps, each bracketed by CUDA events on the launching stream:
+        returns per-step (append s, decode s) and the whole region's seconds."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+        with sampler:
+            with torch.cuda.stream(self.stream):
+                for i in range(reps):
+                    ev[i][0].record(self.stream)
+                    self.g_append.replay()
+                    ev[i][1].record(self.stream)
+                    self.g_decode.replay()
+                    ev[i][2].record(self.stream)
+            torch.cuda.synchronize(self.dev)
+        per = [(e[0].elapsed_time(e[1]) / 1e3, e[1].elapsed_time(e[2]) / 1e3) for e in ev]
+        return per, ev[0][0].elapsed_time(ev[-1][2]) / 1e3
+
+    def close(self):
+        del self.g_append, self.g_decode
+        self.layers = None
+        self.workspace = None
+        torch.cuda.synchronize(self.dev)
+        torch.cuda.empty_cache()
+
+
+def roofline(wl, achieved):
+    peak, peak_kind = measured_peaks()
+    traffic = decode_traffic_record()
+    tv = None
+    if traffic:
+        tv = (traffic.get("workloads", {}).get(wl.name, {}) or {}).get("traffic_bytes_per_launch")
+    return {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": tv,
+            "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+            "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+            "nominal_peak": NOMINAL_HBM_GBS}
+
+
+def per_config_entry(kvq, wl, dev, K, W, world, gw=None):
+    """One workload measured on its own: median over repeats (at least 10,
+    and enough to cover a quarter of a second so the clock sampler sees the
+    region), each repeat one step of every layer."""
+    n_layers = LAYERS.get(wl.name, 1)
+    own = gw is None
+    if own:
+        gw = GpuWorkload(kvq, wl, dev, n_layers)
+    gw.warm(W)
+    probe, t_probe = gw.timed(3, ClockSampler(-1, enabled=False))
+    reps = max(10, K, min(2000, int(math.ceil(0.25 / max(t_probe / 3, 1e-6)))))
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(physical_gpu_index(dev.index))
+    per, _ = gw.timed(reps, sampler)
+    barrier(dev)
+    t_app = statistics.median(a for a, _ in per)
+    t_dec = statistics.median(d for _, d in per)
+    t_app = reduce_max(t_app, dev)
+    t_dec = reduce_max(t_dec, dev)
+    dec_mean = sum(d for _, d in per) / reps
+    pl_dec = t_dec / gw.n_layers
+    pl_app = t_app / gw.n_layers
+    achieved = gw.dec_b / gw.n_layers / pl_dec / 1e9
+    e2e = run_e2e(kvq, wl, gw.layers, gw.workspace, dev, min(K, 20), W, world)
+    entry = {
+        "config": {"B": wl.B, "Hq": wl.Hq, "Hk": wl.Hk, "D": wl.D, "seq_len": gw.hint,
+                   "scale_mode": wl.mode, "layout": wl.layout, "layers_per_step": gw.n_layers,
+                   "split_chunk": gw.chunk, "splits": gw.splits,
+                   "prefill_chunk": wl.prefill_chunk,
+                   "l2": ("inputs larger than L2 (%.0f MB per step)" % ((gw.dec_b + gw.app_b) / 1e6)
+                          if gw.dec_b + gw.app_b > 126e6 else
+                          "inputs L2-resident (%.2f MB per step): a latency figure"
+                          % ((gw.dec_b + gw.app_b) / 1e6))},
+        "repeats": reps, "statistic": "median over repeats",
+        "decode_us_per_layer": round(pl_dec * 1e6, 3),
+        "decode_us_per_layer_mean": round(dec_mean / gw.n_layers * 1e6, 3),
+        "decode_us_per_layer_min": round(min(d for _, d in per) / gw.n_layers * 1e6, 3),
+        "append_us_per_layer": round(pl_app * 1e6, 3),
+        "decode_gbs": round(world * achieved, 2),
+        "roofline": roofline(wl, achieved),
+        "append_gbs": round(world * gw.app_b / t_app / 1e9, 2),
+        "tokens_per_s_per_layer": round(wl.B * QLEN / (pl_app + pl_dec), 1),
+        "algorithmic_bytes_per_decode_call": int(gw.dec_b / gw.n_layers),
+        "e2e": e2e,
+        "clocks": sampler.summary(),
+    }
+    if own:
+        gw.close()
+    return entry
 
 
 def run_kvq(args, wl):
@@ -410,113 +595,71 @@ def run_kvq(args, wl):
     import decode_attention_kvq_b200 as kvq  # fails loudly if libkvq.so is missing
 
     n_layers = args.layers or LAYERS.get(wl.name, 1)
-    layers = build_layers(kvq, wl, n_layers, dev)
-    L0 = layers[0]
-    ws_bytes = (kvq.kvq_decode_workspace_bytes(wl.B, wl.Hq, wl.Hk, wl.D, L0.hint) if QLEN == 1
-                else kvq.kvq_chunk_workspace_bytes(wl.B, wl.Hq, wl.Hk, QLEN, wl.D, L0.hint))
-    workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    chunk, splits = kvq.kvq_decode_plan(wl.B, wl.Hk, L0.hint)
-    # append (+ prefill-chunk append) + split kernel (+ combine kernel when a
-    # sequence spans several chunks: then the call has a workspace)
-    launches_per_layer = (1 + (1 if wl.prefill_chunk else 0)) + 1 + (1 if ws_bytes > 0 else 0)
+    gw = GpuWorkload(kvq, wl, dev, n_layers)
 
-    stream = torch.cuda.Stream(dev)
-    # warm the library once eagerly, then capture the two phases as graphs
-    with torch.cuda.stream(stream):
-        for ly in layers:
-            ly.append(kvq)
-            ly.decode(kvq, workspace)
-    torch.cuda.synchronize(dev)
-    g_append, g_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_append, stream=stream):
-        for ly in layers:
-            ly.append(kvq)
-    with torch.cuda.graph(g_decode, stream=stream):
-        for ly in layers:
-            ly.decode(kvq, workspace)
-    torch.cuda.synchronize(dev)
-
+    # ---- the headline: exactly K steps after W warm-up steps
     K, W = args.steps, args.warmup
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    with torch.cuda.stream(stream):
-        for _ in range(W):
-            g_append.replay()
-            g_decode.replay()
-    torch.cuda.synchronize(dev)
+    gw.warm(W)
     barrier(dev)
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(physical_gpu_index(local))
-    with sampler:
-        with torch.cuda.stream(stream):
-            for i in range(K):
-                ev[i][0].record(stream)
-                g_append.replay()
-                ev[i][1].record(stream)
-                g_decode.replay()
-                ev[i][2].record(stream)
-        torch.cuda.synchronize(dev)
+    per, t_total = gw.timed(K, sampler)
     barrier(dev)
-    t_append = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3          # s over K steps
-    t_decode = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    t_total = ev[0][0].elapsed_time(ev[-1][2]) / 1e3
+    t_append = sum(a for a, _ in per)
+    t_decode = sum(d for _, d in per)
     t_total_max = reduce_max(t_total, dev)
     t_decode_max = reduce_max(t_decode, dev)
     t_append_max = reduce_max(t_append, dev)
 
-    dec_b = sum(decode_bytes(wl, ly.seq_lens_list, 16 if ly.paged else 0) for ly in layers)
-    app_b = sum(append_bytes(wl, QLEN) + (append_bytes(wl, wl.prefill_chunk) if wl.prefill_chunk
-                                       else 0) for _ in layers)
-    value = world * dec_b * K / t_decode_max / 1e9
+    value = world * gw.dec_b * K / t_decode_max / 1e9
     per_layer_decode = t_decode_max / (K * n_layers)
     per_layer_append = t_append_max / (K * n_layers)
     tokens_per_s_per_layer = wl.B * QLEN / (per_layer_append + per_layer_decode)
-    append_gbs = app_b * K / t_append_max / 1e9
-
-    peak, peak_kind = measured_peaks()
-    decode_call_bytes = dec_b / n_layers
+    append_gbs = gw.app_b * K / t_append_max / 1e9
+    decode_call_bytes = gw.dec_b / n_layers
     achieved = decode_call_bytes / per_layer_decode / 1e9
-    traffic = decode_traffic_record()
-    traffic_val = None
-    if traffic and traffic.get("workload") == wl.name:
-        traffic_val = traffic.get("traffic_bytes_per_launch")
+    rl = roofline(wl, achieved)
+    rl["kernel"] = "kvq_decode_attn call (split + combine kernels, per layer)"
+    rl["algorithmic_bytes_per_launch"] = int(decode_call_bytes)
 
     # ---- end to end through the public API from pinned host buffers
-    e2e = run_e2e(kvq, wl, layers, workspace, dev, K, W, world)
+    e2e = run_e2e(kvq, wl, gw.layers, gw.workspace, dev, K, W, world)
 
-    clocks = sampler.summary()
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(1e3 * t_total_max / K, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
         "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hk": wl.Hk, "D": wl.D,
-                   "seq_len": L0.hint, "q_len": QLEN, "scale_mode": wl.mode,
+                   "seq_len": gw.hint, "q_len": QLEN, "scale_mode": wl.mode,
                    "layout": wl.layout,
                    "layers_per_step": n_layers, "parallelism": f"replicas x{world}",
                    "l2": ("inputs larger than L2 (%.0f MB per step)"
-                          % ((dec_b + app_b) / 1e6)),
-                   "split_chunk": chunk, "splits": splits},
+                          % ((gw.dec_b + gw.app_b) / 1e6)),
+                   "split_chunk": gw.chunk, "splits": gw.splits},
         "tokens_per_s_per_layer": round(tokens_per_s_per_layer, 1),
         "append_gbs": round(append_gbs, 2),
         "decode_us_per_layer": round(per_layer_decode * 1e6, 3),
         "append_us_per_layer": round(per_layer_append * 1e6, 3),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic_val,
-                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                     "kernel": "kvq_decode_attn call (split + combine kernels, per layer)",
-                     "algorithmic_bytes_per_launch": int(decode_call_bytes)},
-        "gpu_launches": launches_per_layer * n_layers * K,
-        "clocks": clocks,
+        "roofline": rl,
+        "gpu_launches": gw.launches_per_layer * n_layers * K,
+        "clocks": sampler.summary(),
         "e2e": e2e,
     }
+    # ---- every workload on its own (medians over repeats); the headline's
+    # caches and graphs are reused for its own entry
+    if QLEN == 1 and not args.no_per_config and args.layers == 0:
+        pc = {}
+        for name, w in synth.WORKLOADS.items():
+            pc[name] = per_config_entry(kvq, w, dev, K, W, world,
+                                        gw=gw if name == wl.name else None)
+        line["per_config"] = pc
+    gw.close()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, desc = oracle_sample(wl, args.cpu_layers, args.cpu_budget_s)
-        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1,
-                                "kind": "oracle", "sample": desc}
+        line["cpu_baseline"] = cpu_baseline(wl, args)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
-        del g_append, g_decode
         dist.destroy_process_group()
     return 0
 
@@ -581,7 +724,10 @@ def main(argv=None):
     ap.add_argument("--workload", choices=list(synth.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--layers", type=int, default=0, help="layer caches per step (0: default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the headline workload")
+    ap.add_argument("--cpu-budget-s", type=float, default=10.0,
+                    help="seconds of oracle work per CPU-baseline leg")
     ap.add_argument("--cpu-layers", type=int, default=400)
     ap.add_argument("--qlen", type=int, default=1,
                     help="queries per head per step: > 1 runs chunk attention steps")

@@ -191,3 +191,62 @@ def cache_bytes(layers, Hk, seq, D, group, scale_bytes=4) -> int:
 
 def fp32_cache_bytes(layers, Hk, seq, D) -> int:
     return int(_load().oracle_fp32_cache_bytes(layers, Hk, seq, D))
+
+
+# ------------------------------------------------- all-core baseline build
+_omp_lib = None
+
+
+def _load_omp():
+    global _omp_lib
+    if _omp_lib is None:
+        lib = ctypes.CDLL(_build.build_omp())
+        P, I = ctypes.c_void_p, ctypes.c_int
+        lib.oracle_attn_units.argtypes = [P, I, I, I, I, I, I, P, P, P, P, I, I, P, I, I, P,
+                                          ctypes.c_double, P, I]
+        lib.oracle_attn_units.restype = I
+        _omp_lib = lib
+    return _omp_lib
+
+
+def unit_tables(table: torch.Tensor, Hk: int, num_pages: int) -> torch.Tensor:
+    """Per-(sequence, kv head) page ids of a paged arena seen as one-head
+    pages: page p of head hk becomes p * Hk + hk (entries outside the arena
+    stay -1).  int32 [B * Hk, max_pages]."""
+    t = _cpu(table, torch.int32).to(torch.int64)
+    ok = (t >= 0) & (t < num_pages)
+    hk = torch.arange(Hk, dtype=torch.int64).view(1, Hk, 1)
+    u = torch.where(ok.unsqueeze(1), t.unsqueeze(1) * Hk + hk, torch.full_like(hk, -1))
+    return u.reshape(-1, t.shape[1]).to(torch.int32).contiguous()
+
+
+def attn_units(q, k, v, k_scale, v_scale, seq_lens, attn_scale, mode="per_token",
+               page_size=0, utables=None, num_pages=0, threads=1):
+    """The oracle's decode (q [B,Hq,D]) or chunk (q [B,Hq,T,D]) attention run
+    as one pinned-oracle call per (sequence, kv head) unit on `threads` host
+    threads (baseline timing only; results equal decode_attn / chunk_attn).
+    Paged caches take utables from unit_tables()."""
+    if q.dim() == 3:
+        B, Hq, D = q.shape
+        T = 1
+    else:
+        B, Hq, T, D = q.shape
+    grp = group_of(mode, D)
+    Hk = k.shape[1]
+    qb = _bits16(q)
+    kc, vc = _cpu(k, torch.uint8), _cpu(v, torch.uint8)
+    ks, vs = _cpu(k_scale, torch.float32), _cpu(v_scale, torch.float32)
+    sl = _cpu(seq_lens, torch.int32)
+    out = torch.empty(*q.shape, dtype=torch.float64)
+    if page_size > 0:
+        tb = _cpu(utables, torch.int32)
+        err = _load_omp().oracle_attn_units(
+            qb.data_ptr(), B, Hq, Hk, T, D, grp, kc.data_ptr(), vc.data_ptr(), ks.data_ptr(),
+            vs.data_ptr(), 0, page_size, tb.data_ptr(), tb.shape[1], num_pages, sl.data_ptr(),
+            float(attn_scale), out.data_ptr(), int(threads))
+    else:
+        err = _load_omp().oracle_attn_units(
+            qb.data_ptr(), B, Hq, Hk, T, D, grp, kc.data_ptr(), vc.data_ptr(), ks.data_ptr(),
+            vs.data_ptr(), kc.shape[2], 0, None, 0, 0, sl.data_ptr(), float(attn_scale),
+            out.data_ptr(), int(threads))
+    return out, err
