@@ -64,9 +64,11 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <atomic>
 #include <type_traits>
 #include <unordered_map>
 
+#include "kvq_devonce.h"
 #include "kvq_internal.cuh"
 #include "kvq_ptx.cuh"
 
@@ -1208,16 +1210,21 @@ using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, voi
                               const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                               CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+EncodeFn query_encode_fn() {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<EncodeFn>(ptr);
+    return nullptr;
+}
+
+// The driver's tensor-map encoder, looked up once per process (a
+// function-local static is initialised exactly once even when several host
+// threads get here together; the entry point is the same for every device).
 EncodeFn encode_fn() {
-    static EncodeFn fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeFn>(ptr);
-    }
+    static const EncodeFn fn = query_encode_fn();
     return fn;
 }
 
@@ -1267,18 +1274,24 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
     return cudaSuccess;
 }
 
+// Function attributes belong to the current device's context, so they are
+// set once per device ordinal.
 template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL>
 cudaError_t set_attrs() {
     using Lay = Layout<D, G32, G16>;
-    static bool done = false;
-    if (done) return cudaSuccess;
-    auto kern = decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-    if (e == cudaSuccess) done = true;
-    return e;
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    return once_per_device(done, dev, cudaSuccess, [] {
+        auto kern = decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL>;
+        cudaError_t r =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
+        if (r == cudaSuccess)
+            r = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared);
+        return r;
+    });
 }
 
 template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL>
