@@ -10,7 +10,9 @@ import ctypes
 import pytest
 import torch
 
-from kvq_testutil import ATOL, RTOL_L2, assert_attn_close, bf16_randn, kvq
+import synth
+from kvq_testutil import (ContigCache, PagedCache, assert_attn_close, bf16_randn, f32_scale,
+                          kvq)
 
 pytestmark = pytest.mark.gpu
 
@@ -64,3 +66,62 @@ def test_noalloc_rejects_problems_larger_than_the_scratch():
     assert st == 5 and m.lib.kvq_status_string(st).decode() == "KVQ_ERR_SCRATCH_TOO_SMALL"
     torch.cuda.synchronize()
     assert torch.all(out == 0)                               # nothing was enqueued
+
+
+def _noalloc(m, q, cache, seq, hint, mode, paged):
+    """One kvq_decode_attn_noalloc call through the C ABI."""
+    B, Hq, D = q.shape
+    Hk = cache.k.shape[1]
+    out = torch.full((B, Hq, D), float("nan"), device="cuda")
+    cv = (m.cache_view(cache.k, cache.v, cache.ks, cache.vs, cache.table, 16) if paged else
+          m.cache_view(cache.k, cache.v, cache.ks, cache.vs))
+    st = m.lib.kvq_decode_attn_noalloc(
+        q.data_ptr(), B, Hq, Hk, D, 0 if mode == "per_token" else 1, ctypes.byref(cv),
+        seq.data_ptr(), hint, f32_scale(D), out.data_ptr(), 0, None,
+        torch.cuda.current_stream().cuda_stream)
+    assert st == 0, m.lib.kvq_status_string(st)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("mode", ["per_token", "group32"])
+def test_noalloc_matches_oracle_contiguous(mode):
+    """The scratch-array path against the fp64 oracle and against the
+    workspace entry point, two calls in a row, per-token and group-32."""
+    m = kvq()
+    B, Hq, Hk, D = 3, 32, 8, 128
+    lens = [2900, 1500, 777]
+    S = max(lens)
+    c = ContigCache(B, Hk, S, D, mode)
+    g = torch.Generator().manual_seed(71)
+    kh = (torch.randn(B, Hk, S, D, generator=g)).to(torch.bfloat16)
+    vh = (torch.randn(B, Hk, S, D, generator=g)).to(torch.bfloat16)
+    assert c.append(kh, vh, torch.zeros(B, dtype=torch.int32)) == 0
+    seq = torch.tensor(lens, dtype=torch.int32)
+    assert m.kvq_decode_workspace_bytes(B, Hq, Hk, D, S) > 0
+    for call in range(2):
+        q = bf16_randn((B, Hq, D), seed=80 + call)
+        out = _noalloc(m, q.cuda(), c, seq.cuda(), S, mode, paged=False)
+        ref = c.oracle_decode(q, seq, f32_scale(D))
+        assert_attn_close(out, ref, f"{mode} call {call} vs oracle")
+        ws = c.decode(q, seq, S, attn_scale=f32_scale(D))
+        assert_attn_close(out, ws.cpu().double(), f"{mode} call {call} vs workspace call")
+
+
+def test_noalloc_matches_oracle_paged():
+    """Paged arena through the scratch array, against the oracle."""
+    m = kvq()
+    B, Hq, Hk, D = 4, 32, 8, 128
+    lens = [1200, 3001, 16, 640]
+    table, npages = synth.page_table_for(lens, 16, torch.Generator().manual_seed(5))
+    c = PagedCache(npages, Hk, D, "per_token", table)
+    g = torch.Generator().manual_seed(72)
+    for b, L in enumerate(lens):
+        kh = torch.randn(1, Hk, L, D, generator=g).to(torch.bfloat16)
+        vh = torch.randn(1, Hk, L, D, generator=g).to(torch.bfloat16)
+        assert c.append(kh, vh, torch.zeros(1, dtype=torch.int32), rows=[b]) == 0
+    seq = torch.tensor(lens, dtype=torch.int32)
+    for call in range(2):
+        q = bf16_randn((B, Hq, D), seed=90 + call)
+        out = _noalloc(m, q.cuda(), c, seq.cuda(), max(lens), "per_token", paged=True)
+        assert_attn_close(out, c.oracle_decode(q, seq, f32_scale(D)), f"paged call {call}")
