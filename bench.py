@@ -728,7 +728,7 @@ def main(argv=None):
                     help="time only the headline workload")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0,
                     help="seconds of oracle work per CPU-baseline leg")
-    ap.add_argument("--cpu-layers", type=int, default=400)
+    ap.add_argument("--cpu-layers", type=int, default=1500)
     ap.add_argument("--qlen", type=int, default=1,
                     help="queries per head per step: > 1 runs chunk attention steps")
     args = ap.parse_args(argv)

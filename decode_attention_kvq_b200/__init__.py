@@ -283,3 +283,67 @@ def kvq_cache_bytes(layers, Hk, seq, D, mode="per_token") -> int:
 
 def kvq_version() -> str:
     return lib.kvq_version().decode()
+
+
+class Pager:
+    """Host bookkeeping of a paged arena (kvq_pager_* in include/kvq.h): the
+    free-page allocator, one page table and length per sequence, append,
+    rollback (popn), release and reset, and the rollback rule of
+    sliding-window layers.  The pager's memory is a host buffer this object
+    owns; ``table()`` / ``lens()`` are int32 host tensors over it, to be
+    copied to the device for kvq_append_paged and the attention calls."""
+
+    def __init__(self, num_pages: int, max_seqs: int, max_pages: int, page_size: int = 16,
+                 windows=()):
+        wins = (ctypes.c_int32 * max(len(windows), 1))(*[int(w) for w in windows])
+        nbytes = int(lib.kvq_pager_bytes(num_pages, max_seqs, max_pages, len(windows)))
+        if nbytes == 0:
+            raise ValueError("bad pager sizes")
+        # 16-byte aligned host buffer (torch's CPU allocator aligns to 64 bytes)
+        self._mem = torch.empty(nbytes, dtype=torch.uint8)
+        handle = ctypes.c_void_p()
+        check(lib.kvq_pager_init(self._mem.data_ptr(), nbytes, num_pages, page_size, max_seqs,
+                                 max_pages, wins if windows else None, len(windows),
+                                 ctypes.byref(handle)), "kvq_pager_init")
+        self._h = handle
+        self.num_pages, self.max_seqs, self.max_pages = num_pages, max_seqs, max_pages
+        self.page_size = page_size
+        tp = lib.kvq_pager_table(self._h)
+        lp = lib.kvq_pager_lens(self._h)
+        base = self._mem.data_ptr()
+        # the table and the lengths live inside the pager's buffer
+        self._table = self._mem[tp - base:tp - base + 4 * max_seqs * max_pages].view(
+            torch.int32).view(max_seqs, max_pages)
+        self._lens = self._mem[lp - base:lp - base + 4 * max_seqs].view(torch.int32)
+
+    def append(self, seq: int, n: int) -> int:
+        """Grow sequence seq by n tokens; returns the first write position."""
+        pos = ctypes.c_int64(0)
+        check(lib.kvq_pager_append(self._h, seq, n, ctypes.byref(pos)), "kvq_pager_append")
+        return pos.value
+
+    def popn(self, seq: int, n: int) -> int:
+        return int(lib.kvq_pager_popn(self._h, seq, n))
+
+    def release(self, seq: int) -> None:
+        check(lib.kvq_pager_release(self._h, seq), "kvq_pager_release")
+
+    def reset(self) -> None:
+        lib.kvq_pager_reset(self._h)
+
+    def num_free(self) -> int:
+        return int(lib.kvq_pager_free_pages(self._h))
+
+    def pages_used(self, seq: int) -> int:
+        return int(lib.kvq_pager_pages_used(self._h, seq))
+
+    def seq_len(self, seq: int) -> int:
+        return int(lib.kvq_pager_seq_len(self._h, seq))
+
+    def table(self) -> torch.Tensor:
+        """int32 [max_seqs, max_pages] host view (-1 = no page)."""
+        return self._table
+
+    def lens(self) -> torch.Tensor:
+        """int32 [max_seqs] host view of the lengths."""
+        return self._lens

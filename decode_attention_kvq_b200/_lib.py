@@ -36,6 +36,17 @@ _PROTOS = {
     "kvq_version": (ctypes.c_char_p, []),
     "kvq_decode_attn_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _I, _P, _P]),
     "kvq_noalloc_scratch_bytes": (_SZ, []),
+    "kvq_pager_bytes": (_SZ, [_I, _I, _I, _I]),
+    "kvq_pager_init": (_I, [_P, _SZ, _I, _I, _I, _I, _P, _I, _P]),
+    "kvq_pager_append": (_I, [_P, _I, _I64, _P]),
+    "kvq_pager_popn": (_I64, [_P, _I, _I64]),
+    "kvq_pager_release": (_I, [_P, _I]),
+    "kvq_pager_reset": (None, [_P]),
+    "kvq_pager_free_pages": (_I, [_P]),
+    "kvq_pager_pages_used": (_I, [_P, _I]),
+    "kvq_pager_seq_len": (_I64, [_P, _I]),
+    "kvq_pager_table": (_P, [_P]),
+    "kvq_pager_lens": (_P, [_P]),
 }
 
 for _name, (_res, _args) in _PROTOS.items():

@@ -252,6 +252,7 @@ const char* kvq_status_string(kvq_status status) {
         case KVQ_ERR_CUDA: return "KVQ_ERR_CUDA";
         case KVQ_ERR_DEVICE_FLAG: return "KVQ_ERR_DEVICE_FLAG";
         case KVQ_ERR_SCRATCH_TOO_SMALL: return "KVQ_ERR_SCRATCH_TOO_SMALL";
+        case KVQ_ERR_OUT_OF_PAGES: return "KVQ_ERR_OUT_OF_PAGES";
     }
     return "KVQ_UNKNOWN_STATUS";
 }

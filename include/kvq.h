@@ -49,8 +49,9 @@ typedef enum kvq_status {
     KVQ_ERR_UNSUPPORTED = 2,   /* valid but not built: head_dim or GQA group outside the kernels' set */
     KVQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
     KVQ_ERR_DEVICE_FLAG = 4,   /* kvq_read_error found device-side error bits */
-    KVQ_ERR_SCRATCH_TOO_SMALL = 5  /* kvq_decode_attn_noalloc: the problem needs more split-K
+    KVQ_ERR_SCRATCH_TOO_SMALL = 5, /* kvq_decode_attn_noalloc: the problem needs more split-K
                                       scratch than the library's fixed array holds */
+    KVQ_ERR_OUT_OF_PAGES = 6       /* kvq_pager_append: the free pages cannot hold the tokens */
 } kvq_status;
 
 typedef enum kvq_scale_mode {
@@ -260,6 +261,68 @@ kvq_status kvq_decode_attn_noalloc(const uint16_t *q, int B, int Hq, int Hk, int
 
 /* Size in bytes of the scratch array kvq_decode_attn_noalloc uses (no counterpart on the pages). */
 size_t kvq_noalloc_scratch_bytes(void);
+
+/*
+ * ---- Paged-cache bookkeeping on the host --------------------------------
+ * A pager owns no device memory: it keeps, in caller-provided host memory,
+ * the free-page allocator of one arena of num_pages pages, one page table and
+ * one length per sequence, and the rollback rule of sliding-window layers.
+ * Its table (kvq_pager_table) is the int32 [max_seqs, max_pages] page table,
+ * -1 past each sequence's pages, that kvq_append_paged and the attention
+ * calls read after the caller copies it to the device; kvq_pager_append
+ * returns the write position to pass as d_pos.  Host code only; a pager is
+ * not safe for concurrent use from several host threads.
+ * Source: combs-models 0.2.2, src/kv.rs -- PageAllocator (free-page stack,
+ * page 0 first, freed pages reused last-in first-out), CacheConfig::num_pages,
+ * PagedKVCache::ensure_pages, popn, reset; one sequence there, one table per
+ * sequence here, all sharing the allocator.
+ */
+typedef struct kvq_pager kvq_pager;
+
+/* Host bytes a pager needs (0 on bad sizes).  num_windows: sliding-window
+ * layers whose rollback rule the pager enforces (0 = none). */
+size_t kvq_pager_bytes(int num_pages, int max_seqs, int max_pages, int num_windows);
+
+/* Lays a pager out in `mem` (16-byte aligned, at least kvq_pager_bytes(...)
+ * bytes, owned by the caller for the pager's lifetime): every page free,
+ * every sequence empty.  windows[i] >= 2 are the sliding-window sizes w of
+ * the model's sliding layers (a layer of window w keeps w - 1 past tokens).
+ * Requirements: num_pages, max_seqs, max_pages, page_size >= 1;
+ * max_pages * page_size < 2^31.  Otherwise KVQ_ERR_INVALID_ARG. */
+kvq_status kvq_pager_init(void *mem, size_t bytes, int num_pages, int page_size, int max_seqs,
+                          int max_pages, const int32_t *windows, int num_windows,
+                          kvq_pager **pager);
+
+/* Appends n >= 0 tokens to sequence seq: its table grows to
+ * ceil((len + n) / page_size) pages, each new page popped from the free
+ * stack, and the length becomes len + n; *pos (may be NULL) receives the old
+ * length, the first write position.  KVQ_ERR_OUT_OF_PAGES when the free
+ * pages cannot cover the growth and KVQ_ERR_INVALID_ARG beyond
+ * max_pages * page_size tokens; in both cases nothing changes. */
+kvq_status kvq_pager_append(kvq_pager *pager, int seq, int64_t n, int64_t *pos);
+
+/* Rolls back the last n tokens of sequence seq (n clamped to its length):
+ * pages that no longer hold a token go back onto the free stack, the last
+ * page first.  Returns the number of tokens removed: 0 also when a sliding
+ * layer has already evicted (length > w - 1 for some window w), in which
+ * case nothing changes (the evicted tokens cannot be restored). */
+int64_t kvq_pager_popn(kvq_pager *pager, int seq, int64_t n);
+
+/* Sequence seq finished: all its pages freed, length 0 (no sliding-layer
+ * rule: nothing is rolled back into).  Not on the page, whose cache holds
+ * one sequence. */
+kvq_status kvq_pager_release(kvq_pager *pager, int seq);
+
+/* Every page free, every sequence empty. */
+void kvq_pager_reset(kvq_pager *pager);
+
+int kvq_pager_free_pages(const kvq_pager *pager);
+int kvq_pager_pages_used(const kvq_pager *pager, int seq);
+int64_t kvq_pager_seq_len(const kvq_pager *pager, int seq);
+/* Host views into the pager's memory: table int32 [max_seqs, max_pages]
+ * (-1 = no page) and lengths int32 [max_seqs]. */
+const int32_t *kvq_pager_table(const kvq_pager *pager);
+const int32_t *kvq_pager_lens(const kvq_pager *pager);
 
 /* Human-readable name of a status code (static string). */
 const char *kvq_status_string(kvq_status status);
