@@ -48,6 +48,9 @@ def _load():
         lib.oracle_chunk_attn.argtypes = [P, I, I, I, I, I, I, P, P, P, P, I, I, P, I, I, P,
                                           ctypes.c_double, P]
         lib.oracle_chunk_attn.restype = I
+        lib.oracle_window_attn.argtypes = [P, I, I, I, I, I, I, P, P, P, P, I, I, P, I, I, P, I,
+                                           ctypes.c_double, P]
+        lib.oracle_window_attn.restype = I
         lib.oracle_cache_bytes.argtypes = [I64] * 6
         lib.oracle_cache_bytes.restype = I64
         lib.oracle_fp32_cache_bytes.argtypes = [I64] * 4
@@ -182,6 +185,42 @@ def chunk_attn(q, k, v, k_scale, v_scale, seq_lens, attn_scale=None, mode="per_t
                                         vc.data_ptr(), ks.data_ptr(), vs.data_ptr(),
                                         kc.shape[2], 0, None, 0, 0, sl.data_ptr(),
                                         float(attn_scale), out.data_ptr())
+    return (out, err) if return_err else out
+
+
+def window_attn(q, k, v, k_scale, v_scale, seq_lens, window, attn_scale=None,
+                mode="per_token", page_size=0, table=None, return_err=False):
+    """fp64 sliding-window attention: query i of a sequence of length L (the
+    chunk's T tokens included) sits at position p = L - T + i and attends to
+    positions max(0, p - window + 1) .. p.  q bf16 [B,Hq,D] (a decode step,
+    T = 1) or [B,Hq,T,D]; cache arguments as for decode_attn.  Returns fp64
+    with q's shape."""
+    if q.dim() == 3:
+        B, Hq, D = q.shape
+        T = 1
+    else:
+        B, Hq, T, D = q.shape
+    grp = group_of(mode, D)
+    Hk = k.shape[1]
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    qb = _bits16(q)
+    kc, vc = _cpu(k, torch.uint8), _cpu(v, torch.uint8)
+    ks, vs = _cpu(k_scale, torch.float32), _cpu(v_scale, torch.float32)
+    sl = _cpu(seq_lens, torch.int32)
+    out = torch.empty(*q.shape, dtype=torch.float64)
+    if page_size > 0:
+        tb = _cpu(table, torch.int32)
+        err = _load().oracle_window_attn(qb.data_ptr(), B, Hq, Hk, T, D, grp, kc.data_ptr(),
+                                         vc.data_ptr(), ks.data_ptr(), vs.data_ptr(), 0,
+                                         page_size, tb.data_ptr(), tb.shape[1], kc.shape[0],
+                                         sl.data_ptr(), int(window), float(attn_scale),
+                                         out.data_ptr())
+    else:
+        err = _load().oracle_window_attn(qb.data_ptr(), B, Hq, Hk, T, D, grp, kc.data_ptr(),
+                                         vc.data_ptr(), ks.data_ptr(), vs.data_ptr(),
+                                         kc.shape[2], 0, None, 0, 0, sl.data_ptr(), int(window),
+                                         float(attn_scale), out.data_ptr())
     return (out, err) if return_err else out
 
 

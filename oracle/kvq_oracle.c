@@ -32,6 +32,9 @@
  *    the cache offset is seq_len - q_len and query q_pos sees the positions
  *    up to offset + q_pos) and combs-models 0.2.2, src/kv.rs, attend (a
  *    query at global position p attends the keys at positions <= p).
+ *  - Sliding-window attention: combs-models 0.2.2, src/kv.rs, attend with
+ *    a window w (a query at position p sees the keys p - w + 1 .. p) as
+ *    PagedKVCache::sliding_attention uses it for sliding layers.
  *  - Paged layout: combs-models 0.2.2, src/kv.rs, PagedKVCache (arena
  *    [num_pages, n_kv, page_size, head_dim]; logical token g lives in
  *    physical page table[g / page_size], slot g % page_size).
@@ -313,4 +316,82 @@ int64_t oracle_cache_bytes(int64_t layers, int64_t Hk, int64_t seq, int64_t D, i
 /* fp32 equivalent, as in kv_cache_fp32_equivalent_bytes. */
 int64_t oracle_fp32_cache_bytes(int64_t layers, int64_t Hk, int64_t seq, int64_t D) {
     return layers * 2 * Hk * seq * D * 4;
+}
+
+/*
+ * Sliding-window attention of T queries per (sequence, q head) over the
+ * dequantized cache, in fp64: query i sits at position p = L - T + i (L
+ * counts the chunk's T tokens; T = 1 is a decode step) and attends to the
+ * positions max(0, p - window + 1) .. p -- the causal mask with the window
+ * rule of combs-models 0.2.2, src/kv.rs, attend (a key at position k is
+ * forbidden when k > p or when k + window - 1 < p) as the sliding layers of
+ * PagedKVCache::sliding_attention use it.  window >= 1; the cache arguments
+ * are those of oracle_decode_attn.  L = 0 gives zero rows; 0 < L < T is a
+ * length error (zero rows).
+ */
+int oracle_window_attn(const uint16_t *q, int B, int Hq, int Hk, int T, int D, int group,
+                       const uint8_t *k, const uint8_t *v, const float *k_scale,
+                       const float *v_scale, int max_seq, int page_size,
+                       const int32_t *table, int max_pages, int num_pages,
+                       const int32_t *seq_lens, int window, double attn_scale, double *out) {
+    int err = 0, ng = D / group, G = Hq / Hk;
+    int64_t cap = page_size > 0 ? (int64_t)max_pages * page_size : max_seq;
+    double *z = NULL, *kh = (double *)malloc(sizeof(double) * D);
+    double *acc = (double *)malloc(sizeof(double) * D);
+    int64_t *rows = NULL;
+    for (int b = 0; b < B; ++b) {
+        int64_t L = seq_lens[b];
+        if (L < 0 || L > cap || (L > 0 && L < T)) { err |= ORACLE_ERR_LEN; L = 0; }
+        rows = (int64_t *)realloc(rows, sizeof(int64_t) * (L > 0 ? L : 1));
+        z = (double *)realloc(z, sizeof(double) * (L > 0 ? L : 1));
+        int bad = 0;
+        for (int64_t t = 0; t < L; ++t) {
+            if (page_size > 0) {
+                int32_t phys = table[(int64_t)b * max_pages + t / page_size];
+                if (phys < 0 || phys >= num_pages) { bad = 1; break; }
+                rows[t] = (int64_t)phys * Hk * page_size + t % page_size;
+            } else {
+                rows[t] = (int64_t)b * Hk * max_seq + t;
+            }
+        }
+        if (bad) { err |= ORACLE_ERR_PAGE; L = 0; }
+        for (int h = 0; h < Hq; ++h) {
+            int hk = h / G;
+            int64_t hstride = page_size > 0 ? page_size : max_seq;
+            for (int i = 0; i < T; ++i) {
+                double *o = out + (((int64_t)b * Hq + h) * T + i) * D;
+                if (L == 0) { for (int d = 0; d < D; ++d) o[d] = 0.0; continue; }
+                const uint16_t *qh = q + (((int64_t)b * Hq + h) * T + i) * D;
+                int64_t p = L - T + i;                      /* the query's position */
+                int64_t first = p - window + 1;             /* oldest key the window keeps */
+                if (first < 0) first = 0;
+                double zmax = -INFINITY;
+                for (int64_t t = first; t <= p; ++t) {
+                    int64_t row = rows[t] + (int64_t)hk * hstride;
+                    for (int d = 0; d < D; ++d) {
+                        float s = k_scale[row * ng + d / group];
+                        kh[d] = (double)((float)((int)k[row * D + d] - 128) * s);
+                    }
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += (double)widen_bf16(qh[d]) * kh[d];
+                    z[t] = dot * attn_scale;
+                    if (z[t] > zmax) zmax = z[t];
+                }
+                double l = 0.0;
+                for (int d = 0; d < D; ++d) acc[d] = 0.0;
+                for (int64_t t = first; t <= p; ++t) {
+                    int64_t row = rows[t] + (int64_t)hk * hstride;
+                    double e = exp(z[t] - zmax);
+                    l += e;
+                    for (int d = 0; d < D; ++d) {
+                        float s = v_scale[row * ng + d / group];
+                        acc[d] += e * (double)((float)((int)v[row * D + d] - 128) * s);
+                    }
+                }
+                for (int d = 0; d < D; ++d) o[d] = acc[d] / l;
+            }
+        }
+    }
+    free(z); free(kh); free(acc); free(rows);
+    return err;
 }
