@@ -231,6 +231,41 @@ def kvq_chunk_workspace_bytes(B, Hq, Hk, T, D, max_seq_len_hint, num_splits=0) -
                                              int(num_splits)))
 
 
+def kvq_window_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, window, *,
+                    Hk=None, page_table=None, page_size=0, attn_scale=None, mode="per_token",
+                    out=None, workspace=None, num_splits=0, err=None, stream=None,
+                    view: Optional[CacheView] = None):
+    """Sliding-window attention: q bf16 [B,Hq,D] (a decode step) or
+    [B,Hq,T,D]; query i at position L - T + i sees the positions
+    max(0, p - window + 1) .. p.  Returns fp32 of q's shape."""
+    if q.dim() == 3:
+        B, Hq, D = q.shape
+        T = 1
+    else:
+        B, Hq, T, D = q.shape
+    if Hk is None:
+        Hk = k.shape[1]
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    if view is None:
+        view = cache_view(k, v, k_scale, v_scale, page_table, page_size)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = int(lib.kvq_window_workspace_bytes(B, Hq, Hk, T, D, int(max_seq_len_hint),
+                                                  int(window), int(num_splits)))
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace, None, "workspace") if workspace is not None else 0
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    check(lib.kvq_window_attn(
+        _ptr(q, torch.bfloat16, "q"), B, Hq, Hk, T, D, _mode(mode), ctypes.byref(view),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(max_seq_len_hint), int(window),
+        float(attn_scale), _ptr(out, torch.float32, "out"), ws_ptr, ws_bytes, int(num_splits),
+        _ptr(err, torch.int32, "err"), _stream(stream, q)), "kvq_window_attn")
+    return out
+
+
 def kvq_decode_attn_noalloc(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *,
                             Hk=None, page_table=None, page_size=0, attn_scale=None,
                             mode="per_token", out=None, num_splits=0, err=None, stream=None,

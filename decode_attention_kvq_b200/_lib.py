@@ -28,6 +28,9 @@ _PROTOS = {
     "kvq_chunk_attn": (_I, [_P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _SZ, _I, _P,
                             _P]),
     "kvq_chunk_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "kvq_window_attn": (_I, [_P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _F, _P, _P, _SZ, _I,
+                             _P, _P]),
+    "kvq_window_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "kvq_decode_plan": (_I, [_I, _I, _I, _I, _I, _P, _P]),
     "kvq_dequant": (_I, [_P, _P, _I64, _I, _I, _P, _P]),
     "kvq_status_string": (ctypes.c_char_p, [_I]),

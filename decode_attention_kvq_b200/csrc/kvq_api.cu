@@ -78,10 +78,20 @@ size_t workspace_for(int B, int Hq, int D, int splits) {
 // Decode (T = 1) and chunk (T > 1) attention: the T queries of a (sequence,
 // q head) ride as T rows of the GQA group, so the split kernel sees Hq * T
 // heads, G * T per kv head, and masks each row causally.
+// The longest run of tokens a sequence's queries walk: everything up to the
+// hint, or with a sliding window at most T + window - 1 positions plus the
+// up-to-15 below the window that its 16-aligned base adds.
+int walked_hint(int hint, int T, int window) {
+    if (window <= 0) return hint;
+    const int64_t w = static_cast<int64_t>(window) + T - 1 + 15;
+    return w < hint ? static_cast<int>(w) : hint;
+}
+
 kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_scale_mode mode,
                   const kvq_cache_view* kv, const int32_t* d_seq_lens, int max_seq_len_hint,
-                  float attn_scale, float* out, void* workspace, size_t workspace_bytes,
-                  int num_splits, int32_t* d_err, kvq_stream_t stream) {
+                  int window, float attn_scale, float* out, void* workspace,
+                  size_t workspace_bytes, int num_splits, int32_t* d_err, kvq_stream_t stream) {
+    if (window < 0) return KVQ_ERR_INVALID_ARG;
     if (!q || !kv || !kv->k || !kv->v || !kv->k_scale || !kv->v_scale || !d_seq_lens || !out)
         return KVQ_ERR_INVALID_ARG;
     if (B < 0 || Hq < 1 || Hk < 1 || (Hq % Hk) != 0 || D < 16 || (D % 16) != 0 ||
@@ -115,7 +125,8 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
     if (B == 0) return KVQ_OK;
 
     int chunk = 0, splits = 0;
-    kvq_status st = plan(B, Hk, max_seq_len_hint, num_splits, 0, &chunk, &splits);
+    const int hint = walked_hint(max_seq_len_hint, T, window);
+    kvq_status st = plan(B, Hk, hint, num_splits, 0, &chunk, &splits);
     if (st != KVQ_OK) return st;
     // work items (sequence, kv head, chunk) are counted in 32-bit integers
     if (static_cast<int64_t>(B) * Hk * (splits + 3) >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
@@ -133,6 +144,7 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
     p.ws_l = ws ? ws + n_part * (D + 1) : nullptr;
     p.B = B; p.Hq = Hq * T; p.Hk = Hk; p.G = G; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
     p.qlen = T;
+    p.window = window;
     p.page_size = kv->page_size; p.max_seq = kv->max_seq; p.max_pages = kv->max_pages;
     p.num_pages = kv->num_pages; p.chunk = chunk; p.splits = splits;
     {
@@ -212,7 +224,7 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
                            int max_seq_len_hint, float attn_scale, float* out, void* workspace,
                            size_t workspace_bytes, int num_splits, int32_t* d_err,
                            kvq_stream_t stream) {
-    return attend(q, B, Hq, Hk, 1, D, mode, kv, d_seq_lens, max_seq_len_hint, attn_scale, out,
+    return attend(q, B, Hq, Hk, 1, D, mode, kv, d_seq_lens, max_seq_len_hint, 0, attn_scale, out,
                   workspace, workspace_bytes, num_splits, d_err, stream);
 }
 
@@ -222,8 +234,25 @@ kvq_status kvq_chunk_attn(const uint16_t* q, int B, int Hq, int Hk, int T, int D
                           float* out, void* workspace, size_t workspace_bytes, int num_splits,
                           int32_t* d_err, kvq_stream_t stream) {
     if (T < 1) return KVQ_ERR_INVALID_ARG;
-    return attend(q, B, Hq, Hk, T, D, mode, kv, d_seq_lens, max_seq_len_hint, attn_scale, out,
+    return attend(q, B, Hq, Hk, T, D, mode, kv, d_seq_lens, max_seq_len_hint, 0, attn_scale, out,
                   workspace, workspace_bytes, num_splits, d_err, stream);
+}
+
+kvq_status kvq_window_attn(const uint16_t* q, int B, int Hq, int Hk, int T, int D,
+                           kvq_scale_mode mode, const kvq_cache_view* kv,
+                           const int32_t* d_seq_lens, int max_seq_len_hint, int window,
+                           float attn_scale, float* out, void* workspace, size_t workspace_bytes,
+                           int num_splits, int32_t* d_err, kvq_stream_t stream) {
+    if (T < 1 || window < 1) return KVQ_ERR_INVALID_ARG;
+    return attend(q, B, Hq, Hk, T, D, mode, kv, d_seq_lens, max_seq_len_hint, window, attn_scale,
+                  out, workspace, workspace_bytes, num_splits, d_err, stream);
+}
+
+size_t kvq_window_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_seq_len_hint,
+                                  int window, int num_splits) {
+    if (T < 1 || window < 1 || Hq > INT32_MAX / T) return 0;
+    return kvq_decode_workspace_bytes(B, Hq * T, Hk, D, walked_hint(max_seq_len_hint, T, window),
+                                      num_splits);
 }
 
 size_t kvq_chunk_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_seq_len_hint,

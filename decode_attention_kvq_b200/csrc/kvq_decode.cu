@@ -74,7 +74,7 @@ decode_combine_one(DecodeParams p) {
     const bool active = lane * 4 < D;
     const float* o = p.ws_o + bh * p.splits * D + lane * 4;
     const int64_t cap = p.page_size ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
-    const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
+    const int64_t plan = static_cast<int64_t>(p.splits) * p.chunk;
     const int L0 = p.seq_lens[b];
 
     float Mw = -INFINITY, lw = 0.f;
@@ -117,7 +117,7 @@ decode_combine_one(DecodeParams p) {
     };
     // the first round of loads is issued together with the length
     load(w);
-    const int L = (L0 < 0 || L0 > lim) ? 0 : L0;
+    const int L = max(walked_len(L0, cap, plan, p.qlen, p.window), 0);
     const int ns = (L + p.chunk - 1) / p.chunk;
     if (ns <= 1) return;                        // finished by the split kernel
     fold(w, ns);
@@ -150,7 +150,7 @@ decode_combine_live(DecodeParams p) {
     const bool active = lane * 4 < D;
     const float* o = p.ws_o + bh * p.splits * D + lane * 4;
     const int64_t cap = p.page_size ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
-    const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
+    const int64_t plan = static_cast<int64_t>(p.splits) * p.chunk;
     const int L0 = p.seq_lens[b];
     float mv0[kWords];
 #pragma unroll
@@ -158,7 +158,7 @@ decode_combine_live(DecodeParams p) {
         const int j = 32 * x + lane;
         mv0[x] = j < p.splits ? m[j] : -INFINITY;
     }
-    const int L = (L0 < 0 || L0 > lim) ? 0 : L0;
+    const int L = max(walked_len(L0, cap, plan, p.qlen, p.window), 0);
     const int ns = (L + p.chunk - 1) / p.chunk;
     if (ns <= 1) return;                        // finished by the split kernel
 

@@ -65,6 +65,7 @@
 #include <math.h>
 
 #include <atomic>
+#include <climits>
 #include <type_traits>
 #include <unordered_map>
 
@@ -236,9 +237,11 @@ __device__ __forceinline__ Seg seg_at(int i, int iend, const int* lens, const in
 // and one fold; lanes t and t ^ 2 (the two parities) add their scores.  P''
 // is built once per group pair, each column with its own parity's V scale;
 // the P.V output columns of the other parity are not used.
-// CAUSAL (a chunk of T = p.qlen queries per sequence and q head): the G
-// columns are (head, query i) rows, query fastest, and column i of a sequence
-// of length L sees the positions <= L - T + i (L counts the chunk's tokens).
+// CAUSAL (a chunk of T = p.qlen queries per sequence and q head, or a
+// sliding window): the G columns are (head, query i) rows, query fastest, and
+// column i of a sequence of length L sees the positions <= L - T + i (L
+// counts the chunk's tokens) and, with a window w, >= L - T + i - w + 1.
+// With a window the tokens are counted from the sequence's window base.
 template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL>
 __global__ void __launch_bounds__(nthreads(PAGED), 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -307,7 +310,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (!PAGED && prm.one_item && tid == 32) {
+    if (!PAGED && prm.one_item && !prm.window && tid == 32) {
         // one item per CTA, contiguous cache: the item's first two stages of K
         // and V rows (and their scales) do not depend on the length, so they
         // are prefetched into L2 while the predecessor finishes (more than two
@@ -352,12 +355,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     // ---- lengths and chunk prefix sums (items per sequence: Hk * max(1, chunks))
     if (!one) {
         const int64_t cap = PAGED ? static_cast<int64_t>(prm.max_pages) * prm.page_size : prm.max_seq;
-        const int64_t lim = min(cap, static_cast<int64_t>(prm.splits) * prm.chunk);
+        const int64_t plan = static_cast<int64_t>(prm.splits) * prm.chunk;
 #pragma unroll 1
         for (int b = tid; b < prm.B; b += nthreads(PAGED)) {
-            int L = prm.seq_lens[b];
+            const int Lraw = prm.seq_lens[b];
+            // tokens walked from the window base (all of them without a window)
+            int L = walked_len(Lraw, cap, plan, prm.qlen, prm.window);
             // (a chunk of queries needs its own tokens in the cache: L >= T)
-            if (L < 0 || L > lim || (CAUSAL && L > 0 && L < prm.qlen)) {
+            if (L < 0 || (CAUSAL && Lraw > 0 && Lraw < prm.qlen)) {
                 if (blockIdx.x == 0) raise_flag(prm.d_err, KVQ_DEVERR_LEN);
                 L = 0;
             }
@@ -426,10 +431,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     // planned window reads as 0 (flagged once, by the first consumer thread of
     // the sequence's first CTA)
     auto one_raw = [&]() { return p.seq_lens[one_b]; };
-    auto one_valid = [&](int L) {
+    auto one_valid = [&](int Lraw) {
         const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
-        const int64_t lim = min(cap, static_cast<int64_t>(p.splits) * p.chunk);
-        if (L < 0 || L > lim || (CAUSAL && L > 0 && L < p.qlen)) {
+        int L = walked_len(Lraw, cap, static_cast<int64_t>(p.splits) * p.chunk, p.qlen, p.window);
+        if (L < 0 || (CAUSAL && Lraw > 0 && Lraw < p.qlen)) {
             if (one_j == 0 && one_hk == 0 && tid == 32 * nprod(PAGED)) raise_flag(p.d_err, KVQ_DEVERR_LEN);
             L = 0;
         }
@@ -472,6 +477,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const uint16_t* const qg = p.q;
         const int32_t* const table = p.table;
         int32_t* const d_err = p.d_err;
+        // sliding window: rows are addressed from the sequence's window base
+        const int window = p.window, qlen = p.qlen;
+        const int32_t* const seq_lens = p.seq_lens;
+        const int64_t cap_tok = PAGED ? static_cast<int64_t>(max_pages) * p.page_size : max_seq;
         // floats in each scale array (contiguous layout)
         const int64_t sc_total = static_cast<int64_t>(B) * Hk * max_seq * NG;
         const uint32_t q_bytes = static_cast<uint32_t>(G * D * 2);
@@ -493,6 +502,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 int t1 = sg.t1;
                 uint32_t spec_valid = ~0u;      // paged, ONE item: the first stage's loaded pages
                 const int b = sg.b, hk = sg.hk;
+                int wb = 0;                     // the window base (a multiple of 16)
+                if (CAUSAL && window > 0) {
+                    const int Lr = ONE ? Lone : seq_lens[b];
+                    wb = (Lr >= 0 && Lr <= cap_tok) ? window_base(Lr, qlen, window) : 0;
+                }
                 const uint16_t* qsrc = qg + (static_cast<int64_t>(b) * Hq + hk * G) * D;
                 int seg_tiles = 0;          // tiles issued for this segment
                 if (ONE && pw == 0 && lane == 0) {
@@ -508,10 +522,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 int pbase = sg.t0 >> 4;
                 int32_t pg_cur = -1, pg_nxt = -1;
                 auto load_pages = [&](int first) {
-                    const int idx = first + lane;
+                    const int idx = first + lane;           // counted from the window base
+                    const int ia = (wb >> 4) + idx;         // the logical page
                     int32_t v = -1;
-                    if (16 * idx < t1 && idx < max_pages) {
-                        v = table[static_cast<int64_t>(b) * max_pages + idx];
+                    if (16 * idx < t1 && ia < max_pages) {
+                        v = table[static_cast<int64_t>(b) * max_pages + ia];
                         if (v < 0 || v >= num_pages) v = -1;
                     }
                     return v;
@@ -539,7 +554,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const bool with_q = !ONE && seg_tiles < 2;
                     if (!PAGED) {
                         if (lane == 0) {
-                            const int64_t row0 = (static_cast<int64_t>(b) * Hk + hk) * max_seq + tt0;
+                            const int64_t row0 = (static_cast<int64_t>(b) * Hk + hk) * max_seq + wb + tt0;
                             // scales: whole 16-byte chunks from the aligned float at or
                             // below the tile's first ONE; where the last chunk would run
                             // past the end of the scale array its 1-3 floats are copied
@@ -754,15 +769,18 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         i = sg.next;
         const int b = sg.b, hk = sg.hk;
         const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
-        // chunk of queries: the last position column 8 nt + 2 t + c may see
-        int lim_col[NT][2];
+        // chunk of queries: the last position column 8 nt + 2 t + c may see;
+        // sliding window: the first (both counted from the window base)
+        int lim_col[NT][2], lo_col[NT][2];
         if constexpr (CAUSAL) {
             const int Lseq = one ? one_valid(one_raw()) : lens[b];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
+                for (int c = 0; c < 2; ++c) {
                     lim_col[nt][c] = Lseq - p.qlen + (8 * nt + 2 * t + c) % p.qlen;
+                    lo_col[nt][c] = p.window > 0 ? lim_col[nt][c] - p.window + 1 : INT_MIN;
+                }
         }
         if (!one && sg.ns == 0) {
             // empty (or rejected) sequence: zero rows
@@ -923,12 +941,13 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                             z[u][nt][3] = okB[u] ? z[u][nt][3] * zs[nt][1] : -INFINITY;
                         }
                         if constexpr (CAUSAL) {
-                            // positions past the column's query are masked
+                            // positions past the column's query, or older than its
+                            // sliding window, are masked
                             const int ta = tt0 + rA[u], tb = tt0 + rB[u];
-                            if (ta > lim_col[nt][0]) z[u][nt][0] = -INFINITY;
-                            if (ta > lim_col[nt][1]) z[u][nt][1] = -INFINITY;
-                            if (tb > lim_col[nt][0]) z[u][nt][2] = -INFINITY;
-                            if (tb > lim_col[nt][1]) z[u][nt][3] = -INFINITY;
+                            if (ta > lim_col[nt][0] || ta < lo_col[nt][0]) z[u][nt][0] = -INFINITY;
+                            if (ta > lim_col[nt][1] || ta < lo_col[nt][1]) z[u][nt][1] = -INFINITY;
+                            if (tb > lim_col[nt][0] || tb < lo_col[nt][0]) z[u][nt][2] = -INFINITY;
+                            if (tb > lim_col[nt][1] || tb < lo_col[nt][1]) z[u][nt][3] = -INFINITY;
                         }
                     }
                 // ---- online softmax per head: max over the slice's 32 tokens
@@ -946,8 +965,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         const float mn = fmaxf(m[nt][c], mx);
                         const float al = (mn == -INFINITY) ? 1.f : ptx::ex2(m[nt][c] - mn);
                         float add = 0.f;
-                        // (a chunk query can have seen no position yet: its
-                        // masked scores then give 2^-inf = 0, not NaN)
+                        // (a chunk query, or a windowed one, can have seen no
+                        // position yet: its masked scores then give 2^-inf = 0,
+                        // not NaN)
                         const float mb = (CAUSAL && mn == -INFINITY) ? 0.f : mn;
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
@@ -1321,7 +1341,9 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
 
 template <int D, bool G32, bool PAGED>
 cudaError_t pick_g(const DecodeParams& p, cudaStream_t s) {
-    if (p.qlen > 1)                     // a chunk of queries: causal columns
+    // a chunk of queries (causal columns) or a sliding window: the masked
+    // instantiation (for one decode query the causal mask keeps every position)
+    if (p.qlen > 1 || p.window > 0)
         return p.G > 8 ? launch_tc<D, G32, PAGED, true, false, true>(p, s)
                        : launch_tc<D, G32, PAGED, false, false, true>(p, s);
     if (p.G > 8) return launch_tc<D, G32, PAGED, true, false, false>(p, s);

@@ -66,8 +66,27 @@ struct DecodeParams {
     int one_item;            // the plan's items fit the grid: CTA c takes item c
     int qlen;                // queries per (sequence, q head): 1 for decode, T for a chunk
                              // (Hq and G then count (head, query) rows, query fastest)
+    int window;              // sliding window w (0: none): a query at position p sees p - w + 1 .. p
     float scale_log2;        // attn_scale * log2(e)
 };
+
+// Sliding window: the oldest position any of a sequence's qlen queries sees
+// is L - qlen - window + 1.  The kernels count a sequence's tokens from that
+// position rounded down to a multiple of 16 (whole pages, 16-byte aligned
+// scale rows), mask the few below it, and plan over L - base tokens.
+__host__ __device__ __forceinline__ int window_base(int L, int qlen, int window) {
+    if (window <= 0) return 0;
+    const int lo = L - qlen - window + 1;
+    return lo > 0 ? (lo & ~15) : 0;
+}
+
+// The number of tokens the kernels walk for a sequence of length L (from its
+// window base), or -1 when L is outside [0, cap] or beyond the plan.
+__device__ __forceinline__ int walked_len(int L, int64_t cap, int64_t plan, int qlen, int window) {
+    if (L < 0 || L > cap) return -1;
+    const int n = L - window_base(L, qlen, window);
+    return n > plan ? -1 : n;
+}
 constexpr int kMaxBatch = 1024;                              // sequences per call
 constexpr int kMaxGrid = 1024;                               // persistent CTAs
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);

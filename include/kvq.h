@@ -208,6 +208,39 @@ size_t kvq_chunk_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_se
                                  int num_splits);
 
 /*
+ * kvq_window_attn -- sliding-window attention on the INT8 cache: T >= 1 new
+ * queries per (sequence, q head) (T = 1: a decode step), query i at position
+ * p = L - T + i attending to the positions max(0, p - window + 1) .. p, with
+ * the fused dequantisation of kvq_decode_attn.  Only the last
+ * T + window - 1 positions of each sequence (from a 16-aligned start) are
+ * read, so the work is bounded by the window, not the length.
+ *   q       bf16 [B, Hq, D] (T = 1) or [B, Hq, T, D];  out fp32 of q's shape
+ *   window  w >= 1 keys per query, the newest included (a layer that keeps
+ *           w - 1 past tokens and appends one sees w)
+ *   workspace  at least kvq_window_workspace_bytes(...) bytes
+ *   the other arguments as for kvq_chunk_attn (L counts the T new tokens,
+ *   0 < L < T is a length error).
+ * The cache holds every position (positions are rows, as for the other
+ * calls).  A sliding layer that keeps only its last w tokens in a ring of w
+ * rows (position g in row g % w) decodes with plain kvq_decode_attn over
+ * min(L, w) rows instead: the softmax does not depend on the rows' order.
+ * Requirements: those of kvq_chunk_attn; window < 1 or T < 1 is
+ * KVQ_ERR_INVALID_ARG.
+ * Source: combs-models 0.2.2, src/kv.rs, attend with a window (a key at k is
+ * masked when k > p or k + w - 1 < p) as PagedKVCache::sliding_attention
+ * uses it for sliding layers (transformers' sliding-window layers).
+ */
+kvq_status kvq_window_attn(const uint16_t *q, int B, int Hq, int Hk, int T, int D,
+                           kvq_scale_mode mode, const kvq_cache_view *kv,
+                           const int32_t *d_seq_lens, int max_seq_len_hint, int window,
+                           float attn_scale, float *out, void *workspace, size_t workspace_bytes,
+                           int num_splits, int32_t *d_err, kvq_stream_t stream);
+
+/* Workspace bytes kvq_window_attn needs for these arguments (0 when no split is needed). */
+size_t kvq_window_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_seq_len_hint,
+                                  int window, int num_splits);
+
+/*
  * Split plan kvq_decode_attn uses: KV tokens per split (*chunk) and the
  * largest number of splits of any sequence (*splits).  num_sms <= 0 means the
  * current device's SM count.  Returns KVQ_ERR_INVALID_ARG on bad sizes.
