@@ -51,6 +51,17 @@ def _load():
         lib.oracle_window_attn.argtypes = [P, I, I, I, I, I, I, P, P, P, P, I, I, P, I, I, P, I,
                                            ctypes.c_double, P]
         lib.oracle_window_attn.restype = I
+        lib.oracle_fp8_encode.argtypes = [ctypes.c_float, I]
+        lib.oracle_fp8_encode.restype = ctypes.c_uint8
+        lib.oracle_fp8_decode.argtypes = [ctypes.c_uint8, I]
+        lib.oracle_fp8_decode.restype = ctypes.c_float
+        lib.oracle_fp8_encode_rows.argtypes = [P, I64, I, P]
+        lib.oracle_fp8_encode_rows.restype = None
+        lib.oracle_append_fp8.argtypes = [P, I, I, I, I, I, P, P, I, I, P, I, I]
+        lib.oracle_append_fp8.restype = I
+        lib.oracle_fp8_attn.argtypes = [P, I, I, I, I, I, I, P, P, I, I, P, I, I, P, I,
+                                        ctypes.c_double, P]
+        lib.oracle_fp8_attn.restype = I
         lib.oracle_cache_bytes.argtypes = [I64] * 6
         lib.oracle_cache_bytes.restype = I64
         lib.oracle_fp32_cache_bytes.argtypes = [I64] * 4
@@ -221,6 +232,79 @@ def window_attn(q, k, v, k_scale, v_scale, seq_lens, window, attn_scale=None,
                                          vc.data_ptr(), ks.data_ptr(), vs.data_ptr(),
                                          kc.shape[2], 0, None, 0, 0, sl.data_ptr(), int(window),
                                          float(attn_scale), out.data_ptr())
+    return (out, err) if return_err else out
+
+
+FP8_FORMATS = {"fp8_e4m3": 0, "fp8_e5m2": 1}
+
+
+def fp8_encode(x: torch.Tensor, fmt: str) -> torch.Tensor:
+    """bf16 values -> FP8 bytes (the page's truncating encoders, with the
+    readings stated in kvq_oracle.c)."""
+    xb = _bits16(x)
+    out = torch.empty(x.shape, dtype=torch.uint8)
+    _load().oracle_fp8_encode_rows(xb.data_ptr(), xb.numel(), FP8_FORMATS[fmt], out.data_ptr())
+    return out
+
+
+def fp8_encode_f32(value: float, fmt: str) -> int:
+    """One fp32 value -> its FP8 byte."""
+    return int(_load().oracle_fp8_encode(float(value), FP8_FORMATS[fmt]))
+
+
+def fp8_decode(c: torch.Tensor, fmt: str) -> torch.Tensor:
+    """FP8 bytes -> their exact fp32 values (pure-Python loop: small inputs)."""
+    f = _load().oracle_fp8_decode
+    code = FP8_FORMATS[fmt]
+    flat = _cpu(c, torch.uint8).reshape(-1).tolist()
+    return torch.tensor([f(int(b), code) for b in flat], dtype=torch.float32).reshape(c.shape)
+
+
+def append_fp8(x_new, pos, dst, fmt, page_size=0, table=None) -> int:
+    """Encode x_new bf16 [B,Hk,T,D] into an FP8 cache: contiguous
+    [B,Hk,max_seq,D] at pos[b], or a paged arena [num_pages,Hk,page_size,D]
+    with table [B,max_pages]."""
+    B, Hk, T, D = x_new.shape
+    assert dst.is_contiguous()
+    xb = _bits16(x_new)
+    p = _cpu(pos, torch.int32)
+    if page_size > 0:
+        tb = _cpu(table, torch.int32)
+        return _load().oracle_append_fp8(xb.data_ptr(), B, Hk, T, D, FP8_FORMATS[fmt],
+                                         p.data_ptr(), dst.data_ptr(), 0, page_size,
+                                         tb.data_ptr(), tb.shape[1], dst.shape[0])
+    return _load().oracle_append_fp8(xb.data_ptr(), B, Hk, T, D, FP8_FORMATS[fmt], p.data_ptr(),
+                                     dst.data_ptr(), dst.shape[2], 0, None, 0, 0)
+
+
+def fp8_attn(q, k, v, seq_lens, fmt, window=0, attn_scale=None, page_size=0, table=None,
+             return_err=False):
+    """fp64 attention over an FP8 cache: q bf16 [B,Hq,D] (decode) or
+    [B,Hq,T,D] (causal chunk); window > 0 adds the sliding-window rule.
+    Returns fp64 with q's shape."""
+    if q.dim() == 3:
+        B, Hq, D = q.shape
+        T = 1
+    else:
+        B, Hq, T, D = q.shape
+    Hk = k.shape[1]
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    qb = _bits16(q)
+    kc, vc = _cpu(k, torch.uint8), _cpu(v, torch.uint8)
+    sl = _cpu(seq_lens, torch.int32)
+    out = torch.empty(*q.shape, dtype=torch.float64)
+    f = FP8_FORMATS[fmt]
+    if page_size > 0:
+        tb = _cpu(table, torch.int32)
+        err = _load().oracle_fp8_attn(qb.data_ptr(), B, Hq, Hk, T, D, f, kc.data_ptr(),
+                                      vc.data_ptr(), 0, page_size, tb.data_ptr(), tb.shape[1],
+                                      kc.shape[0], sl.data_ptr(), int(window), float(attn_scale),
+                                      out.data_ptr())
+    else:
+        err = _load().oracle_fp8_attn(qb.data_ptr(), B, Hq, Hk, T, D, f, kc.data_ptr(),
+                                      vc.data_ptr(), kc.shape[2], 0, None, 0, 0, sl.data_ptr(),
+                                      int(window), float(attn_scale), out.data_ptr())
     return (out, err) if return_err else out
 
 

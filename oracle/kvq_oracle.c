@@ -395,3 +395,171 @@ int oracle_window_attn(const uint16_t *q, int B, int Hq, int Hk, int T, int D, i
     free(z); free(kh); free(acc); free(rows);
     return err;
 }
+
+/*
+ * FP8 KV format: every value is stored as one FP8 byte and there is no
+ * scale.  llama-gguf 0.14.0, src/model/kv_quantized.rs, KVCacheFormat::
+ * Fp8E4M3 / Fp8E5M2 with quantize_fp8_e4m3 / quantize_fp8_e5m2 and their
+ * dequantize_* counterparts.  fmt 0 = E4M3 (4 exponent bits, bias 7, 3
+ * mantissa bits), fmt 1 = E5M2 (5 exponent bits, bias 15, 2 mantissa bits).
+ *
+ * The page's encoders TRUNCATE: the mantissa bits below the format's are
+ * dropped (toward zero), numbers below the smallest subnormal become a zero
+ * of their sign, and an exponent above the format's range saturates (E4M3:
+ * to +-448, code 0x7E; E5M2: to +-inf, code 0x7C).  Two readings where the
+ * page's code disagrees with its own decoders: an E4M3 value in [480, 512)
+ * would get exponent 15 and mantissa 7, the NaN pattern of the page's
+ * decoder, so it saturates to 0x7E like the larger ones; an E5M2 value in
+ * [2^16, 2^17) would get exponent 31, the inf/NaN patterns, so it encodes as
+ * inf (0x7C) like the larger ones.  +-0 encodes as 0x00; non-finite inputs
+ * follow the page (NaN -> 0xFF, E4M3 inf -> 0x7F / 0xFF, E5M2 inf -> 0x7C /
+ * 0xFC).
+ */
+uint8_t oracle_fp8_encode(float x, int fmt) {
+    const int ebits = fmt ? 5 : 4, mbits = fmt ? 2 : 3, bias = fmt ? 15 : 7;
+    const int emax = (1 << ebits) - 1;                     /* 15 or 31 */
+    if (isnan(x)) return 0xFF;
+    if (isinf(x)) return fmt ? (x > 0 ? 0x7C : 0xFC) : (x > 0 ? 0x7F : 0xFF);
+    if (x == 0.0f) return 0x00;
+    uint32_t bits;
+    memcpy(&bits, &x, sizeof bits);
+    const uint8_t sign = (uint8_t)(bits >> 31);
+    const int e = (int)((bits >> 23) & 0xFF) - 127;        /* unbiased binary32 exponent */
+    uint32_t sig = bits & 0x7FFFFF;
+    if (e != -127) sig |= 0x800000;                         /* the implicit one, bit 23 */
+    const int E = e + bias;                                 /* biased FP8 exponent */
+    const uint8_t top = (uint8_t)(sign << 7);
+    if (fmt == 0) {
+        if (E > emax) return top | 0x7E;                    /* saturate: 448 */
+    } else {
+        if (E > emax - 1) return top | 0x7C;                /* inf (reading for E = 31) */
+    }
+    if (E <= 0) {
+        const int keep = mbits + E;                         /* significand bits a subnormal keeps */
+        if (keep <= 0) return top;                          /* below the smallest subnormal */
+        return top | (uint8_t)(sig >> (24 - keep));         /* truncated subnormal mantissa */
+    }
+    uint8_t mant = (uint8_t)((sig >> (23 - mbits)) & ((1u << mbits) - 1));
+    uint8_t code = top | (uint8_t)(E << mbits) | mant;
+    if (fmt == 0 && (code & 0x7F) == 0x7F) code = top | 0x7E;   /* reading: not the NaN code */
+    return code;
+}
+
+/* The exact value of an FP8 byte (the page's dequantize_fp8_*). */
+float oracle_fp8_decode(uint8_t c, int fmt) {
+    const int mbits = fmt ? 2 : 3, bias = fmt ? 15 : 7;
+    const uint8_t mag = c & 0x7F;
+    const float sgn = (c & 0x80) ? -1.0f : 1.0f;
+    if (mag == 0) return 0.0f;
+    if (fmt == 0 && mag == 0x7F) return NAN;
+    if (fmt == 1 && mag == 0x7C) return sgn * INFINITY;
+    if (fmt == 1 && mag > 0x7C) return NAN;
+    const int E = mag >> mbits, M = mag & ((1 << mbits) - 1);
+    if (E == 0) return sgn * ldexpf((float)M, 1 - bias - mbits);       /* M * 2^(1-bias-mbits) */
+    return sgn * ldexpf((float)((1 << mbits) + M), E - bias - mbits);  /* 1.M * 2^(E-bias) */
+}
+
+void oracle_fp8_encode_rows(const uint16_t *x, int64_t n, int fmt, uint8_t *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_fp8_encode(widen_bf16(x[i]), fmt);
+}
+
+/*
+ * Append of new tokens x_new [B, Hk, T, D] to an FP8 cache: contiguous
+ * [B, Hk, max_seq, D] (page_size 0) or a paged arena [num_pages, Hk,
+ * page_size, D] with table [B, max_pages]; positions and flags as in
+ * oracle_append_contig / oracle_append_paged.
+ */
+int oracle_append_fp8(const uint16_t *x_new, int B, int Hk, int T, int D, int fmt,
+                      const int32_t *pos, uint8_t *dst, int max_seq, int page_size,
+                      const int32_t *table, int max_pages, int num_pages) {
+    int err = 0;
+    for (int b = 0; b < B; ++b) {
+        int64_t p0 = pos[b];
+        int64_t cap = page_size > 0 ? (int64_t)max_pages * page_size : max_seq;
+        if (p0 < 0 || p0 + T > cap) { err |= ORACLE_ERR_POS; continue; }
+        for (int t = 0; t < T; ++t) {
+            int64_t g = p0 + t;
+            for (int h = 0; h < Hk; ++h) {
+                int64_t row;
+                if (page_size > 0) {
+                    int32_t phys = table[(int64_t)b * max_pages + g / page_size];
+                    if (phys < 0 || phys >= num_pages) { err |= ORACLE_ERR_PAGE; continue; }
+                    row = ((int64_t)phys * Hk + h) * page_size + g % page_size;
+                } else {
+                    row = ((int64_t)b * Hk + h) * max_seq + g;
+                }
+                oracle_fp8_encode_rows(x_new + (((int64_t)b * Hk + h) * T + t) * D, D, fmt,
+                                       dst + row * D);
+            }
+        }
+    }
+    return err;
+}
+
+/*
+ * Attention over an FP8 cache in fp64, k-hat / v-hat the exact values of the
+ * bytes: T queries per (sequence, q head), query i at position p = L - T + i
+ * attending to positions max(0, p - window + 1) .. p (window 0: 0 .. p; T = 1
+ * with window 0 is a decode step over the whole cache).  Cache and length
+ * arguments as in oracle_window_attn, without scales.
+ */
+int oracle_fp8_attn(const uint16_t *q, int B, int Hq, int Hk, int T, int D, int fmt,
+                    const uint8_t *k, const uint8_t *v, int max_seq, int page_size,
+                    const int32_t *table, int max_pages, int num_pages,
+                    const int32_t *seq_lens, int window, double attn_scale, double *out) {
+    int err = 0, G = Hq / Hk;
+    int64_t cap = page_size > 0 ? (int64_t)max_pages * page_size : max_seq;
+    double *z = NULL, *kh = (double *)malloc(sizeof(double) * D);
+    double *acc = (double *)malloc(sizeof(double) * D);
+    int64_t *rows = NULL;
+    for (int b = 0; b < B; ++b) {
+        int64_t L = seq_lens[b];
+        if (L < 0 || L > cap || (L > 0 && L < T)) { err |= ORACLE_ERR_LEN; L = 0; }
+        rows = (int64_t *)realloc(rows, sizeof(int64_t) * (L > 0 ? L : 1));
+        z = (double *)realloc(z, sizeof(double) * (L > 0 ? L : 1));
+        int bad = 0;
+        for (int64_t t = 0; t < L; ++t) {
+            if (page_size > 0) {
+                int32_t phys = table[(int64_t)b * max_pages + t / page_size];
+                if (phys < 0 || phys >= num_pages) { bad = 1; break; }
+                rows[t] = (int64_t)phys * Hk * page_size + t % page_size;
+            } else {
+                rows[t] = (int64_t)b * Hk * max_seq + t;
+            }
+        }
+        if (bad) { err |= ORACLE_ERR_PAGE; L = 0; }
+        for (int h = 0; h < Hq; ++h) {
+            int hk = h / G;
+            int64_t hstride = page_size > 0 ? page_size : max_seq;
+            for (int i = 0; i < T; ++i) {
+                double *o = out + (((int64_t)b * Hq + h) * T + i) * D;
+                if (L == 0) { for (int d = 0; d < D; ++d) o[d] = 0.0; continue; }
+                const uint16_t *qh = q + (((int64_t)b * Hq + h) * T + i) * D;
+                int64_t p = L - T + i;
+                int64_t first = window > 0 ? p - window + 1 : 0;
+                if (first < 0) first = 0;
+                double zmax = -INFINITY;
+                for (int64_t t = first; t <= p; ++t) {
+                    int64_t row = rows[t] + (int64_t)hk * hstride;
+                    for (int d = 0; d < D; ++d) kh[d] = (double)oracle_fp8_decode(k[row * D + d], fmt);
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += (double)widen_bf16(qh[d]) * kh[d];
+                    z[t] = dot * attn_scale;
+                    if (z[t] > zmax) zmax = z[t];
+                }
+                double l = 0.0;
+                for (int d = 0; d < D; ++d) acc[d] = 0.0;
+                for (int64_t t = first; t <= p; ++t) {
+                    int64_t row = rows[t] + (int64_t)hk * hstride;
+                    double e = exp(z[t] - zmax);
+                    l += e;
+                    for (int d = 0; d < D; ++d)
+                        acc[d] += e * (double)oracle_fp8_decode(v[row * D + d], fmt);
+                }
+                for (int d = 0; d < D; ++d) o[d] = acc[d] / l;
+            }
+        }
+    }
+    free(z); free(kh); free(acc); free(rows);
+    return err;
+}
