@@ -32,11 +32,15 @@ from ._lib import KvqError, lib, LIB_PATH, check  # noqa: F401
 
 PER_TOKEN = 0
 GROUP32 = 1
+FP8_E4M3 = 2
+FP8_E5M2 = 3
 DEVERR_POS = 1
 DEVERR_PAGE = 2
 DEVERR_LEN = 4
 
-_MODES = {"per_token": PER_TOKEN, "group32": GROUP32, PER_TOKEN: PER_TOKEN, GROUP32: GROUP32}
+_MODES = {"per_token": PER_TOKEN, "group32": GROUP32, "fp8_e4m3": FP8_E4M3,
+          "fp8_e5m2": FP8_E5M2, PER_TOKEN: PER_TOKEN, GROUP32: GROUP32, FP8_E4M3: FP8_E4M3,
+          FP8_E5M2: FP8_E5M2}
 
 
 class CacheView(ctypes.Structure):
@@ -90,15 +94,18 @@ def _stream(stream, ref: torch.Tensor) -> int:
 
 
 def num_groups(mode, D: int) -> int:
-    return 1 if _mode(mode) == PER_TOKEN else D // 32
+    """Scales per (token, kv head): 1 per token, D / 32 for group-32, 0 for FP8."""
+    m = _mode(mode)
+    return 1 if m == PER_TOKEN else (D // 32 if m == GROUP32 else 0)
 
 
 def kvq_append(k_new, v_new, pos, k_cache, v_cache, k_scale, v_scale, mode="per_token",
                err=None, stream=None):
     """Quantise k_new/v_new bf16 [B,Hk,T,D] into the contiguous cache at pos[b].
 
-    k_cache/v_cache u8 [B,Hk,max_seq,D]; k_scale/v_scale fp32 [B,Hk,max_seq,NG];
-    pos int32 [B]; err optional int32 [1] device error word.
+    k_cache/v_cache u8 [B,Hk,max_seq,D]; k_scale/v_scale fp32 [B,Hk,max_seq,NG]
+    (None in the FP8 modes); pos int32 [B]; err optional int32 [1] device
+    error word.
     """
     B, Hk, T, D = k_new.shape
     check(lib.kvq_append(

@@ -18,13 +18,23 @@ constexpr int kMaxSplits = 4096;     // bound on splits per sequence (combine sm
 
 kvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
 
+bool valid_mode(kvq_scale_mode m) {
+    return m == KVQ_SCALE_PER_TOKEN || m == KVQ_SCALE_GROUP32 || m == KVQ_FP8_E4M3 ||
+           m == KVQ_FP8_E5M2;
+}
+bool is_fp8(kvq_scale_mode m) { return m == KVQ_FP8_E4M3 || m == KVQ_FP8_E5M2; }
+// 0: INT8 with scales, 1: E4M3, 2: E5M2 (the kernels' encoding)
+int fp8_code(kvq_scale_mode m) { return m == KVQ_FP8_E4M3 ? 1 : m == KVQ_FP8_E5M2 ? 2 : 0; }
+
 kvq_status check_append_common(const uint16_t* k_new, const uint16_t* v_new, int B, int Hk, int T,
                                int D, kvq_scale_mode mode, const int32_t* d_pos,
                                const void* kd, const void* vd, const float* ks,
                                const float* vs, const int32_t* d_err) {
-    if (!k_new || !v_new || !d_pos || !kd || !vd || !ks || !vs) return KVQ_ERR_INVALID_ARG;
+    if (!valid_mode(mode)) return KVQ_ERR_INVALID_ARG;
+    const bool scaled = !is_fp8(mode);                 // FP8 modes have no scale arrays
+    if (!k_new || !v_new || !d_pos || !kd || !vd || (scaled && (!ks || !vs)))
+        return KVQ_ERR_INVALID_ARG;
     if (B < 1 || Hk < 1 || T < 1 || D < 16 || D > 256 || (D % 16) != 0) return KVQ_ERR_INVALID_ARG;
-    if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_INVALID_ARG;
     if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
     if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(kd, 16) || !aligned(vd, 16) ||
         !aligned(ks, 16) || !aligned(vs, 16) || !aligned(d_pos, 4) || !aligned(d_err, 4))
@@ -92,12 +102,12 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
                   int window, float attn_scale, float* out, void* workspace,
                   size_t workspace_bytes, int num_splits, int32_t* d_err, kvq_stream_t stream) {
     if (window < 0) return KVQ_ERR_INVALID_ARG;
-    if (!q || !kv || !kv->k || !kv->v || !kv->k_scale || !kv->v_scale || !d_seq_lens || !out)
-        return KVQ_ERR_INVALID_ARG;
+    if (!valid_mode(mode)) return KVQ_ERR_INVALID_ARG;
+    if (!q || !kv || !kv->k || !kv->v || !d_seq_lens || !out) return KVQ_ERR_INVALID_ARG;
+    if (!is_fp8(mode) && (!kv->k_scale || !kv->v_scale)) return KVQ_ERR_INVALID_ARG;
     if (B < 0 || Hq < 1 || Hk < 1 || (Hq % Hk) != 0 || D < 16 || (D % 16) != 0 ||
         max_seq_len_hint < 0 || num_splits < 0 || B > 65535 || Hk > 65535)
         return KVQ_ERR_INVALID_ARG;
-    if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_INVALID_ARG;
     if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
     if (kv->page_size == 16) {
         if (!kv->page_table || !aligned(kv->page_table, 4) || kv->max_pages < 1 ||
@@ -143,6 +153,7 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
     p.ws_m = ws ? ws + n_part * D : nullptr;
     p.ws_l = ws ? ws + n_part * (D + 1) : nullptr;
     p.B = B; p.Hq = Hq * T; p.Hk = Hk; p.G = G; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
+    p.fp8 = fp8_code(mode);
     p.qlen = T;
     p.window = window;
     p.page_size = kv->page_size; p.max_seq = kv->max_seq; p.max_pages = kv->max_pages;
@@ -181,6 +192,7 @@ kvq_status kvq_append(const uint16_t* k_new, const uint16_t* v_new, int B, int H
     p.k_new = k_new; p.v_new = v_new; p.k_dst = k_cache; p.v_dst = v_cache;
     p.k_scale = k_scale; p.v_scale = v_scale; p.pos = d_pos; p.table = nullptr; p.d_err = d_err;
     p.B = B; p.Hk = Hk; p.T = T; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
+    p.fp8 = fp8_code(mode);
     p.max_seq = max_seq; p.page_size = 0;
     return from_cuda(kvq::launch_append(p, static_cast<cudaStream_t>(stream)));
 }
@@ -200,7 +212,8 @@ kvq_status kvq_append_paged(const uint16_t* k_new, const uint16_t* v_new, int B,
     p.k_new = k_new; p.v_new = v_new; p.k_dst = k_arena; p.v_dst = v_arena;
     p.k_scale = k_scale; p.v_scale = v_scale; p.pos = d_pos; p.table = page_table;
     p.d_err = d_err; p.B = B; p.Hk = Hk; p.T = T; p.D = D;
-    p.group32 = mode == KVQ_SCALE_GROUP32; p.max_seq = 0; p.page_size = page_size;
+    p.group32 = mode == KVQ_SCALE_GROUP32; p.fp8 = fp8_code(mode);
+    p.max_seq = 0; p.page_size = page_size;
     p.max_pages = max_pages; p.num_pages = num_pages;
     return from_cuda(kvq::launch_append(p, static_cast<cudaStream_t>(stream)));
 }
@@ -264,13 +277,14 @@ size_t kvq_chunk_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_se
 kvq_status kvq_dequant(const uint8_t* q, const float* scale, int64_t rows, int D,
                        kvq_scale_mode mode, float* out, kvq_stream_t stream) {
     if (rows < 0 || D < 16 || (D % 16) != 0) return KVQ_ERR_INVALID_ARG;
-    if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_INVALID_ARG;
+    if (!valid_mode(mode)) return KVQ_ERR_INVALID_ARG;
     if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
     if (rows == 0) return KVQ_OK;
-    if (!q || !scale || !out || !aligned(q, 16) || !aligned(out, 16) || !aligned(scale, 16))
+    if (!q || (!scale && !is_fp8(mode)) || !out || !aligned(q, 16) || !aligned(out, 16) ||
+        !aligned(scale, 16))
         return KVQ_ERR_INVALID_ARG;
-    return from_cuda(kvq::launch_dequant(q, scale, rows, D, mode == KVQ_SCALE_GROUP32, out,
-                                         static_cast<cudaStream_t>(stream)));
+    return from_cuda(kvq::launch_dequant(q, scale, rows, D, mode == KVQ_SCALE_GROUP32,
+                                         fp8_code(mode), out, static_cast<cudaStream_t>(stream)));
 }
 
 const char* kvq_status_string(kvq_status status) {
@@ -301,7 +315,7 @@ kvq_status kvq_read_error(int32_t* d_err, int32_t* bits, kvq_stream_t stream) {
 }
 
 int64_t kvq_cache_bytes(int64_t layers, int64_t Hk, int64_t seq, int D, kvq_scale_mode mode) {
-    const int64_t ng = mode == KVQ_SCALE_GROUP32 ? D / 32 : 1;
+    const int64_t ng = mode == KVQ_SCALE_GROUP32 ? D / 32 : is_fp8(mode) ? 0 : 1;
     return layers * 2 * Hk * seq * (static_cast<int64_t>(D) + 4 * ng);
 }
 

@@ -1,5 +1,9 @@
 // kvq_append.cu -- quantise new K/V tokens and store them in the INT8 cache.
 //
+// FP8 modes (llama-gguf 0.14.0, src/model/kv_quantized.rs,
+// quantize_fp8_e4m3 / quantize_fp8_e5m2): each value becomes its truncated
+// FP8 byte (fp8_from_bf16), with no scale.
+//
 // Method (abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
 // CudaQuantizedKvCache::quantize_tensor; group-32 variant after realizar
 // 0.8.5 kv_cache_q8_init.rs and combs-models 0.2.2 kv.rs kv_quantize):
@@ -71,6 +75,21 @@ append_kernel(AppendParams p, int lanes_log2) {
     const int nvec = p.D >> 3;                   // 8-value vectors per row
     const bool active = row_ok && sub < nvec;
     const uint16_t* src = (which ? p.v_new : p.k_new) + r * p.D;
+
+    if (p.fp8) {                                 // FP8: one byte a value, no scale
+        if (!active || dst_row < 0) return;
+        const uint4 raw = *reinterpret_cast<const uint4*>(src + sub * 8);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t h = (w[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+            packed[i >> 2] |= fp8_from_bf16(h, p.fp8) << (8 * (i & 3));
+        }
+        uint8_t* dst = (which ? p.v_dst : p.k_dst) + dst_row * p.D + sub * 8;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+        return;
+    }
 
     float x[8];
     float amax = 0.f;

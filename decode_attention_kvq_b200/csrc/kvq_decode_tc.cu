@@ -104,6 +104,25 @@ __device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint
     lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
+// Two FP8 bytes of w (bytes 0, 1 when hi == 0, bytes 2, 3 when hi == 1) ->
+// f16x2 holding their exact values.  F8 == 2 (E5M2): the byte is the top
+// byte of the f16 of the same value.  F8 == 1 (E4M3): the sign stays at bit
+// 15 and the 7 magnitude bits go to bits 7..13, which reads as the value
+// times 2^-8 (normal and subnormal codes alike, the biases being 7 and 15);
+// one f16x2 multiply by 256 (exact) restores it.
+template <int F8>
+__device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t w, int hi) {
+    const uint32_t y = ptx::prmt(w, 0u, hi ? 0x3424u : 0x1404u);
+    if constexpr (F8 == 2) {
+        return y;
+    } else {
+        const uint32_t r = ((y >> 1) & 0x3f803f80u) | (y & 0x80008000u);
+        uint32_t out;
+        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out) : "r"(r), "r"(0x5c005c00u));
+        return out;
+    }
+}
+
 // 8x8 b16 transpose across the warp (fragment of row lane/4, columns
 // 2*(lane%4) and +1, in and out).
 __device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
@@ -242,7 +261,7 @@ __device__ __forceinline__ Seg seg_at(int i, int iend, const int* lens, const in
 // column i of a sequence of length L sees the positions <= L - T + i (L
 // counts the chunk's tokens) and, with a window w, >= L - T + i - w + 1.
 // With a window the tokens are counted from the sequence's window base.
-template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL>
+template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8>
 __global__ void __launch_bounds__(nthreads(PAGED), 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ DecodeParams prm) {
@@ -256,6 +275,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     constexpr int NGV = G32 ? NG : 1;   // V scales per token
     static_assert(!PK || (G32 && !G16), "packing: group-32 scales, at most 4 heads");
     static_assert(!(PK && CAUSAL), "chunk queries: unpacked columns");
+    static_assert(F8 == 0 || !G32, "FP8 caches have no scales");
     constexpr int NVS = PK ? NGRP / 2 : NGV;   // P'' operand sets (PK: group pairs)
 
     extern __shared__ uint8_t smem_raw[];
@@ -335,7 +355,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                                    static_cast<int64_t>(prm.B) * prm.Hk * prm.max_seq * Lay::NG) &
                                ~static_cast<int64_t>(3);
             const int64_t a0 = f0 & ~static_cast<int64_t>(3);
-            if (f1 > a0) {
+            if (F8 == 0 && f1 > a0) {
                 ptx::prefetch_l2(prm.k_scale + a0, static_cast<uint32_t>((f1 - a0) * 4));
                 ptx::prefetch_l2(prm.v_scale + a0, static_cast<uint32_t>((f1 - a0) * 4));
             }
@@ -559,24 +579,28 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                             // below the tile's first ONE; where the last chunk would run
                             // past the end of the scale array its 1-3 floats are copied
                             // by plain loads (before the arrival that publishes them)
-                            const int64_t f0 = row0 * NG;
-                            const int off = static_cast<int>(f0 & 3);
-                            const int64_t c0 = f0 - off;
-                            const int nf = ntok * NG + off;
-                            int nb = (nf + 3) & ~3;
-                            if (c0 + nb > sc_total) {
-                                nb = nf & ~3;
+                            int nb = 0;             // 16-byte chunks of scales (none for FP8)
+                            int64_t c0 = 0;
+                            if constexpr (F8 == 0) {
+                                const int64_t f0 = row0 * NG;
+                                const int off = static_cast<int>(f0 & 3);
+                                c0 = f0 - off;
+                                const int nf = ntok * NG + off;
+                                nb = (nf + 3) & ~3;
+                                if (c0 + nb > sc_total) {
+                                    nb = nf & ~3;
 #pragma unroll 1
-                                for (int e = nb; e < nf; ++e) {
-                                    sts_f32(sks + 4 * e, k_scale[c0 + e]);
-                                    sts_f32(svs + 4 * e, v_scale[c0 + e]);
+                                    for (int e = nb; e < nf; ++e) {
+                                        sts_f32(sks + 4 * e, k_scale[c0 + e]);
+                                        sts_f32(svs + 4 * e, v_scale[c0 + e]);
+                                    }
                                 }
                             }
                             ptx::mbar_arrive_expect_tx(
                                 full, 2 * Lay::KV_BYTES + 8 * nb + (with_q ? q_bytes : 0u));
                             ptx::tma_load_2d(sk, &tm_k, 0, static_cast<int>(row0), full, pol);
                             ptx::tma_load_2d(sv, &tm_v, 0, static_cast<int>(row0), full, pol);
-                            if (nb > 0) {
+                            if (F8 == 0 && nb > 0) {
                                 ptx::bulk_load(sks, k_scale + c0, 4 * nb, full);
                                 ptx::bulk_load(svs, v_scale + c0, 4 * nb, full);
                             }
@@ -623,7 +647,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         if (pg >= 0)
                             ptx::tma_load_2d(sk + lane * 16 * D, &tm_k, 0, (pg * Hk + hk) * 16, full, pol);
 #pragma unroll
-                        for (int it = 0; it < NG; ++it) {
+                        for (int it = 0; it < (F8 ? 0 : NG); ++it) {
                             const int c = lane + 32 * it;
                             const int q = c / (4 * NG), cc = c % (4 * NG);
                             const int pq = __shfl_sync(0xffffffffu, pg, q);
@@ -721,6 +745,19 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             zsq[nt] = pow2i(-sh) * p.scale_log2;
 #pragma unroll
             for (int c = 0; c < NCG; ++c) csq[nt][c] = 0;
+            if constexpr (F8 != 0) {
+                // FP8 keys: Q^T as f16 (the prescaled bf16 values are exact in
+                // f16 down to 2^-14 of the head's max): b0 / b1 of k-step 2 gi
+                // are head_dim 32 gi + 8 t + {0,1} / {2,3}, of k-step 2 gi + 1
+                // {4,5} / {6,7}, matching the K operand's byte pairs
+#pragma unroll
+                for (int gi = 0; gi < NGRP; ++gi) {
+                    qh0[nt][gi] = ptx::pack_f16x2(qf[gi][0] * up, qf[gi][1] * up);
+                    qh1[nt][gi] = ptx::pack_f16x2(qf[gi][2] * up, qf[gi][3] * up);
+                    ql0[nt][gi] = ptx::pack_f16x2(qf[gi][4] * up, qf[gi][5] * up);
+                    ql1[nt][gi] = ptx::pack_f16x2(qf[gi][6] * up, qf[gi][7] * up);
+                }
+            } else {
 #pragma unroll
             for (int gi = 0; gi < NGRP; ++gi) {
                 uint32_t qi[8];
@@ -747,6 +784,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             for (int c = 0; c < NCG; ++c) {
                 csq[nt][c] += __shfl_xor_sync(0xffffffffu, csq[nt][c], 1);
                 csq[nt][c] += __shfl_xor_sync(0xffffffffu, csq[nt][c], 2);
+            }
             }
         }
         // per-head factors of the two heads (columns 2t, 2t+1) this thread
@@ -895,6 +933,30 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                             }
                     }
                 };
+                if constexpr (F8 != 0) {
+                    // FP8 keys: byte pairs to exact f16, two m16n8k16 k-steps per
+                    // 32 head_dim values (A rows: tokens rA, rB; k as in build_q)
+#pragma unroll
+                    for (int gi = 0; gi < NGRP; ++gi)
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const uint2 wa = lds64(sk + swz<D>(rA[u], 32 * gi + 8 * t));
+                            const uint2 wb = lds64(sk + swz<D>(rB[u], 32 * gi + 8 * t));
+                            const uint32_t a0 = fp8x2_to_f16x2<F8>(wa.x, 0);
+                            const uint32_t a1 = fp8x2_to_f16x2<F8>(wb.x, 0);
+                            const uint32_t a2 = fp8x2_to_f16x2<F8>(wa.x, 1);
+                            const uint32_t a3 = fp8x2_to_f16x2<F8>(wb.x, 1);
+                            const uint32_t c0 = fp8x2_to_f16x2<F8>(wa.y, 0);
+                            const uint32_t c1 = fp8x2_to_f16x2<F8>(wb.y, 0);
+                            const uint32_t c2 = fp8x2_to_f16x2<F8>(wa.y, 1);
+                            const uint32_t c3 = fp8x2_to_f16x2<F8>(wb.y, 1);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                ptx::mma_f16(z[u][nt], a0, a1, a2, a3, qh0[nt][gi], qh1[nt][gi]);
+                                ptx::mma_f16(z[u][nt], c0, c1, c2, c3, ql0[nt][gi], ql1[nt][gi]);
+                            }
+                        }
+                } else {
                 zero_acc(0);
 #pragma unroll
                 for (int gi = 0; gi < NGRP; ++gi) {
@@ -919,6 +981,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     }
                 }
                 if constexpr (!G32) fold(0);
+                }
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -988,8 +1051,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
                     for (int gv = 0; gv < NVS; ++gv) {
                         const int cg = PK ? 2 * gv + par : gv;
-                        vsa[u][gv] = okA[u] ? ldsf(svs + (rA[u] * NG + cg) * 4) : 0.f;
-                        vsb[u][gv] = okB[u] ? ldsf(svs + (rB[u] * NG + cg) * 4) : 0.f;
+                        vsa[u][gv] = okA[u] ? (F8 ? 1.f : ldsf(svs + (rA[u] * NG + cg) * 4)) : 0.f;
+                        vsb[u][gv] = okB[u] ? (F8 ? 1.f : ldsf(svs + (rB[u] * NG + cg) * 4)) : 0.f;
                         vmax = fmaxf(vmax, fmaxf(vsa[u][gv], vsb[u][gv]));
                     }
                 if constexpr (PK) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 2));
@@ -1058,10 +1121,18 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         for (int hh = 0; hh < 2; ++hh) {
                             const uint32_t x01 = hh ? xh01 : xl01;
                             const uint32_t x23 = hh ? xh23 : xl23;
-                            const uint32_t a0 = ptx::bytes_to_f16x2(x01, 0x4140u);
-                            const uint32_t a1 = ptx::bytes_to_f16x2(x01, 0x4342u);
-                            const uint32_t a2 = ptx::bytes_to_f16x2(x23, 0x4140u);
-                            const uint32_t a3 = ptx::bytes_to_f16x2(x23, 0x4342u);
+                            uint32_t a0, a1, a2, a3;
+                            if constexpr (F8 != 0) {     // FP8 values, exact in f16
+                                a0 = fp8x2_to_f16x2<F8>(x01, 0);
+                                a1 = fp8x2_to_f16x2<F8>(x01, 1);
+                                a2 = fp8x2_to_f16x2<F8>(x23, 0);
+                                a3 = fp8x2_to_f16x2<F8>(x23, 1);
+                            } else {                     // offset-128 bytes as exact integers
+                                a0 = ptx::bytes_to_f16x2(x01, 0x4140u);
+                                a1 = ptx::bytes_to_f16x2(x01, 0x4342u);
+                                a2 = ptx::bytes_to_f16x2(x23, 0x4140u);
+                                a3 = ptx::bytes_to_f16x2(x23, 0x4342u);
+                            }
 #pragma unroll
                             for (int nt = 0; nt < NT; ++nt) {
                                 ptx::mma_f16(o[mt0 + hh][nt], a0, a1, a2, a3, pbh[gv][nt][0],
@@ -1296,7 +1367,7 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
 
 // Function attributes belong to the current device's context, so they are
 // set once per device ordinal.
-template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL>
+template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8>
 cudaError_t set_attrs() {
     using Lay = Layout<D, G32, G16>;
     static std::atomic<uint64_t> done{0};
@@ -1304,7 +1375,7 @@ cudaError_t set_attrs() {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     return once_per_device(done, dev, cudaSuccess, [] {
-        auto kern = decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL>;
+        auto kern = decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL, F8>;
         cudaError_t r =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
         if (r == cudaSuccess)
@@ -1314,10 +1385,10 @@ cudaError_t set_attrs() {
     });
 }
 
-template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL>
+template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8 = 0>
 cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     using Lay = Layout<D, G32, G16>;
-    cudaError_t e = set_attrs<D, G32, PAGED, G16, PK, CAUSAL>();
+    cudaError_t e = set_attrs<D, G32, PAGED, G16, PK, CAUSAL, F8>();
     if (e != cudaSuccess) return e;
     CUtensorMap mk, mv;
     const int64_t rows = PAGED ? static_cast<int64_t>(p.num_pages) * p.Hk * 16
@@ -1336,7 +1407,7 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL>, mk, mv, p);
+    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL, F8>, mk, mv, p);
 }
 
 template <int D, bool G32, bool PAGED>
@@ -1352,11 +1423,27 @@ cudaError_t pick_g(const DecodeParams& p, cudaStream_t s) {
     return launch_tc<D, G32, PAGED, false, false, false>(p, s);
 }
 
+// FP8 caches (no scales): E4M3 (F8 = 1) or E5M2 (F8 = 2)
+template <int D, bool PAGED, int F8>
+cudaError_t pick_g_fp8(const DecodeParams& p, cudaStream_t s) {
+    const bool masked = p.qlen > 1 || p.window > 0;
+    if (p.G > 8)
+        return masked ? launch_tc<D, false, PAGED, true, false, true, F8>(p, s)
+                      : launch_tc<D, false, PAGED, true, false, false, F8>(p, s);
+    return masked ? launch_tc<D, false, PAGED, false, false, true, F8>(p, s)
+                  : launch_tc<D, false, PAGED, false, false, false, F8>(p, s);
+}
+
+template <int D, bool PAGED>
+cudaError_t pick_fmt(const DecodeParams& p, cudaStream_t s) {
+    if (p.fp8 == 1) return pick_g_fp8<D, PAGED, 1>(p, s);
+    if (p.fp8 == 2) return pick_g_fp8<D, PAGED, 2>(p, s);
+    return p.group32 ? pick_g<D, true, PAGED>(p, s) : pick_g<D, false, PAGED>(p, s);
+}
+
 template <int D>
 cudaError_t pick_layout(const DecodeParams& p, cudaStream_t s) {
-    if (p.page_size)
-        return p.group32 ? pick_g<D, true, true>(p, s) : pick_g<D, false, true>(p, s);
-    return p.group32 ? pick_g<D, true, false>(p, s) : pick_g<D, false, false>(p, s);
+    return p.page_size ? pick_fmt<D, true>(p, s) : pick_fmt<D, false>(p, s);
 }
 
 }  // namespace

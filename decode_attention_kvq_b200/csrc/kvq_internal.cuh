@@ -32,6 +32,7 @@ struct AppendParams {
     int32_t* d_err;
     int B, Hk, T, D;
     int group32;             // 1: 32-value groups, 0: one scale per row
+    int fp8;                 // 0: INT8 with scales, 1: FP8 E4M3, 2: FP8 E5M2 (no scales)
     int max_seq;             // contiguous capacity
     int page_size;           // 0: contiguous, else paged
     int max_pages, num_pages;
@@ -40,7 +41,7 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 
 // --------------------------------------------------------------- dequant
 cudaError_t launch_dequant(const uint8_t* q, const float* scale, int64_t rows, int D,
-                           int group32, float* out, cudaStream_t s);
+                           int group32, int fp8, float* out, cudaStream_t s);
 
 // ---------------------------------------------------------------- decode
 struct DecodeParams {
@@ -58,6 +59,7 @@ struct DecodeParams {
     int32_t* d_err;
     int B, Hq, Hk, G, D;
     int group32;
+    int fp8;                 // 0: INT8 with scales, 1: FP8 E4M3, 2: FP8 E5M2 (no scales)
     int page_size, max_seq, max_pages, num_pages;
     int chunk;               // KV tokens per split
     int splits;              // chunks of the longest sequence
@@ -92,6 +94,36 @@ constexpr int kMaxGrid = 1024;                               // persistent CTAs
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 // tensor-core split kernel (kvq_decode_tc.cu)
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s);
+
+// FP8 code of a bf16 value, truncated toward zero (the format's mantissa bits
+// kept, the rest dropped), from the bf16 fields directly: E4M3 (fmt 1, bias
+// 7, 3 mantissa bits) saturates at +-448 (0x7E, also where the truncated code
+// would be the NaN pattern 0x7F); E5M2 (fmt 2, bias 15, 2 mantissa bits)
+// gives +-inf (0x7C) from 2^16 up.  Below the smallest subnormal: a zero of
+// the value's sign; +-0 -> 0x00; NaN -> 0xFF; inf -> 0x7F / 0xFF (E4M3),
+// 0x7C / 0xFC (E5M2).
+__device__ __forceinline__ uint32_t fp8_from_bf16(uint32_t h, int fmt) {
+    const uint32_t s = (h >> 8) & 0x80u;                 // sign at bit 7
+    const int eb = static_cast<int>((h >> 7) & 0xffu);    // bf16 biased exponent
+    const uint32_t m7 = h & 0x7fu;                        // bf16 mantissa bits
+    const bool e4 = fmt == 1;
+    const int mb = e4 ? 3 : 2;
+    if (eb == 0xff) {
+        if (m7) return 0xffu;
+        return e4 ? (s ? 0xffu : 0x7fu) : (s | 0x7cu);
+    }
+    if ((h & 0x7fffu) == 0) return 0u;                    // +-0
+    const int E = eb - 127 + (e4 ? 7 : 15);               // FP8 biased exponent
+    if (e4 ? E > 15 : E > 30) return s | (e4 ? 0x7eu : 0x7cu);
+    if (E <= 0) {                                         // subnormal (or zero) code
+        const int keep = mb + E;                          // significand bits kept
+        if (keep <= 0 || eb == 0) return s;
+        return s | ((0x80u | m7) >> (8 - keep));          // 8-bit significand, top bits
+    }
+    uint32_t c = s | (static_cast<uint32_t>(E) << mb) | (m7 >> (7 - mb));
+    if (e4 && (c & 0x7fu) == 0x7fu) c = s | 0x7eu;
+    return c;
+}
 
 // Programmatic dependent launch: wait for the preceding grid's writes, and
 // let the next grid in the stream be scheduled early.

@@ -54,9 +54,22 @@ typedef enum kvq_status {
     KVQ_ERR_OUT_OF_PAGES = 6       /* kvq_pager_append: the free pages cannot hold the tokens */
 } kvq_status;
 
+/*
+ * How the cache stores values: INT8 offset-128 bytes with fp32 scales (per
+ * token or per 32-value group), or FP8 bytes with no scale.  The FP8 modes
+ * follow llama-gguf 0.14.0, src/model/kv_quantized.rs, KVCacheFormat::
+ * Fp8E4M3 / Fp8E5M2 with quantize_fp8_e4m3 / quantize_fp8_e5m2: each bf16
+ * value is TRUNCATED toward zero to the format (a zero of its sign below the
+ * smallest subnormal; E4M3 saturates at +-448 -- also for values in
+ * [480, 512), whose truncated code would be the NaN pattern -- and E5M2 gives
+ * +-inf from 2^16 up); attention reads the bytes' exact values.  In FP8 modes
+ * every scale pointer is ignored and may be NULL (NG = 0).
+ */
 typedef enum kvq_scale_mode {
     KVQ_SCALE_PER_TOKEN = 0,   /* one fp32 scale per (token, kv head): NG = 1 */
-    KVQ_SCALE_GROUP32 = 1      /* one fp32 scale per 32 values along head_dim: NG = D / 32 */
+    KVQ_SCALE_GROUP32 = 1,     /* one fp32 scale per 32 values along head_dim: NG = D / 32 */
+    KVQ_FP8_E4M3 = 2,          /* FP8 E4M3 bytes (bias 7, 3 mantissa bits), no scale: NG = 0 */
+    KVQ_FP8_E5M2 = 3           /* FP8 E5M2 bytes (bias 15, 2 mantissa bits), no scale: NG = 0 */
 } kvq_scale_mode;
 
 /* Device-side error bits (OR-ed into *d_err). */
@@ -368,8 +381,10 @@ const char *kvq_status_string(kvq_status status);
 kvq_status kvq_read_error(int32_t *d_err, int32_t *bits, kvq_stream_t stream);
 
 /*
- * Bytes of an INT8 cache with fp32 scales: layers * 2 * Hk * seq * (D + 4 * NG).
- * Source: realizar 0.8.5, kv_cache_q8_init.rs, kv_cache_q8_memory_bytes.
+ * Bytes of an INT8 cache with fp32 scales: layers * 2 * Hk * seq * (D + 4 * NG)
+ * (NG = 0 for the FP8 modes).
+ * Source: realizar 0.8.5, kv_cache_q8_init.rs, kv_cache_q8_memory_bytes;
+ * llama-gguf 0.14.0, kv_quantized.rs, memory_usage (FP8: one byte a value).
  */
 int64_t kvq_cache_bytes(int64_t layers, int64_t Hk, int64_t seq, int D, kvq_scale_mode mode);
 
