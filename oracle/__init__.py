@@ -62,6 +62,16 @@ def _load():
         lib.oracle_fp8_attn.argtypes = [P, I, I, I, I, I, I, P, P, I, I, P, I, I, P, I,
                                         ctypes.c_double, P]
         lib.oracle_fp8_attn.restype = I
+        lib.oracle_append_static.argtypes = [P, I, I, I, I, I, I, P, P, P, I]
+        lib.oracle_append_static.restype = I
+        lib.oracle_static_attn.argtypes = [P, I, I, I, I, I, I, P, P, P, P, I, P, I,
+                                           ctypes.c_double, P]
+        lib.oracle_static_attn.restype = I
+        lib.oracle_append_mixed.argtypes = [P, I, I, I, I, I, P, P, P, P, I, I]
+        lib.oracle_append_mixed.restype = I
+        lib.oracle_mixed_attn.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, I, I, P,
+                                          ctypes.c_double, P]
+        lib.oracle_mixed_attn.restype = I
         lib.oracle_cache_bytes.argtypes = [I64] * 6
         lib.oracle_cache_bytes.restype = I64
         lib.oracle_fp32_cache_bytes.argtypes = [I64] * 4
@@ -305,6 +315,82 @@ def fp8_attn(q, k, v, seq_lens, fmt, window=0, attn_scale=None, page_size=0, tab
         err = _load().oracle_fp8_attn(qb.data_ptr(), B, Hq, Hk, T, D, f, kc.data_ptr(),
                                       vc.data_ptr(), kc.shape[2], 0, None, 0, 0, sl.data_ptr(),
                                       int(window), float(attn_scale), out.data_ptr())
+    return (out, err) if return_err else out
+
+
+STATIC_GRAN = {"per_head": 1, "per_channel": 2}
+MIXED_MODES = {"per_token": 0, "group32": 1, "per_head": 3, "per_channel": 4}
+
+
+def append_static(x_new, pos, cache, scales, gran, calibrate=True) -> int:
+    """Per-head / per-channel quantisation of x_new bf16 [B,Hk,T,D] into the
+    contiguous cache at pos[b]; scales fp32 [B,Hk,1] or [B,Hk,D] are set from
+    this call's tokens (calibrate) or read."""
+    B, Hk, T, D = x_new.shape
+    assert cache.is_contiguous() and scales.is_contiguous() and scales.dtype == torch.float32
+    xb = _bits16(x_new)
+    p = _cpu(pos, torch.int32)
+    return _load().oracle_append_static(xb.data_ptr(), B, Hk, T, D, STATIC_GRAN[gran],
+                                        int(bool(calibrate)), p.data_ptr(), cache.data_ptr(),
+                                        scales.data_ptr(), cache.shape[2])
+
+
+def static_attn(q, k, v, k_scales, v_scales, seq_lens, gran, window=0, attn_scale=None,
+                return_err=False):
+    """fp64 attention over a per-head / per-channel INT8 cache: q bf16 [B,Hq,D]
+    (decode) or [B,Hq,T,D] (causal chunk), optional sliding window."""
+    if q.dim() == 3:
+        B, Hq, D = q.shape
+        T = 1
+    else:
+        B, Hq, T, D = q.shape
+    Hk = k.shape[1]
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    qb = _bits16(q)
+    kc, vc = _cpu(k, torch.uint8), _cpu(v, torch.uint8)
+    ks, vs = _cpu(k_scales, torch.float32), _cpu(v_scales, torch.float32)
+    sl = _cpu(seq_lens, torch.int32)
+    out = torch.empty(*q.shape, dtype=torch.float64)
+    err = _load().oracle_static_attn(qb.data_ptr(), B, Hq, Hk, T, D, STATIC_GRAN[gran],
+                                     kc.data_ptr(), vc.data_ptr(), ks.data_ptr(), vs.data_ptr(),
+                                     kc.shape[2], sl.data_ptr(), int(window), float(attn_scale),
+                                     out.data_ptr())
+    return (out, err) if return_err else out
+
+
+def append_mixed(x_new, lens_old, cache, scales, ring, mode="per_token", window=None) -> int:
+    """Append to a mixed cache: x_new bf16 [B,Hk,T,D] joins the bf16 window
+    ring [B,Hk,W,D]; tokens older than the window's W are quantised into the
+    INT8 part cache [B,Hk,max_seq,D] with the mode's scales."""
+    B, Hk, T, D = x_new.shape
+    W = ring.shape[2] if window is None else int(window)
+    assert ring.dtype == torch.bfloat16 and ring.is_contiguous() and cache.is_contiguous()
+    xb = _bits16(x_new)
+    lo = _cpu(lens_old, torch.int32)
+    return _load().oracle_append_mixed(xb.data_ptr(), B, Hk, T, D, MIXED_MODES[mode],
+                                       lo.data_ptr(), cache.data_ptr(), scales.data_ptr(),
+                                       ring.view(torch.int16).data_ptr(), W, cache.shape[2])
+
+
+def mixed_attn(q, k, v, k_scales, v_scales, rk, rv, seq_lens, mode="per_token",
+               attn_scale=None, window=None, return_err=False):
+    """fp64 decode attention over a mixed cache (INT8 part + bf16 window ring)."""
+    B, Hq, D = q.shape
+    Hk = k.shape[1]
+    W = rk.shape[2] if window is None else int(window)
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    qb = _bits16(q)
+    kc, vc = _cpu(k, torch.uint8), _cpu(v, torch.uint8)
+    ks, vs = _cpu(k_scales, torch.float32), _cpu(v_scales, torch.float32)
+    rkb, rvb = _bits16(rk), _bits16(rv)
+    sl = _cpu(seq_lens, torch.int32)
+    out = torch.empty(B, Hq, D, dtype=torch.float64)
+    err = _load().oracle_mixed_attn(qb.data_ptr(), B, Hq, Hk, D, MIXED_MODES[mode],
+                                    kc.data_ptr(), vc.data_ptr(), ks.data_ptr(), vs.data_ptr(),
+                                    rkb.data_ptr(), rvb.data_ptr(), W, kc.shape[2],
+                                    sl.data_ptr(), float(attn_scale), out.data_ptr())
     return (out, err) if return_err else out
 
 

@@ -563,3 +563,232 @@ int oracle_fp8_attn(const uint16_t *q, int B, int Hq, int Hk, int T, int D, int 
     free(z); free(kh); free(acc); free(rows);
     return err;
 }
+
+/*
+ * Per-head and per-channel scales (abaddon 0.2.0-rc.1,
+ * src/kv_cache_quant_cuda.rs, QuantGranularity::PerHead / PerChannel,
+ * OptimizedQuantizedKvCache::quantize_with_granularity): one fp32 scale per
+ * (sequence, kv head) -- the page's shape (batch, heads, 1, 1) -- or one per
+ * (sequence, kv head, channel) -- (batch, heads, 1, head_dim).  A calibrating
+ * call sets them from all the tokens it quantises: m = max |x| over the
+ * call's tokens and head_dim (per head) or over its tokens (per channel),
+ * floored at 1e-8, s = m / 127.  Reading: the page concatenates a later
+ * call's scales along the token axis, which its own dequantise cannot
+ * broadcast against the tokens, so a sequence keeps the scales of its
+ * calibrating call and later calls quantise with them.  Every value is then
+ * quantised with the per-token rule (round(x / s) + 128, half away from
+ * zero, clamped to [0, 255]; values beyond the calibrated range clamp).
+ *   gran 1 = per head (NS = 1 scale), gran 2 = per channel (NS = D scales).
+ *   x_new [B, Hk, T, D] bf16; cache [B, Hk, max_seq, D] at pos[b];
+ *   scales [B, Hk, NS], read (calibrate == 0) or written (calibrate == 1).
+ */
+int oracle_append_static(const uint16_t *x_new, int B, int Hk, int T, int D, int gran,
+                         int calibrate, const int32_t *pos, uint8_t *cache, float *scales,
+                         int max_seq) {
+    int err = 0, ns = gran == 1 ? 1 : D;
+    for (int b = 0; b < B; ++b) {
+        int64_t p0 = pos[b];
+        if (p0 < 0 || p0 + T > max_seq) { err |= ORACLE_ERR_POS; continue; }
+        for (int h = 0; h < Hk; ++h) {
+            const uint16_t *x = x_new + ((int64_t)b * Hk + h) * T * D;
+            float *s = scales + ((int64_t)b * Hk + h) * ns;
+            if (calibrate) {
+                for (int c = 0; c < ns; ++c) {
+                    float m = 0.0f;
+                    for (int t = 0; t < T; ++t)
+                        for (int d = 0; d < D; ++d) {
+                            if (ns > 1 && d != c) continue;
+                            float a = fabsf(widen_bf16(x[(int64_t)t * D + d]));
+                            if (a > m) m = a;
+                        }
+                    if (m < 1e-8f) m = 1e-8f;
+                    s[c] = m / 127.0f;
+                }
+            }
+            for (int t = 0; t < T; ++t)
+                for (int d = 0; d < D; ++d) {
+                    float r = widen_bf16(x[(int64_t)t * D + d]) / s[ns > 1 ? d : 0];
+                    int v = (int)roundf(r) + 128;
+                    if (v < 0) v = 0;
+                    if (v > 255) v = 255;
+                    cache[(((int64_t)b * Hk + h) * max_seq + p0 + t) * D + d] = (uint8_t)v;
+                }
+        }
+    }
+    return err;
+}
+
+/*
+ * Attention over a contiguous INT8 cache with per-head / per-channel scales
+ * (k-hat = (byte - 128) * s[channel or 0], one fp32 multiply), in fp64: T
+ * queries per (sequence, q head), causal from the chunk's end, with an
+ * optional sliding window (window 0: none), as in oracle_fp8_attn.
+ *   k_scales, v_scales [B, Hk, NS].
+ */
+int oracle_static_attn(const uint16_t *q, int B, int Hq, int Hk, int T, int D, int gran,
+                       const uint8_t *k, const uint8_t *v, const float *k_scales,
+                       const float *v_scales, int max_seq, const int32_t *seq_lens, int window,
+                       double attn_scale, double *out) {
+    int err = 0, G = Hq / Hk, ns = gran == 1 ? 1 : D;
+    double *z = NULL, *kh = (double *)malloc(sizeof(double) * D);
+    double *acc = (double *)malloc(sizeof(double) * D);
+    for (int b = 0; b < B; ++b) {
+        int64_t L = seq_lens[b];
+        if (L < 0 || L > max_seq || (L > 0 && L < T)) { err |= ORACLE_ERR_LEN; L = 0; }
+        z = (double *)realloc(z, sizeof(double) * (L > 0 ? L : 1));
+        for (int h = 0; h < Hq; ++h) {
+            int hk = h / G;
+            const float *sk = k_scales + ((int64_t)b * Hk + hk) * ns;
+            const float *sv = v_scales + ((int64_t)b * Hk + hk) * ns;
+            for (int i = 0; i < T; ++i) {
+                double *o = out + (((int64_t)b * Hq + h) * T + i) * D;
+                if (L == 0) { for (int d = 0; d < D; ++d) o[d] = 0.0; continue; }
+                const uint16_t *qh = q + (((int64_t)b * Hq + h) * T + i) * D;
+                int64_t p = L - T + i;
+                int64_t first = window > 0 ? p - window + 1 : 0;
+                if (first < 0) first = 0;
+                double zmax = -INFINITY;
+                for (int64_t t = first; t <= p; ++t) {
+                    int64_t row = ((int64_t)b * Hk + hk) * max_seq + t;
+                    for (int d = 0; d < D; ++d)
+                        kh[d] = (double)((float)((int)k[row * D + d] - 128) * sk[ns > 1 ? d : 0]);
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += (double)widen_bf16(qh[d]) * kh[d];
+                    z[t] = dot * attn_scale;
+                    if (z[t] > zmax) zmax = z[t];
+                }
+                double l = 0.0;
+                for (int d = 0; d < D; ++d) acc[d] = 0.0;
+                for (int64_t t = first; t <= p; ++t) {
+                    int64_t row = ((int64_t)b * Hk + hk) * max_seq + t;
+                    double e = exp(z[t] - zmax);
+                    l += e;
+                    for (int d = 0; d < D; ++d)
+                        acc[d] += e * (double)((float)((int)v[row * D + d] - 128) * sv[ns > 1 ? d : 0]);
+                }
+                for (int d = 0; d < D; ++d) o[d] = acc[d] / l;
+            }
+        }
+    }
+    free(z); free(kh); free(acc);
+    return err;
+}
+
+/* INT8 value of byte q at (row, d) for the INT8 modes of the mixed cache:
+ * mode 0 per token (scales [rows]), 1 group-32 ([rows, D/32]), 3 per head and
+ * 4 per channel (static scales of the (sequence, kv head): 1 or D floats). */
+static float mixed_int8_value(int mode, const uint8_t *q, const float *scales, int64_t row,
+                              int64_t unit, int D, int d) {
+    float s;
+    if (mode == 0) s = scales[row];
+    else if (mode == 1) s = scales[row * (D / 32) + d / 32];
+    else if (mode == 3) s = scales[unit];
+    else s = scales[unit * D + d];
+    return (float)((int)q[row * D + d] - 128) * s;
+}
+
+/*
+ * Mixed cache (abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
+ * DynamicQuantConfig::unquantized_window, OptimizedQuantizedKvCache::append
+ * and get_kv): the newest W tokens of a sequence stay unquantised (bf16) and
+ * the older ones are INT8.  An append adds the new tokens to the recent
+ * window; when the window holds more than W tokens the oldest ones are
+ * quantised (per the cache's INT8 mode) and move to the INT8 part, so after
+ * any append the INT8 part holds positions 0 .. L - W - 1 and the window the
+ * last min(L, W).  Layout: the INT8 part is a contiguous cache [B, Hk,
+ * max_seq, D] with its scales (mode 0: [B, Hk, max_seq, 1]; 1: [B, Hk,
+ * max_seq, D/32]; 3 / 4: static [B, Hk, 1 or D], read, set earlier by a
+ * calibrating call); the window is a ring [B, Hk, W, D] of bf16 in which
+ * position g sits in row g % W.
+ *   x_new [B, Hk, T, D]; lens_old [B] = L before the append.
+ */
+int oracle_append_mixed(const uint16_t *x_new, int B, int Hk, int T, int D, int mode,
+                        const int32_t *lens_old, uint8_t *cache, float *scales,
+                        uint16_t *ring, int W, int max_seq) {
+    int err = 0, ng = mode == 1 ? D / 32 : 1, ns = mode == 4 ? D : 1;
+    for (int b = 0; b < B; ++b) {
+        int64_t L0 = lens_old[b], L1 = L0 + T;
+        if (L0 < 0 || L1 > max_seq) { err |= ORACLE_ERR_POS; continue; }
+        int64_t q0 = L0 > W ? L0 - W : 0;                  /* INT8 part before */
+        int64_t q1 = L1 > W ? L1 - W : 0;                  /* and after */
+        for (int h = 0; h < Hk; ++h) {
+            int64_t unit = (int64_t)b * Hk + h;
+            /* quantise positions q0 .. q1 - 1, oldest first, from the window
+             * (older than this call) or from the new tokens */
+            for (int64_t g = q0; g < q1; ++g) {
+                const uint16_t *src = g < L0 ? ring + (unit * W + g % W) * D
+                                             : x_new + (unit * T + (g - L0)) * D;
+                int64_t row = unit * max_seq + g;
+                if (mode == 0 || mode == 1) {
+                    oracle_quantize_rows(src, 1, D, mode == 0 ? D : 32, cache + row * D,
+                                         scales + row * ng);
+                } else {
+                    const float *s = scales + unit * ns;
+                    for (int d = 0; d < D; ++d) {
+                        float r = widen_bf16(src[d]) / s[ns > 1 ? d : 0];
+                        int v = (int)roundf(r) + 128;
+                        if (v < 0) v = 0;
+                        if (v > 255) v = 255;
+                        cache[row * D + d] = (uint8_t)v;
+                    }
+                }
+            }
+            /* the new tokens that stay in the window */
+            for (int64_t g = (q1 > L0 ? q1 : L0); g < L1; ++g)
+                memcpy(ring + (unit * W + g % W) * D, x_new + (unit * T + (g - L0)) * D,
+                       sizeof(uint16_t) * D);
+        }
+    }
+    return err;
+}
+
+/*
+ * Decode attention over a mixed cache in fp64 (one query per (sequence, q
+ * head) at the newest position, no mask): positions 0 .. L - W - 1 from the
+ * INT8 part (dequantised per mode), the rest from the bf16 window ring.
+ */
+int oracle_mixed_attn(const uint16_t *q, int B, int Hq, int Hk, int D, int mode,
+                      const uint8_t *k, const uint8_t *v, const float *k_scales,
+                      const float *v_scales, const uint16_t *rk, const uint16_t *rv, int W,
+                      int max_seq, const int32_t *seq_lens, double attn_scale, double *out) {
+    int err = 0, G = Hq / Hk;
+    double *z = NULL, *kh = (double *)malloc(sizeof(double) * D);
+    double *acc = (double *)malloc(sizeof(double) * D);
+    for (int b = 0; b < B; ++b) {
+        int64_t L = seq_lens[b];
+        if (L < 0 || L > max_seq) { err |= ORACLE_ERR_LEN; L = 0; }
+        int64_t Lq = L > W ? L - W : 0;
+        z = (double *)realloc(z, sizeof(double) * (L > 0 ? L : 1));
+        for (int h = 0; h < Hq; ++h) {
+            int hk = h / G;
+            int64_t unit = (int64_t)b * Hk + hk;
+            double *o = out + ((int64_t)b * Hq + h) * D;
+            if (L == 0) { for (int d = 0; d < D; ++d) o[d] = 0.0; continue; }
+            const uint16_t *qh = q + ((int64_t)b * Hq + h) * D;
+            double zmax = -INFINITY;
+            for (int64_t t = 0; t < L; ++t) {
+                for (int d = 0; d < D; ++d)
+                    kh[d] = t < Lq ? (double)mixed_int8_value(mode, k, k_scales,
+                                                              unit * max_seq + t, unit, D, d)
+                                   : (double)widen_bf16(rk[(unit * W + t % W) * D + d]);
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += (double)widen_bf16(qh[d]) * kh[d];
+                z[t] = dot * attn_scale;
+                if (z[t] > zmax) zmax = z[t];
+            }
+            double l = 0.0;
+            for (int d = 0; d < D; ++d) acc[d] = 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                double e = exp(z[t] - zmax);
+                l += e;
+                for (int d = 0; d < D; ++d)
+                    acc[d] += e * (t < Lq ? (double)mixed_int8_value(mode, v, v_scales,
+                                                                     unit * max_seq + t, unit, D, d)
+                                          : (double)widen_bf16(rv[(unit * W + t % W) * D + d]));
+            }
+            for (int d = 0; d < D; ++d) o[d] = acc[d] / l;
+        }
+    }
+    free(z); free(kh); free(acc);
+    return err;
+}
