@@ -34,13 +34,15 @@ PER_TOKEN = 0
 GROUP32 = 1
 FP8_E4M3 = 2
 FP8_E5M2 = 3
+PER_HEAD = 4
+PER_CHANNEL = 5
 DEVERR_POS = 1
 DEVERR_PAGE = 2
 DEVERR_LEN = 4
 
 _MODES = {"per_token": PER_TOKEN, "group32": GROUP32, "fp8_e4m3": FP8_E4M3,
-          "fp8_e5m2": FP8_E5M2, PER_TOKEN: PER_TOKEN, GROUP32: GROUP32, FP8_E4M3: FP8_E4M3,
-          FP8_E5M2: FP8_E5M2}
+          "fp8_e5m2": FP8_E5M2, "per_head": PER_HEAD, "per_channel": PER_CHANNEL}
+_MODES.update({v: v for v in list(_MODES.values())})
 
 
 class CacheView(ctypes.Structure):
@@ -94,9 +96,17 @@ def _stream(stream, ref: torch.Tensor) -> int:
 
 
 def num_groups(mode, D: int) -> int:
-    """Scales per (token, kv head): 1 per token, D / 32 for group-32, 0 for FP8."""
+    """Scales per (token, kv head): 1 per token, D / 32 for group-32, 0 for FP8
+    and for the per-head / per-channel modes (whose scales are per (sequence,
+    kv head): see static_scales)."""
     m = _mode(mode)
     return 1 if m == PER_TOKEN else (D // 32 if m == GROUP32 else 0)
+
+
+def static_scales(mode, D: int) -> int:
+    """Scales per (sequence, kv head) of the per-head (1) / per-channel (D) modes."""
+    m = _mode(mode)
+    return 1 if m == PER_HEAD else (D if m == PER_CHANNEL else 0)
 
 
 def kvq_append(k_new, v_new, pos, k_cache, v_cache, k_scale, v_scale, mode="per_token",
@@ -114,6 +124,21 @@ def kvq_append(k_new, v_new, pos, k_cache, v_cache, k_scale, v_scale, mode="per_
         _ptr(k_cache, torch.uint8, "k_cache"), _ptr(v_cache, torch.uint8, "v_cache"),
         _ptr(k_scale, torch.float32, "k_scale"), _ptr(v_scale, torch.float32, "v_scale"),
         k_cache.shape[2], _ptr(err, torch.int32, "err"), _stream(stream, k_new)), "kvq_append")
+
+
+def kvq_append_calibrate(k_new, v_new, pos, k_cache, v_cache, k_scale, v_scale,
+                         mode="per_head", err=None, stream=None):
+    """Per-head / per-channel quantisation of k_new/v_new bf16 [B,Hk,T,D] into
+    the contiguous cache at pos[b], with the scales (fp32 [B,Hk,1] or
+    [B,Hk,D]) first computed from these tokens."""
+    B, Hk, T, D = k_new.shape
+    check(lib.kvq_append_calibrate(
+        _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        B, Hk, T, D, _mode(mode), _ptr(pos, torch.int32, "pos"),
+        _ptr(k_cache, torch.uint8, "k_cache"), _ptr(v_cache, torch.uint8, "v_cache"),
+        _ptr(k_scale, torch.float32, "k_scale"), _ptr(v_scale, torch.float32, "v_scale"),
+        k_cache.shape[2], _ptr(err, torch.int32, "err"), _stream(stream, k_new)),
+        "kvq_append_calibrate")
 
 
 def kvq_append_paged(k_new, v_new, pos, k_arena, v_arena, k_scale, v_scale, page_table,
@@ -270,6 +295,49 @@ def kvq_window_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, windo
         _ptr(seq_lens, torch.int32, "seq_lens"), int(max_seq_len_hint), int(window),
         float(attn_scale), _ptr(out, torch.float32, "out"), ws_ptr, ws_bytes, int(num_splits),
         _ptr(err, torch.int32, "err"), _stream(stream, q)), "kvq_window_attn")
+    return out
+
+
+def kvq_append_mixed(k_new, v_new, lens_old, k_cache, v_cache, k_scale, v_scale, k_ring,
+                     v_ring, mode="per_token", err=None, stream=None):
+    """Mixed cache append: k_new/v_new bf16 [B,Hk,T,D] join the bf16 window
+    rings [B,Hk,W,D]; tokens leaving the window are quantised into the INT8
+    part (k_cache [B,Hk,max_seq,D] and its scales).  lens_old int32 [B]."""
+    B, Hk, T, D = k_new.shape
+    check(lib.kvq_append_mixed(
+        _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        B, Hk, T, D, _mode(mode), _ptr(lens_old, torch.int32, "lens_old"),
+        _ptr(k_cache, torch.uint8, "k_cache"), _ptr(v_cache, torch.uint8, "v_cache"),
+        _ptr(k_scale, torch.float32, "k_scale"), _ptr(v_scale, torch.float32, "v_scale"),
+        k_cache.shape[2], _ptr(k_ring, torch.bfloat16, "k_ring"),
+        _ptr(v_ring, torch.bfloat16, "v_ring"), k_ring.shape[2], _ptr(err, torch.int32, "err"),
+        _stream(stream, k_new)), "kvq_append_mixed")
+
+
+def kvq_decode_attn_mixed(q, k, v, k_scale, v_scale, k_ring, v_ring, seq_lens, max_seq_len_hint,
+                          *, mode="per_token", attn_scale=None, out=None, workspace=None,
+                          num_splits=0, err=None, stream=None, page_table=None, page_size=0):
+    """Decode attention over a mixed cache (INT8 part + bf16 window rings
+    [B,Hk,W,D]); seq_lens counts every token.  Returns fp32 [B,Hq,D]."""
+    B, Hq, D = q.shape
+    Hk = k.shape[1]
+    W = k_ring.shape[2]
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    view = cache_view(k, v, k_scale, v_scale, page_table, page_size)
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = int(lib.kvq_mixed_workspace_bytes(B, Hq, Hk, D, int(max_seq_len_hint), W,
+                                                 int(num_splits)))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    check(lib.kvq_decode_attn_mixed(
+        _ptr(q, torch.bfloat16, "q"), B, Hq, Hk, D, _mode(mode), ctypes.byref(view),
+        _ptr(k_ring, torch.bfloat16, "k_ring"), _ptr(v_ring, torch.bfloat16, "v_ring"), W,
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(max_seq_len_hint), float(attn_scale),
+        _ptr(out, torch.float32, "out"), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), int(num_splits),
+        _ptr(err, torch.int32, "err"), _stream(stream, q)), "kvq_decode_attn_mixed")
     return out
 
 

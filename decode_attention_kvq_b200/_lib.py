@@ -23,6 +23,12 @@ _PROTOS = {
     "kvq_append": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P]),
     "kvq_append_paged": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I,
                               _P, _P]),
+    "kvq_append_calibrate": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P]),
+    "kvq_append_mixed": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P, _I,
+                              _P, _P]),
+    "kvq_decode_attn_mixed": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _I, _P, _I, _F, _P, _P,
+                                   _SZ, _I, _P, _P]),
+    "kvq_mixed_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "kvq_decode_attn": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _SZ, _I, _P, _P]),
     "kvq_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "kvq_chunk_attn": (_I, [_P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _SZ, _I, _P,

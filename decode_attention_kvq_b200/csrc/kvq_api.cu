@@ -20,7 +20,12 @@ kvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR
 
 bool valid_mode(kvq_scale_mode m) {
     return m == KVQ_SCALE_PER_TOKEN || m == KVQ_SCALE_GROUP32 || m == KVQ_FP8_E4M3 ||
-           m == KVQ_FP8_E5M2;
+           m == KVQ_FP8_E5M2 || m == KVQ_SCALE_PER_HEAD || m == KVQ_SCALE_PER_CHANNEL;
+}
+bool is_static(kvq_scale_mode m) { return m == KVQ_SCALE_PER_HEAD || m == KVQ_SCALE_PER_CHANNEL; }
+// scales per (sequence, kv head) of the per-head / per-channel modes (0: per row)
+int static_ns(kvq_scale_mode m, int D) {
+    return m == KVQ_SCALE_PER_HEAD ? 1 : m == KVQ_SCALE_PER_CHANNEL ? D : 0;
 }
 bool is_fp8(kvq_scale_mode m) { return m == KVQ_FP8_E4M3 || m == KVQ_FP8_E5M2; }
 // 0: INT8 with scales, 1: E4M3, 2: E5M2 (the kernels' encoding)
@@ -36,8 +41,10 @@ kvq_status check_append_common(const uint16_t* k_new, const uint16_t* v_new, int
         return KVQ_ERR_INVALID_ARG;
     if (B < 1 || Hk < 1 || T < 1 || D < 16 || D > 256 || (D % 16) != 0) return KVQ_ERR_INVALID_ARG;
     if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
+    // per-head scales are read one float at a time: 4-byte alignment suffices
+    const uintptr_t sa = mode == KVQ_SCALE_PER_HEAD ? 4 : 16;
     if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(kd, 16) || !aligned(vd, 16) ||
-        !aligned(ks, 16) || !aligned(vs, 16) || !aligned(d_pos, 4) || !aligned(d_err, 4))
+        !aligned(ks, sa) || !aligned(vs, sa) || !aligned(d_pos, 4) || !aligned(d_err, 4))
         return KVQ_ERR_INVALID_ARG;
     return KVQ_OK;
 }
@@ -97,11 +104,18 @@ int walked_hint(int hint, int T, int window) {
     return w < hint ? static_cast<int>(w) : hint;
 }
 
+// mixed cache: split-K slots for every row even without a split (the
+// window kernel folds them)
+size_t mixed_workspace_for(int B, int Hq, int D, int splits) {
+    return static_cast<size_t>(B) * Hq * (splits > 1 ? splits : 1) * (D + 2) * sizeof(float);
+}
+
 kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_scale_mode mode,
                   const kvq_cache_view* kv, const int32_t* d_seq_lens, int max_seq_len_hint,
                   int window, float attn_scale, float* out, void* workspace,
-                  size_t workspace_bytes, int num_splits, int32_t* d_err, kvq_stream_t stream) {
-    if (window < 0) return KVQ_ERR_INVALID_ARG;
+                  size_t workspace_bytes, int num_splits, int32_t* d_err, kvq_stream_t stream,
+                  int recent = 0, const uint16_t* rk = nullptr, const uint16_t* rv = nullptr) {
+    if (window < 0 || recent < 0) return KVQ_ERR_INVALID_ARG;
     if (!valid_mode(mode)) return KVQ_ERR_INVALID_ARG;
     if (!q || !kv || !kv->k || !kv->v || !d_seq_lens || !out) return KVQ_ERR_INVALID_ARG;
     if (!is_fp8(mode) && (!kv->k_scale || !kv->v_scale)) return KVQ_ERR_INVALID_ARG;
@@ -118,8 +132,9 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
     } else {
         return KVQ_ERR_INVALID_ARG;
     }
+    const uintptr_t sa = mode == KVQ_SCALE_PER_HEAD ? 4 : 16;   // per-head: scalar reads
     if (!aligned(q, 16) || !aligned(kv->k, 16) || !aligned(kv->v, 16) ||
-        !aligned(kv->k_scale, 16) || !aligned(kv->v_scale, 16) || !aligned(d_seq_lens, 4) ||
+        !aligned(kv->k_scale, sa) || !aligned(kv->v_scale, sa) || !aligned(d_seq_lens, 4) ||
         !aligned(out, 16) || !aligned(workspace, 16) || !aligned(d_err, 4))
         return KVQ_ERR_INVALID_ARG;
     if (T > 16 || Hq > 65535) return KVQ_ERR_UNSUPPORTED;
@@ -135,12 +150,15 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
     if (B == 0) return KVQ_OK;
 
     int chunk = 0, splits = 0;
-    const int hint = walked_hint(max_seq_len_hint, T, window);
+    // (mixed cache: the split kernel walks the INT8 part, the hint less the window)
+    const int hint = recent ? (max_seq_len_hint > recent ? max_seq_len_hint - recent : 0)
+                            : walked_hint(max_seq_len_hint, T, window);
     kvq_status st = plan(B, Hk, hint, num_splits, 0, &chunk, &splits);
     if (st != KVQ_OK) return st;
     // work items (sequence, kv head, chunk) are counted in 32-bit integers
     if (static_cast<int64_t>(B) * Hk * (splits + 3) >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
-    const size_t need = workspace_for(B, Hq * T, D, splits);
+    const size_t need = recent ? mixed_workspace_for(B, Hq * T, D, splits)
+                               : workspace_for(B, Hq * T, D, splits);
     if (need > 0 && (!workspace || workspace_bytes < need)) return KVQ_ERR_INVALID_ARG;
 
     kvq::DecodeParams p{};
@@ -154,8 +172,12 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
     p.ws_l = ws ? ws + n_part * (D + 1) : nullptr;
     p.B = B; p.Hq = Hq * T; p.Hk = Hk; p.G = G; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
     p.fp8 = fp8_code(mode);
+    p.static_ns = static_ns(mode, D);
     p.qlen = T;
     p.window = window;
+    p.recent = recent;
+    p.rk = rk;
+    p.rv = rv;
     p.page_size = kv->page_size; p.max_seq = kv->max_seq; p.max_pages = kv->max_pages;
     p.num_pages = kv->num_pages; p.chunk = chunk; p.splits = splits;
     {
@@ -173,6 +195,14 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
     // for every (sequence, kv head) it starts (merge, query set-up), so each
     // unit start weighs three items when the items are divided among the CTAs
     p.seg_w = (chunk <= 128 && !p.one_item) ? 3 : 0;
+    if (recent) {                       // mixed cache: INT8 partials, then the window kernel
+        const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+        if (hint > 0) {
+            const cudaError_t e = kvq::launch_decode_split_tc(p, cs);
+            if (e != cudaSuccess) return KVQ_ERR_CUDA;
+        }
+        return from_cuda(kvq::launch_recent_combine(p, cs));
+    }
     return from_cuda(kvq::launch_decode(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -193,6 +223,7 @@ kvq_status kvq_append(const uint16_t* k_new, const uint16_t* v_new, int B, int H
     p.k_scale = k_scale; p.v_scale = v_scale; p.pos = d_pos; p.table = nullptr; p.d_err = d_err;
     p.B = B; p.Hk = Hk; p.T = T; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
     p.fp8 = fp8_code(mode);
+    p.static_ns = static_ns(mode, D);
     p.max_seq = max_seq; p.page_size = 0;
     return from_cuda(kvq::launch_append(p, static_cast<cudaStream_t>(stream)));
 }
@@ -213,9 +244,27 @@ kvq_status kvq_append_paged(const uint16_t* k_new, const uint16_t* v_new, int B,
     p.k_scale = k_scale; p.v_scale = v_scale; p.pos = d_pos; p.table = page_table;
     p.d_err = d_err; p.B = B; p.Hk = Hk; p.T = T; p.D = D;
     p.group32 = mode == KVQ_SCALE_GROUP32; p.fp8 = fp8_code(mode);
+    p.static_ns = static_ns(mode, D);
     p.max_seq = 0; p.page_size = page_size;
     p.max_pages = max_pages; p.num_pages = num_pages;
     return from_cuda(kvq::launch_append(p, static_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_append_calibrate(const uint16_t* k_new, const uint16_t* v_new, int B, int Hk,
+                                int T, int D, kvq_scale_mode mode, const int32_t* d_pos,
+                                uint8_t* k_cache, uint8_t* v_cache, float* k_scale,
+                                float* v_scale, int max_seq, int32_t* d_err, kvq_stream_t stream) {
+    if (!is_static(mode)) return KVQ_ERR_INVALID_ARG;
+    kvq_status st = check_append_common(k_new, v_new, B, Hk, T, D, mode, d_pos, k_cache, v_cache,
+                                        k_scale, v_scale, d_err);
+    if (st != KVQ_OK) return st;
+    if (max_seq < 1) return KVQ_ERR_INVALID_ARG;
+    kvq::AppendParams p{};
+    p.k_new = k_new; p.v_new = v_new; p.k_dst = k_cache; p.v_dst = v_cache;
+    p.k_scale = k_scale; p.v_scale = v_scale; p.pos = d_pos; p.table = nullptr; p.d_err = d_err;
+    p.B = B; p.Hk = Hk; p.T = T; p.D = D; p.static_ns = static_ns(mode, D);
+    p.max_seq = max_seq; p.page_size = 0;
+    return from_cuda(kvq::launch_append_calibrate(p, static_cast<cudaStream_t>(stream)));
 }
 
 kvq_status kvq_decode_plan(int B, int Hk, int max_seq_len_hint, int num_splits, int num_sms,
@@ -251,6 +300,53 @@ kvq_status kvq_chunk_attn(const uint16_t* q, int B, int Hq, int Hk, int T, int D
                   workspace, workspace_bytes, num_splits, d_err, stream);
 }
 
+kvq_status kvq_append_mixed(const uint16_t* k_new, const uint16_t* v_new, int B, int Hk, int T,
+                            int D, kvq_scale_mode mode, const int32_t* d_lens_old,
+                            uint8_t* k_cache, uint8_t* v_cache, float* k_scale, float* v_scale,
+                            int max_seq, uint16_t* k_ring, uint16_t* v_ring, int window,
+                            int32_t* d_err, kvq_stream_t stream) {
+    if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32 && !is_static(mode))
+        return KVQ_ERR_INVALID_ARG;
+    kvq_status st = check_append_common(k_new, v_new, B, Hk, T, D, mode, d_lens_old, k_cache,
+                                        v_cache, k_scale, v_scale, d_err);
+    if (st != KVQ_OK) return st;
+    if (max_seq < 1 || window < 1 || window > kvq::kMaxRecent || !k_ring || !v_ring ||
+        !aligned(k_ring, 16) || !aligned(v_ring, 16))
+        return KVQ_ERR_INVALID_ARG;
+    kvq::AppendParams p{};
+    p.k_new = k_new; p.v_new = v_new; p.k_dst = k_cache; p.v_dst = v_cache;
+    p.k_scale = k_scale; p.v_scale = v_scale; p.pos = d_lens_old; p.table = nullptr;
+    p.d_err = d_err; p.B = B; p.Hk = Hk; p.T = T; p.D = D;
+    p.group32 = mode == KVQ_SCALE_GROUP32; p.static_ns = static_ns(mode, D);
+    p.max_seq = max_seq; p.page_size = 0;
+    return from_cuda(kvq::launch_append_mixed(p, k_ring, v_ring, window,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_decode_attn_mixed(const uint16_t* q, int B, int Hq, int Hk, int D,
+                                 kvq_scale_mode mode, const kvq_cache_view* kv,
+                                 const uint16_t* k_ring, const uint16_t* v_ring, int window,
+                                 const int32_t* d_seq_lens, int max_seq_len_hint,
+                                 float attn_scale, float* out, void* workspace,
+                                 size_t workspace_bytes, int num_splits, int32_t* d_err,
+                                 kvq_stream_t stream) {
+    if (window < 1 || window > kvq::kMaxRecent || !k_ring || !v_ring || !aligned(k_ring, 16) ||
+        !aligned(v_ring, 16))
+        return KVQ_ERR_INVALID_ARG;
+    if (B > 0 && !workspace) return KVQ_ERR_INVALID_ARG;
+    return attend(q, B, Hq, Hk, 1, D, mode, kv, d_seq_lens, max_seq_len_hint, 0, attn_scale, out,
+                  workspace, workspace_bytes, num_splits, d_err, stream, window, k_ring, v_ring);
+}
+
+size_t kvq_mixed_workspace_bytes(int B, int Hq, int Hk, int D, int max_seq_len_hint, int window,
+                                 int num_splits) {
+    int chunk = 0, splits = 0;
+    if (B < 1 || Hq < 1 || D < 1 || window < 1) return 0;
+    const int hint = max_seq_len_hint > window ? max_seq_len_hint - window : 0;
+    if (plan(B, Hk, hint, num_splits, 0, &chunk, &splits) != KVQ_OK) return 0;
+    return mixed_workspace_for(B, Hq, D, splits);
+}
+
 kvq_status kvq_window_attn(const uint16_t* q, int B, int Hq, int Hk, int T, int D,
                            kvq_scale_mode mode, const kvq_cache_view* kv,
                            const int32_t* d_seq_lens, int max_seq_len_hint, int window,
@@ -281,10 +377,11 @@ kvq_status kvq_dequant(const uint8_t* q, const float* scale, int64_t rows, int D
     if (mode == KVQ_SCALE_GROUP32 && (D % 32) != 0) return KVQ_ERR_INVALID_ARG;
     if (rows == 0) return KVQ_OK;
     if (!q || (!scale && !is_fp8(mode)) || !out || !aligned(q, 16) || !aligned(out, 16) ||
-        !aligned(scale, 16))
+        !aligned(scale, mode == KVQ_SCALE_PER_HEAD ? 4 : 16))
         return KVQ_ERR_INVALID_ARG;
     return from_cuda(kvq::launch_dequant(q, scale, rows, D, mode == KVQ_SCALE_GROUP32,
-                                         fp8_code(mode), out, static_cast<cudaStream_t>(stream)));
+                                         fp8_code(mode), static_ns(mode, D), out,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 const char* kvq_status_string(kvq_status status) {
@@ -315,7 +412,8 @@ kvq_status kvq_read_error(int32_t* d_err, int32_t* bits, kvq_stream_t stream) {
 }
 
 int64_t kvq_cache_bytes(int64_t layers, int64_t Hk, int64_t seq, int D, kvq_scale_mode mode) {
-    const int64_t ng = mode == KVQ_SCALE_GROUP32 ? D / 32 : is_fp8(mode) ? 0 : 1;
+    // per-head / per-channel scales are per (sequence, kv head), not per token
+    const int64_t ng = mode == KVQ_SCALE_GROUP32 ? D / 32 : (is_fp8(mode) || is_static(mode)) ? 0 : 1;
     return layers * 2 * Hk * seq * (static_cast<int64_t>(D) + 4 * ng);
 }
 

@@ -104,6 +104,22 @@ append_kernel(AppendParams p, int lanes_log2) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
     }
+    if (p.static_ns) {                           // per head / per channel: stored scales
+        if (!active || dst_row < 0) return;
+        const float* sc = (which ? p.v_scale : p.k_scale) +
+                          (static_cast<int64_t>(b) * p.Hk + h) * p.static_ns;
+        uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float si = sc[p.static_ns > 1 ? sub * 8 + i : 0];
+            int v = static_cast<int>(roundf(__fdiv_rn(x[i], si))) + 128;
+            v = v < 0 ? 0 : (v > 255 ? 255 : v);
+            packed[i >> 2] |= static_cast<uint32_t>(v) << (8 * (i & 3));
+        }
+        uint8_t* dst = (which ? p.v_dst : p.k_dst) + dst_row * p.D + sub * 8;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+        return;
+    }
     // reduce inside the group of lanes sharing one scale
     const int red_lanes = p.group32 ? 4 : P;
     for (int off = 1; off < red_lanes; off <<= 1)
@@ -129,7 +145,190 @@ append_kernel(AppendParams p, int lanes_log2) {
     }
 }
 
+// Per-head / per-channel calibration (abaddon 0.2.0-rc.1,
+// OptimizedQuantizedKvCache::quantize_with_granularity), contiguous caches:
+// one CTA per (K or V, b, h).  Thread (c, r) owns channel c and the tokens
+// t = r (mod lanes); the maxima are reduced through shared memory (over the
+// token lanes per channel, or over everything per head), the scales written,
+// then the same threads quantise their tokens with them.
+constexpr int kCalThreads = 256;
+__global__ void __launch_bounds__(kCalThreads)
+calibrate_kernel(AppendParams p) {
+    grid_dep_wait();
+    grid_dep_launch();
+    __shared__ float red[kCalThreads];
+    __shared__ float scl[256];
+    const int units = p.B * p.Hk;
+    const int which = blockIdx.x / units;
+    const int bh = blockIdx.x % units;
+    const int b = bh / p.Hk;
+    const int D = p.D, T = p.T, tid = threadIdx.x;
+    const int lanes = kCalThreads / D;           // token lanes per channel (D <= 256)
+    const int c = tid % D, r = tid / D;
+    const bool act = r < lanes;
+    const int64_t p0 = p.pos[b];
+    if (p0 < 0 || p0 + T > p.max_seq) {          // the whole unit is skipped
+        if (tid == 0 && which == 0 && bh % p.Hk == 0) raise_flag(p.d_err, KVQ_DEVERR_POS);
+        return;
+    }
+    const uint16_t* x = (which ? p.v_new : p.k_new) + static_cast<int64_t>(bh) * T * D;
+    float m = 0.f;
+    if (act)
+        for (int t = r; t < T; t += lanes)
+            m = fmaxf(m, fabsf(bf16_bits_to_f32(x[static_cast<int64_t>(t) * D + c])));
+    red[tid] = m;
+    __syncthreads();
+    float* sc = (which ? p.v_scale : p.k_scale) + static_cast<int64_t>(bh) * p.static_ns;
+    if (p.static_ns > 1) {                       // per channel: over the token lanes
+        if (act && r == 0) {
+            for (int k = 1; k < lanes; ++k) m = fmaxf(m, red[k * D + c]);
+            const float s = __fdiv_rn(m < 1e-8f ? 1e-8f : m, 127.0f);
+            scl[c] = s;
+            sc[c] = s;
+        }
+    } else {                                     // per head: over every thread
+        for (int off = kCalThreads / 2; off > 0; off >>= 1) {
+            if (tid < off) red[tid] = fmaxf(red[tid], red[tid + off]);
+            __syncthreads();
+        }
+        if (tid == 0) {
+            const float s = __fdiv_rn(red[0] < 1e-8f ? 1e-8f : red[0], 127.0f);
+            scl[0] = s;
+            sc[0] = s;
+        }
+    }
+    __syncthreads();
+    if (!act) return;
+    const float s = scl[p.static_ns > 1 ? c : 0];
+    uint8_t* dst = (which ? p.v_dst : p.k_dst) + (static_cast<int64_t>(bh) * p.max_seq + p0) * D;
+    for (int t = r; t < T; t += lanes) {
+        const float xv = bf16_bits_to_f32(x[static_cast<int64_t>(t) * D + c]);
+        int v = static_cast<int>(roundf(__fdiv_rn(xv, s))) + 128;
+        v = v < 0 ? 0 : (v > 255 ? 255 : v);
+        dst[static_cast<int64_t>(t) * D + c] = static_cast<uint8_t>(v);
+    }
+}
+
+// Mixed cache append (abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
+// OptimizedQuantizedKvCache::append): one CTA per (K or V, b, h).  With the
+// old length L0 and the new L1 = L0 + T, the window keeps the last W tokens,
+// so positions max(0, L0 - W) .. max(0, L1 - W) - 1 leave it: first each of
+// them is quantised into the INT8 part (a warp per position: from the ring
+// if it was appended earlier, else from the new tokens), then, behind a
+// barrier (a new token can land in the ring row an old one is read from),
+// the new tokens that stay are copied into the ring (row g % W).
+__global__ void __launch_bounds__(kAppendThreads)
+append_mixed_kernel(AppendParams p, uint16_t* k_ring, uint16_t* v_ring, int W) {
+    grid_dep_wait();
+    grid_dep_launch();
+    const int units = p.B * p.Hk;
+    const int which = blockIdx.x / units;
+    const int bh = blockIdx.x % units;
+    const int b = bh / p.Hk;
+    const int D = p.D, T = p.T;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t L0 = p.pos[b], L1 = L0 + T;
+    const int64_t q0 = L0 > W ? L0 - W : 0, q1 = L1 > W ? L1 - W : 0;
+    if (L0 < 0 || q1 > p.max_seq) {
+        if (threadIdx.x == 0 && which == 0 && bh % p.Hk == 0) raise_flag(p.d_err, KVQ_DEVERR_POS);
+        return;
+    }
+    const uint16_t* x = (which ? p.v_new : p.k_new) + static_cast<int64_t>(bh) * T * D;
+    uint16_t* ring = (which ? v_ring : k_ring) + static_cast<int64_t>(bh) * W * D;
+    uint8_t* dst = (which ? p.v_dst : p.k_dst) + static_cast<int64_t>(bh) * p.max_seq * D;
+    float* sdst = which ? p.v_scale : p.k_scale;
+    const int nvec = D >> 3;
+    const bool act = lane < nvec;
+    for (int64_t g = q0 + warp; g < q1; g += kAppendThreads / 32) {
+        const uint16_t* src = g < L0 ? ring + (g % W) * D : x + (g - L0) * D;
+        float xv[8];
+        float amax = 0.f;
+        if (act) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(src + lane * 8);
+            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                xv[2 * i] = bf16_bits_to_f32(w4[i] & 0xffffu);
+                xv[2 * i + 1] = bf16_bits_to_f32(w4[i] >> 16);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(xv[i]));
+        }
+        float sc[8];
+        if (p.static_ns) {                        // stored per-head / per-channel scales
+            const float* st = sdst + static_cast<int64_t>(bh) * p.static_ns;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sc[i] = act ? st[p.static_ns > 1 ? lane * 8 + i : 0] : 1.f;
+        } else {                                  // per token or per 32-value group
+            const int red = p.group32 ? 4 : 32;
+            for (int off = 1; off < red; off <<= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            const float s = __fdiv_rn(amax < 1e-8f ? 1e-8f : amax, 127.0f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sc[i] = s;
+            if (act) {
+                const int64_t row = static_cast<int64_t>(bh) * p.max_seq + g;
+                if (p.group32) {
+                    if ((lane & 3) == 0) sdst[row * (D >> 5) + (lane >> 2)] = s;
+                } else if (lane == 0) {
+                    sdst[row] = s;
+                }
+            }
+        }
+        if (act) {
+            uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                int v = static_cast<int>(roundf(__fdiv_rn(xv[i], sc[i]))) + 128;
+                v = v < 0 ? 0 : (v > 255 ? 255 : v);
+                packed[i >> 2] |= static_cast<uint32_t>(v) << (8 * (i & 3));
+            }
+            *reinterpret_cast<uint2*>(dst + g * D + lane * 8) = make_uint2(packed[0], packed[1]);
+        }
+    }
+    __syncthreads();
+    const int64_t g0 = q1 > L0 ? q1 : L0;         // the new tokens that stay in the window
+    for (int64_t i = threadIdx.x; i < (L1 - g0) * nvec; i += kAppendThreads) {
+        const int64_t g = g0 + i / nvec;
+        const int c = static_cast<int>(i % nvec);
+        *reinterpret_cast<uint4*>(ring + (g % W) * D + c * 8) =
+            *reinterpret_cast<const uint4*>(x + (g - L0) * D + c * 8);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_append_mixed(const AppendParams& p, uint16_t* k_ring, uint16_t* v_ring, int W,
+                                cudaStream_t s) {
+    const int64_t blocks = 2ll * p.B * p.Hk;
+    if (blocks > 0x7fffffffll || W < 1 || p.D > 256) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    cfg.blockDim = dim3(kAppendThreads, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, append_mixed_kernel, p, k_ring, v_ring, W);
+}
+
+cudaError_t launch_append_calibrate(const AppendParams& p, cudaStream_t s) {
+    if (p.D > 256 || p.D < 1) return cudaErrorInvalidValue;
+    const int64_t blocks = 2ll * p.B * p.Hk;
+    if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    cfg.blockDim = dim3(kCalThreads, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, calibrate_kernel, p);
+}
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
     const int nvec = p.D >> 3;

@@ -117,7 +117,7 @@ decode_combine_one(DecodeParams p) {
     };
     // the first round of loads is issued together with the length
     load(w);
-    const int L = max(walked_len(L0, cap, plan, p.qlen, p.window), 0);
+    const int L = max(walked_len(L0, cap, plan, p.qlen, p.window, p.recent), 0);
     const int ns = (L + p.chunk - 1) / p.chunk;
     if (ns <= 1) return;                        // finished by the split kernel
     fold(w, ns);
@@ -158,7 +158,7 @@ decode_combine_live(DecodeParams p) {
         const int j = 32 * x + lane;
         mv0[x] = j < p.splits ? m[j] : -INFINITY;
     }
-    const int L = max(walked_len(L0, cap, plan, p.qlen, p.window), 0);
+    const int L = max(walked_len(L0, cap, plan, p.qlen, p.window, p.recent), 0);
     const int ns = (L + p.chunk - 1) / p.chunk;
     if (ns <= 1) return;                        // finished by the split kernel
 
@@ -253,6 +253,95 @@ size_t combine_one_spread_smem(int rows) {
 }
 
 }  // namespace
+
+// Mixed cache (abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
+// OptimizedQuantizedKvCache::get_kv: the INT8 part dequantised, then the
+// unquantised recent tokens): one CTA per (b, q head).  The newest
+// min(L, W) tokens sit in the bf16 ring (position g in row g % W); their
+// partial (m, l, o) is computed here in fp32 from the bf16 values, then
+// folded with the split kernel's INT8 partials (every slot below the INT8
+// part's chunk count with a finite m) into the output row.
+__global__ void __launch_bounds__(kThreads)
+decode_recent_combine(DecodeParams p) {
+    __shared__ float s_z[kMaxRecent];   // the window's scores
+    __shared__ float s_red[kWarps];
+    grid_dep_wait();                    // the split kernel's partials are complete
+    grid_dep_launch();
+    const int64_t bh = blockIdx.x;
+    const int b = static_cast<int>(bh / p.Hq);
+    const int h = static_cast<int>(bh % p.Hq);
+    const int hk = h / p.G;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int D = p.D, W = p.recent;
+    float* out = p.out + bh * D;
+    const int64_t cap = p.page_size ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
+    const int64_t plan = static_cast<int64_t>(p.splits) * p.chunk;
+    const int L = p.seq_lens[b];
+    const int n8 = walked_len(L, cap, plan, 1, 0, W);   // INT8 part walked by the split kernel
+    if (n8 < 0) {                                       // flagged by the split kernel
+        for (int d = tid; d < D; d += kThreads) out[d] = 0.f;
+        return;
+    }
+    const int Lq = L > W ? L - W : 0;
+    const int nr = L - Lq;                              // tokens in the window
+    const uint16_t* qh = p.q + bh * D;
+    const int64_t ring0 = (static_cast<int64_t>(b) * p.Hk + hk) * W;
+    // ---- window scores (log2 domain), one warp per token, lanes over head_dim
+    float mloc = -INFINITY;
+    for (int i = w; i < nr; i += kWarps) {
+        const uint16_t* kr = p.rk + (ring0 + (Lq + i) % W) * D;
+        float dot = 0.f;
+        for (int d = lane; d < D; d += 32)
+            dot = fmaf(bf16_bits_to_f32(qh[d]), bf16_bits_to_f32(kr[d]), dot);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        const float z = dot * p.scale_log2;
+        if (lane == 0) s_z[i] = z;
+        mloc = fmaxf(mloc, z);
+    }
+    if (lane == 0) s_red[w] = mloc;
+    __syncthreads();
+    float mr = -INFINITY;
+#pragma unroll
+    for (int x = 0; x < kWarps; ++x) mr = fmaxf(mr, s_red[x]);
+    // ---- INT8 partials: the running max over them and the window
+    const int ns = (n8 + p.chunk - 1) / p.chunk;
+    const float* m8 = p.ws_m + bh * p.splits;
+    const float* l8 = p.ws_l + bh * p.splits;
+    float M = mr;
+    for (int j = 0; j < ns; ++j) M = fmaxf(M, m8[j]);
+    // ---- each thread: its head_dim values of the weighted sums
+    float lsum = 0.f;
+    for (int i = 0; i < nr; ++i) lsum += exp2f(s_z[i] - M);
+    for (int j = 0; j < ns; ++j)
+        if (m8[j] != -INFINITY) lsum = fmaf(exp2f(m8[j] - M), l8[j], lsum);
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    for (int d = tid; d < D; d += kThreads) {
+        float acc = 0.f;
+        for (int i = 0; i < nr; ++i) {
+            const uint16_t* vr = p.rv + (ring0 + (Lq + i) % W) * D;
+            acc = fmaf(exp2f(s_z[i] - M), bf16_bits_to_f32(vr[d]), acc);
+        }
+        for (int j = 0; j < ns; ++j)
+            if (m8[j] != -INFINITY)
+                acc = fmaf(exp2f(m8[j] - M), p.ws_o[(bh * p.splits + j) * D + d], acc);
+        out[d] = acc * inv;
+    }
+}
+
+cudaError_t launch_recent_combine(const DecodeParams& p, cudaStream_t s) {
+    if (p.recent < 1 || p.recent > kMaxRecent) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.B * p.Hq, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_recent_combine, p);
+}
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
     cudaError_t e = launch_decode_split_tc(p, s);

@@ -261,7 +261,7 @@ __device__ __forceinline__ Seg seg_at(int i, int iend, const int* lens, const in
 // column i of a sequence of length L sees the positions <= L - T + i (L
 // counts the chunk's tokens) and, with a window w, >= L - T + i - w + 1.
 // With a window the tokens are counted from the sequence's window base.
-template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8>
+template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8, bool ST>
 __global__ void __launch_bounds__(nthreads(PAGED), 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ DecodeParams prm) {
@@ -276,6 +276,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     static_assert(!PK || (G32 && !G16), "packing: group-32 scales, at most 4 heads");
     static_assert(!(PK && CAUSAL), "chunk queries: unpacked columns");
     static_assert(F8 == 0 || !G32, "FP8 caches have no scales");
+    static_assert(!ST || (F8 == 0 && !G32), "per-head / per-channel scales: INT8, no groups");
+    // no scale rows in the ring: FP8 (no scales) and per-head / per-channel
+    // scales (one set per (sequence, kv head), folded into Q and the output)
+    constexpr bool NOSC = F8 != 0 || ST;
     constexpr int NVS = PK ? NGRP / 2 : NGV;   // P'' operand sets (PK: group pairs)
 
     extern __shared__ uint8_t smem_raw[];
@@ -355,7 +359,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                                    static_cast<int64_t>(prm.B) * prm.Hk * prm.max_seq * Lay::NG) &
                                ~static_cast<int64_t>(3);
             const int64_t a0 = f0 & ~static_cast<int64_t>(3);
-            if (F8 == 0 && f1 > a0) {
+            if (!NOSC && f1 > a0) {
                 ptx::prefetch_l2(prm.k_scale + a0, static_cast<uint32_t>((f1 - a0) * 4));
                 ptx::prefetch_l2(prm.v_scale + a0, static_cast<uint32_t>((f1 - a0) * 4));
             }
@@ -380,7 +384,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int b = tid; b < prm.B; b += nthreads(PAGED)) {
             const int Lraw = prm.seq_lens[b];
             // tokens walked from the window base (all of them without a window)
-            int L = walked_len(Lraw, cap, plan, prm.qlen, prm.window);
+            int L = walked_len(Lraw, cap, plan, prm.qlen, prm.window, prm.recent);
             // (a chunk of queries needs its own tokens in the cache: L >= T)
             if (L < 0 || (CAUSAL && Lraw > 0 && Lraw < prm.qlen)) {
                 if (blockIdx.x == 0) raise_flag(prm.d_err, KVQ_DEVERR_LEN);
@@ -453,7 +457,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     auto one_raw = [&]() { return p.seq_lens[one_b]; };
     auto one_valid = [&](int Lraw) {
         const int64_t cap = PAGED ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
-        int L = walked_len(Lraw, cap, static_cast<int64_t>(p.splits) * p.chunk, p.qlen, p.window);
+        int L = walked_len(Lraw, cap, static_cast<int64_t>(p.splits) * p.chunk, p.qlen, p.window,
+                           p.recent);
         if (L < 0 || (CAUSAL && Lraw > 0 && Lraw < p.qlen)) {
             if (one_j == 0 && one_hk == 0 && tid == 32 * nprod(PAGED)) raise_flag(p.d_err, KVQ_DEVERR_LEN);
             L = 0;
@@ -581,7 +586,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                             // by plain loads (before the arrival that publishes them)
                             int nb = 0;             // 16-byte chunks of scales (none for FP8)
                             int64_t c0 = 0;
-                            if constexpr (F8 == 0) {
+                            if constexpr (!NOSC) {
                                 const int64_t f0 = row0 * NG;
                                 const int off = static_cast<int>(f0 & 3);
                                 c0 = f0 - off;
@@ -600,7 +605,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                                 full, 2 * Lay::KV_BYTES + 8 * nb + (with_q ? q_bytes : 0u));
                             ptx::tma_load_2d(sk, &tm_k, 0, static_cast<int>(row0), full, pol);
                             ptx::tma_load_2d(sv, &tm_v, 0, static_cast<int>(row0), full, pol);
-                            if (F8 == 0 && nb > 0) {
+                            if (!NOSC && nb > 0) {
                                 ptx::bulk_load(sks, k_scale + c0, 4 * nb, full);
                                 ptx::bulk_load(svs, v_scale + c0, 4 * nb, full);
                             }
@@ -647,7 +652,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         if (pg >= 0)
                             ptx::tma_load_2d(sk + lane * 16 * D, &tm_k, 0, (pg * Hk + hk) * 16, full, pol);
 #pragma unroll
-                        for (int it = 0; it < (F8 ? 0 : NG); ++it) {
+                        for (int it = 0; it < (NOSC ? 0 : NG); ++it) {
                             const int c = lane + 32 * it;
                             const int q = c / (4 * NG), cc = c % (4 * NG);
                             const int pq = __shfl_sync(0xffffffffu, pg, q);
@@ -713,7 +718,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     // 16+4t..16+4t+3 (b1) of k-step gi hold head_dim 32*gi + 8*t +
     // {0..3} and {4..7}: the same permutation of head_dim as the
     // K operand's bytes, so the dot products are unchanged.
-    auto build_q = [&](uint32_t sq) {
+    // ksc: per-head / per-channel K scales of the segment's (sequence, kv
+    // head), folded into Q (q_d * s_d) before the fixed-point digits
+    auto build_q = [&](uint32_t sq, const float* ksc) {
         float zsq[NT];
         int csq[NT][NCG];              // sum of the head's Qi (per 32-value group)
 #pragma unroll
@@ -730,6 +737,18 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 for (int e = 0; e < 4; ++e) {
                     qf[gi][2 * e] = bf16_bits_to_f32(w[e] & 0xffffu);
                     qf[gi][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
+                }
+                if constexpr (ST) {
+                    if (p.static_ns > 1) {
+                        const float4 s0 = *reinterpret_cast<const float4*>(ksc + 32 * gi + 8 * t);
+                        const float4 s1 = *reinterpret_cast<const float4*>(ksc + 32 * gi + 8 * t + 4);
+                        qf[gi][0] *= s0.x; qf[gi][1] *= s0.y; qf[gi][2] *= s0.z; qf[gi][3] *= s0.w;
+                        qf[gi][4] *= s1.x; qf[gi][5] *= s1.y; qf[gi][6] *= s1.z; qf[gi][7] *= s1.w;
+                    } else {
+                        const float s0 = ksc[0];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) qf[gi][e] *= s0;
+                    }
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(qf[gi][e]));
@@ -836,9 +855,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         kv = 64;
         bool have_q = false;            // Q fragments of this segment are built
+        const float* ksc = ST ? p.k_scale + (static_cast<int64_t>(b) * p.Hk + hk) * p.static_ns
+                              : nullptr;
         if (one) {                      // the query rows came ahead of stage 0
             wait(bar_q, 0);
-            build_q(sbase + Lay::Q_OFF);
+            build_q(sbase + Lay::Q_OFF, ksc);
             have_q = true;
         }
         // contiguous layout: the stage's scales start sc_off bytes in (the copies
@@ -864,7 +885,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const uint32_t svs = sv + Lay::KV_BYTES + Lay::SC_FLOATS * 4 + sc_off;
             if (!have_q) {
                 have_q = true;
-                build_q(sk + Lay::Q_OFF);
+                build_q(sk + Lay::Q_OFF, ksc);
             }
             const int tok0 = tt0 + 32 * wg;               // first token of this warp's slice
             if (tok0 < t1) {
@@ -921,8 +942,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const int cg = PK ? 2 * kg + par : kg;
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const float ksa = ldsf(sks + (rA[u] * NG + cg) * 4);
-                        const float ksb = ldsf(sks + (rB[u] * NG + cg) * 4);
+                        const float ksa = ST ? 1.f : ldsf(sks + (rA[u] * NG + cg) * 4);
+                        const float ksb = ST ? 1.f : ldsf(sks + (rB[u] * NG + cg) * 4);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -1051,8 +1072,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
                     for (int gv = 0; gv < NVS; ++gv) {
                         const int cg = PK ? 2 * gv + par : gv;
-                        vsa[u][gv] = okA[u] ? (F8 ? 1.f : ldsf(svs + (rA[u] * NG + cg) * 4)) : 0.f;
-                        vsb[u][gv] = okB[u] ? (F8 ? 1.f : ldsf(svs + (rB[u] * NG + cg) * 4)) : 0.f;
+                        vsa[u][gv] = okA[u] ? (NOSC ? 1.f : ldsf(svs + (rA[u] * NG + cg) * 4)) : 0.f;
+                        vsb[u][gv] = okB[u] ? (NOSC ? 1.f : ldsf(svs + (rB[u] * NG + cg) * 4)) : 0.f;
                         vmax = fmaxf(vmax, fmaxf(vsa[u][gv], vsb[u][gv]));
                     }
                 if constexpr (PK) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 2));
@@ -1184,8 +1205,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // segment that is the whole (b, kv head) writes the final rows
         // (one item per CTA: the final rows of a one-chunk or empty sequence come
         // from its chunk 0; chunks past the length write nothing)
-        const bool final_rows = one ? sg.j0 == 0 && sg.ns <= 1 : sg.j0 == 0 && sg.j1 == sg.ns - 1;
-        const bool part_rows = one ? sg.ns > 1 && sg.j0 < sg.ns : !final_rows;
+        // (mixed cache: partials only, the window kernel writes the rows)
+        const bool final_rows =
+            !p.recent && (one ? sg.j0 == 0 && sg.ns <= 1 : sg.j0 == 0 && sg.j1 == sg.ns - 1);
+        const bool part_rows = p.recent ? (one ? sg.j0 < sg.ns : true)
+                                        : (one ? sg.ns > 1 && sg.j0 < sg.ns : !final_rows);
         const int seg_j0 = sg.j0;
         // the previous segment's readers are done with the maxima and the slots
         if (merges > 0) wait(bar_mfree, (merges - 1) & 1);
@@ -1266,6 +1290,16 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 s1 = fmaf(fw[w], v.y, s1);
                 s2 = fmaf(fw[w], v.z, s2);
                 s3 = fmaf(fw[w], v.w, s3);
+            }
+            if constexpr (ST) {         // per-head / per-channel V scales on the output
+                const float* vsc = p.v_scale + (static_cast<int64_t>(b) * p.Hk + hk) * p.static_ns;
+                if (p.static_ns > 1) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(vsc + 4 * k);
+                    s0 *= w4.x; s1 *= w4.y; s2 *= w4.z; s3 *= w4.w;
+                } else {
+                    const float w1 = vsc[0];
+                    s0 *= w1; s1 *= w1; s2 *= w1; s3 *= w1;
+                }
             }
             const int64_t row = bh0 + h;
             if (final_rows) {
@@ -1367,7 +1401,7 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
 
 // Function attributes belong to the current device's context, so they are
 // set once per device ordinal.
-template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8>
+template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8, bool ST>
 cudaError_t set_attrs() {
     using Lay = Layout<D, G32, G16>;
     static std::atomic<uint64_t> done{0};
@@ -1375,7 +1409,7 @@ cudaError_t set_attrs() {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     return once_per_device(done, dev, cudaSuccess, [] {
-        auto kern = decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL, F8>;
+        auto kern = decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL, F8, ST>;
         cudaError_t r =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
         if (r == cudaSuccess)
@@ -1385,10 +1419,10 @@ cudaError_t set_attrs() {
     });
 }
 
-template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8 = 0>
+template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8 = 0, bool ST = false>
 cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     using Lay = Layout<D, G32, G16>;
-    cudaError_t e = set_attrs<D, G32, PAGED, G16, PK, CAUSAL, F8>();
+    cudaError_t e = set_attrs<D, G32, PAGED, G16, PK, CAUSAL, F8, ST>();
     if (e != cudaSuccess) return e;
     CUtensorMap mk, mv;
     const int64_t rows = PAGED ? static_cast<int64_t>(p.num_pages) * p.Hk * 16
@@ -1407,7 +1441,8 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL, F8>, mk, mv, p);
+    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL, F8, ST>, mk, mv,
+                              p);
 }
 
 template <int D, bool G32, bool PAGED>
@@ -1434,8 +1469,20 @@ cudaError_t pick_g_fp8(const DecodeParams& p, cudaStream_t s) {
                   : launch_tc<D, false, PAGED, false, false, false, F8>(p, s);
 }
 
+// per-head / per-channel scales (one set per (sequence, kv head))
+template <int D, bool PAGED>
+cudaError_t pick_g_static(const DecodeParams& p, cudaStream_t s) {
+    const bool masked = p.qlen > 1 || p.window > 0;
+    if (p.G > 8)
+        return masked ? launch_tc<D, false, PAGED, true, false, true, 0, true>(p, s)
+                      : launch_tc<D, false, PAGED, true, false, false, 0, true>(p, s);
+    return masked ? launch_tc<D, false, PAGED, false, false, true, 0, true>(p, s)
+                  : launch_tc<D, false, PAGED, false, false, false, 0, true>(p, s);
+}
+
 template <int D, bool PAGED>
 cudaError_t pick_fmt(const DecodeParams& p, cudaStream_t s) {
+    if (p.static_ns) return pick_g_static<D, PAGED>(p, s);
     if (p.fp8 == 1) return pick_g_fp8<D, PAGED, 1>(p, s);
     if (p.fp8 == 2) return pick_g_fp8<D, PAGED, 2>(p, s);
     return p.group32 ? pick_g<D, true, PAGED>(p, s) : pick_g<D, false, PAGED>(p, s);

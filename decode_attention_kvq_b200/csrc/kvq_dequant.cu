@@ -53,6 +53,27 @@ dequant_fp8_kernel(const uint8_t* __restrict__ q, int64_t n_vec, int fmt,
     }
 }
 
+// Per-head (ns = 1) / per-channel (ns = D) scales: `scale` holds the
+// (sequence, kv head)'s scales, applied to every row.
+__global__ void __launch_bounds__(kDequantThreads)
+dequant_static_kernel(const uint8_t* __restrict__ q, const float* __restrict__ scale,
+                      int64_t n_vec, int D, int ns, float* __restrict__ out) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kDequantThreads;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kDequantThreads + threadIdx.x; i < n_vec;
+         i += stride) {
+        const int64_t e = i * 16;
+        const int d0 = static_cast<int>(e % D);
+        const uint4 raw = *reinterpret_cast<const uint4*>(q + e);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        float* o = out + e;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float s = scale[ns > 1 ? d0 + j : 0];
+            o[j] = __fmul_rn(static_cast<float>(static_cast<int>((w[j >> 2] >> (8 * (j & 3))) & 0xffu) - 128), s);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kDequantThreads)
 dequant_kernel(const uint8_t* __restrict__ q, const float* __restrict__ scale, int64_t n_vec,
                int D, int group32, float* __restrict__ out) {
@@ -81,7 +102,7 @@ dequant_kernel(const uint8_t* __restrict__ q, const float* __restrict__ scale, i
 }  // namespace
 
 cudaError_t launch_dequant(const uint8_t* q, const float* scale, int64_t rows, int D,
-                           int group32, int fp8, float* out, cudaStream_t s) {
+                           int group32, int fp8, int static_ns, float* out, cudaStream_t s) {
     const int64_t n_vec = rows * D / 16;
     if (n_vec == 0) return cudaSuccess;
     int dev = 0, sms = 148;
@@ -90,7 +111,10 @@ cudaError_t launch_dequant(const uint8_t* q, const float* scale, int64_t rows, i
     int64_t blocks = (n_vec + kDequantThreads - 1) / kDequantThreads;
     const int64_t cap = static_cast<int64_t>(sms) * 8;   // grid-stride beyond 8 blocks per SM
     if (blocks > cap) blocks = cap;
-    if (fp8)
+    if (static_ns)
+        dequant_static_kernel<<<static_cast<unsigned>(blocks), kDequantThreads, 0, s>>>(
+            q, scale, n_vec, D, static_ns, out);
+    else if (fp8)
         dequant_fp8_kernel<<<static_cast<unsigned>(blocks), kDequantThreads, 0, s>>>(q, n_vec, fp8,
                                                                                  out);
     else

@@ -33,15 +33,22 @@ struct AppendParams {
     int B, Hk, T, D;
     int group32;             // 1: 32-value groups, 0: one scale per row
     int fp8;                 // 0: INT8 with scales, 1: FP8 E4M3, 2: FP8 E5M2 (no scales)
+    int static_ns;           // per-head (1) / per-channel (D) scales per (b, kv head); 0: per row
     int max_seq;             // contiguous capacity
     int page_size;           // 0: contiguous, else paged
     int max_pages, num_pages;
 };
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+// per-head / per-channel scales set from the call's tokens, then the tokens quantised
+cudaError_t launch_append_calibrate(const AppendParams& p, cudaStream_t s);
+// mixed cache: tokens leaving the bf16 window (ring [B, Hk, W, D]) are quantised
+// into the INT8 part, the new ones enter the window; p.pos holds the old lengths
+cudaError_t launch_append_mixed(const AppendParams& p, uint16_t* k_ring, uint16_t* v_ring, int W,
+                                cudaStream_t s);
 
 // --------------------------------------------------------------- dequant
 cudaError_t launch_dequant(const uint8_t* q, const float* scale, int64_t rows, int D,
-                           int group32, int fp8, float* out, cudaStream_t s);
+                           int group32, int fp8, int static_ns, float* out, cudaStream_t s);
 
 // ---------------------------------------------------------------- decode
 struct DecodeParams {
@@ -60,6 +67,7 @@ struct DecodeParams {
     int B, Hq, Hk, G, D;
     int group32;
     int fp8;                 // 0: INT8 with scales, 1: FP8 E4M3, 2: FP8 E5M2 (no scales)
+    int static_ns;           // per-head (1) / per-channel (D) scales per (b, kv head); 0: per token
     int page_size, max_seq, max_pages, num_pages;
     int chunk;               // KV tokens per split
     int splits;              // chunks of the longest sequence
@@ -69,6 +77,10 @@ struct DecodeParams {
     int qlen;                // queries per (sequence, q head): 1 for decode, T for a chunk
                              // (Hq and G then count (head, query) rows, query fastest)
     int window;              // sliding window w (0: none): a query at position p sees p - w + 1 .. p
+    int recent;              // mixed cache: the newest `recent` tokens are bf16 in a ring (0: none);
+                             // the split kernel walks the INT8 part and writes partials only
+    const uint16_t* rk;      // mixed cache: bf16 rings [B, Hk, recent, D] (K and V)
+    const uint16_t* rv;
     float scale_log2;        // attn_scale * log2(e)
 };
 
@@ -82,16 +94,23 @@ __host__ __device__ __forceinline__ int window_base(int L, int qlen, int window)
     return lo > 0 ? (lo & ~15) : 0;
 }
 
-// The number of tokens the kernels walk for a sequence of length L (from its
-// window base), or -1 when L is outside [0, cap] or beyond the plan.
-__device__ __forceinline__ int walked_len(int L, int64_t cap, int64_t plan, int qlen, int window) {
-    if (L < 0 || L > cap) return -1;
-    const int n = L - window_base(L, qlen, window);
+// The number of tokens the kernels walk for a sequence of length L: its INT8
+// part (all of it, or L - recent for a mixed cache) from its window base; -1
+// when L < 0 or the INT8 part is beyond the capacity or the plan.
+__device__ __forceinline__ int walked_len(int L, int64_t cap, int64_t plan, int qlen, int window,
+                                          int recent = 0) {
+    if (L < 0) return -1;
+    int n = L > recent ? L - recent : 0;
+    if (n > cap) return -1;
+    n -= window_base(n, qlen, window);
     return n > plan ? -1 : n;
 }
 constexpr int kMaxBatch = 1024;                              // sequences per call
+constexpr int kMaxRecent = 2048;                             // mixed cache: bf16 window tokens
 constexpr int kMaxGrid = 1024;                               // persistent CTAs
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+// mixed cache: the bf16 window's partial and the INT8 partials into the output
+cudaError_t launch_recent_combine(const DecodeParams& p, cudaStream_t s);
 // tensor-core split kernel (kvq_decode_tc.cu)
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s);
 

@@ -9,8 +9,9 @@
  *    calls, and never synchronises the stream (except kvq_read_error).
  *  - bf16 tensors are passed as uint16_t* (the raw bf16 bits).
  *  - Every pointer that is read or written with vector loads must be 16-byte
- *    aligned (all tensor arguments except d_pos, d_seq_lens, page_table and
- *    d_err, which need 4-byte alignment).  torch allocations satisfy this.
+ *    aligned (all tensor arguments except d_pos, d_seq_lens, page_table,
+ *    d_err and the per-head scale arrays, which need 4-byte alignment).
+ *    torch allocations satisfy this.
  *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy
  *    default stream.  All work is enqueued on it, in order.
  *  - Argument faults the host can see are reported synchronously as
@@ -69,8 +70,26 @@ typedef enum kvq_scale_mode {
     KVQ_SCALE_PER_TOKEN = 0,   /* one fp32 scale per (token, kv head): NG = 1 */
     KVQ_SCALE_GROUP32 = 1,     /* one fp32 scale per 32 values along head_dim: NG = D / 32 */
     KVQ_FP8_E4M3 = 2,          /* FP8 E4M3 bytes (bias 7, 3 mantissa bits), no scale: NG = 0 */
-    KVQ_FP8_E5M2 = 3           /* FP8 E5M2 bytes (bias 15, 2 mantissa bits), no scale: NG = 0 */
+    KVQ_FP8_E5M2 = 3,          /* FP8 E5M2 bytes (bias 15, 2 mantissa bits), no scale: NG = 0 */
+    KVQ_SCALE_PER_HEAD = 4,    /* INT8, one fp32 scale per (sequence, kv head): scales [B, Hk, 1] */
+    KVQ_SCALE_PER_CHANNEL = 5  /* INT8, one per (sequence, kv head, channel): scales [B, Hk, D] */
 } kvq_scale_mode;
+
+/*
+ * Per-head and per-channel modes (abaddon 0.2.0-rc.1,
+ * src/kv_cache_quant_cuda.rs, QuantGranularity::PerHead / PerChannel,
+ * OptimizedQuantizedKvCache::quantize_with_granularity): the scale arrays are
+ * not per token but per (sequence, kv head) -- the page's shapes (batch,
+ * heads, 1, 1) and (batch, heads, 1, head_dim) -- for contiguous caches and
+ * paged arenas alike.  kvq_append_calibrate sets them from one call's tokens
+ * (max |x| over the tokens and head_dim, or over the tokens per channel,
+ * floored at 1e-8, divided by 127) and quantises those tokens; kvq_append /
+ * kvq_append_paged in these modes quantise with the stored scales (the page
+ * concatenates later calls' scales along the token axis, which its own
+ * dequantise cannot broadcast: here a sequence keeps the scales of its
+ * calibrating call).  Every value uses the per-token rounding rule; values
+ * beyond the calibrated range clamp to the byte range.
+ */
 
 /* Device-side error bits (OR-ed into *d_err). */
 #define KVQ_DEVERR_POS 1u    /* append range [pos, pos + T) outside [0, capacity) */
@@ -122,6 +141,24 @@ kvq_status kvq_append_paged(const uint16_t *k_new, const uint16_t *v_new, int B,
                             uint8_t *v_arena, float *k_scale, float *v_scale,
                             const int32_t *page_table, int max_pages, int num_pages,
                             int page_size, int32_t *d_err, kvq_stream_t stream);
+
+/*
+ * kvq_append_calibrate -- per-head / per-channel quantisation of T new tokens
+ * per (sequence, kv head) into a contiguous cache: first the scales of each
+ * (sequence, kv head) are computed from these T tokens (mode
+ * KVQ_SCALE_PER_HEAD: one from all T * D values; KVQ_SCALE_PER_CHANNEL: one
+ * per channel from its T values) and written to k_scale / v_scale
+ * ([B, Hk, 1] or [B, Hk, D]), then the tokens are quantised with them at
+ * positions d_pos[b] .. d_pos[b] + T - 1 (bit-exact with that definition).
+ * Other arguments, requirements and errors as for kvq_append; a sequence
+ * whose range leaves the capacity is skipped (its scales untouched).
+ * Source: abaddon 0.2.0-rc.1, kv_cache_quant_cuda.rs,
+ * OptimizedQuantizedKvCache::quantize_with_granularity.
+ */
+kvq_status kvq_append_calibrate(const uint16_t *k_new, const uint16_t *v_new, int B, int Hk,
+                                int T, int D, kvq_scale_mode mode, const int32_t *d_pos,
+                                uint8_t *k_cache, uint8_t *v_cache, float *k_scale,
+                                float *v_scale, int max_seq, int32_t *d_err, kvq_stream_t stream);
 
 /*
  * Where decode attention finds the INT8 cache.  page_size == 0 selects the
@@ -260,6 +297,59 @@ size_t kvq_window_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_s
  */
 kvq_status kvq_decode_plan(int B, int Hk, int max_seq_len_hint, int num_splits, int num_sms,
                            int *chunk, int *splits);
+
+/*
+ * ---- Mixed cache: the newest tokens unquantised --------------------------
+ * A sequence's newest `window` tokens stay bf16 in a ring and the older ones
+ * are INT8 (abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
+ * DynamicQuantConfig::unquantized_window -- 128 by default -- and
+ * OptimizedQuantizedKvCache::append / get_kv).  After any append of a
+ * sequence of length L, positions 0 .. L - window - 1 are in the INT8 part (a
+ * contiguous cache [B, Hk, max_seq, D] with the mode's scales) and the last
+ * min(L, window) in the ring, bf16 [B, Hk, window, D], position g in row
+ * g % window.
+ */
+
+/*
+ * kvq_append_mixed -- append T new tokens per (sequence, kv head): they join
+ * the window, and the tokens that leave it (positions max(0, L0 - window) ..
+ * max(0, L0 + T - window) - 1, L0 = d_lens_old[b] the length before the
+ * call) are quantised into the INT8 part with the mode's rule (per token,
+ * group-32, or the stored per-head / per-channel scales).  Bit-exact with
+ * that definition.
+ *   k_new, v_new  bf16 [B, Hk, T, D];  d_lens_old int32 [B] (device)
+ *   k_cache ... max_seq  the INT8 part, as for kvq_append
+ *   k_ring, v_ring  bf16 [B, Hk, window, D];  1 <= window <= 2048
+ * Modes: KVQ_SCALE_PER_TOKEN, GROUP32, PER_HEAD, PER_CHANNEL.  A sequence
+ * whose INT8 part would exceed max_seq (or L0 < 0) is skipped and flagged
+ * with KVQ_DEVERR_POS.  The caller advances its lengths by T.
+ */
+kvq_status kvq_append_mixed(const uint16_t *k_new, const uint16_t *v_new, int B, int Hk, int T,
+                            int D, kvq_scale_mode mode, const int32_t *d_lens_old,
+                            uint8_t *k_cache, uint8_t *v_cache, float *k_scale, float *v_scale,
+                            int max_seq, uint16_t *k_ring, uint16_t *v_ring, int window,
+                            int32_t *d_err, kvq_stream_t stream);
+
+/*
+ * kvq_decode_attn_mixed -- decode attention over a mixed cache: the query
+ * attends to the INT8 part (fused dequantisation, split-K, any mode and
+ * layout of kvq_decode_attn; kv views it) and to the bf16 window, in one
+ * softmax.  d_seq_lens counts every token (INT8 part + window); the other
+ * arguments as for kvq_decode_attn, with a workspace of at least
+ * kvq_mixed_workspace_bytes(...) bytes (never 0: the INT8 partials of every
+ * row pass through it).
+ */
+kvq_status kvq_decode_attn_mixed(const uint16_t *q, int B, int Hq, int Hk, int D,
+                                 kvq_scale_mode mode, const kvq_cache_view *kv,
+                                 const uint16_t *k_ring, const uint16_t *v_ring, int window,
+                                 const int32_t *d_seq_lens, int max_seq_len_hint,
+                                 float attn_scale, float *out, void *workspace,
+                                 size_t workspace_bytes, int num_splits, int32_t *d_err,
+                                 kvq_stream_t stream);
+
+/* Workspace bytes kvq_decode_attn_mixed needs for these arguments. */
+size_t kvq_mixed_workspace_bytes(int B, int Hq, int Hk, int D, int max_seq_len_hint, int window,
+                                 int num_splits);
 
 /*
  * kvq_dequant -- x = (byte - 128) * scale, one fp32 multiply per element,
