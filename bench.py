@@ -62,20 +62,42 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def _ng(wl):
+    """Scales per (token, kv head) of the workload's cache format."""
+    return {"per_token": 1, "group32": wl.D // 32}.get(wl.mode, 0)
+
+
+def _static_ns(wl):
+    """Scales per (sequence, kv head): per-head 1, per-channel D, else 0."""
+    return {"per_head": 1, "per_channel": wl.D}.get(wl.mode, 0)
+
+
 def decode_bytes(wl, seq_lens, page_size=0):
-    """Algorithmic bytes of one decode call: K/V bytes + scales, Q, output,
-    page-table entries."""
-    ng = 1 if wl.mode == "per_token" else wl.D // 32
-    kv = sum(wl.Hk * L * (2 * wl.D + 2 * 4 * ng) for L in seq_lens)
+    """Algorithmic bytes of one decode call: the attended K/V bytes + their
+    scales (per token, or per (sequence, kv head)), the bf16 window of a mixed
+    cache, Q, output, page-table entries."""
+    ng = _ng(wl)
+    kv = 0
+    for L in seq_lens:
+        n8 = L
+        if wl.window:
+            n8 = min(L, wl.window + QLEN - 1)
+        if wl.recent:
+            n8 = max(L - wl.recent, 0)
+            kv += wl.Hk * (L - n8) * 2 * wl.D * 2           # bf16 window
+        kv += wl.Hk * n8 * (2 * wl.D + 2 * 4 * ng) + wl.Hk * 2 * 4 * _static_ns(wl)
     qo = wl.B * wl.Hq * wl.D * (2 + 4) * QLEN
     pt = sum((L + 15) // 16 * 4 for L in seq_lens) if page_size else 0
     return kv + qo + pt
 
 
 def append_bytes(wl, T):
-    ng = 1 if wl.mode == "per_token" else wl.D // 32
+    ng = _ng(wl)
     rd = T * wl.B * wl.Hk * wl.D * 2 * 2
     wr = T * wl.B * wl.Hk * (2 * wl.D + 2 * 4 * ng)
+    if wl.recent:                  # the token leaving the window is read back, the new one written
+        rd += T * wl.B * wl.Hk * wl.D * 2 * 2
+        wr += T * wl.B * wl.Hk * wl.D * 2 * 2
     return rd + wr
 
 
@@ -200,23 +222,33 @@ def decode_sources_hash():
 
 # ---------------------------------------------------------------- workload
 class Layer:
-    """One layer's INT8 cache on the GPU with its decode-step inputs."""
+    """One layer's KV cache on the GPU with its decode-step inputs: INT8 with
+    per-token / group-32 / per-channel scales, or FP8; contiguous or paged;
+    optionally a mixed cache (bf16 window ring) or sliding-window attention."""
 
     def __init__(self, kvq, wl, inp, dev, keep_host=False):
         self.wl = wl
         B, Hk, D = wl.B, wl.Hk, wl.D
-        ng = 1 if wl.mode == "per_token" else D // 32
+        ng = _ng(wl)
+        ns = _static_ns(wl)
         self.paged = wl.layout == "paged"
         cached = inp.cached
         self.seq_lens_list = [int(x) for x in inp.seq_lens]
         self.hint = max(self.seq_lens_list)
+
+        def scales(lead):
+            if ns:                      # per (sequence, kv head)
+                return torch.zeros(B, Hk, ns, device=dev)
+            if ng == 0:                 # FP8: none
+                return None
+            return torch.zeros(*lead, ng, device=dev)
+
         if self.paged:
             shape = (inp.num_pages, Hk, 16, D)
             self.table = inp.page_table.to(dev)
             self.k = torch.zeros(shape, dtype=torch.uint8, device=dev)
             self.v = torch.zeros_like(self.k)
-            self.ks = torch.zeros(inp.num_pages, Hk, 16, ng, device=dev)
-            self.vs = torch.zeros_like(self.ks)
+            self.ks, self.vs = scales((inp.num_pages, Hk, 16)), scales((inp.num_pages, Hk, 16))
             for b in range(B):
                 L = int(cached[b])
                 kv_k = inp.k_hist[b:b + 1, :, :L].contiguous().to(dev)
@@ -229,16 +261,31 @@ class Layer:
             self.table = None
             self.k = torch.zeros(B, Hk, S, D, dtype=torch.uint8, device=dev)
             self.v = torch.zeros_like(self.k)
-            self.ks = torch.zeros(B, Hk, S, ng, device=dev)
-            self.vs = torch.zeros_like(self.ks)
+            self.ks, self.vs = scales((B, Hk, S)), scales((B, Hk, S))
             Lmax = int(cached.max())
-            chunk = 8192
-            for p0 in range(0, Lmax, chunk):
-                T = min(chunk, Lmax - p0)
-                kvq.kvq_append(inp.k_hist[:, :, p0:p0 + T].contiguous().to(dev),
-                               inp.v_hist[:, :, p0:p0 + T].contiguous().to(dev),
-                               torch.full((B,), p0, dtype=torch.int32, device=dev),
-                               self.k, self.v, self.ks, self.vs, wl.mode)
+            if wl.recent:               # mixed cache: the history through the window
+                self.rk = torch.zeros(B, Hk, wl.recent, D, dtype=torch.bfloat16, device=dev)
+                self.rv = torch.zeros_like(self.rk)
+                lens = torch.zeros(B, dtype=torch.int32, device=dev)
+                for p0 in range(0, Lmax, 8192):
+                    T = min(8192, Lmax - p0)
+                    kvq.kvq_append_mixed(inp.k_hist[:, :, p0:p0 + T].contiguous().to(dev),
+                                         inp.v_hist[:, :, p0:p0 + T].contiguous().to(dev),
+                                         lens, self.k, self.v, self.ks, self.vs, self.rk,
+                                         self.rv, wl.mode)
+                    lens += T
+            else:
+                chunk = 8192
+                for p0 in range(0, Lmax, chunk):
+                    T = min(chunk, Lmax - p0)
+                    args = (inp.k_hist[:, :, p0:p0 + T].contiguous().to(dev),
+                            inp.v_hist[:, :, p0:p0 + T].contiguous().to(dev),
+                            torch.full((B,), p0, dtype=torch.int32, device=dev),
+                            self.k, self.v, self.ks, self.vs, wl.mode)
+                    if ns and p0 == 0:  # per-channel: the first chunk sets the scales
+                        kvq.kvq_append_calibrate(*args)
+                    else:
+                        kvq.kvq_append(*args)
         self.k_new = inp.k_new.to(dev)
         self.v_new = inp.v_new.to(dev)
         self.q = inp.q.to(dev)
@@ -251,16 +298,33 @@ class Layer:
         if keep_host:
             self.host = inp
         # prefill chunk re-append (long-context workload): rewrite the last chunk
-        self.chunk_T = wl.prefill_chunk
+        self.chunk_T = wl.prefill_chunk if not wl.recent else 0
         if self.chunk_T:
             p0 = int(cached[0]) - self.chunk_T
             self.chunk_k = inp.k_hist[:, :, p0:p0 + self.chunk_T].contiguous().to(dev)
             self.chunk_v = inp.v_hist[:, :, p0:p0 + self.chunk_T].contiguous().to(dev)
             self.chunk_pos = torch.full((B,), p0, dtype=torch.int32, device=dev)
 
+    def workspace_bytes(self, kvq):
+        wl, hint = self.wl, self.hint
+        if wl.recent:
+            return int(kvq.lib.kvq_mixed_workspace_bytes(wl.B, wl.Hq, wl.Hk, wl.D, hint,
+                                                         wl.recent, 0))
+        if wl.window:
+            return int(kvq.lib.kvq_window_workspace_bytes(wl.B, wl.Hq, wl.Hk, QLEN, wl.D, hint,
+                                                          wl.window, 0))
+        if QLEN == 1:
+            return kvq.kvq_decode_workspace_bytes(wl.B, wl.Hq, wl.Hk, wl.D, hint)
+        return kvq.kvq_chunk_workspace_bytes(wl.B, wl.Hq, wl.Hk, QLEN, wl.D, hint)
+
     def append(self, kvq, k_new=None, v_new=None, stream=None):
         k_new = self.k_new if k_new is None else k_new
         v_new = self.v_new if v_new is None else v_new
+        if self.wl.recent:
+            # the step's token joins the window; the one leaving it is quantised
+            kvq.kvq_append_mixed(k_new, v_new, self.pos, self.k, self.v, self.ks, self.vs,
+                                 self.rk, self.rv, self.wl.mode, stream=stream)
+            return
         if self.chunk_T:
             kvq.kvq_append(self.chunk_k, self.chunk_v, self.chunk_pos, self.k, self.v, self.ks,
                            self.vs, self.wl.mode, stream=stream)
@@ -272,12 +336,22 @@ class Layer:
                            self.wl.mode, stream=stream)
 
     def decode(self, kvq, workspace, q=None, out=None, stream=None):
-        call = kvq.kvq_decode_attn if self.qlen == 1 else kvq.kvq_chunk_attn
-        call(self.q if q is None else q, self.k, self.v, self.ks, self.vs,
-                            self.seq_lens, self.hint, mode=self.wl.mode,
-                            out=self.out if out is None else out, workspace=workspace,
-                            page_table=self.table, page_size=16 if self.paged else 0,
-                            view=self.view, stream=stream)
+        q = self.q if q is None else q
+        out = self.out if out is None else out
+        wl = self.wl
+        common = dict(mode=wl.mode, out=out, workspace=workspace, stream=stream)
+        if wl.recent:
+            kvq.kvq_decode_attn_mixed(q, self.k, self.v, self.ks, self.vs, self.rk, self.rv,
+                                      self.seq_lens, self.hint, **common)
+        elif wl.window:
+            kvq.kvq_window_attn(q, self.k, self.v, self.ks, self.vs, self.seq_lens, self.hint,
+                                wl.window, page_table=self.table,
+                                page_size=16 if self.paged else 0, view=self.view, **common)
+        else:
+            call = kvq.kvq_decode_attn if self.qlen == 1 else kvq.kvq_chunk_attn
+            call(q, self.k, self.v, self.ks, self.vs, self.seq_lens, self.hint,
+                 page_table=self.table, page_size=16 if self.paged else 0, view=self.view,
+                 **common)
 
 
 def build_layers(kvq, wl, n_layers, dev, keep_host=False):
@@ -453,14 +527,12 @@ class GpuWorkload:
         self.n_layers = n_layers
         L0 = self.layers[0]
         self.hint = L0.hint
-        ws_bytes = (kvq.kvq_decode_workspace_bytes(wl.B, wl.Hq, wl.Hk, wl.D, L0.hint)
-                    if QLEN == 1 else
-                    kvq.kvq_chunk_workspace_bytes(wl.B, wl.Hq, wl.Hk, QLEN, wl.D, L0.hint))
+        ws_bytes = L0.workspace_bytes(kvq)
         self.workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
         self.chunk, self.splits = kvq.kvq_decode_plan(wl.B, wl.Hk, L0.hint)
         # append (+ prefill-chunk append) + split kernel (+ combine kernel when a
         # sequence spans several chunks: then the call has a workspace)
-        self.launches_per_layer = ((1 + (1 if wl.prefill_chunk else 0)) + 1 +
+        self.launches_per_layer = ((1 + (1 if L0.chunk_T else 0)) + 1 +
                                    (1 if ws_bytes > 0 else 0))
         self.stream = torch.cuda.Stream(dev)
         with torch.cuda.stream(self.stream):       # warm the library once eagerly
@@ -650,7 +722,7 @@ def run_kvq(args, wl):
     # caches and graphs are reused for its own entry
     if QLEN == 1 and not args.no_per_config and args.layers == 0:
         pc = {}
-        for name, w in synth.WORKLOADS.items():
+        for name, w in synth.ALL_WORKLOADS.items():
             pc[name] = per_config_entry(kvq, w, dev, K, W, world,
                                         gw=gw if name == wl.name else None)
         line["per_config"] = pc
@@ -721,7 +793,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
-    ap.add_argument("--workload", choices=list(synth.WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", choices=list(synth.ALL_WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--layers", type=int, default=0, help="layer caches per step (0: default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
@@ -737,8 +809,10 @@ def main(argv=None):
         ap.error("--qlen must be at least 1")
     QLEN = args.qlen
     args.warmup = max(args.warmup, 3)     # timing rule: at least 3 untimed warm-up steps
-    wl = synth.WORKLOADS[args.workload]
+    wl = synth.ALL_WORKLOADS[args.workload]
     if args.impl == "reference":
+        if args.workload not in synth.WORKLOADS:
+            ap.error("the reference arm runs the five parity workloads")
         return run_reference(args, wl)
     return run_kvq(args, wl)
 

@@ -6,6 +6,8 @@ quantisation or attention arithmetic.
 """
 from .workloads import (  # noqa: F401
     WORKLOADS,
+    EXTRA_WORKLOADS,
+    ALL_WORKLOADS,
     Workload,
     bf16_normal,
     lengths_uniform,

@@ -31,7 +31,7 @@ class Workload:
     Hq: int
     Hk: int
     D: int
-    mode: str               # "per_token" | "group32"
+    mode: str               # "per_token" | "group32" | "fp8_e4m3" | "fp8_e5m2" | "per_channel" ...
     layout: str             # "contiguous" | "paged"
     len_lo: int             # cached length before the decode append (inclusive range)
     len_hi: int
@@ -40,6 +40,8 @@ class Workload:
     outlier_factor: float = 1.0
     prefill_chunk: int = 0  # tokens per append call when building the cache
     seed: int = 0
+    window: int = 0         # sliding-window attention over the last `window` positions (0: none)
+    recent: int = 0         # mixed cache: the newest `recent` tokens kept bf16 (0: none)
 
     @property
     def G(self) -> int:
@@ -47,7 +49,8 @@ class Workload:
 
     @property
     def NG(self) -> int:
-        return 1 if self.mode == "per_token" else self.D // 32
+        """Scales per (token, kv head)."""
+        return {"per_token": 1, "group32": self.D // 32}.get(self.mode, 0)
 
 
 WORKLOADS = {
@@ -62,6 +65,23 @@ WORKLOADS = {
     "long_context": Workload("long_context", 1, 64, 8, 128, "per_token", "contiguous",
                              131072, 131072, 1.0, 0.02, 20.0, prefill_chunk=2048, seed=1005),
 }
+
+
+# The same shapes and data with the other cache formats and attention forms
+# (measurement lines for them; the five workloads above are the parity and
+# headline cases).
+EXTRA_WORKLOADS = {
+    "long_context_fp8_e4m3": dataclasses.replace(WORKLOADS["long_context"],
+                                                 name="long_context_fp8_e4m3", mode="fp8_e4m3"),
+    "long_context_per_channel": dataclasses.replace(WORKLOADS["long_context"],
+                                                    name="long_context_per_channel",
+                                                    mode="per_channel"),
+    "long_context_window4096": dataclasses.replace(WORKLOADS["long_context"],
+                                                   name="long_context_window4096", window=4096),
+    "llama3_8b_layer_mixed128": dataclasses.replace(WORKLOADS["llama3_8b_layer"],
+                                                    name="llama3_8b_layer_mixed128", recent=128),
+}
+ALL_WORKLOADS = {**WORKLOADS, **EXTRA_WORKLOADS}
 
 
 def _gen(seed: int) -> torch.Generator:
