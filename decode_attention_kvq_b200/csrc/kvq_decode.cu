@@ -256,84 +256,175 @@ size_t combine_one_spread_smem(int rows) {
 
 // Mixed cache (abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
 // OptimizedQuantizedKvCache::get_kv: the INT8 part dequantised, then the
-// unquantised recent tokens): one CTA per (b, q head).  The newest
-// min(L, W) tokens sit in the bf16 ring (position g in row g % W); their
-// partial (m, l, o) is computed here in fp32 from the bf16 values, then
-// folded with the split kernel's INT8 partials (every slot below the INT8
-// part's chunk count with a finite m) into the output row.
-__global__ void __launch_bounds__(kThreads)
+// unquantised recent tokens): one CTA per (b, kv head) and its G query heads.
+// The newest min(L, W) tokens sit in the bf16 ring (position g in row g % W);
+// they are walked in tiles of kRecTile tokens staged in shared memory (K and V
+// rows by 16-byte loads), with an online softmax per head in fp32: scores by
+// one warp per token (lanes over head_dim, all G heads at once), then each
+// thread updates its (head, head_dim) outputs from the tile's V rows.  The
+// split kernel's INT8 partials (every slot below the INT8 part's chunk count
+// with a finite m) are folded in at the end and the rows written.
+constexpr int kRecThreads = 256;
+constexpr int kRecWarps = kRecThreads / 32;
+constexpr int kRecTile = 16;                    // window tokens per shared-memory tile
+constexpr int kRecMaxG = 16;
+__global__ void __launch_bounds__(kRecThreads)
 decode_recent_combine(DecodeParams p) {
-    __shared__ float s_z[kMaxRecent];   // the window's scores
-    __shared__ float s_red[kWarps];
+    __shared__ __align__(16) float s_q[kRecMaxG * 256];             // the G query rows (fp32)
+    __shared__ __align__(16) uint16_t s_k[kRecTile * 256], s_v[kRecTile * 256];
+    __shared__ float s_p[kRecMaxG][kRecTile];                       // scores, then weights
+    __shared__ float s_m[kRecMaxG], s_l[kRecMaxG], s_a[kRecMaxG];   // running max, sum, rescale
     grid_dep_wait();                    // the split kernel's partials are complete
     grid_dep_launch();
-    const int64_t bh = blockIdx.x;
-    const int b = static_cast<int>(bh / p.Hq);
-    const int h = static_cast<int>(bh % p.Hq);
-    const int hk = h / p.G;
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int D = p.D, W = p.recent;
-    float* out = p.out + bh * D;
+    const int unit = blockIdx.x;                        // b * Hk + hk
+    const int b = unit / p.Hk;
+    const int G = p.G, D = p.D, W = p.recent;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t bh0 = static_cast<int64_t>(unit) * G;  // first q row (b * Hq + hk * G)
     const int64_t cap = p.page_size ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
     const int64_t plan = static_cast<int64_t>(p.splits) * p.chunk;
     const int L = p.seq_lens[b];
     const int n8 = walked_len(L, cap, plan, 1, 0, W);   // INT8 part walked by the split kernel
     if (n8 < 0) {                                       // flagged by the split kernel
-        for (int d = tid; d < D; d += kThreads) out[d] = 0.f;
+        for (int i = tid; i < G * D; i += kRecThreads) p.out[bh0 * D + i] = 0.f;
         return;
     }
     const int Lq = L > W ? L - W : 0;
     const int nr = L - Lq;                              // tokens in the window
-    const uint16_t* qh = p.q + bh * D;
-    const int64_t ring0 = (static_cast<int64_t>(b) * p.Hk + hk) * W;
-    // ---- window scores (log2 domain), one warp per token, lanes over head_dim
-    float mloc = -INFINITY;
-    for (int i = w; i < nr; i += kWarps) {
-        const uint16_t* kr = p.rk + (ring0 + (Lq + i) % W) * D;
-        float dot = 0.f;
-        for (int d = lane; d < D; d += 32)
-            dot = fmaf(bf16_bits_to_f32(qh[d]), bf16_bits_to_f32(kr[d]), dot);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-        const float z = dot * p.scale_log2;
-        if (lane == 0) s_z[i] = z;
-        mloc = fmaxf(mloc, z);
+    for (int i = tid; i < G * D; i += kRecThreads)
+        s_q[i] = bf16_bits_to_f32(p.q[bh0 * D + i]);
+    if (tid < G) {
+        s_m[tid] = -INFINITY;
+        s_l[tid] = 0.f;
     }
-    if (lane == 0) s_red[w] = mloc;
-    __syncthreads();
-    float mr = -INFINITY;
+    // this thread's (head, head_dim) outputs: pairs tid + kRecThreads * k
+    constexpr int kMaxPairs = kRecMaxG * 256 / kRecThreads;
+    float o[kMaxPairs];
 #pragma unroll
-    for (int x = 0; x < kWarps; ++x) mr = fmaxf(mr, s_red[x]);
-    // ---- INT8 partials: the running max over them and the window
-    const int ns = (n8 + p.chunk - 1) / p.chunk;
-    const float* m8 = p.ws_m + bh * p.splits;
-    const float* l8 = p.ws_l + bh * p.splits;
-    float M = mr;
-    for (int j = 0; j < ns; ++j) M = fmaxf(M, m8[j]);
-    // ---- each thread: its head_dim values of the weighted sums
-    float lsum = 0.f;
-    for (int i = 0; i < nr; ++i) lsum += exp2f(s_z[i] - M);
-    for (int j = 0; j < ns; ++j)
-        if (m8[j] != -INFINITY) lsum = fmaf(exp2f(m8[j] - M), l8[j], lsum);
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    for (int d = tid; d < D; d += kThreads) {
-        float acc = 0.f;
-        for (int i = 0; i < nr; ++i) {
-            const uint16_t* vr = p.rv + (ring0 + (Lq + i) % W) * D;
-            acc = fmaf(exp2f(s_z[i] - M), bf16_bits_to_f32(vr[d]), acc);
+    for (int k = 0; k < kMaxPairs; ++k) o[k] = 0.f;
+    const int npair = G * D;
+    const int64_t ring0 = static_cast<int64_t>(unit) * W;
+    const int vec = D / 8;                              // 16-byte chunks per row
+    for (int i0 = 0; i0 < nr; i0 += kRecTile) {
+        const int n = min(kRecTile, nr - i0);
+        __syncthreads();                                // the previous tile is consumed
+        for (int c = tid; c < n * vec; c += kRecThreads) {
+            const int t = c / vec, x = c % vec;
+            const int64_t row = ring0 + (Lq + i0 + t) % W;
+            reinterpret_cast<uint4*>(s_k)[t * vec + x] =
+                reinterpret_cast<const uint4*>(p.rk + row * D)[x];
+            reinterpret_cast<uint4*>(s_v)[t * vec + x] =
+                reinterpret_cast<const uint4*>(p.rv + row * D)[x];
         }
-        for (int j = 0; j < ns; ++j)
-            if (m8[j] != -INFINITY)
-                acc = fmaf(exp2f(m8[j] - M), p.ws_o[(bh * p.splits + j) * D + d], acc);
-        out[d] = acc * inv;
+        __syncthreads();
+        // scores (log2 domain): one warp per token, lanes over head_dim
+        for (int t = warp; t < n; t += kRecWarps) {
+            float acc[kRecMaxG];
+#pragma unroll
+            for (int h = 0; h < kRecMaxG; ++h) acc[h] = 0.f;
+            for (int d = lane; d < D; d += 32) {
+                const float kv = bf16_bits_to_f32(s_k[t * D + d]);
+#pragma unroll
+                for (int h = 0; h < kRecMaxG; ++h)
+                    if (h < G) acc[h] = fmaf(s_q[h * D + d], kv, acc[h]);
+            }
+#pragma unroll
+            for (int h = 0; h < kRecMaxG; ++h) {
+                if (h >= G) break;
+                float a = acc[h];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+                if (lane == 0) s_p[h][t] = a * p.scale_log2;
+            }
+        }
+        __syncthreads();
+        // online softmax per head (one thread per head)
+        if (tid < G) {
+            float mt = -INFINITY;
+            for (int t = 0; t < n; ++t) mt = fmaxf(mt, s_p[tid][t]);
+            const float mn = fmaxf(s_m[tid], mt);
+            const float a = exp2f(s_m[tid] - mn);       // 0 while the max was -inf
+            float add = 0.f;
+            for (int t = 0; t < n; ++t) {
+                const float e = exp2f(s_p[tid][t] - mn);
+                s_p[tid][t] = e;
+                add += e;
+            }
+            s_l[tid] = s_l[tid] * a + add;
+            s_m[tid] = mn;
+            s_a[tid] = a;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < kMaxPairs; ++k) {
+            const int idx = tid + kRecThreads * k;
+            if (idx >= npair) break;
+            const int h = idx / D, d = idx % D;
+            float acc = o[k] * s_a[h];
+            for (int t = 0; t < n; ++t) acc = fmaf(s_p[h][t], bf16_bits_to_f32(s_v[t * D + d]), acc);
+            o[k] = acc;
+        }
+    }
+    __syncthreads();
+    // the INT8 partials of each head: their max and weighted sum (warp per head)
+    const int ns = (n8 + p.chunk - 1) / p.chunk;
+    for (int h = warp; h < G; h += kRecWarps) {
+        const float* m8 = p.ws_m + (bh0 + h) * p.splits;
+        const float* l8 = p.ws_l + (bh0 + h) * p.splits;
+        float M = s_m[h];
+        for (int j = lane; j < ns; j += 32) M = fmaxf(M, m8[j]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float ls = 0.f;
+        for (int j = lane; j < ns; j += 32)
+            if (m8[j] != -INFINITY) ls = fmaf(exp2f(m8[j] - M), l8[j], ls);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
+        if (lane == 0) {
+            const float aw = s_m[h] == -INFINITY ? 0.f : exp2f(s_m[h] - M);
+            const float tot = ls + s_l[h] * aw;
+            s_a[h] = aw;                                // the window's weight
+            s_l[h] = tot > 0.f ? 1.f / tot : 0.f;       // the normaliser
+            s_m[h] = M;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kMaxPairs; ++k) {
+        const int idx = tid + kRecThreads * k;
+        if (idx >= npair) break;
+        const int h = idx / D, d = idx % D;
+        const int64_t row = bh0 + h;
+        const float M = s_m[h];
+        const float* m8 = p.ws_m + row * p.splits;
+        const float* o8 = p.ws_o + row * p.splits * D + d;
+        float acc = o[k] * s_a[h];
+        int j = 0;
+        for (; j + 4 <= ns; j += 4) {                   // four slots' loads in flight
+            float mj[4], oj[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                mj[u] = m8[j + u];
+                oj[u] = o8[static_cast<int64_t>(j + u) * D];
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (mj[u] != -INFINITY) acc = fmaf(exp2f(mj[u] - M), oj[u], acc);
+        }
+        for (; j < ns; ++j) {
+            const float mj = m8[j];
+            if (mj != -INFINITY) acc = fmaf(exp2f(mj - M), o8[static_cast<int64_t>(j) * D], acc);
+        }
+        p.out[row * D + d] = acc * s_l[h];
     }
 }
 
 cudaError_t launch_recent_combine(const DecodeParams& p, cudaStream_t s) {
-    if (p.recent < 1 || p.recent > kMaxRecent) return cudaErrorInvalidValue;
+    if (p.recent < 1 || p.recent > kMaxRecent || p.G > kRecMaxG || p.D > 256 || p.qlen != 1)
+        return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.B * p.Hq, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.gridDim = dim3(p.B * p.Hk, 1, 1);
+    cfg.blockDim = dim3(kRecThreads, 1, 1);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
