@@ -137,10 +137,26 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
         !aligned(kv->k_scale, sa) || !aligned(kv->v_scale, sa) || !aligned(d_seq_lens, 4) ||
         !aligned(out, 16) || !aligned(workspace, 16) || !aligned(d_err, 4))
         return KVQ_ERR_INVALID_ARG;
-    if (T > 16 || Hq > 65535) return KVQ_ERR_UNSUPPORTED;
+    if (Hq > 65535) return KVQ_ERR_UNSUPPORTED;
+    // more than 16 (head, query) rows per kv head: the dense chunk kernel on
+    // the tcgen05 tensor cores
+    const bool dense = static_cast<int64_t>(Hq / Hk) * T > 16;
+    if (dense) {
+        if (!kvq::chunk_tc_supported(D, Hq / Hk, T, mode == KVQ_SCALE_GROUP32, is_fp8(mode),
+                                     static_ns(mode, D), kv->page_size, window, recent))
+            return KVQ_ERR_UNSUPPORTED;
+        if (static_cast<int64_t>(B) * Hq * T >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+        if (B == 0) return KVQ_OK;
+        if (static_cast<int64_t>(B) * Hk * kv->max_seq >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+        kvq::DecodeParams p{};
+        p.q = q; p.k = kv->k; p.v = kv->v; p.k_scale = kv->k_scale; p.v_scale = kv->v_scale;
+        p.seq_lens = d_seq_lens; p.out = out; p.d_err = d_err;
+        p.B = B; p.Hk = Hk; p.D = D; p.max_seq = kv->max_seq;
+        p.scale_log2 = attn_scale * 1.4426950408889634f;
+        return from_cuda(kvq::launch_chunk_tc(p, Hq, Hq / Hk, T, static_cast<cudaStream_t>(stream)));
+    }
     const int G = Hq / Hk * T;          // rows per kv head: (head, query), query fastest
     if (D != 64 && D != 128) return KVQ_ERR_UNSUPPORTED;
-    if (G > 16) return KVQ_ERR_UNSUPPORTED;
     // the split kernel keeps every sequence length in shared memory
     if (B > kvq::kMaxBatch) return KVQ_ERR_UNSUPPORTED;
     // TMA row coordinates are 32-bit
@@ -366,7 +382,8 @@ size_t kvq_window_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_s
 
 size_t kvq_chunk_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_seq_len_hint,
                                  int num_splits) {
-    if (T < 1 || Hq > INT32_MAX / T) return 0;
+    if (T < 1 || Hq > INT32_MAX / T || Hk < 1) return 0;
+    if (static_cast<int64_t>(Hq / Hk) * T > 16) return 0;   // the dense kernel needs none
     return kvq_decode_workspace_bytes(B, Hq * T, Hk, D, max_seq_len_hint, num_splits);
 }
 

@@ -1495,6 +1495,10 @@ cudaError_t pick_layout(const DecodeParams& p, cudaStream_t s) {
 
 }  // namespace
 
+cudaError_t make_tile_map(CUtensorMap* map, const void* base, int D, int64_t rows, int box_rows) {
+    return make_map(map, base, D, rows, box_rows);
+}
+
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s) {
     if (p.grid < 1) return cudaErrorInvalidValue;
     if (p.D == 128) return pick_layout<128>(p, s);

@@ -3,6 +3,7 @@
 // the public ABI; the public declarations live in include/kvq.h.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -143,6 +144,17 @@ __device__ __forceinline__ uint32_t fp8_from_bf16(uint32_t h, int fmt) {
     if (e4 && (c & 0x7fu) == 0x7fu) c = s | 0x7eu;
     return c;
 }
+
+// 2-D u8 TMA tensor map over `rows` rows of D bytes (box of box_rows rows,
+// 128-byte swizzle for D = 128, 64-byte for D = 64), cached per host thread.
+cudaError_t make_tile_map(CUtensorMap* map, const void* base, int D, int64_t rows, int box_rows);
+
+// Dense chunk attention on the tcgen05 tensor cores (kvq_chunk_tc.cu): the
+// shapes it covers, and its launch (dp as built for the chunk, Hq / G / T the
+// call's own head count, group and chunk length).
+bool chunk_tc_supported(int D, int G, int T, int group32, int fp8, int static_ns, int page_size,
+                        int window, int recent);
+cudaError_t launch_chunk_tc(const DecodeParams& dp, int Hq, int G, int T, cudaStream_t s);
 
 // Programmatic dependent launch: wait for the preceding grid's writes, and
 // let the next grid in the stream be scheduled early.

@@ -151,7 +151,10 @@ def test_decode_rejects_bad_arguments(kvq):
     assert call(mode=1, D=48) == 1
     assert call(D=256) == 2                 # valid, kernel not built for it
     assert call(D=32) == 2
-    assert call(Hq=8 * 32, Hk=8) == 2       # GQA group above the built tile (16)
+    # a GQA group above 16 rows runs on the dense tcgen05 kernel, which covers
+    # head_dim 128, per-token scales, contiguous caches: other shapes are refused
+    assert call(Hq=8 * 32, Hk=8, D=64) == 2
+    assert call(Hq=8 * 32, Hk=8, mode=1) == 2
     assert call(B=1025) == 2                # more sequences than the split kernel caches
     assert call(out=FAKE + 4) == 1          # misaligned output
     cv_bad_scale = kvq.CacheView(FAKE, FAKE, FAKE + 8, FAKE, 0, 4096, 0, 0, 0)
@@ -176,8 +179,12 @@ def test_chunk_rejects_bad_arguments(kvq):
         return lib.kvq_chunk_attn(*a.values())
     assert call(T=0) == 1
     assert call(q=None) == 1
-    assert call(T=5) == 2                   # (Hq / Hk) * T = 20 rows per kv head
-    assert call(Hq=64, T=3) == 2            # 24 rows
+    # more than 16 rows per kv head: the dense kernel, head_dim 128, per-token,
+    # contiguous, no window only
+    assert call(T=5, D=64) == 2             # (Hq / Hk) * T = 20 rows per kv head
+    assert call(Hq=64, T=3, mode=1) == 2    # 24 rows, group-32 scales
+    pv = kvq.CacheView(FAKE, FAKE, FAKE, FAKE, 16, 0, FAKE, 4, 4)
+    assert call(T=5, kv=ctypes.byref(pv)) == 2     # paged
     assert call(out=FAKE + 4) == 1
 
 
@@ -187,6 +194,7 @@ def test_chunk_workspace_is_the_decode_workspace_of_the_rows(kvq):
         assert kvq.kvq_chunk_workspace_bytes(B, Hq, Hk, T, D, hint, ns) == \
             kvq.kvq_decode_workspace_bytes(B, Hq * T, Hk, D, hint, ns)
     assert kvq.kvq_chunk_workspace_bytes(1, 32, 8, 0, 128, 4097, 0) == 0
+    assert kvq.kvq_chunk_workspace_bytes(1, 32, 8, 5, 128, 4097, 0) == 0   # dense: none
 
 
 @needs_no_gpu

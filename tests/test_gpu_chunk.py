@@ -106,7 +106,9 @@ def test_chunk_longer_than_its_sequence_is_a_length_error():
     assert_attn_close(out[1:], c.oracle_chunk(q, sl, f32_scale(D))[1:], "valid sequence")
 
 
-def test_chunk_rows_beyond_sixteen_per_kv_head_are_unsupported():
+def test_chunk_rows_beyond_sixteen_per_kv_head_at_d64_are_unsupported():
+    """More than 16 rows per kv head run on the dense kernel, which covers
+    head_dim 128 only."""
     m = kvq()
     c = _contig(1, 1, 64, "per_token", [40], seed=121)
     q = bf16_randn((1, 4, 5, 64), seed=122)      # G * T = 20
