@@ -72,6 +72,22 @@ def _static_ns(wl):
     return {"per_head": 1, "per_channel": wl.D}.get(wl.mode, 0)
 
 
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s on this machine's B200s (burst), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def chunk_flops(wl, seq_lens, T):
+    """Useful flops of one chunk-attention call: every (query, head) row times
+    the keys it sees (L - T + i + 1 for query i), 2 D for Q.K^T and 2 D for P.V."""
+    pairs = sum(T * (L - T) + T * (T + 1) // 2 for L in seq_lens)
+    return pairs * wl.Hq * wl.D * 2 * 2
+
+
 def decode_bytes(wl, seq_lens, page_size=0):
     """Algorithmic bytes of one decode call: the attended K/V bytes + their
     scales (per token, or per (sequence, kv head)), the bf16 window of a mixed
@@ -298,7 +314,8 @@ class Layer:
         if keep_host:
             self.host = inp
         # prefill chunk re-append (long-context workload): rewrite the last chunk
-        self.chunk_T = wl.prefill_chunk if not wl.recent else 0
+        # (a chunk step's own tokens are the chunk: no separate re-append then)
+        self.chunk_T = wl.prefill_chunk if (not wl.recent and QLEN == 1) else 0
         if self.chunk_T:
             p0 = int(cached[0]) - self.chunk_T
             self.chunk_k = inp.k_hist[:, :, p0:p0 + self.chunk_T].contiguous().to(dev)
@@ -551,7 +568,7 @@ class GpuWorkload:
         self.dec_b = sum(decode_bytes(wl, ly.seq_lens_list, 16 if ly.paged else 0)
                          for ly in self.layers)
         self.app_b = n_layers * (append_bytes(wl, QLEN) +
-                                 (append_bytes(wl, wl.prefill_chunk) if wl.prefill_chunk else 0))
+                                 (append_bytes(wl, L0.chunk_T) if L0.chunk_T else 0))
 
     def warm(self, W):
         with torch.cuda.stream(self.stream):
@@ -649,6 +666,47 @@ def per_config_entry(kvq, wl, dev, K, W, world, gw=None):
     return entry
 
 
+def prefill_entry(kvq, wl, dev, K, W, world, T):
+    """A prefill step of the workload's shape: append a T-token chunk per
+    (sequence, kv head), then T queries per head attend causally (the dense
+    chunk kernel when (Hq / Hk) * T > 16).  Tensor-bound: useful flops over the
+    measured bf16 peak; median over repeats."""
+    global QLEN
+    saved = QLEN
+    QLEN = T
+    try:
+        gw = GpuWorkload(kvq, wl, dev, 1)
+        gw.warm(max(W, 3))
+        _, t_probe = gw.timed(2, ClockSampler(-1, enabled=False))
+        reps = max(10, min(200, int(math.ceil(0.25 / max(t_probe / 2, 1e-6)))))
+        sampler = ClockSampler(physical_gpu_index(dev.index))
+        per, _ = gw.timed(reps, sampler)
+        t_app = reduce_max(statistics.median(a for a, _ in per), dev)
+        t_att = reduce_max(statistics.median(d for _, d in per), dev)
+        L0 = gw.layers[0]
+        flops = chunk_flops(wl, L0.seq_lens_list, T)
+        peak, kind = measured_tensor_peak()
+        achieved = flops / t_att / 1e12
+        entry = {
+            "config": {"B": wl.B, "Hq": wl.Hq, "Hk": wl.Hk, "D": wl.D, "q_len": T,
+                       "seq_len": L0.hint, "scale_mode": wl.mode, "layout": wl.layout},
+            "repeats": reps, "statistic": "median over repeats",
+            "attention_ms": round(t_att * 1e3, 4), "append_us": round(t_app * 1e6, 3),
+            "append_gbs": round(world * append_bytes(wl, T) / t_app / 1e9, 2),
+            "tokens_per_s": round(world * wl.B * T / (t_app + t_att), 1),
+            "useful_flops": int(flops),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                         "peak_source": f"{kind} dense bf16 (MEASURED_PEAKS.json bf16_tflops)",
+                         "kernel_ceiling_frac": round(2 / 3, 4)},
+            "clocks": sampler.summary(),
+        }
+        gw.close()
+        return entry
+    finally:
+        QLEN = saved
+
+
 def run_kvq(args, wl):
     import torch.distributed as dist
 
@@ -725,6 +783,8 @@ def run_kvq(args, wl):
         for name, w in synth.ALL_WORKLOADS.items():
             pc[name] = per_config_entry(kvq, w, dev, K, W, world,
                                         gw=gw if name == wl.name else None)
+        pc["long_context_prefill2048"] = prefill_entry(kvq, synth.WORKLOADS["long_context"], dev,
+                                                       K, W, world, 2048)
         line["per_config"] = pc
     gw.close()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

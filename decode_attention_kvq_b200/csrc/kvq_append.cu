@@ -9,9 +9,11 @@
 // 0.8.5 kv_cache_q8_init.rs and combs-models 0.2.2 kv.rs kv_quantize):
 //   m = max(max_i |x_i|, 1e-8);  s = m / 127;
 //   byte_i = clamp(round_half_away(x_i / s) + 128, 0, 255);  scale = s (fp32).
-// Both divisions are IEEE round-to-nearest fp32 divisions (__fdiv_rn), and
-// roundf rounds half away from zero, so the bytes and scales are bit-exact
-// with that definition.
+// Both divisions are IEEE round-to-nearest fp32 divisions, and roundf rounds
+// half away from zero, so the bytes and scales are bit-exact with that
+// definition; the per-element quotient is taken by a reciprocal multiply
+// except within 1e-4 of a rounding tie (round_quotient), which gives the same
+// byte.
 //
 // Mapping: one "row" is the D values of one (which in {K, V}, b, h, t).  A
 // row is handled by P = next_pow2(D / 8) lanes of a warp, each lane loading
@@ -24,6 +26,21 @@
 
 namespace kvq {
 namespace {
+
+// round_half_away(x / s) for the IEEE-rounded fp32 quotient x / s, mostly
+// without a division.  r = x * inv, inv = 1 / s rounded once and the product
+// rounded once, is within 2^-23 |x / s| of the quotient, i.e. within 2.3e-5
+// of the rounded quotient wherever |x / s| <= 128 (every in-range byte).  So
+// unless r lies within 1e-4 of a point halfway between two integers, the
+// rounded quotient lies strictly inside the same interval (k - 0.5, k + 0.5)
+// and rounds to the same integer as r; those near-ties take the IEEE division.
+// Beyond |x / s| = 128 both roundings clamp to the same byte.
+__device__ __forceinline__ int round_quotient(float x, float s, float inv) {
+    const float r = __fmul_rn(x, inv);
+    const float a = fabsf(r);
+    if (fabsf(a - floorf(a) - 0.5f) < 1e-4f) return static_cast<int>(roundf(__fdiv_rn(x, s)));
+    return static_cast<int>(roundf(r));
+}
 
 constexpr int kAppendThreads = 256;
 
@@ -112,7 +129,7 @@ append_kernel(AppendParams p, int lanes_log2) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const float si = sc[p.static_ns > 1 ? sub * 8 + i : 0];
-            int v = static_cast<int>(roundf(__fdiv_rn(x[i], si))) + 128;
+            int v = round_quotient(x[i], si, __frcp_rn(si)) + 128;
             v = v < 0 ? 0 : (v > 255 ? 255 : v);
             packed[i >> 2] |= static_cast<uint32_t>(v) << (8 * (i & 3));
         }
@@ -128,10 +145,11 @@ append_kernel(AppendParams p, int lanes_log2) {
     if (!active || dst_row < 0) return;
     const float m = amax < 1e-8f ? 1e-8f : amax;
     const float s = __fdiv_rn(m, 127.0f);
+    const float inv = __frcp_rn(s);
     uint32_t packed[2] = {0u, 0u};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        int v = static_cast<int>(roundf(__fdiv_rn(x[i], s))) + 128;
+        int v = round_quotient(x[i], s, inv) + 128;
         v = v < 0 ? 0 : (v > 255 ? 255 : v);
         packed[i >> 2] |= static_cast<uint32_t>(v) << (8 * (i & 3));
     }
@@ -200,10 +218,11 @@ calibrate_kernel(AppendParams p) {
     __syncthreads();
     if (!act) return;
     const float s = scl[p.static_ns > 1 ? c : 0];
+    const float inv = __frcp_rn(s);
     uint8_t* dst = (which ? p.v_dst : p.k_dst) + (static_cast<int64_t>(bh) * p.max_seq + p0) * D;
     for (int t = r; t < T; t += lanes) {
         const float xv = bf16_bits_to_f32(x[static_cast<int64_t>(t) * D + c]);
-        int v = static_cast<int>(roundf(__fdiv_rn(xv, s))) + 128;
+        int v = round_quotient(xv, s, inv) + 128;
         v = v < 0 ? 0 : (v > 255 ? 255 : v);
         dst[static_cast<int64_t>(t) * D + c] = static_cast<uint8_t>(v);
     }
@@ -279,7 +298,7 @@ append_mixed_kernel(AppendParams p, uint16_t* k_ring, uint16_t* v_ring, int W) {
             uint32_t packed[2] = {0u, 0u};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                int v = static_cast<int>(roundf(__fdiv_rn(xv[i], sc[i]))) + 128;
+                int v = round_quotient(xv[i], sc[i], __frcp_rn(sc[i])) + 128;
                 v = v < 0 ? 0 : (v > 255 ? 255 : v);
                 packed[i >> 2] |= static_cast<uint32_t>(v) << (8 * (i & 3));
             }

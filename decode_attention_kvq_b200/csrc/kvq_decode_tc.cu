@@ -62,6 +62,7 @@
 //    which every wait of the CTA returns at once); barriers are reached by
 //    every participating thread unconditionally.
 #include <cuda.h>
+#include <cuda_fp8.h>
 #include <math.h>
 
 #include <atomic>
@@ -106,20 +107,18 @@ __device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint
 
 // Two FP8 bytes of w (bytes 0, 1 when hi == 0, bytes 2, 3 when hi == 1) ->
 // f16x2 holding their exact values.  F8 == 2 (E5M2): the byte is the top
-// byte of the f16 of the same value.  F8 == 1 (E4M3): the sign stays at bit
-// 15 and the 7 magnitude bits go to bits 7..13, which reads as the value
-// times 2^-8 (normal and subnormal codes alike, the biases being 7 and 15);
-// one f16x2 multiply by 256 (exact) restores it.
+// byte of the f16 of the same value.  F8 == 1 (E4M3): the hardware fp8x2 ->
+// f16x2 conversion.
 template <int F8>
 __device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t w, int hi) {
-    const uint32_t y = ptx::prmt(w, 0u, hi ? 0x3424u : 0x1404u);
     if constexpr (F8 == 2) {
-        return y;
+        return ptx::prmt(w, 0u, hi ? 0x3424u : 0x1404u);
     } else {
-        const uint32_t r = ((y >> 1) & 0x3f803f80u) | (y & 0x80008000u);
-        uint32_t out;
-        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out) : "r"(r), "r"(0x5c005c00u));
-        return out;
+        // the two bytes as an fp8x2 value (first byte in the low half), one
+        // hardware conversion to f16x2 (exact: E4M3 values are f16 values)
+        const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+            static_cast<__nv_fp8x2_storage_t>((w >> (hi ? 16 : 0)) & 0xffffu), __NV_E4M3);
+        return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
     }
 }
 

@@ -134,3 +134,25 @@ def test_dequant_roundtrip_of_appended_cache():
     # half-step bound against the bf16 source
     bound = c.oks.repeat_interleave(32, dim=-1) * (0.5 + 2.0 ** -18 + 2.0 ** -17)
     assert torch.all((ref - k.float()).abs() <= bound)
+
+
+@pytest.mark.parametrize("mode", ["per_token", "group32"])
+def test_append_ties_and_large_sweep_bit_exact(mode):
+    """The quotient x / s is taken by a reciprocal multiply away from rounding
+    ties and by the IEEE division near them: rows of exact ties (max 127, so
+    s = 1 and x = k + 0.5), rows of values that are ties only up to bf16
+    rounding, and a sweep of 2M values over many magnitudes, all bit-exact."""
+    B, Hk, T, D = 2, 4, 2048, 128
+    g = torch.Generator().manual_seed(77)
+    x = torch.randn(B, Hk, T, D, generator=g) * torch.pow(
+        2.0, torch.randint(-12, 12, (B, Hk, T, 1), generator=g).float())
+    k = torch.randint(-127, 127, (B, Hk, 64, D), generator=g).float()
+    x[:, :, :64] = k + 0.5                                   # exact ties (s = 1)
+    x[:, :, :64, 0] = 127.0
+    m = torch.rand(B, Hk, 64, 1, generator=g) * 10 + 0.1     # near-ties after bf16 rounding
+    x[:, :, 64:128] = (k + 0.5) * m / 127.0
+    x[:, :, 64:128, 0] = m[..., 0]
+    xb = x.to(torch.bfloat16)
+    c = ContigCache(B, Hk, T, D, mode)
+    assert c.append(xb, -xb, torch.zeros(B, dtype=torch.int32)) == 0
+    c.assert_bit_exact()
