@@ -352,6 +352,30 @@ class Layer:
             kvq.kvq_append(k_new, v_new, self.pos, self.k, self.v, self.ks, self.vs,
                            self.wl.mode, stream=stream)
 
+    @property
+    def fusable(self):
+        """The step can run as one kvq_append_decode call (INT8 per-token or
+        group-32 decode without a window or a bf16 recent window)."""
+        wl = self.wl
+        return (self.qlen == 1 and not wl.window and not wl.recent and
+                wl.mode in ("per_token", "group32"))
+
+    def step_fused(self, kvq, workspace, k_new=None, v_new=None, q=None, out=None, stream=None):
+        """The decode step through the one-call entry point: the new token is
+        quantised inside the decode kernel (the prefill-chunk re-append of the
+        long-context workload stays its own call)."""
+        k_new = self.k_new if k_new is None else k_new
+        v_new = self.v_new if v_new is None else v_new
+        q = self.q if q is None else q
+        out = self.out if out is None else out
+        if self.chunk_T:
+            kvq.kvq_append(self.chunk_k, self.chunk_v, self.chunk_pos, self.k, self.v, self.ks,
+                           self.vs, self.wl.mode, stream=stream)
+        kvq.kvq_append_decode(q, k_new, v_new, self.k, self.v, self.ks, self.vs, self.seq_lens,
+                              self.hint, page_table=self.table,
+                              page_size=16 if self.paged else 0, view=self.view,
+                              mode=self.wl.mode, out=out, workspace=workspace, stream=stream)
+
     def decode(self, kvq, workspace, q=None, out=None, stream=None):
         q = self.q if q is None else q
         out = self.out if out is None else out
@@ -545,7 +569,7 @@ class GpuWorkload:
         L0 = self.layers[0]
         self.hint = L0.hint
         ws_bytes = L0.workspace_bytes(kvq)
-        self.workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.workspace = kvq.new_workspace(max(ws_bytes, 16), dev)
         self.chunk, self.splits = kvq.kvq_decode_plan(wl.B, wl.Hk, L0.hint)
         # append (+ prefill-chunk append) + split kernel (+ combine kernel when a
         # sequence spans several chunks: then the call has a workspace)
@@ -564,6 +588,17 @@ class GpuWorkload:
         with torch.cuda.graph(self.g_decode, stream=self.stream):
             for ly in self.layers:
                 ly.decode(kvq, self.workspace)
+        # the same step through the one-call entry point, where it applies
+        self.g_fused = None
+        if L0.fusable:
+            with torch.cuda.stream(self.stream):
+                for ly in self.layers:
+                    ly.step_fused(kvq, self.workspace)
+            torch.cuda.synchronize(dev)
+            self.g_fused = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.g_fused, stream=self.stream):
+                for ly in self.layers:
+                    ly.step_fused(kvq, self.workspace)
         torch.cuda.synchronize(dev)
         self.dec_b = sum(decode_bytes(wl, ly.seq_lens_list, 16 if ly.paged else 0)
                          for ly in self.layers)
@@ -593,8 +628,43 @@ class GpuWorkload:
         per = [(e[0].elapsed_time(e[1]) / 1e3, e[1].elapsed_time(e[2]) / 1e3) for e in ev]
         return per, ev[0][0].elapsed_time(ev[-1][2]) / 1e3
 
+    def timed_fused(self, reps, sampler):
+        """reps one-call steps (g_fused), each bracketed by CUDA events on the
+        launching stream: per-step seconds."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        with torch.cuda.stream(self.stream):
+            for _ in range(3):
+                self.g_fused.replay()
+        with sampler:
+            with torch.cuda.stream(self.stream):
+                for i in range(reps):
+                    ev[i][0].record(self.stream)
+                    self.g_fused.replay()
+                    ev[i][1].record(self.stream)
+            torch.cuda.synchronize(self.dev)
+        return [e[0].elapsed_time(e[1]) / 1e3 for e in ev]
+
+    def fused_entry(self, reps, world, dev):
+        """The one-call step: per-layer time, tokens/s per layer and the bytes it
+        moves (decode + append) against the HBM roofline; median over reps."""
+        if self.g_fused is None:
+            return None
+        sampler = ClockSampler(physical_gpu_index(dev.index))
+        per = self.timed_fused(reps, sampler)
+        t = reduce_max(statistics.median(per), dev)
+        pl = t / self.n_layers
+        moved = (self.dec_b + self.app_b) / self.n_layers
+        achieved = moved / pl / 1e9
+        peak, _ = measured_peaks()
+        return {"call": "kvq_append_decode (new token quantised inside the decode kernel)",
+                "repeats": reps, "statistic": "median over repeats",
+                "us_per_layer": round(pl * 1e6, 3),
+                "tokens_per_s_per_layer": round(world * self.wl.B * QLEN / pl, 1),
+                "bytes_per_layer": int(moved), "gbs": round(world * achieved, 2),
+                "frac": round(achieved / peak, 4), "clocks": sampler.summary()}
+
     def close(self):
-        del self.g_append, self.g_decode
+        del self.g_append, self.g_decode, self.g_fused
         self.layers = None
         self.workspace = None
         torch.cuda.synchronize(self.dev)
@@ -639,6 +709,7 @@ def per_config_entry(kvq, wl, dev, K, W, world, gw=None):
     pl_app = t_app / gw.n_layers
     achieved = gw.dec_b / gw.n_layers / pl_dec / 1e9
     e2e = run_e2e(kvq, wl, gw.layers, gw.workspace, dev, min(K, 20), W, world)
+    fused = gw.fused_entry(reps, world, dev)
     entry = {
         "config": {"B": wl.B, "Hq": wl.Hq, "Hk": wl.Hk, "D": wl.D, "seq_len": gw.hint,
                    "scale_mode": wl.mode, "layout": wl.layout, "layers_per_step": gw.n_layers,
@@ -656,8 +727,12 @@ def per_config_entry(kvq, wl, dev, K, W, world, gw=None):
         "decode_gbs": round(world * achieved, 2),
         "roofline": roofline(wl, achieved),
         "append_gbs": round(world * gw.app_b / t_app / 1e9, 2),
-        "tokens_per_s_per_layer": round(wl.B * QLEN / (pl_app + pl_dec), 1),
+        "tokens_per_s_per_layer": round(world * wl.B * QLEN /
+                                        min(pl_app + pl_dec,
+                                            fused["us_per_layer"] * 1e-6 if fused else 1e9), 1),
+        "tokens_per_s_per_layer_two_calls": round(world * wl.B * QLEN / (pl_app + pl_dec), 1),
         "algorithmic_bytes_per_decode_call": int(gw.dec_b / gw.n_layers),
+        "fused_step": fused,
         "e2e": e2e,
         "clocks": sampler.summary(),
     }
@@ -754,6 +829,9 @@ def run_kvq(args, wl):
 
     # ---- end to end through the public API from pinned host buffers
     e2e = run_e2e(kvq, wl, gw.layers, gw.workspace, dev, K, W, world)
+    # ---- the same step as one call per layer (new token quantised inside the
+    # decode kernel), K more steps
+    fused = gw.fused_entry(max(K, 10), world, dev)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -767,7 +845,11 @@ def run_kvq(args, wl):
                    "l2": ("inputs larger than L2 (%.0f MB per step)"
                           % ((gw.dec_b + gw.app_b) / 1e6)),
                    "split_chunk": gw.chunk, "splits": gw.splits},
-        "tokens_per_s_per_layer": round(tokens_per_s_per_layer, 1),
+        "tokens_per_s_per_layer": round(world * max(tokens_per_s_per_layer,
+                                                    fused["tokens_per_s_per_layer"] / world
+                                                    if fused else 0.0), 1),
+        "tokens_per_s_per_layer_two_calls": round(world * tokens_per_s_per_layer, 1),
+        "fused_step": fused,
         "append_gbs": round(append_gbs, 2),
         "decode_us_per_layer": round(per_layer_decode * 1e6, 3),
         "append_us_per_layer": round(per_layer_append * 1e6, 3),
@@ -799,8 +881,9 @@ def run_kvq(args, wl):
 def run_e2e(kvq, wl, layers, workspace, dev, K, W, world):
     """Same metric through the public Python API with host buffers: each step
     copies every layer's q / k_new / v_new from pinned host memory (one packed
-    copy for the step), runs kvq_append + kvq_decode_attn eagerly for every
-    layer, and copies all the outputs back (one packed copy)."""
+    copy for the step), runs the decode step eagerly for every layer (one
+    kvq_append_decode call where the cache format allows, else kvq_append +
+    kvq_decode_attn), and copies all the outputs back (one packed copy)."""
     n = len(layers)
     # the step's inputs, packed layer after layer: q, k_new, v_new (bf16)
     parts = [t for ly in layers for t in (ly.q, ly.k_new, ly.v_new)]
@@ -826,8 +909,12 @@ def run_e2e(kvq, wl, layers, workspace, dev, K, W, world):
             d_in.copy_(h_in, non_blocking=True)
             for i, ly in enumerate(layers):
                 q, k_new, v_new = views[3 * i:3 * i + 3]
-                ly.append(kvq, k_new, v_new, stream=stream)
-                ly.decode(kvq, workspace, q=q, out=out_views[i], stream=stream)
+                if ly.fusable:
+                    ly.step_fused(kvq, workspace, k_new, v_new, q=q, out=out_views[i],
+                                  stream=stream)
+                else:
+                    ly.append(kvq, k_new, v_new, stream=stream)
+                    ly.decode(kvq, workspace, q=q, out=out_views[i], stream=stream)
             h_out.copy_(d_out, non_blocking=True)
 
     for _ in range(max(W, 1)):

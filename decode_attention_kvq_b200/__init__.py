@@ -180,6 +180,11 @@ def cache_view(k, v, k_scale, v_scale, page_table=None, page_size=0) -> CacheVie
     return cv
 
 
+def new_workspace(nbytes, device) -> torch.Tensor:
+    """A split-K workspace of nbytes bytes (its contents are scratch)."""
+    return torch.empty(int(nbytes), dtype=torch.uint8, device=device)
+
+
 def kvq_decode_workspace_bytes(B, Hq, Hk, D, max_seq_len_hint, num_splits=0) -> int:
     return int(lib.kvq_decode_workspace_bytes(B, Hq, Hk, D, max_seq_len_hint, num_splits))
 
@@ -214,7 +219,7 @@ def kvq_decode_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *, Hk
     if workspace is None:               # (a given workspace's size is checked by the call)
         need = kvq_decode_workspace_bytes(B, Hq, Hk, D, max_seq_len_hint, num_splits)
         if need > 0:
-            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+            workspace = new_workspace(need, q.device)
     ws_ptr = _ptr(workspace, None, "workspace") if workspace is not None else 0
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     check(lib.kvq_decode_attn(
@@ -222,6 +227,39 @@ def kvq_decode_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *, Hk
         _ptr(seq_lens, torch.int32, "seq_lens"), int(max_seq_len_hint), float(attn_scale),
         _ptr(out, torch.float32, "out"), ws_ptr, ws_bytes, int(num_splits),
         _ptr(err, torch.int32, "err"), _stream(stream, q)), "kvq_decode_attn")
+    return out
+
+
+def kvq_append_decode(q, k_new, v_new, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *,
+                      Hk=None, page_table=None, page_size=0, attn_scale=None,
+                      mode="per_token", out=None, workspace=None, num_splits=0, err=None,
+                      stream=None, view: Optional[CacheView] = None):
+    """One decode step in one call: k_new / v_new bf16 [B,Hk,1,D] are quantised
+    into position seq_lens[b] - 1 of the cache (written in place), then q bf16
+    [B,Hq,D] attends to positions 0 .. seq_lens[b] - 1; returns fp32 [B,Hq,D].
+    seq_lens counts the tokens INCLUDING the new one.  Cache arguments as for
+    kvq_decode_attn (per_token or group32 mode)."""
+    B, Hq, D = q.shape
+    if Hk is None:
+        Hk = k.shape[1]
+    if attn_scale is None:
+        attn_scale = 1.0 / math.sqrt(D)
+    if view is None:
+        view = cache_view(k, v, k_scale, v_scale, page_table, page_size)
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
+    if workspace is None:               # (a given workspace's size is checked by the call)
+        need = kvq_decode_workspace_bytes(B, Hq, Hk, D, max_seq_len_hint, num_splits)
+        if need > 0:
+            workspace = new_workspace(need, q.device)
+    ws_ptr = _ptr(workspace, None, "workspace") if workspace is not None else 0
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    check(lib.kvq_append_decode(
+        _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
+        _ptr(v_new, torch.bfloat16, "v_new"), B, Hq, Hk, D, _mode(mode), ctypes.byref(view),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(max_seq_len_hint), float(attn_scale),
+        _ptr(out, torch.float32, "out"), ws_ptr, ws_bytes, int(num_splits),
+        _ptr(err, torch.int32, "err"), _stream(stream, q)), "kvq_append_decode")
     return out
 
 
@@ -247,7 +285,7 @@ def kvq_chunk_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, *, Hk=
     if workspace is None:               # (a given workspace's size is checked by the call)
         need = kvq_chunk_workspace_bytes(B, Hq, Hk, T, D, max_seq_len_hint, num_splits)
         if need > 0:
-            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+            workspace = new_workspace(need, q.device)
     ws_ptr = _ptr(workspace, None, "workspace") if workspace is not None else 0
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     check(lib.kvq_chunk_attn(
@@ -287,7 +325,7 @@ def kvq_window_attn(q, k, v, k_scale, v_scale, seq_lens, max_seq_len_hint, windo
         need = int(lib.kvq_window_workspace_bytes(B, Hq, Hk, T, D, int(max_seq_len_hint),
                                                   int(window), int(num_splits)))
         if need > 0:
-            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+            workspace = new_workspace(need, q.device)
     ws_ptr = _ptr(workspace, None, "workspace") if workspace is not None else 0
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     check(lib.kvq_window_attn(

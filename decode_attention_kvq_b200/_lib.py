@@ -30,6 +30,8 @@ _PROTOS = {
                                    _SZ, _I, _P, _P]),
     "kvq_mixed_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "kvq_decode_attn": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _SZ, _I, _P, _P]),
+    "kvq_append_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _SZ, _I,
+                               _P, _P]),
     "kvq_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "kvq_chunk_attn": (_I, [_P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _SZ, _I, _P,
                             _P]),

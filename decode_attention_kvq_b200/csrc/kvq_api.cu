@@ -87,6 +87,7 @@ kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk
     return KVQ_OK;
 }
 
+// [o: n_part * D][m: n_part][l: n_part] floats
 size_t workspace_for(int B, int Hq, int D, int splits) {
     if (splits <= 1) return 0;
     return static_cast<size_t>(B) * Hq * splits * (D + 2) * sizeof(float);
@@ -114,7 +115,8 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
                   const kvq_cache_view* kv, const int32_t* d_seq_lens, int max_seq_len_hint,
                   int window, float attn_scale, float* out, void* workspace,
                   size_t workspace_bytes, int num_splits, int32_t* d_err, kvq_stream_t stream,
-                  int recent = 0, const uint16_t* rk = nullptr, const uint16_t* rv = nullptr) {
+                  int recent = 0, const uint16_t* rk = nullptr, const uint16_t* rv = nullptr,
+                  const uint16_t* k_new = nullptr, const uint16_t* v_new = nullptr) {
     if (window < 0 || recent < 0) return KVQ_ERR_INVALID_ARG;
     if (!valid_mode(mode)) return KVQ_ERR_INVALID_ARG;
     if (!q || !kv || !kv->k || !kv->v || !d_seq_lens || !out) return KVQ_ERR_INVALID_ARG;
@@ -139,12 +141,12 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
         return KVQ_ERR_INVALID_ARG;
     if (Hq > 65535) return KVQ_ERR_UNSUPPORTED;
     // more than 16 (head, query) rows per kv head: the dense chunk kernel on
-    // the tcgen05 tensor cores
+    // the tcgen05 tensor cores where it covers the shape (otherwise the
+    // CUDA-core split kernel below)
     const bool dense = static_cast<int64_t>(Hq / Hk) * T > 16;
-    if (dense) {
-        if (!kvq::chunk_tc_supported(D, Hq / Hk, T, mode == KVQ_SCALE_GROUP32, is_fp8(mode),
-                                     static_ns(mode, D), kv->page_size, window, recent))
-            return KVQ_ERR_UNSUPPORTED;
+    if (dense && !k_new &&
+        kvq::chunk_tc_supported(D, Hq / Hk, T, mode == KVQ_SCALE_GROUP32, is_fp8(mode),
+                                static_ns(mode, D), kv->page_size, window, recent)) {
         if (static_cast<int64_t>(B) * Hq * T >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
         if (B == 0) return KVQ_OK;
         if (static_cast<int64_t>(B) * Hk * kv->max_seq >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
@@ -155,14 +157,18 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
         p.scale_log2 = attn_scale * 1.4426950408889634f;
         return from_cuda(kvq::launch_chunk_tc(p, Hq, Hq / Hk, T, static_cast<cudaStream_t>(stream)));
     }
+    if (static_cast<int64_t>(Hq / Hk) * T > (1ll << 19)) return KVQ_ERR_UNSUPPORTED;
     const int G = Hq / Hk * T;          // rows per kv head: (head, query), query fastest
-    if (D != 64 && D != 128) return KVQ_ERR_UNSUPPORTED;
-    // the split kernel keeps every sequence length in shared memory
-    if (B > kvq::kMaxBatch) return KVQ_ERR_UNSUPPORTED;
-    // TMA row coordinates are 32-bit
+    // The tensor-core split kernel takes D 64 / 128, at most 16 rows per kv
+    // head, at most kMaxBatch sequences (their lengths sit in shared memory)
+    // and caches whose TMA row coordinates fit 32 bits; every other shape runs
+    // on the CUDA-core split kernel.
     const int64_t rows = kv->page_size ? static_cast<int64_t>(kv->num_pages) * Hk * 16
                                        : static_cast<int64_t>(B) * Hk * kv->max_seq;
-    if (rows >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+    const bool simt = dense || (D != 64 && D != 128) || B > kvq::kMaxBatch ||
+                      rows >= (1ll << 31);
+    // the mixed cache's window kernel folds at most 16 rows per kv head
+    if (recent && G > 16) return KVQ_ERR_UNSUPPORTED;
     if (B == 0) return KVQ_OK;
 
     int chunk = 0, splits = 0;
@@ -186,6 +192,11 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
     p.ws_o = ws;
     p.ws_m = ws ? ws + n_part * D : nullptr;
     p.ws_l = ws ? ws + n_part * (D + 1) : nullptr;
+    if (k_new) {                        // fused append: the view's arrays are written
+        p.k_new = k_new; p.v_new = v_new;
+        p.k_w = const_cast<uint8_t*>(kv->k); p.v_w = const_cast<uint8_t*>(kv->v);
+        p.ks_w = const_cast<float*>(kv->k_scale); p.vs_w = const_cast<float*>(kv->v_scale);
+    }
     p.B = B; p.Hq = Hq * T; p.Hk = Hk; p.G = G; p.D = D; p.group32 = mode == KVQ_SCALE_GROUP32;
     p.fp8 = fp8_code(mode);
     p.static_ns = static_ns(mode, D);
@@ -196,7 +207,10 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
     p.rv = rv;
     p.page_size = kv->page_size; p.max_seq = kv->max_seq; p.max_pages = kv->max_pages;
     p.num_pages = kv->num_pages; p.chunk = chunk; p.splits = splits;
-    {
+    if (simt) {
+        p.grid = 0;                     // one CTA per item (and block of rows)
+        p.one_item = 1;
+    } else {
         int dev = 0, sms = 0;
         if (cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -214,12 +228,13 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
     if (recent) {                       // mixed cache: INT8 partials, then the window kernel
         const cudaStream_t cs = static_cast<cudaStream_t>(stream);
         if (hint > 0) {
-            const cudaError_t e = kvq::launch_decode_split_tc(p, cs);
+            const cudaError_t e = simt ? kvq::launch_decode_simt(p, cs)
+                                       : kvq::launch_decode_split_tc(p, cs);
             if (e != cudaSuccess) return KVQ_ERR_CUDA;
         }
         return from_cuda(kvq::launch_recent_combine(p, cs));
     }
-    return from_cuda(kvq::launch_decode(p, static_cast<cudaStream_t>(stream)));
+    return from_cuda(kvq::launch_decode(p, static_cast<cudaStream_t>(stream), simt));
 }
 
 }  // namespace
@@ -306,6 +321,20 @@ kvq_status kvq_decode_attn(const uint16_t* q, int B, int Hq, int Hk, int D, kvq_
                   workspace, workspace_bytes, num_splits, d_err, stream);
 }
 
+kvq_status kvq_append_decode(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                             int B, int Hq, int Hk, int D, kvq_scale_mode mode,
+                             const kvq_cache_view* kv, const int32_t* d_seq_lens,
+                             int max_seq_len_hint, float attn_scale, float* out, void* workspace,
+                             size_t workspace_bytes, int num_splits, int32_t* d_err,
+                             kvq_stream_t stream) {
+    if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return KVQ_ERR_INVALID_ARG;
+    if (!valid_mode(mode)) return KVQ_ERR_INVALID_ARG;
+    if (mode != KVQ_SCALE_PER_TOKEN && mode != KVQ_SCALE_GROUP32) return KVQ_ERR_UNSUPPORTED;
+    return attend(q, B, Hq, Hk, 1, D, mode, kv, d_seq_lens, max_seq_len_hint, 0, attn_scale, out,
+                  workspace, workspace_bytes, num_splits, d_err, stream, 0, nullptr, nullptr,
+                  k_new, v_new);
+}
+
 kvq_status kvq_chunk_attn(const uint16_t* q, int B, int Hq, int Hk, int T, int D,
                           kvq_scale_mode mode, const kvq_cache_view* kv,
                           const int32_t* d_seq_lens, int max_seq_len_hint, float attn_scale,
@@ -383,7 +412,8 @@ size_t kvq_window_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_s
 size_t kvq_chunk_workspace_bytes(int B, int Hq, int Hk, int T, int D, int max_seq_len_hint,
                                  int num_splits) {
     if (T < 1 || Hq > INT32_MAX / T || Hk < 1) return 0;
-    if (static_cast<int64_t>(Hq / Hk) * T > 16) return 0;   // the dense kernel needs none
+    // (above 16 rows per kv head the dense kernel needs none, but the shapes it
+    // does not cover run on the CUDA-core split kernel, which does)
     return kvq_decode_workspace_bytes(B, Hq * T, Hk, D, max_seq_len_hint, num_splits);
 }
 

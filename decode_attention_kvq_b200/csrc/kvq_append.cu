@@ -12,8 +12,8 @@
 // Both divisions are IEEE round-to-nearest fp32 divisions, and roundf rounds
 // half away from zero, so the bytes and scales are bit-exact with that
 // definition; the per-element quotient is taken by a reciprocal multiply
-// except within 1e-4 of a rounding tie (round_quotient), which gives the same
-// byte.
+// except within 1e-4 of a rounding tie (round_quotient in kvq_internal.cuh),
+// which gives the same byte.
 //
 // Mapping: one "row" is the D values of one (which in {K, V}, b, h, t).  A
 // row is handled by P = next_pow2(D / 8) lanes of a warp, each lane loading
@@ -26,21 +26,6 @@
 
 namespace kvq {
 namespace {
-
-// round_half_away(x / s) for the IEEE-rounded fp32 quotient x / s, mostly
-// without a division.  r = x * inv, inv = 1 / s rounded once and the product
-// rounded once, is within 2^-23 |x / s| of the quotient, i.e. within 2.3e-5
-// of the rounded quotient wherever |x / s| <= 128 (every in-range byte).  So
-// unless r lies within 1e-4 of a point halfway between two integers, the
-// rounded quotient lies strictly inside the same interval (k - 0.5, k + 0.5)
-// and rounds to the same integer as r; those near-ties take the IEEE division.
-// Beyond |x / s| = 128 both roundings clamp to the same byte.
-__device__ __forceinline__ int round_quotient(float x, float s, float inv) {
-    const float r = __fmul_rn(x, inv);
-    const float a = fabsf(r);
-    if (fabsf(a - floorf(a) - 0.5f) < 1e-4f) return static_cast<int>(roundf(__fdiv_rn(x, s)));
-    return static_cast<int>(roundf(r));
-}
 
 constexpr int kAppendThreads = 256;
 
@@ -61,9 +46,13 @@ append_kernel(AppendParams p, int lanes_log2) {
 
     const int which = row_ok && row >= rows_per_tensor;    // 0: K, 1: V
     const int64_t r = row_ok ? row - which * rows_per_tensor : 0;
-    const int t = static_cast<int>(r % p.T);
-    const int h = static_cast<int>((r / p.T) % p.Hk);
-    const int b = static_cast<int>(r / (static_cast<int64_t>(p.T) * p.Hk));
+    // (row, kv head, token) in 32-bit arithmetic (the host keeps 2 B Hk T
+    // below 2^31): 64-bit divisions would cost more than the rest of the row
+    const uint32_t r32 = static_cast<uint32_t>(r);
+    const uint32_t bh = r32 / static_cast<uint32_t>(p.T);
+    const int t = static_cast<int>(r32 - bh * static_cast<uint32_t>(p.T));
+    const int b = static_cast<int>(bh / static_cast<uint32_t>(p.Hk));
+    const int h = static_cast<int>(bh - static_cast<uint32_t>(b) * static_cast<uint32_t>(p.Hk));
 
     // ---- destination row (skip and flag when out of range)
     int64_t dst_row = -1;
@@ -129,9 +118,7 @@ append_kernel(AppendParams p, int lanes_log2) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const float si = sc[p.static_ns > 1 ? sub * 8 + i : 0];
-            int v = round_quotient(x[i], si, __frcp_rn(si)) + 128;
-            v = v < 0 ? 0 : (v > 255 ? 255 : v);
-            packed[i >> 2] |= static_cast<uint32_t>(v) << (8 * (i & 3));
+            packed[i >> 2] |= q8_byte(x[i], si, __frcp_rn(si)) << (8 * (i & 3));
         }
         uint8_t* dst = (which ? p.v_dst : p.k_dst) + dst_row * p.D + sub * 8;
         *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
@@ -143,16 +130,11 @@ append_kernel(AppendParams p, int lanes_log2) {
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
 
     if (!active || dst_row < 0) return;
-    const float m = amax < 1e-8f ? 1e-8f : amax;
-    const float s = __fdiv_rn(m, 127.0f);
+    const float s = q8_scale(amax);
     const float inv = __frcp_rn(s);
     uint32_t packed[2] = {0u, 0u};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        int v = round_quotient(x[i], s, inv) + 128;
-        v = v < 0 ? 0 : (v > 255 ? 255 : v);
-        packed[i >> 2] |= static_cast<uint32_t>(v) << (8 * (i & 3));
-    }
+    for (int i = 0; i < 8; ++i) packed[i >> 2] |= q8_byte(x[i], s, inv) << (8 * (i & 3));
     uint8_t* dst = (which ? p.v_dst : p.k_dst) + dst_row * p.D + sub * 8;
     *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
     float* sdst = which ? p.v_scale : p.k_scale;
@@ -200,7 +182,7 @@ calibrate_kernel(AppendParams p) {
     if (p.static_ns > 1) {                       // per channel: over the token lanes
         if (act && r == 0) {
             for (int k = 1; k < lanes; ++k) m = fmaxf(m, red[k * D + c]);
-            const float s = __fdiv_rn(m < 1e-8f ? 1e-8f : m, 127.0f);
+            const float s = q8_scale(m);
             scl[c] = s;
             sc[c] = s;
         }
@@ -210,7 +192,7 @@ calibrate_kernel(AppendParams p) {
             __syncthreads();
         }
         if (tid == 0) {
-            const float s = __fdiv_rn(red[0] < 1e-8f ? 1e-8f : red[0], 127.0f);
+            const float s = q8_scale(red[0]);
             scl[0] = s;
             sc[0] = s;
         }
@@ -222,9 +204,7 @@ calibrate_kernel(AppendParams p) {
     uint8_t* dst = (which ? p.v_dst : p.k_dst) + (static_cast<int64_t>(bh) * p.max_seq + p0) * D;
     for (int t = r; t < T; t += lanes) {
         const float xv = bf16_bits_to_f32(x[static_cast<int64_t>(t) * D + c]);
-        int v = round_quotient(xv, s, inv) + 128;
-        v = v < 0 ? 0 : (v > 255 ? 255 : v);
-        dst[static_cast<int64_t>(t) * D + c] = static_cast<uint8_t>(v);
+        dst[static_cast<int64_t>(t) * D + c] = static_cast<uint8_t>(q8_byte(xv, s, inv));
     }
 }
 
@@ -282,7 +262,7 @@ append_mixed_kernel(AppendParams p, uint16_t* k_ring, uint16_t* v_ring, int W) {
             const int red = p.group32 ? 4 : 32;
             for (int off = 1; off < red; off <<= 1)
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-            const float s = __fdiv_rn(amax < 1e-8f ? 1e-8f : amax, 127.0f);
+            const float s = q8_scale(amax);
 #pragma unroll
             for (int i = 0; i < 8; ++i) sc[i] = s;
             if (act) {
@@ -297,11 +277,8 @@ append_mixed_kernel(AppendParams p, uint16_t* k_ring, uint16_t* v_ring, int W) {
         if (act) {
             uint32_t packed[2] = {0u, 0u};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                int v = round_quotient(xv[i], sc[i], __frcp_rn(sc[i])) + 128;
-                v = v < 0 ? 0 : (v > 255 ? 255 : v);
-                packed[i >> 2] |= static_cast<uint32_t>(v) << (8 * (i & 3));
-            }
+            for (int i = 0; i < 8; ++i)
+                packed[i >> 2] |= q8_byte(xv[i], sc[i], __frcp_rn(sc[i])) << (8 * (i & 3));
             *reinterpret_cast<uint2*>(dst + g * D + lane * 8) = make_uint2(packed[0], packed[1]);
         }
     }
@@ -350,6 +327,7 @@ cudaError_t launch_append_calibrate(const AppendParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
+    if (2ll * p.B * p.Hk * p.T >= (1ll << 31)) return cudaErrorInvalidValue;   // 32-bit row index
     const int nvec = p.D >> 3;
     int lanes_log2 = 0;
     while ((1 << lanes_log2) < nvec) ++lanes_log2;

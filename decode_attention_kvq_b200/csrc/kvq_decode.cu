@@ -1,7 +1,8 @@
-// kvq_decode.cu -- decode attention driver: the persistent split kernel
-// (kvq_decode_tc.cu) followed, when the plan splits a sequence, by the combine
-// kernel below (launched as a programmatic dependent so its launch overlaps
-// the split kernel).
+// kvq_decode.cu -- decode attention driver: the split kernel (the persistent
+// tensor-core one of kvq_decode_tc.cu, or the CUDA-core one of
+// kvq_decode_simt.cu) followed, when the plan splits a sequence, by the
+// combine kernel below (launched as a programmatic dependent so its launch
+// overlaps the split kernel).
 //
 // Combine (flash-decoding): for each (sequence, q head) whose kv head's
 // chunks were split over several CTAs, the partial states (o_k, m_k, l_k) in
@@ -58,7 +59,8 @@ __device__ __forceinline__ void finish_row(float* out_row, int D, float Mw, floa
 
 // One item per CTA (one_item): CTA c of the split kernel held item c of the
 // plan, so chunk j < ns of every unit holds a partial and nothing else does.
-// One CTA per (b, q head); lane l of a warp owns head_dim [4l, 4l + 4).
+// One CTA per (b, q head) and 128 columns of head_dim (blockIdx.y: columns
+// 128 y ..); lane l of a warp owns columns [4l, 4l + 4) of those.
 __global__ void __launch_bounds__(kThreads)
 decode_combine_one(DecodeParams p) {
     __shared__ float s_m[kWarps], s_l[kWarps];
@@ -71,8 +73,9 @@ decode_combine_one(DecodeParams p) {
     const float* m = p.ws_m + bh * p.splits;
     const float* lv = p.ws_l + bh * p.splits;
     const int D = p.D;
-    const bool active = lane * 4 < D;
-    const float* o = p.ws_o + bh * p.splits * D + lane * 4;
+    const int dh = 128 * static_cast<int>(blockIdx.y);   // this CTA's first column
+    const bool active = dh + lane * 4 < D;
+    const float* o = p.ws_o + bh * p.splits * D + dh + lane * 4;
     const int64_t cap = p.page_size ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
     const int64_t plan = static_cast<int64_t>(p.splits) * p.chunk;
     const int L0 = p.seq_lens[b];
@@ -126,14 +129,15 @@ decode_combine_one(DecodeParams p) {
         load(k0);
         fold(k0, ns);
     }
-    finish_row<false>(p.out + bh * D, D, Mw, lw, acc, s_m, s_l, s_acc);
+    finish_row<false>(p.out + bh * D + dh, min(D - dh, 128), Mw, lw, acc, s_m, s_l, s_acc);
 }
 
 // Blocks of several items per CTA (one_item == 0): a unit's partials are its
 // chunk slots j < ns with finite m.  The first kWords * 32 m slots are loaded
 // together with the length; a ballot per 32 slots picks the live ones, and
 // warp w loads and folds those with j % kWarps == w (at most kBatch per 32
-// slots).  One CTA per (b, q head); lane l of a warp owns head_dim [4l, 4l + 4).
+// slots).  One CTA per (b, q head) and 128 columns of head_dim (blockIdx.y);
+// lane l of a warp owns columns [4l, 4l + 4) of those.
 constexpr int kWords = 4;
 __global__ void __launch_bounds__(kThreads)
 decode_combine_live(DecodeParams p) {
@@ -147,8 +151,9 @@ decode_combine_live(DecodeParams p) {
     const float* m = p.ws_m + bh * p.splits;
     const float* lv = p.ws_l + bh * p.splits;
     const int D = p.D;
-    const bool active = lane * 4 < D;
-    const float* o = p.ws_o + bh * p.splits * D + lane * 4;
+    const int dh = 128 * static_cast<int>(blockIdx.y);   // this CTA's first column
+    const bool active = dh + lane * 4 < D;
+    const float* o = p.ws_o + bh * p.splits * D + dh + lane * 4;
     const int64_t cap = p.page_size ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
     const int64_t plan = static_cast<int64_t>(p.splits) * p.chunk;
     const int L0 = p.seq_lens[b];
@@ -207,7 +212,7 @@ decode_combine_live(DecodeParams p) {
 #pragma unroll 1
     for (int base = 32 * kWords; base < ns; base += 32)
         word(base, base + lane < ns ? m[base + lane] : -INFINITY);
-    finish_row<true>(p.out + bh * D, D, Mw, lw, acc, s_m, s_l, s_acc);
+    finish_row<true>(p.out + bh * D + dh, min(D - dh, 128), Mw, lw, acc, s_m, s_l, s_acc);
 }
 
 // Dynamic shared memory for decode_combine_one so that at most k =
@@ -434,11 +439,11 @@ cudaError_t launch_recent_combine(const DecodeParams& p, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, decode_recent_combine, p);
 }
 
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
-    cudaError_t e = launch_decode_split_tc(p, s);
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s, bool simt) {
+    cudaError_t e = simt ? launch_decode_simt(p, s) : launch_decode_split_tc(p, s);
     if (e != cudaSuccess || p.splits <= 1) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.B * p.Hq, 1, 1);
+    cfg.gridDim = dim3(p.B * p.Hq, (p.D + 127) / 128, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;

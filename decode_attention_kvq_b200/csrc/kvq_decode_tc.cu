@@ -260,10 +260,99 @@ __device__ __forceinline__ Seg seg_at(int i, int iend, const int* lens, const in
 // column i of a sequence of length L sees the positions <= L - T + i (L
 // counts the chunk's tokens) and, with a window w, >= L - T + i - w + 1.
 // With a window the tokens are counted from the sequence's window base.
-template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8, bool ST>
+// Fused append: the warp whose 32-token slice of a landed stage holds the
+// new token (position tok of unit (b, hk), stage row r) quantises it -- the
+// append kernels' quantiser -- into the stage's K and V rows and scales (sk,
+// sv, sks, svs: shared-memory addresses) and into the cache, before any of
+// its MMA operands are read.  Lane l takes head_dim values [l * VPL,
+// (l + 1) * VPL) of k_new and v_new.  Only the fused instantiation of the
+// split kernel (VAR == 2) contains it.
+template <int D, bool G32, bool PAGED>
+__device__ __forceinline__ void patch_new_token(const DecodeParams& p, uint32_t sk, uint32_t sv,
+                                             uint32_t sks, uint32_t svs, int r, int tok, int b,
+                                             int hk) {
+    constexpr int VPL = D / 32;          // values per lane
+    constexpr int NG = G32 ? D / 32 : 1;
+    const int lane = threadIdx.x & 31;
+    uint32_t kx[2] = {0u, 0u}, vx[2] = {0u, 0u};
+    const int64_t nrow = (static_cast<int64_t>(b) * p.Hk + hk) * D + lane * VPL;
+    if constexpr (VPL == 4) {
+        const uint2 a = *reinterpret_cast<const uint2*>(p.k_new + nrow);
+        const uint2 c = *reinterpret_cast<const uint2*>(p.v_new + nrow);
+        kx[0] = a.x; kx[1] = a.y;
+        vx[0] = c.x; vx[1] = c.y;
+    } else {
+        kx[0] = *reinterpret_cast<const uint32_t*>(p.k_new + nrow);
+        vx[0] = *reinterpret_cast<const uint32_t*>(p.v_new + nrow);
+    }
+    float xk[VPL], xv[VPL];
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) {
+        xk[e] = bf16_bits_to_f32((kx[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+        xv[e] = bf16_bits_to_f32((vx[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+    }
+    float ak = 0.f, av = 0.f;
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) {
+        ak = fmaxf(ak, fabsf(xk[e]));
+        av = fmaxf(av, fabsf(xv[e]));
+    }
+    // per token: over the warp; group-32: over the 32 / VPL lanes of a group
+    constexpr int RED = G32 ? 32 / VPL : 32;
+#pragma unroll
+    for (int off = 1; off < RED; off <<= 1) {
+        ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, off));
+        av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, off));
+    }
+    const float sck = q8_scale(ak), scv = q8_scale(av);
+    const float ik = __frcp_rn(sck), iv = __frcp_rn(scv);
+    uint32_t bk = 0u, bv = 0u;
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) {
+        bk |= q8_byte(xk[e], sck, ik) << (8 * e);
+        bv |= q8_byte(xv[e], scv, iv) << (8 * e);
+    }
+    const int gidx = G32 ? (lane * VPL) >> 5 : 0;
+    const bool lead = G32 ? ((lane * VPL) & 31) == 0 : lane == 0;
+    const uint32_t off = swz<D>(static_cast<uint32_t>(r), static_cast<uint32_t>(lane * VPL));
+    int64_t crow;
+    if constexpr (PAGED) {
+        const int32_t pg = p.table[static_cast<int64_t>(b) * p.max_pages + (tok >> 4)];
+        crow = (static_cast<int64_t>(pg) * p.Hk + hk) * 16 + (tok & 15);
+    } else {
+        crow = (static_cast<int64_t>(b) * p.Hk + hk) * p.max_seq + tok;
+    }
+    if constexpr (VPL == 4) {
+        sts_u32(sk + off, bk);
+        sts_u32(sv + off, bv);
+        *reinterpret_cast<uint32_t*>(p.k_w + crow * D + lane * VPL) = bk;
+        *reinterpret_cast<uint32_t*>(p.v_w + crow * D + lane * VPL) = bv;
+    } else {
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(sk + off), "h"(static_cast<uint16_t>(bk)) : "memory");
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(sv + off), "h"(static_cast<uint16_t>(bv)) : "memory");
+        *reinterpret_cast<uint16_t*>(p.k_w + crow * D + lane * VPL) = static_cast<uint16_t>(bk);
+        *reinterpret_cast<uint16_t*>(p.v_w + crow * D + lane * VPL) = static_cast<uint16_t>(bv);
+    }
+    if (lead) {
+        sts_f32(sks + (r * NG + gidx) * 4, sck);
+        sts_f32(svs + (r * NG + gidx) * 4, scv);
+        p.ks_w[crow * NG + gidx] = sck;
+        p.vs_w[crow * NG + gidx] = scv;
+    }
+    // the slot is refilled by TMA (async proxy) after these generic writes
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+}
+
+
+template <int D, bool G32, bool PAGED, bool G16, bool PK, int VAR, int F8, bool ST>
 __global__ void __launch_bounds__(nthreads(PAGED), 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ DecodeParams prm) {
+    // VAR: 0 decode, 1 masked (chunks of queries, sliding windows), 2 decode
+    // with the fused append of the step's new token
+    constexpr bool CAUSAL = VAR == 1;
+    constexpr bool FUSED = VAR == 2;
     using Lay = Layout<D, G32, G16>;
     constexpr int NG = Lay::NG;
     constexpr int NST = Lay::NST;
@@ -276,6 +365,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     static_assert(!(PK && CAUSAL), "chunk queries: unpacked columns");
     static_assert(F8 == 0 || !G32, "FP8 caches have no scales");
     static_assert(!ST || (F8 == 0 && !G32), "per-head / per-channel scales: INT8, no groups");
+    static_assert(!FUSED || (F8 == 0 && !ST), "fused append: INT8 per token / group-32");
     // no scale rows in the ring: FP8 (no scales) and per-head / per-channel
     // scales (one set per (sequence, kv head), folded into Q and the output)
     constexpr bool NOSC = F8 != 0 || ST;
@@ -819,9 +909,19 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
     };
 
+    // ---- in-kernel combine (flash-decoding): fold a split unit's partial
+    // states, slots j < ns of rows bh0 .. bh0 + G - 1 (a slot whose m is -inf
+    // holds none), into its output rows:
+    //   M = max_j m_j,  w_j = 2^(m_j - M),  out = sum_j w_j o_j / sum_j w_j l_j.
+    // tpi adjacent threads share the slots of one (row, 16-byte chunk), each
+    // folding batches of eight slots per round of L2 loads, then merge their
+    // states by shuffles.
+    // ---- fused append (decode, INT8 per token / group-32): patch_new_token
+
 #pragma unroll 1
     for (int i = ibeg; i < iend;) {
-        const Seg sg = one ? one_seg(one_valid(one_raw())) : seg_at(i, iend, lens, nsv, cum, B, p.chunk);
+        const int Lone = one ? one_valid(one_raw()) : 0;
+        const Seg sg = one ? one_seg(Lone) : seg_at(i, iend, lens, nsv, cum, B, p.chunk);
         i = sg.next;
         const int b = sg.b, hk = sg.hk;
         const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + hk * G;   // first q head of the group
@@ -829,7 +929,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // sliding window: the first (both counted from the window base)
         int lim_col[NT][2], lo_col[NT][2];
         if constexpr (CAUSAL) {
-            const int Lseq = one ? one_valid(one_raw()) : lens[b];
+            const int Lseq = one ? Lone : lens[b];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -872,6 +972,20 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // one item per CTA: at least the one stage the producer issued before
         // it knew the length
         const int ntiles = max(one ? 1 : 0, (t1 - t0 + TT - 1) / TT);
+        // fused append: the new token (position L - 1, fa_tok) lies in one
+        // stage of this segment, in the slice of one warp of the group that
+        // takes that stage; that warp quantises it there (-1: not this warp)
+        int fa_tok = -1;
+        if constexpr (FUSED) {
+            if (p.k_new != nullptr) {
+                const int tok = (one ? Lone : lens[b]) - 1;
+                if (tok >= t0 && tok < t1) {
+                    const int itn = (tok - t0) / TT;
+                    if (((c_count + itn) & 1) == grp && ((tok - t0 - itn * TT) >> 5) == wg)
+                        fa_tok = tok;
+                }
+            }
+        }
 #pragma unroll 1
         for (int it = 0; it < ntiles; ++it, ++c_count) {
             if ((c_count & 1) != grp) continue;           // the other group's stage
@@ -892,6 +1006,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 int rA[2], rB[2], V0[2], V1[2];
                 bool okA[2], okB[2];
                 const uint32_t pmask = PAGED ? lds32(sk + Lay::MASK_OFF) : 0u;
+                if constexpr (FUSED) {
+                    // (paged: only into a page that was loaded; a missing one
+                    // was flagged by the producer and its tokens are masked)
+                    if (fa_tok >= tt0 && fa_tok < tt0 + TT &&
+                        (!PAGED || ((pmask >> ((fa_tok - tt0) >> 4)) & 1u)))
+                        patch_new_token<D, G32, PAGED>(p, sk, sv, sks, svs, fa_tok - tt0, fa_tok,
+                                                       b, hk);
+                }
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     const int base = 32 * wg + 16 * u;
@@ -1400,7 +1522,7 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int D, int64_t rows, in
 
 // Function attributes belong to the current device's context, so they are
 // set once per device ordinal.
-template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8, bool ST>
+template <int D, bool G32, bool PAGED, bool G16, bool PK, int VAR, int F8, bool ST>
 cudaError_t set_attrs() {
     using Lay = Layout<D, G32, G16>;
     static std::atomic<uint64_t> done{0};
@@ -1408,7 +1530,7 @@ cudaError_t set_attrs() {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     return once_per_device(done, dev, cudaSuccess, [] {
-        auto kern = decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL, F8, ST>;
+        auto kern = decode_split_tc<D, G32, PAGED, G16, PK, VAR, F8, ST>;
         cudaError_t r =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
         if (r == cudaSuccess)
@@ -1418,10 +1540,10 @@ cudaError_t set_attrs() {
     });
 }
 
-template <int D, bool G32, bool PAGED, bool G16, bool PK, bool CAUSAL, int F8 = 0, bool ST = false>
+template <int D, bool G32, bool PAGED, bool G16, bool PK, int VAR, int F8 = 0, bool ST = false>
 cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     using Lay = Layout<D, G32, G16>;
-    cudaError_t e = set_attrs<D, G32, PAGED, G16, PK, CAUSAL, F8, ST>();
+    cudaError_t e = set_attrs<D, G32, PAGED, G16, PK, VAR, F8, ST>();
     if (e != cudaSuccess) return e;
     CUtensorMap mk, mv;
     const int64_t rows = PAGED ? static_cast<int64_t>(p.num_pages) * p.Hk * 16
@@ -1440,7 +1562,7 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16, PK, CAUSAL, F8, ST>, mk, mv,
+    return cudaLaunchKernelEx(&cfg, decode_split_tc<D, G32, PAGED, G16, PK, VAR, F8, ST>, mk, mv,
                               p);
 }
 
@@ -1449,12 +1571,20 @@ cudaError_t pick_g(const DecodeParams& p, cudaStream_t s) {
     // a chunk of queries (causal columns) or a sliding window: the masked
     // instantiation (for one decode query the causal mask keeps every position)
     if (p.qlen > 1 || p.window > 0)
-        return p.G > 8 ? launch_tc<D, G32, PAGED, true, false, true>(p, s)
-                       : launch_tc<D, G32, PAGED, false, false, true>(p, s);
-    if (p.G > 8) return launch_tc<D, G32, PAGED, true, false, false>(p, s);
+        return p.G > 8 ? launch_tc<D, G32, PAGED, true, false, 1>(p, s)
+                       : launch_tc<D, G32, PAGED, false, false, 1>(p, s);
+    // the step's new token quantised inside the kernel (kvq_append_decode):
+    // its own instantiation, so the plain decode code carries none of it
+    if (p.k_new != nullptr) {
+        if (p.G > 8) return launch_tc<D, G32, PAGED, true, false, 2>(p, s);
+        if constexpr (G32)
+            if (p.G <= 4) return launch_tc<D, G32, PAGED, false, true, 2>(p, s);
+        return launch_tc<D, G32, PAGED, false, false, 2>(p, s);
+    }
+    if (p.G > 8) return launch_tc<D, G32, PAGED, true, false, 0>(p, s);
     if constexpr (G32)
-        if (p.G <= 4) return launch_tc<D, G32, PAGED, false, true, false>(p, s);
-    return launch_tc<D, G32, PAGED, false, false, false>(p, s);
+        if (p.G <= 4) return launch_tc<D, G32, PAGED, false, true, 0>(p, s);
+    return launch_tc<D, G32, PAGED, false, false, 0>(p, s);
 }
 
 // FP8 caches (no scales): E4M3 (F8 = 1) or E5M2 (F8 = 2)
@@ -1462,10 +1592,10 @@ template <int D, bool PAGED, int F8>
 cudaError_t pick_g_fp8(const DecodeParams& p, cudaStream_t s) {
     const bool masked = p.qlen > 1 || p.window > 0;
     if (p.G > 8)
-        return masked ? launch_tc<D, false, PAGED, true, false, true, F8>(p, s)
-                      : launch_tc<D, false, PAGED, true, false, false, F8>(p, s);
-    return masked ? launch_tc<D, false, PAGED, false, false, true, F8>(p, s)
-                  : launch_tc<D, false, PAGED, false, false, false, F8>(p, s);
+        return masked ? launch_tc<D, false, PAGED, true, false, 1, F8>(p, s)
+                      : launch_tc<D, false, PAGED, true, false, 0, F8>(p, s);
+    return masked ? launch_tc<D, false, PAGED, false, false, 1, F8>(p, s)
+                  : launch_tc<D, false, PAGED, false, false, 0, F8>(p, s);
 }
 
 // per-head / per-channel scales (one set per (sequence, kv head))
@@ -1473,10 +1603,10 @@ template <int D, bool PAGED>
 cudaError_t pick_g_static(const DecodeParams& p, cudaStream_t s) {
     const bool masked = p.qlen > 1 || p.window > 0;
     if (p.G > 8)
-        return masked ? launch_tc<D, false, PAGED, true, false, true, 0, true>(p, s)
-                      : launch_tc<D, false, PAGED, true, false, false, 0, true>(p, s);
-    return masked ? launch_tc<D, false, PAGED, false, false, true, 0, true>(p, s)
-                  : launch_tc<D, false, PAGED, false, false, false, 0, true>(p, s);
+        return masked ? launch_tc<D, false, PAGED, true, false, 1, 0, true>(p, s)
+                      : launch_tc<D, false, PAGED, true, false, 0, 0, true>(p, s);
+    return masked ? launch_tc<D, false, PAGED, false, false, 1, 0, true>(p, s)
+                  : launch_tc<D, false, PAGED, false, false, 0, 0, true>(p, s);
 }
 
 template <int D, bool PAGED>

@@ -20,6 +20,39 @@ __device__ __forceinline__ void raise_flag(int32_t* d_err, uint32_t bits) {
     if (d_err) atomicOr(reinterpret_cast<int*>(d_err), static_cast<int>(bits));
 }
 
+// ------------------------------------------------- INT8 quantiser (append)
+// Method (abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
+// CudaQuantizedKvCache::quantize_tensor): s = max(max |x|, 1e-8) / 127 and
+// byte = clamp(round_half_away(x / s) + 128, 0, 255), both divisions IEEE
+// round-to-nearest fp32.  Every kernel that quantises (the append kernels and
+// the decode kernel's fused append) uses these, so their bytes agree.
+
+// the scale of a row (or 32-value group) from its absolute maximum
+__device__ __forceinline__ float q8_scale(float amax) {
+    return __fdiv_rn(amax < 1e-8f ? 1e-8f : amax, 127.0f);
+}
+
+// round_half_away(x / s) for the IEEE-rounded fp32 quotient x / s, mostly
+// without a division.  r = x * inv, inv = 1 / s rounded once and the product
+// rounded once, is within 2^-23 |x / s| of the quotient, i.e. within 2.3e-5
+// of the rounded quotient wherever |x / s| <= 128 (every in-range byte).  So
+// unless r lies within 1e-4 of a point halfway between two integers, the
+// rounded quotient lies strictly inside the same interval (k - 0.5, k + 0.5)
+// and rounds to the same integer as r; those near-ties take the IEEE division.
+// Beyond |x / s| = 128 both roundings clamp to the same byte.
+__device__ __forceinline__ int round_quotient(float x, float s, float inv) {
+    const float r = __fmul_rn(x, inv);
+    const float a = fabsf(r);
+    if (fabsf(a - floorf(a) - 0.5f) < 1e-4f) return static_cast<int>(roundf(__fdiv_rn(x, s)));
+    return static_cast<int>(roundf(r));
+}
+
+// the stored byte of x under scale s (inv = __frcp_rn(s))
+__device__ __forceinline__ uint32_t q8_byte(float x, float s, float inv) {
+    const int v = round_quotient(x, s, inv) + 128;
+    return static_cast<uint32_t>(v < 0 ? 0 : (v > 255 ? 255 : v));
+}
+
 // ---------------------------------------------------------------- append
 struct AppendParams {
     const uint16_t* k_new;   // [B, Hk, T, D] bf16
@@ -83,7 +116,18 @@ struct DecodeParams {
     const uint16_t* rk;      // mixed cache: bf16 rings [B, Hk, recent, D] (K and V)
     const uint16_t* rv;
     float scale_log2;        // attn_scale * log2(e)
+    // fused append (decode, INT8 per token / group-32): the step's new token
+    // k_new / v_new bf16 [B, Hk, 1, D] is quantised into position L - 1 of
+    // the cache (written through k_w / v_w / ks_w / vs_w, the same memory as
+    // k / v / k_scale / v_scale) by the CTA whose range holds it; null: none
+    const uint16_t* k_new;
+    const uint16_t* v_new;
+    uint8_t* k_w;
+    uint8_t* v_w;
+    float* ks_w;
+    float* vs_w;
 };
+
 
 // Sliding window: the oldest position any of a sequence's qlen queries sees
 // is L - qlen - window + 1.  The kernels count a sequence's tokens from that
@@ -109,7 +153,12 @@ __device__ __forceinline__ int walked_len(int L, int64_t cap, int64_t plan, int 
 constexpr int kMaxBatch = 1024;                              // sequences per call
 constexpr int kMaxRecent = 2048;                             // mixed cache: bf16 window tokens
 constexpr int kMaxGrid = 1024;                               // persistent CTAs
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+// the split kernel (tensor-core, or the CUDA-core one when simt) and, where
+// the partials are not folded in it, the combine kernel
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s, bool simt = false);
+// CUDA-core split kernel (kvq_decode_simt.cu): any D % 16 == 0 up to 256,
+// any rows per kv head, one item per CTA
+cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t s);
 // mixed cache: the bf16 window's partial and the INT8 partials into the output
 cudaError_t launch_recent_combine(const DecodeParams& p, cudaStream_t s);
 // tensor-core split kernel (kvq_decode_tc.cu)

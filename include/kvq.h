@@ -201,10 +201,13 @@ typedef struct kvq_cache_view {
  *   num_splits  0 = automatic; otherwise the requested number of KV splits
  *               per sequence (split-K / flash-decoding)
  *   d_err       int32 [1] or NULL (KVQ_DEVERR_LEN, KVQ_DEVERR_PAGE)
- * Requirements: Hq % Hk == 0 and Hq / Hk <= 16; D in {64, 128}; GROUP32
- * needs D % 32 == 0; B * Hk * max_seq (contiguous) or num_pages * Hk * 16
- * (paged) below 2^31 rows; B <= 1024 and B * Hk * splits below 2^31
- * (otherwise KVQ_ERR_UNSUPPORTED).
+ * Requirements: Hq % Hk == 0; 16 <= D <= 256 with D % 16 == 0 (GROUP32:
+ * D % 32 == 0); B <= 65535, Hq <= 65535 (otherwise KVQ_ERR_INVALID_ARG /
+ * KVQ_ERR_UNSUPPORTED); B * Hk * splits below 2^31 (KVQ_ERR_UNSUPPORTED).
+ * D in {64, 128} with Hq / Hk <= 16, B <= 1024 and the cache below 2^31
+ * rows of D bytes runs on the tensor-core split kernel; every other shape
+ * on the CUDA-core split kernel (same results within the stated bar,
+ * lower throughput).
  * Source: abaddon 0.2.0-rc.1, kv_cache_quant_cuda.rs, module doc "Fused
  * approach" and CudaQuantizedKvCache::forward_attention (scores with
  * on-the-fly K dequantisation, softmax, P.V with on-the-fly V
@@ -224,6 +227,39 @@ size_t kvq_decode_workspace_bytes(int B, int Hq, int Hk, int D, int max_seq_len_
                                   int num_splits);
 
 /*
+ * kvq_append_decode -- one decode step in one call: the step's new token of
+ * every (sequence, kv head) is quantised into the cache at position
+ * L_b - 1, then the step's query attends to positions 0 .. L_b - 1, with the
+ * same fused dequantisation as kvq_decode_attn.  The result (cache bytes,
+ * scales and output) is that of kvq_append (or kvq_append_paged) with
+ * d_pos[b] = L_b - 1 followed by kvq_decode_attn; the quantisation is the
+ * same bit-exact rule.  The token is quantised by the CTA whose range of the
+ * cache holds position L_b - 1, into its shared-memory tile and into the
+ * cache, so no separate append launch runs.
+ *   k_new, v_new  bf16 [B, Hk, 1, D]   the step's new keys / values (read)
+ *   kv          cache view as for kvq_decode_attn; its k, v, k_scale and
+ *               v_scale arrays are WRITTEN at position L_b - 1 (they must be
+ *               writable device memory)
+ *   d_seq_lens  int32 [B]  L_b, the length INCLUDING the new token; 0: no
+ *               token is written and the output row is zero
+ *   the other arguments as for kvq_decode_attn (workspace: at least
+ *   kvq_decode_workspace_bytes(...) bytes).
+ * Requirements: those of kvq_decode_attn, with mode PER_TOKEN or GROUP32
+ * (other modes: KVQ_ERR_UNSUPPORTED).  A sequence whose length is beyond the
+ * capacity writes nothing and is flagged KVQ_DEVERR_LEN; a missing page of
+ * position L_b - 1 writes nothing and is flagged KVQ_DEVERR_PAGE.
+ * Source: abaddon 0.2.0-rc.1, kv_cache_quant_cuda.rs, CudaQuantizedKvCache::
+ * append followed by forward_attention (a decode step appends its token and
+ * attends to the cache that now holds it).
+ */
+kvq_status kvq_append_decode(const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
+                             int B, int Hq, int Hk, int D, kvq_scale_mode mode,
+                             const kvq_cache_view *kv, const int32_t *d_seq_lens,
+                             int max_seq_len_hint, float attn_scale, float *out, void *workspace,
+                             size_t workspace_bytes, int num_splits, int32_t *d_err,
+                             kvq_stream_t stream);
+
+/*
  * kvq_chunk_attn -- a chunk of T new queries per (sequence, q head), causal
  * from the chunk's end: the chunk's T tokens are the last T positions of the
  * sequence (appended before the call), so query i sits at position
@@ -239,8 +275,11 @@ size_t kvq_decode_workspace_bytes(int B, int Hq, int Hk, int D, int max_seq_len_
  *               kvq_decode_attn
  *   the other arguments as for kvq_decode_attn.
  * Requirements: those of kvq_decode_attn with the GQA group counted in
- * (head, query) rows: (Hq / Hk) * T <= 16 (otherwise KVQ_ERR_UNSUPPORTED).
- * T < 1 is KVQ_ERR_INVALID_ARG.
+ * (head, query) rows, (Hq / Hk) * T <= 2^19.  More than 16 rows per kv head
+ * run on the dense tcgen05 kernel when D = 128, the scales are per token,
+ * the cache is contiguous and there is no window (that kernel needs no
+ * workspace); otherwise on the CUDA-core split kernel.  T < 1 is
+ * KVQ_ERR_INVALID_ARG.
  * Source: abaddon 0.2.0-rc.1, kv_cache_quant_cuda.rs,
  * CudaQuantizedKvCache::forward_attention (prefill with q_len > 1: the cache
  * offset is seq_len - q_len and query q_pos sees the positions up to

@@ -149,13 +149,16 @@ def test_decode_rejects_bad_arguments(kvq):
     assert call(Hq=30) == 1                 # Hq % Hk != 0
     assert call(D=100) == 1
     assert call(mode=1, D=48) == 1
-    assert call(D=256) == 2                 # valid, kernel not built for it
-    assert call(D=32) == 2
-    # a GQA group above 16 rows runs on the dense tcgen05 kernel, which covers
-    # head_dim 128, per-token scales, contiguous caches: other shapes are refused
-    assert call(Hq=8 * 32, Hk=8, D=64) == 2
-    assert call(Hq=8 * 32, Hk=8, mode=1) == 2
-    assert call(B=1025) == 2                # more sequences than the split kernel caches
+    # shapes outside the tensor-core kernels (other head dims, more than 16
+    # rows per kv head outside the dense kernel, more than 1024 sequences) are
+    # accepted for the CUDA-core kernel: validation passes and the call stops
+    # at the device query, which fails here without a GPU (KVQ_ERR_CUDA)
+    assert call(D=256) == 3
+    assert call(D=32) == 3
+    assert call(D=48) == 3
+    assert call(Hq=8 * 32, Hk=8, D=64) == 3
+    assert call(Hq=8 * 32, Hk=8, mode=1) == 3
+    assert call(B=1025) == 3
     assert call(out=FAKE + 4) == 1          # misaligned output
     cv_bad_scale = kvq.CacheView(FAKE, FAKE, FAKE + 8, FAKE, 0, 4096, 0, 0, 0)
     assert call(kv=ctypes.byref(cv_bad_scale)) == 1
@@ -164,6 +167,31 @@ def test_decode_rejects_bad_arguments(kvq):
     assert call(kv=ctypes.byref(bad_page)) == 1
     no_table = kvq.CacheView(FAKE, FAKE, FAKE, FAKE, 16, 0, None, 4, 4)
     assert call(kv=ctypes.byref(no_table)) == 1
+
+
+@needs_no_gpu
+def test_append_decode_rejects_bad_arguments(kvq):
+    lib = kvq.lib
+    cv = kvq.CacheView(FAKE, FAKE, FAKE, FAKE, 0, 4096, 0, 0, 0)
+    ok = dict(q=FAKE, kn=FAKE, vn=FAKE, B=1, Hq=32, Hk=8, D=128, mode=0, kv=ctypes.byref(cv),
+              sl=FAKE, hint=4096, scale=0.088, out=FAKE, ws=FAKE, wsb=1 << 30, ns=0, err=None,
+              s=None)
+
+    def call(**over):
+        a = dict(ok)
+        a.update(over)
+        return lib.kvq_append_decode(*a.values())
+    assert call(kn=None) == 1
+    assert call(vn=None) == 1
+    assert call(vn=FAKE + 2) == 1           # misaligned new values
+    assert call(q=None) == 1
+    assert call(mode=9) == 1
+    for m in (2, 3, 4, 5):                  # FP8, per-head, per-channel: not fused
+        assert call(mode=m) == 2
+    assert call(Hq=30) == 1
+    # any head dim and group size (the CUDA-core kernel): past validation
+    assert call(Hq=8 * 32) == 3
+    assert call(D=256) == 3
 
 
 @needs_no_gpu
@@ -179,12 +207,13 @@ def test_chunk_rejects_bad_arguments(kvq):
         return lib.kvq_chunk_attn(*a.values())
     assert call(T=0) == 1
     assert call(q=None) == 1
-    # more than 16 rows per kv head: the dense kernel, head_dim 128, per-token,
-    # contiguous, no window only
-    assert call(T=5, D=64) == 2             # (Hq / Hk) * T = 20 rows per kv head
-    assert call(Hq=64, T=3, mode=1) == 2    # 24 rows, group-32 scales
+    # more than 16 rows per kv head outside the dense kernel's shapes (head_dim
+    # 128, per-token, contiguous, no window): accepted for the CUDA-core kernel
+    # (the call then stops at the device query: no GPU here)
+    assert call(T=5, D=64) == 3             # (Hq / Hk) * T = 20 rows per kv head
+    assert call(Hq=64, T=3, mode=1) == 3    # 24 rows, group-32 scales
     pv = kvq.CacheView(FAKE, FAKE, FAKE, FAKE, 16, 0, FAKE, 4, 4)
-    assert call(T=5, kv=ctypes.byref(pv)) == 2     # paged
+    assert call(T=5, kv=ctypes.byref(pv)) == 3     # paged
     assert call(out=FAKE + 4) == 1
 
 
@@ -194,7 +223,9 @@ def test_chunk_workspace_is_the_decode_workspace_of_the_rows(kvq):
         assert kvq.kvq_chunk_workspace_bytes(B, Hq, Hk, T, D, hint, ns) == \
             kvq.kvq_decode_workspace_bytes(B, Hq * T, Hk, D, hint, ns)
     assert kvq.kvq_chunk_workspace_bytes(1, 32, 8, 0, 128, 4097, 0) == 0
-    assert kvq.kvq_chunk_workspace_bytes(1, 32, 8, 5, 128, 4097, 0) == 0   # dense: none
+    # above 16 rows per kv head: sized for the CUDA-core kernel too
+    assert kvq.kvq_chunk_workspace_bytes(1, 32, 8, 5, 128, 4097, 0) == \
+        kvq.kvq_decode_workspace_bytes(1, 32 * 5, 8, 128, 4097, 0)
 
 
 @needs_no_gpu

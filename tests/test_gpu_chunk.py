@@ -106,11 +106,12 @@ def test_chunk_longer_than_its_sequence_is_a_length_error():
     assert_attn_close(out[1:], c.oracle_chunk(q, sl, f32_scale(D))[1:], "valid sequence")
 
 
-def test_chunk_rows_beyond_sixteen_per_kv_head_at_d64_are_unsupported():
-    """More than 16 rows per kv head run on the dense kernel, which covers
-    head_dim 128 only."""
-    m = kvq()
+def test_chunk_rows_beyond_sixteen_per_kv_head_at_d64():
+    """More than 16 rows per kv head at head_dim 64, a shape the dense kernel
+    does not cover: the CUDA-core split kernel takes it."""
     c = _contig(1, 1, 64, "per_token", [40], seed=121)
     q = bf16_randn((1, 4, 5, 64), seed=122)      # G * T = 20
-    with pytest.raises(m.KvqError):
-        c.chunk(q, torch.tensor([40], dtype=torch.int32), 40)
+    sl = torch.tensor([40], dtype=torch.int32)
+    assert_attn_close(c.chunk(q, sl, 40, attn_scale=f32_scale(64)),
+                      c.oracle_chunk(q, sl, f32_scale(64)), "G*T=20 at D=64")
+    assert kvq().kvq_read_error(c.err) == 0

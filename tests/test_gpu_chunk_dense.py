@@ -68,14 +68,18 @@ def test_dense_chunk_length_rules():
     assert_attn_close(out, ref, "all rows")
 
 
-def test_dense_chunk_unsupported_variants():
-    m = kvq()
+def test_dense_shapes_outside_the_tcgen05_kernel():
+    """A dense chunk the tcgen05 kernel does not cover (group-32 scales) runs
+    on the CUDA-core split kernel, within the bar of the oracle."""
     c = ContigCache(1, 1, 64, 128, "group32")
-    q = bf16_randn((1, 8, 4, 128), seed=9).cuda()
-    with pytest.raises(m.KvqError) as ei:
-        m.kvq_chunk_attn(q, c.k, c.v, c.ks, c.vs, torch.tensor([64], dtype=torch.int32).cuda(),
-                         64, mode="group32")
-    assert ei.value.status == 2
+    kn = bf16_randn((1, 1, 64, 128), seed=10)
+    vn = bf16_randn((1, 1, 64, 128), seed=11)
+    assert c.append(kn, vn, torch.zeros(1, dtype=torch.int32)) == 0
+    q = bf16_randn((1, 8, 4, 128), seed=9)          # 32 rows per kv head
+    sl = torch.tensor([64], dtype=torch.int32)
+    out = c.chunk(q, sl, 64, attn_scale=f32_scale(128))
+    assert_attn_close(out, c.oracle_chunk(q, sl, f32_scale(128)), "dense group-32")
+    assert kvq().kvq_read_error(c.err) == 0
 
 
 def test_dense_chunk_long_context_full_size_sampled_rows():
