@@ -4,6 +4,7 @@
 // kvq_read_error, whose job is to read the device error word.
 #include <stdint.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "kvq_internal.cuh"
@@ -17,6 +18,30 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 constexpr int kMaxSplits = 4096;     // bound on splits per sequence (combine smem)
 
 kvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+// SM count of the current device, read once per device (a device's SM count
+// does not change while the process runs; the attribute query costs more
+// than the rest of a call's host work)
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sms[kMaxDevices];
+
+bool current_sms(int* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (dev >= 0 && dev < kMaxDevices) {
+        const int c = g_sms[dev].load(std::memory_order_relaxed);
+        if (c > 0) {
+            *out = c;
+            return true;
+        }
+    }
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return false;
+    if (dev >= 0 && dev < kMaxDevices) g_sms[dev].store(sms, std::memory_order_relaxed);
+    *out = sms;
+    return true;
+}
 
 bool valid_mode(kvq_scale_mode m) {
     return m == KVQ_SCALE_PER_TOKEN || m == KVQ_SCALE_GROUP32 || m == KVQ_FP8_E4M3 ||
@@ -52,12 +77,7 @@ kvq_status check_append_common(const uint16_t* k_new, const uint16_t* v_new, int
 kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk_out,
                 int* splits_out) {
     if (B < 0 || Hk < 1 || hint < 0 || num_splits < 0) return KVQ_ERR_INVALID_ARG;
-    if (num_sms <= 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return KVQ_ERR_CUDA;
-    }
+    if (num_sms <= 0 && !current_sms(&num_sms)) return KVQ_ERR_CUDA;
     int64_t chunk;
     if (hint <= 16) {
         chunk = 16;
@@ -211,10 +231,8 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
         p.grid = 0;                     // one CTA per item (and block of rows)
         p.one_item = 1;
     } else {
-        int dev = 0, sms = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return KVQ_ERR_CUDA;
+        int sms = 0;
+        if (!current_sms(&sms)) return KVQ_ERR_CUDA;
         const int64_t items = static_cast<int64_t>(B) * Hk * splits;
         p.grid = static_cast<int>(items < sms ? items : sms);   // persistent: one CTA per SM
         if (p.grid > kvq::kMaxGrid) p.grid = kvq::kMaxGrid;

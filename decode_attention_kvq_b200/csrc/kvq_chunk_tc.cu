@@ -14,23 +14,31 @@
 //    r = i * G + h (query i, head h of the group), so the rows share K and V
 //    and their causal limits lie within 128 / G positions.  It walks the KV
 //    positions up to its last row's limit in tiles of 128 tokens.
-//  * Warp 4 (one lane) streams K and V tiles (TMA 2-D, 128-byte swizzle) and
+//  * Warp 8 (one lane) streams K and V tiles (TMA 2-D, 128-byte swizzle) and
 //    their fp32 scales (bulk copies) through a two-stage ring.
-//  * Warp 5 (one lane) issues the tensor-core work: S = Q K^T on tcgen05
+//  * Warp 9 (one lane) issues the tensor-core work: S = Q K^T on tcgen05
 //    kind::i8 -- Q as a per-row power-of-two prescaled 16-bit integer in two
 //    byte digits (signed hi, unsigned lo), the K bytes as loaded, so
 //    S = 256 S_hi + S_lo - 128 sum(Qi) is exact in int32 -- into two 128-
 //    column TMEM accumulators; then P V on kind::f16 into a third (fp32, a
 //    fresh one per tile), with P'' = 2^(z - m) * v_scale * 2^kv split into f16
 //    hi + lo parts and V as the exact f16 integers byte - 128.
-//  * Warps 0-3 (thread i = row i = TMEM lane i) read the scores with
-//    tcgen05.ld, apply the K scale, the row's prescale, attn_scale and log2(e),
-//    mask causally, keep the online softmax per row, fold each tile's P V
-//    into a running sum in TMEM (fp32, with the row's rescale), write P'' and
-//    the f16 V tile into shared memory in the canonical swizzled layouts, and
-//    finally read the sum back and write the row.
+//  * Warps 0-7 own the rows, two warps per row: warp w reads TMEM lanes
+//    32 (w % 4) .. + 31 (row i = TMEM lane i) and takes half h = w / 4 of the
+//    row's 128 columns -- tokens 64 h .. 64 h + 63 of a tile and head_dim
+//    64 h .. 64 h + 63 of the output -- so two row warps share each
+//    scheduler.  They read the scores with tcgen05.ld, apply the K scale, the
+//    row's prescale, attn_scale and log2(e), mask causally, exchange the
+//    halves' maxima through shared memory, keep the online softmax per row,
+//    fold each tile's P V into a running sum in TMEM (fp32, with the row's
+//    rescale), write P'' and the f16 V tile into shared memory in the
+//    canonical swizzled layouts, and finally read the sum back and write the
+//    row.  Per tile, the K scales and the V scales times the P'' prescale are
+//    first copied into aligned shared-memory vectors.
 //  * Every mbarrier wait is bounded; a timeout sets KVQ_DEVERR_TIMEOUT, every
-//    role then skips its remaining work, and the CTA frees its tensor memory.
+//    role then skips its remaining work (the row warps still pass every
+//    named barrier of every tile, so none waits for another that left), and
+//    the CTA frees its tensor memory.
 #include <cuda.h>
 #include <math.h>
 
@@ -46,7 +54,9 @@ namespace {
 constexpr int kRows = 128;                 // (query, head) rows per CTA: the MMA M
 constexpr int kTok = 128;                  // KV tokens per tile
 constexpr int kDim = 128;                  // head_dim handled here
-constexpr int kThreads = 192;              // warps 0-3 rows, 4 producer, 5 MMA
+constexpr int kThreads = 320;              // warps 0-7 rows, 8 producer, 9 MMA
+constexpr int kRowThreads = 256;
+constexpr int kProdWarp = 8, kMmaWarp = 9;
 constexpr int kTmemCols = 512;             // S_hi 128 | S_lo 128 | O tile 128 | O run 128
 // The tensor cores add each P.V k-step into O; over a long key range that is
 // tens of thousands of accumulations into one fp32 accumulator, and the error
@@ -65,7 +75,10 @@ constexpr int kV16 = kStage0 + 2 * kStageBytes;   // V as f16 [2 atoms][128 tok]
 constexpr int kPhi = kV16 + 32768;                // P'' hi [2 atoms][128 rows][128 B], K-major
 constexpr int kPlo = kPhi + 32768;
 constexpr int kMisc = kPlo + 32768;               // barriers, tensor-memory address, flags
-constexpr int kSmem = kMisc + 256 + 1024;         // + base alignment slack
+// row-warp vectors: K scales [2][128], V scales x 2^kv [2][128] (by tile
+// parity), the halves' maxima [2][128] and a spare pair [2][128]
+constexpr int kAux = kMisc + 256;
+constexpr int kSmem = kAux + 4096 + 1024;         // + base alignment slack
 
 struct ChunkParams {
     const uint16_t* q;        // [B, Hq, T, D] bf16
@@ -182,7 +195,11 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const uint32_t bar_qready = bar_full + 64;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMisc + 96);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMisc + 100);
-    float* red = reinterpret_cast<float*>(smem + kMisc + 128);   // [4] per-warp V-scale maxima
+    float* red = reinterpret_cast<float*>(smem + kMisc + 128);   // [8] per-warp V-scale maxima
+    float* kal = reinterpret_cast<float*>(smem + kAux);          // [2][128] K scales
+    float* vsu = kal + 256;                                      // [2][128] V scales * 2^kv
+    float* xch = vsu + 256;                                      // [2][128] halves' maxima
+    float* lx = xch + 256;                                       // [2][128] spare pair
 
     // ---- the CTA's (sequence, kv head, row tile) and its KV range
     const int tph = p.tiles_per_head;
@@ -203,13 +220,13 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(bar_full + 8 * s, 1);
-            ptx::mbar_init(bar_empty + 8 * s, 1 + 4);   // K: the MMA commit; V: four row warps
+            ptx::mbar_init(bar_empty + 8 * s, 1 + 8);   // K: the MMA commit; V: eight row warps
         }
         ptx::mbar_init(bar_sfull, 1);
-        ptx::mbar_init(bar_sfree, 4);
-        ptx::mbar_init(bar_pfull, 4);
+        ptx::mbar_init(bar_sfree, 8);
+        ptx::mbar_init(bar_pfull, 8);
         ptx::mbar_init(bar_odone, 1);
-        ptx::mbar_init(bar_qready, 4);
+        ptx::mbar_init(bar_qready, 8);
         *abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&tm_k);
@@ -242,7 +259,7 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const int sc_off = static_cast<int>(unit_row & 3);
     const int64_t sc_total = static_cast<int64_t>(p.B) * p.Hk * p.max_seq;
 
-    if (warp == 4) {
+    if (warp == kProdWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t pol = ptx::policy_evict_first();
@@ -276,7 +293,7 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             for (int j = max(ntile - 2, 0); j < ntile; ++j)
                 ptx::mbar_wait(bar_full + 8 * (j & 1), (j >> 1) & 1);
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
         if (lane == 0 && ntile > 0 && wait(bar_qready, 0)) {
             const uint64_t dq_hi = smem_desc(sb + kQhi, 16, 1024);
@@ -312,23 +329,26 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         }
     } else {
         // ------------------------------------------------------------ rows
-        const int i_row = tid;                          // TMEM lane
+        const int i_row = 32 * (warp & 3) + lane;       // TMEM lane
+        const int hf = warp >> 2;                       // half of the row's columns
         const int r = r_first + i_row;
         const int qi = r / G, h = r - qi * G;
         const bool valid = L >= 0 && qi < T;
         const int pos = L - T + qi;                     // the query's position
         const int64_t orow = (static_cast<int64_t>(b) * p.Hq + hk * G + h) * T + qi;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        // ---- Q digits of this row into the swizzled A tiles
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        auto row_sync = [] { ptx::named_bar_sync(1, kRowThreads); };
+        // ---- Q digits of this row (this half's 64 head_dim values) into the
+        // swizzled A tiles; the row's max |q| and digit sum over both halves
         float zs = 0.f;
         int cq = 0;
         {
-            float qf[kDim];
+            float qf[64];
             float amax = 0.f;
             if (valid) {
-                const uint4* src = reinterpret_cast<const uint4*>(p.q + orow * kDim);
+                const uint4* src = reinterpret_cast<const uint4*>(p.q + orow * kDim + 64 * hf);
 #pragma unroll
-                for (int c = 0; c < kDim / 8; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     const uint4 raw = src[c];
                     const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
@@ -338,11 +358,14 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     }
                 }
 #pragma unroll
-                for (int d = 0; d < kDim; ++d) amax = fmaxf(amax, fabsf(qf[d]));
+                for (int d = 0; d < 64; ++d) amax = fmaxf(amax, fabsf(qf[d]));
             } else {
 #pragma unroll
-                for (int d = 0; d < kDim; ++d) qf[d] = 0.f;
+                for (int d = 0; d < 64; ++d) qf[d] = 0.f;
             }
+            lx[128 * hf + i_row] = amax;
+            row_sync();
+            amax = fmaxf(lx[i_row], lx[128 + i_row]);
             int sh = 0;
             if (amax > 0.f) {
                 const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127;
@@ -352,14 +375,15 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             zs = pow2i_f(-sh) * p.scale_log2;
             int qsum = 0;
 #pragma unroll
-            for (int c = 0; c < kDim / 16; ++c) {       // 16 values = one 16-byte chunk per digit
+            for (int cc = 0; cc < 4; ++cc) {            // 16 values = one 16-byte chunk per digit
+                const int c = 4 * hf + cc;
                 uint32_t hi[4], lo[4];
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
                     uint32_t hw = 0, lw = 0;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int v = min(max(__float2int_rn(qf[16 * c + 4 * w + e] * up), -32767), 32767);
+                        const int v = min(max(__float2int_rn(qf[16 * cc + 4 * w + e] * up), -32767), 32767);
                         qsum += v;
                         hw |= ((static_cast<uint32_t>(v) >> 8) & 0xffu) << (8 * e);
                         lw |= (static_cast<uint32_t>(v) & 0xffu) << (8 * e);
@@ -371,50 +395,45 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 *reinterpret_cast<uint4*>(smem + kQhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
                 *reinterpret_cast<uint4*>(smem + kQlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
-            cq = 128 * qsum;
+            xch[128 * hf + i_row] = __int_as_float(qsum);
+            row_sync();
+            cq = 128 * (__float_as_int(xch[i_row]) + __float_as_int(xch[128 + i_row]));
         }
         fence_async_smem();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar_qready);
 
-        float m_run = -INFINITY, l_run = 0.f;
+        float m_run = -INFINITY, l_run = 0.f;            // l_run: this half's tokens
         int kv = 64;                                     // P'' prescale exponent (CTA-uniform)
         float f_prev = 1.f;                              // rescale of the running sum (see the fold)
+        bool live = true;                                // no wait has given up
         for (int j = 0; j < ntile; ++j) {
             const int s = j & 1;
             const int t0 = j * kTok;
             const float* ksc = reinterpret_cast<const float*>(smem + kStage0 + s * kStageBytes + kStKs) + sc_off;
             const float* vsc = reinterpret_cast<const float*>(smem + kStage0 + s * kStageBytes + kStVs) + sc_off;
-            if (!wait(bar_full + 8 * s, (j >> 1) & 1)) break;
-            if (!wait(bar_sfull, j & 1)) break;
-            tc_fence_after();
-            // ---- pass 1: the row's maximum over the tile
-            float zmax = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sh_[32], sl_[32];
-                tmem_ld32(lane_base + kColShi + 32 * c, sh_);
-                tmem_ld32(lane_base + kColSlo + 32 * c, sl_);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int t = t0 + 32 * c + e;
-                    const int S = static_cast<int>(sh_[e]) * 256 + static_cast<int>(sl_[e]) - cq;
-                    const float z = static_cast<float>(S) * ksc[32 * c + e] * zs;
-                    if (valid && t <= pos) zmax = fmaxf(zmax, z);
-                }
-            }
-            // ---- the tile's largest V scale over its real tokens (the same for
-            // every row): the P'' prescale 2^kv only drops, and a drop rescales O
-            float drop = 1.f;
+            float* kal_j = kal + 128 * s;
+            float* vsu_j = vsu + 128 * s;
+            live = live && wait(bar_full + 8 * s, (j >> 1) & 1);
+            // ---- the tile's scales: token i_row's K scale and V scale (0 past
+            // the keys), the largest V scale over the tile (the same for every
+            // row): the P'' prescale 2^kv only drops, and a drop rescales O
+            const bool real = t0 + i_row < t_hi;
+            const float ks_i = (live && real) ? ksc[i_row] : 0.f;
+            const float vs_i = (live && real) ? vsc[i_row] : 0.f;
             {
-                float vm = (t0 + i_row < t_hi) ? vsc[i_row] : 0.f;
+                float vm = vs_i;
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
                 if (lane == 0) red[warp] = vm;
-                ptx::named_bar_sync(1, 128);
-                vm = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-                ptx::named_bar_sync(1, 128);             // red is read before the next tile writes it
+                if (hf == 0) kal_j[i_row] = ks_i;
+            }
+            row_sync();
+            float drop = 1.f;
+            {
+                float vm = red[0];
+#pragma unroll
+                for (int w = 1; w < 8; ++w) vm = fmaxf(vm, red[w]);
                 if (vm > 0.f) {
                     const int ev = static_cast<int>((__float_as_uint(vm) >> 23) & 0xffu) - 127;
                     const int kn = max(min(kv, 14 - ev), -120);
@@ -423,19 +442,55 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                         kv = kn;
                     }
                 }
+                if (hf == 0) vsu_j[i_row] = vs_i * pow2i_f(kv);
             }
-            const float m_new = fmaxf(m_run, zmax);
+            row_sync();                                  // red read; kal, vsu written
+            live = live && wait(bar_sfull, j & 1);
+            tc_fence_after();
+            // ---- pass 1: the maximum of S * k_scale over this half's tokens
+            // (tiles wholly at or below the row's position need no mask)
+            const int tb = t0 + 64 * hf;                 // this half's first token
+            const bool unmasked = valid && tb + 63 <= pos;
+            float xmax = -INFINITY;
+            if (live) {
+#pragma unroll 1
+                for (int cl = 0; cl < 2; ++cl) {
+                    const int c = 2 * hf + cl;
+                    uint32_t sh_[32], sl_[32];
+                    tmem_ld32(lane_base + kColShi + 32 * c, sh_);
+                    tmem_ld32(lane_base + kColSlo + 32 * c, sl_);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 k4 = *reinterpret_cast<const float4*>(kal_j + 32 * c + 4 * e4);
+                        const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int e = 4 * e4 + u;
+                            const int S = static_cast<int>(sh_[e]) * 256 + static_cast<int>(sl_[e]) - cq;
+                            const float x = static_cast<float>(S) * kk[u];
+                            if (unmasked || (valid && t0 + 32 * c + e <= pos)) xmax = fmaxf(xmax, x);
+                        }
+                    }
+                }
+            }
+            xch[128 * hf + i_row] = xmax;
+            row_sync();
+            const float xm = fmaxf(xch[i_row], xch[128 + i_row]);
+            const float m_new = fmaxf(m_run, xm * zs);
             const float mb = m_new == -INFINITY ? 0.f : m_new;
             const float alpha = m_run == -INFINITY ? 1.f : ptx::ex2(m_run - mb);
             // the previous P.V is done: P, V16 free, O stable
-            if (j >= 1 && !wait(bar_odone, (j - 1) & 1)) break;
+            if (j >= 1) live = live && wait(bar_odone, (j - 1) & 1);
             tc_fence_after();
-            // fold the previous tile's P.V into the running sum: run = run * f + tile,
-            // f the previous tile's rescale (the running sum is relative to the
-            // tile's maximum and prescale)
-            if (j >= 1) {
+            // fold the previous tile's P.V into the running sum (this half's
+            // head_dim columns): run = run * f + tile, f the previous tile's
+            // rescale (the running sum is relative to the tile's maximum and
+            // prescale)
+            if (live && j >= 1) {
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int cl = 0; cl < 2; ++cl) {
+                    const int c = 2 * hf + cl;
                     uint32_t ot[32], orn[32];
                     tmem_ld32(lane_base + kColO + 32 * c, ot);
                     if (j >= 2) tmem_ld32(lane_base + kColRun + 32 * c, orn);
@@ -450,44 +505,54 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 tmem_wait_st();
             }
             f_prev = alpha * drop;                       // applies to the running sum at the next fold
-            // ---- pass 2: P'' = 2^(z - m) * v_scale * 2^kv as f16 hi + lo
-            const float up = pow2i_f(kv);
+            // ---- pass 2: P'' = 2^(z - m) * v_scale * 2^kv as f16 hi + lo for
+            // this half's tokens (P atom hf)
             float lsum = 0.f;
+            if (live) {
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sh_[32], sl_[32];
-                tmem_ld32(lane_base + kColShi + 32 * c, sh_);
-                tmem_ld32(lane_base + kColSlo + 32 * c, sl_);
-                tmem_wait_ld();
-                uint32_t ph[16], pl[16];
+                for (int cl = 0; cl < 2; ++cl) {
+                    const int c = 2 * hf + cl;
+                    uint32_t sh_[32], sl_[32];
+                    tmem_ld32(lane_base + kColShi + 32 * c, sh_);
+                    tmem_ld32(lane_base + kColSlo + 32 * c, sl_);
+                    tmem_wait_ld();
+                    uint32_t ph[16], pl[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float pp[2];
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 k4 = *reinterpret_cast<const float4*>(kal_j + 32 * c + 4 * e4);
+                        const float4 v4 = *reinterpret_cast<const float4*>(vsu_j + 32 * c + 4 * e4);
+                        const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+                        const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+                        float pp[4];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int t = t0 + 32 * c + e + u;
-                        const int S = static_cast<int>(sh_[e + u]) * 256 + static_cast<int>(sl_[e + u]) - cq;
-                        const float z = static_cast<float>(S) * ksc[32 * c + e + u] * zs;
-                        const bool on = valid && t <= pos;
-                        const float pe = on ? ptx::ex2(z - mb) : 0.f;
-                        lsum += pe;
-                        pp[u] = on ? pe * vsc[32 * c + e + u] * up : 0.f;
+                        for (int u = 0; u < 4; ++u) {
+                            const int e = 4 * e4 + u;
+                            const int S = static_cast<int>(sh_[e]) * 256 + static_cast<int>(sl_[e]) - cq;
+                            const float x = static_cast<float>(S) * kk[u];
+                            const bool on = unmasked || (valid && t0 + 32 * c + e <= pos);
+                            const float pe = on ? ptx::ex2(fmaf(x, zs, -mb)) : 0.f;
+                            lsum += pe;
+                            pp[u] = pe * vv[u];
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; u += 2) {
+                            const __half2 hh = __floats2half2_rn(pp[u], pp[u + 1]);
+                            const float2 hfl = __half22float2(hh);
+                            const __half2 ll = __floats2half2_rn(pp[u] - hfl.x, pp[u + 1] - hfl.y);
+                            ph[2 * e4 + (u >> 1)] = *reinterpret_cast<const uint32_t*>(&hh);
+                            pl[2 * e4 + (u >> 1)] = *reinterpret_cast<const uint32_t*>(&ll);
+                        }
                     }
-                    const __half2 hh = __floats2half2_rn(pp[0], pp[1]);
-                    const float2 hf = __half22float2(hh);
-                    const __half2 ll = __floats2half2_rn(pp[0] - hf.x, pp[1] - hf.y);
-                    ph[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
-                    pl[e >> 1] = *reinterpret_cast<const uint32_t*>(&ll);
-                }
-                // tokens 32c .. 32c + 31: atom c / 2, chunks 4 (c % 2) .. + 3
+                    // tokens 32c .. 32c + 31: atom c / 2 = hf, chunks 4 cl .. + 3
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const int kc = 4 * (c & 1) + x;
-                    const uint32_t off = (c >> 1) * 16384 + i_row * 128 + ((kc ^ (i_row & 7)) << 4);
-                    *reinterpret_cast<uint4*>(smem + kPhi + off) =
-                        make_uint4(ph[4 * x], ph[4 * x + 1], ph[4 * x + 2], ph[4 * x + 3]);
-                    *reinterpret_cast<uint4*>(smem + kPlo + off) =
-                        make_uint4(pl[4 * x], pl[4 * x + 1], pl[4 * x + 2], pl[4 * x + 3]);
+                    for (int x = 0; x < 4; ++x) {
+                        const int kc = 4 * cl + x;
+                        const uint32_t off = hf * 16384 + i_row * 128 + ((kc ^ (i_row & 7)) << 4);
+                        *reinterpret_cast<uint4*>(smem + kPhi + off) =
+                            make_uint4(ph[4 * x], ph[4 * x + 1], ph[4 * x + 2], ph[4 * x + 3]);
+                        *reinterpret_cast<uint4*>(smem + kPlo + off) =
+                            make_uint4(pl[4 * x], pl[4 * x + 1], pl[4 * x + 2], pl[4 * x + 3]);
+                    }
                 }
             }
             tc_fence_before();
@@ -495,11 +560,13 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             if (lane == 0) ptx::mbar_arrive(bar_sfree);     // S read: the next Q K^T may start
             l_run = l_run * alpha + lsum;
             m_run = m_new;
-            // ---- V tile row i_row as exact f16 (byte - 128) into the MN-major B tile
-            {
+            // ---- V tile row i_row (this half's head_dim) as exact f16
+            // (byte - 128) into the MN-major B tile (atom hf)
+            if (live) {
                 const uint8_t* vrow = smem + kStage0 + s * kStageBytes + kStV + i_row * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {            // 16 head_dim values per source chunk
+                for (int cc = 0; cc < 4; ++cc) {         // 16 head_dim values per source chunk
+                    const int c = 4 * hf + cc;
                     const uint4 raw = *reinterpret_cast<const uint4*>(vrow + ((c ^ (i_row & 7)) << 4));
                     const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
                     uint32_t f[8];
@@ -508,9 +575,8 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                         f[2 * w] = ptx::bytes_to_f16x2(w4[w], 0x4140u);
                         f[2 * w + 1] = ptx::bytes_to_f16x2(w4[w], 0x4342u);
                     }
-                    const int a = c >> 2;                // d = 16 c: atom d / 64
-                    const int k0 = 2 * (c & 3);          // chunks (d % 64) / 8 and + 1
-                    const uint32_t base = kV16 + a * 16384 + i_row * 128;
+                    const int k0 = 2 * cc;               // chunks (d % 64) / 8 and + 1
+                    const uint32_t base = kV16 + hf * 16384 + i_row * 128;
                     *reinterpret_cast<uint4*>(smem + base + ((k0 ^ (i_row & 7)) << 4)) =
                         make_uint4(f[0], f[1], f[2], f[3]);
                     *reinterpret_cast<uint4*>(smem + base + (((k0 + 1) ^ (i_row & 7)) << 4)) =
@@ -525,12 +591,16 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 ptx::mbar_arrive(bar_empty + 8 * s);    // V and scales consumed
             }
         }
-        // ---- the row: (run * f + last tile) * 2^-kv / l
-        if (ntile > 0 && wait(bar_odone, (ntile - 1) & 1)) {
+        // ---- the row: (run * f + last tile) * 2^-kv / l, l over both halves
+        lx[128 * hf + i_row] = l_run;
+        row_sync();
+        const float l_tot = lx[i_row] + lx[128 + i_row];
+        if (ntile > 0 && live && wait(bar_odone, (ntile - 1) & 1)) {
             tc_fence_after();
-            const float f = (valid && l_run > 0.f) ? pow2i_f(-kv) / l_run : 0.f;
+            const float f = (valid && l_tot > 0.f) ? pow2i_f(-kv) / l_tot : 0.f;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int cl = 0; cl < 2; ++cl) {
+                const int c = 2 * hf + cl;
                 uint32_t ot[32], orn[32];
                 tmem_ld32(lane_base + kColO + 32 * c, ot);
                 if (ntile >= 2) tmem_ld32(lane_base + kColRun + 32 * c, orn);
@@ -547,10 +617,10 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                         dst[x] = make_float4(o_[4 * x], o_[4 * x + 1], o_[4 * x + 2], o_[4 * x + 3]);
                 }
             }
-        } else if (valid || (L < 0 && qi < T)) {
+        } else if (ntile == 0 && (valid || (L < 0 && qi < T))) {
             // no key (an empty or rejected sequence): a zero row
-            float4* dst = reinterpret_cast<float4*>(p.out + orow * kDim);
-            for (int x = 0; x < kDim / 4; ++x) dst[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+            float4* dst = reinterpret_cast<float4*>(p.out + orow * kDim + 64 * hf);
+            for (int x = 0; x < 16; ++x) dst[x] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
     tc_fence_before();
