@@ -43,6 +43,7 @@ _PROTOS = {
     "kvq_dequant": (_I, [_P, _P, _I64, _I, _I, _P, _P]),
     "kvq_status_string": (ctypes.c_char_p, [_I]),
     "kvq_read_error": (_I, [_P, _P, _P]),
+    "kvq_check_error": (_I, [_P, _P]),
     "kvq_cache_bytes": (_I64, [_I64, _I64, _I64, _I, _I]),
     "kvq_version": (ctypes.c_char_p, []),
     "kvq_decode_attn_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _I, _P, _P]),

@@ -476,6 +476,10 @@ kvq_status kvq_read_error(int32_t* d_err, int32_t* bits, kvq_stream_t stream) {
     return h ? KVQ_ERR_DEVICE_FLAG : KVQ_OK;
 }
 
+kvq_status kvq_check_error(int32_t* d_err, kvq_stream_t stream) {
+    return kvq_read_error(d_err, nullptr, stream);
+}
+
 int64_t kvq_cache_bytes(int64_t layers, int64_t Hk, int64_t seq, int D, kvq_scale_mode mode) {
     // per-head / per-channel scales are per (sequence, kv head), not per token
     const int64_t ng = mode == KVQ_SCALE_GROUP32 ? D / 32 : (is_fp8(mode) || is_static(mode)) ? 0 : 1;

@@ -36,23 +36,21 @@ append_kernel(AppendParams p, int lanes_log2) {
     const int P = 1 << lanes_log2;               // lanes per row
     const int lane = threadIdx.x & 31;
     const int sub = lane & (P - 1);              // lane index inside the row
-    const int rows_per_warp = 32 >> lanes_log2;
-    const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * kAppendThreads + threadIdx.x) >> 5;
-    const int64_t row = warp_global * rows_per_warp + (lane >> lanes_log2);
-    const int64_t rows_per_tensor = static_cast<int64_t>(p.B) * p.Hk * p.T;
+    // CTA = one (K or V, sequence, kv head) unit (blockIdx.x) and a block of
+    // its tokens (blockIdx.y): the unit's indices are the same for the whole
+    // CTA, and a lane's token is its row within the block
+    const int units = p.B * p.Hk;
+    const int which = static_cast<int>(blockIdx.x) >= units;      // 0: K, 1: V
+    const int bh = static_cast<int>(blockIdx.x) - which * units;
+    const int b = bh / p.Hk;
+    const int h = bh - b * p.Hk;
+    const int rows_per_cta = (static_cast<int>(blockDim.x) >> 5) * (32 >> lanes_log2);
+    const int t = static_cast<int>(blockIdx.y) * rows_per_cta +
+                  (static_cast<int>(threadIdx.x) >> 5) * (32 >> lanes_log2) + (lane >> lanes_log2);
     // Every lane stays to the end of the shuffles below (full-warp masks);
-    // lanes past the last row just carry no data.
-    const bool row_ok = row < 2 * rows_per_tensor;
-
-    const int which = row_ok && row >= rows_per_tensor;    // 0: K, 1: V
-    const int64_t r = row_ok ? row - which * rows_per_tensor : 0;
-    // (row, kv head, token) in 32-bit arithmetic (the host keeps 2 B Hk T
-    // below 2^31): 64-bit divisions would cost more than the rest of the row
-    const uint32_t r32 = static_cast<uint32_t>(r);
-    const uint32_t bh = r32 / static_cast<uint32_t>(p.T);
-    const int t = static_cast<int>(r32 - bh * static_cast<uint32_t>(p.T));
-    const int b = static_cast<int>(bh / static_cast<uint32_t>(p.Hk));
-    const int h = static_cast<int>(bh - static_cast<uint32_t>(b) * static_cast<uint32_t>(p.Hk));
+    // lanes past the last token just carry no data.
+    const bool row_ok = t < p.T;
+    const int64_t r = static_cast<int64_t>(bh) * p.T + (row_ok ? t : 0);   // source row
 
     // ---- destination row (skip and flag when out of range)
     int64_t dst_row = -1;
@@ -67,12 +65,10 @@ append_kernel(AppendParams p, int lanes_log2) {
             if (p0 < 0 || p0 + p.T > cap) {
                 flag = KVQ_DEVERR_POS;
             } else {
-                const int64_t g = p0 + t;
-                const int32_t page =
-                    p.table[static_cast<int64_t>(b) * p.max_pages + g / p.page_size];
+                const int64_t g = p0 + t;                // (pages of 16 tokens)
+                const int32_t page = p.table[static_cast<int64_t>(b) * p.max_pages + (g >> 4)];
                 if (page < 0 || page >= p.num_pages) flag = KVQ_DEVERR_PAGE;
-                else dst_row = (static_cast<int64_t>(page) * p.Hk + h) * p.page_size
-                               + g % p.page_size;
+                else dst_row = (static_cast<int64_t>(page) * p.Hk + h) * 16 + (g & 15);
             }
         }
     }
@@ -327,17 +323,20 @@ cudaError_t launch_append_calibrate(const AppendParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
-    if (2ll * p.B * p.Hk * p.T >= (1ll << 31)) return cudaErrorInvalidValue;   // 32-bit row index
     const int nvec = p.D >> 3;
     int lanes_log2 = 0;
     while ((1 << lanes_log2) < nvec) ++lanes_log2;
-    const int64_t rows = 2ll * p.B * p.Hk * p.T;
-    const int rows_per_block = (kAppendThreads / 32) * (32 >> lanes_log2);
-    const int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
-    if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
+    // one CTA per (K or V, sequence, kv head) and block of tokens; a small
+    // append takes only the warps its tokens need
+    const int64_t units = 2ll * p.B * p.Hk;
+    const int64_t lanes = static_cast<int64_t>(p.T) << lanes_log2;
+    const int threads = static_cast<int>(lanes >= kAppendThreads ? kAppendThreads : (lanes + 31) / 32 * 32);
+    const int rows_per_block = (threads / 32) * (32 >> lanes_log2);
+    const int64_t tblocks = (p.T + rows_per_block - 1) / rows_per_block;
+    if (units > 0x7fffffffll || tblocks > 65535) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
-    cfg.blockDim = dim3(kAppendThreads, 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(units), static_cast<unsigned>(tblocks), 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

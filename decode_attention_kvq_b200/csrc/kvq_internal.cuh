@@ -39,12 +39,16 @@ __device__ __forceinline__ float q8_scale(float amax) {
 // unless r lies within 1e-4 of a point halfway between two integers, the
 // rounded quotient lies strictly inside the same interval (k - 0.5, k + 0.5)
 // and rounds to the same integer as r; those near-ties take the IEEE division.
-// Beyond |x / s| = 128 both roundings clamp to the same byte.
+// With t = |r| + 0.5 (exact while |r| < 2^22), |r| is within 1e-4 of a tie
+// exactly when t is within 1e-4 of an integer, and round_half_away(|r|) is
+// floor(t).  Beyond |x / s| = 128 every rounding clamps to the same byte (at
+// and above 2^22 every t is an integer: the division decides).
 __device__ __forceinline__ int round_quotient(float x, float s, float inv) {
     const float r = __fmul_rn(x, inv);
-    const float a = fabsf(r);
-    if (fabsf(a - floorf(a) - 0.5f) < 1e-4f) return static_cast<int>(roundf(__fdiv_rn(x, s)));
-    return static_cast<int>(roundf(r));
+    const float t = __fadd_rn(fabsf(r), 0.5f);
+    if (fabsf(__fadd_rn(t, -rintf(t))) < 1e-4f) return static_cast<int>(roundf(__fdiv_rn(x, s)));
+    const int k = static_cast<int>(floorf(t));
+    return r < 0.f ? -k : k;
 }
 
 // the stored byte of x under scale s (inv = __frcp_rn(s))

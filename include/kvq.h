@@ -509,6 +509,11 @@ const char *kvq_status_string(kvq_status status);
  */
 kvq_status kvq_read_error(int32_t *d_err, int32_t *bits, kvq_stream_t stream);
 
+/* kvq_read_error without the bits: synchronises `stream`, clears the device
+ * error word and returns KVQ_OK (it was 0) or KVQ_ERR_DEVICE_FLAG (for
+ * tests; the name of the helper in the boundary's plan). */
+kvq_status kvq_check_error(int32_t *d_err, kvq_stream_t stream);
+
 /*
  * Bytes of an INT8 cache with fp32 scales: layers * 2 * Hk * seq * (D + 4 * NG)
  * (NG = 0 for the FP8 modes).

@@ -195,6 +195,13 @@ def test_append_decode_rejects_bad_arguments(kvq):
 
 
 @needs_no_gpu
+def test_error_word_helpers_reject_bad_pointers(kvq):
+    assert kvq.lib.kvq_read_error(None, None, None) == 1
+    assert kvq.lib.kvq_check_error(None, None) == 1
+    assert kvq.lib.kvq_check_error(FAKE + 2, None) == 1      # misaligned word
+
+
+@needs_no_gpu
 def test_chunk_rejects_bad_arguments(kvq):
     lib = kvq.lib
     cv = kvq.CacheView(FAKE, FAKE, FAKE, FAKE, 0, 4096, 0, 0, 0)
