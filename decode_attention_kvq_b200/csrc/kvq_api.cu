@@ -187,8 +187,6 @@ kvq_status attend(const uint16_t* q, int B, int Hq, int Hk, int T, int D, kvq_sc
                                        : static_cast<int64_t>(B) * Hk * kv->max_seq;
     const bool simt = dense || (D != 64 && D != 128) || B > kvq::kMaxBatch ||
                       rows >= (1ll << 31);
-    // the mixed cache's window kernel folds at most 16 rows per kv head
-    if (recent && G > 16) return KVQ_ERR_UNSUPPORTED;
     if (B == 0) return KVQ_OK;
 
     int chunk = 0, splits = 0;

@@ -17,7 +17,9 @@
 
 #include <atomic>
 
+#include "kvq_devonce.h"
 #include "kvq_internal.cuh"
+#include "kvq_ptx.cuh"
 
 namespace kvq {
 namespace {
@@ -261,182 +263,216 @@ size_t combine_one_spread_smem(int rows) {
 
 // Mixed cache (abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
 // OptimizedQuantizedKvCache::get_kv: the INT8 part dequantised, then the
-// unquantised recent tokens): one CTA per (b, kv head) and its G query heads.
-// The newest min(L, W) tokens sit in the bf16 ring (position g in row g % W);
-// they are walked in tiles of kRecTile tokens staged in shared memory (K and V
-// rows by 16-byte loads), with an online softmax per head in fp32: scores by
-// one warp per token (lanes over head_dim, all G heads at once), then each
-// thread updates its (head, head_dim) outputs from the tile's V rows.  The
-// split kernel's INT8 partials (every slot below the INT8 part's chunk count
-// with a finite m) are folded in at the end and the rows written.
+// unquantised recent tokens): one CTA per (b, q head).  The newest min(L, W)
+// tokens sit in the bf16 ring of the head's kv head (position g in row
+// g % W).  They are walked in tiles of up to tw tokens (the whole window when
+// it fits the dynamic shared memory), each tile's K and V rows brought in by
+// one round of asynchronous 16-byte copies, with an online softmax in fp32:
+// the tile's scores by the eight warps (a warp per token, lanes over
+// head_dim), its maximum and weights by one warp (lanes over tokens), then
+// thread d updates output value d.  The split kernel's INT8 partials of the
+// row (every slot below the INT8 part's chunk count with a finite m) are
+// folded in at the end; the first kRecPre slots' m, l and values are loaded
+// before the window work, so their latency overlaps it.
+namespace {
 constexpr int kRecThreads = 256;
 constexpr int kRecWarps = kRecThreads / 32;
-constexpr int kRecTile = 16;                    // window tokens per shared-memory tile
-constexpr int kRecMaxG = 16;
+constexpr int kRecSmem = 96 * 1024;             // dynamic shared memory budget of a tile
+constexpr int kRecMaxSlots = 64;                // INT8 partials staged per round
+constexpr int kRecPre = 16;                     // partial slots prefetched into registers
+
+int recent_tile(int W, int D) {                 // window tokens per tile
+    const int fit = (kRecSmem - 64) / (4 * D + 4);
+    return W < fit ? W : fit;
+}
+size_t recent_smem(int tw, int D) { return static_cast<size_t>(tw) * (4 * D + 4); }
+
 __global__ void __launch_bounds__(kRecThreads)
-decode_recent_combine(DecodeParams p) {
-    __shared__ __align__(16) float s_q[kRecMaxG * 256];             // the G query rows (fp32)
-    __shared__ __align__(16) uint16_t s_k[kRecTile * 256], s_v[kRecTile * 256];
-    __shared__ float s_p[kRecMaxG][kRecTile];                       // scores, then weights
-    __shared__ float s_m[kRecMaxG], s_l[kRecMaxG], s_a[kRecMaxG];   // running max, sum, rescale
+decode_recent_combine(DecodeParams p, int tw) {
+    extern __shared__ __align__(16) uint8_t rec_smem[];
+    uint16_t* s_k = reinterpret_cast<uint16_t*>(rec_smem);            // [tw][D]
+    uint16_t* s_v = s_k + static_cast<size_t>(tw) * p.D;              // [tw][D]
+    float* s_p = reinterpret_cast<float*>(s_v + static_cast<size_t>(tw) * p.D);   // [tw]
+    __shared__ __align__(16) float s_q[256];                          // the query row (fp32)
+    __shared__ float s_st[4];                                         // m, l, tile rescale
+    __shared__ float s_m8[kRecMaxSlots], s_l8[kRecMaxSlots];
     grid_dep_wait();                    // the split kernel's partials are complete
     grid_dep_launch();
-    const int unit = blockIdx.x;                        // b * Hk + hk
-    const int b = unit / p.Hk;
-    const int G = p.G, D = p.D, W = p.recent;
+    const int64_t row = blockIdx.x;                     // b * Hq + q head
+    const int b = static_cast<int>(row / p.Hq);
+    const int unit = static_cast<int>(row / p.G);       // b * Hk + kv head
+    const int D = p.D, W = p.recent;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t bh0 = static_cast<int64_t>(unit) * G;  // first q row (b * Hq + hk * G)
     const int64_t cap = p.page_size ? static_cast<int64_t>(p.max_pages) * p.page_size : p.max_seq;
     const int64_t plan = static_cast<int64_t>(p.splits) * p.chunk;
     const int L = p.seq_lens[b];
     const int n8 = walked_len(L, cap, plan, 1, 0, W);   // INT8 part walked by the split kernel
     if (n8 < 0) {                                       // flagged by the split kernel
-        for (int i = tid; i < G * D; i += kRecThreads) p.out[bh0 * D + i] = 0.f;
+        for (int d = tid; d < D; d += kRecThreads) p.out[row * D + d] = 0.f;
         return;
     }
     const int Lq = L > W ? L - W : 0;
     const int nr = L - Lq;                              // tokens in the window
-    for (int i = tid; i < G * D; i += kRecThreads)
-        s_q[i] = bf16_bits_to_f32(p.q[bh0 * D + i]);
-    if (tid < G) {
-        s_m[tid] = -INFINITY;
-        s_l[tid] = 0.f;
+    const int ns = (n8 + p.chunk - 1) / p.chunk;        // INT8 partial slots
+    const float* m8 = p.ws_m + row * p.splits;
+    const float* l8 = p.ws_l + row * p.splits;
+    const float* o8 = p.ws_o + row * p.splits * D + (tid < D ? tid : 0);
+    // the first slots' m, l (shared) and this thread's values (registers)
+    const int npre = min(ns, kRecPre);
+    if (tid < npre) {
+        s_m8[tid] = m8[tid];
+        s_l8[tid] = l8[tid];
     }
-    // this thread's (head, head_dim) outputs: pairs tid + kRecThreads * k
-    constexpr int kMaxPairs = kRecMaxG * 256 / kRecThreads;
-    float o[kMaxPairs];
+    float ovp[kRecPre];
 #pragma unroll
-    for (int k = 0; k < kMaxPairs; ++k) o[k] = 0.f;
-    const int npair = G * D;
+    for (int u = 0; u < kRecPre; ++u) ovp[u] = u < npre ? o8[static_cast<int64_t>(u) * D] : 0.f;
+    for (int d = tid; d < D; d += kRecThreads) s_q[d] = bf16_bits_to_f32(p.q[row * D + d]);
+    if (tid == 0) {
+        s_st[0] = -INFINITY;
+        s_st[1] = 0.f;
+    }
+    float o = 0.f;                                      // output value d = tid
     const int64_t ring0 = static_cast<int64_t>(unit) * W;
     const int vec = D / 8;                              // 16-byte chunks per row
-    for (int i0 = 0; i0 < nr; i0 += kRecTile) {
-        const int n = min(kRecTile, nr - i0);
+    const uint32_t sk_a = ptx::smem_u32(s_k), sv_a = ptx::smem_u32(s_v);
+    for (int i0 = 0; i0 < nr; i0 += tw) {
+        const int n = min(tw, nr - i0);
         __syncthreads();                                // the previous tile is consumed
         for (int c = tid; c < n * vec; c += kRecThreads) {
-            const int t = c / vec, x = c % vec;
-            const int64_t row = ring0 + (Lq + i0 + t) % W;
-            reinterpret_cast<uint4*>(s_k)[t * vec + x] =
-                reinterpret_cast<const uint4*>(p.rk + row * D)[x];
-            reinterpret_cast<uint4*>(s_v)[t * vec + x] =
-                reinterpret_cast<const uint4*>(p.rv + row * D)[x];
+            const int t = c / vec, x = c - (c / vec) * vec;
+            const int64_t rr = ring0 + (Lq + i0 + t) % W;
+            ptx::cp_async_16(sk_a + 16u * static_cast<uint32_t>(c), p.rk + rr * D + 8 * x);
+            ptx::cp_async_16(sv_a + 16u * static_cast<uint32_t>(c), p.rv + rr * D + 8 * x);
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");
         __syncthreads();
-        // scores (log2 domain): one warp per token, lanes over head_dim
-        for (int t = warp; t < n; t += kRecWarps) {
-            float acc[kRecMaxG];
-#pragma unroll
-            for (int h = 0; h < kRecMaxG; ++h) acc[h] = 0.f;
+        // scores (log2 domain): a warp takes four tokens at a time (lanes over
+        // head_dim), their four reduction trees interleaved
+        for (int t0 = 4 * warp; t0 < n; t0 += 4 * kRecWarps) {
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
             for (int d = lane; d < D; d += 32) {
-                const float kv = bf16_bits_to_f32(s_k[t * D + d]);
+                const float qd = s_q[d];
 #pragma unroll
-                for (int h = 0; h < kRecMaxG; ++h)
-                    if (h < G) acc[h] = fmaf(s_q[h * D + d], kv, acc[h]);
+                for (int u = 0; u < 4; ++u)
+                    if (t0 + u < n) a[u] = fmaf(qd, bf16_bits_to_f32(s_k[(t0 + u) * D + d]), a[u]);
             }
 #pragma unroll
-            for (int h = 0; h < kRecMaxG; ++h) {
-                if (h >= G) break;
-                float a = acc[h];
+            for (int off = 16; off > 0; off >>= 1)
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-                if (lane == 0) s_p[h][t] = a * p.scale_log2;
+                for (int u = 0; u < 4; ++u) a[u] += __shfl_xor_sync(0xffffffffu, a[u], off);
+            if (lane < 4 && t0 + lane < n) {
+                const float v = lane == 0 ? a[0] : lane == 1 ? a[1] : lane == 2 ? a[2] : a[3];
+                s_p[t0 + lane] = v * p.scale_log2;
             }
         }
         __syncthreads();
-        // online softmax per head (one thread per head)
-        if (tid < G) {
+        // online softmax over the tile: one warp, lanes over tokens
+        if (warp == 0) {
             float mt = -INFINITY;
-            for (int t = 0; t < n; ++t) mt = fmaxf(mt, s_p[tid][t]);
-            const float mn = fmaxf(s_m[tid], mt);
-            const float a = exp2f(s_m[tid] - mn);       // 0 while the max was -inf
+            for (int t = lane; t < n; t += 32) mt = fmaxf(mt, s_p[t]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+            const float mo = s_st[0];
+            const float mn = fmaxf(mo, mt);
             float add = 0.f;
-            for (int t = 0; t < n; ++t) {
-                const float e = exp2f(s_p[tid][t] - mn);
-                s_p[tid][t] = e;
+            for (int t = lane; t < n; t += 32) {
+                const float e = exp2f(s_p[t] - mn);
+                s_p[t] = e;
                 add += e;
             }
-            s_l[tid] = s_l[tid] * a + add;
-            s_m[tid] = mn;
-            s_a[tid] = a;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) add += __shfl_xor_sync(0xffffffffu, add, off);
+            if (lane == 0) {
+                const float a = exp2f(mo - mn);         // 0 while the max was -inf
+                s_st[1] = s_st[1] * a + add;
+                s_st[0] = mn;
+                s_st[2] = a;
+            }
         }
         __syncthreads();
+        if (tid < D) {                                  // four partial sums: a short chain
+            float ac[4] = {o * s_st[2], 0.f, 0.f, 0.f};
+            int t = 0;
+            for (; t + 4 <= n; t += 4)
 #pragma unroll
-        for (int k = 0; k < kMaxPairs; ++k) {
-            const int idx = tid + kRecThreads * k;
-            if (idx >= npair) break;
-            const int h = idx / D, d = idx % D;
-            float acc = o[k] * s_a[h];
-            for (int t = 0; t < n; ++t) acc = fmaf(s_p[h][t], bf16_bits_to_f32(s_v[t * D + d]), acc);
-            o[k] = acc;
+                for (int u = 0; u < 4; ++u)
+                    ac[u] = fmaf(s_p[t + u], bf16_bits_to_f32(s_v[(t + u) * D + tid]), ac[u]);
+            for (; t < n; ++t) ac[0] = fmaf(s_p[t], bf16_bits_to_f32(s_v[t * D + tid]), ac[0]);
+            o = (ac[0] + ac[1]) + (ac[2] + ac[3]);
         }
     }
     __syncthreads();
-    // the INT8 partials of each head: their max and weighted sum (warp per head)
-    const int ns = (n8 + p.chunk - 1) / p.chunk;
-    for (int h = warp; h < G; h += kRecWarps) {
-        const float* m8 = p.ws_m + (bh0 + h) * p.splits;
-        const float* l8 = p.ws_l + (bh0 + h) * p.splits;
-        float M = s_m[h];
-        for (int j = lane; j < ns; j += 32) M = fmaxf(M, m8[j]);
+    // the row's INT8 partials: their maximum and weighted sum, then output d;
+    // empty slots (m = -inf) are dropped by selection (no load behind a branch)
+    float M = s_st[0];
+    float lsum = 0.f;                                   // relative to M, the window's l not included
+    float acc = 0.f;
+    const float mw = s_st[0], lw = s_st[1];
+    auto rescale = [&](int nj) {                        // the new maximum over nj staged slots
+        float Mn = M;
+        for (int j = 0; j < nj; ++j) Mn = fmaxf(Mn, s_m8[j]);
+        const float a = M == -INFINITY ? 0.f : exp2f(M - Mn);
+        acc *= a;
+        lsum *= a;
+        M = Mn;
+    };
+    auto add = [&](int j, float value) {                // staged slot j with this thread's value
+        const float mj = s_m8[j];
+        const bool live = mj != -INFINITY;
+        const float w = live ? exp2f(mj - M) : 0.f;
+        acc = live ? fmaf(w, value, acc) : acc;
+        lsum = live ? fmaf(w, s_l8[j], lsum) : lsum;
+    };
+    rescale(npre);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        float ls = 0.f;
-        for (int j = lane; j < ns; j += 32)
-            if (m8[j] != -INFINITY) ls = fmaf(exp2f(m8[j] - M), l8[j], ls);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
-        if (lane == 0) {
-            const float aw = s_m[h] == -INFINITY ? 0.f : exp2f(s_m[h] - M);
-            const float tot = ls + s_l[h] * aw;
-            s_a[h] = aw;                                // the window's weight
-            s_l[h] = tot > 0.f ? 1.f / tot : 0.f;       // the normaliser
-            s_m[h] = M;
+    for (int u = 0; u < kRecPre; ++u)
+        if (u < npre) add(u, ovp[u]);
+#pragma unroll 1
+    for (int j0 = npre; j0 < ns; j0 += kRecMaxSlots) {
+        const int nj = min(kRecMaxSlots, ns - j0);
+        __syncthreads();                                // s_m8, s_l8 free
+        if (tid < nj) {
+            s_m8[tid] = m8[j0 + tid];
+            s_l8[tid] = l8[j0 + tid];
         }
+        __syncthreads();
+        rescale(nj);
+        for (int j = 0; j < nj; ++j) add(j, o8[static_cast<int64_t>(j0 + j) * D]);
     }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < kMaxPairs; ++k) {
-        const int idx = tid + kRecThreads * k;
-        if (idx >= npair) break;
-        const int h = idx / D, d = idx % D;
-        const int64_t row = bh0 + h;
-        const float M = s_m[h];
-        const float* m8 = p.ws_m + row * p.splits;
-        const float* o8 = p.ws_o + row * p.splits * D + d;
-        float acc = o[k] * s_a[h];
-        int j = 0;
-        for (; j + 4 <= ns; j += 4) {                   // four slots' loads in flight
-            float mj[4], oj[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                mj[u] = m8[j + u];
-                oj[u] = o8[static_cast<int64_t>(j + u) * D];
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (mj[u] != -INFINITY) acc = fmaf(exp2f(mj[u] - M), oj[u], acc);
-        }
-        for (; j < ns; ++j) {
-            const float mj = m8[j];
-            if (mj != -INFINITY) acc = fmaf(exp2f(mj - M), o8[static_cast<int64_t>(j) * D], acc);
-        }
-        p.out[row * D + d] = acc * s_l[h];
+    if (tid < D) {
+        const float aw = mw == -INFINITY ? 0.f : exp2f(mw - M);
+        const float tot = lsum + lw * aw;
+        p.out[row * D + tid] = tot > 0.f ? (acc + o * aw) / tot : 0.f;
     }
 }
 
+}  // namespace
+
 cudaError_t launch_recent_combine(const DecodeParams& p, cudaStream_t s) {
-    if (p.recent < 1 || p.recent > kMaxRecent || p.G > kRecMaxG || p.D > 256 || p.qlen != 1)
+    if (p.recent < 1 || p.recent > kMaxRecent || p.D > 256 || p.qlen != 1 ||
+        static_cast<int64_t>(p.B) * p.Hq > 0x7fffffffll)
         return cudaErrorInvalidValue;
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = once_per_device(done, dev, cudaSuccess, [] {
+        return cudaFuncSetAttribute(decode_recent_combine,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kRecSmem);
+    });
+    if (e != cudaSuccess) return e;
+    const int tw = recent_tile(p.recent, p.D);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.B * p.Hk, 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(static_cast<int64_t>(p.B) * p.Hq), 1, 1);
     cfg.blockDim = dim3(kRecThreads, 1, 1);
+    cfg.dynamicSmemBytes = recent_smem(tw, p.D);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_recent_combine, p);
+    return cudaLaunchKernelEx(&cfg, decode_recent_combine, p, tw);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s, bool simt) {

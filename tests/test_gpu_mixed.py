@@ -118,3 +118,18 @@ def test_mixed_many_units(mode):
     c.assert_bit_exact()
     c.check_decode(Hk * 8, seed=7)
     c.check_decode(Hk * 2, seed=8, num_splits=5)
+
+
+@pytest.mark.parametrize("D,G,W", [(128, 32, 2048), (96, 4, 200), (256, 8, 40)])
+def test_mixed_wide_groups_long_windows_other_head_dims(D, G, W):
+    """The window kernel takes one CTA per (sequence, q head): 32 heads per kv
+    head, the longest window (2048 tokens, many tiles), and head dims whose
+    INT8 part runs on the CUDA-core split kernel."""
+    B, Hk, S = 2, 2, 3000
+    c = MixedPair(B, Hk, S, D, W, "per_token", seed=D + G)
+    c.append([2500, 100], seed=3)
+    c.assert_bit_exact()
+    c.check_decode(Hk * G, seed=4)
+    c.append([1, 1], seed=5)
+    c.assert_bit_exact()
+    c.check_decode(Hk * G, seed=6, num_splits=3)
