@@ -2,10 +2,9 @@
 // that cannot allocate device memory.
 //
 // Some callers cannot call cudaMalloc (or any allocator) at the point where
-// they run attention: code executing inside a CUDA graph capture that must
-// not allocate, embedded or plugin hosts that hand the library only their
-// own input/output buffers, or runtimes whose allocator is not reachable
-// from this C interface.  kvq_decode_attn needs a split-K scratch workspace
+// they run attention: embedded or plugin hosts that hand the library only
+// their own input/output buffers, or runtimes whose allocator is not
+// reachable from this C interface.  kvq_decode_attn needs a split-K scratch workspace
 // from its caller; this entry point instead uses a fixed-size scratch array
 // that lives in the library itself (a file-scope __device__ array, present on
 // every GPU that loads the library until the process exits).

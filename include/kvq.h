@@ -407,10 +407,10 @@ kvq_status kvq_dequant(const uint8_t *q, const float *scale, int64_t rows, int D
  * kvq_decode_attn_noalloc -- kvq_decode_attn for callers that cannot allocate
  * device memory.  The pages this library follows have no counterpart of this
  * call; it exists for integration.  Some callers cannot call cudaMalloc (or
- * any allocator) where they run attention: code inside a CUDA graph capture
- * that must not allocate, plugin or embedded hosts that only hand over their
- * own input and output buffers, runtimes whose allocator this C interface
- * cannot reach.  This entry point takes the same arguments as
+ * any allocator) where they run attention: plugin or embedded hosts that
+ * only hand over their own input and output buffers, runtimes whose
+ * allocator this C interface cannot reach.  This entry point takes the same
+ * arguments as
  * kvq_decode_attn minus the workspace, and uses instead a split-K scratch
  * array that lives inside the library: a file-scope __device__ array of
  * kvq_noalloc_scratch_bytes() bytes (16 MiB), present on every GPU that loads
@@ -418,8 +418,7 @@ kvq_status kvq_dequant(const uint8_t *q, const float *scale, int64_t rows, int D
  *  - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
  *    library routine is called.
  *  - The first call on a device looks up the array's device address with
- *    cudaGetSymbolAddress (with that device current) and caches it; make that
- *    first call before any stream capture.
+ *    cudaGetSymbolAddress (with that device current) and caches it.
  *  - Problems whose split-K scratch (kvq_decode_workspace_bytes for the same
  *    arguments) exceeds the array return KVQ_ERR_SCRATCH_TOO_SMALL before
  *    anything is enqueued.
