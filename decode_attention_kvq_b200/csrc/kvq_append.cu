@@ -16,10 +16,10 @@
 // which gives the same byte.
 //
 // Mapping: one "row" is the D values of one (which in {K, V}, b, h, t).  A
-// row is handled by P = next_pow2(D / 8) lanes of a warp, each lane loading
-// 8 bf16 (16 bytes) and storing 8 bytes; the absolute maximum is reduced
-// with xor shuffles inside the row (per token) or inside each 4-lane
-// quarter that covers 32 values (group-32).  The kernel is HBM-bound: per
+// row is handled by P = next_pow2(D / 16) lanes of a warp, each lane loading
+// 16 bf16 (two 16-byte loads) and storing 16 bytes; the absolute maximum is
+// reduced with xor shuffles inside the row (per token) or inside each lane
+// pair that covers 32 values (group-32).  The kernel is HBM-bound: per
 // row it reads 2*D bytes and writes D + 4*NG bytes.  It is launched as a
 // programmatic dependent (waits for the preceding grid before reading).
 #include "kvq_internal.cuh"
@@ -74,68 +74,68 @@ append_kernel(AppendParams p, int lanes_log2) {
     }
     if (flag && sub == 0) raise_flag(p.d_err, flag);
 
-    const int nvec = p.D >> 3;                   // 8-value vectors per row
+    const int nvec = p.D >> 4;                   // 16-value vectors per row (lanes)
     const bool active = row_ok && sub < nvec;
     const uint16_t* src = (which ? p.v_new : p.k_new) + r * p.D;
+    uint8_t* dst = (which ? p.v_dst : p.k_dst) + dst_row * p.D + sub * 16;
 
+    // the lane's 16 values: two 16-byte loads
+    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (active) {
+        const uint4 a = *reinterpret_cast<const uint4*>(src + sub * 16);
+        const uint4 c = *reinterpret_cast<const uint4*>(src + sub * 16 + 8);
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+        w[4] = c.x; w[5] = c.y; w[6] = c.z; w[7] = c.w;
+    }
     if (p.fp8) {                                 // FP8: one byte a value, no scale
         if (!active || dst_row < 0) return;
-        const uint4 raw = *reinterpret_cast<const uint4*>(src + sub * 8);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-        uint32_t packed[2] = {0u, 0u};
+        uint32_t packed[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t h = (w[i >> 1] >> (16 * (i & 1))) & 0xffffu;
-            packed[i >> 2] |= fp8_from_bf16(h, p.fp8) << (8 * (i & 3));
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t hb = (w[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+            packed[i >> 2] |= fp8_from_bf16(hb, p.fp8) << (8 * (i & 3));
         }
-        uint8_t* dst = (which ? p.v_dst : p.k_dst) + dst_row * p.D + sub * 8;
-        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
         return;
     }
 
-    float x[8];
+    float x[16];
     float amax = 0.f;
-    if (active) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(src + sub * 8);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            x[2 * i] = bf16_bits_to_f32(w[i] & 0xffffu);
-            x[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    for (int i = 0; i < 8; ++i) {
+        x[2 * i] = bf16_bits_to_f32(w[i] & 0xffffu);
+        x[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
     }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
     if (p.static_ns) {                           // per head / per channel: stored scales
         if (!active || dst_row < 0) return;
         const float* sc = (which ? p.v_scale : p.k_scale) +
                           (static_cast<int64_t>(b) * p.Hk + h) * p.static_ns;
-        uint32_t packed[2] = {0u, 0u};
+        uint32_t packed[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float si = sc[p.static_ns > 1 ? sub * 8 + i : 0];
+        for (int i = 0; i < 16; ++i) {
+            const float si = sc[p.static_ns > 1 ? sub * 16 + i : 0];
             packed[i >> 2] |= q8_byte(x[i], si, __frcp_rn(si)) << (8 * (i & 3));
         }
-        uint8_t* dst = (which ? p.v_dst : p.k_dst) + dst_row * p.D + sub * 8;
-        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
         return;
     }
-    // reduce inside the group of lanes sharing one scale
-    const int red_lanes = p.group32 ? 4 : P;
+    // reduce inside the group of lanes sharing one scale (group-32: two lanes)
+    const int red_lanes = p.group32 ? 2 : P;
     for (int off = 1; off < red_lanes; off <<= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
 
     if (!active || dst_row < 0) return;
     const float s = q8_scale(amax);
     const float inv = __frcp_rn(s);
-    uint32_t packed[2] = {0u, 0u};
+    uint32_t packed[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) packed[i >> 2] |= q8_byte(x[i], s, inv) << (8 * (i & 3));
-    uint8_t* dst = (which ? p.v_dst : p.k_dst) + dst_row * p.D + sub * 8;
-    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+    for (int i = 0; i < 16; ++i) packed[i >> 2] |= q8_byte(x[i], s, inv) << (8 * (i & 3));
+    *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     float* sdst = which ? p.v_scale : p.k_scale;
     if (p.group32) {
-        if ((sub & 3) == 0) sdst[dst_row * (p.D >> 5) + (sub >> 2)] = s;
+        if ((sub & 1) == 0) sdst[dst_row * (p.D >> 5) + (sub >> 1)] = s;
     } else if (sub == 0) {
         sdst[dst_row] = s;
     }
@@ -323,7 +323,7 @@ cudaError_t launch_append_calibrate(const AppendParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
-    const int nvec = p.D >> 3;
+    const int nvec = p.D >> 4;                   // lanes per row: 16 values each
     int lanes_log2 = 0;
     while ((1 << lanes_log2) < nvec) ++lanes_log2;
     // one CTA per (K or V, sequence, kv head) and block of tokens; a small

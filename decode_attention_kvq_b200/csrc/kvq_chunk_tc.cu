@@ -447,10 +447,13 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             row_sync();                                  // red read; kal, vsu written
             live = live && wait(bar_sfull, j & 1);
             tc_fence_after();
-            // ---- pass 1: the maximum of S * k_scale over this half's tokens
-            // (tiles wholly at or below the row's position need no mask)
+            // ---- pass 1: x = S * k_scale over this half's tokens (-inf where the
+            // causal mask drops the key), its maximum, and x written back over
+            // the S_hi columns so that pass 2 reads one tile and no mask
+            // (a warp whose rows all see the whole half skips the mask test)
             const int tb = t0 + 64 * hf;                 // this half's first token
             const bool unmasked = valid && tb + 63 <= pos;
+            const bool warp_unmasked = __all_sync(0xffffffffu, unmasked);
             float xmax = -INFINITY;
             if (live) {
 #pragma unroll 1
@@ -460,19 +463,39 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     tmem_ld32(lane_base + kColShi + 32 * c, sh_);
                     tmem_ld32(lane_base + kColSlo + 32 * c, sl_);
                     tmem_wait_ld();
+                    if (warp_unmasked) {
 #pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 k4 = *reinterpret_cast<const float4*>(kal_j + 32 * c + 4 * e4);
-                        const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            const float4 k4 = *reinterpret_cast<const float4*>(kal_j + 32 * c + 4 * e4);
+                            const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int e = 4 * e4 + u;
-                            const int S = static_cast<int>(sh_[e]) * 256 + static_cast<int>(sl_[e]) - cq;
-                            const float x = static_cast<float>(S) * kk[u];
-                            if (unmasked || (valid && t0 + 32 * c + e <= pos)) xmax = fmaxf(xmax, x);
+                            for (int u = 0; u < 4; ++u) {
+                                const int e = 4 * e4 + u;
+                                const int S = static_cast<int>(sh_[e]) * 256 + static_cast<int>(sl_[e]) - cq;
+                                const float x = static_cast<float>(S) * kk[u];
+                                xmax = fmaxf(xmax, x);
+                                sh_[e] = __float_as_uint(x);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            const float4 k4 = *reinterpret_cast<const float4*>(kal_j + 32 * c + 4 * e4);
+                            const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int e = 4 * e4 + u;
+                                const int S = static_cast<int>(sh_[e]) * 256 + static_cast<int>(sl_[e]) - cq;
+                                const bool on = valid && t0 + 32 * c + e <= pos;
+                                const float x = on ? static_cast<float>(S) * kk[u] : -INFINITY;
+                                xmax = fmaxf(xmax, x);
+                                sh_[e] = __float_as_uint(x);
+                            }
                         }
                     }
+                    tmem_st32(lane_base + kColShi + 32 * c, sh_);
                 }
+                tmem_wait_st();
             }
             xch[128 * hf + i_row] = xmax;
             row_sync();
@@ -505,32 +528,25 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 tmem_wait_st();
             }
             f_prev = alpha * drop;                       // applies to the running sum at the next fold
-            // ---- pass 2: P'' = 2^(z - m) * v_scale * 2^kv as f16 hi + lo for
-            // this half's tokens (P atom hf)
+            // ---- pass 2: P'' = 2^(x zs - m) * v_scale * 2^kv as f16 hi + lo for
+            // this half's tokens (P atom hf); x = -inf (masked) gives 0
             float lsum = 0.f;
             if (live) {
 #pragma unroll 1
                 for (int cl = 0; cl < 2; ++cl) {
                     const int c = 2 * hf + cl;
-                    uint32_t sh_[32], sl_[32];
-                    tmem_ld32(lane_base + kColShi + 32 * c, sh_);
-                    tmem_ld32(lane_base + kColSlo + 32 * c, sl_);
+                    uint32_t xs[32];
+                    tmem_ld32(lane_base + kColShi + 32 * c, xs);
                     tmem_wait_ld();
                     uint32_t ph[16], pl[16];
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 k4 = *reinterpret_cast<const float4*>(kal_j + 32 * c + 4 * e4);
                         const float4 v4 = *reinterpret_cast<const float4*>(vsu_j + 32 * c + 4 * e4);
-                        const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
                         const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
                         float pp[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            const int e = 4 * e4 + u;
-                            const int S = static_cast<int>(sh_[e]) * 256 + static_cast<int>(sl_[e]) - cq;
-                            const float x = static_cast<float>(S) * kk[u];
-                            const bool on = unmasked || (valid && t0 + 32 * c + e <= pos);
-                            const float pe = on ? ptx::ex2(fmaf(x, zs, -mb)) : 0.f;
+                            const float pe = ptx::ex2(fmaf(__uint_as_float(xs[4 * e4 + u]), zs, -mb));
                             lsum += pe;
                             pp[u] = pe * vv[u];
                         }
