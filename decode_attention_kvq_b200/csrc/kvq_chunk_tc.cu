@@ -196,6 +196,10 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMisc + 96);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMisc + 100);
     float* red = reinterpret_cast<float*>(smem + kMisc + 128);   // [8] per-warp V-scale maxima
+    // [8] per-warp "a row's maximum grew this tile"; [2] by tile parity: P.V of
+    // the tile adds onto the O tile (1) or starts it afresh (0)
+    volatile int* grew = reinterpret_cast<volatile int*>(smem + kMisc + 160);
+    volatile int* pv_acc = reinterpret_cast<volatile int*>(smem + kMisc + 192);
     float* kal = reinterpret_cast<float*>(smem + kAux);          // [2][128] K scales
     float* vsu = kal + 256;                                      // [2][128] V scales * 2^kv
     float* xch = vsu + 256;                                      // [2][128] halves' maxima
@@ -314,14 +318,17 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 tc_commit(bar_empty + 8 * s);       // K consumed
                 if (!wait(bar_pfull, j & 1)) break;
                 tc_fence_after();
-                // O += P'' V: eight k-steps of 16 tokens per part; P rows are
-                // two 64-token atoms, V16 k-steps advance 16 rows of 128 bytes
+                // O (+)= P'' V: eight k-steps of 16 tokens per part; P rows are
+                // two 64-token atoms, V16 k-steps advance 16 rows of 128 bytes.
+                // The tile's first k-step starts the O tile afresh unless the
+                // rows left it unfolded (then the tile adds onto it)
+                const bool onto = j > 0 && pv_acc[j & 1] != 0;
                 for (int part = 0; part < 2; ++part) {
                     const uint32_t pb = sb + (part ? kPlo : kPhi);
                     for (int k = 0; k < 8; ++k) {
                         const uint64_t da = smem_desc(pb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
                         const uint64_t dv = smem_desc(sb + kV16 + k * 2048, 16384, 1024);
-                        tc_mma<false>(tmem + kColO, da, dv, kIdescPv, (part > 0 || k > 0));
+                        tc_mma<false>(tmem + kColO, da, dv, kIdescPv, (onto || part > 0 || k > 0));
                     }
                 }
                 tc_commit(bar_odone);
@@ -405,7 +412,17 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 
         float m_run = -INFINITY, l_run = 0.f;            // l_run: this half's tokens
         int kv = 64;                                     // P'' prescale exponent (CTA-uniform)
-        float f_prev = 1.f;                              // rescale of the running sum (see the fold)
+        // Lazy fold: the O tile adds up the P.V of consecutive tiles while no
+        // row's maximum grows and the prescale stays (they share one scale),
+        // up to kFoldEvery tiles; it is folded into the running sum (O run)
+        // before the P.V of a tile that changes the scale, or at the limit:
+        // run = run * f_run + tile, f_run the factor from the running sum's
+        // scale to the O tile's (one factor per fold: between folds every
+        // factor is 1)
+        constexpr int kFoldEvery = 8;
+        float f_run = 1.f;
+        bool has_run = false;                            // O run holds a sum
+        int n_acc = 0;                                   // tiles summed in the O tile
         bool live = true;                                // no wait has given up
         for (int j = 0; j < ntile; ++j) {
             const int s = j & 1;
@@ -498,36 +515,49 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 tmem_wait_st();
             }
             xch[128 * hf + i_row] = xmax;
+            {
+                const bool g = __any_sync(0xffffffffu, xmax * zs > m_run);
+                if (lane == 0) grew[warp] = g ? 1 : 0;
+            }
             row_sync();
             const float xm = fmaxf(xch[i_row], xch[128 + i_row]);
             const float m_new = fmaxf(m_run, xm * zs);
             const float mb = m_new == -INFINITY ? 0.f : m_new;
-            const float alpha = m_run == -INFINITY ? 1.f : ptx::ex2(m_run - mb);
+            const float alpha = (m_run == -INFINITY || m_new <= m_run) ? 1.f : ptx::ex2(m_run - mb);
+            bool any_grew = false;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) any_grew = any_grew || grew[w] != 0;
+            // fold the O tile into the running sum before this tile's P.V (a
+            // CTA-wide decision: every row reads the same flags)
+            const bool fold_now = j >= 1 && (any_grew || drop != 1.f || n_acc >= kFoldEvery);
             // the previous P.V is done: P, V16 free, O stable
             if (j >= 1) live = live && wait(bar_odone, (j - 1) & 1);
             tc_fence_after();
-            // fold the previous tile's P.V into the running sum (this half's
-            // head_dim columns): run = run * f + tile, f the previous tile's
-            // rescale (the running sum is relative to the tile's maximum and
-            // prescale)
-            if (live && j >= 1) {
+            // the fold (this half's head_dim columns)
+            if (live && fold_now) {
 #pragma unroll 1
                 for (int cl = 0; cl < 2; ++cl) {
                     const int c = 2 * hf + cl;
                     uint32_t ot[32], orn[32];
                     tmem_ld32(lane_base + kColO + 32 * c, ot);
-                    if (j >= 2) tmem_ld32(lane_base + kColRun + 32 * c, orn);
+                    if (has_run) tmem_ld32(lane_base + kColRun + 32 * c, orn);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        orn[e] = __float_as_uint(j >= 2 ? fmaf(__uint_as_float(orn[e]), f_prev,
-                                                               __uint_as_float(ot[e]))
-                                                        : __uint_as_float(ot[e]));
+                        orn[e] = __float_as_uint(has_run ? fmaf(__uint_as_float(orn[e]), f_run,
+                                                                __uint_as_float(ot[e]))
+                                                         : __uint_as_float(ot[e]));
                     tmem_st32(lane_base + kColRun + 32 * c, orn);
                 }
                 tmem_wait_st();
             }
-            f_prev = alpha * drop;                       // applies to the running sum at the next fold
+            if (fold_now) {
+                has_run = true;
+                f_run = alpha * drop;                    // the running sum's scale -> this tile's
+                n_acc = 0;
+            }
+            ++n_acc;
+            if (tid == 0) pv_acc[s] = (j >= 1 && !fold_now) ? 1 : 0;   // read after pfull
             // ---- pass 2: P'' = 2^(x zs - m) * v_scale * 2^kv as f16 hi + lo for
             // this half's tokens (P atom hf); x = -inf (masked) gives 0
             float lsum = 0.f;
@@ -607,7 +637,7 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 ptx::mbar_arrive(bar_empty + 8 * s);    // V and scales consumed
             }
         }
-        // ---- the row: (run * f + last tile) * 2^-kv / l, l over both halves
+        // ---- the row: (run * f_run + O tile) * 2^-kv / l, l over both halves
         lx[128 * hf + i_row] = l_run;
         row_sync();
         const float l_tot = lx[i_row] + lx[128 + i_row];
@@ -619,13 +649,13 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 const int c = 2 * hf + cl;
                 uint32_t ot[32], orn[32];
                 tmem_ld32(lane_base + kColO + 32 * c, ot);
-                if (ntile >= 2) tmem_ld32(lane_base + kColRun + 32 * c, orn);
+                if (has_run) tmem_ld32(lane_base + kColRun + 32 * c, orn);
                 tmem_wait_ld();
                 float o_[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
-                    o_[e] = (ntile >= 2 ? fmaf(__uint_as_float(orn[e]), f_prev, __uint_as_float(ot[e]))
-                                        : __uint_as_float(ot[e])) * f;
+                    o_[e] = (has_run ? fmaf(__uint_as_float(orn[e]), f_run, __uint_as_float(ot[e]))
+                                     : __uint_as_float(ot[e])) * f;
                 if (valid) {
                     float4* dst = reinterpret_cast<float4*>(p.out + orow * kDim + 32 * c);
 #pragma unroll
