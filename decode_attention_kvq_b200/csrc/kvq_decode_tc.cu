@@ -32,11 +32,12 @@
 //    two stages, its query rows by 1-D bulk copies; all complete on the
 //    stage's mbarrier.  It refills a slot as soon as its consumers released
 //    it.  The consumers form two groups of four warps that take alternate
-//    stages; a warp takes 32 tokens of its group's stage as two 16-token MMA
-//    tiles.
+//    stages (with 9 to 16 heads: every stage, group g taking heads 8g ..
+//    8g + 7); a warp takes 32 tokens of its group's stage as two 16-token
+//    MMA tiles.
 //  * S^T = K . Q^T on the integer MMA (mma.sync m16n8k32, s32 accumulate),
-//    with the query heads of the GQA group as the N = 8 dimension (two
-//    n-tiles when G > 8): the K bytes are the A operand as loaded, and Q is
+//    with 8 query heads of the GQA group as the N = 8 dimension: the K
+//    bytes are the A operand as loaded, and Q is
 //    a per-head power-of-two prescaled 16-bit integer in two byte digits, so
 //    S = 256 S_hi + S_lo - 128 sum(Qi) is exact.  The K scale (per token, or
 //    per 32-value group with one fold per group), the prescale, attn_scale
@@ -143,7 +144,7 @@ struct Layout {
     static constexpr int Q_BYTES = (G16 ? 16 : 8) * D * 2;           // bf16 query rows
     static constexpr int MASK_OFF = Q_OFF + Q_BYTES;                 // paged: valid-page bits
     static constexpr int STAGE = ((MASK_OFF + 16) + 1023) / 1024 * 1024;
-    static constexpr int NV = (G16 ? 2 : 1) * (D / 16) * 4;        // o floats per lane
+    static constexpr int NV = (D / 16) * 4;                         // o floats per lane
     static constexpr int MERGE_BYTES = NW * NV * 32 * 4;
     static constexpr int LENS_BYTES = (3 * kMaxB + 1) * 4;          // lengths, chunks, prefix sums
     static constexpr int PARAM_BYTES = 256;                         // the kernel parameters
@@ -263,14 +264,16 @@ __device__ __forceinline__ Seg seg_at(int i, int iend, const int* lens, const in
 // Fused append: the warp whose 32-token slice of a landed stage holds the
 // new token (position tok of unit (b, hk), stage row r) quantises it -- the
 // append kernels' quantiser -- into the stage's K and V rows and scales (sk,
-// sv, sks, svs: shared-memory addresses) and into the cache, before any of
-// its MMA operands are read.  Lane l takes head_dim values [l * VPL,
+// sv, sks, svs: shared-memory addresses) and, if to_cache, into the cache,
+// before any of its MMA operands are read.  (G16: the slice's warp of each
+// group does this; both write the same bits into the stage, and only group
+// 0's writes the cache.)  Lane l takes head_dim values [l * VPL,
 // (l + 1) * VPL) of k_new and v_new.  Only the fused instantiation of the
 // split kernel (VAR == 2) contains it.
 template <int D, bool G32, bool PAGED>
 __device__ __forceinline__ void patch_new_token(const DecodeParams& p, uint32_t sk, uint32_t sv,
                                              uint32_t sks, uint32_t svs, int r, int tok, int b,
-                                             int hk) {
+                                             int hk, bool to_cache) {
     constexpr int VPL = D / 32;          // values per lane
     constexpr int NG = G32 ? D / 32 : 1;
     const int lane = threadIdx.x & 31;
@@ -325,19 +328,25 @@ __device__ __forceinline__ void patch_new_token(const DecodeParams& p, uint32_t 
     if constexpr (VPL == 4) {
         sts_u32(sk + off, bk);
         sts_u32(sv + off, bv);
-        *reinterpret_cast<uint32_t*>(p.k_w + crow * D + lane * VPL) = bk;
-        *reinterpret_cast<uint32_t*>(p.v_w + crow * D + lane * VPL) = bv;
+        if (to_cache) {
+            *reinterpret_cast<uint32_t*>(p.k_w + crow * D + lane * VPL) = bk;
+            *reinterpret_cast<uint32_t*>(p.v_w + crow * D + lane * VPL) = bv;
+        }
     } else {
         asm volatile("st.shared.u16 [%0], %1;" ::"r"(sk + off), "h"(static_cast<uint16_t>(bk)) : "memory");
         asm volatile("st.shared.u16 [%0], %1;" ::"r"(sv + off), "h"(static_cast<uint16_t>(bv)) : "memory");
-        *reinterpret_cast<uint16_t*>(p.k_w + crow * D + lane * VPL) = static_cast<uint16_t>(bk);
-        *reinterpret_cast<uint16_t*>(p.v_w + crow * D + lane * VPL) = static_cast<uint16_t>(bv);
+        if (to_cache) {
+            *reinterpret_cast<uint16_t*>(p.k_w + crow * D + lane * VPL) = static_cast<uint16_t>(bk);
+            *reinterpret_cast<uint16_t*>(p.v_w + crow * D + lane * VPL) = static_cast<uint16_t>(bv);
+        }
     }
     if (lead) {
         sts_f32(sks + (r * NG + gidx) * 4, sck);
         sts_f32(svs + (r * NG + gidx) * 4, scv);
-        p.ks_w[crow * NG + gidx] = sck;
-        p.vs_w[crow * NG + gidx] = scv;
+        if (to_cache) {
+            p.ks_w[crow * NG + gidx] = sck;
+            p.vs_w[crow * NG + gidx] = scv;
+        }
     }
     // the slot is refilled by TMA (async proxy) after these generic writes
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -359,7 +368,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     constexpr int NV = Lay::NV;
     constexpr int NGRP = D / 32;        // 32-value groups over head_dim
     constexpr int MT = D / 16;          // m-tiles of O^T over head_dim (PV)
-    constexpr int NT = G16 ? 2 : 1;     // n-tiles of 8 query heads
+    // n-tiles of 8 query heads per warp.  G16 (9 to 16 heads): the two groups
+    // split the heads (group grp takes heads 8 grp .. 8 grp + 7) and both work
+    // every stage, so a warp still holds one n-tile of state
+    constexpr int NT = 1;
     constexpr int NGV = G32 ? NG : 1;   // V scales per token
     static_assert(!PK || (G32 && !G16), "packing: group-32 scales, at most 4 heads");
     static_assert(!(PK && CAUSAL), "chunk queries: unpacked columns");
@@ -395,7 +407,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     volatile int* abort_flag = reinterpret_cast<volatile int*>(mrg_l + 16 * NW + 4);
     static_assert(2 * NST * 8 + 2 * 16 * NW * 4 + 16 + 4 <= Lay::MISC_BYTES,
                   "barriers, maxima, flag");
-    float* mslot = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);   // [NW][8 NT heads][D]
+    float* mslot = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);   // [NW][8 heads][D]
     int* lens = reinterpret_cast<int*>(smem + Lay::LENS_OFF);                     // [B]
     int* nsv = lens + kMaxB;                                                     // [B] chunks
     int* cum = nsv + kMaxB;                                                      // [B + 1]
@@ -416,7 +428,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // the producer's expect_tx arrival (paged: one per producer warp, plus
             // one cp.async arrival per lane of producer warp 0 for the scales)
             ptx::mbar_init(bar_full + 8 * s, PAGED ? 2 + 32 : 1);
-            ptx::mbar_init(bar_empty + 8 * s, WPG);
+            ptx::mbar_init(bar_empty + 8 * s, G16 ? 2 * WPG : WPG);
         }
         ptx::mbar_init(bar_mfree, NW);
         ptx::mbar_init(bar_q, 1);
@@ -784,6 +796,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int ctid = tid - 32 * nprod(PAGED);      // consumer thread index
     if (one) grid_dep_wait();           // before the length read and any global write
     const int grp = cw / WPG, wg = cw % WPG;
+    const int hofs = G16 ? 8 * grp : 0;          // the warp's first query head (column)
     const int sig_g = sigma(g);
     const int sig_a = sigma(2 * t), sig_b = sigma(2 * t + 1);
 
@@ -814,7 +827,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         int csq[NT][NCG];              // sum of the head's Qi (per 32-value group)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const int h = PK ? (g & 3) : 8 * nt + g;
+            const int h = PK ? (g & 3) : hofs + 8 * nt + g;
             float qf[NGRP][8];
             float amax = 0.f;
 #pragma unroll
@@ -934,7 +947,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    lim_col[nt][c] = Lseq - p.qlen + (8 * nt + 2 * t + c) % p.qlen;
+                    lim_col[nt][c] = Lseq - p.qlen + (hofs + 8 * nt + 2 * t + c) % p.qlen;
                     lo_col[nt][c] = p.window > 0 ? lim_col[nt][c] - p.window + 1 : INT_MIN;
                 }
         }
@@ -981,14 +994,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const int tok = (one ? Lone : lens[b]) - 1;
                 if (tok >= t0 && tok < t1) {
                     const int itn = (tok - t0) / TT;
-                    if (((c_count + itn) & 1) == grp && ((tok - t0 - itn * TT) >> 5) == wg)
+                    if ((G16 || ((c_count + itn) & 1) == grp) && ((tok - t0 - itn * TT) >> 5) == wg)
                         fa_tok = tok;
                 }
             }
         }
 #pragma unroll 1
         for (int it = 0; it < ntiles; ++it, ++c_count) {
-            if ((c_count & 1) != grp) continue;           // the other group's stage
+            if (!G16 && (c_count & 1) != grp) continue;   // the other group's stage
             const int s = c_count % NST;
             wait(bar_full + 8 * s, (c_count / NST) & 1);
             const int tt0 = t0 + it * TT;
@@ -1012,7 +1025,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     if (fa_tok >= tt0 && fa_tok < tt0 + TT &&
                         (!PAGED || ((pmask >> ((fa_tok - tt0) >> 4)) & 1u)))
                         patch_new_token<D, G32, PAGED>(p, sk, sv, sks, svs, fa_tok - tt0, fa_tok,
-                                                       b, hk);
+                                                       b, hk, !G16 || grp == 0);
                 }
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
@@ -1342,7 +1355,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 8);
                 l[nt][c] += __shfl_xor_sync(0xffffffffu, l[nt][c], 16);
                 if (g == 0) {
-                    const int hm = PK ? 2 * (t & 1) + c : 8 * nt + 2 * t + c;
+                    const int hm = PK ? 2 * (t & 1) + c : hofs + 8 * nt + 2 * t + c;
                     mrg_m[hm * NW + cw] = m[nt][c];
                     mrg_l[hm * NW + cw] = l[nt][c];
                 }
@@ -1373,39 +1386,46 @@ decode_split_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         ptx::named_bar_sync(1, NCONS);
         // one thread per (head, 16-byte chunk of its row): the head's segment
-        // max M and sum Ls over the eight warps, the weights 2^(m_w - M) (over
-        // Ls when the rows are final), and the weighted sum of the eight slots
+        // max M and sum Ls over the warps that hold the head (all eight; G16:
+        // the four of its group), the weights 2^(m_w - M) (over Ls when the
+        // rows are final), and the weighted sum of their slots
         constexpr int NCH = D / 4;
-        constexpr int NITEM = 8 * NT * NCH;
-        static_assert(NW == 8, "two 16-byte loads of per-warp maxima and sums");
+        constexpr int NWH = G16 ? WPG : NW;           // warps holding one head
+        constexpr int NITEM = (G16 ? 16 : 8) * NCH;
+        static_assert(NW == 8 && NWH % 4 == 0, "16-byte loads of per-warp maxima and sums");
 #pragma unroll
         for (int it = 0; it < (NITEM + NCONS - 1) / NCONS; ++it) {
             const int idx = ctid + it * NCONS;
             const int h = idx / NCH, k = idx % NCH;
             if (idx >= NITEM || h >= G) continue;
-            float mw[NW], fw[NW], lw[NW];
-            *reinterpret_cast<float4*>(mw) = *reinterpret_cast<const float4*>(mrg_m + h * NW);
-            *reinterpret_cast<float4*>(mw + 4) = *reinterpret_cast<const float4*>(mrg_m + h * NW + 4);
-            *reinterpret_cast<float4*>(lw) = *reinterpret_cast<const float4*>(mrg_l + h * NW);
-            *reinterpret_cast<float4*>(lw + 4) = *reinterpret_cast<const float4*>(mrg_l + h * NW + 4);
+            const int wb = G16 ? WPG * (h >> 3) : 0;   // the head's first warp
+            const int hl = G16 ? (h & 7) : h;           // its row in a warp's slot
+            float mw[NWH], fw[NWH], lw[NWH];
+#pragma unroll
+            for (int x = 0; x < NWH / 4; ++x) {
+                *reinterpret_cast<float4*>(mw + 4 * x) =
+                    *reinterpret_cast<const float4*>(mrg_m + h * NW + wb + 4 * x);
+                *reinterpret_cast<float4*>(lw + 4 * x) =
+                    *reinterpret_cast<const float4*>(mrg_l + h * NW + wb + 4 * x);
+            }
             float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < NW; ++w) M = fmaxf(M, mw[w]);
+            for (int w = 0; w < NWH; ++w) M = fmaxf(M, mw[w]);
             float Ls = 0.f;
 #pragma unroll
-            for (int w = 0; w < NW; ++w) {
+            for (int w = 0; w < NWH; ++w) {
                 fw[w] = mw[w] == -INFINITY ? 0.f : ptx::ex2(mw[w] - M);
                 Ls += lw[w] * fw[w];
             }
             if (final_rows) {
                 const float r = Ls > 0.f ? __frcp_rn(Ls) : 0.f;
 #pragma unroll
-                for (int w = 0; w < NW; ++w) fw[w] *= r;
+                for (int w = 0; w < NWH; ++w) fw[w] *= r;
             }
             float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-            const float* src = mslot + h * D + 4 * (k ^ mswz<D, G32>(h));
+            const float* src = mslot + hl * D + 4 * (k ^ mswz<D, G32>(hl)) + wb * NV * 32;
 #pragma unroll
-            for (int w = 0; w < NW; ++w) {
+            for (int w = 0; w < NWH; ++w) {
                 const float4 v = *reinterpret_cast<const float4*>(src + w * NV * 32);
                 s0 = fmaf(fw[w], v.x, s0);
                 s1 = fmaf(fw[w], v.y, s1);
