@@ -22,19 +22,24 @@
 //    S = 256 S_hi + S_lo - 128 sum(Qi) is exact in int32 -- into two 128-
 //    column TMEM accumulators; then P V on kind::f16 into a third (fp32, a
 //    fresh one per tile), with P'' = 2^(z - m) * v_scale * 2^kv split into f16
-//    hi + lo parts and V as the exact f16 integers byte - 128.
+//    hi + lo parts and V as the exact f16 integers byte - 128.  The next
+//    tile's Q K^T is issued as soon as the rows hold this tile's scores in
+//    registers, ahead of this tile's P V.
 //  * Warps 0-7 own the rows, two warps per row: warp w reads TMEM lanes
 //    32 (w % 4) .. + 31 (row i = TMEM lane i) and takes half h = w / 4 of the
 //    row's 128 columns -- tokens 64 h .. 64 h + 63 of a tile and head_dim
 //    64 h .. 64 h + 63 of the output -- so two row warps share each
-//    scheduler.  They read the scores with tcgen05.ld, apply the K scale, the
-//    row's prescale, attn_scale and log2(e), mask causally, exchange the
-//    halves' maxima through shared memory, keep the online softmax per row,
-//    fold each tile's P V into a running sum in TMEM (fp32, with the row's
-//    rescale), write P'' and the f16 V tile into shared memory in the
-//    canonical swizzled layouts, and finally read the sum back and write the
-//    row.  Per tile, the K scales and the V scales times the P'' prescale are
-//    first copied into aligned shared-memory vectors.
+//    scheduler.  They read the scores with tcgen05.ld into registers, apply
+//    the K scale, the row's prescale, attn_scale and log2(e), mask causally,
+//    exchange the halves' maxima through shared memory, keep the online
+//    softmax per row, fold the P V of tiles into a running sum in TMEM (fp32,
+//    with the row's rescale), write P'' into shared memory in the canonical
+//    swizzled layout, and finally read the sum back and write the row.
+//  * Warps 10 and 11 help ahead of the rows: per tile, warp 10 copies the K
+//    scales and the V scales times the P'' prescale into aligned shared-
+//    memory vectors (with the prescale's drop), and both write the tile's V
+//    as exact f16 into the MN-major B tile once the previous P V has read
+//    it.
 //  * Every mbarrier wait is bounded; a timeout sets KVQ_DEVERR_TIMEOUT, every
 //    role then skips its remaining work (the row warps still pass every
 //    named barrier of every tile, so none waits for another that left), and
@@ -54,9 +59,9 @@ namespace {
 constexpr int kRows = 128;                 // (query, head) rows per CTA: the MMA M
 constexpr int kTok = 128;                  // KV tokens per tile
 constexpr int kDim = 128;                  // head_dim handled here
-constexpr int kThreads = 320;              // warps 0-7 rows, 8 producer, 9 MMA
+constexpr int kThreads = 384;              // warps 0-7 rows, 8 producer, 9 MMA, 10-11 helpers
 constexpr int kRowThreads = 256;
-constexpr int kProdWarp = 8, kMmaWarp = 9;
+constexpr int kProdWarp = 8, kMmaWarp = 9, kAuxWarp = 10;   // helpers: warps 10 and 11
 constexpr int kTmemCols = 512;             // S_hi 128 | S_lo 128 | O tile 128 | O run 128
 // The tensor cores add each P.V k-step into O; over a long key range that is
 // tens of thousands of accumulations into one fp32 accumulator, and the error
@@ -151,6 +156,26 @@ __device__ __forceinline__ void tmem_st32(uint32_t addr, const uint32_t (&r)[32]
           "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
+// 16 consecutive 32-bit columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(addr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};"
+        ::"r"(addr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+          "r"(r[14]), "r"(r[15])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -193,13 +218,17 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const uint32_t bar_pfull = bar_full + 48;
     const uint32_t bar_odone = bar_full + 56;
     const uint32_t bar_qready = bar_full + 64;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMisc + 96);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMisc + 100);
-    float* red = reinterpret_cast<float*>(smem + kMisc + 128);   // [8] per-warp V-scale maxima
+    const uint32_t bar_aready = bar_full + 72;       // [2] by tile parity: the tile's vectors
+    const uint32_t bar_afree = bar_full + 88;        // [2] by tile parity: rows done with them
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMisc + 104);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMisc + 108);
     // [8] per-warp "a row's maximum grew this tile"; [2] by tile parity: P.V of
-    // the tile adds onto the O tile (1) or starts it afresh (0)
+    // the tile adds onto the O tile (1) or starts it afresh (0); [2] by tile
+    // parity: the prescale's drop factor and exponent after the tile
     volatile int* grew = reinterpret_cast<volatile int*>(smem + kMisc + 160);
     volatile int* pv_acc = reinterpret_cast<volatile int*>(smem + kMisc + 192);
+    volatile float* tdrop = reinterpret_cast<volatile float*>(smem + kMisc + 208);
+    volatile int* tkv = reinterpret_cast<volatile int*>(smem + kMisc + 216);
     float* kal = reinterpret_cast<float*>(smem + kAux);          // [2][128] K scales
     float* vsu = kal + 256;                                      // [2][128] V scales * 2^kv
     float* xch = vsu + 256;                                      // [2][128] halves' maxima
@@ -224,11 +253,14 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(bar_full + 8 * s, 1);
-            ptx::mbar_init(bar_empty + 8 * s, 1 + 8);   // K: the MMA commit; V: eight row warps
+            // K: the MMA commit; V and the scales: the two helper warps
+            ptx::mbar_init(bar_empty + 8 * s, 1 + 2);
+            ptx::mbar_init(bar_aready + 8 * s, 1);
+            ptx::mbar_init(bar_afree + 8 * s, 8);
         }
         ptx::mbar_init(bar_sfull, 1);
         ptx::mbar_init(bar_sfree, 8);
-        ptx::mbar_init(bar_pfull, 8);
+        ptx::mbar_init(bar_pfull, 8 + 2);           // P'' by the rows, V16 by the helpers
         ptx::mbar_init(bar_odone, 1);
         ptx::mbar_init(bar_qready, 8);
         *abort_flag = 0;
@@ -299,40 +331,144 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
+        // Order on the tensor pipe: S(0), then per tile j: S(j + 1) as soon as
+        // the rows hold tile j's scores in registers (sfree, after their first
+        // pass) and its K has landed, and P.V(j) once P'' and V16 are written
+        // (pfull).  So the next tile's scores are computed while the rows
+        // finish tile j, and P.V(j) runs during their first pass over j + 1.
         if (lane == 0 && ntile > 0 && wait(bar_qready, 0)) {
             const uint64_t dq_hi = smem_desc(sb + kQhi, 16, 1024);
             const uint64_t dq_lo = smem_desc(sb + kQlo, 16, 1024);
-            for (int j = 0; j < ntile; ++j) {
+            // S = Q K^T of tile j: four k-steps of 32 bytes per digit
+            // (descriptor start addresses advance in 16-byte units)
+            auto issue_s = [&](int j) {
                 const int s = j & 1;
-                if (!wait(bar_full + 8 * s, (j >> 1) & 1)) break;
-                if (j >= 1 && !wait(bar_sfree, (j - 1) & 1)) break;
+                if (!wait(bar_full + 8 * s, (j >> 1) & 1)) return false;
                 tc_fence_after();
                 const uint64_t dk = smem_desc(sb + kStage0 + s * kStageBytes + kStK, 16, 1024);
-                // S = Q K^T: four k-steps of 32 bytes per digit (descriptor
-                // start addresses advance in 16-byte units)
                 for (int k = 0; k < 4; ++k)
                     tc_mma<true>(tmem + kColShi, dq_hi + 2 * k, dk + 2 * k, kIdescQkHi, k > 0);
                 for (int k = 0; k < 4; ++k)
                     tc_mma<true>(tmem + kColSlo, dq_lo + 2 * k, dk + 2 * k, kIdescQkLo, k > 0);
                 tc_commit(bar_sfull);
                 tc_commit(bar_empty + 8 * s);       // K consumed
-                if (!wait(bar_pfull, j & 1)) break;
-                tc_fence_after();
-                // O (+)= P'' V: eight k-steps of 16 tokens per part; P rows are
-                // two 64-token atoms, V16 k-steps advance 16 rows of 128 bytes.
-                // The tile's first k-step starts the O tile afresh unless the
-                // rows left it unfolded (then the tile adds onto it)
-                const bool onto = j > 0 && pv_acc[j & 1] != 0;
-                for (int part = 0; part < 2; ++part) {
-                    const uint32_t pb = sb + (part ? kPlo : kPhi);
-                    for (int k = 0; k < 8; ++k) {
-                        const uint64_t da = smem_desc(pb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                        const uint64_t dv = smem_desc(sb + kV16 + k * 2048, 16384, 1024);
-                        tc_mma<false>(tmem + kColO, da, dv, kIdescPv, (onto || part > 0 || k > 0));
+                return true;
+            };
+            if (issue_s(0)) {
+                for (int j = 0; j < ntile; ++j) {
+                    if (j + 1 < ntile) {
+                        // the rows have read S_hi and S_lo of tile j
+                        if (!wait(bar_sfree, j & 1)) break;
+                        tc_fence_after();
+                        if (!issue_s(j + 1)) break;
                     }
+                    if (!wait(bar_pfull, j & 1)) break;
+                    tc_fence_after();
+                    // O (+)= P'' V: eight k-steps of 16 tokens per part; P rows are
+                    // two 64-token atoms, V16 k-steps advance 16 rows of 128 bytes.
+                    // The tile's first k-step starts the O tile afresh unless the
+                    // rows left it unfolded (then the tile adds onto it)
+                    const bool onto = j > 0 && pv_acc[j & 1] != 0;
+                    for (int part = 0; part < 2; ++part) {
+                        const uint32_t pb = sb + (part ? kPlo : kPhi);
+                        for (int k = 0; k < 8; ++k) {
+                            const uint64_t da = smem_desc(pb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                            const uint64_t dv = smem_desc(sb + kV16 + k * 2048, 16384, 1024);
+                            tc_mma<false>(tmem + kColO, da, dv, kIdescPv, (onto || part > 0 || k > 0));
+                        }
+                    }
+                    tc_commit(bar_odone);
                 }
-                tc_commit(bar_odone);
             }
+        }
+    } else if (warp >= kAuxWarp) {
+        // ------------------------------------------------------------ helpers
+        // Per tile j, ahead of the rows: warp 10 copies the K scales and the
+        // V scales times the P'' prescale 2^kv into the aligned vectors of the
+        // tile's parity (tokens 4 lane .. 4 lane + 3; 0 past the keys), with the
+        // largest V scale over the tile: 2^kv only drops, and a drop rescales
+        // O.  Then both warps write the tile's V rows as exact f16 (byte - 128)
+        // into the MN-major B tile (warp 10 + a: rows 64 a .. 64 a + 63), once
+        // the previous P.V has read it.
+        const int a = warp - kAuxWarp;
+        int kv = 64;
+        auto vectors = [&](int j) {
+            const int s = j & 1;
+            if (!wait(bar_full + 8 * s, (j >> 1) & 1)) return false;
+            if (j >= 2 && !wait(bar_afree + 8 * s, ((j >> 1) - 1) & 1)) return false;
+            const float* ksc = reinterpret_cast<const float*>(smem + kStage0 + s * kStageBytes + kStKs) + sc_off;
+            const float* vsc = reinterpret_cast<const float*>(smem + kStage0 + s * kStageBytes + kStVs) + sc_off;
+            float ks[4], vs[4];
+            float vm = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int tok = 4 * lane + e;
+                const bool real = j * kTok + tok < t_hi;
+                ks[e] = real ? ksc[tok] : 0.f;
+                vs[e] = real ? vsc[tok] : 0.f;
+                vm = fmaxf(vm, vs[e]);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+            float drop = 1.f;
+            if (vm > 0.f) {
+                const int ev = static_cast<int>((__float_as_uint(vm) >> 23) & 0xffu) - 127;
+                const int kn = max(min(kv, 14 - ev), -120);
+                if (kn < kv) {
+                    drop = pow2i_f(kn - kv);
+                    kv = kn;
+                }
+            }
+            const float up = pow2i_f(kv);
+            *reinterpret_cast<float4*>(kal + 128 * s + 4 * lane) = make_float4(ks[0], ks[1], ks[2], ks[3]);
+            *reinterpret_cast<float4*>(vsu + 128 * s + 4 * lane) =
+                make_float4(vs[0] * up, vs[1] * up, vs[2] * up, vs[3] * up);
+            if (lane == 0) {
+                tdrop[s] = drop;
+                tkv[s] = kv;
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_aready + 8 * s);
+            return true;
+        };
+        auto v16 = [&](int j) {
+            const int s = j & 1;
+            if (a == 1 && !wait(bar_full + 8 * s, (j >> 1) & 1)) return false;
+            if (j >= 1 && !wait(bar_odone, (j - 1) & 1)) return false;   // P.V(j - 1) read V16
+#pragma unroll 1
+            for (int r2 = 0; r2 < 2; ++r2) {
+                const int row = 64 * a + 32 * r2 + lane;             // token of the tile
+                const uint8_t* vrow = smem + kStage0 + s * kStageBytes + kStV + row * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {            // 16 head_dim values per source chunk
+                    const uint4 raw = *reinterpret_cast<const uint4*>(vrow + ((c ^ (row & 7)) << 4));
+                    const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+                    uint32_t f[8];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        f[2 * w] = ptx::bytes_to_f16x2(w4[w], 0x4140u);
+                        f[2 * w + 1] = ptx::bytes_to_f16x2(w4[w], 0x4342u);
+                    }
+                    const int k0 = 2 * (c & 3);          // chunks (d % 64) / 8 and + 1 of atom c / 4
+                    const uint32_t base = kV16 + (c >> 2) * 16384 + row * 128;
+                    *reinterpret_cast<uint4*>(smem + base + ((k0 ^ (row & 7)) << 4)) =
+                        make_uint4(f[0], f[1], f[2], f[3]);
+                    *reinterpret_cast<uint4*>(smem + base + (((k0 + 1) ^ (row & 7)) << 4)) =
+                        make_uint4(f[4], f[5], f[6], f[7]);
+                }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(bar_pfull);
+                ptx::mbar_arrive(bar_empty + 8 * s);    // V and scales consumed
+            }
+            return true;
+        };
+        bool ok = ntile > 0 && (a != 0 || vectors(0));
+        for (int j = 0; ok && j < ntile; ++j) {
+            if (a == 0 && j + 1 < ntile && !vectors(j + 1)) break;
+            ok = v16(j);
         }
     } else {
         // ------------------------------------------------------------ rows
@@ -427,57 +563,30 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         for (int j = 0; j < ntile; ++j) {
             const int s = j & 1;
             const int t0 = j * kTok;
-            const float* ksc = reinterpret_cast<const float*>(smem + kStage0 + s * kStageBytes + kStKs) + sc_off;
-            const float* vsc = reinterpret_cast<const float*>(smem + kStage0 + s * kStageBytes + kStVs) + sc_off;
-            float* kal_j = kal + 128 * s;
-            float* vsu_j = vsu + 128 * s;
-            live = live && wait(bar_full + 8 * s, (j >> 1) & 1);
-            // ---- the tile's scales: token i_row's K scale and V scale (0 past
-            // the keys), the largest V scale over the tile (the same for every
-            // row): the P'' prescale 2^kv only drops, and a drop rescales O
-            const bool real = t0 + i_row < t_hi;
-            const float ks_i = (live && real) ? ksc[i_row] : 0.f;
-            const float vs_i = (live && real) ? vsc[i_row] : 0.f;
-            {
-                float vm = vs_i;
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
-                if (lane == 0) red[warp] = vm;
-                if (hf == 0) kal_j[i_row] = ks_i;
-            }
-            row_sync();
-            float drop = 1.f;
-            {
-                float vm = red[0];
-#pragma unroll
-                for (int w = 1; w < 8; ++w) vm = fmaxf(vm, red[w]);
-                if (vm > 0.f) {
-                    const int ev = static_cast<int>((__float_as_uint(vm) >> 23) & 0xffu) - 127;
-                    const int kn = max(min(kv, 14 - ev), -120);
-                    if (kn < kv) {
-                        drop = pow2i_f(kn - kv);
-                        kv = kn;
-                    }
-                }
-                if (hf == 0) vsu_j[i_row] = vs_i * pow2i_f(kv);
-            }
-            row_sync();                                  // red read; kal, vsu written
+            const float* kal_j = kal + 128 * s;
+            const float* vsu_j = vsu + 128 * s;
+            // the tile's K scales, V scales * 2^kv and prescale drop (helpers)
+            live = live && wait(bar_aready + 8 * s, (j >> 1) & 1);
+            const float drop = live ? tdrop[s] : 1.f;
+            if (live) kv = tkv[s];
             live = live && wait(bar_sfull, j & 1);
             tc_fence_after();
             // ---- pass 1: x = S * k_scale over this half's tokens (-inf where the
-            // causal mask drops the key), its maximum, and x written back over
-            // the S_hi columns so that pass 2 reads one tile and no mask
+            // causal mask drops the key) and its maximum; x stays in registers
+            // (xr), so pass 2 needs no mask, no integer reconstruction and no
+            // tensor memory, and S is free for the next tile's Q K^T at once
             // (a warp whose rows all see the whole half skips the mask test)
             const int tb = t0 + 64 * hf;                 // this half's first token
             const bool unmasked = valid && tb + 63 <= pos;
             const bool warp_unmasked = __all_sync(0xffffffffu, unmasked);
             float xmax = -INFINITY;
+            uint32_t xr[2][32];
             if (live) {
-#pragma unroll 1
+#pragma unroll
                 for (int cl = 0; cl < 2; ++cl) {
                     const int c = 2 * hf + cl;
-                    uint32_t sh_[32], sl_[32];
-                    tmem_ld32(lane_base + kColShi + 32 * c, sh_);
+                    uint32_t sl_[32];
+                    tmem_ld32(lane_base + kColShi + 32 * c, xr[cl]);
                     tmem_ld32(lane_base + kColSlo + 32 * c, sl_);
                     tmem_wait_ld();
                     if (warp_unmasked) {
@@ -488,10 +597,10 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
                                 const int e = 4 * e4 + u;
-                                const int S = static_cast<int>(sh_[e]) * 256 + static_cast<int>(sl_[e]) - cq;
+                                const int S = static_cast<int>(xr[cl][e]) * 256 + static_cast<int>(sl_[e]) - cq;
                                 const float x = static_cast<float>(S) * kk[u];
                                 xmax = fmaxf(xmax, x);
-                                sh_[e] = __float_as_uint(x);
+                                xr[cl][e] = __float_as_uint(x);
                             }
                         }
                     } else {
@@ -502,18 +611,20 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
                                 const int e = 4 * e4 + u;
-                                const int S = static_cast<int>(sh_[e]) * 256 + static_cast<int>(sl_[e]) - cq;
+                                const int S = static_cast<int>(xr[cl][e]) * 256 + static_cast<int>(sl_[e]) - cq;
                                 const bool on = valid && t0 + 32 * c + e <= pos;
                                 const float x = on ? static_cast<float>(S) * kk[u] : -INFINITY;
                                 xmax = fmaxf(xmax, x);
-                                sh_[e] = __float_as_uint(x);
+                                xr[cl][e] = __float_as_uint(x);
                             }
                         }
                     }
-                    tmem_st32(lane_base + kColShi + 32 * c, sh_);
                 }
-                tmem_wait_st();
             }
+            // S_hi / S_lo read into registers: the next Q K^T may start
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_sfree);
             xch[128 * hf + i_row] = xmax;
             {
                 const bool g = __any_sync(0xffffffffu, xmax * zs > m_run);
@@ -533,21 +644,21 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             // the previous P.V is done: P, V16 free, O stable
             if (j >= 1) live = live && wait(bar_odone, (j - 1) & 1);
             tc_fence_after();
-            // the fold (this half's head_dim columns)
+            // the fold (this half's head_dim columns, in 16-column pieces)
             if (live && fold_now) {
 #pragma unroll 1
-                for (int cl = 0; cl < 2; ++cl) {
-                    const int c = 2 * hf + cl;
-                    uint32_t ot[32], orn[32];
-                    tmem_ld32(lane_base + kColO + 32 * c, ot);
-                    if (has_run) tmem_ld32(lane_base + kColRun + 32 * c, orn);
+                for (int cl = 0; cl < 4; ++cl) {
+                    const int c = 4 * hf + cl;           // 16-column pieces
+                    uint32_t ot[16], orn[16];
+                    tmem_ld16(lane_base + kColO + 16 * c, ot);
+                    if (has_run) tmem_ld16(lane_base + kColRun + 16 * c, orn);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
+                    for (int e = 0; e < 16; ++e)
                         orn[e] = __float_as_uint(has_run ? fmaf(__uint_as_float(orn[e]), f_run,
                                                                 __uint_as_float(ot[e]))
                                                          : __uint_as_float(ot[e]));
-                    tmem_st32(lane_base + kColRun + 32 * c, orn);
+                    tmem_st16(lane_base + kColRun + 16 * c, orn);
                 }
                 tmem_wait_st();
             }
@@ -562,12 +673,10 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             // this half's tokens (P atom hf); x = -inf (masked) gives 0
             float lsum = 0.f;
             if (live) {
-#pragma unroll 1
+#pragma unroll
                 for (int cl = 0; cl < 2; ++cl) {
                     const int c = 2 * hf + cl;
-                    uint32_t xs[32];
-                    tmem_ld32(lane_base + kColShi + 32 * c, xs);
-                    tmem_wait_ld();
+                    const uint32_t (&xs)[32] = xr[cl];
                     uint32_t ph[16], pl[16];
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
@@ -601,40 +710,14 @@ chunk_attn_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar_sfree);     // S read: the next Q K^T may start
             l_run = l_run * alpha + lsum;
             m_run = m_new;
-            // ---- V tile row i_row (this half's head_dim) as exact f16
-            // (byte - 128) into the MN-major B tile (atom hf)
-            if (live) {
-                const uint8_t* vrow = smem + kStage0 + s * kStageBytes + kStV + i_row * 128;
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {         // 16 head_dim values per source chunk
-                    const int c = 4 * hf + cc;
-                    const uint4 raw = *reinterpret_cast<const uint4*>(vrow + ((c ^ (i_row & 7)) << 4));
-                    const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-                    uint32_t f[8];
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        f[2 * w] = ptx::bytes_to_f16x2(w4[w], 0x4140u);
-                        f[2 * w + 1] = ptx::bytes_to_f16x2(w4[w], 0x4342u);
-                    }
-                    const int k0 = 2 * cc;               // chunks (d % 64) / 8 and + 1
-                    const uint32_t base = kV16 + hf * 16384 + i_row * 128;
-                    *reinterpret_cast<uint4*>(smem + base + ((k0 ^ (i_row & 7)) << 4)) =
-                        make_uint4(f[0], f[1], f[2], f[3]);
-                    *reinterpret_cast<uint4*>(smem + base + (((k0 + 1) ^ (i_row & 7)) << 4)) =
-                        make_uint4(f[4], f[5], f[6], f[7]);
-                }
-            }
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
+                ptx::mbar_arrive(bar_afree + 8 * s);    // this parity's vectors read
                 ptx::mbar_arrive(bar_pfull);
-                ptx::mbar_arrive(bar_empty + 8 * s);    // V and scales consumed
             }
         }
         // ---- the row: (run * f_run + O tile) * 2^-kv / l, l over both halves
