@@ -263,31 +263,56 @@ size_t combine_one_spread_smem(int rows) {
 
 // Mixed cache (abaddon 0.2.0-rc.1, src/kv_cache_quant_cuda.rs,
 // OptimizedQuantizedKvCache::get_kv: the INT8 part dequantised, then the
-// unquantised recent tokens): one CTA per (b, q head).  The newest min(L, W)
-// tokens sit in the bf16 ring of the head's kv head (position g in row
-// g % W).  They are walked in tiles of up to tw tokens (the whole window when
-// it fits the dynamic shared memory), each tile's K and V rows brought in by
-// one round of asynchronous 16-byte copies, with an online softmax in fp32:
-// the tile's scores by the eight warps (a warp per token, lanes over
-// head_dim), its maximum and weights by one warp (lanes over tokens), then
-// thread d updates output value d.  The split kernel's INT8 partials of the
-// row (every slot below the INT8 part's chunk count with a finite m) are
-// folded in at the end; the first kRecPre slots' m, l and values are loaded
-// before the window work, so their latency overlaps it.
+// unquantised recent tokens): a cluster of kRecParts CTAs per (b, q head).
+// The newest min(L, W) tokens sit in the bf16 ring of the head's kv head
+// (position g in row g % W); CTA (cluster rank) r takes the r-th quarter of
+// them and the row's INT8 partial slots j with j % kRecParts == r (every
+// slot below the INT8 part's chunk count with a finite m).  Its window
+// tokens are walked in tiles of up to tw tokens (all of them when they fit
+// the dynamic shared memory), each tile's K and V rows brought in by one
+// round of asynchronous 16-byte copies, with an online softmax in fp32: the
+// tile's scores by the eight warps (a warp per token, lanes over head_dim),
+// its maximum and weights by one warp (lanes over tokens), then P.V with the
+// tokens split among the threads of each output value.  Its slots' m, l and
+// values are loaded before the window work, so their latency overlaps it.
+// Each CTA leaves its state (max M, sum l and unnormalised output, relative
+// to M) in shared memory; after a cluster barrier rank 0 reads the others'
+// through distributed shared memory and writes the row, and a second
+// barrier keeps every CTA's shared memory alive until it has.
 namespace {
 constexpr int kRecThreads = 256;
 constexpr int kRecWarps = kRecThreads / 32;
+constexpr int kRecParts = 4;                    // CTAs (one cluster) per (b, q head)
 constexpr int kRecSmem = 96 * 1024;             // dynamic shared memory budget of a tile
 constexpr int kRecMaxSlots = 64;                // INT8 partials staged per round
 constexpr int kRecPre = 16;                     // partial slots prefetched into registers
 
-int recent_tile(int W, int D) {                 // window tokens per tile
+int recent_tile(int W, int D) {                 // window tokens per tile (per CTA)
+    const int w = (W + kRecParts - 1) / kRecParts;
     const int fit = (kRecSmem - 64) / (4 * D + 4);
-    return W < fit ? W : fit;
+    return w < fit ? w : fit;
 }
 size_t recent_smem(int tw, int D) { return static_cast<size_t>(tw) * (4 * D + 4); }
 
-__global__ void __launch_bounds__(kRecThreads)
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// a float in CTA `rank`'s shared memory at this CTA's address `a` of the same variable
+__device__ __forceinline__ float ld_peer_f32(uint32_t a, uint32_t rank) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    return v;
+}
+
+__global__ void __cluster_dims__(kRecParts, 1, 1) __launch_bounds__(kRecThreads)
 decode_recent_combine(DecodeParams p, int tw) {
     extern __shared__ __align__(16) uint8_t rec_smem[];
     uint16_t* s_k = reinterpret_cast<uint16_t*>(rec_smem);            // [tw][D]
@@ -296,9 +321,13 @@ decode_recent_combine(DecodeParams p, int tw) {
     __shared__ __align__(16) float s_q[256];                          // the query row (fp32)
     __shared__ float s_st[4];                                         // m, l, tile rescale
     __shared__ float s_m8[kRecMaxSlots], s_l8[kRecMaxSlots];
+    __shared__ __align__(16) float s_red[kRecThreads];                // P.V part sums
+    __shared__ __align__(16) float s_fo[256];                         // this CTA's state
+    __shared__ float s_fm, s_fl;
     grid_dep_wait();                    // the split kernel's partials are complete
     grid_dep_launch();
-    const int64_t row = blockIdx.x;                     // b * Hq + q head
+    const int r = static_cast<int>(cluster_rank());
+    const int64_t row = blockIdx.x / kRecParts;         // b * Hq + q head
     const int b = static_cast<int>(row / p.Hq);
     const int unit = static_cast<int>(row / p.G);       // b * Hk + kv head
     const int D = p.D, W = p.recent;
@@ -308,24 +337,31 @@ decode_recent_combine(DecodeParams p, int tw) {
     const int L = p.seq_lens[b];
     const int n8 = walked_len(L, cap, plan, 1, 0, W);   // INT8 part walked by the split kernel
     if (n8 < 0) {                                       // flagged by the split kernel
-        for (int d = tid; d < D; d += kRecThreads) p.out[row * D + d] = 0.f;
+        // (the same for every CTA of the cluster: all of them leave here)
+        if (r == 0)
+            for (int d = tid; d < D; d += kRecThreads) p.out[row * D + d] = 0.f;
         return;
     }
     const int Lq = L > W ? L - W : 0;
     const int nr = L - Lq;                              // tokens in the window
+    const int i_lo = static_cast<int>(static_cast<int64_t>(nr) * r / kRecParts);
+    const int i_hi = static_cast<int>(static_cast<int64_t>(nr) * (r + 1) / kRecParts);
     const int ns = (n8 + p.chunk - 1) / p.chunk;        // INT8 partial slots
+    const int nsr = ns > r ? (ns - r + kRecParts - 1) / kRecParts : 0;   // this CTA's slots
     const float* m8 = p.ws_m + row * p.splits;
     const float* l8 = p.ws_l + row * p.splits;
     const float* o8 = p.ws_o + row * p.splits * D + (tid < D ? tid : 0);
-    // the first slots' m, l (shared) and this thread's values (registers)
-    const int npre = min(ns, kRecPre);
+    // the first of this CTA's slots (j = r + kRecParts u): m, l (shared) and
+    // this thread's values (registers)
+    const int npre = min(nsr, kRecPre);
     if (tid < npre) {
-        s_m8[tid] = m8[tid];
-        s_l8[tid] = l8[tid];
+        s_m8[tid] = m8[r + kRecParts * tid];
+        s_l8[tid] = l8[r + kRecParts * tid];
     }
     float ovp[kRecPre];
 #pragma unroll
-    for (int u = 0; u < kRecPre; ++u) ovp[u] = u < npre ? o8[static_cast<int64_t>(u) * D] : 0.f;
+    for (int u = 0; u < kRecPre; ++u)
+        ovp[u] = u < npre ? o8[static_cast<int64_t>(r + kRecParts * u) * D] : 0.f;
     for (int d = tid; d < D; d += kRecThreads) s_q[d] = bf16_bits_to_f32(p.q[row * D + d]);
     if (tid == 0) {
         s_st[0] = -INFINITY;
@@ -335,8 +371,9 @@ decode_recent_combine(DecodeParams p, int tw) {
     const int64_t ring0 = static_cast<int64_t>(unit) * W;
     const int vec = D / 8;                              // 16-byte chunks per row
     const uint32_t sk_a = ptx::smem_u32(s_k), sv_a = ptx::smem_u32(s_v);
-    for (int i0 = 0; i0 < nr; i0 += tw) {
-        const int n = min(tw, nr - i0);
+    const int parts = D <= kRecThreads / 2 ? kRecThreads / D : 1;   // P.V threads per value
+    for (int i0 = i_lo; i0 < i_hi; i0 += tw) {
+        const int n = min(tw, i_hi - i0);
         __syncthreads();                                // the previous tile is consumed
         for (int c = tid; c < n * vec; c += kRecThreads) {
             const int t = c / vec, x = c - (c / vec) * vec;
@@ -390,20 +427,33 @@ decode_recent_combine(DecodeParams p, int tw) {
             }
         }
         __syncthreads();
-        if (tid < D) {                                  // four partial sums: a short chain
-            float ac[4] = {o * s_st[2], 0.f, 0.f, 0.f};
-            int t = 0;
-            for (; t + 4 <= n; t += 4)
+        // P.V: the tile's tokens split among `parts` threads per output value
+        // (token t to part t % parts), four partial sums each, then summed
+        // into the running value by the part-0 threads
+        {
+            const int part = tid / D, d = tid - part * D;
+            if (part < parts) {
+                float ac[4] = {0.f, 0.f, 0.f, 0.f};
+                int t = part;
+                for (; t + 3 * parts < n; t += 4 * parts)
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    ac[u] = fmaf(s_p[t + u], bf16_bits_to_f32(s_v[(t + u) * D + tid]), ac[u]);
-            for (; t < n; ++t) ac[0] = fmaf(s_p[t], bf16_bits_to_f32(s_v[t * D + tid]), ac[0]);
-            o = (ac[0] + ac[1]) + (ac[2] + ac[3]);
+                    for (int u = 0; u < 4; ++u)
+                        ac[u] = fmaf(s_p[t + u * parts],
+                                     bf16_bits_to_f32(s_v[(t + u * parts) * D + d]), ac[u]);
+                for (; t < n; t += parts) ac[0] = fmaf(s_p[t], bf16_bits_to_f32(s_v[t * D + d]), ac[0]);
+                s_red[tid] = (ac[0] + ac[1]) + (ac[2] + ac[3]);
+            }
+            __syncthreads();
+            if (tid < D) {
+                float sum = o * s_st[2];
+                for (int q = 0; q < parts; ++q) sum += s_red[q * D + tid];
+                o = sum;
+            }
         }
     }
     __syncthreads();
-    // the row's INT8 partials: their maximum and weighted sum, then output d;
-    // empty slots (m = -inf) are dropped by selection (no load behind a branch)
+    // this CTA's INT8 partials: their maximum and weighted sum; empty slots
+    // (m = -inf) are dropped by selection (no load behind a branch)
     float M = s_st[0];
     float lsum = 0.f;                                   // relative to M, the window's l not included
     float acc = 0.f;
@@ -428,29 +478,57 @@ decode_recent_combine(DecodeParams p, int tw) {
     for (int u = 0; u < kRecPre; ++u)
         if (u < npre) add(u, ovp[u]);
 #pragma unroll 1
-    for (int j0 = npre; j0 < ns; j0 += kRecMaxSlots) {
-        const int nj = min(kRecMaxSlots, ns - j0);
+    for (int u0 = npre; u0 < nsr; u0 += kRecMaxSlots) {
+        const int nj = min(kRecMaxSlots, nsr - u0);
         __syncthreads();                                // s_m8, s_l8 free
         if (tid < nj) {
-            s_m8[tid] = m8[j0 + tid];
-            s_l8[tid] = l8[j0 + tid];
+            s_m8[tid] = m8[r + kRecParts * (u0 + tid)];
+            s_l8[tid] = l8[r + kRecParts * (u0 + tid)];
         }
         __syncthreads();
         rescale(nj);
-        for (int j = 0; j < nj; ++j) add(j, o8[static_cast<int64_t>(j0 + j) * D]);
+        for (int j = 0; j < nj; ++j) add(j, o8[static_cast<int64_t>(r + kRecParts * (u0 + j)) * D]);
     }
-    if (tid < D) {
+    // this CTA's state, relative to its maximum M
+    {
         const float aw = mw == -INFINITY ? 0.f : exp2f(mw - M);
-        const float tot = lsum + lw * aw;
-        p.out[row * D + tid] = tot > 0.f ? (acc + o * aw) / tot : 0.f;
+        if (tid == 0) {
+            s_fm = M;
+            s_fl = lsum + lw * aw;
+        }
+        if (tid < D) s_fo[tid] = acc + o * aw;
     }
+    cluster_sync_all();                                 // every CTA's state is written
+    if (r == 0) {
+        float fm[kRecParts], fl[kRecParts], fo[kRecParts];
+        const uint32_t am = ptx::smem_u32(&s_fm), al = ptx::smem_u32(&s_fl);
+        const uint32_t ao = ptx::smem_u32(&s_fo[tid < D ? tid : 0]);
+#pragma unroll
+        for (int q = 0; q < kRecParts; ++q) {
+            fm[q] = ld_peer_f32(am, q);
+            fl[q] = ld_peer_f32(al, q);
+            fo[q] = tid < D ? ld_peer_f32(ao, q) : 0.f;
+        }
+        float Mx = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kRecParts; ++q) Mx = fmaxf(Mx, fm[q]);
+        float tot = 0.f, val = 0.f;
+#pragma unroll
+        for (int q = 0; q < kRecParts; ++q) {
+            const float w = fm[q] == -INFINITY ? 0.f : exp2f(fm[q] - Mx);
+            tot = fmaf(w, fl[q], tot);
+            val = fmaf(w, fo[q], val);
+        }
+        if (tid < D) p.out[row * D + tid] = tot > 0.f ? val / tot : 0.f;
+    }
+    cluster_sync_all();                                 // rank 0 has read every CTA's state
 }
 
 }  // namespace
 
 cudaError_t launch_recent_combine(const DecodeParams& p, cudaStream_t s) {
     if (p.recent < 1 || p.recent > kMaxRecent || p.D > 256 || p.qlen != 1 ||
-        static_cast<int64_t>(p.B) * p.Hq > 0x7fffffffll)
+        static_cast<int64_t>(p.B) * p.Hq * kRecParts > 0x7fffffffll)
         return cudaErrorInvalidValue;
     static std::atomic<uint64_t> done{0};
     int dev = 0;
@@ -463,7 +541,7 @@ cudaError_t launch_recent_combine(const DecodeParams& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int tw = recent_tile(p.recent, p.D);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(static_cast<int64_t>(p.B) * p.Hq), 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(static_cast<int64_t>(p.B) * p.Hq * kRecParts), 1, 1);
     cfg.blockDim = dim3(kRecThreads, 1, 1);
     cfg.dynamicSmemBytes = recent_smem(tw, p.D);
     cfg.stream = s;
