@@ -122,9 +122,10 @@ def test_mixed_many_units(mode):
 
 @pytest.mark.parametrize("D,G,W", [(128, 32, 2048), (96, 4, 200), (256, 8, 40)])
 def test_mixed_wide_groups_long_windows_other_head_dims(D, G, W):
-    """The window kernel takes one CTA per (sequence, q head): 32 heads per kv
-    head, the longest window (2048 tokens, many tiles), and head dims whose
-    INT8 part runs on the CUDA-core split kernel."""
+    """The window kernel takes a cluster of four CTAs per (sequence, q head):
+    32 heads per kv head, the longest window (2048 tokens, 512 per CTA in
+    several tiles), and head dims whose INT8 part runs on the CUDA-core split
+    kernel."""
     B, Hk, S = 2, 2, 3000
     c = MixedPair(B, Hk, S, D, W, "per_token", seed=D + G)
     c.append([2500, 100], seed=3)
