@@ -92,7 +92,12 @@ kvq_status plan(int B, int Hk, int hint, int num_splits, int num_sms, int* chunk
         const int64_t units = static_cast<int64_t>(B > 0 ? B : 1) * Hk;
         const int64_t per_unit = num_sms / units;
         if (per_unit >= 8) {
-            chunk = ceil_div(ceil_div(hint, per_unit), 16) * 16;
+            // a short sequence (at most four 128-token stages, which the CTA's
+            // two consumer groups take in two rounds) stays one chunk: its
+            // CTA writes the final rows, and no combine launch follows, which
+            // costs more than the stages that splitting would spread
+            chunk = hint <= 4 * 128 ? ceil_div(hint, 16) * 16
+                                    : ceil_div(ceil_div(hint, per_unit), 16) * 16;
         } else {
             chunk = 128;
         }
