@@ -87,6 +87,19 @@ def test_decode_plan_fills_the_machine(kvq):
     assert 16 < splits <= 64
 
 
+def test_decode_plan_keeps_short_sequences_whole(kvq):
+    # few units and at most four 128-token stages: one chunk, no combine
+    assert kvq.kvq_decode_plan(1, 1, 257, 0, num_sms=148) == (272, 1)
+    assert kvq.kvq_decode_plan(2, 2, 512, 0, num_sms=148) == (512, 1)
+    # one token more: split over the SMs again
+    chunk, splits = kvq.kvq_decode_plan(1, 1, 513, 0, num_sms=148)
+    assert splits > 1 and splits * chunk >= 513
+    # many units keep one-stage chunks whatever the length
+    assert kvq.kvq_decode_plan(64, 8, 300, 0, num_sms=148) == (128, 3)
+    # an explicit split count still splits a short sequence
+    assert kvq.kvq_decode_plan(1, 1, 257, 4, num_sms=148)[1] == 4
+
+
 def test_workspace_formula(kvq):
     if torch.cuda.is_available():
         pytest.skip("formula check uses an explicit SM count; covered on the GPU")
